@@ -1,0 +1,369 @@
+/*
+ * moe_oracle.c -- float64 CPU oracle for the forward pass of a top-k routed
+ * mixture-of-experts SwiGLU FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the independent checker of the
+ * CUDA library: only the tests, the smoke check and the timed CPU baseline
+ * of the benchmark may load it.  It shares no code, header, table or helper
+ * with the CUDA path; it reads the same raw input bits (bf16 or fp32) and
+ * nothing else.
+ *
+ * Every value is widened to double on load (bf16 -> double and fp32 -> double
+ * are exact), every sum is a plain left-to-right double sum, and there is no
+ * blocking, fusion or reordering beyond what the method states.  The code
+ * follows the pages step by step:
+ *
+ *   route      "Tutorial 11: Mixture of Experts (MoE)", section 2 "The Router"
+ *              (route_topk: router logits, softmax over all experts, top-k,
+ *              gather of the kept scores, optional renormalisation), and
+ *              "Small MoE Architecture, in depth", section "A small MoE layer
+ *              in PyTorch" (sigmoid scores, gates = the kept raw scores).
+ *   permute    "Tutorial 11", section 3 "Expert Computation", Step 1 (sort the
+ *              flattened expert ids; the grouped order) and "Small MoE
+ *              Architecture, in depth" (per-expert counts by bincount).
+ *   forward    "Tutorial 11", section 3 Steps 2-3 and section 4 "The Complete
+ *              MoE Layer" (per-row expert SwiGLU, weighted sum over the k
+ *              selected experts); the SwiGLU expert is down(silu(gate x) *
+ *              up x) as in the Expert module of "Small MoE Architecture, in
+ *              depth"; the always-on shared expert is added to every token as
+ *              in the same module, scaled by sigmoid(w_s . x).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - top-k slot order: keys in descending order, ties to the lower expert
+ *     index (the pages' argpartition leaves the order open; torch.topk sorts).
+ *   - selection key: the logit for softmax scoring (softmax is monotone, so
+ *     ranking logits ranks probabilities) and sigmoid(logit) for sigmoid.
+ *   - "softmax over those four scores" (Small models, sparse experts, "How it
+ *     works" step 3) equals full softmax followed by renormalisation of the k
+ *     kept probabilities; that configuration is {softmax, norm_topk = 1}.
+ *   - the shared expert's gate is sigmoid(w_s . x); its logit takes no part
+ *     in the top-k selection.
+ *   - silu(u) = u / (1 + exp(-u)); no biases anywhere.
+ *
+ * Pins: this file is checked, not trusted -- see tests/test_oracle_pins.py
+ * (the route_topk worked example, a dense all-experts formulation, a
+ * loop-over-experts formulation, E = 1 / k = 1 dense SwiGLU, invariants).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_BF16 = 0, ORACLE_F32 = 1 };
+enum { ORACLE_SOFTMAX = 0, ORACLE_SIGMOID = 1 };
+
+/* Layer shape and options.  T tokens of width d, E routed experts of hidden
+ * width h, k experts per token, h_shared = 0 means no shared expert. */
+typedef struct {
+    int64_t T;
+    int32_t d, E, h, k;
+    int32_t norm_topk;
+    int32_t score;
+    int32_t h_shared;
+    int32_t dtype;
+} oracle_cfg;
+
+/* Element i of a stored tensor, widened exactly to double. */
+static double elem(const void *base, int64_t i, int32_t dtype)
+{
+    if (dtype == ORACLE_F32)
+        return (double)((const float *)base)[i];
+    uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+static double silu(double u) { return u / (1.0 + exp(-u)); }
+
+static int cfg_ok(const oracle_cfg *c)
+{
+    if (!c || c->T < 0 || c->d < 1 || c->E < 1 || c->h < 1) return 0;
+    if (c->k < 1 || c->k > c->E) return 0;
+    if (c->score != ORACLE_SOFTMAX && c->score != ORACLE_SIGMOID) return 0;
+    if (c->dtype != ORACLE_BF16 && c->dtype != ORACLE_F32) return 0;
+    if (c->h_shared < 0) return 0;
+    return 1;
+}
+
+/* Router logits of one token: l_e = sum_i x_i * Wr[e, i] (a bias-free linear
+ * layer, "Tutorial 11" section 2 step 1; the router of "Small MoE
+ * Architecture, in depth" is nn.Linear(d, n_experts, bias=False)). */
+static void router_logits(const oracle_cfg *c, const void *x, const void *wr,
+                          int64_t t, double *logits)
+{
+    for (int32_t e = 0; e < c->E; ++e) {
+        double s = 0.0;
+        for (int32_t i = 0; i < c->d; ++i)
+            s += elem(x, t * c->d + i, c->dtype) * elem(wr, (int64_t)e * c->d + i, c->dtype);
+        logits[e] = s;
+    }
+}
+
+/* Selection keys: logits under softmax (monotone map), sigmoid otherwise. */
+static void selection_keys(const oracle_cfg *c, const double *logits, double *keys)
+{
+    for (int32_t e = 0; e < c->E; ++e)
+        keys[e] = (c->score == ORACLE_SIGMOID) ? sigmoid(logits[e]) : logits[e];
+}
+
+/* The k best experts, best first: repeatedly take the largest key not yet
+ * taken, scanning experts in increasing index so that ties go to the lower
+ * index.  O(k * E), plain on purpose. */
+static void select_topk(const oracle_cfg *c, const double *keys, char *taken, int32_t *ids)
+{
+    memset(taken, 0, (size_t)c->E);
+    for (int32_t j = 0; j < c->k; ++j) {
+        int32_t best = -1;
+        for (int32_t e = 0; e < c->E; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || keys[e] > keys[best]) best = e;
+        }
+        taken[best] = 1;
+        ids[j] = best;
+    }
+}
+
+/* Scores over all experts: softmax with the maximum subtracted ("Tutorial 11"
+ * section 2 step 2), or the element-wise sigmoid ("Small MoE Architecture, in
+ * depth", forward: scores = sigmoid(router(x))). */
+static void expert_scores(const oracle_cfg *c, const double *logits, double *scores)
+{
+    if (c->score == ORACLE_SIGMOID) {
+        for (int32_t e = 0; e < c->E; ++e) scores[e] = sigmoid(logits[e]);
+        return;
+    }
+    double m = logits[0];
+    for (int32_t e = 1; e < c->E; ++e)
+        if (logits[e] > m) m = logits[e];
+    double z = 0.0;
+    for (int32_t e = 0; e < c->E; ++e) z += exp(logits[e] - m);
+    for (int32_t e = 0; e < c->E; ++e) scores[e] = exp(logits[e] - m) / z;
+}
+
+/* Routes one token: ids[0..k), gates[0..k), the full score row and the
+ * shared-expert gate.  Gates are the selected scores ("Tutorial 11" section 2
+ * step 4), divided by their sum when norm_topk is set (step 5; the worked
+ * example under "Why Normalize Selected Probabilities?"). */
+static void route_one(const oracle_cfg *c, const void *x, const void *wr, const void *w_sg,
+                      int64_t t, double *logits, double *keys, double *scores, char *taken,
+                      int32_t *ids, double *gates, double *shared_gate)
+{
+    router_logits(c, x, wr, t, logits);
+    selection_keys(c, logits, keys);
+    select_topk(c, keys, taken, ids);
+    expert_scores(c, logits, scores);
+    double sum = 0.0;
+    for (int32_t j = 0; j < c->k; ++j) {
+        gates[j] = scores[ids[j]];
+        sum += gates[j];
+    }
+    if (c->norm_topk)
+        for (int32_t j = 0; j < c->k; ++j) gates[j] /= sum;
+    if (shared_gate) {
+        double s = 0.0;
+        if (c->h_shared > 0 && w_sg) {
+            for (int32_t i = 0; i < c->d; ++i)
+                s += elem(x, t * c->d + i, c->dtype) * elem(w_sg, i, c->dtype);
+            *shared_gate = sigmoid(s);
+        } else {
+            *shared_gate = 0.0;
+        }
+    }
+}
+
+static int nthreads_used(int requested)
+{
+#ifdef _OPENMP
+    if (requested > 0) return requested;
+    return omp_get_max_threads();
+#else
+    (void)requested;
+    return 1;
+#endif
+}
+
+/* Routes tokens [t0, t1).  ids and gates are [T, k] (indexed by absolute
+ * token), probs is an optional [T, E] score matrix, shared_gate an optional
+ * [T] vector.  Returns 0 on success, -1 on a bad argument. */
+int oracle_route(const oracle_cfg *c, const void *x, const void *wr, const void *w_sg,
+                 int64_t t0, int64_t t1, int32_t *ids, double *gates, double *probs,
+                 double *shared_gate, int nthreads)
+{
+    if (!cfg_ok(c) || !x || !wr || !ids || !gates || t0 < 0 || t1 > c->T || t0 > t1) return -1;
+    int nt = nthreads_used(nthreads);
+    int bad = 0;
+#pragma omp parallel num_threads(nt)
+    {
+        double *logits = malloc(sizeof(double) * (size_t)c->E * 3);
+        char *taken = malloc((size_t)c->E);
+        if (!logits || !taken) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            double *keys = logits + c->E, *scores = logits + 2 * c->E;
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = t0; t < t1; ++t) {
+                route_one(c, x, wr, w_sg, t, logits, keys, scores, taken, ids + t * c->k,
+                          gates + t * c->k, shared_gate ? shared_gate + t : NULL);
+                if (probs)
+                    for (int32_t e = 0; e < c->E; ++e) probs[t * c->E + e] = scores[e];
+            }
+        }
+        free(logits);
+        free(taken);
+    }
+    return bad ? -1 : 0;
+}
+
+/* Margin of the selection for tokens [t0, t1): the smallest gap between
+ * adjacent keys among the top min(k + 1, E) keys in descending order.  A
+ * margin above the numerical error of a faster implementation means that it
+ * must find the same experts in the same slot order. */
+int oracle_topk_margin(const oracle_cfg *c, const void *x, const void *wr, int64_t t0, int64_t t1,
+                       double *margin, int nthreads)
+{
+    if (!cfg_ok(c) || !x || !wr || !margin || t0 < 0 || t1 > c->T || t0 > t1) return -1;
+    int nt = nthreads_used(nthreads);
+    int32_t m = c->k + 1 <= c->E ? c->k + 1 : c->E;
+    int bad = 0;
+#pragma omp parallel num_threads(nt)
+    {
+        double *logits = malloc(sizeof(double) * (size_t)c->E * 2);
+        char *taken = malloc((size_t)c->E);
+        int32_t *order = malloc(sizeof(int32_t) * (size_t)m);
+        if (!logits || !taken || !order) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            double *keys = logits + c->E;
+            oracle_cfg cm = *c;
+            cm.k = m;
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = t0; t < t1; ++t) {
+                router_logits(c, x, wr, t, logits);
+                selection_keys(c, logits, keys);
+                select_topk(&cm, keys, taken, order);
+                double g = INFINITY;
+                for (int32_t j = 0; j + 1 < m; ++j) {
+                    double gap = keys[order[j]] - keys[order[j + 1]];
+                    if (gap < g) g = gap;
+                }
+                margin[t - t0] = g;
+            }
+        }
+        free(logits);
+        free(taken);
+        free(order);
+    }
+    return bad ? -1 : 0;
+}
+
+/* Groups the T*k assignments by expert.  Assignment r = t*k + j carries
+ * expert ids[r].  counts[e] = number of assignments to e; offsets is the
+ * exclusive prefix sum of counts (E + 1 entries); sorted_rows lists the
+ * assignments expert by expert, each expert's in increasing r (a stable sort
+ * by expert id, "Tutorial 11" section 3 Step 1); inv_rows is its inverse,
+ * inv_rows[sorted_rows[i]] = i.  Returns -1 on an id outside [0, E). */
+int oracle_permute(const oracle_cfg *c, const int32_t *ids, int32_t *counts, int32_t *offsets,
+                   int32_t *sorted_rows, int32_t *inv_rows)
+{
+    if (!cfg_ok(c) || !ids || !counts || !offsets || !sorted_rows || !inv_rows) return -1;
+    int64_t R = c->T * c->k;
+    for (int64_t r = 0; r < R; ++r)
+        if (ids[r] < 0 || ids[r] >= c->E) return -1;
+    for (int32_t e = 0; e < c->E; ++e) {
+        int32_t n = 0;
+        for (int64_t r = 0; r < R; ++r) n += (ids[r] == e);
+        counts[e] = n;
+    }
+    offsets[0] = 0;
+    for (int32_t e = 0; e < c->E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int64_t pos = 0;
+    for (int32_t e = 0; e < c->E; ++e)
+        for (int64_t r = 0; r < R; ++r)
+            if (ids[r] == e) sorted_rows[pos++] = (int32_t)r;
+    for (int64_t i = 0; i < R; ++i) inv_rows[sorted_rows[i]] = (int32_t)i;
+    return 0;
+}
+
+/* One SwiGLU expert applied to token t, scaled by g and added to out[d]:
+ * out += g * Wd . (silu(Wg . x) * (Wu . x)).  Wg, Wu are [hid, d] and Wd is
+ * [d, hid], all row-major; `a` is scratch of length hid. */
+static void swiglu_expert_add(const oracle_cfg *c, const void *x, int64_t t, const void *wg,
+                              const void *wu, const void *wd, int64_t w_off_in, int64_t w_off_out,
+                              int32_t hid, double g, double *a, double *out)
+{
+    for (int32_t n = 0; n < hid; ++n) {
+        double u = 0.0, v = 0.0;
+        for (int32_t i = 0; i < c->d; ++i) {
+            double xi = elem(x, t * c->d + i, c->dtype);
+            u += elem(wg, w_off_in + (int64_t)n * c->d + i, c->dtype) * xi;
+            v += elem(wu, w_off_in + (int64_t)n * c->d + i, c->dtype) * xi;
+        }
+        a[n] = silu(u) * v;
+    }
+    for (int32_t i = 0; i < c->d; ++i) {
+        double o = 0.0;
+        for (int32_t n = 0; n < hid; ++n)
+            o += elem(wd, w_off_out + (int64_t)i * hid + n, c->dtype) * a[n];
+        out[i] += g * o;
+    }
+}
+
+/* Full layer output for the listed tokens: y[i, :] is token tokens[i]'s
+ * output row, y = sum_j gate_j * expert_{ids_j}(x) (+ sigmoid(w_s . x) *
+ * shared(x) when h_shared > 0).  W_gate/W_up are [E, h, d], W_down [E, d, h];
+ * the shared expert's weights are [h_shared, d], [h_shared, d], [d, h_shared]
+ * and w_s is [d].  Routing is recomputed per token, so any subset of tokens
+ * can be evaluated on its own.  Returns the number of threads used, or -1. */
+int oracle_forward(const oracle_cfg *c, const void *x, const void *wr, const void *wg,
+                   const void *wu, const void *wd, const void *sh_g, const void *sh_u,
+                   const void *sh_d, const void *w_sg, const int64_t *tokens, int64_t n_tokens,
+                   double *y, int nthreads)
+{
+    if (!cfg_ok(c) || !x || !wr || !wg || !wu || !wd || !tokens || !y || n_tokens < 0) return -1;
+    if (c->h_shared > 0 && (!sh_g || !sh_u || !sh_d || !w_sg)) return -1;
+    for (int64_t i = 0; i < n_tokens; ++i)
+        if (tokens[i] < 0 || tokens[i] >= c->T) return -1;
+    int nt = nthreads_used(nthreads);
+    int32_t hmax = c->h > c->h_shared ? c->h : c->h_shared;
+    int bad = 0;
+#pragma omp parallel num_threads(nt)
+    {
+        double *logits = malloc(sizeof(double) * ((size_t)c->E * 3 + (size_t)c->k + (size_t)hmax));
+        char *taken = malloc((size_t)c->E);
+        int32_t *ids = malloc(sizeof(int32_t) * (size_t)c->k);
+        if (!logits || !taken || !ids) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            double *keys = logits + c->E, *scores = logits + 2 * c->E;
+            double *gates = logits + 3 * c->E, *a = gates + c->k;
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t i = 0; i < n_tokens; ++i) {
+                int64_t t = tokens[i];
+                double sg = 0.0;
+                route_one(c, x, wr, w_sg, t, logits, keys, scores, taken, ids, gates, &sg);
+                double *out = y + i * c->d;
+                for (int32_t q = 0; q < c->d; ++q) out[q] = 0.0;
+                for (int32_t j = 0; j < c->k; ++j) {
+                    int64_t e = ids[j];
+                    swiglu_expert_add(c, x, t, wg, wu, wd, e * c->h * c->d, e * c->d * c->h, c->h,
+                                      gates[j], a, out);
+                }
+                if (c->h_shared > 0)
+                    swiglu_expert_add(c, x, t, sh_g, sh_u, sh_d, 0, 0, c->h_shared, sg, a, out);
+            }
+        }
+        free(logits);
+        free(taken);
+        free(ids);
+    }
+    return bad ? -1 : nt;
+}

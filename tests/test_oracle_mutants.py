@@ -1,0 +1,77 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU,
+in a temporary directory), builds it, and runs the pin checks of
+test_oracle_pins against that build: at least one pin must fail.  The
+committed oracle itself is never modified.
+"""
+import os
+import shutil
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
+
+# (name, exact text in the oracle, planted mistake)
+MUTANTS = [
+    ("tie_to_higher_index", "keys[e] > keys[best]) best = e;", "keys[e] >= keys[best]) best = e;"),
+    ("sigmoid_sign", "return 1.0 / (1.0 + exp(-v));", "return 1.0 / (1.0 + exp(v));"),
+    ("silu_sign", "return u / (1.0 + exp(-u));", "return u / (1.0 + exp(u));"),
+    ("renorm_dropped", "if (c->norm_topk)\n", "if (0 && c->norm_topk)\n"),
+    ("gate_from_slot_index", "gates[j] = scores[ids[j]];", "gates[j] = scores[j];"),
+    ("down_transposed", "elem(wd, w_off_out + (int64_t)i * hid + n, c->dtype)",
+     "elem(wd, w_off_out + (int64_t)n * c->d + i, c->dtype)"),
+    ("gate_up_swapped", "a[n] = silu(u) * v;", "a[n] = silu(v) * u;"),
+    ("router_transposed", "elem(wr, (int64_t)e * c->d + i, c->dtype)",
+     "elem(wr, (int64_t)i * c->E + e, c->dtype)"),
+    ("softmax_no_normaliser", "scores[e] = exp(logits[e] - m) / z;",
+     "scores[e] = exp(logits[e] - m);"),
+    ("permutation_unstable", "for (int64_t r = 0; r < R; ++r)\n            if (ids[r] == e) sorted_rows[pos++]",
+     "for (int64_t r = R - 1; r >= 0; --r)\n            if (ids[r] == e) sorted_rows[pos++]"),
+    ("offsets_inclusive", "offsets[e + 1] = offsets[e] + counts[e];",
+     "offsets[e + 1] = offsets[e] + counts[e] + (e == 0);"),
+    ("shared_gate_sign", "*shared_gate = sigmoid(s);", "*shared_gate = sigmoid(-s);"),
+    ("gate_weight_dropped", "out[i] += g * o;", "out[i] += o;"),
+    ("selection_by_raw_logit_under_sigmoid",
+     "keys[e] = (c->score == ORACLE_SIGMOID) ? sigmoid(logits[e]) : logits[e];",
+     "keys[e] = (c->score == ORACLE_SIGMOID) ? -logits[e] : logits[e];"),
+]
+
+
+@pytest.mark.parametrize("name,orig,bad", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, orig, bad):
+    src = open(SRC).read()
+    assert src.count(orig) == 1, f"mutation anchor for {name} not found exactly once"
+    msrc = tmp_path / "moe_oracle_mutant.c"
+    msrc.write_text(src.replace(orig, bad))
+    so = str(tmp_path / f"liboracle_{name}.so")
+    oracle.build(force=True, source=str(msrc), output=so)
+    old = pins.LIB_PATH
+    pins.LIB_PATH = so
+    failed = []
+    try:
+        for check in pins.PIN_CHECKS:
+            try:
+                check()
+            except (AssertionError, ValueError, IndexError):
+                failed.append(check.__name__)
+    finally:
+        pins.LIB_PATH = old
+        oracle._lib_cache.pop(so, None)
+    assert failed, f"planted mistake '{name}' passed every pin"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    so = str(tmp_path / "liboracle_copy.so")
+    shutil.copy(SRC, tmp_path / "copy.c")
+    oracle.build(force=True, source=str(tmp_path / "copy.c"), output=so)
+    old = pins.LIB_PATH
+    pins.LIB_PATH = so
+    try:
+        for check in pins.PIN_CHECKS:
+            check()
+    finally:
+        pins.LIB_PATH = old

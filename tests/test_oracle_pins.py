@@ -1,0 +1,334 @@
+"""Pins of the float64 oracle to facts that do not come from the oracle itself.
+
+* the routing worked example printed on "Tutorial 11: Mixture of Experts
+  (MoE)", section 2 (golden file, run through the oracle's full route);
+* the identity between "softmax over the kept scores" ("Small models, sparse
+  experts", section "How it works") and full softmax + renormalisation;
+* brute force over all k-subsets for the selected expert set;
+* a full sort (numpy lexsort) for slot order and tie-breaking;
+* the dense compute-all-experts-then-mask formulation and the
+  loop-over-experts index_add formulation (numpy, float64, matrix ops);
+* the E = 1, k = 1 special case, which is the textbook dense SwiGLU FFN;
+* invariants: distinct ids, counts summing to T*k, a stable permutation
+  (numpy's stable argsort), gates summing to one under renormalisation.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import dense
+from sparse_mixture_experts_sigmoid_b200 import synth
+from sparse_mixture_experts_sigmoid_b200.workloads import WORKLOADS, Workload
+
+from support import OracleInputs, bits, ocfg
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+LIB_PATH = None  # the mutation tests rebind this to a mutated build
+
+
+def lib():
+    return oracle.load(LIB_PATH)
+
+
+def _golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            out[key] = vals
+    return out
+
+
+# ---------------------------------------------------------------- worked example
+
+def _worked_example_layer(norm):
+    g = _golden("route_worked_example.txt")
+    p = np.array([float(v) for v in g["probs"]])
+    E, d = p.size, 8
+    c = oracle.Cfg(T=1, d=d, E=E, h=8, k=int(g["top_k"][0]), norm_topk=norm, dtype="f32")
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0                                    # x = e_0, so logit_e = Wr[e, 0]
+    wr = np.zeros((E, d), np.float32)
+    wr[:, 0] = np.log(p).astype(np.float32)          # softmax(ln p) = p since sum(p) = 1
+    return g, p, c, x, wr
+
+
+def check_worked_example():
+    g, p, c, x, wr = _worked_example_layer(norm=True)
+    ids, gates, probs, _ = oracle.route(c, x, wr, want_probs=True, lib=lib())
+    assert abs(p.sum() - 1.0) < 1e-15
+    np.testing.assert_array_equal(ids[0], [int(v) for v in g["ids"]])
+    num = [float(v) for v in g["normalised_exact_num"]]
+    den = float(g["normalised_exact_den"][0])
+    np.testing.assert_allclose(gates[0], np.array(num) / den, atol=1e-6)
+    np.testing.assert_allclose(np.round(gates[0], 3), [float(v) for v in g["normalised"]], atol=0)
+    np.testing.assert_allclose(probs[0], p, atol=1e-6)
+    # the non-renormalised twin returns the raw probabilities of the kept experts
+    _, _, c0, _, _ = _worked_example_layer(norm=False)
+    ids0, gates0, _, _ = oracle.route(c0, x, wr, lib=lib())
+    np.testing.assert_array_equal(ids0[0], ids[0])
+    np.testing.assert_allclose(gates0[0], [float(v) for v in g["scores"]], atol=1e-6)
+
+
+def test_worked_example():
+    check_worked_example()
+
+
+# ---------------------------------------------------------------- routing
+
+def _random_case(rng, T, d, E, k, dtype="f32", score="softmax", norm=True, scale=1.0):
+    c = oracle.Cfg(T=T, d=d, E=E, h=8, k=k, norm_topk=norm, score=score, dtype=dtype)
+    x = (rng.standard_normal((T, d)) * scale).astype(np.float32)
+    wr = (rng.standard_normal((E, d)) * 0.3).astype(np.float32)
+    if dtype == "bf16":
+        x = _to_bf16_bits(x)
+        wr = _to_bf16_bits(wr)
+    return c, x, wr
+
+
+def _to_bf16_bits(a):
+    u = np.ascontiguousarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)   # round to nearest even
+    return r
+
+
+def check_routing_brute_force():
+    rng = np.random.default_rng(11)
+    for score in ("softmax", "sigmoid"):
+        for E, k in [(5, 2), (6, 3), (4, 4), (7, 1)]:
+            c, x, wr = _random_case(rng, 25, 9, E, k, score=score)
+            ids, _, _, _ = oracle.route(c, x, wr, lib=lib())
+            L = dense.to_f64(x) @ dense.to_f64(wr).T
+            for t in range(c.T):
+                # the kept set maximises the sum of logits over all k-subsets
+                # (distinct continuous keys; sigmoid is monotone so the set is the same)
+                best = max(itertools.combinations(range(E), k), key=lambda s: L[t, list(s)].sum())
+                assert set(ids[t].tolist()) == set(best)
+                # slots are ordered best first
+                assert all(L[t, ids[t, j]] > L[t, ids[t, j + 1]] for j in range(k - 1))
+
+
+def test_routing_brute_force():
+    check_routing_brute_force()
+
+
+def check_routing_vs_full_sort_and_ties():
+    rng = np.random.default_rng(12)
+    for score in ("softmax", "sigmoid"):
+        for norm in (True, False):
+            c, x, wr = _random_case(rng, 30, 16, 12, 4, score=score, norm=norm)
+            # duplicate router rows -> exactly tied keys; ties go to the lower index
+            wr[7] = wr[2]
+            wr[9] = wr[2]
+            wr[11] = wr[0]
+            ids, gates, probs, _ = oracle.route(c, x, wr, want_probs=True, lib=lib())
+            ids_ref, gates_ref, _ = dense.route_matrix(dense.to_f64(x), dense.to_f64(wr), c.k,
+                                                       score, norm)
+            np.testing.assert_array_equal(ids, ids_ref)
+            np.testing.assert_allclose(gates, gates_ref, rtol=1e-13, atol=1e-15)
+            for t in range(c.T):
+                s = list(ids[t])
+                for a, b in ((2, 7), (7, 9), (0, 11)):
+                    if a in s and b in s:
+                        assert s.index(a) < s.index(b)
+
+
+def test_routing_vs_full_sort_and_ties():
+    check_routing_vs_full_sort_and_ties()
+
+
+def test_softmax_over_kept_equals_renormalised_softmax():
+    """'softmax over those four scores' == full softmax then renormalise the kept."""
+    rng = np.random.default_rng(13)
+    c, x, wr = _random_case(rng, 64, 20, 16, 4, norm=True, scale=2.0)
+    ids, gates, _, _ = oracle.route(c, x, wr, lib=lib())
+    L = dense.to_f64(x) @ dense.to_f64(wr).T
+    kept = np.take_along_axis(L, ids.astype(np.int64), axis=1)
+    z = np.exp(kept - kept.max(axis=1, keepdims=True))
+    np.testing.assert_allclose(gates, z / z.sum(axis=1, keepdims=True), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(gates.sum(axis=1), 1.0, atol=1e-15)
+
+
+def check_margin():
+    rng = np.random.default_rng(14)
+    for score in ("softmax", "sigmoid"):
+        c, x, wr = _random_case(rng, 20, 10, 9, 3, score=score)
+        m = oracle.topk_margin(c, x, wr, lib=lib())
+        L = dense.to_f64(x) @ dense.to_f64(wr).T
+        key = 1.0 / (1.0 + np.exp(-L)) if score == "sigmoid" else L
+        srt = -np.sort(-key, axis=1)[:, :c.k + 1]
+        np.testing.assert_allclose(m, (srt[:, :-1] - srt[:, 1:]).min(axis=1), rtol=1e-12)
+
+
+def test_margin():
+    check_margin()
+
+
+# ---------------------------------------------------------------- whole layer
+
+SMALL_CASES = [
+    # (T, d, E, h, k, score, norm, h_shared, dtype)
+    (37, 24, 6, 20, 2, "softmax", True, 0, "f32"),
+    (29, 16, 5, 12, 3, "softmax", False, 0, "bf16"),
+    (31, 24, 7, 16, 2, "sigmoid", True, 0, "bf16"),
+    (23, 16, 4, 20, 1, "sigmoid", False, 28, "f32"),
+    (19, 32, 6, 8, 4, "softmax", False, 40, "bf16"),
+]
+
+
+def _small_layer(case, seed):
+    T, d, E, h, k, score, norm, hs, dt = case
+    w = Workload("small", T=T, d=d, E=E, h=h, k=k, score=score, norm_topk=norm, h_shared=hs,
+                 dtype=dt, seed=seed, router_std=0.3, weight_std=0.3)
+    return w, OracleInputs(synth.make_layer(w, "cpu"))
+
+
+def check_dense_formulation():
+    for i, case in enumerate(SMALL_CASES):
+        w, a = _small_layer(case, 100 + i)
+        c = ocfg(w)
+        y = oracle.forward(c, a.x, a.wr, a.wg, a.wu, a.wd, a.shared, lib=lib())
+        y_ref, ids_ref, gates_ref = dense.dense_forward(c, a.x, a.wr, a.wg, a.wu, a.wd, a.shared)
+        scale = np.abs(y_ref).max()
+        assert scale > 0
+        np.testing.assert_allclose(y, y_ref, rtol=0, atol=1e-12 * scale)
+        ids, gates, _, sg = oracle.route(c, a.x, a.wr, a.w_sg, lib=lib())
+        np.testing.assert_array_equal(ids, ids_ref)
+        np.testing.assert_allclose(gates, gates_ref, rtol=1e-13, atol=1e-15)
+        if w.h_shared:
+            sg_ref = 1.0 / (1.0 + np.exp(-(dense.to_f64(a.x) @ dense.to_f64(a.w_sg))))
+            np.testing.assert_allclose(sg, sg_ref, rtol=1e-13)
+
+
+def test_dense_formulation():
+    check_dense_formulation()
+
+
+def check_tiny_workload():
+    w = WORKLOADS["tiny"]
+    a = OracleInputs(synth.make_layer(w, "cpu"))
+    c = ocfg(w)
+    y = oracle.forward(c, a.x, a.wr, a.wg, a.wu, a.wd, lib=lib())
+    y_dense, _, _ = dense.dense_forward(c, a.x, a.wr, a.wg, a.wu, a.wd)
+    y_loop = dense.loop_over_experts_forward(c, a.x, a.wr, a.wg, a.wu, a.wd)
+    scale = np.abs(y_dense).max()
+    np.testing.assert_allclose(y, y_dense, rtol=0, atol=1e-12 * scale)
+    np.testing.assert_allclose(y, y_loop, rtol=0, atol=1e-12 * scale)
+    # a subset of tokens evaluates to the same rows
+    sub = np.array([63, 0, 17], np.int64)
+    np.testing.assert_allclose(oracle.forward(c, a.x, a.wr, a.wg, a.wu, a.wd, tokens=sub,
+                                              lib=lib()), y[sub], rtol=0, atol=0)
+
+
+def test_tiny_workload_three_formulations():
+    check_tiny_workload()
+
+
+def check_loop_over_experts():
+    for i, case in enumerate(SMALL_CASES[:3] + SMALL_CASES[4:]):
+        w, a = _small_layer(case, 200 + i)
+        c = ocfg(w)
+        y = oracle.forward(c, a.x, a.wr, a.wg, a.wu, a.wd, a.shared, lib=lib())
+        y_ref = dense.loop_over_experts_forward(c, a.x, a.wr, a.wg, a.wu, a.wd, a.shared)
+        np.testing.assert_allclose(y, y_ref, rtol=0, atol=1e-12 * np.abs(y_ref).max())
+
+
+def test_loop_over_experts():
+    check_loop_over_experts()
+
+
+def check_single_expert_is_dense_swiglu():
+    for score, norm in (("softmax", False), ("softmax", True), ("sigmoid", True)):
+        w = Workload("one", T=17, d=24, E=1, h=40, k=1, score=score, norm_topk=norm,
+                     dtype="f32", seed=7, weight_std=0.3, router_std=0.3)
+        a = OracleInputs(synth.make_layer(w, "cpu"))
+        c = ocfg(w)
+        y = oracle.forward(c, a.x, a.wr, a.wg, a.wu, a.wd, lib=lib())
+        ref = dense.dense_swiglu(dense.to_f64(a.x), dense.to_f64(a.wg[0]), dense.to_f64(a.wu[0]),
+                                 dense.to_f64(a.wd[0]))
+        np.testing.assert_allclose(y, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+        ids, gates, _, _ = oracle.route(c, a.x, a.wr, lib=lib())
+        assert (ids == 0).all() and np.all(gates == 1.0)
+    # sigmoid without renormalisation: gate = sigmoid(logit)
+    w = Workload("one", T=9, d=16, E=1, h=8, k=1, score="sigmoid", norm_topk=False, dtype="f32",
+                 seed=8, weight_std=0.3, router_std=0.3)
+    a = OracleInputs(synth.make_layer(w, "cpu"))
+    c = ocfg(w)
+    y = oracle.forward(c, a.x, a.wr, a.wg, a.wu, a.wd, lib=lib())
+    l = dense.to_f64(a.x) @ dense.to_f64(a.wr[0])
+    ref = (1 / (1 + np.exp(-l)))[:, None] * dense.dense_swiglu(
+        dense.to_f64(a.x), dense.to_f64(a.wg[0]), dense.to_f64(a.wu[0]), dense.to_f64(a.wd[0]))
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+
+
+def test_single_expert_is_dense_swiglu():
+    check_single_expert_is_dense_swiglu()
+
+
+# ---------------------------------------------------------------- grouping invariants
+
+def check_permutation_invariants():
+    rng = np.random.default_rng(15)
+    for T, E, k in [(50, 7, 3), (1, 4, 4), (64, 8, 2), (40, 16, 1)]:
+        c = oracle.Cfg(T=T, d=8, E=E, h=8, k=k)
+        # distinct ids per token, skewed towards expert 0 so some experts are empty
+        ids = np.stack([rng.choice(E, size=k, replace=False,
+                                   p=np.r_[0.5, np.full(E - 1, 0.5 / (E - 1))])
+                        for _ in range(T)]).astype(np.int32)
+        counts, offsets, srt, inv = oracle.permute(c, ids, lib=lib())
+        flat = ids.reshape(-1)
+        np.testing.assert_array_equal(counts, np.bincount(flat, minlength=E))
+        assert counts.sum() == T * k
+        np.testing.assert_array_equal(offsets, np.r_[0, np.cumsum(counts)])
+        np.testing.assert_array_equal(srt, np.argsort(flat, kind="stable"))
+        np.testing.assert_array_equal(inv[srt], np.arange(T * k))
+        for e in range(E):
+            seg = srt[offsets[e]:offsets[e + 1]]
+            assert (flat[seg] == e).all()
+
+
+def test_permutation_invariants():
+    check_permutation_invariants()
+
+
+def test_route_invariants_on_workload_shapes():
+    """Distinct ids, renormalised gates sum to one, unnormalised sum below one."""
+    for name in ("tiny", "gemma_upcycle"):
+        w = WORKLOADS[name].with_(T=48)
+        layer = synth.make_layer(w, "cpu")
+        c = ocfg(w)
+        ids, gates, _, _ = oracle.route(c, bits(layer.x), bits(layer.w_router))
+        for t in range(w.T):
+            assert len(set(ids[t].tolist())) == w.k
+        s = gates.sum(axis=1)
+        if w.norm_topk:
+            np.testing.assert_allclose(s, 1.0, atol=1e-12)
+        else:
+            assert (s < 1.0).all()
+
+
+def test_oracle_rejects_bad_arguments():
+    c = oracle.Cfg(T=2, d=4, E=3, h=4, k=4, dtype="f32")        # k > E
+    x = np.zeros((2, 4), np.float32)
+    wr = np.zeros((3, 4), np.float32)
+    with pytest.raises(ValueError):
+        oracle.route(c, x, wr)
+    c = oracle.Cfg(T=1, d=4, E=3, h=4, k=1)
+    with pytest.raises(ValueError):
+        oracle.permute(c, np.array([3], np.int32))                 # id out of range
+
+
+# The checks the mutation tests run against deliberately broken builds.
+PIN_CHECKS = [check_worked_example, check_routing_brute_force, check_routing_vs_full_sort_and_ties,
+              check_margin, check_dense_formulation, check_tiny_workload, check_loop_over_experts,
+              check_single_expert_is_dense_swiglu, check_permutation_invariants]
+
+assert math.isclose(64 ** (1 / 3), 4.0)
