@@ -1,0 +1,220 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the forward pass of a top-k routed
+ * mixture-of-experts (MoE) SwiGLU FFN layer on an NVIDIA B200 (sm_100a).
+ *
+ * The layer (one token row x of width d):
+ *
+ *   l_e    = x . W_router[e]                       e = 0..E-1, bias-free
+ *   s_e    = softmax(l)_e  or  sigmoid(l_e)        score function
+ *   ids    = the k experts with the largest keys, best first; the key is
+ *            l_e under softmax (same order as s_e) and s_e under sigmoid;
+ *            equal keys go to the lower expert index
+ *   g_j    = s_{ids_j}, divided by sum_j s_{ids_j} when norm_topk is set
+ *   y      = sum_j g_j * W_down[ids_j] (silu(W_gate[ids_j] x) * (W_up[ids_j] x))
+ *          + sigmoid(w_s . x) * S_down (silu(S_gate x) * (S_up x))  (shared
+ *            expert, only when h_shared > 0)
+ *   silu(u) = u * sigmoid(u)
+ *
+ * Sources: "Tutorial 11: Mixture of Experts (MoE)" -- section 2 "The Router"
+ * (route_topk: logits, softmax over all experts, top-k, gather of the kept
+ * scores, optional renormalisation), section 3 "Expert Computation" (group
+ * rows by expert, grouped expert linears, unsort and weighted sum), section 4
+ * "The Complete MoE Layer" (weight shapes); "Small MoE Architecture, in depth"
+ * -- section "A small MoE layer in PyTorch" (sigmoid scores, SwiGLU experts,
+ * shared expert added to every token).  The sigmoid gate on the shared expert
+ * and the tie rule are this library's readings where the pages are silent.
+ *
+ * Conventions for every entry point:
+ *  - Tensors are row-major and contiguous, in DEVICE memory owned by the
+ *    caller, on the current CUDA device.  The library allocates nothing,
+ *    frees nothing and never synchronises the stream; all work is enqueued
+ *    on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *  - Element type of x, weights, act and y: bf16 (MOE_BF16) or fp32
+ *    (MOE_F32), as cfg->dtype says.  Scores, gates and accumulators are
+ *    fp32; ids and permutations are int32.
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns an error and enqueues nothing.  MOE_ERR_CUDA means
+ *    a launch failed (cudaGetLastError); the stream may hold earlier work.
+ *  - Errors found on the device (an out-of-range expert id handed to
+ *    moe_permute, a bounded wait that ran out) set a device flag that
+ *    moe_device_status() reads.
+ *  - Limits: 1 <= k <= min(E, MOE_MAX_TOPK), 1 <= E <= MOE_MAX_EXPERTS,
+ *    d, h and h_shared multiples of 8, T * k < 2^31, T * max(d, h) < 2^40.
+ *    Valid shapes outside the limits return MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_MAX_EXPERTS 512
+#define MOE_MAX_TOPK 16
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,    /* null pointer, negative size, k outside [1, E], bad enum */
+    MOE_ERR_UNSUPPORTED = 2,    /* a valid shape outside the limits above */
+    MOE_ERR_WORKSPACE = 3,      /* workspace pointer null or smaller than required */
+    MOE_ERR_CUDA = 4,           /* a CUDA call or kernel launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out (from moe_device_status) */
+    MOE_ERR_DEVICE_INPUT = 6    /* a kernel met an invalid device input (from moe_device_status) */
+} moe_status;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_fn;
+typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
+
+/* Layer shape and options.  All fields are plain integers so the struct has
+ * one layout in every language binding. */
+typedef struct {
+    int64_t T;         /* tokens (rows of x and y); 0 is allowed and does nothing */
+    int32_t d;         /* model width */
+    int32_t E;         /* routed experts */
+    int32_t h;         /* hidden width of each routed expert */
+    int32_t k;         /* experts per token */
+    int32_t norm_topk; /* nonzero: divide the k gates by their sum */
+    int32_t score;     /* moe_score_fn */
+    int32_t h_shared;  /* hidden width of the always-on shared expert; 0 = none */
+    int32_t dtype;     /* moe_dtype of x, the weights, act and y */
+} moe_config;
+
+/* Device pointers into a moe_forward workspace (see moe_workspace_layout).
+ * Pointers of absent parts are NULL. */
+typedef struct {
+    int32_t *ids;         /* [T, k]  selected experts, best first */
+    float *gates;         /* [T, k]  gate of each selected expert */
+    float *shared_gate;   /* [T]     sigmoid(w_s . x); NULL without a shared expert */
+    int32_t *counts;      /* [E]     assignments per expert */
+    int32_t *offsets;     /* [E + 1] exclusive prefix sum of counts */
+    int32_t *sorted_rows; /* [T*k]   assignments r = t*k + j grouped by expert, stable */
+    int32_t *inv_rows;    /* [T*k]   inverse permutation: inv_rows[sorted_rows[i]] = i */
+    void *act;            /* [T*k, h] silu(gate)*up rows in grouped order (dtype) */
+    void *act_shared;     /* [T, h_shared] shared-expert activations; NULL if absent */
+    float *y_acc;         /* [T, d]  fp32 accumulator; NULL when dtype is MOE_F32 */
+} moe_workspace_views;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *moe_status_string(moe_status status);
+
+/* Checks a configuration against the rules and limits above (host only). */
+moe_status moe_validate(const moe_config *cfg);
+
+/* Bytes of device workspace that moe_forward needs for cfg (host only).
+ * The same workspace also serves moe_combine. */
+moe_status moe_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/* Carves a workspace of ws_bytes bytes at device address ws into the named
+ * parts that moe_forward fills (host only; nothing is read or written on the
+ * device).  ws must be 256-byte aligned. */
+moe_status moe_workspace_layout(const moe_config *cfg, void *ws, size_t ws_bytes,
+                                moe_workspace_views *views);
+
+/* Router: logits, scores, top-k selection and gates for all T tokens.
+ *   x        [T, d]        dtype
+ *   w_router [E, d]        dtype
+ *   w_shared_gate [d]      dtype, or NULL (then shared_gate must be NULL)
+ *   ids      [T, k] int32  out: selected experts, best first
+ *   gates    [T, k] fp32   out
+ *   probs    [T, E] fp32   out, optional (NULL): every expert's score s_e
+ *   shared_gate [T] fp32   out, optional: sigmoid(w_s . x)
+ * "Tutorial 11", section 2 (route_topk); "Small MoE Architecture, in depth",
+ * forward of SmallMoE (sigmoid scores, gates from the raw scores). */
+moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router,
+                     const void *w_shared_gate, int32_t *ids, float *gates, float *probs,
+                     float *shared_gate, void *stream);
+
+/* Grouping: counts, offsets and the stable permutation of the T*k
+ * assignments by expert, and its inverse.
+ *   ids         [T, k] int32 in [0, E)   (an id outside sets MOE_ERR_DEVICE_INPUT on
+ *                                          the device flag and leaves outputs unspecified)
+ *   counts      [E] int32 out;  offsets [E + 1] int32 out (offsets[0] = 0)
+ *   sorted_rows [T*k] int32 out: for each expert in turn, its assignments
+ *               r = t*k + j in increasing r
+ *   inv_rows    [T*k] int32 out: inv_rows[sorted_rows[i]] = i
+ * "Tutorial 11", section 3, Step 1 (argsort of the flattened ids; the unsort
+ * index of Step 3 is inv_rows). */
+moe_status moe_permute(const moe_config *cfg, const int32_t *ids, int32_t *counts,
+                       int32_t *offsets, int32_t *sorted_rows, int32_t *inv_rows, void *stream);
+
+/* Grouped gate/up projection with the SwiGLU product fused:
+ *   act[i, :] = silu(W_gate[e] x_t) * (W_up[e] x_t)   for grouped row i of
+ *   expert e, where t = sorted_rows[i] / k.
+ *   x [T, d]; w_gate, w_up [E, h, d]; offsets [E + 1]; sorted_rows [T*k];
+ *   act [T*k, h] out (dtype), grouped order.  Rows of x are read in place by
+ *   index: no copy of x or of any weight is made.
+ * "Tutorial 11", section 3, Step 2 (grouped_expert_linear for gate and up,
+ * silu(gate) * up); the expert of "Small MoE Architecture, in depth". */
+moe_status moe_grouped_swiglu(const moe_config *cfg, const void *x, const void *w_gate,
+                              const void *w_up, const int32_t *offsets,
+                              const int32_t *sorted_rows, void *act, void *stream);
+
+/* Grouped down projection fused with the gate-weighted combine:
+ *   y[t, :] = sum over the k assignments r = t*k + j of gates[r] * W_down[e] act[inv(r), :]
+ *   act [T*k, h] (dtype, grouped order); w_down [E, d, h]; offsets [E + 1];
+ *   sorted_rows [T*k]; gates [T, k] fp32; y [T, d] out (dtype, overwritten).
+ *   ws / ws_bytes: for MOE_BF16 an fp32 accumulator of T*d floats is needed
+ *   (any workspace of moe_workspace_size bytes works); for MOE_F32 ws may be
+ *   NULL.  The summation order over the k experts is not fixed.
+ * "Tutorial 11", section 3, Steps 2-3 (grouped down linear, unsort, weighted
+ * sum over the k experts). */
+moe_status moe_combine(const moe_config *cfg, const void *act, const void *w_down,
+                       const int32_t *offsets, const int32_t *sorted_rows, const float *gates,
+                       void *y, void *ws, size_t ws_bytes, void *stream);
+
+/* The whole layer: route, group, grouped SwiGLU, down projection and combine,
+ * plus the shared expert when cfg->h_shared > 0.
+ *   x [T, d]; w_router [E, d]; w_gate, w_up [E, h, d]; w_down [E, d, h];
+ *   sh_gate, sh_up [h_shared, d], sh_down [d, h_shared], w_shared_gate [d]
+ *   (all four NULL when h_shared == 0); y [T, d] out (dtype).
+ *   ws: device workspace of at least moe_workspace_size(cfg) bytes, 256-byte
+ *   aligned; afterwards it holds the routing results (moe_workspace_layout).
+ * "Tutorial 11", section 4 (Moe.__call__); "Small MoE Architecture, in
+ * depth", SmallMoE.forward (shared expert). */
+moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
+                       const void *w_gate, const void *w_up, const void *w_down,
+                       const void *sh_gate, const void *sh_up, const void *sh_down,
+                       const void *w_shared_gate, void *y, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* Largest T*k that moe_forward serves with the CUDA-core small-batch kernels
+ * (one warp per weight row, weights streamed once); larger batches use the
+ * tensor-core grouped GEMM. */
+int32_t moe_decode_max_rows(void);
+
+/* Stages of moe_forward, in launch order. */
+typedef enum {
+    MOE_STAGE_ROUTE = 0,
+    MOE_STAGE_PERMUTE = 1,
+    MOE_STAGE_GATE_UP = 2,
+    MOE_STAGE_SHARED_GATE_UP = 3,
+    MOE_STAGE_DOWN = 4,
+    MOE_STAGE_SHARED_DOWN = 5,
+    MOE_STAGE_FINALIZE = 6,
+    MOE_STAGE_COUNT = 7
+} moe_stage;
+
+/* Profiling hook for the calling host thread.  With events != NULL (n must be
+ * MOE_STAGE_COUNT + 1 cudaEvent_t handles, created by the caller), every later
+ * moe_forward call on this thread records events[0] on its stream before its
+ * first launch and events[i + 1] after stage i; a stage that does not run
+ * records an empty interval.  events == NULL turns the hook off.  Host only. */
+moe_status moe_profile_events(void *const *events, int32_t n);
+
+/* Number of kernels this library has launched in this process (all threads). */
+int64_t moe_launch_count(void);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * flag: MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_INPUT if a kernel set it
+ * since the last call, MOE_OK otherwise, MOE_ERR_CUDA if the stream itself
+ * reports an error.  Blocking; meant for tests and debugging. */
+moe_status moe_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

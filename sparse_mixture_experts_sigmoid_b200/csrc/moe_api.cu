@@ -1,0 +1,363 @@
+// C ABI of libmoe.so: argument validation, workspace layout and the launch
+// sequence of the MoE layer forward pass.  Declarations and contracts are in
+// include/moe.h.
+#include <atomic>
+#include <mutex>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+// Device error word: kernels OR kErrTimeout / kErrInput into it.
+__device__ uint32_t g_device_error;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+uint32_t *g_err_ptr[kMaxDevices];
+int g_sms[kMaxDevices];
+
+int current_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return -1;
+    return d;
+}
+
+// Device address of g_device_error on the current device (looked up once per device).
+uint32_t *err_ptr() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<uint32_t *>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+enum Part { P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_N };
+
+struct Layout {
+    size_t off[P_N];
+    size_t size[P_N];
+    size_t total;
+};
+
+Layout make_layout(const moe_config &c) {
+    Layout L{};
+    const size_t R = (size_t)c.T * c.k, esz = c.dtype == MOE_F32 ? 4 : 2;
+    L.size[P_IDS] = R * 4;
+    L.size[P_GATES] = R * 4;
+    L.size[P_SG] = c.h_shared > 0 ? (size_t)c.T * 4 : 0;
+    L.size[P_COUNTS] = (size_t)c.E * 4;
+    L.size[P_OFFSETS] = ((size_t)c.E + 1) * 4;
+    L.size[P_SORTED] = R * 4;
+    L.size[P_INV] = R * 4;
+    L.size[P_ACT] = R * (size_t)c.h * esz;
+    L.size[P_ACTS] = c.h_shared > 0 ? (size_t)c.T * c.h_shared * esz : 0;
+    L.size[P_YACC] = c.dtype == MOE_BF16 ? (size_t)c.T * c.d * 4 : 0;
+    size_t o = 0;
+    for (int i = 0; i < P_N; ++i) {
+        L.off[i] = o;
+        o += align256(L.size[i]);
+    }
+    L.total = o;
+    return L;
+}
+
+template <typename T>
+T *part(void *ws, const Layout &L, Part p) {
+    return L.size[p] ? reinterpret_cast<T *>(static_cast<char *>(ws) + L.off[p]) : nullptr;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+std::atomic<int64_t> g_launches{0};
+
+// Per-thread profiling events (moe_profile_events).
+thread_local cudaEvent_t t_events[MOE_STAGE_COUNT + 1];
+thread_local bool t_profile = false;
+
+void mark(int i, cudaStream_t s) {
+    if (t_profile) cudaEventRecord(t_events[i], s);
+}
+
+// The tensor-core grouped GEMM serves batches above this many assignments.
+constexpr int32_t kDecodeMaxRows = 1 << 30;
+
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int num_sms() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_sms[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        g_sms[dev] = v;
+    }
+    return g_sms[dev];
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null pointer, bad size, k outside [1, E] or bad enum";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape outside the library's limits";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace null, misaligned or too small";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
+        case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a kernel's bounded wait ran out";
+        case MOE_ERR_DEVICE_INPUT: return "MOE_ERR_DEVICE_INPUT: a kernel met an invalid device input";
+    }
+    return "unknown moe_status";
+}
+
+moe_status moe_validate(const moe_config *c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (c->T < 0 || c->d < 1 || c->E < 1 || c->h < 1 || c->k < 1 || c->k > c->E || c->h_shared < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (c->dtype != MOE_BF16 && c->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+    if (c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (c->d % 8 || c->h % 8 || c->h_shared % 8) return MOE_ERR_UNSUPPORTED;
+    if (c->T * (int64_t)c->k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    int64_t w = c->d > c->h ? c->d : c->h;
+    if (c->h_shared > w) w = c->h_shared;
+    if (c->T * w >= (int64_t)1 << 40) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_config *c, size_t *bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    *bytes = make_layout(*c).total;
+    return MOE_OK;
+}
+
+moe_status moe_workspace_layout(const moe_config *c, void *ws, size_t ws_bytes, moe_workspace_views *v) {
+    if (!v) return MOE_ERR_INVALID_ARG;
+    const moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    const Layout L = make_layout(*c);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
+    v->ids = part<int32_t>(ws, L, P_IDS);
+    v->gates = part<float>(ws, L, P_GATES);
+    v->shared_gate = part<float>(ws, L, P_SG);
+    v->counts = part<int32_t>(ws, L, P_COUNTS);
+    v->offsets = part<int32_t>(ws, L, P_OFFSETS);
+    v->sorted_rows = part<int32_t>(ws, L, P_SORTED);
+    v->inv_rows = part<int32_t>(ws, L, P_INV);
+    v->act = part<void>(ws, L, P_ACT);
+    v->act_shared = part<void>(ws, L, P_ACTS);
+    v->y_acc = part<float>(ws, L, P_YACC);
+    return MOE_OK;
+}
+
+int32_t moe_decode_max_rows(void) { return kDecodeMaxRows; }
+
+moe_status moe_route(const moe_config *c, const void *x, const void *w_router, const void *w_shared_gate,
+                     int32_t *ids, float *gates, float *probs, float *shared_gate, void *stream) {
+    moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (c->T == 0) return MOE_OK;
+    if (!x || !w_router || !ids || !gates) return MOE_ERR_INVALID_ARG;
+    if (shared_gate && !w_shared_gate) return MOE_ERR_INVALID_ARG;
+    RouterArgs a{};
+    a.x = x;
+    a.w_router = w_router;
+    a.w_shared_gate = shared_gate ? w_shared_gate : nullptr;
+    a.T = c->T;
+    a.d = c->d;
+    a.E = c->E;
+    a.k = c->k;
+    a.norm_topk = c->norm_topk != 0;
+    a.score = c->score;
+    a.ids = ids;
+    a.gates = gates;
+    a.probs = probs;
+    a.shared_gate = shared_gate;
+    a.zero_rows = nullptr;
+    return cuda_status(launch_router(a, c->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(const moe_config *c, const int32_t *ids, int32_t *counts, int32_t *offsets,
+                       int32_t *sorted_rows, int32_t *inv_rows, void *stream) {
+    moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0 && (!ids || !sorted_rows || !inv_rows)) return MOE_ERR_INVALID_ARG;
+    uint32_t *err = err_ptr();
+    if (!err) return MOE_ERR_CUDA;
+    PermuteArgs a{ids, (int)(c->T * c->k), c->E, counts, offsets, sorted_rows, inv_rows, err};
+    return cuda_status(launch_permute(a, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_grouped_swiglu(const moe_config *c, const void *x, const void *w_gate, const void *w_up,
+                              const int32_t *offsets, const int32_t *sorted_rows, void *act, void *stream) {
+    moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (c->T == 0) return MOE_OK;
+    if (!x || !w_gate || !w_up || !offsets || !sorted_rows || !act) return MOE_ERR_INVALID_ARG;
+    uint32_t *err = err_ptr();
+    if (!err) return MOE_ERR_CUDA;
+    SegGateUpArgs a{};
+    a.x = x;
+    a.w_gate = w_gate;
+    a.w_up = w_up;
+    a.seg = Segments{offsets, sorted_rows, c->E, c->k, c->T * c->k};
+    a.T = c->T;
+    a.d = c->d;
+    a.hid = c->h;
+    a.act = act;
+    return cuda_status(launch_seg_gateup(a, c->dtype, static_cast<cudaStream_t>(stream), err));
+}
+
+moe_status moe_combine(const moe_config *c, const void *act, const void *w_down, const int32_t *offsets,
+                       const int32_t *sorted_rows, const float *gates, void *y, void *ws, size_t ws_bytes,
+                       void *stream) {
+    moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (c->T == 0) return MOE_OK;
+    if (!act || !w_down || !offsets || !sorted_rows || !gates || !y) return MOE_ERR_INVALID_ARG;
+    const bool bf16 = c->dtype == MOE_BF16;
+    const size_t need = bf16 ? (size_t)c->T * c->d * 4 : 0;
+    if (bf16 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15))) return MOE_ERR_WORKSPACE;
+    uint32_t *err = err_ptr();
+    if (!err) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *acc = bf16 ? static_cast<float *>(ws) : static_cast<float *>(y);
+    cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)c->T * c->d * 4, s);
+    SegDownArgs a{};
+    a.act = act;
+    a.w_down = w_down;
+    a.seg = Segments{offsets, sorted_rows, c->E, c->k, c->T * c->k};
+    a.T = c->T;
+    a.d = c->d;
+    a.hid = c->h;
+    a.gates = gates;
+    a.y_acc = acc;
+    if (e == cudaSuccess) e = launch_seg_down(a, c->dtype, s, err);
+    if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
+    return cuda_status(e);
+}
+
+moe_status moe_forward(const moe_config *c, const void *x, const void *w_router, const void *w_gate,
+                       const void *w_up, const void *w_down, const void *sh_gate, const void *sh_up,
+                       const void *sh_down, const void *w_shared_gate, void *y, void *ws, size_t ws_bytes,
+                       void *stream) {
+    moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (c->T == 0) return MOE_OK;
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !y) return MOE_ERR_INVALID_ARG;
+    const bool shared = c->h_shared > 0;
+    if (shared && (!sh_gate || !sh_up || !sh_down || !w_shared_gate)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*c);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
+    uint32_t *err = err_ptr();
+    if (!err) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = c->dtype == MOE_BF16;
+
+    int32_t *ids = part<int32_t>(ws, L, P_IDS);
+    float *gates = part<float>(ws, L, P_GATES);
+    float *sg = part<float>(ws, L, P_SG);
+    int32_t *counts = part<int32_t>(ws, L, P_COUNTS);
+    int32_t *offsets = part<int32_t>(ws, L, P_OFFSETS);
+    int32_t *srt = part<int32_t>(ws, L, P_SORTED);
+    int32_t *inv = part<int32_t>(ws, L, P_INV);
+    void *act = part<void>(ws, L, P_ACT);
+    void *acts = part<void>(ws, L, P_ACTS);
+    float *acc = bf16 ? part<float>(ws, L, P_YACC) : static_cast<float *>(y);
+
+    RouterArgs ra{};
+    ra.x = x;
+    ra.w_router = w_router;
+    ra.w_shared_gate = shared ? w_shared_gate : nullptr;
+    ra.T = c->T;
+    ra.d = c->d;
+    ra.E = c->E;
+    ra.k = c->k;
+    ra.norm_topk = c->norm_topk != 0;
+    ra.score = c->score;
+    ra.ids = ids;
+    ra.gates = gates;
+    ra.probs = nullptr;
+    ra.shared_gate = sg;
+    ra.zero_rows = acc;
+    mark(0, s);
+    cudaError_t e = launch_router(ra, c->dtype, s);
+    mark(1 + MOE_STAGE_ROUTE, s);
+
+    const int R = (int)(c->T * c->k);
+    if (e == cudaSuccess) {
+        PermuteArgs pa{ids, R, c->E, counts, offsets, srt, inv, err};
+        e = launch_permute(pa, s);
+    }
+    mark(1 + MOE_STAGE_PERMUTE, s);
+    const Segments routed{offsets, srt, c->E, c->k, (int64_t)R};
+    const Segments dense{nullptr, nullptr, 1, 1, c->T};
+    if (e == cudaSuccess) {
+        SegGateUpArgs ga{x, w_gate, w_up, routed, c->T, c->d, c->h, act};
+        e = launch_seg_gateup(ga, c->dtype, s, err);
+    }
+    mark(1 + MOE_STAGE_GATE_UP, s);
+    if (e == cudaSuccess && shared) {
+        SegGateUpArgs ga{x, sh_gate, sh_up, dense, c->T, c->d, c->h_shared, acts};
+        e = launch_seg_gateup(ga, c->dtype, s, err);
+    }
+    mark(1 + MOE_STAGE_SHARED_GATE_UP, s);
+    if (e == cudaSuccess) {
+        SegDownArgs da{act, w_down, routed, c->T, c->d, c->h, gates, acc};
+        e = launch_seg_down(da, c->dtype, s, err);
+    }
+    mark(1 + MOE_STAGE_DOWN, s);
+    if (e == cudaSuccess && shared) {
+        SegDownArgs da{acts, sh_down, dense, c->T, c->d, c->h_shared, sg, acc};
+        e = launch_seg_down(da, c->dtype, s, err);
+    }
+    mark(1 + MOE_STAGE_SHARED_DOWN, s);
+    if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
+    mark(1 + MOE_STAGE_FINALIZE, s);
+    return cuda_status(e);
+}
+
+moe_status moe_profile_events(void *const *events, int32_t n) {
+    if (!events) {
+        t_profile = false;
+        return MOE_OK;
+    }
+    if (n != MOE_STAGE_COUNT + 1) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i <= MOE_STAGE_COUNT; ++i) {
+        if (!events[i]) return MOE_ERR_INVALID_ARG;
+        t_events[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    t_profile = true;
+    return MOE_OK;
+}
+
+int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+moe_status moe_device_status(void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v & kErrTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+    if (v & kErrInput) return MOE_ERR_DEVICE_INPUT;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,125 @@
+// Internal declarations shared by the CUDA translation units of libmoe.so.
+// Not part of the public ABI (that is include/moe.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Device error flag bits (the flag lives in moe_api.cu; kernels get its address).
+enum : uint32_t { kErrTimeout = 1u, kErrInput = 2u };
+
+// ------------------------------------------------------------------ element helpers
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// Eight consecutive elements as fp32 from one 16-byte (bf16) or two 16-byte (fp32) loads.
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+    float4 a = *reinterpret_cast<const float4 *>(p);
+    float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+// Same, bypassing L1 (streamed once).
+__device__ __forceinline__ void load8_stream(const __nv_bfloat16 *p, float (&v)[8]) {
+    uint4 u = __ldcs(reinterpret_cast<const uint4 *>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void load8_stream(const float *p, float (&v)[8]) {
+    float4 a = __ldcs(reinterpret_cast<const float4 *>(p));
+    float4 b = __ldcs(reinterpret_cast<const float4 *>(p + 4));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ------------------------------------------------------------------ kernel launchers
+// Each returns the launch's cudaError_t (cudaGetLastError after the launch).
+
+struct RouterArgs {
+    const void *x, *w_router, *w_shared_gate;
+    int64_t T;
+    int d, E, k, norm_topk, score;
+    int32_t *ids;
+    float *gates, *probs, *shared_gate;
+    float *zero_rows;   // optional [T, d] fp32 buffer to clear (the combine accumulator)
+};
+cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t s);
+
+struct PermuteArgs {
+    const int32_t *ids;
+    int R, E;
+    int32_t *counts, *offsets, *sorted_rows, *inv_rows;
+    uint32_t *err;
+};
+cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t s);
+
+// A group of rows that one weight set serves: either the routed experts
+// (offsets/sorted_rows give each expert's rows; the token of grouped row i is
+// sorted_rows[i] / k) or one dense segment (the shared expert: row i is token i).
+struct Segments {
+    const int32_t *offsets;      // [E + 1]; NULL for the dense segment
+    const int32_t *sorted_rows;  // [R]; NULL for the dense segment
+    int E, k;                    // experts (1 for dense) and experts per token
+    int64_t rows;                // R for routed, T for dense
+};
+
+struct SegGateUpArgs {
+    const void *x, *w_gate, *w_up;   // x [T, d]; weights [E, hid, d]
+    Segments seg;
+    int64_t T;
+    int d, hid;
+    void *act;                       // [rows, hid]
+};
+cudaError_t launch_seg_gateup(const SegGateUpArgs &a, int dtype, cudaStream_t s, uint32_t *err);
+
+struct SegDownArgs {
+    const void *act, *w_down;        // act [rows, hid]; w_down [E, d, hid]
+    Segments seg;
+    int64_t T;
+    int d, hid;
+    const float *gates;              // routed: [R] gate per assignment; dense: [T] per token
+    float *y_acc;                    // [T, d] fp32, accumulated into
+};
+cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uint32_t *err);
+
+cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s);
+
+int num_sms();
+
+// Counts one kernel launch (for moe_launch_count).
+void note_launch();
+
+}  // namespace moe

@@ -1,0 +1,312 @@
+// Router: fused GEMV (router logits), softmax or sigmoid scoring, register
+// top-k with renormalisation.
+//
+// "Tutorial 11: Mixture of Experts (MoE)", section 2 "The Router" (route_topk:
+// logits = x . W_router^T, softmax over all experts, top-k, gather, optional
+// renormalisation); "Small MoE Architecture, in depth", SmallMoE.forward
+// (sigmoid scores; gates are the kept raw scores).
+//
+// Layout of the work: a CTA of 8 warps owns 8*TW consecutive tokens, each warp
+// TW of them.  W_router (plus the shared-expert gate vector w_s as row E) is
+// streamed through shared memory in chunks of KC columns with a two-stage
+// cp.async pipeline, so every CTA reads W_router from L2 once.  Inside a warp,
+// EL lanes span the experts (lane e % EL holds experts e, e + EL, ...) and
+// CG = 32 / EL lane groups split the chunk's columns; the CG partial sums are
+// folded with shuffles.  All arithmetic is fp32 on exact bf16/fp32 inputs.
+// Selection is k rounds of a warp arg-max over (key, -index), so equal keys
+// resolve to the lower expert index.
+#include <float.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
+    uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+struct Geo {
+    int Ep;     // rows staged: E (+1 for the shared gate)
+    int EL;     // lanes across experts
+    int KC;     // columns per chunk
+    int ldw;    // staged row stride, elements
+};
+
+template <typename Tin>
+__device__ __forceinline__ void stage_chunk(const RouterArgs &a, const Geo &g, Tin *ws, Tin *xs,
+                                            int64_t t0, int NT, int c0) {
+    constexpr int V = 16 / sizeof(Tin);  // elements per 16-byte vector
+    const Tin *wr = static_cast<const Tin *>(a.w_router);
+    const Tin *wsg = static_cast<const Tin *>(a.w_shared_gate);
+    const Tin *x = static_cast<const Tin *>(a.x);
+    const int vpr = g.KC / V;
+    const int nw = g.Ep * vpr;
+    for (int i = threadIdx.x; i < nw; i += kThreads) {
+        int row = i / vpr, col = (i - row * vpr) * V;
+        int gc = c0 + col;
+        const Tin *src = row < a.E ? wr + (int64_t)row * a.d + gc : wsg + gc;
+        bool ok = gc < a.d;
+        cp_async16(ws + row * g.ldw + col, ok ? src : wr, ok ? 16 : 0);
+    }
+    const int nx = NT * vpr;
+    for (int i = threadIdx.x; i < nx; i += kThreads) {
+        int tok = i / vpr, col = (i - tok * vpr) * V;
+        int gc = c0 + col;
+        int64_t t = t0 + tok;
+        bool ok = gc < a.d && t < a.T;
+        cp_async16(xs + tok * g.KC + col, ok ? x + t * a.d + gc : x, ok ? 16 : 0);
+    }
+}
+
+template <typename Tin, int TW, int EPL>
+__global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    constexpr int NT = kWarps * TW;
+    Tin *wbuf[2], *xbuf[2];
+    {
+        Tin *p = reinterpret_cast<Tin *>(smem_raw);
+        const int wsz = g.Ep * g.ldw, xsz = NT * g.KC;
+        wbuf[0] = p;
+        wbuf[1] = p + wsz;
+        xbuf[0] = p + 2 * wsz;
+        xbuf[1] = p + 2 * wsz + xsz;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t0 = (int64_t)blockIdx.x * NT;
+    const int CG = 32 / g.EL;
+    const int cg = lane / g.EL, le = lane % g.EL;
+    const int nchunks = (a.d + g.KC - 1) / g.KC;
+    const int NS = g.KC / 8;
+
+    float acc[TW][EPL];
+#pragma unroll
+    for (int i = 0; i < TW; ++i)
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) acc[i][q] = 0.f;
+
+    stage_chunk<Tin>(a, g, wbuf[0], xbuf[0], t0, NT, 0);
+    cp_async_commit();
+    for (int c = 0; c < nchunks; ++c) {
+        if (c + 1 < nchunks) {
+            stage_chunk<Tin>(a, g, wbuf[(c + 1) & 1], xbuf[(c + 1) & 1], t0, NT, (c + 1) * g.KC);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const Tin *W = wbuf[c & 1];
+        const Tin *X = xbuf[c & 1] + warp * TW * g.KC;
+        for (int s = cg; s < NS; s += CG) {
+            float xv[TW][8];
+#pragma unroll
+            for (int i = 0; i < TW; ++i) load8(X + i * g.KC + s * 8, xv[i]);
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = le + g.EL * q;
+                if (e < g.Ep) {
+                    float w[8];
+                    load8(W + e * g.ldw + s * 8, w);
+#pragma unroll
+                    for (int i = 0; i < TW; ++i) {
+                        float v = acc[i][q];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) v = fmaf(w[u], xv[i][u], v);
+                        acc[i][q] = v;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+    // fold the column groups
+    for (int o = g.EL; o < 32; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < TW; ++i)
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) acc[i][q] += __shfl_xor_sync(0xffffffffu, acc[i][q], o);
+
+    // clear this CTA's rows of the combine accumulator
+    if (a.zero_rows) {
+        const int64_t tend = min(a.T, t0 + NT);
+        const int64_t n4 = (tend - t0) * a.d / 4;
+        float4 *z = reinterpret_cast<float4 *>(a.zero_rows + t0 * a.d);
+        for (int64_t i = threadIdx.x; i < n4; i += kThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    const bool sigm = a.score == MOE_SCORE_SIGMOID;
+#pragma unroll
+    for (int i = 0; i < TW; ++i) {
+        const int64_t t = t0 + warp * TW + i;
+        if (t >= a.T) break;
+        // softmax statistics over the E routed experts
+        float m = -FLT_MAX;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = le + g.EL * q;
+            if (cg == 0 && e < a.E) m = fmaxf(m, acc[i][q]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float z = 0.f;
+        if (!sigm) {
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = le + g.EL * q;
+                if (cg == 0 && e < a.E) z += expf(acc[i][q] - m);
+            }
+            z = warp_sum(z);
+        }
+        float key[EPL];
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) key[q] = sigm ? 1.f / (1.f + expf(-acc[i][q])) : acc[i][q];
+
+        uint32_t taken = 0;
+        int my_e = 0;
+        float my_l = 0.f;
+        for (int j = 0; j < a.k; ++j) {
+            float bk = -FLT_MAX;
+            int be = 0x7fffffff;
+            float bl = 0.f;
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = le + g.EL * q;
+                const bool ok = cg == 0 && e < a.E && !((taken >> q) & 1u);
+                if (ok && (key[q] > bk || (key[q] == bk && e < be))) {
+                    bk = key[q];
+                    be = e;
+                    bl = acc[i][q];
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
+                int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+                if (ok_ > bk || (ok_ == bk && oe < be)) {
+                    bk = ok_;
+                    be = oe;
+                    bl = ol;
+                }
+            }
+            if (be >= a.E) be = j;  // only reachable with non-finite logits; keeps ids in range
+            if (le == be % g.EL && cg == 0) taken |= 1u << (be / g.EL);
+            if (lane == j) {
+                my_e = be;
+                my_l = bl;
+            }
+        }
+        float sc = 0.f;
+        if (lane < a.k) sc = sigm ? 1.f / (1.f + expf(-my_l)) : expf(my_l - m) / z;
+        if (a.norm_topk) {
+            const float ssum = warp_sum(lane < a.k ? sc : 0.f);
+            sc = sc / ssum;
+        }
+        if (lane < a.k) {
+            a.ids[t * a.k + lane] = my_e;
+            a.gates[t * a.k + lane] = sc;
+        }
+        if (a.probs) {
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = le + g.EL * q;
+                if (cg == 0 && e < a.E)
+                    a.probs[t * a.E + e] = sigm ? 1.f / (1.f + expf(-acc[i][q])) : expf(acc[i][q] - m) / z;
+            }
+        }
+        if (a.shared_gate && a.w_shared_gate) {
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = le + g.EL * q;
+                if (cg == 0 && e == a.E) a.shared_gate[t] = 1.f / (1.f + expf(-acc[i][q]));
+            }
+        }
+    }
+}
+
+int pow2ceil(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+template <typename Tin, int TW, int EPL>
+cudaError_t launch_t(const RouterArgs &a, const Geo &g, cudaStream_t s) {
+    constexpr int NT = kWarps * TW;
+    const size_t smem = sizeof(Tin) * (2 * (size_t)g.Ep * g.ldw + 2 * (size_t)NT * g.KC);
+    auto kern = router_kernel<Tin, TW, EPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((a.T + NT - 1) / NT);
+    kern<<<grid, kThreads, smem, s>>>(a, g);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <typename Tin, int EPL>
+cudaError_t launch_e(const RouterArgs &a, const Geo &g, int TW, cudaStream_t s) {
+    if constexpr (EPL <= 8) {
+        if (TW >= 4) return launch_t<Tin, 4, EPL>(a, g, s);
+    }
+    if constexpr (EPL <= 16) {
+        if (TW >= 2) return launch_t<Tin, 2, EPL>(a, g, s);
+    }
+    return launch_t<Tin, 1, EPL>(a, g, s);
+}
+
+template <typename Tin>
+cudaError_t launch_dt(const RouterArgs &a, cudaStream_t s) {
+    Geo g;
+    g.Ep = a.E + (a.w_shared_gate ? 1 : 0);
+    int EPL;
+    if (g.Ep <= 32) {
+        g.EL = pow2ceil(g.Ep < 4 ? 4 : g.Ep);
+        EPL = 1;
+    } else {
+        g.EL = 32;
+        EPL = pow2ceil((g.Ep + 31) / 32);
+    }
+    // chunk width: up to 512 columns while the staged router rows stay near 32 KB
+    const int pad = 16 / (int)sizeof(Tin);
+    int KC = 64;
+    const int dpad = (a.d + 63) / 64 * 64;
+    while (KC < 512 && KC * 2 <= dpad && (size_t)g.Ep * (KC * 2 + pad) * sizeof(Tin) <= 32768) KC *= 2;
+    // wide fp32 rows with many experts: narrower chunks keep two stages under ~150 KB
+    if (2 * (size_t)g.Ep * (KC + pad) * sizeof(Tin) > 150000) KC = 32;
+    g.KC = KC;
+    g.ldw = KC + pad;
+    // tokens per warp: as many as keep at least ~2 CTAs per SM busy
+    const int64_t target = 2LL * num_sms();
+    int TW = 1;
+    if ((a.T + 8 * 4 - 1) / (8 * 4) >= target) TW = 4;
+    else if ((a.T + 8 * 2 - 1) / (8 * 2) >= target) TW = 2;
+    switch (EPL) {
+        case 1: return launch_e<Tin, 1>(a, g, TW, s);
+        case 2: return launch_e<Tin, 2>(a, g, TW, s);
+        case 4: return launch_e<Tin, 4>(a, g, TW, s);
+        case 8: return launch_e<Tin, 8>(a, g, TW, s);
+        case 16: return launch_e<Tin, 16>(a, g, TW, s);
+        case 32: return launch_e<Tin, 32>(a, g, TW, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t s) {
+    if (a.T <= 0) return cudaSuccess;
+    return dtype == MOE_F32 ? launch_dt<float>(a, s) : launch_dt<__nv_bfloat16>(a, s);
+}
+
+}  // namespace moe

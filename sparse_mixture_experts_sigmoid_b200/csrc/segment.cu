@@ -1,0 +1,247 @@
+// Small-batch grouped expert kernels (CUDA cores): one warp per (expert,
+// output row).  The warp streams that weight row once with 16-byte loads and
+// applies it to every grouped row of the expert, so weights are read once per
+// call; this is the bandwidth-bound path for decode-sized batches, where an
+// expert sees a handful of rows and a tensor-core tile would be mostly empty.
+//
+//   gate/up : act[i, n] = silu(W_gate[e, n] . x_t) * (W_up[e, n] . x_t)
+//   down    : y_acc[t, n] += g_i * (W_down[e, n] . act[i])
+//
+// "Tutorial 11: Mixture of Experts (MoE)", section 3, Steps 2-3 (grouped
+// expert linears, silu(gate) * up, weighted sum); "Small MoE Architecture, in
+// depth", Expert.forward (the SwiGLU expert) and the batch-1 decode remarks in
+// "Why small changes the MoE trade-off" (decode reads only the chosen experts).
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int RB = 4;  // grouped rows per pass over a weight row
+
+// Builds, in shared memory, the list of experts that own at least one row.
+__device__ int list_experts(const Segments &sg, int *list, int *beg, int *end) {
+    __shared__ int s_n;
+    if (sg.offsets == nullptr) {
+        if (threadIdx.x == 0) {
+            list[0] = 0;
+            beg[0] = 0;
+            end[0] = (int)sg.rows;
+            s_n = 1;
+        }
+        __syncthreads();
+        return s_n;
+    }
+    if (threadIdx.x == 0) s_n = 0;
+    __syncthreads();
+    // ordered compaction: each warp takes 32 experts at a time
+    for (int base = 0; base < sg.E; base += kThreads) {
+        const int e = base + threadIdx.x;
+        int b = 0, en = 0;
+        bool has = false;
+        if (e < sg.E) {
+            b = sg.offsets[e];
+            en = sg.offsets[e + 1];
+            has = en > b;
+        }
+        __shared__ int wcount[kWarps];
+        const unsigned m = __ballot_sync(0xffffffffu, has);
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        if (lane == 0) wcount[warp] = __popc(m);
+        __syncthreads();
+        int before = s_n;
+        for (int w = 0; w < warp; ++w) before += wcount[w];
+        if (has) {
+            const int pos = before + __popc(m & ((1u << lane) - 1u));
+            list[pos] = e;
+            beg[pos] = b;
+            end[pos] = en;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int add = 0;
+            for (int w = 0; w < kWarps; ++w) add += wcount[w];
+            s_n += add;
+        }
+        __syncthreads();
+    }
+    return s_n;
+}
+
+__device__ __forceinline__ float dot8(const float (&a)[8], const float (&b)[8], float acc) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc = fmaf(a[u], b[u], acc);
+    return acc;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) seg_gateup_kernel(SegGateUpArgs a, uint32_t *err) {
+    extern __shared__ int sm[];
+    int *list = sm, *beg = sm + a.seg.E, *end = sm + 2 * a.seg.E;
+    const int ne = list_experts(a.seg, list, beg, end);
+    const T *x = static_cast<const T *>(a.x);
+    const T *wg = static_cast<const T *>(a.w_gate);
+    const T *wu = static_cast<const T *>(a.w_up);
+    T *act = static_cast<T *>(a.act);
+    const int lane = threadIdx.x & 31;
+    const int64_t nitems = (int64_t)ne * a.hid;
+    const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t nw = (int64_t)gridDim.x * kWarps;
+    for (int64_t item = gw; item < nitems; item += nw) {
+        const int li = (int)(item / a.hid);
+        const int n = (int)(item - (int64_t)li * a.hid);
+        const int e = list[li];
+        const T *grow = wg + ((int64_t)e * a.hid + n) * a.d;
+        const T *urow = wu + ((int64_t)e * a.hid + n) * a.d;
+        for (int r0 = beg[li]; r0 < end[li]; r0 += RB) {
+            int64_t tok[RB];
+#pragma unroll
+            for (int b = 0; b < RB; ++b) {
+                const int r = r0 + b;
+                int64_t t = -1;
+                if (r < end[li]) {
+                    t = a.seg.sorted_rows ? a.seg.sorted_rows[r] / a.seg.k : r;
+                    if (t < 0 || t >= a.T) {
+                        if (lane == 0) atomicOr(err, kErrInput);
+                        t = -1;
+                    }
+                }
+                tok[b] = t;
+            }
+            float ag[RB], au[RB];
+#pragma unroll
+            for (int b = 0; b < RB; ++b) ag[b] = au[b] = 0.f;
+            for (int c = lane * 8; c < a.d; c += 256) {
+                float gv[8], uv[8];
+                load8_stream(grow + c, gv);
+                load8_stream(urow + c, uv);
+#pragma unroll
+                for (int b = 0; b < RB; ++b) {
+                    if (tok[b] >= 0) {
+                        float xv[8];
+                        load8(x + tok[b] * a.d + c, xv);
+                        ag[b] = dot8(gv, xv, ag[b]);
+                        au[b] = dot8(uv, xv, au[b]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < RB; ++b) {
+                const float g = warp_sum(ag[b]);
+                const float u = warp_sum(au[b]);
+                if (lane == b && tok[b] >= 0) act[(int64_t)(r0 + b) * a.hid + n] = from_f32<T>(silu_f(g) * u);
+            }
+        }
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) seg_down_kernel(SegDownArgs a, uint32_t *err) {
+    extern __shared__ int sm[];
+    int *list = sm, *beg = sm + a.seg.E, *end = sm + 2 * a.seg.E;
+    const int ne = list_experts(a.seg, list, beg, end);
+    const T *act = static_cast<const T *>(a.act);
+    const T *wd = static_cast<const T *>(a.w_down);
+    const int lane = threadIdx.x & 31;
+    const int64_t nitems = (int64_t)ne * a.d;
+    const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t nw = (int64_t)gridDim.x * kWarps;
+    for (int64_t item = gw; item < nitems; item += nw) {
+        const int li = (int)(item / a.d);
+        const int n = (int)(item - (int64_t)li * a.d);
+        const int e = list[li];
+        const T *row = wd + ((int64_t)e * a.d + n) * a.hid;
+        for (int r0 = beg[li]; r0 < end[li]; r0 += RB) {
+            float acc[RB];
+#pragma unroll
+            for (int b = 0; b < RB; ++b) acc[b] = 0.f;
+            const int nb = min(RB, end[li] - r0);
+            for (int c = lane * 8; c < a.hid; c += 256) {
+                float wv[8];
+                load8_stream(row + c, wv);
+#pragma unroll
+                for (int b = 0; b < RB; ++b) {
+                    if (b < nb) {
+                        float av[8];
+                        load8(act + (int64_t)(r0 + b) * a.hid + c, av);
+                        acc[b] = dot8(wv, av, acc[b]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < RB; ++b) {
+                const float v = warp_sum(acc[b]);
+                if (lane == b && b < nb) {
+                    const int r = r0 + b;
+                    const int64_t slot = a.seg.sorted_rows ? a.seg.sorted_rows[r] : r;
+                    const int64_t t = a.seg.sorted_rows ? slot / a.seg.k : r;
+                    if (t < 0 || t >= a.T) {
+                        atomicOr(err, kErrInput);
+                    } else {
+                        atomicAdd(a.y_acc + t * a.d + n, a.gates[slot] * v);
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <typename T>
+__global__ void finalize_kernel(const float *y_acc, T *y, int64_t n) {
+    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (i + 8 <= n) {
+        const float4 a = *reinterpret_cast<const float4 *>(y_acc + i);
+        const float4 b = *reinterpret_cast<const float4 *>(y_acc + i + 4);
+        __align__(16) __nv_bfloat16 o[8] = {__float2bfloat16_rn(a.x), __float2bfloat16_rn(a.y),
+                                            __float2bfloat16_rn(a.z), __float2bfloat16_rn(a.w),
+                                            __float2bfloat16_rn(b.x), __float2bfloat16_rn(b.y),
+                                            __float2bfloat16_rn(b.z), __float2bfloat16_rn(b.w)};
+        *reinterpret_cast<uint4 *>(y + i) = *reinterpret_cast<const uint4 *>(o);
+    } else {
+        for (int64_t j = i; j < n; ++j) y[j] = __float2bfloat16_rn(y_acc[j]);
+    }
+}
+
+int grid_for(int64_t items) {
+    const int64_t cap = 4LL * num_sms();
+    const int64_t need = (items + kWarps - 1) / kWarps;
+    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_seg_gateup(const SegGateUpArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
+    if (a.seg.rows <= 0) return cudaSuccess;
+    const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
+    const int grid = grid_for((int64_t)a.seg.E * a.hid);
+    if (dtype == MOE_F32)
+        seg_gateup_kernel<float><<<grid, kThreads, smem, s>>>(a, err);
+    else
+        seg_gateup_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a, err);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
+    if (a.seg.rows <= 0) return cudaSuccess;
+    const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
+    const int grid = grid_for((int64_t)a.seg.E * a.d);
+    if (dtype == MOE_F32)
+        seg_down_kernel<float><<<grid, kThreads, smem, s>>>(a, err);
+    else
+        seg_down_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a, err);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t blocks = (n / 8 + threads) / threads + 1;
+    finalize_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(y_acc, static_cast<__nv_bfloat16 *>(y), n);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,124 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/moe.h declares, and rejects bad arguments before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_mixture_experts_sigmoid_b200 import binding as B
+from sparse_mixture_experts_sigmoid_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert {"moe_route", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward"} <= names
+    L = B.lib()
+    for n in sorted(names):
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert set(B.EXPORTED) <= names
+
+
+def test_status_strings():
+    for s in range(7):
+        assert B.lib().moe_status_string(s).decode().startswith(B.STATUS_NAMES[s])
+    assert b"unknown" in B.lib().moe_status_string(99)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0), 1), (dict(k=9), 1), (dict(T=-1), 1), (dict(d=0), 1), (dict(score=2), 1),
+    (dict(E=513, k=2), 2), (dict(k=17, E=32), 2), (dict(d=12), 2), (dict(h=100), 2),
+    (dict(h_shared=12), 2), (dict(h_shared=-8), 1), (dict(T=1 << 30, k=4), 2),
+])
+def test_validate_rejects(kw, status):
+    base = dict(T=16, d=64, E=8, h=128, k=2, norm_topk=1, score=0, h_shared=0, dtype=0)
+    base.update(kw)
+    cfg = B.MoEConfig(**base)
+    assert B.validate(cfg) == status
+
+
+def test_validate_accepts_all_workloads():
+    for w in WORKLOADS.values():
+        assert B.validate(B.config_of(w)) == 0, w.name
+
+
+def test_null_pointers_rejected_before_launch():
+    cfg = B.config_of(WORKLOADS["tiny"])
+    L = B.lib()
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    assert L.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, None, None, None) == 1
+    assert L.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None) == 1  # shared_gate w/o w_s
+    assert L.moe_permute(ctypes.byref(cfg), fake, None, fake, fake, fake, None) == 1
+    assert L.moe_grouped_swiglu(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, None) == 1
+    assert L.moe_combine(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, None, 0, None) == 1
+    args = [fake] * 5 + [None] * 4 + [fake]
+    assert L.moe_forward(ctypes.byref(cfg), *args, None, 0, None) == 3        # no workspace
+    assert L.moe_forward(ctypes.byref(cfg), *args, P(0x10000), 16, None) == 3  # too small
+    qcfg = B.config_of(WORKLOADS["qwen_shared"])
+    assert L.moe_forward(ctypes.byref(qcfg), *args, P(0x10000), 1 << 40, None) == 1  # shared weights missing
+    bf = B.config(16, 64, 8, 128, 2)
+    assert L.moe_combine(ctypes.byref(bf), fake, fake, fake, fake, fake, fake, None, 0, None) == 3
+
+
+def test_zero_tokens_is_a_no_op():
+    cfg = B.config(0, 64, 8, 128, 2)
+    P = ctypes.c_void_p
+    assert B.lib().moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None) == 0
+    assert B.lib().moe_forward(ctypes.byref(cfg), *([None] * 10), None, 0, None) == 0
+
+
+def test_workspace_layout_is_disjoint_and_aligned():
+    for w in WORKLOADS.values():
+        cfg = B.config_of(w)
+        n = B.workspace_size(cfg)
+        base = 1 << 40
+        v = B.WorkspaceViews()
+        assert B.lib().moe_workspace_layout(ctypes.byref(cfg), ctypes.c_void_p(base), n, ctypes.byref(v)) == 0
+        R = w.T * w.k
+        esz = w.elem_bytes()
+        sizes = {"ids": R * 4, "gates": R * 4, "shared_gate": w.T * 4 if w.h_shared else 0,
+                 "counts": w.E * 4, "offsets": (w.E + 1) * 4, "sorted_rows": R * 4, "inv_rows": R * 4,
+                 "act": R * w.h * esz, "act_shared": w.T * w.h_shared * esz,
+                 "y_acc": w.T * w.d * 4 if w.dtype == "bf16" else 0}
+        spans = []
+        for name, size in sizes.items():
+            p = getattr(v, name)
+            if size == 0:
+                assert not p, name
+                continue
+            assert p % 256 == 0 and base <= p and p + size <= base + n, name
+            spans.append((p, p + size))
+        spans.sort()
+        for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+            assert a1 <= b0
+        # misaligned or short workspaces are refused
+        assert B.lib().moe_workspace_layout(ctypes.byref(cfg), ctypes.c_void_p(base + 16), n,
+                                            ctypes.byref(v)) == 3
+        assert B.lib().moe_workspace_layout(ctypes.byref(cfg), ctypes.c_void_p(base), n - 1,
+                                            ctypes.byref(v)) == 3
+
+
+def test_workspace_never_holds_per_token_weight_copies():
+    """The naive dispatch on "Small models, sparse experts" ("Dispatch decides
+    everything") gathers each token's expert weights: a [2048, 512, 640] fp32
+    tensor, 2.68 GB, for one projection of one layer.  The workspace here holds
+    activations only and must stay orders of magnitude below that."""
+    naive = 2048 * 512 * 640 * 4
+    assert naive == 2_684_354_560
+    w = WORKLOADS["gemma_upcycle"]
+    assert B.workspace_size(B.config_of(w)) < naive / 50

@@ -1,0 +1,53 @@
+"""Measurement arithmetic, pinned to the decode-ceiling worked example printed
+on "Small MoE Architecture, in depth" ("Worked example: the batch-1 budget on
+a device") and to closed forms of the layer's work."""
+import os
+
+import numpy as np
+
+from sparse_mixture_experts_sigmoid_b200 import roofline
+from sparse_mixture_experts_sigmoid_b200.workloads import WORKLOADS
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "decode_ceiling.txt")
+
+
+def test_decode_ceiling_worked_example():
+    rows, params = [], {}
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        parts = line.split()
+        if len(parts) == 2:
+            params[parts[0]] = float(parts[1])
+        else:
+            rows.append((parts[0], *map(float, parts[1:])))
+    assert len(rows) == 3
+    for name, total, active, fp_gb, ceil_tps in rows:
+        fp, tps = roofline.batch1_decode_ceiling(total, active, params["bytes_per_param"], params["mem_gb_s"])
+        assert f"{fp:4.2f}" == f"{fp_gb:4.2f}", name
+        assert round(tps) == ceil_tps, name
+
+
+def test_layer_work_closed_forms():
+    w = WORKLOADS["mixtral_prefill"]
+    counts = np.full(w.E, w.R // w.E)
+    lw = roofline.layer_work(w, counts)
+    assert lw["flops"] == 2.0 * 4096 * 2 * 3 * 4096 * 14336 + 2.0 * 4096 * 8 * 4096
+    # all 8 experts active: 8 * 3 * 14336 * 4096 * 2 bytes of weights, ~2.82 GB
+    assert abs(lw["bytes"] - (8 * 3 * 14336 * 4096 * 2 + 8 * 4096 * 2 + 2 * 4096 * 4096 * 2)) == 0
+    d = WORKLOADS["mixtral_decode"]
+    dw = roofline.layer_work(d, np.r_[1, 1, np.zeros(6)])
+    # decode reads only the two chosen experts: 704.6 MB of expert weights
+    assert abs(2 * 3 * 14336 * 4096 * 2 / 1e6 - 704.6) < 0.1
+    assert dw["bytes"] == 2 * 3 * 14336 * 4096 * 2 + 8 * 4096 * 2 + 2 * 4096 * 2
+    # stage flops add up to the layer's
+    for name in ("gemma_upcycle", "qwen_shared"):
+        w = WORKLOADS[name]
+        sw = roofline.stage_work(w, np.ones(w.E))
+        assert abs(sum(v["flops"] for v in sw.values()) - w.flops()) < 1e-6 * w.flops()
+
+
+def test_peaks_file_or_fallback(tmp_path):
+    p = roofline.measured_peaks(str(tmp_path / "missing.json"))
+    assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0
