@@ -1,0 +1,646 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, TMEM
+// accumulators, TMA), for the variable-size expert segments of a MoE layer.
+//
+//   GATEUP: act[i, n] = silu(W_gate[e, n] . a_i) * (W_up[e, n] . a_i)
+//   DOWN  : y_acc[t_i, n] += g_i * (W_down[e, n] . a_i)
+//
+// where i runs over the grouped rows of expert e.  "Tutorial 11: Mixture of
+// Experts (MoE)", section 3 "Expert Computation" (tokens grouped by expert, a
+// grouped matrix multiply per projection, silu(gate) * up, weighted sum back
+// in token order); "Small models, sparse experts", section "Dispatch decides
+// everything" (read each token's expert weights in place, no gathered weight
+// copies, no padding of groups to a common length).
+//
+// Design (sm_100a):
+//  * Persistent CTAs, one per SM, walk a tile list derived on the device from
+//    the expert offsets: tiles are 128 grouped rows x (128 gate + 128 up
+//    columns) for GATEUP, 128 x 256 for DOWN; expert-major, and inside an
+//    expert the row tiles vary fastest so CTAs running at the same time share
+//    one weight tile through L2.  Partial row tiles at a segment's end are
+//    computed and masked, never padded in memory.
+//  * Warp roles: warps 0-3 epilogue (TMEM lane quarters 0-3), warp 4 TMA
+//    producer, warp 5 TMEM allocator + single-thread MMA issuer, warps 6-9
+//    (gather mode) load token rows x[t] by index with 16-byte cp.async straight
+//    into the 128-byte-swizzled K-major layout that the MMA descriptor reads.
+//  * Weights (and contiguous A operands) arrive by TMA 2D tiles, 128-byte
+//    swizzle, no multicast.  A 4-stage shared-memory ring (48 KB per stage)
+//    is guarded by full/empty mbarriers; the MMA thread frees a stage with
+//    tcgen05.commit.
+//  * One tcgen05.mma.cta_group::1 of M=128, N=256 per 32-byte K slice
+//    (kind::f16 for bf16, kind::tf32 for fp32), fp32 accumulators in TMEM,
+//    double-buffered (2 x 256 columns) so the epilogue of tile i overlaps the
+//    main loop of tile i+1.
+//  * Epilogues: GATEUP reads gate and up columns of the same row from TMEM
+//    (tcgen05.ld 32x32b), applies silu(g)*u and stores act; DOWN scales each
+//    row by its gate and adds it into the fp32 accumulator with 16-byte vector
+//    reductions (the combine over the k experts of a token).
+//  * Every mbarrier wait is bounded (4 s of %globaltimer); on expiry the CTA
+//    raises the device timeout flag, the other roles stop at their next wait,
+//    outstanding copies are drained and TMEM is released before exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * 128;     // one A stage: 128 rows x 128 bytes
+constexpr int kBBytes = 256 * 128;    // one B stage: 256 rows x 128 bytes
+constexpr int kEpiWarps = 4;
+constexpr int kTmaWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kGatherWarp0 = 6;
+constexpr int kGatherThreads = 128;
+constexpr int kLag = 2;               // cp.async groups kept in flight per gather thread
+constexpr int kTmemCols = 512;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+enum { GATEUP = 0, DOWN = 1 };
+
+using Params = GemmParams;
+
+struct Ctrl {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort;
+    int n_mtiles;
+    int pad;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase of parity `parity` to complete.  Returns false if
+// the CTA is aborting or the limit ran out (which raises the device flag).
+__device__ __noinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int *abort, uint32_t *err) {
+    if (mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(b, parity)) return true;
+        if ((i & 63) == 0) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicOr(err, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+template <typename T>
+__device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc);
+template <>
+__device__ __forceinline__ void mma<__nv_bfloat16>(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                   uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+template <>
+__device__ __forceinline__ void mma<float>(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// 32 lanes x 16 columns of 32-bit words from TMEM: thread i gets row (lane base + i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row core groups 1024 bytes apart (SBO), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc(const void *p) {
+    const uint32_t a = smem_u32(p);
+    return (uint64_t)((a & 0x3FFFF) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor: fp32 accumulator, A/B format (1 = bf16, 2 = tf32),
+// both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+template <typename T>
+constexpr uint32_t instr_desc(int M, int N) {
+    constexpr uint32_t fmt = sizeof(T) == 2 ? 1u : 2u;
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ tile list
+
+// One warp: per-expert row-tile counts and their prefix sum (tile_start), and
+// the validated segment offsets (seg_off).  Offsets outside [0, rows] or
+// decreasing are reported and treated as empty segments.
+__device__ void build_tiles(const Params &p, int *tile_start, int *seg_off, int *n_mtiles) {
+    const int lane = threadIdx.x & 31;
+    if (p.offsets == nullptr) {
+        if (lane == 0) {
+            seg_off[0] = 0;
+            seg_off[1] = (int)p.rows;
+            tile_start[0] = 0;
+            tile_start[1] = (int)((p.rows + BM - 1) / BM);
+            *n_mtiles = tile_start[1];
+        }
+        return;
+    }
+    int carry = 0;
+    bool bad = false;
+    for (int base = 0; base < p.E; base += 32) {
+        const int e = base + lane;
+        int b = 0, en = 0;
+        if (e < p.E) {
+            b = p.offsets[e];
+            en = p.offsets[e + 1];
+            if (b < 0 || en < b || en > p.rows) {
+                bad = true;
+                en = b = 0;
+            }
+        }
+        const int mt = (en - b + BM - 1) / BM;
+        int incl = mt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (e < p.E) {
+            tile_start[e] = carry + incl - mt;
+            seg_off[e] = b;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kErrInput);
+    if (lane == 0) {
+        tile_start[p.E] = carry;
+        *n_mtiles = carry;
+    }
+}
+
+struct Tile {
+    int e, m, n;
+};
+
+__device__ __forceinline__ Tile decode(int id, int n_tiles, const int *tile_start, int E) {
+    const int q = id / n_tiles;
+    int lo = 0, hi = E;  // first j in [0, E] with tile_start[j] > q, minus one
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= q) lo = mid;
+        else hi = mid - 1;
+    }
+    // lo = the last index with tile_start[lo] <= q; a run of empty experts shares
+    // its start with the next non-empty one, so lo lands on the expert owning q
+    Tile t;
+    t.e = lo;
+    const int mt = tile_start[lo + 1] - tile_start[lo];
+    const int local = id - tile_start[lo] * n_tiles;
+    t.n = local / mt;
+    t.m = local - t.n * mt;
+    return t;
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int MODE, bool GATHER, typename T>
+__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, Params p) {
+    constexpr int BK = 128 / (int)sizeof(T);   // elements per 128-byte K block
+    constexpr int BN_OUT = MODE == GATEUP ? 128 : 256;
+    constexpr uint32_t kIdesc = instr_desc<T>(BM, 256);
+    constexpr int V = 16 / (int)sizeof(T);     // elements per 16-byte chunk
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + kStages * kABytes;
+    Ctrl *ctrl = reinterpret_cast<Ctrl *>(sB + kStages * kBBytes);
+    int *tile_start = reinterpret_cast<int *>(ctrl + 1);
+    int *seg_off = tile_start + (p.E + 1);
+    int *seg_end = seg_off + (p.E + 1);
+    volatile int *abort = &ctrl->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&ctrl->full[s], GATHER ? 1 + kGatherThreads : 1);
+            mbar_init(&ctrl->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&ctrl->tfull[a], 1);
+            mbar_init(&ctrl->tempty[a], kEpiWarps * 32);
+        }
+        ctrl->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) tmem_alloc(&ctrl->tmem_base, kTmemCols);
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&tmB0);
+            if (MODE == GATEUP) prefetch_tmap(&tmB1);
+            if (!GATHER) prefetch_tmap(&tmA);
+        }
+        build_tiles(p, tile_start, seg_off, &ctrl->n_mtiles);
+        __syncwarp();
+        // per-expert segment ends (offsets validated above)
+        if (p.offsets == nullptr) {
+            if (lane == 0) seg_end[0] = (int)p.rows;
+        } else {
+            for (int e = lane; e < p.E; e += 32) {
+                int b = p.offsets[e], en = p.offsets[e + 1];
+                if (b < 0 || en < b || en > p.rows) en = b = 0;
+                seg_end[e] = en;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = ctrl->tmem_base;
+    const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
+    const int total = ctrl->n_mtiles * n_tiles;
+    const int nk = (p.K + BK - 1) / BK;
+    const int nE = p.offsets ? p.E : 1;
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
+                const Tile tl = decode(id, n_tiles, tile_start, nE);
+                const int a_row = seg_off[tl.e] + tl.m * BM;
+                const int b_row = tl.e * p.N + tl.n * BN_OUT;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!wait_bar(&ctrl->empty[s], ph ^ 1, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(&ctrl->full[s], kBBytes + (GATHER ? 0 : kABytes));
+                    if (!GATHER) tma_load_2d(&tmA, sA + s * kABytes, &ctrl->full[s], kb * BK, a_row);
+                    if (MODE == GATEUP) {
+                        tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
+                        tma_load_2d(&tmB1, sB + s * kBBytes + kBBytes / 2, &ctrl->full[s], kb * BK, b_row);
+                    } else {
+                        tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
+                    }
+                }
+            }
+            if (!ok) {
+                // aborting: let the copies already issued land before the CTA exits
+                for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j) {
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait(&ctrl->full[j % kStages], (j / kStages) & 1) &&
+                           globaltimer() - t0 < 100000000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++tc) {
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * 256;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!wait_bar(&ctrl->full[s], ph, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc(sA + s * kABytes);
+                    const uint64_t bd = smem_desc(sB + s * kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // four 32-byte K slices per 128-byte block
+                        mma<T>(d_tmem, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb | kk) != 0);
+                    mma_commit(&ctrl->empty[s]);
+                }
+                if (ok) mma_commit(&ctrl->tfull[acc]);
+            }
+        }
+    } else if (warp < kEpiWarps) {
+        uint32_t tc = 0;
+        const int row = warp * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        for (int id = blockIdx.x; id < total; id += gridDim.x, ++tc) {
+            const Tile tl = decode(id, n_tiles, tile_start, nE);
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
+            tc_fence_after();
+            const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM + row;
+            const bool valid = r < seg_end[tl.e];
+            const uint32_t tbase = tmem + acc * 256 + lane_base;
+            if constexpr (MODE == GATEUP) {
+                T *act = static_cast<T *>(p.act);
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 16) {
+                    float g[16], u[16];
+                    tmem_ld16(tbase + c, g);
+                    tmem_ld16(tbase + 128 + c, u);
+                    tmem_wait_ld();
+                    const int col = tl.n * 128 + c;
+                    if (valid && col < p.N) {
+                        T *dst = act + r * p.N + col;
+#pragma unroll
+                        for (int h8 = 0; h8 < 2; ++h8) {
+                            if (col + 8 * h8 < p.N) {
+                                if constexpr (sizeof(T) == 2) {
+                                    uint32_t w[4];
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        const int i0 = 8 * h8 + 2 * q;
+                                        __nv_bfloat162 b2 = __floats2bfloat162_rn(silu_f(g[i0]) * u[i0],
+                                                                                  silu_f(g[i0 + 1]) * u[i0 + 1]);
+                                        w[q] = *reinterpret_cast<uint32_t *>(&b2);
+                                    }
+                                    *reinterpret_cast<uint4 *>(dst + 8 * h8) = make_uint4(w[0], w[1], w[2], w[3]);
+                                } else {
+                                    float o[8];
+#pragma unroll
+                                    for (int q = 0; q < 8; ++q) o[q] = silu_f(g[8 * h8 + q]) * u[8 * h8 + q];
+                                    float *fd = reinterpret_cast<float *>(dst + 8 * h8);
+                                    *reinterpret_cast<float4 *>(fd) = make_float4(o[0], o[1], o[2], o[3]);
+                                    *reinterpret_cast<float4 *>(fd + 4) = make_float4(o[4], o[5], o[6], o[7]);
+                                }
+                            }
+                        }
+                    }
+                }
+            } else {
+                int64_t t = -1;
+                float gate = 0.f;
+                if (valid) {
+                    if (p.sorted_rows) {
+                        const int v = p.sorted_rows[r];
+                        t = v / p.k;
+                        gate = (v >= 0 && v < p.rows) ? p.gates[v] : 0.f;
+                    } else {
+                        t = r;
+                        gate = p.gates[r];
+                    }
+                    if (t < 0 || t >= p.T) {
+                        atomicOr(p.err, kErrInput);
+                        t = -1;
+                    }
+                }
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 16) {
+                    float v[16];
+                    tmem_ld16(tbase + c, v);
+                    tmem_wait_ld();
+                    const int col = tl.n * 256 + c;
+                    if (t >= 0) {
+                        float *dst = p.y_acc + t * p.N + col;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (col + 4 * q < p.N)
+                                atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
+                                          make_float4(gate * v[4 * q], gate * v[4 * q + 1], gate * v[4 * q + 2],
+                                                      gate * v[4 * q + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&ctrl->tempty[acc]);
+        }
+    } else if (GATHER && warp >= kGatherWarp0) {
+        const int g = threadIdx.x - kGatherWarp0 * 32;   // 0..127
+        const int c = g & 7;                             // 16-byte chunk of the 128-byte row
+        const int rg = g >> 3;                           // rows rg, rg + 16, ..., rg + 112
+        const int swz = (c ^ (rg & 7)) << 4;             // 128-byte swizzle: chunk ^ (row mod 8)
+        const T *x = static_cast<const T *>(p.x);
+        uint32_t it = 0;
+        int pending = 0;
+        bool ok = true;
+        for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
+            const Tile tl = decode(id, n_tiles, tile_start, nE);
+            const int64_t row0 = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM;
+            const int64_t rend = seg_end[tl.e];
+            const T *src[8];
+            uint32_t okmask = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int64_t r = row0 + rg + 16 * q;
+                src[q] = x;
+                if (r < rend) {
+                    const int v = p.sorted_rows[r];
+                    const int64_t t = v / p.k;
+                    if (v >= 0 && t < p.T) {
+                        src[q] = x + t * p.K + c * V;
+                        okmask |= 1u << q;
+                    } else {
+                        atomicOr(p.err, kErrInput);
+                    }
+                }
+            }
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!wait_bar(&ctrl->empty[s], ph ^ 1, abort, p.err)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *dst = sA + s * kABytes + rg * 128 + swz;
+                const bool colok = kb * BK + c * V < p.K;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (okmask & (1u << q))
+                        cp_async16(dst + q * 16 * 128, colok ? (const void *)(src[q] + kb * BK) : (const void *)x,
+                                   colok ? 16 : 0);
+                cp_async_commit();
+                if (pending == kLag) {
+                    cp_async_wait<kLag>();
+                    fence_proxy_async();
+                    mbar_arrive(&ctrl->full[(it - kLag) % kStages]);
+                } else {
+                    ++pending;
+                }
+            }
+        }
+        cp_async_wait<0>();
+        fence_proxy_async();
+        if (ok)
+            for (uint32_t j = it - pending; j < it; ++j) mbar_arrive(&ctrl->full[j % kStages]);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2D row-major [rows, cols] tensor, box of box_rows x (128 bytes), 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap *m, const void *base, bool f32, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const uint32_t esz = f32 ? 4 : 2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * esz};
+    cuuint32_t box[2] = {128 / esz, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, bool GATHER, typename T>
+cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
+    const Params &p = L.p;
+    constexpr int BN_OUT = MODE == GATEUP ? 128 : 256;
+    const bool f32 = sizeof(T) == 4;
+    CUtensorMap mA, mB0, mB1;
+    const int nE = p.offsets ? p.E : 1;
+    if (!make_map(&mB0, L.b0, f32, (uint64_t)nE * p.N, p.K, MODE == GATEUP ? 128 : 256)) return cudaErrorInvalidValue;
+    if (MODE == GATEUP) {
+        if (!make_map(&mB1, L.b1, f32, (uint64_t)nE * p.N, p.K, 128)) return cudaErrorInvalidValue;
+    } else {
+        mB1 = mB0;
+    }
+    if (!GATHER) {
+        if (!make_map(&mA, L.a_src, f32, (uint64_t)p.rows, p.K, 128)) return cudaErrorInvalidValue;
+    } else {
+        mA = mB0;
+    }
+    const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
+    const int64_t max_m = p.rows / BM + nE;
+    const int64_t max_tiles = max_m * n_tiles;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
+    const size_t smem = 1024 + (size_t)kStages * (kABytes + kBBytes) + sizeof(Ctrl) + 3 * sizeof(int) * (p.E + 1);
+    auto kern = grouped_gemm_kernel<MODE, GATHER, T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, GATHER ? 320 : 192, smem, s>>>(mA, mB0, mB1, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace gg
+
+cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s) {
+    const GemmParams &p = L.p;
+    if (p.rows <= 0) return cudaSuccess;
+    const bool f32 = L.dtype == MOE_F32;
+    if (L.mode == gg::GATEUP) {
+        if (L.gather)
+            return f32 ? gg::launch_t<gg::GATEUP, true, float>(L, s) : gg::launch_t<gg::GATEUP, true, __nv_bfloat16>(L, s);
+        return f32 ? gg::launch_t<gg::GATEUP, false, float>(L, s) : gg::launch_t<gg::GATEUP, false, __nv_bfloat16>(L, s);
+    }
+    return f32 ? gg::launch_t<gg::DOWN, false, float>(L, s) : gg::launch_t<gg::DOWN, false, __nv_bfloat16>(L, s);
+}
+
+}  // namespace moe

@@ -85,8 +85,56 @@ void mark(int i, cudaStream_t s) {
     if (t_profile) cudaEventRecord(t_events[i], s);
 }
 
-// The tensor-core grouped GEMM serves batches above this many assignments.
-constexpr int32_t kDecodeMaxRows = 1 << 30;
+// The tensor-core grouped GEMM serves batches above this many assignments;
+// smaller ones (decode) use the CUDA-core segment kernels.
+constexpr int32_t kDecodeMaxRows = 64;
+
+GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const void *wu, const int32_t *offsets,
+                       const int32_t *srt, void *act, uint32_t *err) {
+    GemmLaunch L{};
+    L.mode = 0;
+    L.gather = true;
+    L.dtype = c.dtype;
+    L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.d, c.h, x, act, nullptr, nullptr, err};
+    L.b0 = wg;
+    L.b1 = wu;
+    return L;
+}
+GemmLaunch gemm_gateup_dense(const moe_config &c, const void *x, const void *wg, const void *wu, void *act,
+                             uint32_t *err) {
+    GemmLaunch L{};
+    L.mode = 0;
+    L.gather = false;
+    L.dtype = c.dtype;
+    L.p = GemmParams{nullptr, nullptr, 1, 1, c.T, c.T, c.d, c.h_shared, x, act, nullptr, nullptr, err};
+    L.a_src = x;
+    L.b0 = wg;
+    L.b1 = wu;
+    return L;
+}
+GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const int32_t *offsets,
+                     const int32_t *srt, const float *gates, float *acc, uint32_t *err) {
+    GemmLaunch L{};
+    L.mode = 1;
+    L.gather = false;
+    L.dtype = c.dtype;
+    L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.h, c.d, nullptr, nullptr, acc, gates, err};
+    L.a_src = act;
+    L.b0 = wd;
+    return L;
+}
+GemmLaunch gemm_down_dense(const moe_config &c, const void *act, const void *wd, const float *sg, float *acc,
+                           uint32_t *err) {
+    GemmLaunch L{};
+    L.mode = 1;
+    L.gather = false;
+    L.dtype = c.dtype;
+    L.p = GemmParams{nullptr, nullptr, 1, 1, c.T, c.T, c.h_shared, c.d, nullptr, nullptr, acc, sg, err};
+    L.a_src = act;
+    L.b0 = wd;
+    return L;
+}
+bool use_gemm(const moe_config &c) { return c.T * c.k > kDecodeMaxRows; }
 
 }  // namespace
 
@@ -221,6 +269,9 @@ moe_status moe_grouped_swiglu(const moe_config *c, const void *x, const void *w_
     a.d = c->d;
     a.hid = c->h;
     a.act = act;
+    if (use_gemm(*c))
+        return cuda_status(launch_grouped_gemm(gemm_gateup(*c, x, w_gate, w_up, offsets, sorted_rows, act, err),
+                                               static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_seg_gateup(a, c->dtype, static_cast<cudaStream_t>(stream), err));
 }
 
@@ -248,7 +299,9 @@ moe_status moe_combine(const moe_config *c, const void *act, const void *w_down,
     a.hid = c->h;
     a.gates = gates;
     a.y_acc = acc;
-    if (e == cudaSuccess) e = launch_seg_down(a, c->dtype, s, err);
+    if (e == cudaSuccess)
+        e = use_gemm(*c) ? launch_grouped_gemm(gemm_down(*c, act, w_down, offsets, sorted_rows, gates, acc, err), s)
+                         : launch_seg_down(a, c->dtype, s, err);
     if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
     return cuda_status(e);
 }
@@ -308,24 +361,29 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     mark(1 + MOE_STAGE_PERMUTE, s);
     const Segments routed{offsets, srt, c->E, c->k, (int64_t)R};
     const Segments dense{nullptr, nullptr, 1, 1, c->T};
+    const bool gemm = use_gemm(*c);
     if (e == cudaSuccess) {
         SegGateUpArgs ga{x, w_gate, w_up, routed, c->T, c->d, c->h, act};
-        e = launch_seg_gateup(ga, c->dtype, s, err);
+        e = gemm ? launch_grouped_gemm(gemm_gateup(*c, x, w_gate, w_up, offsets, srt, act, err), s)
+                 : launch_seg_gateup(ga, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_GATE_UP, s);
     if (e == cudaSuccess && shared) {
         SegGateUpArgs ga{x, sh_gate, sh_up, dense, c->T, c->d, c->h_shared, acts};
-        e = launch_seg_gateup(ga, c->dtype, s, err);
+        e = gemm ? launch_grouped_gemm(gemm_gateup_dense(*c, x, sh_gate, sh_up, acts, err), s)
+                 : launch_seg_gateup(ga, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_SHARED_GATE_UP, s);
     if (e == cudaSuccess) {
         SegDownArgs da{act, w_down, routed, c->T, c->d, c->h, gates, acc};
-        e = launch_seg_down(da, c->dtype, s, err);
+        e = gemm ? launch_grouped_gemm(gemm_down(*c, act, w_down, offsets, srt, gates, acc, err), s)
+                 : launch_seg_down(da, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_DOWN, s);
     if (e == cudaSuccess && shared) {
         SegDownArgs da{acts, sh_down, dense, c->T, c->d, c->h_shared, sg, acc};
-        e = launch_seg_down(da, c->dtype, s, err);
+        e = gemm ? launch_grouped_gemm(gemm_down_dense(*c, acts, sh_down, sg, acc, err), s)
+                 : launch_seg_down(da, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_SHARED_DOWN, s);
     if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);

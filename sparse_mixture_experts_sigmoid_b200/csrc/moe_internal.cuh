@@ -117,6 +117,30 @@ cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uin
 
 cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s);
 
+// Tensor-core grouped GEMM (grouped_gemm.cu).
+struct GemmParams {
+    const int32_t *offsets;      // [E + 1] grouped row offsets; nullptr: one dense segment of `rows` rows
+    const int32_t *sorted_rows;  // grouped row -> assignment t*k + j (routed only)
+    int E, k;
+    int64_t rows;                // grouped rows (R routed, T dense)
+    int64_t T;
+    int K, N;                    // reduction length and output width
+    const void *x;               // gather source [T, K] (gate/up of routed experts)
+    void *act;                   // gate/up output [rows, N]
+    float *y_acc;                // down output [T, N] fp32, accumulated into
+    const float *gates;          // down: routed [R] by assignment, dense [T]
+    uint32_t *err;
+};
+struct GemmLaunch {
+    int mode;             // 0: gate/up with SwiGLU epilogue, 1: down with gate-weighted combine
+    bool gather;          // A rows gathered from x by index (routed gate/up); else TMA from a_src
+    int dtype;            // MOE_BF16 or MOE_F32 (tf32 MMA)
+    GemmParams p;
+    const void *a_src;    // contiguous A operand [rows, K] when !gather
+    const void *b0, *b1;  // weights [E*N, K] (b1: up projection for gate/up)
+};
+cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s);
+
 int num_sms();
 
 // Counts one kernel launch (for moe_launch_count).
