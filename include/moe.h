@@ -165,6 +165,26 @@ moe_status moe_combine(const moe_config *cfg, const void *act, const void *w_dow
                        const int32_t *offsets, const int32_t *sorted_rows, const float *gates,
                        void *y, void *ws, size_t ws_bytes, void *stream);
 
+/* moe_combine without a workspace, for callers that cannot allocate device
+ * memory (for example a plugin inside an engine that pre-plans all device
+ * memory, or code under a fixed memory budget).  The pages have no
+ * counterpart: this is an interface choice of this library.
+ *   Same arguments and result as moe_combine, minus ws / ws_bytes.  For
+ *   MOE_BF16 the fp32 accumulator is a static device array of
+ *   MOE_NOALLOC_MAX_ACC_FLOATS floats (16 MiB) that every GPU loading the
+ *   library holds until exit; T * d above that limit returns
+ *   MOE_ERR_WORKSPACE and enqueues nothing.  The call allocates nothing and
+ *   calls no allocating routine.
+ *   The first call on a device looks up the array's device address (a
+ *   one-time, per-device set-up with that device current); make that first
+ *   call before any stream capture.  All calls share the array and it keeps
+ *   the last call's contents: each call clears the part it uses, and calls
+ *   that overlap on the GPU (unordered streams) race on it. */
+#define MOE_NOALLOC_MAX_ACC_FLOATS (4u << 20)
+moe_status moe_combine_noalloc(const moe_config *cfg, const void *act, const void *w_down,
+                               const int32_t *offsets, const int32_t *sorted_rows, const float *gates,
+                               void *y, void *stream);
+
 /* The whole layer: route, group, grouped SwiGLU, down projection and combine,
  * plus the shared expert when cfg->h_shared > 0.
  *   x [T, d]; w_router [E, d]; w_gate, w_up [E, h, d]; w_down [E, d, h];

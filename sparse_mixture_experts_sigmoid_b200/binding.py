@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_DEVICE_INPUT"}
 EXPORTED = ["moe_status_string", "moe_validate", "moe_workspace_size", "moe_workspace_layout", "moe_route",
             "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_decode_max_rows",
-            "moe_device_status", "moe_profile_events", "moe_launch_count"]
+            "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc"]
 STAGES = ["route", "permute", "gate_up", "shared_gate_up", "down", "shared_down", "finalize"]
 
 
@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "moe_device_status": ([P], ctypes.c_int),
             "moe_profile_events": ([ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32], ctypes.c_int),
             "moe_launch_count": ([], ctypes.c_int64),
+            "moe_combine_noalloc": ([C, P, P, P, P, P, P, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -218,6 +219,21 @@ def combine(cfg: MoEConfig, act, w_down, offsets, sorted_rows, gates, ws=None, s
                              _ptr(gates, "gates", (cfg.T, cfg.k), torch.float32), _ptr(y, "y"),
                              _ptr(ws, "ws"), 0 if ws is None else ws.numel() * ws.element_size(),
                              _stream(stream)), "moe_combine")
+    return y
+
+
+def combine_noalloc(cfg: MoEConfig, act, w_down, offsets, sorted_rows, gates, y=None, stream=None):
+    """moe_combine_noalloc: like combine() but the library's static accumulator
+    replaces the workspace (for callers that cannot allocate device memory)."""
+    et = _elem_dtype(cfg)
+    if y is None:
+        y = torch.empty(cfg.T, cfg.d, dtype=et, device=act.device)
+    _check(lib().moe_combine_noalloc(ctypes.byref(cfg), _ptr(act, "act", (cfg.T * cfg.k, cfg.h), et),
+                                     _ptr(w_down, "w_down", (cfg.E, cfg.d, cfg.h), et),
+                                     _ptr(offsets, "offsets", (cfg.E + 1,), torch.int32),
+                                     _ptr(sorted_rows, "sorted_rows", (cfg.T * cfg.k,), torch.int32),
+                                     _ptr(gates, "gates", (cfg.T, cfg.k), torch.float32),
+                                     _ptr(y, "y", (cfg.T, cfg.d), et), _stream(stream)), "moe_combine_noalloc")
     return y
 
 

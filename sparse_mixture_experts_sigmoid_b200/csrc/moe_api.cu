@@ -138,6 +138,13 @@ bool use_gemm(const moe_config &c) { return c.T * c.k > kDecodeMaxRows; }
 
 }  // namespace
 
+uint32_t *device_error_word() { return err_ptr(); }
+bool gemm_path(const moe_config &c) { return use_gemm(c); }
+GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const int32_t *offsets,
+                     const int32_t *srt, const float *gates, float *acc, uint32_t *err) {
+    return gemm_down(c, act, wd, offsets, srt, gates, acc, err);
+}
+
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int num_sms() {

@@ -141,6 +141,12 @@ struct GemmLaunch {
 };
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s);
 
+// Launch planning shared by the entry points (defined in moe_api.cu).
+uint32_t *device_error_word();   // the library's device error word on the current device
+bool gemm_path(const moe_config &c);   // tensor-core GEMM (true) or segment kernels (false)
+GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const int32_t *offsets,
+                     const int32_t *srt, const float *gates, float *acc, uint32_t *err);
+
 int num_sms();
 
 // Counts one kernel launch (for moe_launch_count).
