@@ -34,10 +34,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
 L2_FLUSH_BYTES = 256 << 20
 # stage -> (kernel name in the ncu launch list, source file whose hash keys the traffic figure)
-STAGE_KERNEL = {"route": ("router_kernel", "router.cu"), "permute": ("permute_kernel", "permute.cu"),
-                "gate_up": ("seg_gateup_kernel", "segment.cu"), "shared_gate_up": ("seg_gateup_kernel", "segment.cu"),
-                "down": ("seg_down_kernel", "segment.cu"), "shared_down": ("seg_down_kernel", "segment.cu"),
+STAGE_KERNEL = {"route": ("router_tc_kernel", "router_tc.cu"), "permute": ("scatter_kernel", "permute.cu"),
+                "gate_up": ("grouped_gemm_kernel", "grouped_gemm.cu"),
+                "shared_gate_up": ("grouped_gemm_kernel", "grouped_gemm.cu"),
+                "down": ("grouped_gemm_kernel", "grouped_gemm.cu"),
+                "shared_down": ("grouped_gemm_kernel", "grouped_gemm.cu"),
                 "finalize": ("finalize_kernel", "segment.cu")}
+# kernels of the small-batch path (at most 64 assignments)
+STAGE_KERNEL_SMALL = {"route": ("router_kernel", "router.cu"), "gate_up": ("seg_gateup_kernel", "segment.cu"),
+                      "down": ("seg_down_kernel", "segment.cu")}
 
 
 def parse():
@@ -213,23 +218,36 @@ def bench_ours(args, w, ws_n, rank, local):
     torch.cuda.synchronize()
     counts = B.workspace_views(cfg, wsbuf)["counts"].cpu().numpy()
 
-    ev = [B.StageEvents() for _ in range(K)]
+    # timed region: K steps, each bracketed by CUDA events on the launching stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     sampler = ClockSampler(local)
     with sampler:
         barrier(ws_n)
         l0 = B.launch_count()
         for i in range(K):
             flush.zero_()
-            with ev[i]:
-                B.forward_layer(cfg, layer, y=y, ws=wsbuf)
+            starts[i].record()
+            B.forward_layer(cfg, layer, y=y, ws=wsbuf)
+            stops[i].record()
         barrier(ws_n)
         launches = B.launch_count() - l0
     assert B.device_status() == 0, "device error flag set during the timed region"
-    step_ms = [e.events[0].elapsed_time(e.events[-1]) for e in ev]
-    stage = {n: statistics.fmean(e.stage_ms()[n] for e in ev) for n in B.STAGES}
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
     ms_local = statistics.fmean(step_ms)
     ms = reduce_max(ms_local, ws_n)
     value = ws_n * w.T / (ms / 1e3)
+
+    # per-kernel breakdown: the same steps again with the library recording an
+    # event after each stage (the dominant kernel's roofline comes from these)
+    ev = [B.StageEvents() for _ in range(K)]
+    barrier(ws_n)
+    for i in range(K):
+        flush.zero_()
+        with ev[i]:
+            B.forward_layer(cfg, layer, y=y, ws=wsbuf)
+    barrier(ws_n)
+    stage = {n: statistics.fmean(e.stage_ms()[n] for e in ev) for n in B.STAGES}
 
     # end to end through the public API: pinned host x in, y back to pinned host
     e2e = None
@@ -269,6 +287,8 @@ def bench_ours(args, w, ws_n, rank, local):
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     t = stage[dom] / 1e3
     kname, ksrc = STAGE_KERNEL[dom]
+    if w.R <= B.decode_max_rows() and dom in STAGE_KERNEL_SMALL:
+        kname, ksrc = STAGE_KERNEL_SMALL[dom]
     if by > 0 and fl / by < ridge:
         roof = {"bound": "hbm", "achieved": by / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:

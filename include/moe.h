@@ -130,15 +130,22 @@ moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router,
 /* Grouping: counts, offsets and the stable permutation of the T*k
  * assignments by expert, and its inverse.
  *   ids         [T, k] int32 in [0, E)   (an id outside sets MOE_ERR_DEVICE_INPUT on
- *                                          the device flag and leaves outputs unspecified)
+ *                                          the device flag, publishes empty experts
+ *                                          and leaves sorted_rows/inv_rows unwritten)
  *   counts      [E] int32 out;  offsets [E + 1] int32 out (offsets[0] = 0)
  *   sorted_rows [T*k] int32 out: for each expert in turn, its assignments
  *               r = t*k + j in increasing r
  *   inv_rows    [T*k] int32 out: inv_rows[sorted_rows[i]] = i
+ *   ws, ws_bytes: device scratch of at least moe_permute_workspace_size(cfg)
+ *               bytes, 16-byte aligned, overlapping no other argument
  * "Tutorial 11", section 3, Step 1 (argsort of the flattened ids; the unsort
  * index of Step 3 is inv_rows). */
 moe_status moe_permute(const moe_config *cfg, const int32_t *ids, int32_t *counts,
-                       int32_t *offsets, int32_t *sorted_rows, int32_t *inv_rows, void *stream);
+                       int32_t *offsets, int32_t *sorted_rows, int32_t *inv_rows, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/* Bytes of scratch that moe_permute needs for cfg (host only). */
+moe_status moe_permute_workspace_size(const moe_config *cfg, size_t *bytes);
 
 /* Grouped gate/up projection with the SwiGLU product fused:
  *   act[i, :] = silu(W_gate[e] x_t) * (W_up[e] x_t)   for grouped row i of

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_DEVICE_INPUT"}
 EXPORTED = ["moe_status_string", "moe_validate", "moe_workspace_size", "moe_workspace_layout", "moe_route",
             "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_decode_max_rows",
-            "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc"]
+            "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size"]
 STAGES = ["route", "permute", "gate_up", "shared_gate_up", "down", "shared_down", "finalize"]
 
 
@@ -62,7 +62,8 @@ def lib() -> ctypes.CDLL:
             "moe_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_workspace_layout": ([C, P, S, ctypes.POINTER(WorkspaceViews)], ctypes.c_int),
             "moe_route": ([C, P, P, P, P, P, P, P, P], ctypes.c_int),
-            "moe_permute": ([C, P, P, P, P, P, P], ctypes.c_int),
+            "moe_permute": ([C, P, P, P, P, P, P, S, P], ctypes.c_int),
+            "moe_permute_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_grouped_swiglu": ([C, P, P, P, P, P, P, P], ctypes.c_int),
             "moe_combine": ([C, P, P, P, P, P, P, P, S, P], ctypes.c_int),
             "moe_forward": ([C, P, P, P, P, P, P, P, P, P, P, P, S, P], ctypes.c_int),
@@ -181,9 +182,17 @@ def route(cfg: MoEConfig, x, w_router, w_shared_gate=None, want_probs=False, str
     return ids, gates, probs, sg
 
 
-def permute(cfg: MoEConfig, ids, stream=None):
+def permute_workspace_size(cfg: MoEConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_permute_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "moe_permute_workspace_size")
+    return n.value
+
+
+def permute(cfg: MoEConfig, ids, ws=None, stream=None):
     """Returns (counts[E], offsets[E+1], sorted_rows[T*k], inv_rows[T*k]), int32."""
     dev = ids.device
+    if ws is None:
+        ws = torch.empty(max(permute_workspace_size(cfg), 16), dtype=torch.uint8, device=dev)
     R = cfg.T * cfg.k
     counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
     offsets = torch.empty(cfg.E + 1, dtype=torch.int32, device=dev)
@@ -191,7 +200,8 @@ def permute(cfg: MoEConfig, ids, stream=None):
     inv = torch.empty(max(R, 1), dtype=torch.int32, device=dev)[:R]
     _check(lib().moe_permute(ctypes.byref(cfg), _ptr(ids, "ids", (cfg.T, cfg.k), torch.int32),
                              _ptr(counts, "counts"), _ptr(offsets, "offsets"), _ptr(srt, "sorted_rows"),
-                             _ptr(inv, "inv_rows"), _stream(stream)), "moe_permute")
+                             _ptr(inv, "inv_rows"), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
+                             _stream(stream)), "moe_permute")
     return counts, offsets, srt, inv
 
 

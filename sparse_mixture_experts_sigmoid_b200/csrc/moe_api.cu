@@ -38,7 +38,7 @@ uint32_t *err_ptr() {
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-enum Part { P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_N };
+enum Part { P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_PERM, P_N };
 
 struct Layout {
     size_t off[P_N];
@@ -59,6 +59,7 @@ Layout make_layout(const moe_config &c) {
     L.size[P_ACT] = R * (size_t)c.h * esz;
     L.size[P_ACTS] = c.h_shared > 0 ? (size_t)c.T * c.h_shared * esz : 0;
     L.size[P_YACC] = c.dtype == MOE_BF16 ? (size_t)c.T * c.d * 4 : 0;
+    L.size[P_PERM] = permute_workspace_bytes((int64_t)R, c.E);
     size_t o = 0;
     for (int i = 0; i < P_N; ++i) {
         L.off[i] = o;
@@ -244,19 +245,32 @@ moe_status moe_route(const moe_config *c, const void *x, const void *w_router, c
     a.probs = probs;
     a.shared_gate = shared_gate;
     a.zero_rows = nullptr;
+    a.err = err_ptr();
+    if (!a.err) return MOE_ERR_CUDA;
     return cuda_status(launch_router(a, c->dtype, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_permute_workspace_size(const moe_config *c, size_t *bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    *bytes = permute_workspace_bytes(c->T * c->k, c->E);
+    return MOE_OK;
+}
+
 moe_status moe_permute(const moe_config *c, const int32_t *ids, int32_t *counts, int32_t *offsets,
-                       int32_t *sorted_rows, int32_t *inv_rows, void *stream) {
+                       int32_t *sorted_rows, int32_t *inv_rows, void *ws, size_t ws_bytes, void *stream) {
     moe_status st = moe_validate(c);
     if (st != MOE_OK) return st;
     if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
     if (c->T > 0 && (!ids || !sorted_rows || !inv_rows)) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0 && (!ws || ws_bytes < permute_workspace_bytes(c->T * c->k, c->E) ||
+                     (reinterpret_cast<uintptr_t>(ws) & 15)))
+        return MOE_ERR_WORKSPACE;
     uint32_t *err = err_ptr();
     if (!err) return MOE_ERR_CUDA;
     PermuteArgs a{ids, (int)(c->T * c->k), c->E, counts, offsets, sorted_rows, inv_rows, err};
-    return cuda_status(launch_permute(a, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_permute(a, static_cast<int32_t *>(ws), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_grouped_swiglu(const moe_config *c, const void *x, const void *w_gate, const void *w_up,
@@ -356,6 +370,7 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     ra.probs = nullptr;
     ra.shared_gate = sg;
     ra.zero_rows = acc;
+    ra.err = err;
     mark(0, s);
     cudaError_t e = launch_router(ra, c->dtype, s);
     mark(1 + MOE_STAGE_ROUTE, s);
@@ -363,7 +378,7 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     const int R = (int)(c->T * c->k);
     if (e == cudaSuccess) {
         PermuteArgs pa{ids, R, c->E, counts, offsets, srt, inv, err};
-        e = launch_permute(pa, s);
+        e = launch_permute(pa, part<int32_t>(ws, L, P_PERM), s);
     }
     mark(1 + MOE_STAGE_PERMUTE, s);
     const Segments routed{offsets, srt, c->E, c->k, (int64_t)R};

@@ -75,8 +75,12 @@ struct RouterArgs {
     int32_t *ids;
     float *gates, *probs, *shared_gate;
     float *zero_rows;   // optional [T, d] fp32 buffer to clear (the combine accumulator)
+    uint32_t *err;      // device error word
 };
+// Tensor-core router (router_tc.cu) when supported, else the CUDA-core router.
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t s);
+bool router_tc_supported(const RouterArgs &a, int dtype);
+cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t s);
 
 struct PermuteArgs {
     const int32_t *ids;
@@ -84,7 +88,9 @@ struct PermuteArgs {
     int32_t *counts, *offsets, *sorted_rows, *inv_rows;
     uint32_t *err;
 };
-cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t s);
+// table: scratch of permute_workspace_bytes(R, E) bytes.
+size_t permute_workspace_bytes(int64_t R, int E);
+cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, cudaStream_t s);
 
 // A group of rows that one weight set serves: either the routed experts
 // (offsets/sorted_rows give each expert's rows; the token of grouped row i is

@@ -6,146 +6,176 @@
 // 3 unsorts with the inverse index); "Small MoE Architecture, in depth"
 // (per-expert load by bincount).
 //
-// One CTA of 32 warps.  Warp w owns the contiguous slice [w*S, (w+1)*S) of the
-// assignments.  Pass 1 counts per (warp, expert) in shared memory; a 32-lane
-// __match_any_sync groups the lanes holding the same expert so one lane adds
-// the group's popcount (no atomics: a warp owns its counter row).  The counts
-// are scanned over warps and over experts, so every (warp, expert) pair knows
-// where its rows start.  Pass 2 walks the slice again in order; a lane's rank
-// inside its match group plus the running per-(warp, expert) cursor is its
-// position, which keeps the order of r inside each expert (stable).
+// Three kernels over blocks of kChunk consecutive assignments:
+//  1. histogram: each CTA counts its block's assignments per expert in shared
+//     memory (lanes holding the same expert are grouped with __match_any_sync
+//     so one lane adds the group's size) and writes one row of a [B, E+1]
+//     table (the last column counts out-of-range ids);
+//  2. scan (one CTA): column sums give the per-expert counts, their exclusive
+//     scan the offsets, and each table entry becomes the position where that
+//     block's rows of that expert start (offset + the counts of earlier blocks);
+//  3. scatter: each CTA ranks its assignments inside the block -- lane rank in
+//     the match group plus the counts of earlier warps for the same expert --
+//     so rows of one expert keep increasing r order (a stable sort by expert).
+// An out-of-range id anywhere makes the scan report MOE_ERR_DEVICE_INPUT and
+// publish empty experts, and the scatter writes nothing.
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kWarps = 32;
-constexpr int kThreads = kWarps * 32;
+constexpr int kChunk = 1024;     // assignments per block
+constexpr int kThreads = 1024;   // one assignment per thread in the scatter
+constexpr int kWarps = kThreads / 32;
 
-__global__ void __launch_bounds__(kThreads) permute_kernel(PermuteArgs a) {
-    extern __shared__ int32_t sm[];
-    int32_t *cnt = sm;                    // [kWarps][E]: counts, then start positions
-    int32_t *tot = sm + kWarps * a.E;     // [E]
-    int32_t *off = tot + a.E;             // [E + 1]
-    __shared__ int32_t warp_tot[kWarps];
-    __shared__ int bad;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i < kWarps * a.E; i += kThreads) cnt[i] = 0;
-    if (threadIdx.x == 0) bad = 0;
+__global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a, int32_t *table) {
+    extern __shared__ int32_t cnt[];   // [E + 1]
+    const int b = blockIdx.x;
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
-
-    const int S = (a.R + kWarps - 1) / kWarps;
-    const int beg = min(a.R, warp * S), end = min(a.R, beg + S);
-    int32_t *mycnt = cnt + warp * a.E;
-
-    // pass 1: per-warp counts
-    for (int base = beg; base < end; base += 32) {
-        const int r = base + lane;
-        int e = r < end ? a.ids[r] : -1;
-        if (r < end && (e < 0 || e >= a.E)) {
-            bad = 1;
-            e = -1;
+    const int beg = b * kChunk, end = min(a.R, beg + kChunk);
+    for (int r0 = beg; r0 < end; r0 += blockDim.x) {
+        const int r = r0 + threadIdx.x;
+        int e = -1;
+        if (r < end) {
+            e = a.ids[r];
+            if (e < 0 || e >= a.E) e = a.E;   // counted in the error column
         }
         const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int leader = __ffs(peers) - 1;
-        if (e >= 0 && lane == leader) mycnt[e] += __popc(peers);
-        __syncwarp();
+        if (e >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&cnt[e], __popc(peers));
     }
     __syncthreads();
-    if (bad) {
-        // invalid input: report it and leave every expert empty so no later
-        // stage reads through an out-of-range index
-        for (int i = threadIdx.x; i <= a.E; i += kThreads) {
+    int32_t *row = table + (int64_t)b * (a.E + 1);
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) row[i] = cnt[i];
+}
+
+// One CTA.  Expert column g of the block table is handled by tpe consecutive
+// threads (a power of two <= 32), thread j summing the contiguous block range
+// [j*S, (j+1)*S); the partial sums are scanned inside the group with shuffles.
+__global__ void __launch_bounds__(1024) scan_kernel(PermuteArgs a, int32_t *table, int nblocks, int tpe) {
+    __shared__ int32_t tots[MOE_MAX_EXPERTS + 1];
+    __shared__ int32_t offs[MOE_MAX_EXPERTS + 1];
+    const int lane = threadIdx.x & 31;
+    const int g = threadIdx.x / tpe, j = threadIdx.x % tpe;
+    const int S = (nblocks + tpe - 1) / tpe;
+    const int b0 = min(nblocks, j * S), b1 = min(nblocks, b0 + S);
+    const bool col = g <= a.E;
+    int local = 0;
+    if (col) {
+#pragma unroll 8
+        for (int b = b0; b < b1; ++b) local += table[(int64_t)b * (a.E + 1) + g];
+    }
+    int incl = local;
+    for (int o = 1; o < tpe; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (j >= o) incl += u;
+    }
+    const int tot = __shfl_sync(0xffffffffu, incl, (lane / tpe) * tpe + tpe - 1);
+    if (col && j == 0) tots[g] = tot;
+    __syncthreads();
+    if (tots[a.E] != 0) {
+        // out-of-range ids: publish empty experts and tell the scatter to stop
+        for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
             a.offsets[i] = 0;
             if (i < a.E) a.counts[i] = 0;
         }
-        if (threadIdx.x == 0) atomicOr(a.err, kErrInput);
+        if (threadIdx.x == 0) {
+            atomicOr(a.err, kErrInput);
+            table[(int64_t)nblocks * (a.E + 1)] = 1;
+        }
         return;
     }
-    // scan over warps for each expert
-    for (int e = threadIdx.x; e < a.E; e += kThreads) {
-        int run = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            const int c = cnt[w * a.E + e];
-            cnt[w * a.E + e] = run;
-            run += c;
-        }
-        tot[e] = run;
-    }
-    __syncthreads();
-    // exclusive scan over experts (E <= 1024 items, chunked per warp)
-    {
-        const int per = (a.E + kThreads - 1) / kThreads;   // items per thread (1 for E <= 1024)
-        int local = 0;
-        const int e0 = threadIdx.x * per;
-        for (int i = 0; i < per; ++i)
-            if (e0 + i < a.E) local += tot[e0 + i];
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) warp_tot[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            int wv = warp_tot[lane];
+    // exclusive scan over experts (warp 0, 32 experts per step)
+    if (threadIdx.x < 32) {
+        int carry = 0;
+        for (int base = 0; base < a.E; base += 32) {
+            const int e = base + lane;
+            const int v = e < a.E ? tots[e] : 0;
+            int in = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, wv, o);
-                if (lane >= o) wv += v;
+                const int u = __shfl_up_sync(0xffffffffu, in, o);
+                if (lane >= o) in += u;
             }
-            warp_tot[lane] = wv;   // inclusive over warps
+            if (e < a.E) offs[e] = carry + in - v;
+            carry += __shfl_sync(0xffffffffu, in, 31);
         }
-        __syncthreads();
-        int run = incl - local + (warp > 0 ? warp_tot[warp - 1] : 0);
-        for (int i = 0; i < per; ++i) {
-            if (e0 + i < a.E) {
-                off[e0 + i] = run;
-                run += tot[e0 + i];
-            }
-        }
-        if (threadIdx.x == kThreads - 1) off[a.E] = warp_tot[kWarps - 1];
+        if (lane == 0) offs[a.E] = carry;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e <= a.E; e += kThreads) {
-        a.offsets[e] = off[e];
-        if (e < a.E) a.counts[e] = tot[e];
-    }
-    // pass 2: stable scatter
-    for (int base = beg; base < end; base += 32) {
-        const int r = base + lane;
-        const int e = r < end ? a.ids[r] : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int leader = __ffs(peers) - 1;
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        int pos = 0;
-        if (e >= 0) pos = off[e] + mycnt[e] + rank;
-        __syncwarp();
-        if (e >= 0) {
-            a.sorted_rows[pos] = r;
-            a.inv_rows[r] = pos;
-            if (lane == leader) mycnt[e] += __popc(peers);
+    if (g < a.E) {
+        if (j == 0) {
+            a.offsets[g] = offs[g];
+            a.counts[g] = tots[g];
         }
-        __syncwarp();
+        int run = offs[g] + incl - local;   // start of block b0's rows of expert g
+        for (int b = b0; b < b1; ++b) {
+            int32_t *p = table + (int64_t)b * (a.E + 1) + g;
+            const int c = *p;
+            *p = run;
+            run += c;
+        }
+    }
+    if (threadIdx.x == 0) {
+        a.offsets[a.E] = offs[a.E];
+        table[(int64_t)nblocks * (a.E + 1)] = 0;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) scatter_kernel(PermuteArgs a, const int32_t *table, int nblocks) {
+    extern __shared__ int32_t wc[];   // [kWarps][E]: per-warp counts, then per-warp starts
+    if (table[(int64_t)nblocks * (a.E + 1)]) return;
+    const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kWarps * a.E; i += kThreads) wc[i] = 0;
+    __syncthreads();
+    const int r = b * kChunk + threadIdx.x;
+    const int e = r < a.R ? a.ids[r] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * a.E + e] = __popc(peers);
+    __syncthreads();
+    const int32_t *base = table + (int64_t)b * (a.E + 1);
+    for (int x = threadIdx.x; x < a.E; x += kThreads) {
+        int run = base[x];
+        for (int w = 0; w < kWarps; ++w) {
+            const int c = wc[w * a.E + x];
+            wc[w * a.E + x] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    if (e >= 0) {
+        const int pos = wc[warp * a.E + e] + rank;
+        a.sorted_rows[pos] = r;
+        a.inv_rows[r] = pos;
     }
 }
 
 }  // namespace
 
-cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t s) {
+size_t permute_workspace_bytes(int64_t R, int E) {
+    const int64_t nblocks = (R + kChunk - 1) / kChunk;
+    return sizeof(int32_t) * ((size_t)nblocks * (E + 1) + 1);
+}
+
+cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, cudaStream_t s) {
     if (a.R <= 0) {
         // no assignments: every expert is empty
         cudaError_t e = cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
         return e;
     }
-    const size_t smem = sizeof(int32_t) * ((size_t)kWarps * a.E + 2 * (size_t)a.E + 1);
-    cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    const int nblocks = (a.R + kChunk - 1) / kChunk;
+    hist_kernel<<<nblocks, 256, sizeof(int32_t) * (a.E + 1), s>>>(a, table);
+    note_launch();
+    int tpe = 1;
+    while (tpe < 32 && 2 * tpe * (a.E + 1) <= 1024 && tpe < nblocks) tpe *= 2;
+    scan_kernel<<<1, 1024, 0, s>>>(a, table, nblocks, tpe);
+    note_launch();
+    const size_t smem = sizeof(int32_t) * (size_t)kWarps * a.E;
+    cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    permute_kernel<<<1, kThreads, smem, s>>>(a);
+    scatter_kernel<<<nblocks, kThreads, smem, s>>>(a, table, nblocks);
     note_launch();
     return cudaGetLastError();
 }

@@ -306,6 +306,7 @@ cudaError_t launch_dt(const RouterArgs &a, cudaStream_t s) {
 
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
+    if (router_tc_supported(a, dtype)) return launch_router_tc(a, s);
     return dtype == MOE_F32 ? launch_dt<float>(a, s) : launch_dt<__nv_bfloat16>(a, s);
 }
 

@@ -63,7 +63,9 @@ def test_null_pointers_rejected_before_launch():
     fake = P(0x1000)
     assert L.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, None, None, None) == 1
     assert L.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None) == 1  # shared_gate w/o w_s
-    assert L.moe_permute(ctypes.byref(cfg), fake, None, fake, fake, fake, None) == 1
+    assert L.moe_permute(ctypes.byref(cfg), fake, None, fake, fake, fake, fake, 1 << 20, None) == 1
+    assert L.moe_permute(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, 0, None) == 3
+    assert L.moe_permute(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, 4, None) == 3
     assert L.moe_grouped_swiglu(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, None) == 1
     assert L.moe_combine(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, None, 0, None) == 1
     args = [fake] * 5 + [None] * 4 + [fake]
@@ -95,6 +97,7 @@ def test_workspace_layout_is_disjoint_and_aligned():
                  "counts": w.E * 4, "offsets": (w.E + 1) * 4, "sorted_rows": R * 4, "inv_rows": R * 4,
                  "act": R * w.h * esz, "act_shared": w.T * w.h_shared * esz,
                  "y_acc": w.T * w.d * 4 if w.dtype == "bf16" else 0}
+        assert n >= sum(sizes.values()) + B.permute_workspace_size(cfg)
         spans = []
         for name, size in sizes.items():
             p = getattr(v, name)
