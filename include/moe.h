@@ -121,11 +121,17 @@ moe_status moe_workspace_layout(const moe_config *cfg, void *ws, size_t ws_bytes
  *   gates    [T, k] fp32   out
  *   probs    [T, E] fp32   out, optional (NULL): every expert's score s_e
  *   shared_gate [T] fp32   out, optional: sigmoid(w_s . x)
+ *   ws, ws_bytes: device scratch of at least moe_route_workspace_size(cfg)
+ *            bytes, 256-byte aligned (may be NULL when that size is 0)
  * "Tutorial 11", section 2 (route_topk); "Small MoE Architecture, in depth",
  * forward of SmallMoE (sigmoid scores, gates from the raw scores). */
 moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router,
                      const void *w_shared_gate, int32_t *ids, float *gates, float *probs,
-                     float *shared_gate, void *stream);
+                     float *shared_gate, void *ws, size_t ws_bytes, void *stream);
+
+/* Bytes of scratch that moe_route needs for cfg (host only; 0 for batches
+ * served by the CUDA-core router). */
+moe_status moe_route_workspace_size(const moe_config *cfg, size_t *bytes);
 
 /* Grouping: counts, offsets and the stable permutation of the T*k
  * assignments by expert, and its inverse.

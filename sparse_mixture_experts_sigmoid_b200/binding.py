@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_DEVICE_INPUT"}
 EXPORTED = ["moe_status_string", "moe_validate", "moe_workspace_size", "moe_workspace_layout", "moe_route",
             "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_decode_max_rows",
-            "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size"]
+            "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size",
+            "moe_route_workspace_size"]
 STAGES = ["route", "permute", "gate_up", "shared_gate_up", "down", "shared_down", "finalize"]
 
 
@@ -61,7 +62,8 @@ def lib() -> ctypes.CDLL:
             "moe_validate": ([C], ctypes.c_int),
             "moe_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_workspace_layout": ([C, P, S, ctypes.POINTER(WorkspaceViews)], ctypes.c_int),
-            "moe_route": ([C, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "moe_route": ([C, P, P, P, P, P, P, P, P, S, P], ctypes.c_int),
+            "moe_route_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_permute": ([C, P, P, P, P, P, P, S, P], ctypes.c_int),
             "moe_permute_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_grouped_swiglu": ([C, P, P, P, P, P, P, P], ctypes.c_int),
@@ -166,10 +168,19 @@ def workspace_views(cfg: MoEConfig, ws: torch.Tensor) -> dict:
     return out
 
 
-def route(cfg: MoEConfig, x, w_router, w_shared_gate=None, want_probs=False, stream=None):
+def route_workspace_size(cfg: MoEConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_route_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "moe_route_workspace_size")
+    return n.value
+
+
+def route(cfg: MoEConfig, x, w_router, w_shared_gate=None, want_probs=False, ws=None, stream=None):
     """Returns (ids[T,k] int32, gates[T,k] f32, probs[T,E] | None, shared_gate[T] | None)."""
     et = _elem_dtype(cfg)
     dev = x.device
+    if ws is None:
+        n = route_workspace_size(cfg)
+        ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
     ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
     gates = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
     probs = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev) if want_probs else None
@@ -177,7 +188,8 @@ def route(cfg: MoEConfig, x, w_router, w_shared_gate=None, want_probs=False, str
     _check(lib().moe_route(ctypes.byref(cfg), _ptr(x, "x", (cfg.T, cfg.d), et),
                            _ptr(w_router, "w_router", (cfg.E, cfg.d), et),
                            _ptr(w_shared_gate, "w_shared_gate", (cfg.d,), et), _ptr(ids, "ids"),
-                           _ptr(gates, "gates"), _ptr(probs, "probs"), _ptr(sg, "shared_gate"), _stream(stream)),
+                           _ptr(gates, "gates"), _ptr(probs, "probs"), _ptr(sg, "shared_gate"), _ptr(ws, "ws"),
+                           0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)),
            "moe_route")
     return ids, gates, probs, sg
 

@@ -38,13 +38,18 @@ uint32_t *err_ptr() {
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-enum Part { P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_PERM, P_N };
+enum Part { P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_PERM, P_LOGITS, P_N };
 
 struct Layout {
     size_t off[P_N];
     size_t size[P_N];
     size_t total;
 };
+
+// Scratch of the tensor-core router (fp32 logits), 0 when the CUDA-core router runs.
+size_t router_scratch_bytes(const moe_config &c) {
+    return router_tc_supported(c.T, c.E, c.dtype) ? router_tc_workspace_bytes(c.T, c.E, c.h_shared > 0) : 0;
+}
 
 Layout make_layout(const moe_config &c) {
     Layout L{};
@@ -60,6 +65,7 @@ Layout make_layout(const moe_config &c) {
     L.size[P_ACTS] = c.h_shared > 0 ? (size_t)c.T * c.h_shared * esz : 0;
     L.size[P_YACC] = c.dtype == MOE_BF16 ? (size_t)c.T * c.d * 4 : 0;
     L.size[P_PERM] = permute_workspace_bytes((int64_t)R, c.E);
+    L.size[P_LOGITS] = router_scratch_bytes(c);
     size_t o = 0;
     for (int i = 0; i < P_N; ++i) {
         L.off[i] = o;
@@ -223,13 +229,24 @@ moe_status moe_workspace_layout(const moe_config *c, void *ws, size_t ws_bytes, 
 
 int32_t moe_decode_max_rows(void) { return kDecodeMaxRows; }
 
+moe_status moe_route_workspace_size(const moe_config *c, size_t *bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    *bytes = router_scratch_bytes(*c);
+    return MOE_OK;
+}
+
 moe_status moe_route(const moe_config *c, const void *x, const void *w_router, const void *w_shared_gate,
-                     int32_t *ids, float *gates, float *probs, float *shared_gate, void *stream) {
+                     int32_t *ids, float *gates, float *probs, float *shared_gate, void *ws, size_t ws_bytes,
+                     void *stream) {
     moe_status st = moe_validate(c);
     if (st != MOE_OK) return st;
     if (c->T == 0) return MOE_OK;
     if (!x || !w_router || !ids || !gates) return MOE_ERR_INVALID_ARG;
     if (shared_gate && !w_shared_gate) return MOE_ERR_INVALID_ARG;
+    const size_t need = router_scratch_bytes(*c);
+    if (need && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255))) return MOE_ERR_WORKSPACE;
     RouterArgs a{};
     a.x = x;
     a.w_router = w_router;
@@ -247,7 +264,8 @@ moe_status moe_route(const moe_config *c, const void *x, const void *w_router, c
     a.zero_rows = nullptr;
     a.err = err_ptr();
     if (!a.err) return MOE_ERR_CUDA;
-    return cuda_status(launch_router(a, c->dtype, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_router(a, c->dtype, need ? static_cast<float *>(ws) : nullptr,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_permute_workspace_size(const moe_config *c, size_t *bytes) {
@@ -369,10 +387,10 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     ra.gates = gates;
     ra.probs = nullptr;
     ra.shared_gate = sg;
-    ra.zero_rows = acc;
+    ra.zero_rows = use_gemm(*c) ? acc : nullptr;   // the small-batch path writes y directly
     ra.err = err;
     mark(0, s);
-    cudaError_t e = launch_router(ra, c->dtype, s);
+    cudaError_t e = launch_router(ra, c->dtype, part<float>(ws, L, P_LOGITS), s);
     mark(1 + MOE_STAGE_ROUTE, s);
 
     const int R = (int)(c->T * c->k);
@@ -396,17 +414,22 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
                  : launch_seg_gateup(ga, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_SHARED_GATE_UP, s);
-    if (e == cudaSuccess) {
-        SegDownArgs da{act, w_down, routed, c->T, c->d, c->h, gates, acc};
-        e = gemm ? launch_grouped_gemm(gemm_down(*c, act, w_down, offsets, srt, gates, acc, err), s)
-                 : launch_seg_down(da, c->dtype, s, err);
+    if (!gemm) {
+        // small batch: down projection, gate-weighted combine and the shared
+        // expert in one pass that writes y
+        if (e == cudaSuccess) {
+            DownDirectArgs da{act, w_down, ids, inv, gates, shared ? acts : nullptr, shared ? sh_down : nullptr,
+                              sg, c->T, c->d, c->h, c->E, c->k, c->h_shared, y};
+            e = launch_down_direct(da, c->dtype, s, err);
+        }
+        mark(1 + MOE_STAGE_DOWN, s);
+        mark(1 + MOE_STAGE_SHARED_DOWN, s);
+        mark(1 + MOE_STAGE_FINALIZE, s);
+        return cuda_status(e);
     }
+    if (e == cudaSuccess) e = launch_grouped_gemm(gemm_down(*c, act, w_down, offsets, srt, gates, acc, err), s);
     mark(1 + MOE_STAGE_DOWN, s);
-    if (e == cudaSuccess && shared) {
-        SegDownArgs da{acts, sh_down, dense, c->T, c->d, c->h_shared, sg, acc};
-        e = gemm ? launch_grouped_gemm(gemm_down_dense(*c, acts, sh_down, sg, acc, err), s)
-                 : launch_seg_down(da, c->dtype, s, err);
-    }
+    if (e == cudaSuccess && shared) e = launch_grouped_gemm(gemm_down_dense(*c, acts, sh_down, sg, acc, err), s);
     mark(1 + MOE_STAGE_SHARED_DOWN, s);
     if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
     mark(1 + MOE_STAGE_FINALIZE, s);

@@ -77,10 +77,12 @@ struct RouterArgs {
     float *zero_rows;   // optional [T, d] fp32 buffer to clear (the combine accumulator)
     uint32_t *err;      // device error word
 };
-// Tensor-core router (router_tc.cu) when supported, else the CUDA-core router.
-cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t s);
-bool router_tc_supported(const RouterArgs &a, int dtype);
-cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t s);
+// Router: the tensor-core logits GEMM + warp-per-token selection (router_tc.cu)
+// when supported and scratch is given, else the CUDA-core routers (router.cu).
+cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaStream_t s);
+bool router_tc_supported(int64_t T, int E, int dtype);
+size_t router_tc_workspace_bytes(int64_t T, int E, bool shared);
+cudaError_t launch_router_tc(const RouterArgs &a, float *scratch, cudaStream_t s);
 
 struct PermuteArgs {
     const int32_t *ids;
@@ -120,6 +122,19 @@ struct SegDownArgs {
     float *y_acc;                    // [T, d] fp32, accumulated into
 };
 cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uint32_t *err);
+
+// Small-batch down projection + combine written straight into y (no accumulator).
+struct DownDirectArgs {
+    const void *act, *w_down;          // act [R, h] grouped order; w_down [E, d, h]
+    const int32_t *ids, *inv_rows;     // [T*k]
+    const float *gates;                // [T*k]
+    const void *act_shared, *sh_down;  // shared expert: act_shared [T, h_shared], sh_down [d, h_shared]; or null
+    const float *shared_gate;          // [T]
+    int64_t T;
+    int d, h, E, k, h_shared;
+    void *y;                           // [T, d]
+};
+cudaError_t launch_down_direct(const DownDirectArgs &a, int dtype, cudaStream_t s, uint32_t *err);
 
 cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s);
 

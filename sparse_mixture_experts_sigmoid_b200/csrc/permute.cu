@@ -18,7 +18,8 @@
 //     the match group plus the counts of earlier warps for the same expert --
 //     so rows of one expert keep increasing r order (a stable sort by expert).
 // An out-of-range id anywhere makes the scan report MOE_ERR_DEVICE_INPUT and
-// publish empty experts, and the scatter writes nothing.
+// publish empty experts, and the scatter writes nothing.  Up to kChunk
+// assignments the three steps run fused in one CTA.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -151,6 +152,74 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(PermuteArgs a, const 
     }
 }
 
+// All three steps in one CTA when every assignment fits in one block
+// (R <= kChunk): per-warp counts, scans over warps and experts, scatter.
+__global__ void __launch_bounds__(kThreads) permute_small_kernel(PermuteArgs a) {
+    extern __shared__ int32_t sm[];
+    int32_t *wc = sm;                       // [kWarps][E]
+    int32_t *tot = sm + kWarps * a.E;       // [E]
+    int32_t *off = tot + a.E;               // [E + 1]
+    __shared__ int bad;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kWarps * a.E; i += kThreads) wc[i] = 0;
+    if (threadIdx.x == 0) bad = 0;
+    __syncthreads();
+    const int r = threadIdx.x;
+    int e = r < a.R ? a.ids[r] : -1;
+    if (r < a.R && (e < 0 || e >= a.E)) {
+        bad = 1;
+        e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * a.E + e] = __popc(peers);
+    __syncthreads();
+    if (bad) {
+        for (int i = threadIdx.x; i <= a.E; i += kThreads) {
+            a.offsets[i] = 0;
+            if (i < a.E) a.counts[i] = 0;
+        }
+        if (threadIdx.x == 0) atomicOr(a.err, kErrInput);
+        return;
+    }
+    for (int x = threadIdx.x; x < a.E; x += kThreads) {
+        int run = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int c = wc[w * a.E + x];
+            wc[w * a.E + x] = run;
+            run += c;
+        }
+        tot[x] = run;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 0; base < a.E; base += 32) {
+            const int x = base + lane;
+            const int v = x < a.E ? tot[x] : 0;
+            int in = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, in, o);
+                if (lane >= o) in += u;
+            }
+            if (x < a.E) off[x] = carry + in - v;
+            carry += __shfl_sync(0xffffffffu, in, 31);
+        }
+        if (lane == 0) off[a.E] = carry;
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x <= a.E; x += kThreads) {
+        a.offsets[x] = off[x];
+        if (x < a.E) a.counts[x] = tot[x];
+    }
+    if (e >= 0) {
+        const int pos = off[e] + wc[warp * a.E + e] + rank;
+        a.sorted_rows[pos] = r;
+        a.inv_rows[r] = pos;
+    }
+}
+
 }  // namespace
 
 size_t permute_workspace_bytes(int64_t R, int E) {
@@ -164,6 +233,15 @@ cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, cudaStream_t s)
         cudaError_t e = cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
         return e;
+    }
+    if (a.R <= kChunk) {
+        const size_t smem = sizeof(int32_t) * ((size_t)kWarps * a.E + 2 * (size_t)a.E + 1);
+        cudaError_t e = cudaFuncSetAttribute(permute_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        permute_small_kernel<<<1, kThreads, smem, s>>>(a);
+        note_launch();
+        return cudaGetLastError();
     }
     const int nblocks = (a.R + kChunk - 1) / kChunk;
     hist_kernel<<<nblocks, 256, sizeof(int32_t) * (a.E + 1), s>>>(a, table);

@@ -24,6 +24,7 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
+constexpr int64_t kSmallT = 64;   // batches up to this many tokens use one CTA per token
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
     uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -235,6 +236,123 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
     }
 }
 
+// Router for small batches: one CTA of 8 warps per token.  The token's row is
+// staged in shared memory as fp32; warp w computes the logits of experts w,
+// w + 8, ... (lane l takes the 8-element slices l, l + 32, ... of the row with
+// 16-byte loads, all issued before the reduction), so the router weights are
+// streamed by the whole CTA at once.  Warp 0 then selects the top k with the
+// same arg-max rounds as the batched router.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
+    extern __shared__ float sm[];
+    float *sx = sm;              // [d] the token's row
+    float *lg = sm + a.d;        // [E + 1] logits (shared gate last)
+    const int64_t t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Tin *x = static_cast<const Tin *>(a.x) + t * a.d;
+    for (int c = threadIdx.x * 8; c < a.d; c += kThreads * 8) {
+        float v[8];
+        load8(x + c, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sx[c + u] = v[u];
+    }
+    if (a.zero_rows) {
+        float4 *z = reinterpret_cast<float4 *>(a.zero_rows + t * a.d);
+        for (int i = threadIdx.x; i < a.d / 4; i += kThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    const Tin *wr = static_cast<const Tin *>(a.w_router);
+    const int Ep = a.E + (a.w_shared_gate ? 1 : 0);
+    for (int e = warp; e < Ep; e += kWarps) {
+        const Tin *row = e < a.E ? wr + (int64_t)e * a.d : static_cast<const Tin *>(a.w_shared_gate);
+        float acc = 0.f;
+#pragma unroll 4
+        for (int c = lane * 8; c < a.d; c += 256) {
+            float w[8];
+            load8(row + c, w);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc = fmaf(w[u], sx[c + u], acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) lg[e] = acc;
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    constexpr int EPL = MOE_MAX_EXPERTS / 32;
+    const bool sigm = a.score == MOE_SCORE_SIGMOID;
+    float l[EPL], key[EPL];
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) {
+        const int e = lane + 32 * q;
+        l[q] = e < a.E ? lg[e] : -FLT_MAX;
+        key[q] = sigm ? 1.f / (1.f + expf(-l[q])) : l[q];
+    }
+    float m = -FLT_MAX;
+#pragma unroll
+    for (int q = 0; q < EPL; ++q)
+        if (lane + 32 * q < a.E) m = fmaxf(m, l[q]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float z = 0.f;
+    if (!sigm) {
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+            if (lane + 32 * q < a.E) z += expf(l[q] - m);
+        z = warp_sum(z);
+    }
+    uint32_t taken = 0;
+    int my_e = 0;
+    float my_l = 0.f;
+    for (int j = 0; j < a.k; ++j) {
+        float bk = -FLT_MAX, bl = 0.f;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane + 32 * q;
+            if (e < a.E && !((taken >> q) & 1u) && (key[q] > bk || (key[q] == bk && e < be))) {
+                bk = key[q];
+                be = e;
+                bl = l[q];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+            if (ok_ > bk || (ok_ == bk && oe < be)) {
+                bk = ok_;
+                be = oe;
+                bl = ol;
+            }
+        }
+        if (be >= a.E) be = j;   // only reachable with non-finite logits; keeps ids in range
+        if (lane == (be & 31)) taken |= 1u << (be >> 5);
+        if (lane == j) {
+            my_e = be;
+            my_l = bl;
+        }
+    }
+    float sc = 0.f;
+    if (lane < a.k) sc = sigm ? 1.f / (1.f + expf(-my_l)) : expf(my_l - m) / z;
+    if (a.norm_topk) {
+        const float ssum = warp_sum(lane < a.k ? sc : 0.f);
+        sc = sc / ssum;
+    }
+    if (lane < a.k) {
+        a.ids[t * a.k + lane] = my_e;
+        a.gates[t * a.k + lane] = sc;
+    }
+    if (a.probs) {
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane + 32 * q;
+            if (e < a.E) a.probs[t * a.E + e] = sigm ? key[q] : expf(l[q] - m) / z;
+        }
+    }
+    if (lane == 0 && a.shared_gate && a.w_shared_gate) a.shared_gate[t] = 1.f / (1.f + expf(-lg[a.E]));
+}
+
 int pow2ceil(int v) {
     int p = 1;
     while (p < v) p <<= 1;
@@ -304,9 +422,25 @@ cudaError_t launch_dt(const RouterArgs &a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t s) {
+cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
-    if (router_tc_supported(a, dtype)) return launch_router_tc(a, s);
+    if (scratch && router_tc_supported(a.T, a.E, dtype)) return launch_router_tc(a, scratch, s);
+    if (a.T <= kSmallT) {
+        const size_t smem = sizeof(float) * ((size_t)a.d + a.E + 1);
+        if (dtype == MOE_F32) {
+            cudaError_t e = cudaFuncSetAttribute(router_small_kernel<float>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            router_small_kernel<float><<<(unsigned)a.T, kThreads, smem, s>>>(a);
+        } else {
+            cudaError_t e = cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            router_small_kernel<__nv_bfloat16><<<(unsigned)a.T, kThreads, smem, s>>>(a);
+        }
+        note_launch();
+        return cudaGetLastError();
+    }
     return dtype == MOE_F32 ? launch_dt<float>(a, s) : launch_dt<__nv_bfloat16>(a, s);
 }
 

@@ -112,7 +112,29 @@ __global__ void __launch_bounds__(kThreads) seg_gateup_kernel(SegGateUpArgs a, u
             float ag[RB], au[RB];
 #pragma unroll
             for (int b = 0; b < RB; ++b) ag[b] = au[b] = 0.f;
-            for (int c = lane * 8; c < a.d; c += 256) {
+            // four 256-column chunks per round: 8 weight loads in flight per lane
+            int c = lane * 8;
+            for (; c + 3 * 256 < a.d; c += 4 * 256) {
+                float gv[4][8], uv[4][8];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    load8_stream(grow + c + u * 256, gv[u]);
+                    load8_stream(urow + c + u * 256, uv[u]);
+                }
+#pragma unroll
+                for (int b = 0; b < RB; ++b) {
+                    if (tok[b] >= 0) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            float xv[8];
+                            load8(x + tok[b] * a.d + c + u * 256, xv);
+                            ag[b] = dot8(gv[u], xv, ag[b]);
+                            au[b] = dot8(uv[u], xv, au[b]);
+                        }
+                    }
+                }
+            }
+            for (; c < a.d; c += 256) {
                 float gv[8], uv[8];
                 load8_stream(grow + c, gv);
                 load8_stream(urow + c, uv);
@@ -187,6 +209,69 @@ __global__ void __launch_bounds__(kThreads) seg_down_kernel(SegDownArgs a, uint3
     }
 }
 
+// Down projection and combine for small batches, written straight into y:
+// one warp per output element (t, n) sums the k selected experts' rows
+//   y[t, n] = sum_j g[t, j] * (W_down[e_j, n] . act[inv(t*k + j)])
+//           (+ sigmoid gate * (S_down[n] . act_shared[t]) with a shared expert),
+// streaming each weight row once with 16-byte loads, four chunks per round.
+// No accumulator, no atomics and no separate conversion pass.
+template <typename T>
+__device__ __forceinline__ float row_dot(const T *w, const T *v, int n, int lane) {
+    float acc = 0.f;
+    int c = lane * 8;
+    for (; c + 3 * 256 < n; c += 4 * 256) {
+        float wv[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) load8_stream(w + c + u * 256, wv[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float av[8];
+            load8(v + c + u * 256, av);
+            acc = dot8(wv[u], av, acc);
+        }
+    }
+    for (; c < n; c += 256) {
+        float wv[8], av[8];
+        load8_stream(w + c, wv);
+        load8(v + c, av);
+        acc = dot8(wv, av, acc);
+    }
+    return acc;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) down_direct_kernel(DownDirectArgs a, uint32_t *err) {
+    const T *act = static_cast<const T *>(a.act);
+    const T *wd = static_cast<const T *>(a.w_down);
+    T *y = static_cast<T *>(a.y);
+    const int lane = threadIdx.x & 31;
+    const int64_t nitems = a.T * a.d;
+    const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t nw = (int64_t)gridDim.x * kWarps;
+    for (int64_t item = gw; item < nitems; item += nw) {
+        const int64_t t = item / a.d;
+        const int n = (int)(item - t * a.d);
+        float acc = 0.f;
+        for (int j = 0; j < a.k; ++j) {
+            const int64_t slot = t * a.k + j;
+            const int e = a.ids[slot];
+            const int r = a.inv_rows[slot];
+            if (e < 0 || e >= a.E || r < 0 || r >= a.T * a.k) {
+                if (lane == 0) atomicOr(err, kErrInput);
+                continue;
+            }
+            acc += a.gates[slot] * row_dot(wd + ((int64_t)e * a.d + n) * a.h, act + (int64_t)r * a.h, a.h, lane);
+        }
+        if (a.sh_down) {
+            const T *sd = static_cast<const T *>(a.sh_down);
+            const T *as = static_cast<const T *>(a.act_shared);
+            acc += a.shared_gate[t] * row_dot(sd + (int64_t)n * a.h_shared, as + t * a.h_shared, a.h_shared, lane);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) y[item] = from_f32<T>(acc);
+    }
+}
+
 template <typename T>
 __global__ void finalize_kernel(const float *y_acc, T *y, int64_t n) {
     const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
@@ -231,6 +316,17 @@ cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uin
         seg_down_kernel<float><<<grid, kThreads, smem, s>>>(a, err);
     else
         seg_down_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a, err);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_down_direct(const DownDirectArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
+    if (a.T <= 0) return cudaSuccess;
+    const int grid = grid_for(a.T * a.d);
+    if (dtype == MOE_F32)
+        down_direct_kernel<float><<<grid, kThreads, 0, s>>>(a, err);
+    else
+        down_direct_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(a, err);
     note_launch();
     return cudaGetLastError();
 }

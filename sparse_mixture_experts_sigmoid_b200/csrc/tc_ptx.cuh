@@ -75,9 +75,26 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *m, void *dst, uin
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
+// Four rows (r0..r3) of a 2D tensor, 128 bytes each at column c0, into four
+// consecutive 128-byte rows of shared memory (swizzled by address as the
+// tensor map says).  The tensor map's box is one row high.
+__device__ __forceinline__ void tma_gather4(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int r0, int r1,
+                                            int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+          "r"(smem_u32(bar))
+        : "memory");
+}
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                  : "memory");
+}
+// Arrive on the barrier when all of this thread's earlier cp.async copies have
+// completed; the arrival counts toward the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N> __device__ __forceinline__ void cp_async_wait() {

@@ -61,8 +61,11 @@ def test_null_pointers_rejected_before_launch():
     L = B.lib()
     P = ctypes.c_void_p
     fake = P(0x1000)
-    assert L.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, None, None, None) == 1
-    assert L.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None) == 1  # shared_gate w/o w_s
+    assert L.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, None, None, None, 0, None) == 1
+    assert L.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None, 0, None) == 1  # no w_s
+    big = B.config_of(WORKLOADS["olmoe_zipf"])
+    assert B.route_workspace_size(big) == 8192 * 64 * 4
+    assert L.moe_route(ctypes.byref(big), fake, fake, None, fake, fake, None, None, None, 0, None) == 3
     assert L.moe_permute(ctypes.byref(cfg), fake, None, fake, fake, fake, fake, 1 << 20, None) == 1
     assert L.moe_permute(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, 0, None) == 3
     assert L.moe_permute(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, 4, None) == 3
@@ -80,7 +83,7 @@ def test_null_pointers_rejected_before_launch():
 def test_zero_tokens_is_a_no_op():
     cfg = B.config(0, 64, 8, 128, 2)
     P = ctypes.c_void_p
-    assert B.lib().moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None) == 0
+    assert B.lib().moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None, 0, None) == 0
     assert B.lib().moe_forward(ctypes.byref(cfg), *([None] * 10), None, 0, None) == 0
 
 
