@@ -52,9 +52,16 @@ namespace gg {
 using namespace tc;
 
 constexpr int BM = 128;
-constexpr int kStages = 4;
 constexpr int kABytes = BM * 128;     // one A stage: 128 rows x 128 bytes
-constexpr int kBBytes = 256 * 128;    // one B stage: 256 rows x 128 bytes
+constexpr int kMaxStages = 8;
+// Shared-memory ring depth for an MMA N of BN: as many stages as fit in 192 KB.
+constexpr int stages_for(int BN) {
+    const int s = 196608 / (kABytes + BN * 128);
+    return s > kMaxStages ? kMaxStages : s;
+}
+#ifndef MOE_GG_L2_PROMOTION
+#define MOE_GG_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
@@ -67,8 +74,8 @@ enum { GATEUP = 0, DOWN = 1 };
 using Params = GemmParams;
 
 struct Ctrl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint32_t tmem_base;
@@ -152,13 +159,15 @@ __device__ __forceinline__ Tile decode(int id, int n_tiles, const int *tile_star
 
 // ------------------------------------------------------------------ kernel
 
-template <int MODE, bool GATHER, typename T>
+template <int MODE, bool GATHER, typename T, int BN>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, Params p) {
     constexpr int BK = 128 / (int)sizeof(T);   // elements per 128-byte K block
-    constexpr int BN_OUT = MODE == GATEUP ? 128 : 256;
-    constexpr uint32_t kIdesc = instr_desc<T>(BM, 256);
+    constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;   // output columns per tile
+    constexpr int kStages = stages_for(BN);
+    constexpr int kBBytes = BN * 128;                      // one B stage: BN rows x 128 bytes
+    constexpr uint32_t kIdesc = instr_desc<T>(BM, BN);
     constexpr int V = 16 / (int)sizeof(T);     // elements per 16-byte chunk
 
     extern __shared__ uint8_t smem_raw[];
@@ -258,7 +267,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
                 if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + acc * 256;
+                const uint32_t d_tmem = tmem + acc * BN;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
@@ -288,16 +297,16 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             tc_fence_after();
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM + row;
             const bool valid = r < seg_end[tl.e];
-            const uint32_t tbase = tmem + acc * 256 + lane_base;
+            const uint32_t tbase = tmem + acc * BN + lane_base;
             if constexpr (MODE == GATEUP) {
                 T *act = static_cast<T *>(p.act);
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 16) {
+                for (int c = 0; c < BN_OUT; c += 16) {
                     float g[16], u[16];
                     tmem_ld16(tbase + c, g);
-                    tmem_ld16(tbase + 128 + c, u);
+                    tmem_ld16(tbase + BN_OUT + c, u);
                     tmem_wait_ld();
-                    const int col = tl.n * 128 + c;
+                    const int col = tl.n * BN_OUT + c;
                     if (valid && col < p.N) {
                         T *dst = act + r * p.N + col;
 #pragma unroll
@@ -343,11 +352,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                     }
                 }
 #pragma unroll 1
-                for (int c = 0; c < 256; c += 16) {
+                for (int c = 0; c < BN; c += 16) {
                     float v[16];
                     tmem_ld16(tbase + c, v);
                     tmem_wait_ld();
-                    const int col = tl.n * 256 + c;
+                    const int col = tl.n * BN + c;
                     if (t >= 0) {
                         float *dst = p.y_acc + t * p.N + col;
 #pragma unroll
@@ -370,20 +379,35 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         const int rg = g >> 3;                           // rows rg, rg + 16, ..., rg + 112
         const int swz = (c ^ (rg & 7)) << 4;             // 128-byte swizzle: chunk ^ (row mod 8)
         const T *x = static_cast<const T *>(p.x);
-        uint32_t it = 0;
-        bool ok = true;
-        for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
+        // the assignment ids of this thread's eight rows, loaded one tile ahead so
+        // the index loads of the next tile overlap the copies of the current one
+        auto load_ids = [&](int id, int (&v)[8]) {
+            if (id >= total) return;
             const Tile tl = decode(id, n_tiles, tile_start, nE);
             const int64_t row0 = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM;
             const int64_t rend = seg_end[tl.e];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int64_t r = row0 + rg + 16 * q;
+                v[q] = r < rend ? p.sorted_rows[r] : -1;
+            }
+        };
+        int vnext[8];
+        load_ids(blockIdx.x, vnext);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
+            int vcur[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) vcur[q] = vnext[q];
+            load_ids(id + gridDim.x, vnext);
             const T *src[8];
             uint32_t okmask = 0;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const int64_t r = row0 + rg + 16 * q;
                 src[q] = x;
-                if (r < rend) {
-                    const int v = p.sorted_rows[r];
+                const int v = vcur[q];
+                if (v != -1) {
                     const int64_t t = v / p.k;
                     if (v >= 0 && t < p.T) {
                         src[q] = x + t * p.K + c * V;
@@ -423,16 +447,18 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
 // ------------------------------------------------------------------ host side
 
-template <int MODE, bool GATHER, typename T>
+template <int MODE, bool GATHER, typename T, int BN>
 cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
     const Params &p = L.p;
-    constexpr int BN_OUT = MODE == GATEUP ? 128 : 256;
+    constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
+    constexpr int kStages = stages_for(BN);
     const bool f32 = sizeof(T) == 4;
     CUtensorMap mA, mB0, mB1;
     const int nE = p.offsets ? p.E : 1;
-    if (!make_map(&mB0, L.b0, f32, (uint64_t)nE * p.N, p.K, MODE == GATEUP ? 128 : 256)) return cudaErrorInvalidValue;
+    const CUtensorMapL2promotion wp = MOE_GG_L2_PROMOTION;
+    if (!make_map(&mB0, L.b0, f32, (uint64_t)nE * p.N, p.K, BN_OUT, wp)) return cudaErrorInvalidValue;
     if (MODE == GATEUP) {
-        if (!make_map(&mB1, L.b1, f32, (uint64_t)nE * p.N, p.K, 128)) return cudaErrorInvalidValue;
+        if (!make_map(&mB1, L.b1, f32, (uint64_t)nE * p.N, p.K, BN_OUT, wp)) return cudaErrorInvalidValue;
     } else {
         mB1 = mB0;
     }
@@ -445,13 +471,18 @@ cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
     const int64_t max_m = p.rows / BM + nE;
     const int64_t max_tiles = max_m * n_tiles;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
-    const size_t smem = 1024 + (size_t)kStages * (kABytes + kBBytes) + sizeof(Ctrl) + 3 * sizeof(int) * (p.E + 1);
-    auto kern = grouped_gemm_kernel<MODE, GATHER, T>;
+    const size_t smem = 1024 + (size_t)kStages * (kABytes + BN * 128) + sizeof(Ctrl) + 3 * sizeof(int) * (p.E + 1);
+    auto kern = grouped_gemm_kernel<MODE, GATHER, T, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, GATHER ? 320 : 192, smem, s>>>(mA, mB0, mB1, p);
     note_launch();
     return cudaGetLastError();
+}
+
+template <int MODE, bool GATHER, typename T>
+cudaError_t launch_bn(const GemmLaunch &L, cudaStream_t s) {
+    return L.narrow ? launch_t<MODE, GATHER, T, 128>(L, s) : launch_t<MODE, GATHER, T, 256>(L, s);
 }
 
 }  // namespace gg
@@ -462,10 +493,12 @@ cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s) {
     const bool f32 = L.dtype == MOE_F32;
     if (L.mode == gg::GATEUP) {
         if (L.gather)
-            return f32 ? gg::launch_t<gg::GATEUP, true, float>(L, s) : gg::launch_t<gg::GATEUP, true, __nv_bfloat16>(L, s);
-        return f32 ? gg::launch_t<gg::GATEUP, false, float>(L, s) : gg::launch_t<gg::GATEUP, false, __nv_bfloat16>(L, s);
+            return f32 ? gg::launch_bn<gg::GATEUP, true, float>(L, s)
+                       : gg::launch_bn<gg::GATEUP, true, __nv_bfloat16>(L, s);
+        return f32 ? gg::launch_bn<gg::GATEUP, false, float>(L, s)
+                   : gg::launch_bn<gg::GATEUP, false, __nv_bfloat16>(L, s);
     }
-    return f32 ? gg::launch_t<gg::DOWN, false, float>(L, s) : gg::launch_t<gg::DOWN, false, __nv_bfloat16>(L, s);
+    return f32 ? gg::launch_bn<gg::DOWN, false, float>(L, s) : gg::launch_bn<gg::DOWN, false, __nv_bfloat16>(L, s);
 }
 
 }  // namespace moe

@@ -96,6 +96,16 @@ void mark(int i, cudaStream_t s) {
 // smaller ones (decode) use the CUDA-core segment kernels.
 constexpr int32_t kDecodeMaxRows = 64;
 
+#ifndef MOE_NARROW_TILES
+#define MOE_NARROW_TILES 0
+#endif
+#ifndef MOE_NARROW_ROWS_PER_EXPERT
+#define MOE_NARROW_ROWS_PER_EXPERT 128
+#endif
+// Few rows per expert make the expert GEMMs weight-streaming (HBM) bound:
+// narrower N tiles give more tiles and a deeper ring of loads in flight.
+bool narrow_tiles(const moe_config &c) { return c.T * c.k < (int64_t)MOE_NARROW_ROWS_PER_EXPERT * c.E; }
+
 GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const void *wu, const int32_t *offsets,
                        const int32_t *srt, void *act, uint32_t *err) {
     GemmLaunch L{};
@@ -103,6 +113,7 @@ GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const
     L.gather = true;
     L.dtype = c.dtype;
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.d, c.h, x, act, nullptr, nullptr, err};
+    L.narrow = narrow_tiles(c) && MOE_NARROW_TILES;
     L.b0 = wg;
     L.b1 = wu;
     return L;
@@ -126,6 +137,7 @@ GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const
     L.gather = false;
     L.dtype = c.dtype;
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.h, c.d, nullptr, nullptr, acc, gates, err};
+    L.narrow = narrow_tiles(c) && MOE_NARROW_TILES;
     L.a_src = act;
     L.b0 = wd;
     return L;
@@ -142,6 +154,7 @@ GemmLaunch gemm_down_dense(const moe_config &c, const void *act, const void *wd,
     return L;
 }
 bool use_gemm(const moe_config &c) { return c.T * c.k > kDecodeMaxRows; }
+
 
 }  // namespace
 
@@ -288,7 +301,7 @@ moe_status moe_permute(const moe_config *c, const int32_t *ids, int32_t *counts,
     uint32_t *err = err_ptr();
     if (!err) return MOE_ERR_CUDA;
     PermuteArgs a{ids, (int)(c->T * c->k), c->E, counts, offsets, sorted_rows, inv_rows, err};
-    return cuda_status(launch_permute(a, static_cast<int32_t *>(ws), static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_permute(a, static_cast<int32_t *>(ws), false, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_grouped_swiglu(const moe_config *c, const void *x, const void *w_gate, const void *w_up,
@@ -389,6 +402,10 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     ra.shared_gate = sg;
     ra.zero_rows = use_gemm(*c) ? acc : nullptr;   // the small-batch path writes y directly
     ra.err = err;
+    // the tensor-core router also builds the grouping histogram
+    const bool fused_hist = L.size[P_LOGITS] && c->T * c->k > permute_chunk();
+    ra.hist = fused_hist ? part<int32_t>(ws, L, P_PERM) : nullptr;
+    ra.hist_chunk = permute_chunk();
     mark(0, s);
     cudaError_t e = launch_router(ra, c->dtype, part<float>(ws, L, P_LOGITS), s);
     mark(1 + MOE_STAGE_ROUTE, s);
@@ -396,7 +413,7 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     const int R = (int)(c->T * c->k);
     if (e == cudaSuccess) {
         PermuteArgs pa{ids, R, c->E, counts, offsets, srt, inv, err};
-        e = launch_permute(pa, part<int32_t>(ws, L, P_PERM), s);
+        e = launch_permute(pa, part<int32_t>(ws, L, P_PERM), fused_hist, s);
     }
     mark(1 + MOE_STAGE_PERMUTE, s);
     const Segments routed{offsets, srt, c->E, c->k, (int64_t)R};

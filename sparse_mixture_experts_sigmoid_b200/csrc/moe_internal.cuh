@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/moe.h"
+#include "moe.h"  // include/ is on the include path
 
 namespace moe {
 
@@ -57,7 +57,10 @@ __device__ __forceinline__ void load8_stream(const float *p, float (&v)[8]) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-__device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
+// silu(u) = u * sigmoid(u) = u / (1 + exp(-u)).  The fast divide is exact enough
+// here: for u < -87 the denominator overflows to +inf or past 2^126 and the
+// result flushes to zero, which is silu's limit there.
+__device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -76,6 +79,8 @@ struct RouterArgs {
     float *gates, *probs, *shared_gate;
     float *zero_rows;   // optional [T, d] fp32 buffer to clear (the combine accumulator)
     uint32_t *err;      // device error word
+    int32_t *hist;      // optional [B, E+1] block histogram for grouping (tensor-core router only)
+    int hist_chunk;     // assignments per histogram block
 };
 // Router: the tensor-core logits GEMM + warp-per-token selection (router_tc.cu)
 // when supported and scratch is given, else the CUDA-core routers (router.cu).
@@ -90,9 +95,11 @@ struct PermuteArgs {
     int32_t *counts, *offsets, *sorted_rows, *inv_rows;
     uint32_t *err;
 };
-// table: scratch of permute_workspace_bytes(R, E) bytes.
+// table: scratch of permute_workspace_bytes(R, E) bytes, a [B, E+1] histogram of
+// blocks of permute_chunk() assignments; table_ready: the router already filled it.
 size_t permute_workspace_bytes(int64_t R, int E);
-cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, cudaStream_t s);
+int permute_chunk();
+cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, bool table_ready, cudaStream_t s);
 
 // A group of rows that one weight set serves: either the routed experts
 // (offsets/sorted_rows give each expert's rows; the token of grouped row i is
@@ -156,6 +163,7 @@ struct GemmLaunch {
     int mode;             // 0: gate/up with SwiGLU epilogue, 1: down with gate-weighted combine
     bool gather;          // A rows gathered from x by index (routed gate/up); else TMA from a_src
     int dtype;            // MOE_BF16 or MOE_F32 (tf32 MMA)
+    bool narrow;          // MMA N = 128 and a deeper ring (few rows per expert) instead of N = 256
     GemmParams p;
     const void *a_src;    // contiguous A operand [rows, K] when !gather
     const void *b0, *b1;  // weights [E*N, K] (b1: up projection for gate/up)

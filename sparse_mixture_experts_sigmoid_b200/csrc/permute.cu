@@ -6,20 +6,21 @@
 // 3 unsorts with the inverse index); "Small MoE Architecture, in depth"
 // (per-expert load by bincount).
 //
-// Three kernels over blocks of kChunk consecutive assignments:
-//  1. histogram: each CTA counts its block's assignments per expert in shared
-//     memory (lanes holding the same expert are grouped with __match_any_sync
-//     so one lane adds the group's size) and writes one row of a [B, E+1]
-//     table (the last column counts out-of-range ids);
-//  2. scan (one CTA): column sums give the per-expert counts, their exclusive
-//     scan the offsets, and each table entry becomes the position where that
-//     block's rows of that expert start (offset + the counts of earlier blocks);
-//  3. scatter: each CTA ranks its assignments inside the block -- lane rank in
-//     the match group plus the counts of earlier warps for the same expert --
-//     so rows of one expert keep increasing r order (a stable sort by expert).
-// An out-of-range id anywhere makes the scan report MOE_ERR_DEVICE_INPUT and
-// publish empty experts, and the scatter writes nothing.  Up to kChunk
-// assignments the three steps run fused in one CTA.
+// Over blocks of kChunk consecutive assignments:
+//  1. histogram: per block and expert, the number of assignments, in a
+//     [B, E+1] table (the last column counts out-of-range ids).  Either the
+//     histogram kernel below builds it (each CTA counts its block in shared
+//     memory; lanes holding the same expert are grouped with __match_any_sync
+//     so one lane adds the group's size) or the router's selection kernel
+//     accumulates it while it writes the ids.
+//  2. scan + scatter: each CTA derives the per-expert counts, their exclusive
+//     scan (the offsets) and its block's start for each expert from the table,
+//     then ranks its assignments inside the block -- lane rank in the match
+//     group plus the counts of earlier warps for the same expert -- so rows of
+//     one expert keep increasing r order (a stable sort by expert).
+// An out-of-range id anywhere reports MOE_ERR_DEVICE_INPUT, publishes empty
+// experts and writes no permutation.  Up to kChunk assignments everything runs
+// in one CTA.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -50,94 +51,79 @@ __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a, int32_t *table
     for (int i = threadIdx.x; i <= a.E; i += blockDim.x) row[i] = cnt[i];
 }
 
-// One CTA.  Expert column g of the block table is handled by tpe consecutive
-// threads (a power of two <= 32), thread j summing the contiguous block range
-// [j*S, (j+1)*S); the partial sums are scanned inside the group with shuffles.
-__global__ void __launch_bounds__(1024) scan_kernel(PermuteArgs a, int32_t *table, int nblocks, int tpe) {
-    __shared__ int32_t tots[MOE_MAX_EXPERTS + 1];
-    __shared__ int32_t offs[MOE_MAX_EXPERTS + 1];
-    const int lane = threadIdx.x & 31;
-    const int g = threadIdx.x / tpe, j = threadIdx.x % tpe;
-    const int S = (nblocks + tpe - 1) / tpe;
-    const int b0 = min(nblocks, j * S), b1 = min(nblocks, b0 + S);
-    const bool col = g <= a.E;
-    int local = 0;
-    if (col) {
-#pragma unroll 8
-        for (int b = b0; b < b1; ++b) local += table[(int64_t)b * (a.E + 1) + g];
-    }
-    int incl = local;
-    for (int o = 1; o < tpe; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (j >= o) incl += u;
-    }
-    const int tot = __shfl_sync(0xffffffffu, incl, (lane / tpe) * tpe + tpe - 1);
-    if (col && j == 0) tots[g] = tot;
+// Scan + stable scatter: every CTA reads the whole [B, E+1] histogram table,
+// forms the per-expert totals, their exclusive scan (the offsets) and the
+// start of its own block's rows of each expert, then ranks its assignments
+// (lane rank in the match group plus the counts of earlier warps).  CTA 0
+// publishes counts and offsets.  A non-zero error column anywhere reports
+// MOE_ERR_DEVICE_INPUT, publishes empty experts and writes nothing else.
+__global__ void __launch_bounds__(kThreads) scatter_kernel(PermuteArgs a, const int32_t *table, int nblocks) {
+    extern __shared__ int32_t sm[];
+    int32_t *wc = sm;                       // [kWarps][E]: per-warp counts, then per-warp starts
+    int32_t *tot = wc + kWarps * a.E;       // [E]
+    int32_t *base = tot + a.E;              // [E] start of this block's rows of each expert
+    int32_t *off = base + a.E;              // [E + 1]
+    __shared__ int bad;
+    const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kWarps * a.E; i += kThreads) wc[i] = 0;
+    if (threadIdx.x == 0) bad = 0;
     __syncthreads();
-    if (tots[a.E] != 0) {
-        // out-of-range ids: publish empty experts and tell the scatter to stop
-        for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
-            a.offsets[i] = 0;
-            if (i < a.E) a.counts[i] = 0;
+    for (int e = threadIdx.x; e <= a.E; e += kThreads) {
+        int t = 0, before = 0;
+#pragma unroll 4
+        for (int q = 0; q < nblocks; ++q) {
+            const int c = table[(int64_t)q * (a.E + 1) + e];
+            t += c;
+            before += q < b ? c : 0;
         }
-        if (threadIdx.x == 0) {
-            atomicOr(a.err, kErrInput);
-            table[(int64_t)nblocks * (a.E + 1)] = 1;
+        if (e < a.E) {
+            tot[e] = t;
+            base[e] = before;
+        } else if (t) {
+            bad = 1;
+        }
+    }
+    __syncthreads();
+    if (bad) {
+        if (b == 0) {
+            for (int i = threadIdx.x; i <= a.E; i += kThreads) {
+                a.offsets[i] = 0;
+                if (i < a.E) a.counts[i] = 0;
+            }
+            if (threadIdx.x == 0) atomicOr(a.err, kErrInput);
         }
         return;
     }
-    // exclusive scan over experts (warp 0, 32 experts per step)
-    if (threadIdx.x < 32) {
+    if (warp == 0) {
         int carry = 0;
-        for (int base = 0; base < a.E; base += 32) {
-            const int e = base + lane;
-            const int v = e < a.E ? tots[e] : 0;
+        for (int e0 = 0; e0 < a.E; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < a.E ? tot[e] : 0;
             int in = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int u = __shfl_up_sync(0xffffffffu, in, o);
                 if (lane >= o) in += u;
             }
-            if (e < a.E) offs[e] = carry + in - v;
+            if (e < a.E) off[e] = carry + in - v;
             carry += __shfl_sync(0xffffffffu, in, 31);
         }
-        if (lane == 0) offs[a.E] = carry;
+        if (lane == 0) off[a.E] = carry;
     }
     __syncthreads();
-    if (g < a.E) {
-        if (j == 0) {
-            a.offsets[g] = offs[g];
-            a.counts[g] = tots[g];
+    if (b == 0)
+        for (int e = threadIdx.x; e <= a.E; e += kThreads) {
+            a.offsets[e] = off[e];
+            if (e < a.E) a.counts[e] = tot[e];
         }
-        int run = offs[g] + incl - local;   // start of block b0's rows of expert g
-        for (int b = b0; b < b1; ++b) {
-            int32_t *p = table + (int64_t)b * (a.E + 1) + g;
-            const int c = *p;
-            *p = run;
-            run += c;
-        }
-    }
-    if (threadIdx.x == 0) {
-        a.offsets[a.E] = offs[a.E];
-        table[(int64_t)nblocks * (a.E + 1)] = 0;
-    }
-}
-
-__global__ void __launch_bounds__(kThreads) scatter_kernel(PermuteArgs a, const int32_t *table, int nblocks) {
-    extern __shared__ int32_t wc[];   // [kWarps][E]: per-warp counts, then per-warp starts
-    if (table[(int64_t)nblocks * (a.E + 1)]) return;
-    const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < kWarps * a.E; i += kThreads) wc[i] = 0;
-    __syncthreads();
     const int r = b * kChunk + threadIdx.x;
     const int e = r < a.R ? a.ids[r] : -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * a.E + e] = __popc(peers);
     __syncthreads();
-    const int32_t *base = table + (int64_t)b * (a.E + 1);
     for (int x = threadIdx.x; x < a.E; x += kThreads) {
-        int run = base[x];
+        int run = off[x] + base[x];
         for (int w = 0; w < kWarps; ++w) {
             const int c = wc[w * a.E + x];
             wc[w * a.E + x] = run;
@@ -224,10 +210,10 @@ __global__ void __launch_bounds__(kThreads) permute_small_kernel(PermuteArgs a) 
 
 size_t permute_workspace_bytes(int64_t R, int E) {
     const int64_t nblocks = (R + kChunk - 1) / kChunk;
-    return sizeof(int32_t) * ((size_t)nblocks * (E + 1) + 1);
+    return sizeof(int32_t) * (size_t)nblocks * (E + 1);
 }
 
-cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, cudaStream_t s) {
+cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, bool table_ready, cudaStream_t s) {
     if (a.R <= 0) {
         // no assignments: every expert is empty
         cudaError_t e = cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), s);
@@ -244,18 +230,18 @@ cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, cudaStream_t s)
         return cudaGetLastError();
     }
     const int nblocks = (a.R + kChunk - 1) / kChunk;
-    hist_kernel<<<nblocks, 256, sizeof(int32_t) * (a.E + 1), s>>>(a, table);
-    note_launch();
-    int tpe = 1;
-    while (tpe < 32 && 2 * tpe * (a.E + 1) <= 1024 && tpe < nblocks) tpe *= 2;
-    scan_kernel<<<1, 1024, 0, s>>>(a, table, nblocks, tpe);
-    note_launch();
-    const size_t smem = sizeof(int32_t) * (size_t)kWarps * a.E;
+    if (!table_ready) {
+        hist_kernel<<<nblocks, 256, sizeof(int32_t) * (a.E + 1), s>>>(a, table);
+        note_launch();
+    }
+    const size_t smem = sizeof(int32_t) * ((size_t)kWarps * a.E + 3 * (size_t)a.E + 1);
     cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     scatter_kernel<<<nblocks, kThreads, smem, s>>>(a, table, nblocks);
     note_launch();
     return cudaGetLastError();
 }
+
+int permute_chunk() { return kChunk; }
 
 }  // namespace moe

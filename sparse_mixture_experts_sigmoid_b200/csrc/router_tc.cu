@@ -52,6 +52,8 @@ struct LogitsArgs {
     bool shared;
     float *logits;   // [T, LS]
     uint32_t *err;
+    int32_t *hist;   // grouping histogram to clear for the selection kernel (or null)
+    int64_t hist_ints;
 };
 
 struct Ctrl {
@@ -110,6 +112,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmW);
         if (a.shared) prefetch_tmap(&tmS);
     }
+    // clear the grouping histogram that the selection kernel accumulates into
+    if (a.hist)
+        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < a.hist_ints; i += (int64_t)gridDim.x * kThreads)
+            a.hist[i] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -291,6 +297,11 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
     if (lane < a.k) {
         a.ids[t * a.k + lane] = my_e;
         a.gates[t * a.k + lane] = sc;
+        if (a.hist) {
+            // per-block expert histogram for the grouping step
+            const int64_t r = t * a.k + lane;
+            atomicAdd(a.hist + (r / a.hist_chunk) * (a.E + 1) + my_e, 1);
+        }
     }
     if (a.probs) {
 #pragma unroll
@@ -334,7 +345,8 @@ cudaError_t launch_router_tc(const RouterArgs &a, float *scratch, cudaStream_t s
     } else {
         mS = mW;
     }
-    LogitsArgs la{a.T, a.d, a.E, g.nrw, g.LS, shared, scratch, a.err};
+    const int64_t hist_ints = a.hist ? ((a.T * a.k + a.hist_chunk - 1) / a.hist_chunk) * (a.E + 1) : 0;
+    LogitsArgs la{a.T, a.d, a.E, g.nrw, g.LS, shared, scratch, a.err, a.hist, hist_ints};
     const size_t smem = 1024 + (size_t)kStages * kStage + sizeof(Ctrl);
     cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -188,7 +188,8 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2D row-major [rows, cols] tensor, box of box_rows x (128 bytes), 128-byte swizzle, zero fill.
-inline bool make_map(CUtensorMap *m, const void *base, bool f32, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+inline bool make_map(CUtensorMap *m, const void *base, bool f32, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                     CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     auto fn = encode_fn();
     if (!fn) return false;
     const uint32_t esz = f32 ? 4 : 2;
@@ -198,7 +199,7 @@ inline bool make_map(CUtensorMap *m, const void *base, bool f32, uint64_t rows, 
     cuuint32_t estr[2] = {1, 1};
     return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_SWIZZLE_128B, promo,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
