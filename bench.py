@@ -144,17 +144,23 @@ def barrier(ws: int):
     torch.cuda.synchronize()
 
 
-def traffic_for(kernel: str, src: str, workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel's source
-    is unchanged since (profiles/traffic.json keys each figure by a source hash)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def source_hash(src: str) -> str:
+    """Hash of a kernel's translation unit plus the shared device headers."""
+    d = os.path.join(ROOT, "sparse_mixture_experts_sigmoid_b200", "csrc")
+    h = hashlib.sha256()
+    for f in [src] + sorted(x for x in os.listdir(d) if x.endswith(".cuh")):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(stage: str, src: str, workload: str):
+    """DRAM bytes per launch of a stage's kernel from a committed ncu capture
+    (profiles/traffic.json), if the kernel's source is unchanged since."""
     try:
-        with open(path) as f:
-            table = json.load(f)
-        ent = table[kernel][workload]
-        h = hashlib.sha256(open(os.path.join(ROOT, "sparse_mixture_experts_sigmoid_b200", "csrc", src),
-                                "rb").read()).hexdigest()[:16]
-        return float(ent["bytes_per_launch"]) if ent.get("src_sha") == h else None
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            ent = json.load(f)[stage][workload]
+        return float(ent["bytes_per_launch"]) if ent.get("src_sha") == source_hash(src) else None
     except (OSError, KeyError, ValueError):
         return None
 
@@ -301,7 +307,7 @@ def bench_ours(args, w, ws_n, rank, local):
     else:
         roof = {"bound": "tensor", "achieved": fl / t / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for(kname, ksrc, w.name)
+    roof["traffic"] = traffic_for(dom, ksrc, w.name)
     roof.update({"kernel": kname, "stage": dom, "ms_per_launch": stage[dom],
                  "algorithmic_bytes": by, "algorithmic_flops": fl, "peak_source": peaks["source"]})
     lw = roofline.layer_work(w, counts)

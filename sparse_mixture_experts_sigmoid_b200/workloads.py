@@ -79,6 +79,9 @@ WORKLOADS: dict[str, Workload] = {
                             h_shared=5632, seed=4),
     "mixtral_prefill": Workload("mixtral_prefill", T=4096, d=4096, E=8, h=14336, k=2, seed=5),
     "mixtral_decode": Workload("mixtral_decode", T=1, d=4096, E=8, h=14336, k=2, seed=5),
+    # small case of the Mixtral-like expert shape (2 experts, 0.7 GB of weights) for
+    # full profiler captures, which must stay a few GB on the device
+    "mixtral_e2_profile": Workload("mixtral_e2_profile", T=2048, d=4096, E=2, h=14336, k=2, seed=6),
 }
 
 # The workload that the headline benchmark line is quoted on.
