@@ -43,6 +43,7 @@
 //    outstanding copies are drained and TMEM is released before exit.
 #include <algorithm>
 
+#include "grouped_tiles.cuh"
 #include "moe_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -83,79 +84,6 @@ struct Ctrl {
     int n_mtiles;
     int pad;
 };
-
-// ------------------------------------------------------------------ tile list
-
-// One warp: per-expert row-tile counts and their prefix sum (tile_start), and
-// the validated segment offsets (seg_off).  Offsets outside [0, rows] or
-// decreasing are reported and treated as empty segments.
-__device__ void build_tiles(const Params &p, int *tile_start, int *seg_off, int *n_mtiles) {
-    const int lane = threadIdx.x & 31;
-    if (p.offsets == nullptr) {
-        if (lane == 0) {
-            seg_off[0] = 0;
-            seg_off[1] = (int)p.rows;
-            tile_start[0] = 0;
-            tile_start[1] = (int)((p.rows + BM - 1) / BM);
-            *n_mtiles = tile_start[1];
-        }
-        return;
-    }
-    int carry = 0;
-    bool bad = false;
-    for (int base = 0; base < p.E; base += 32) {
-        const int e = base + lane;
-        int b = 0, en = 0;
-        if (e < p.E) {
-            b = p.offsets[e];
-            en = p.offsets[e + 1];
-            if (b < 0 || en < b || en > p.rows) {
-                bad = true;
-                en = b = 0;
-            }
-        }
-        const int mt = (en - b + BM - 1) / BM;
-        int incl = mt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (e < p.E) {
-            tile_start[e] = carry + incl - mt;
-            seg_off[e] = b;
-        }
-        carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kErrInput);
-    if (lane == 0) {
-        tile_start[p.E] = carry;
-        *n_mtiles = carry;
-    }
-}
-
-struct Tile {
-    int e, m, n;
-};
-
-__device__ __forceinline__ Tile decode(int id, int n_tiles, const int *tile_start, int E) {
-    const int q = id / n_tiles;
-    int lo = 0, hi = E;  // first j in [0, E] with tile_start[j] > q, minus one
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (tile_start[mid] <= q) lo = mid;
-        else hi = mid - 1;
-    }
-    // lo = the last index with tile_start[lo] <= q; a run of empty experts shares
-    // its start with the next non-empty one, so lo lands on the expert owning q
-    Tile t;
-    t.e = lo;
-    const int mt = tile_start[lo + 1] - tile_start[lo];
-    const int local = id - tile_start[lo] * n_tiles;
-    t.n = local / mt;
-    t.m = local - t.n * mt;
-    return t;
-}
 
 // ------------------------------------------------------------------ kernel
 
@@ -201,7 +129,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             if (MODE == GATEUP) prefetch_tmap(&tmB1);
             if (!GATHER) prefetch_tmap(&tmA);
         }
-        build_tiles(p, tile_start, seg_off, &ctrl->n_mtiles);
+        build_tiles<BM>(p, tile_start, seg_off, &ctrl->n_mtiles);
         __syncwarp();
         // per-expert segment ends (offsets validated above)
         if (p.offsets == nullptr) {

@@ -1,0 +1,86 @@
+// Device-side tile list of the grouped GEMMs: per-expert row-block counts and
+// their prefix sum, built from the expert offsets by one warp, and the mapping
+// of a tile id to (expert, column block, row block).  Tiles are expert-major;
+// inside an expert the row blocks vary fastest, so CTAs running at the same
+// time share one weight tile through L2.
+#pragma once
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace gg {
+
+// One warp: per-expert counts of RB-row blocks and their prefix sum
+// (tile_start), and the validated segment offsets (seg_off).  Offsets outside
+// [0, rows] or decreasing are reported and treated as empty segments.
+template <int RB>
+__device__ void build_tiles(const GemmParams &p, int *tile_start, int *seg_off, int *n_mtiles) {
+    const int lane = threadIdx.x & 31;
+    if (p.offsets == nullptr) {
+        if (lane == 0) {
+            seg_off[0] = 0;
+            seg_off[1] = (int)p.rows;
+            tile_start[0] = 0;
+            tile_start[1] = (int)((p.rows + RB - 1) / RB);
+            *n_mtiles = tile_start[1];
+        }
+        return;
+    }
+    int carry = 0;
+    bool bad = false;
+    for (int base = 0; base < p.E; base += 32) {
+        const int e = base + lane;
+        int b = 0, en = 0;
+        if (e < p.E) {
+            b = p.offsets[e];
+            en = p.offsets[e + 1];
+            if (b < 0 || en < b || en > p.rows) {
+                bad = true;
+                en = b = 0;
+            }
+        }
+        const int mt = (en - b + RB - 1) / RB;
+        int incl = mt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (e < p.E) {
+            tile_start[e] = carry + incl - mt;
+            seg_off[e] = b;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kErrInput);
+    if (lane == 0) {
+        tile_start[p.E] = carry;
+        *n_mtiles = carry;
+    }
+}
+
+struct Tile {
+    int e, m, n;
+};
+
+__device__ __forceinline__ Tile decode(int id, int n_tiles, const int *tile_start, int E) {
+    const int q = id / n_tiles;
+    int lo = 0, hi = E;  // first j in [0, E] with tile_start[j] > q, minus one
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= q) lo = mid;
+        else hi = mid - 1;
+    }
+    // lo = the last index with tile_start[lo] <= q; a run of empty experts shares
+    // its start with the next non-empty one, so lo lands on the expert owning q
+    Tile t;
+    t.e = lo;
+    const int mt = tile_start[lo + 1] - tile_start[lo];
+    const int local = id - tile_start[lo] * n_tiles;
+    t.n = local / mt;
+    t.m = local - t.n * mt;
+    return t;
+}
+
+}  // namespace gg
+}  // namespace moe

@@ -96,15 +96,11 @@ void mark(int i, cudaStream_t s) {
 // smaller ones (decode) use the CUDA-core segment kernels.
 constexpr int32_t kDecodeMaxRows = 64;
 
-#ifndef MOE_NARROW_TILES
-#define MOE_NARROW_TILES 0
-#endif
-#ifndef MOE_NARROW_ROWS_PER_EXPERT
-#define MOE_NARROW_ROWS_PER_EXPERT 128
-#endif
-// Few rows per expert make the expert GEMMs weight-streaming (HBM) bound:
-// narrower N tiles give more tiles and a deeper ring of loads in flight.
-bool narrow_tiles(const moe_config &c) { return c.T * c.k < (int64_t)MOE_NARROW_ROWS_PER_EXPERT * c.E; }
+// MMA N of the expert GEMMs: 256 unless the output width is not a multiple of
+// the wide tile (128 output columns for gate/up, 256 for down), where the last
+// column tile would load weight rows of the next expert for nothing; then 128.
+bool narrow_gateup(const moe_config &c) { return c.h % 128 != 0; }
+bool narrow_down(const moe_config &c) { return c.d % 256 != 0; }
 
 GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const void *wu, const int32_t *offsets,
                        const int32_t *srt, void *act, uint32_t *err) {
@@ -113,7 +109,7 @@ GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const
     L.gather = true;
     L.dtype = c.dtype;
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.d, c.h, x, act, nullptr, nullptr, err};
-    L.narrow = narrow_tiles(c) && MOE_NARROW_TILES;
+    L.narrow = narrow_gateup(c);
     L.b0 = wg;
     L.b1 = wu;
     return L;
@@ -137,7 +133,7 @@ GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const
     L.gather = false;
     L.dtype = c.dtype;
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.h, c.d, nullptr, nullptr, acc, gates, err};
-    L.narrow = narrow_tiles(c) && MOE_NARROW_TILES;
+    L.narrow = narrow_down(c);
     L.a_src = act;
     L.b0 = wd;
     return L;

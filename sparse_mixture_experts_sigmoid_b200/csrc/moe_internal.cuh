@@ -163,7 +163,7 @@ struct GemmLaunch {
     int mode;             // 0: gate/up with SwiGLU epilogue, 1: down with gate-weighted combine
     bool gather;          // A rows gathered from x by index (routed gate/up); else TMA from a_src
     int dtype;            // MOE_BF16 or MOE_F32 (tf32 MMA)
-    bool narrow;          // MMA N = 128 and a deeper ring (few rows per expert) instead of N = 256
+    bool narrow;          // MMA N = 128 (6-stage ring) instead of N = 256 (4 stages)
     GemmParams p;
     const void *a_src;    // contiguous A operand [rows, K] when !gather
     const void *b0, *b1;  // weights [E*N, K] (b1: up projection for gate/up)
