@@ -123,12 +123,15 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         fence_barrier_init();
     }
     if (warp == kMmaWarp) tmem_alloc(&ctrl->tmem_base, kTmemCols);
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tmap(&tmB0);
+        if (MODE == GATEUP) prefetch_tmap(&tmB1);
+        if (!GATHER) prefetch_tmap(&tmA);
+    }
+    // everything above overlaps the previous kernel's tail; the offsets, x,
+    // act and y_acc are read or written only after it has completed
+    pdl_wait();
     if (warp == kTmaWarp) {
-        if (lane == 0) {
-            prefetch_tmap(&tmB0);
-            if (MODE == GATEUP) prefetch_tmap(&tmB1);
-            if (!GATHER) prefetch_tmap(&tmA);
-        }
         build_tiles<BM>(p, tile_start, seg_off, &ctrl->n_mtiles);
         __syncwarp();
         // per-expert segment ends (offsets validated above)
@@ -145,6 +148,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_launch_dependents();   // this CTA's TMEM is allocated
 
     const uint32_t tmem = ctrl->tmem_base;
     const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
@@ -403,9 +407,7 @@ cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
     auto kern = grouped_gemm_kernel<MODE, GATHER, T, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, GATHER ? 320 : 192, smem, s>>>(mA, mB0, mB1, p);
-    note_launch();
-    return cudaGetLastError();
+    return launch_kernel(kern, grid, GATHER ? 320 : 192, smem, s, mA, mB0, mB1, p);
 }
 
 template <int MODE, bool GATHER, typename T>

@@ -2,6 +2,7 @@
 // sequence of the MoE layer forward pass.  Declarations and contracts are in
 // include/moe.h.
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -162,6 +163,14 @@ GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const
 }
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("MOE_PDL");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
 
 int num_sms() {
     const int dev = current_device();

@@ -181,4 +181,40 @@ int num_sms();
 // Counts one kernel launch (for moe_launch_count).
 void note_launch();
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of a pass is launched with programmatic stream serialization, so
+// the next kernel in the stream can be scheduled (and run its prologue: barrier
+// set-up, TMEM allocation, tensor-map prefetch) while this one drains.  Each
+// kernel therefore calls pdl_wait() before its first global-memory access --
+// it returns once every earlier kernel of the stream has completed and its
+// writes are visible -- and pdl_launch_dependents() once its own TMEM (if any)
+// is allocated, so a dependent CTA can never hold TMEM that an earlier CTA on
+// the same SM still has to allocate.  Without the launch attribute both are
+// no-ops.  MOE_PDL=0 in the environment launches without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+bool pdl_enabled();
+
+// Launches kern<<<grid, block, smem, s>>>(args...) with the attribute above and
+// counts it.
+template <typename... P, typename... A>
+cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<A &&>(args)...);
+    note_launch();
+    return e;
+}
+
 }  // namespace moe

@@ -31,6 +31,8 @@ constexpr int kThreads = 1024;   // one assignment per thread in the scatter
 constexpr int kWarps = kThreads / 32;
 
 __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a, int32_t *table) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t cnt[];   // [E + 1]
     const int b = blockIdx.x;
     for (int i = threadIdx.x; i <= a.E; i += blockDim.x) cnt[i] = 0;
@@ -58,6 +60,8 @@ __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a, int32_t *table
 // publishes counts and offsets.  A non-zero error column anywhere reports
 // MOE_ERR_DEVICE_INPUT, publishes empty experts and writes nothing else.
 __global__ void __launch_bounds__(kThreads) scatter_kernel(PermuteArgs a, const int32_t *table, int nblocks) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t sm[];
     int32_t *wc = sm;                       // [kWarps][E]: per-warp counts, then per-warp starts
     int32_t *tot = wc + kWarps * a.E;       // [E]
@@ -141,6 +145,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(PermuteArgs a, const 
 // All three steps in one CTA when every assignment fits in one block
 // (R <= kChunk): per-warp counts, scans over warps and experts, scatter.
 __global__ void __launch_bounds__(kThreads) permute_small_kernel(PermuteArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t sm[];
     int32_t *wc = sm;                       // [kWarps][E]
     int32_t *tot = sm + kWarps * a.E;       // [E]
@@ -225,21 +231,17 @@ cudaError_t launch_permute(const PermuteArgs &a, int32_t *table, bool table_read
         cudaError_t e = cudaFuncSetAttribute(permute_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
-        permute_small_kernel<<<1, kThreads, smem, s>>>(a);
-        note_launch();
-        return cudaGetLastError();
+        return launch_kernel(permute_small_kernel, 1, kThreads, smem, s, a);
     }
     const int nblocks = (a.R + kChunk - 1) / kChunk;
     if (!table_ready) {
-        hist_kernel<<<nblocks, 256, sizeof(int32_t) * (a.E + 1), s>>>(a, table);
-        note_launch();
+        const cudaError_t e = launch_kernel(hist_kernel, nblocks, 256, sizeof(int32_t) * (a.E + 1), s, a, table);
+        if (e != cudaSuccess) return e;
     }
     const size_t smem = sizeof(int32_t) * ((size_t)kWarps * a.E + 3 * (size_t)a.E + 1);
     cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    scatter_kernel<<<nblocks, kThreads, smem, s>>>(a, table, nblocks);
-    note_launch();
-    return cudaGetLastError();
+    return launch_kernel(scatter_kernel, nblocks, kThreads, smem, s, a, static_cast<const int32_t *>(table), nblocks);
 }
 
 int permute_chunk() { return kChunk; }

@@ -72,6 +72,8 @@ __device__ __forceinline__ void stage_chunk(const RouterArgs &a, const Geo &g, T
 
 template <typename Tin, int TW, int EPL>
 __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     constexpr int NT = kWarps * TW;
     Tin *wbuf[2], *xbuf[2];
@@ -244,6 +246,8 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
 // same arg-max rounds as the batched router.
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ float sm[];
     float *sx = sm;              // [d] the token's row
     float *lg = sm + a.d;        // [E + 1] logits (shared gate last)
@@ -367,9 +371,7 @@ cudaError_t launch_t(const RouterArgs &a, const Geo &g, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((a.T + NT - 1) / NT);
-    kern<<<grid, kThreads, smem, s>>>(a, g);
-    note_launch();
-    return cudaGetLastError();
+    return launch_kernel(kern, grid, kThreads, smem, s, a, g);
 }
 
 template <typename Tin, int EPL>
@@ -431,15 +433,13 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaSt
             cudaError_t e = cudaFuncSetAttribute(router_small_kernel<float>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
-            router_small_kernel<float><<<(unsigned)a.T, kThreads, smem, s>>>(a);
+            return launch_kernel(router_small_kernel<float>, (unsigned)a.T, kThreads, smem, s, a);
         } else {
             cudaError_t e = cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
-            router_small_kernel<__nv_bfloat16><<<(unsigned)a.T, kThreads, smem, s>>>(a);
+            return launch_kernel(router_small_kernel<__nv_bfloat16>, (unsigned)a.T, kThreads, smem, s, a);
         }
-        note_launch();
-        return cudaGetLastError();
     }
     return dtype == MOE_F32 ? launch_dt<float>(a, s) : launch_dt<__nv_bfloat16>(a, s);
 }

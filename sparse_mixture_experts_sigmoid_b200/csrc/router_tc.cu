@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmW);
         if (a.shared) prefetch_tmap(&tmS);
     }
+    pdl_wait();   // the prologue above overlaps the previous kernel's tail
     // clear the grouping histogram that the selection kernel accumulates into
     if (a.hist)
         for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < a.hist_ints; i += (int64_t)gridDim.x * kThreads)
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_launch_dependents();   // this CTA's TMEM is allocated
 
     const uint32_t tmem = ctrl->tmem_base;
     const int n_tiles = a.LS / BN;
@@ -226,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // One warp per token: scoring, top-k and gates from a row of logits.
 template <int EPL>
 __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const float *logits, int LS, int nrw) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * 8 + warp;
     if (t >= a.T) return;
@@ -352,20 +356,14 @@ cudaError_t launch_router_tc(const RouterArgs &a, float *scratch, cudaStream_t s
     if (e != cudaSuccess) return e;
     const int total = (int)((a.T + BM - 1) / BM) * (g.LS / BN);
     const int grid = total < num_sms() ? total : num_sms();
-    router_logits_kernel<<<grid, kThreads, smem, s>>>(mX, mW, mS, la);
-    note_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_kernel(router_logits_kernel, grid, kThreads, smem, s, mX, mW, mS, la);
+    if (e != cudaSuccess) return e;
     const unsigned sgrid = (unsigned)((a.T + 7) / 8);
-    if (a.E <= 64)
-        router_select_kernel<2><<<sgrid, 256, 0, s>>>(a, scratch, g.LS, g.nrw);
-    else if (a.E <= 128)
-        router_select_kernel<4><<<sgrid, 256, 0, s>>>(a, scratch, g.LS, g.nrw);
-    else if (a.E <= 256)
-        router_select_kernel<8><<<sgrid, 256, 0, s>>>(a, scratch, g.LS, g.nrw);
-    else
-        router_select_kernel<16><<<sgrid, 256, 0, s>>>(a, scratch, g.LS, g.nrw);
-    note_launch();
-    return cudaGetLastError();
+    const float *lg = scratch;
+    if (a.E <= 64) return launch_kernel(router_select_kernel<2>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
+    if (a.E <= 128) return launch_kernel(router_select_kernel<4>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
+    if (a.E <= 256) return launch_kernel(router_select_kernel<8>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
+    return launch_kernel(router_select_kernel<16>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
 }
 
 }  // namespace moe

@@ -77,6 +77,8 @@ __device__ __forceinline__ float dot8(const float (&a)[8], const float (&b)[8], 
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) seg_gateup_kernel(SegGateUpArgs a, uint32_t *err) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int sm[];
     int *list = sm, *beg = sm + a.seg.E, *end = sm + 2 * a.seg.E;
     const int ne = list_experts(a.seg, list, beg, end);
@@ -160,6 +162,8 @@ __global__ void __launch_bounds__(kThreads) seg_gateup_kernel(SegGateUpArgs a, u
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) seg_down_kernel(SegDownArgs a, uint32_t *err) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int sm[];
     int *list = sm, *beg = sm + a.seg.E, *end = sm + 2 * a.seg.E;
     const int ne = list_experts(a.seg, list, beg, end);
@@ -241,6 +245,8 @@ __device__ __forceinline__ float row_dot(const T *w, const T *v, int n, int lane
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) down_direct_kernel(DownDirectArgs a, uint32_t *err) {
+    pdl_wait();
+    pdl_launch_dependents();
     const T *act = static_cast<const T *>(a.act);
     const T *wd = static_cast<const T *>(a.w_down);
     T *y = static_cast<T *>(a.y);
@@ -274,6 +280,8 @@ __global__ void __launch_bounds__(kThreads) down_direct_kernel(DownDirectArgs a,
 
 template <typename T>
 __global__ void finalize_kernel(const float *y_acc, T *y, int64_t n) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
     if (i + 8 <= n) {
         const float4 a = *reinterpret_cast<const float4 *>(y_acc + i);
@@ -301,11 +309,8 @@ cudaError_t launch_seg_gateup(const SegGateUpArgs &a, int dtype, cudaStream_t s,
     const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
     const int grid = grid_for((int64_t)a.seg.E * a.hid);
     if (dtype == MOE_F32)
-        seg_gateup_kernel<float><<<grid, kThreads, smem, s>>>(a, err);
-    else
-        seg_gateup_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a, err);
-    note_launch();
-    return cudaGetLastError();
+        return launch_kernel(seg_gateup_kernel<float>, grid, kThreads, smem, s, a, err);
+    return launch_kernel(seg_gateup_kernel<__nv_bfloat16>, grid, kThreads, smem, s, a, err);
 }
 
 cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
@@ -313,31 +318,24 @@ cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uin
     const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
     const int grid = grid_for((int64_t)a.seg.E * a.d);
     if (dtype == MOE_F32)
-        seg_down_kernel<float><<<grid, kThreads, smem, s>>>(a, err);
-    else
-        seg_down_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a, err);
-    note_launch();
-    return cudaGetLastError();
+        return launch_kernel(seg_down_kernel<float>, grid, kThreads, smem, s, a, err);
+    return launch_kernel(seg_down_kernel<__nv_bfloat16>, grid, kThreads, smem, s, a, err);
 }
 
 cudaError_t launch_down_direct(const DownDirectArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
     if (a.T <= 0) return cudaSuccess;
     const int grid = grid_for(a.T * a.d);
     if (dtype == MOE_F32)
-        down_direct_kernel<float><<<grid, kThreads, 0, s>>>(a, err);
-    else
-        down_direct_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(a, err);
-    note_launch();
-    return cudaGetLastError();
+        return launch_kernel(down_direct_kernel<float>, grid, kThreads, 0, s, a, err);
+    return launch_kernel(down_direct_kernel<__nv_bfloat16>, grid, kThreads, 0, s, a, err);
 }
 
 cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s) {
     if (n <= 0) return cudaSuccess;
     const int threads = 256;
     const int64_t blocks = (n / 8 + threads) / threads + 1;
-    finalize_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(y_acc, static_cast<__nv_bfloat16 *>(y), n);
-    note_launch();
-    return cudaGetLastError();
+    return launch_kernel(finalize_kernel<__nv_bfloat16>, (unsigned)blocks, threads, 0, s, y_acc,
+                         static_cast<__nv_bfloat16 *>(y), n);
 }
 
 }  // namespace moe
