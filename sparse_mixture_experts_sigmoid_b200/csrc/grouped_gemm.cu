@@ -128,27 +128,26 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         if (MODE == GATEUP) prefetch_tmap(&tmB1);
         if (!GATHER) prefetch_tmap(&tmA);
     }
-    // everything above overlaps the previous kernel's tail; the offsets, x,
-    // act and y_acc are read or written only after it has completed
-    pdl_wait();
-    if (warp == kTmaWarp) {
-        build_tiles<BM>(p, tile_start, seg_off, &ctrl->n_mtiles);
-        __syncwarp();
-        // per-expert segment ends (offsets validated above)
-        if (p.offsets == nullptr) {
-            if (lane == 0) seg_end[0] = (int)p.rows;
-        } else {
-            for (int e = lane; e < p.E; e += 32) {
-                int b = p.offsets[e], en = p.offsets[e + 1];
-                if (b < 0 || en < b || en > p.rows) en = b = 0;
-                seg_end[e] = en;
-            }
-        }
-    }
+    // everything above overlaps the previous kernel's tail.  Data the previous
+    // kernel may still be writing (act, sorted rows, offsets right after the
+    // grouping step) is read only after pdl_wait(); what p.early marks as
+    // complete already (weights, the layer input, offsets from further back)
+    // is read before it, so the first weight tiles are in flight early.
+    const bool early_tiles = (p.early & kEarlyTiles) != 0;
+    if (!early_tiles) pdl_wait();
+    if (warp == kTmaWarp) build_tiles<BM>(p, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    pdl_launch_dependents();   // this CTA's TMEM is allocated
+    // dependents are released only after this CTA's TMEM is allocated and after
+    // the wait: every thread but the producer waits here, the producer once it
+    // has issued the early loads
+    if (!early_tiles) {
+        pdl_launch_dependents();
+    } else if (!(warp == kTmaWarp && lane == 0)) {
+        pdl_wait();
+        pdl_launch_dependents();
+    }
 
     const uint32_t tmem = ctrl->tmem_base;
     const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
@@ -158,6 +157,32 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
+            auto load_b = [&](int s, int kb, int b_row) {
+                if (MODE == GATEUP) {
+                    tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
+                    tma_load_2d(&tmB1, sB + s * kBBytes + kBBytes / 2, &ctrl->full[s], kb * BK, b_row);
+                } else {
+                    tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
+                }
+            };
+            const bool early_a = !GATHER && (p.early & kEarlyA) != 0;
+            // the first kStages stages are free: fill them with weight tiles (and
+            // the A tiles, when they are complete already) before waiting
+            uint32_t pre = 0;
+            if (early_tiles) {
+                for (int id = blockIdx.x; id < total && pre < (uint32_t)kStages; id += gridDim.x) {
+                    const Tile tl = decode(id, n_tiles, tile_start, nE);
+                    const int a_row = seg_off[tl.e] + tl.m * BM;
+                    const int b_row = tl.e * p.N + tl.n * BN_OUT;
+                    for (int kb = 0; kb < nk && pre < (uint32_t)kStages; ++kb, ++pre) {
+                        mbar_expect_tx(&ctrl->full[pre], kBBytes + (GATHER ? 0 : kABytes));
+                        if (early_a) tma_load_2d(&tmA, sA + pre * kABytes, &ctrl->full[pre], kb * BK, a_row);
+                        load_b((int)pre, kb, b_row);
+                    }
+                }
+                pdl_wait();
+                pdl_launch_dependents();
+            }
             uint32_t it = 0;
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
@@ -167,18 +192,18 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
+                    if (it < pre) {
+                        // issued above; only the A tile may still be missing
+                        if (!GATHER && !early_a) tma_load_2d(&tmA, sA + s * kABytes, &ctrl->full[s], kb * BK, a_row);
+                        continue;
+                    }
                     if (!wait_bar(&ctrl->empty[s], ph ^ 1, abort, p.err)) {
                         ok = false;
                         break;
                     }
                     mbar_expect_tx(&ctrl->full[s], kBBytes + (GATHER ? 0 : kABytes));
                     if (!GATHER) tma_load_2d(&tmA, sA + s * kABytes, &ctrl->full[s], kb * BK, a_row);
-                    if (MODE == GATEUP) {
-                        tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
-                        tma_load_2d(&tmB1, sB + s * kBBytes + kBBytes / 2, &ctrl->full[s], kb * BK, b_row);
-                    } else {
-                        tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
-                    }
+                    load_b(s, kb, b_row);
                 }
             }
             if (!ok) {
@@ -219,6 +244,15 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             }
         }
     } else if (warp < kEpiWarps) {
+        if (MODE == GATEUP && p.zero) {
+            // clear this CTA's share of the down GEMM's accumulator while the
+            // first tile's operands stream in
+            const int64_t n4 = p.zero_floats / 4;
+            const int64_t per = (n4 + gridDim.x - 1) / gridDim.x;
+            const int64_t b = (int64_t)blockIdx.x * per, e = min(n4, b + per);
+            float4 *z = reinterpret_cast<float4 *>(p.zero);
+            for (int64_t i = b + threadIdx.x; i < e; i += kEpiWarps * 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         uint32_t tc = 0;
         const int row = warp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;

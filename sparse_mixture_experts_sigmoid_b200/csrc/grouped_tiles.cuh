@@ -11,51 +11,66 @@ namespace moe {
 namespace gg {
 
 // One warp: per-expert counts of RB-row blocks and their prefix sum
-// (tile_start), and the validated segment offsets (seg_off).  Offsets outside
-// [0, rows] or decreasing are reported and treated as empty segments.
+// (tile_start), the validated segment bounds (seg_off, seg_end), and the total
+// (n_mtiles).  Lane l owns the C = ceil(E / 32) consecutive experts starting
+// at l * C, so all offsets are read with one round of independent loads.
+// Offsets outside [0, rows] or decreasing are reported and treated as empty
+// segments.
 template <int RB>
-__device__ void build_tiles(const GemmParams &p, int *tile_start, int *seg_off, int *n_mtiles) {
+__device__ void build_tiles(const GemmParams &p, int *tile_start, int *seg_off, int *seg_end, int *n_mtiles) {
     const int lane = threadIdx.x & 31;
     if (p.offsets == nullptr) {
         if (lane == 0) {
             seg_off[0] = 0;
-            seg_off[1] = (int)p.rows;
+            seg_end[0] = (int)p.rows;
             tile_start[0] = 0;
             tile_start[1] = (int)((p.rows + RB - 1) / RB);
             *n_mtiles = tile_start[1];
         }
         return;
     }
-    int carry = 0;
+    constexpr int kMaxC = (MOE_MAX_EXPERTS + 31) / 32;
+    const int C = (p.E + 31) / 32;
+    const int e0 = lane * C;
+    int o[kMaxC + 1];
+#pragma unroll
+    for (int j = 0; j <= kMaxC; ++j)
+        if (j <= C && e0 + j <= p.E) o[j] = p.offsets[e0 + j];
+    int mt[kMaxC];
+    int sum = 0;
     bool bad = false;
-    for (int base = 0; base < p.E; base += 32) {
-        const int e = base + lane;
-        int b = 0, en = 0;
-        if (e < p.E) {
-            b = p.offsets[e];
-            en = p.offsets[e + 1];
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j) {
+        mt[j] = 0;
+        if (j < C && e0 + j < p.E) {
+            int b = o[j], en = o[j + 1];
             if (b < 0 || en < b || en > p.rows) {
                 bad = true;
                 en = b = 0;
             }
+            seg_off[e0 + j] = b;
+            seg_end[e0 + j] = en;
+            mt[j] = (en - b + RB - 1) / RB;
+            sum += mt[j];
         }
-        const int mt = (en - b + RB - 1) / RB;
-        int incl = mt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (e < p.E) {
-            tile_start[e] = carry + incl - mt;
-            seg_off[e] = b;
-        }
-        carry += __shfl_sync(0xffffffffu, incl, 31);
     }
+    int incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j)
+        if (j < C && e0 + j < p.E) {
+            tile_start[e0 + j] = run;
+            run += mt[j];
+        }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kErrInput);
-    if (lane == 0) {
-        tile_start[p.E] = carry;
-        *n_mtiles = carry;
+    if (lane == 31) {
+        tile_start[p.E] = incl;
+        *n_mtiles = incl;
     }
 }
 

@@ -49,7 +49,7 @@ struct Layout {
 
 // Scratch of the tensor-core router (fp32 logits), 0 when the CUDA-core router runs.
 size_t router_scratch_bytes(const moe_config &c) {
-    return router_tc_supported(c.T, c.E, c.dtype) ? router_tc_workspace_bytes(c.T, c.E, c.h_shared > 0) : 0;
+    return router_tc_supported(c.T, c.E, c.dtype) ? router_tc_workspace_bytes(c.T, c.d, c.E, c.h_shared > 0) : 0;
 }
 
 Layout make_layout(const moe_config &c) {
@@ -163,6 +163,17 @@ GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const
 }
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// Bytes of gate/up weights prefetched into L2 during routing (MOE_L2_PREFETCH_MB,
+// default 64; 0 turns it off).
+size_t l2_prefetch_budget() {
+    static const size_t v = [] {
+        const char *e = std::getenv("MOE_L2_PREFETCH_MB");
+        const long mb = e ? std::atol(e) : 64;
+        return (size_t)(mb > 0 ? mb : 0) << 20;
+    }();
+    return v;
+}
 
 bool pdl_enabled() {
     static const bool on = [] {
@@ -405,12 +416,20 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     ra.gates = gates;
     ra.probs = nullptr;
     ra.shared_gate = sg;
-    ra.zero_rows = use_gemm(*c) ? acc : nullptr;   // the small-batch path writes y directly
+    ra.zero_rows = nullptr;   // the gate/up GEMM clears the accumulator; the small-batch path writes y
     ra.err = err;
     // the tensor-core router also builds the grouping histogram
     const bool fused_hist = L.size[P_LOGITS] && c->T * c->k > permute_chunk();
     ra.hist = fused_hist ? part<int32_t>(ws, L, P_PERM) : nullptr;
     ra.hist_chunk = permute_chunk();
+    if (use_gemm(*c) && (int64_t)c->T * c->k >= 4LL * c->E) {
+        // most experts are active: prefetch the expert weights the gate/up GEMM
+        // reads first (its tiles walk the experts in order) while routing runs
+        const size_t per = (size_t)c->E * c->h * c->d * (c->dtype == MOE_F32 ? 4 : 2);
+        ra.l2_prefetch[0] = w_gate;
+        ra.l2_prefetch[1] = w_up;
+        ra.l2_prefetch_bytes = per < l2_prefetch_budget() / 2 ? per : l2_prefetch_budget() / 2;
+    }
     mark(0, s);
     cudaError_t e = launch_router(ra, c->dtype, part<float>(ws, L, P_LOGITS), s);
     mark(1 + MOE_STAGE_ROUTE, s);
@@ -426,14 +445,17 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     const bool gemm = use_gemm(*c);
     if (e == cudaSuccess) {
         SegGateUpArgs ga{x, w_gate, w_up, routed, c->T, c->d, c->h, act};
-        e = gemm ? launch_grouped_gemm(gemm_gateup(*c, x, w_gate, w_up, offsets, srt, act, err), s)
-                 : launch_seg_gateup(ga, c->dtype, s, err);
+        GemmLaunch gl = gemm_gateup(*c, x, w_gate, w_up, offsets, srt, act, err);
+        gl.p.zero = acc;   // the down GEMM accumulates into it two kernels later
+        gl.p.zero_floats = c->T * c->d;
+        e = gemm ? launch_grouped_gemm(gl, s) : launch_seg_gateup(ga, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_GATE_UP, s);
     if (e == cudaSuccess && shared) {
         SegGateUpArgs ga{x, sh_gate, sh_up, dense, c->T, c->d, c->h_shared, acts};
-        e = gemm ? launch_grouped_gemm(gemm_gateup_dense(*c, x, sh_gate, sh_up, acts, err), s)
-                 : launch_seg_gateup(ga, c->dtype, s, err);
+        GemmLaunch gl = gemm_gateup_dense(*c, x, sh_gate, sh_up, acts, err);
+        gl.p.early = kEarlyTiles | kEarlyA;   // x and the weights are layer inputs
+        e = gemm ? launch_grouped_gemm(gl, s) : launch_seg_gateup(ga, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_SHARED_GATE_UP, s);
     if (!gemm) {
@@ -449,9 +471,16 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
         mark(1 + MOE_STAGE_FINALIZE, s);
         return cuda_status(e);
     }
-    if (e == cudaSuccess) e = launch_grouped_gemm(gemm_down(*c, act, w_down, offsets, srt, gates, acc, err), s);
+    // the grouping step ran two or more kernels back, so the offsets are
+    // complete when the down GEMM starts; act is read after the wait
+    GemmLaunch dl = gemm_down(*c, act, w_down, offsets, srt, gates, acc, err);
+    dl.p.early = kEarlyTiles;
+    if (e == cudaSuccess) e = launch_grouped_gemm(dl, s);
     mark(1 + MOE_STAGE_DOWN, s);
-    if (e == cudaSuccess && shared) e = launch_grouped_gemm(gemm_down_dense(*c, acts, sh_down, sg, acc, err), s);
+    // the shared expert's act came from the kernel before the routed down GEMM
+    GemmLaunch sdl = gemm_down_dense(*c, acts, sh_down, sg, acc, err);
+    sdl.p.early = kEarlyTiles | kEarlyA;
+    if (e == cudaSuccess && shared) e = launch_grouped_gemm(sdl, s);
     mark(1 + MOE_STAGE_SHARED_DOWN, s);
     if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
     mark(1 + MOE_STAGE_FINALIZE, s);

@@ -81,12 +81,17 @@ struct RouterArgs {
     uint32_t *err;      // device error word
     int32_t *hist;      // optional [B, E+1] block histogram for grouping (tensor-core router only)
     int hist_chunk;     // assignments per histogram block
+    // optional: the first l2_prefetch_bytes of each of two weight tensors that the
+    // grouped GEMM after the router reads first, brought into L2 while routing
+    // runs (tensor-core router only; a hint, no data dependence)
+    const void *l2_prefetch[2];
+    size_t l2_prefetch_bytes;
 };
 // Router: the tensor-core logits GEMM + warp-per-token selection (router_tc.cu)
 // when supported and scratch is given, else the CUDA-core routers (router.cu).
 cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaStream_t s);
 bool router_tc_supported(int64_t T, int E, int dtype);
-size_t router_tc_workspace_bytes(int64_t T, int E, bool shared);
+size_t router_tc_workspace_bytes(int64_t T, int d, int E, bool shared);
 cudaError_t launch_router_tc(const RouterArgs &a, float *scratch, cudaStream_t s);
 
 struct PermuteArgs {
@@ -158,6 +163,16 @@ struct GemmParams {
     float *y_acc;                // down output [T, N] fp32, accumulated into
     const float *gates;          // down: routed [R] by assignment, dense [T]
     uint32_t *err;
+    float *zero;                 // gate/up only, optional: [zero_floats] fp32 to clear (the
+    int64_t zero_floats;         // down GEMM's accumulator), spread over the CTAs
+    // kEarly* bits: what the kernel may read before the previous kernel in the
+    // stream has completed (see pdl_wait).  Set only where every kernel between
+    // the producer of that data and this one is known.
+    int early;
+};
+enum : int {
+    kEarlyTiles = 1,   // offsets (and hence the tile list) and the weights
+    kEarlyA = 2,       // the contiguous A operand
 };
 struct GemmLaunch {
     int mode;             // 0: gate/up with SwiGLU epilogue, 1: down with gate-weighted combine
@@ -181,16 +196,25 @@ int num_sms();
 // Counts one kernel launch (for moe_launch_count).
 void note_launch();
 
+// Asynchronous prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // Every kernel of a pass is launched with programmatic stream serialization, so
 // the next kernel in the stream can be scheduled (and run its prologue: barrier
 // set-up, TMEM allocation, tensor-map prefetch) while this one drains.  Each
-// kernel therefore calls pdl_wait() before its first global-memory access --
-// it returns once every earlier kernel of the stream has completed and its
-// writes are visible -- and pdl_launch_dependents() once its own TMEM (if any)
-// is allocated, so a dependent CTA can never hold TMEM that an earlier CTA on
-// the same SM still has to allocate.  Without the launch attribute both are
-// no-ops.  MOE_PDL=0 in the environment launches without the attribute.
+// kernel calls pdl_wait() before it touches data the previous kernel may still
+// be writing (or reading) -- it returns once every earlier kernel of the
+// stream has completed and its writes are visible -- and calls
+// pdl_launch_dependents() only after its own pdl_wait() has returned and its
+// TMEM (if any) is allocated.  Hence (a) a dependent CTA never holds TMEM that
+// an earlier CTA on the same SM still has to allocate, and (b) when a kernel
+// starts, every kernel two or more places back in the stream has completed,
+// so data produced there (and the layer's inputs) may be read before
+// pdl_wait().  Without the launch attribute both calls are no-ops.  MOE_PDL=0
+// in the environment launches without the attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -26,8 +26,11 @@
 namespace moe {
 namespace {
 
-constexpr int kChunk = 1024;     // assignments per block
-constexpr int kThreads = 1024;   // one assignment per thread in the scatter
+#ifndef MOE_PERMUTE_CHUNK
+#define MOE_PERMUTE_CHUNK 1024
+#endif
+constexpr int kChunk = MOE_PERMUTE_CHUNK;   // assignments per block
+constexpr int kThreads = kChunk;            // one assignment per thread in the scatter
 constexpr int kWarps = kThreads / 32;
 
 __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a, int32_t *table) {

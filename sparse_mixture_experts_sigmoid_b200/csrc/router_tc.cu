@@ -2,13 +2,16 @@
 //
 //  1. router_logits_kernel: the router logits l = x . W_router^T (plus the
 //     shared-expert gate logit w_s . x) as a tcgen05 GEMM over tiles of 128
-//     tokens x 64 logit columns, fp32 accumulators in TMEM, stored as fp32
-//     rows of a [T, LS] scratch matrix.
-//  2. router_select_kernel: one warp per token reads its row of logits, forms
-//     softmax statistics or sigmoid scores, takes the top k by k rounds of a
-//     warp arg-max over (key, -index) -- equal keys go to the lower expert
-//     index -- and writes ids, gates (optionally renormalised), the full score
-//     row and the shared gate.
+//     tokens x BN logit columns x one chunk of the K range, fp32 accumulators
+//     in TMEM.  Each tile writes its partial sums as fp32 rows of a
+//     [S, T, LSP] scratch array (S chunks of K).  Splitting K across CTAs
+//     puts ~256 CTAs (two per SM) on the layer, so the read of x is spread
+//     over every SM however few token tiles there are.
+//  2. router_select_kernel: one warp per token adds its S partial rows in
+//     chunk order, forms softmax statistics or sigmoid scores, takes the top k
+//     by k rounds of a warp arg-max over (key, -index) -- equal keys go to the
+//     lower expert index -- and writes ids, gates (optionally renormalised),
+//     the full score row and the shared gate.
 //
 // "Tutorial 11: Mixture of Experts (MoE)", section 2 "The Router" (route_topk:
 // logits = x . W_router^T, softmax over all experts, top-k, gather of the kept
@@ -16,15 +19,19 @@
 // SmallMoE.forward (sigmoid scores; gates are the kept raw scores).
 //
 // Exactness: x and W_router are bf16, so every product is exact in fp32.  The
-// K loop is split over 8 TMEM accumulators (k-block kb accumulates into
-// kb % 8) that the epilogue adds on the CUDA cores, so no accumulation chain
-// inside the tensor core is longer than ceil(d / 512) k-blocks; this keeps
-// the logits within ~1e-6 of a float64 sum (a single long chain measured 4e-6
-// on the gates).  Scores, selection and gates are fp32 on the CUDA cores.
+// K range is cut into S chunks (one per CTA) and, inside a CTA, k-block kb of
+// the chunk accumulates into TMEM accumulator kb % G; the epilogue adds the G
+// accumulators and the selection kernel the S chunks, both on the CUDA cores
+// in a fixed order.  No accumulation chain inside the tensor core is longer
+// than ceil(kpc / G) k-blocks of 64, which keeps the logits within ~1e-6 of a
+// float64 sum (a single long chain measured 4e-6 on the gates).  Scores,
+// selection and gates are fp32 on the CUDA cores.
 //
 // Logit columns: [0, E) are the router rows; when the shared expert is
 // present its gate vector w_s is column nrw = E rounded up to 8 (so its 8-row
-// TMA box lands on a 1024-byte swizzle atom); LS = columns rounded up to 64.
+// TMA box lands on a 1024-byte swizzle atom).  BN is the smallest of 16..128
+// covering the columns; LSP, the stored row length, is the column count
+// rounded up to 16.
 #include <float.h>
 
 #include "moe_internal.cuh"
@@ -36,35 +43,51 @@ namespace rt {
 using namespace tc;
 
 constexpr int BM = 128;
-constexpr int BN = 64;
-constexpr int kStages = 8;
-constexpr int G = 8;                      // K-split accumulators: 8 x 64 = 512 TMEM columns
-constexpr int kABytes = BM * 128;         // 16 KB
-constexpr int kBBytes = BN * 128;         // 8 KB
-constexpr int kStage = kABytes + kBBytes;
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4, kTmaWarp = 4, kMmaWarp = 5;
-constexpr uint32_t kCols = 512;
+constexpr uint32_t kCols = 256;       // TMEM columns per CTA: two CTAs share an SM
+#ifndef MOE_ROUTER_TARGET_CTAS
+#define MOE_ROUTER_TARGET_CTAS 256
+#endif
+#ifndef MOE_ROUTER_MAX_BN
+#define MOE_ROUTER_MAX_BN 128
+#endif
+constexpr int kTargetCtas = MOE_ROUTER_TARGET_CTAS;   // the K split aims at about this many CTAs
+constexpr int kMaxBN = MOE_ROUTER_MAX_BN;
+constexpr int kMaxChunks = 8;         // K chunks the selection kernel adds
+constexpr int kABytes = BM * 128;     // 16 KB: 128 tokens x 64 bf16
+constexpr int kMaxStages = 5;
+
+template <int BN>
+struct Shape {
+    static constexpr int kBBytes = BN * 128;
+    static constexpr int kStage = kABytes + kBBytes;
+    // about 96 KB of ring per CTA, so two CTAs fit on an SM
+    static constexpr int kStages = BN >= 128 ? 3 : (BN >= 64 ? 4 : kMaxStages);
+    static constexpr int G = (int)kCols / BN > 8 ? 8 : (int)kCols / BN;   // K-split accumulators
+};
 
 struct LogitsArgs {
     int64_t T;
-    int d, E, nrw, LS;
+    int d, E, nrw, LSP;   // LSP: stored partial row length
+    int n_tiles, S, kpc;  // column tiles, K chunks, k-blocks per chunk
     bool shared;
-    float *logits;   // [T, LS]
+    float *partial;       // [S, T, LSP]
     uint32_t *err;
-    int32_t *hist;   // grouping histogram to clear for the selection kernel (or null)
+    int32_t *hist;        // grouping histogram to clear for the selection kernel (or null)
     int64_t hist_ints;
 };
 
 struct Ctrl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    uint64_t tfull, tempty;
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t tfull;
     uint32_t tmem_base;
     int abort;
 };
 
 // Sum of the ng partial accumulators (BN columns apart) for 16 columns.
+template <int BN, int G>
 __device__ __forceinline__ void load_logits(uint32_t taddr, int ng, float (&v)[16]) {
 #pragma unroll
     for (int q = 0; q < 16; ++q) v[q] = 0.f;
@@ -86,9 +109,13 @@ __device__ __forceinline__ void load_logits(uint32_t taddr, int ng, float (&v)[1
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 2)
     router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                         const __grid_constant__ CUtensorMap tmS, LogitsArgs a) {
+                         const __grid_constant__ CUtensorMap tmWB, const __grid_constant__ CUtensorMap tmS,
+                         LogitsArgs a) {
+    using Sh = Shape<BN>;
+    constexpr int kStages = Sh::kStages, kStage = Sh::kStage, G = Sh::G;
     constexpr uint32_t kIdesc = instr_desc<__nv_bfloat16>(BM, BN);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -102,7 +129,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&ctrl->empty[s], 1);
         }
         mbar_init(&ctrl->tfull, 1);
-        mbar_init(&ctrl->tempty, kEpiWarps * 32);
         ctrl->abort = 0;
         fence_barrier_init();
     }
@@ -110,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kTmaWarp && lane == 0) {
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmW);
+        prefetch_tmap(&tmWB);
         if (a.shared) prefetch_tmap(&tmS);
     }
     pdl_wait();   // the prologue above overlaps the previous kernel's tail
@@ -123,42 +150,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_launch_dependents();   // this CTA's TMEM is allocated
 
     const uint32_t tmem = ctrl->tmem_base;
-    const int n_tiles = a.LS / BN;
-    const int total = (int)((a.T + BM - 1) / BM) * n_tiles;
     const int nk = (a.d + 63) / 64;
+    // one tile per CTA: id -> (token tile m, column tile n, K chunk c), chunks fastest
+    const int per_m = a.n_tiles * a.S;
+    const int id = blockIdx.x;
+    const int m = id / per_m, rem = id - m * per_m, n = rem / a.S, c = rem - n * a.S;
+    const int kb0 = c * a.kpc, kb1 = min(nk, kb0 + a.kpc);
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
+            // a tile of router rows only comes in one BN-row box per K block
+            // (rows past E read as zeros); other tiles use 8-row boxes: router
+            // rows below nrw, the shared gate row at nrw, and other rows are
+            // never read
+            const bool whole = a.E >= BN && !(a.shared && a.nrw >= n * BN && a.nrw < n * BN + BN);
+            int nbox = 0;
+            for (int j = 0; j < BN / 8; ++j) {
+                const int r = n * BN + 8 * j;
+                nbox += (r < a.nrw) || (a.shared && r == a.nrw);
+            }
+            if (whole) nbox = BN / 8;
             uint32_t it = 0;
             bool ok = true;
-            for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-                const int m = id / n_tiles, n = id - m * n_tiles;
-                // 8-row boxes of the tile's logit rows: router rows below nrw, the
-                // shared gate row at nrw; other rows are never read
-                int nbox = 0;
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                const int s = it % kStages;
+                if (!wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, a.err)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = smem + s * kStage;
+                mbar_expect_tx(&ctrl->full[s], kABytes + nbox * 1024);
+                tma_load_2d(&tmX, st, &ctrl->full[s], kb * 64, m * BM);
+                if (whole) {
+                    tma_load_2d(&tmWB, st + kABytes, &ctrl->full[s], kb * 64, n * BN);
+                    continue;
+                }
                 for (int j = 0; j < BN / 8; ++j) {
                     const int r = n * BN + 8 * j;
-                    nbox += (r < a.nrw) || (a.shared && r == a.nrw);
-                }
-                for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % kStages;
-                    if (!wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, a.err)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *st = smem + s * kStage;
-                    mbar_expect_tx(&ctrl->full[s], kABytes + nbox * 1024);
-                    tma_load_2d(&tmX, st, &ctrl->full[s], kb * 64, m * BM);
-                    for (int j = 0; j < BN / 8; ++j) {
-                        const int r = n * BN + 8 * j;
-                        if (r < a.nrw)
-                            tma_load_2d(&tmW, st + kABytes + j * 1024, &ctrl->full[s], kb * 64, r);
-                        else if (a.shared && r == a.nrw)
-                            tma_load_2d(&tmS, st + kABytes + j * 1024, &ctrl->full[s], kb * 64, 0);
-                    }
+                    if (r < a.nrw)
+                        tma_load_2d(&tmW, st + kABytes + j * 1024, &ctrl->full[s], kb * 64, r);
+                    else if (a.shared && r == a.nrw)
+                        tma_load_2d(&tmS, st + kABytes + j * 1024, &ctrl->full[s], kb * 64, 0);
                 }
             }
             if (!ok) {
+                // aborting: let the copies already issued land before the CTA exits
                 for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j) {
                     const uint64_t t0 = globaltimer();
                     while (!mbar_try_wait(&ctrl->full[j % kStages], (j / kStages) & 1) &&
@@ -169,53 +205,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
-            uint32_t it = 0, tc = 0;
             bool ok = true;
-            for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++tc) {
-                if (!wait_bar(&ctrl->tempty, (tc & 1) ^ 1, abort, a.err)) break;
-                tc_fence_after();
-                for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % kStages;
-                    if (!wait_bar(&ctrl->full[s], (it / kStages) & 1, abort, a.err)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t ad = smem_desc(smem + s * kStage);
-                    const uint64_t bd = smem_desc(smem + s * kStage + kABytes);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma<__nv_bfloat16>(tmem + (kb % G) * BN, ad + 2 * kk, bd + 2 * kk, kIdesc,
-                                           (kb >= G || kk > 0) ? 1u : 0u);
-                    mma_commit(&ctrl->empty[s]);
+            for (int kb = kb0; kb < kb1; ++kb) {
+                const uint32_t it = (uint32_t)(kb - kb0);
+                const int s = it % kStages;
+                if (!wait_bar(&ctrl->full[s], (it / kStages) & 1, abort, a.err)) {
+                    ok = false;
+                    break;
                 }
-                if (ok) mma_commit(&ctrl->tfull);
+                tc_fence_after();
+                const uint64_t ad = smem_desc(smem + s * kStage);
+                const uint64_t bd = smem_desc(smem + s * kStage + kABytes);
+                const int j = kb - kb0;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma<__nv_bfloat16>(tmem + (j % G) * BN, ad + 2 * kk, bd + 2 * kk, kIdesc,
+                                       (j >= G || kk > 0) ? 1u : 0u);
+                mma_commit(&ctrl->empty[s]);
             }
+            if (ok) mma_commit(&ctrl->tfull);
         }
     } else {
-        const int row = warp * 32 + lane;
+        // epilogue: each warp takes its 32 TMEM lanes (tokens), adds the G
+        // accumulators, stages the rows in the (now idle) ring and writes each
+        // row with one coalesced warp store
+        constexpr int kLd = BN + 4;   // staged row stride in floats (conflict-free float4 stores)
+        float *stg = reinterpret_cast<float *>(smem) + warp * 32 * kLd;
         const uint32_t tb = tmem + ((uint32_t)(warp * 32) << 16);
-        const int ng = nk < G ? nk : G;
-        uint32_t tc = 0;
-        for (int id = blockIdx.x; id < total; id += gridDim.x, ++tc) {
-            const int m = id / n_tiles, n = id - m * n_tiles;
-            if (!wait_bar(&ctrl->tfull, tc & 1, abort, a.err)) break;
+        const int ng = kb1 - kb0 < G ? kb1 - kb0 : G;
+        const int ncols = min(BN, a.LSP - n * BN);   // multiple of 16
+        if (wait_bar(&ctrl->tfull, 0, abort, a.err)) {
             tc_fence_after();
-            const int64_t t = (int64_t)m * BM + row;
-            float *dst = a.logits + t * a.LS + n * BN;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
+            for (int col = 0; col < ncols; col += 16) {
                 float v[16];
-                load_logits(tb + c, ng, v);
-                if (t < a.T) {
+                load_logits<BN, G>(tb + col, ng, v);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<float4 *>(dst + c + 4 * q) =
-                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                }
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4 *>(stg + lane * kLd + col + 4 * q) =
+                        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
+            __syncwarp();
+            const int64_t t0 = (int64_t)m * BM + warp * 32;
+            float *dst = a.partial + ((int64_t)c * a.T + t0) * a.LSP + n * BN;
+            for (int rr = 0; rr < 32 && t0 + rr < a.T; ++rr)
+                for (int q = lane * 4; q < ncols; q += 128)
+                    *reinterpret_cast<float4 *>(dst + (int64_t)rr * a.LSP + q) =
+                        *reinterpret_cast<const float4 *>(stg + rr * kLd + q);
             tc_fence_before();
-            mbar_arrive(&ctrl->tempty);
         }
     }
 
@@ -227,19 +264,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // One warp per token: scoring, top-k and gates from a row of logits.
 template <int EPL>
-__global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const float *logits, int LS, int nrw) {
+__global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const float *partial, int LSP, int S,
+                                                            int nrw) {
     pdl_wait();
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+    if (a.l2_prefetch_bytes && lane == 0) {
+        // start streaming the weights the next GEMM reads first into L2; the
+        // routing kernels leave HBM idle (64 KB per warp and tensor)
+        constexpr size_t kChunk = 65536;
+        const size_t n = (a.l2_prefetch_bytes + kChunk - 1) / kChunk;
+        for (size_t c = (size_t)t; c < 2 * n; c += (size_t)gridDim.x * 8) {
+            const size_t off = (c % n) * kChunk;
+            const size_t len = a.l2_prefetch_bytes - off < kChunk ? a.l2_prefetch_bytes - off : kChunk;
+            if (len >= 16) prefetch_l2(static_cast<const char *>(a.l2_prefetch[c / n]) + off, (uint32_t)(len & ~size_t(15)));
+        }
+    }
     if (t >= a.T) return;
-    const float *row = logits + t * LS;
     const bool sigm = a.score == MOE_SCORE_SIGMOID;
+    // the token's logits: its S partial rows added in chunk order
+    const int64_t slab = a.T * (int64_t)LSP;
+    const float *row = partial + t * LSP;
     float l[EPL], key[EPL];
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) l[q] = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+        if (c < S) {
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = lane + 32 * q;
+                if (e < a.E) l[q] += row[c * slab + e];
+            }
+        }
+    }
 #pragma unroll
     for (int q = 0; q < EPL; ++q) {
         const int e = lane + 32 * q;
-        l[q] = e < a.E ? row[e] : -FLT_MAX;
+        if (e >= a.E) l[q] = -FLT_MAX;
         key[q] = sigm ? 1.f / (1.f + expf(-l[q])) : l[q];
     }
     if (a.zero_rows) {
@@ -314,23 +377,69 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
             if (e < a.E) a.probs[t * a.E + e] = sigm ? key[q] : expf(l[q] - m) / z;
         }
     }
-    if (lane == 0 && a.shared_gate && a.w_shared_gate) a.shared_gate[t] = 1.f / (1.f + expf(-row[nrw]));
+    if (lane == 0 && a.shared_gate && a.w_shared_gate) {
+        float ls = 0.f;
+        for (int c = 0; c < S; ++c) ls += row[c * slab + nrw];
+        a.shared_gate[t] = 1.f / (1.f + expf(-ls));
+    }
 }
 
-struct Geometry {
-    int nrw, LS;
+// Tiling of the logits GEMM for a batch (a pure function of the shape).
+struct Plan {
+    int nrw, L, BN, LSP, n_tiles, nk, S, kpc;
+    int64_t m_tiles;
 };
-Geometry geometry(int E, bool shared) {
-    Geometry g;
-    g.nrw = (E + 7) / 8 * 8;
-    g.LS = (g.nrw + (shared ? 1 : 0) + BN - 1) / BN * BN;
-    return g;
+Plan plan(int64_t T, int d, int E, bool shared) {
+    Plan p;
+    p.nrw = (E + 7) / 8 * 8;
+    p.L = p.nrw + (shared ? 1 : 0);
+    p.BN = 16;
+    while (p.BN < p.L && p.BN < kMaxBN) p.BN *= 2;
+    p.n_tiles = (p.L + p.BN - 1) / p.BN;
+    p.LSP = (p.L + 15) / 16 * 16;
+    p.nk = (d + 63) / 64;
+    p.m_tiles = (T + BM - 1) / BM;
+    const int64_t tiles = p.m_tiles * p.n_tiles;
+    int64_t S = kTargetCtas / tiles;
+    S = S < 1 ? 1 : (S > p.nk ? p.nk : S);
+    S = S > kMaxChunks ? kMaxChunks : S;
+    p.kpc = (int)((p.nk + S - 1) / S);
+    p.S = (p.nk + p.kpc - 1) / p.kpc;
+    return p;
+}
+
+template <int BN>
+cudaError_t launch_logits(const RouterArgs &a, const Plan &p, float *partial, cudaStream_t s) {
+    const bool shared = a.w_shared_gate != nullptr;
+    CUtensorMap mX, mW, mWB, mS;
+    if (!make_map(&mX, a.x, false, (uint64_t)a.T, a.d, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&mW, a.w_router, false, (uint64_t)a.E, a.d, 8)) return cudaErrorInvalidValue;
+    if (a.E >= BN) {
+        if (!make_map(&mWB, a.w_router, false, (uint64_t)a.E, a.d, BN)) return cudaErrorInvalidValue;
+    } else {
+        mWB = mW;   // unused: tiles of fewer than BN router rows take 8-row boxes
+    }
+    if (shared) {
+        if (!make_map(&mS, a.w_shared_gate, false, 1, a.d, 8)) return cudaErrorInvalidValue;
+    } else {
+        mS = mW;
+    }
+    const int64_t hist_ints = a.hist ? ((a.T * a.k + a.hist_chunk - 1) / a.hist_chunk) * (a.E + 1) : 0;
+    LogitsArgs la{a.T, a.d, a.E, p.nrw, p.LSP, p.n_tiles, p.S, p.kpc, shared, partial, a.err, a.hist, hist_ints};
+    const size_t smem = 1024 + (size_t)Shape<BN>::kStages * Shape<BN>::kStage + sizeof(Ctrl);
+    auto kern = router_logits_kernel<BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = p.m_tiles * p.n_tiles * p.S;   // one tile per CTA
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    return launch_kernel(kern, (unsigned)grid, kThreads, smem, s, mX, mW, mWB, mS, la);
 }
 
 }  // namespace rt
 
-size_t router_tc_workspace_bytes(int64_t T, int E, bool shared) {
-    return sizeof(float) * (size_t)T * rt::geometry(E, shared).LS;
+size_t router_tc_workspace_bytes(int64_t T, int d, int E, bool shared) {
+    const rt::Plan p = rt::plan(T, d, E, shared);
+    return sizeof(float) * (size_t)p.S * (size_t)T * p.LSP;
 }
 
 bool router_tc_supported(int64_t T, int E, int dtype) {
@@ -339,31 +448,21 @@ bool router_tc_supported(int64_t T, int E, int dtype) {
 
 cudaError_t launch_router_tc(const RouterArgs &a, float *scratch, cudaStream_t s) {
     using namespace rt;
-    const bool shared = a.w_shared_gate != nullptr;
-    const Geometry g = geometry(a.E, shared);
-    CUtensorMap mX, mW, mS;
-    if (!tc::make_map(&mX, a.x, false, (uint64_t)a.T, a.d, BM)) return cudaErrorInvalidValue;
-    if (!tc::make_map(&mW, a.w_router, false, (uint64_t)a.E, a.d, 8)) return cudaErrorInvalidValue;
-    if (shared) {
-        if (!tc::make_map(&mS, a.w_shared_gate, false, 1, a.d, 8)) return cudaErrorInvalidValue;
-    } else {
-        mS = mW;
+    const Plan p = plan(a.T, a.d, a.E, a.w_shared_gate != nullptr);
+    cudaError_t e;
+    switch (p.BN) {
+        case 16: e = launch_logits<16>(a, p, scratch, s); break;
+        case 32: e = launch_logits<32>(a, p, scratch, s); break;
+        case 64: e = launch_logits<64>(a, p, scratch, s); break;
+        default: e = launch_logits<128>(a, p, scratch, s); break;
     }
-    const int64_t hist_ints = a.hist ? ((a.T * a.k + a.hist_chunk - 1) / a.hist_chunk) * (a.E + 1) : 0;
-    LogitsArgs la{a.T, a.d, a.E, g.nrw, g.LS, shared, scratch, a.err, a.hist, hist_ints};
-    const size_t smem = 1024 + (size_t)kStages * kStage + sizeof(Ctrl);
-    cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int total = (int)((a.T + BM - 1) / BM) * (g.LS / BN);
-    const int grid = total < num_sms() ? total : num_sms();
-    e = launch_kernel(router_logits_kernel, grid, kThreads, smem, s, mX, mW, mS, la);
     if (e != cudaSuccess) return e;
     const unsigned sgrid = (unsigned)((a.T + 7) / 8);
-    const float *lg = scratch;
-    if (a.E <= 64) return launch_kernel(router_select_kernel<2>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
-    if (a.E <= 128) return launch_kernel(router_select_kernel<4>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
-    if (a.E <= 256) return launch_kernel(router_select_kernel<8>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
-    return launch_kernel(router_select_kernel<16>, sgrid, 256, 0, s, a, lg, g.LS, g.nrw);
+    const float *pt = scratch;
+    if (a.E <= 64) return launch_kernel(router_select_kernel<2>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
+    if (a.E <= 128) return launch_kernel(router_select_kernel<4>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
+    if (a.E <= 256) return launch_kernel(router_select_kernel<8>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
+    return launch_kernel(router_select_kernel<16>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
 }
 
 }  // namespace moe

@@ -64,7 +64,9 @@ def test_null_pointers_rejected_before_launch():
     assert L.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, None, None, None, 0, None) == 1
     assert L.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None, 0, None) == 1  # no w_s
     big = B.config_of(WORKLOADS["olmoe_zipf"])
-    assert B.route_workspace_size(big) == 8192 * 64 * 4
+    # fp32 partial logits: one [T, 64] slab per chunk of the K range
+    n = B.route_workspace_size(big)
+    assert n >= 8192 * 64 * 4 and n % (8192 * 64 * 4) == 0 and n // (8192 * 64 * 4) <= 2048 // 64
     assert L.moe_route(ctypes.byref(big), fake, fake, None, fake, fake, None, None, None, 0, None) == 3
     assert L.moe_permute(ctypes.byref(cfg), fake, None, fake, fake, fake, fake, 1 << 20, None) == 1
     assert L.moe_permute(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, 0, None) == 3
