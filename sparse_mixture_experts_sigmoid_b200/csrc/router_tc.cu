@@ -283,26 +283,50 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
     }
     if (t >= a.T) return;
     const bool sigm = a.score == MOE_SCORE_SIGMOID;
-    // the token's logits: its S partial rows added in chunk order
+    // the token's logits: lane owns experts lane * EPL .. + EPL - 1; its S
+    // partial rows are read with vector loads, a group of chunks at a time with
+    // all loads issued before the adds, and added in chunk order
     const int64_t slab = a.T * (int64_t)LSP;
     const float *row = partial + t * LSP;
+    const int e0 = lane * EPL;
+    const bool mine = e0 < LSP;   // then all EPL columns lie inside the row (LSP % 16 == 0)
     float l[EPL], key[EPL];
 #pragma unroll
     for (int q = 0; q < EPL; ++q) l[q] = 0.f;
+    constexpr int kGroup = EPL <= 8 ? 8 : 4;
 #pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c) {
-        if (c < S) {
+    for (int c0 = 0; c0 < kMaxChunks; c0 += kGroup) {
+        if (c0 < S) {
+            float v[kGroup][EPL];
 #pragma unroll
-            for (int q = 0; q < EPL; ++q) {
-                const int e = lane + 32 * q;
-                if (e < a.E) l[q] += row[c * slab + e];
+            for (int g = 0; g < kGroup; ++g) {
+                const int c = c0 + g < S ? c0 + g : S - 1;   // clamped: always a valid row
+                const float *src = row + c * slab + (mine ? e0 : 0);
+#pragma unroll
+                for (int q = 0; q < EPL; q += (EPL >= 4 ? 4 : EPL)) {
+                    if constexpr (EPL >= 4) {
+                        const float4 u = *reinterpret_cast<const float4 *>(src + q);
+                        v[g][q] = u.x;
+                        v[g][q + 1] = u.y;
+                        v[g][q + 2] = u.z;
+                        v[g][q + 3] = u.w;
+                    } else {
+                        const float2 u = *reinterpret_cast<const float2 *>(src + q);
+                        v[g][q] = u.x;
+                        v[g][q + 1] = u.y;
+                    }
+                }
             }
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g)
+                if (c0 + g < S)
+#pragma unroll
+                    for (int q = 0; q < EPL; ++q) l[q] += v[g][q];
         }
     }
 #pragma unroll
     for (int q = 0; q < EPL; ++q) {
-        const int e = lane + 32 * q;
-        if (e >= a.E) l[q] = -FLT_MAX;
+        if (!mine || e0 + q >= a.E) l[q] = -FLT_MAX;
         key[q] = sigm ? 1.f / (1.f + expf(-l[q])) : l[q];
     }
     if (a.zero_rows) {
@@ -312,14 +336,14 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
     float m = -FLT_MAX;
 #pragma unroll
     for (int q = 0; q < EPL; ++q)
-        if (lane + 32 * q < a.E) m = fmaxf(m, l[q]);
+        if (e0 + q < a.E) m = fmaxf(m, l[q]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float z = 0.f;
     if (!sigm) {
 #pragma unroll
         for (int q = 0; q < EPL; ++q)
-            if (lane + 32 * q < a.E) z += expf(l[q] - m);
+            if (e0 + q < a.E) z += expf(l[q] - m);
         z = warp_sum(z);
     }
     uint32_t taken = 0;
@@ -330,7 +354,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
         int be = 0x7fffffff;
 #pragma unroll
         for (int q = 0; q < EPL; ++q) {
-            const int e = lane + 32 * q;
+            const int e = e0 + q;
             if (e < a.E && !((taken >> q) & 1u) && (key[q] > bk || (key[q] == bk && e < be))) {
                 bk = key[q];
                 be = e;
@@ -349,7 +373,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
             }
         }
         if (be >= a.E) be = j;   // only reachable with non-finite logits; keeps ids in range
-        if (lane == (be & 31)) taken |= 1u << (be >> 5);
+        if (lane == be / EPL) taken |= 1u << (be % EPL);
         if (lane == j) {
             my_e = be;
             my_l = bl;
@@ -373,7 +397,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
     if (a.probs) {
 #pragma unroll
         for (int q = 0; q < EPL; ++q) {
-            const int e = lane + 32 * q;
+            const int e = e0 + q;
             if (e < a.E) a.probs[t * a.E + e] = sigm ? key[q] : expf(l[q] - m) / z;
         }
     }
