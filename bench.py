@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
 L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
 # stage -> (kernel name in the ncu launch list, source file whose hash keys the traffic figure)
-STAGE_KERNEL = {"route": ("router_tc_kernel", "router_tc.cu"), "permute": ("scatter_kernel", "permute.cu"),
+STAGE_KERNEL = {"route": ("router_logits_kernel", "router_tc.cu"), "permute": ("scatter_kernel", "permute.cu"),
                 "gate_up": ("grouped_gemm_kernel", "grouped_gemm.cu"),
                 "shared_gate_up": ("grouped_gemm_kernel", "grouped_gemm.cu"),
                 "down": ("grouped_gemm_kernel", "grouped_gemm.cu"),

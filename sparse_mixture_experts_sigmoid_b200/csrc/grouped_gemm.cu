@@ -140,11 +140,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     __syncthreads();
     tc_fence_after();
     // dependents are released only after this CTA's TMEM is allocated and after
-    // the wait: every thread but the producer waits here, the producer once it
-    // has issued the early loads
+    // the wait.  With early loads the producer warp skips the wait here (a warp
+    // waits as a whole) and its issuing lane waits once it has issued them.
     if (!early_tiles) {
         pdl_launch_dependents();
-    } else if (!(warp == kTmaWarp && lane == 0)) {
+    } else if (warp != kTmaWarp) {
         pdl_wait();
         pdl_launch_dependents();
     }
