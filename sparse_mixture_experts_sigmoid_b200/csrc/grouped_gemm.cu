@@ -157,12 +157,19 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
+            // weights that no other tile reads again stream through L2 with an
+            // evict-first policy, so what is reused from L2 (prefetched weights,
+            // the gathered rows, act, the combine accumulator) stays
+            const uint64_t wpol = l2_evict_first_policy();
             auto load_b = [&](int s, int kb, int b_row) {
-                if (MODE == GATEUP) {
-                    tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
-                    tma_load_2d(&tmB1, sB + s * kBBytes + kBBytes / 2, &ctrl->full[s], kb * BK, b_row);
+                if (p.stream_weights) {
+                    tma_load_2d_hint(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row, wpol);
+                    if (MODE == GATEUP)
+                        tma_load_2d_hint(&tmB1, sB + s * kBBytes + kBBytes / 2, &ctrl->full[s], kb * BK, b_row, wpol);
                 } else {
                     tma_load_2d(&tmB0, sB + s * kBBytes, &ctrl->full[s], kb * BK, b_row);
+                    if (MODE == GATEUP)
+                        tma_load_2d(&tmB1, sB + s * kBBytes + kBBytes / 2, &ctrl->full[s], kb * BK, b_row);
                 }
             };
             const bool early_a = !GATHER && (p.early & kEarlyA) != 0;

@@ -103,6 +103,9 @@ constexpr int32_t kDecodeMaxRows = 64;
 bool narrow_gateup(const moe_config &c) { return c.h % 128 != 0; }
 bool narrow_down(const moe_config &c) { return c.d % 256 != 0; }
 
+// Experts average at most one 128-row tile: every weight tile is read once.
+bool one_tile_per_expert(const moe_config &c) { return (int64_t)c.T * c.k <= 128LL * c.E; }
+
 GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const void *wu, const int32_t *offsets,
                        const int32_t *srt, void *act, uint32_t *err) {
     GemmLaunch L{};
@@ -111,6 +114,7 @@ GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const
     L.dtype = c.dtype;
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.d, c.h, x, act, nullptr, nullptr, err};
     L.narrow = narrow_gateup(c);
+    L.p.stream_weights = one_tile_per_expert(c);
     L.b0 = wg;
     L.b1 = wu;
     return L;
@@ -135,6 +139,7 @@ GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const
     L.dtype = c.dtype;
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.h, c.d, nullptr, nullptr, acc, gates, err};
     L.narrow = narrow_down(c);
+    L.p.stream_weights = one_tile_per_expert(c);
     L.a_src = act;
     L.b0 = wd;
     return L;
@@ -163,17 +168,6 @@ GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const
 }
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
-
-// Bytes of gate/up weights prefetched into L2 during routing (MOE_L2_PREFETCH_MB,
-// default 64; 0 turns it off).
-size_t l2_prefetch_budget() {
-    static const size_t v = [] {
-        const char *e = std::getenv("MOE_L2_PREFETCH_MB");
-        const long mb = e ? std::atol(e) : 64;
-        return (size_t)(mb > 0 ? mb : 0) << 20;
-    }();
-    return v;
-}
 
 bool pdl_enabled() {
     static const bool on = [] {
@@ -422,14 +416,6 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     const bool fused_hist = L.size[P_LOGITS] && c->T * c->k > permute_chunk();
     ra.hist = fused_hist ? part<int32_t>(ws, L, P_PERM) : nullptr;
     ra.hist_chunk = permute_chunk();
-    if (use_gemm(*c) && (int64_t)c->T * c->k >= 4LL * c->E) {
-        // most experts are active: prefetch the expert weights the gate/up GEMM
-        // reads first (its tiles walk the experts in order) while routing runs
-        const size_t per = (size_t)c->E * c->h * c->d * (c->dtype == MOE_F32 ? 4 : 2);
-        ra.l2_prefetch[0] = w_gate;
-        ra.l2_prefetch[1] = w_up;
-        ra.l2_prefetch_bytes = per < l2_prefetch_budget() / 2 ? per : l2_prefetch_budget() / 2;
-    }
     mark(0, s);
     cudaError_t e = launch_router(ra, c->dtype, part<float>(ws, L, P_LOGITS), s);
     mark(1 + MOE_STAGE_ROUTE, s);

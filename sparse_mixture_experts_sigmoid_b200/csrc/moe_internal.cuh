@@ -81,11 +81,6 @@ struct RouterArgs {
     uint32_t *err;      // device error word
     int32_t *hist;      // optional [B, E+1] block histogram for grouping (tensor-core router only)
     int hist_chunk;     // assignments per histogram block
-    // optional: the first l2_prefetch_bytes of each of two weight tensors that the
-    // grouped GEMM after the router reads first, brought into L2 while routing
-    // runs (tensor-core router only; a hint, no data dependence)
-    const void *l2_prefetch[2];
-    size_t l2_prefetch_bytes;
 };
 // Router: the tensor-core logits GEMM + warp-per-token selection (router_tc.cu)
 // when supported and scratch is given, else the CUDA-core routers (router.cu).
@@ -163,6 +158,7 @@ struct GemmParams {
     float *y_acc;                // down output [T, N] fp32, accumulated into
     const float *gates;          // down: routed [R] by assignment, dense [T]
     uint32_t *err;
+    bool stream_weights;         // each weight tile is read by one tile only: load it evict-first
     float *zero;                 // gate/up only, optional: [zero_floats] fp32 to clear (the
     int64_t zero_floats;         // down GEMM's accumulator), spread over the CTAs
     // kEarly* bits: what the kernel may read before the previous kernel in the
@@ -195,11 +191,6 @@ int num_sms();
 
 // Counts one kernel launch (for moe_launch_count).
 void note_launch();
-
-// Asynchronous prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 
 // ------------------------------------------------------------------ programmatic dependent launch
 // Every kernel of a pass is launched with programmatic stream serialization, so

@@ -262,26 +262,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == kMmaWarp) tmem_dealloc(tmem, kCols);
 }
 
-// One warp per token: scoring, top-k and gates from a row of logits.
+// The selection for token t by one warp (see router_select_kernel).
 template <int EPL>
-__global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const float *partial, int LSP, int S,
-                                                            int nrw) {
-    pdl_wait();
-    pdl_launch_dependents();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-    if (a.l2_prefetch_bytes && lane == 0) {
-        // start streaming the weights the next GEMM reads first into L2; the
-        // routing kernels leave HBM idle (64 KB per warp and tensor)
-        constexpr size_t kChunk = 65536;
-        const size_t n = (a.l2_prefetch_bytes + kChunk - 1) / kChunk;
-        for (size_t c = (size_t)t; c < 2 * n; c += (size_t)gridDim.x * 8) {
-            const size_t off = (c % n) * kChunk;
-            const size_t len = a.l2_prefetch_bytes - off < kChunk ? a.l2_prefetch_bytes - off : kChunk;
-            if (len >= 16) prefetch_l2(static_cast<const char *>(a.l2_prefetch[c / n]) + off, (uint32_t)(len & ~size_t(15)));
-        }
-    }
-    if (t >= a.T) return;
+__device__ __forceinline__ void select_token(const RouterArgs &a, const float *partial, int LSP, int S, int nrw,
+                                             int64_t t, int lane) {
     const bool sigm = a.score == MOE_SCORE_SIGMOID;
     // the token's logits: lane owns experts lane * EPL .. + EPL - 1; its S
     // partial rows are read with vector loads, a group of chunks at a time with
@@ -406,6 +390,17 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const 
         for (int c = 0; c < S; ++c) ls += row[c * slab + nrw];
         a.shared_gate[t] = 1.f / (1.f + expf(-ls));
     }
+}
+
+// One warp per token: scoring, top-k and gates from a row of logits.
+template <int EPL>
+__global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const float *partial, int LSP, int S,
+                                                            int nrw) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+    if (t < a.T) select_token<EPL>(a, partial, LSP, S, nrw, t, lane);
 }
 
 // Tiling of the logits GEMM for a batch (a pure function of the shape).

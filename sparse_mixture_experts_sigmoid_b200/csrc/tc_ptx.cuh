@@ -75,17 +75,21 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *m, void *dst, uin
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
-// Four rows (r0..r3) of a 2D tensor, 128 bytes each at column c0, into four
-// consecutive 128-byte rows of shared memory (swizzled by address as the
-// tensor map says).  The tensor map's box is one row high.
-__device__ __forceinline__ void tma_gather4(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
+// The same load with an L2 cache policy (from createpolicy).
+__device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int c1,
+                                                 uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-          "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
+}
+// L2 policy under which the lines a streamed operand brings in are evicted
+// first, so data reused through L2 (activations, the combine accumulator) stays.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
