@@ -273,39 +273,45 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             const uint32_t tbase = tmem + acc * BN + lane_base;
             if constexpr (MODE == GATEUP) {
                 T *act = static_cast<T *>(p.act);
-#pragma unroll 1
-                for (int c = 0; c < BN_OUT; c += 16) {
-                    float g[16], u[16];
-                    tmem_ld16(tbase + c, g);
-                    tmem_ld16(tbase + BN_OUT + c, u);
-                    tmem_wait_ld();
+                // silu(g) * u for 16 output columns from column c of the tile
+                auto store16 = [&](int c, const float(&g)[16], const float(&u)[16]) {
                     const int col = tl.n * BN_OUT + c;
-                    if (valid && col < p.N) {
-                        T *dst = act + r * p.N + col;
+                    if (!valid || col >= p.N) return;
+                    T *dst = act + r * p.N + col;
 #pragma unroll
-                        for (int h8 = 0; h8 < 2; ++h8) {
-                            if (col + 8 * h8 < p.N) {
-                                if constexpr (sizeof(T) == 2) {
-                                    uint32_t w[4];
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        if (col + 8 * h8 >= p.N) continue;
+                        if constexpr (sizeof(T) == 2) {
+                            uint32_t w[4];
 #pragma unroll
-                                    for (int q = 0; q < 4; ++q) {
-                                        const int i0 = 8 * h8 + 2 * q;
-                                        __nv_bfloat162 b2 = __floats2bfloat162_rn(silu_f(g[i0]) * u[i0],
-                                                                                  silu_f(g[i0 + 1]) * u[i0 + 1]);
-                                        w[q] = *reinterpret_cast<uint32_t *>(&b2);
-                                    }
-                                    *reinterpret_cast<uint4 *>(dst + 8 * h8) = make_uint4(w[0], w[1], w[2], w[3]);
-                                } else {
-                                    float o[8];
-#pragma unroll
-                                    for (int q = 0; q < 8; ++q) o[q] = silu_f(g[8 * h8 + q]) * u[8 * h8 + q];
-                                    float *fd = reinterpret_cast<float *>(dst + 8 * h8);
-                                    *reinterpret_cast<float4 *>(fd) = make_float4(o[0], o[1], o[2], o[3]);
-                                    *reinterpret_cast<float4 *>(fd + 4) = make_float4(o[4], o[5], o[6], o[7]);
-                                }
+                            for (int q = 0; q < 4; ++q) {
+                                const int i0 = 8 * h8 + 2 * q;
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(silu_f(g[i0]) * u[i0],
+                                                                          silu_f(g[i0 + 1]) * u[i0 + 1]);
+                                w[q] = *reinterpret_cast<uint32_t *>(&b2);
                             }
+                            *reinterpret_cast<uint4 *>(dst + 8 * h8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        } else {
+                            float o[8];
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) o[q] = silu_f(g[8 * h8 + q]) * u[8 * h8 + q];
+                            float *fd = reinterpret_cast<float *>(dst + 8 * h8);
+                            *reinterpret_cast<float4 *>(fd) = make_float4(o[0], o[1], o[2], o[3]);
+                            *reinterpret_cast<float4 *>(fd + 4) = make_float4(o[4], o[5], o[6], o[7]);
                         }
                     }
+                };
+                // 32 output columns per TMEM wait: four loads in flight at a time
+#pragma unroll 1
+                for (int c = 0; c < BN_OUT; c += 32) {
+                    float g[2][16], u[2][16];
+                    tmem_ld16(tbase + c, g[0]);
+                    tmem_ld16(tbase + c + 16, g[1]);
+                    tmem_ld16(tbase + BN_OUT + c, u[0]);
+                    tmem_ld16(tbase + BN_OUT + c + 16, u[1]);
+                    tmem_wait_ld();
+                    store16(c, g[0], u[0]);
+                    store16(c + 16, g[1], u[1]);
                 }
             } else {
                 int64_t t = -1;
@@ -324,20 +330,23 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                         t = -1;
                     }
                 }
+                // 32 columns per TMEM wait: two loads in flight at a time
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    float v[16];
-                    tmem_ld16(tbase + c, v);
+                for (int c = 0; c < BN; c += 32) {
+                    float v[2][16];
+                    tmem_ld16(tbase + c, v[0]);
+                    tmem_ld16(tbase + c + 16, v[1]);
                     tmem_wait_ld();
-                    const int col = tl.n * BN + c;
-                    if (t >= 0) {
+#pragma unroll
+                    for (int hh = 0; hh < 2 && t >= 0; ++hh) {
+                        const int col = tl.n * BN + c + 16 * hh;
                         float *dst = p.y_acc + t * p.N + col;
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             if (col + 4 * q < p.N)
                                 atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
-                                          make_float4(gate * v[4 * q], gate * v[4 * q + 1], gate * v[4 * q + 2],
-                                                      gate * v[4 * q + 3]));
+                                          make_float4(gate * v[hh][4 * q], gate * v[hh][4 * q + 1],
+                                                      gate * v[hh][4 * q + 2], gate * v[hh][4 * q + 3]));
                     }
                 }
             }
