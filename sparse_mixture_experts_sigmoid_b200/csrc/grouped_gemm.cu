@@ -239,6 +239,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                         ok = false;
                         break;
                     }
+                    // gathered rows were written by cp.async (generic proxy); the
+                    // MMA reads them through the async proxy
+                    if constexpr (GATHER) fence_proxy_async();
                     tc_fence_after();
                     const uint64_t ad = smem_desc(sA + s * kABytes);
                     const uint64_t bd = smem_desc(sB + s * kBBytes);
