@@ -43,9 +43,7 @@
 //    outstanding copies are drained and TMEM is released before exit.
 #include <algorithm>
 
-#include "grouped_tiles.cuh"
-#include "moe_internal.cuh"
-#include "tc_ptx.cuh"
+#include "grouped_parts.cuh"
 
 namespace moe {
 namespace gg {
@@ -69,8 +67,6 @@ constexpr int kMmaWarp = 5;
 constexpr int kGatherWarp0 = 6;
 constexpr int kGatherThreads = 128;
 constexpr int kTmemCols = 512;
-
-enum { GATEUP = 0, DOWN = 1 };
 
 using Params = GemmParams;
 
@@ -96,7 +92,6 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     constexpr int kStages = stages_for(BN);
     constexpr int kBBytes = BN * 128;                      // one B stage: BN rows x 128 bytes
     constexpr uint32_t kIdesc = instr_desc<T>(BM, BN);
-    constexpr int V = 16 / (int)sizeof(T);     // elements per 16-byte chunk
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -272,156 +267,13 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM + row;
-            const bool valid = r < seg_end[tl.e];
-            const uint32_t tbase = tmem + acc * BN + lane_base;
-            if constexpr (MODE == GATEUP) {
-                T *act = static_cast<T *>(p.act);
-                // silu(g) * u for 16 output columns from column c of the tile
-                auto store16 = [&](int c, const float(&g)[16], const float(&u)[16]) {
-                    const int col = tl.n * BN_OUT + c;
-                    if (!valid || col >= p.N) return;
-                    T *dst = act + r * p.N + col;
-#pragma unroll
-                    for (int h8 = 0; h8 < 2; ++h8) {
-                        if (col + 8 * h8 >= p.N) continue;
-                        if constexpr (sizeof(T) == 2) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const int i0 = 8 * h8 + 2 * q;
-                                __nv_bfloat162 b2 = __floats2bfloat162_rn(silu_f(g[i0]) * u[i0],
-                                                                          silu_f(g[i0 + 1]) * u[i0 + 1]);
-                                w[q] = *reinterpret_cast<uint32_t *>(&b2);
-                            }
-                            *reinterpret_cast<uint4 *>(dst + 8 * h8) = make_uint4(w[0], w[1], w[2], w[3]);
-                        } else {
-                            float o[8];
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) o[q] = silu_f(g[8 * h8 + q]) * u[8 * h8 + q];
-                            float *fd = reinterpret_cast<float *>(dst + 8 * h8);
-                            *reinterpret_cast<float4 *>(fd) = make_float4(o[0], o[1], o[2], o[3]);
-                            *reinterpret_cast<float4 *>(fd + 4) = make_float4(o[4], o[5], o[6], o[7]);
-                        }
-                    }
-                };
-                // 32 output columns per TMEM wait: four loads in flight at a time
-#pragma unroll 1
-                for (int c = 0; c < BN_OUT; c += 32) {
-                    float g[2][16], u[2][16];
-                    tmem_ld16(tbase + c, g[0]);
-                    tmem_ld16(tbase + c + 16, g[1]);
-                    tmem_ld16(tbase + BN_OUT + c, u[0]);
-                    tmem_ld16(tbase + BN_OUT + c + 16, u[1]);
-                    tmem_wait_ld();
-                    store16(c, g[0], u[0]);
-                    store16(c + 16, g[1], u[1]);
-                }
-            } else {
-                int64_t t = -1;
-                float gate = 0.f;
-                if (valid) {
-                    if (p.sorted_rows) {
-                        const int v = p.sorted_rows[r];
-                        t = v / p.k;
-                        gate = (v >= 0 && v < p.rows) ? p.gates[v] : 0.f;
-                    } else {
-                        t = r;
-                        gate = p.gates[r];
-                    }
-                    if (t < 0 || t >= p.T) {
-                        atomicOr(p.err, kErrInput);
-                        t = -1;
-                    }
-                }
-                // 32 columns per TMEM wait: two loads in flight at a time
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    float v[2][16];
-                    tmem_ld16(tbase + c, v[0]);
-                    tmem_ld16(tbase + c + 16, v[1]);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int hh = 0; hh < 2 && t >= 0; ++hh) {
-                        const int col = tl.n * BN + c + 16 * hh;
-                        float *dst = p.y_acc + t * p.N + col;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (col + 4 * q < p.N)
-                                atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
-                                          make_float4(gate * v[hh][4 * q], gate * v[hh][4 * q + 1],
-                                                      gate * v[hh][4 * q + 2], gate * v[hh][4 * q + 3]));
-                    }
-                }
-            }
+            epilogue_row<MODE, T, BN>(p, tl.n, r, r < seg_end[tl.e], tmem + acc * BN + lane_base);
             tc_fence_before();
             mbar_arrive(&ctrl->tempty[acc]);
         }
     } else if (GATHER && warp >= kGatherWarp0) {
-        // gather producers: token rows of x by index, 16-byte cp.async into the
-        // swizzled K-major layout (8 threads per row, 16 rows per pass)
-        const int g = threadIdx.x - kGatherWarp0 * 32;   // 0..127
-        const int c = g & 7;                             // 16-byte chunk of the 128-byte row
-        const int rg = g >> 3;                           // rows rg, rg + 16, ..., rg + 112
-        const int swz = (c ^ (rg & 7)) << 4;             // 128-byte swizzle: chunk ^ (row mod 8)
-        const T *x = static_cast<const T *>(p.x);
-        // the assignment ids of this thread's eight rows, loaded one tile ahead so
-        // the index loads of the next tile overlap the copies of the current one
-        auto load_ids = [&](int id, int (&v)[8]) {
-            if (id >= total) return;
-            const Tile tl = decode(id, n_tiles, tile_start, nE);
-            const int64_t row0 = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM;
-            const int64_t rend = seg_end[tl.e];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int64_t r = row0 + rg + 16 * q;
-                v[q] = r < rend ? p.sorted_rows[r] : -1;
-            }
-        };
-        int vnext[8];
-        load_ids(blockIdx.x, vnext);
-        uint32_t it = 0;
-        bool ok = true;
-        for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-            int vcur[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) vcur[q] = vnext[q];
-            load_ids(id + gridDim.x, vnext);
-            const T *src[8];
-            uint32_t okmask = 0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                src[q] = x;
-                const int v = vcur[q];
-                if (v != -1) {
-                    const int64_t t = v / p.k;
-                    if (v >= 0 && t < p.T) {
-                        src[q] = x + t * p.K + c * V;
-                        okmask |= 1u << q;
-                    } else {
-                        atomicOr(p.err, kErrInput);
-                    }
-                }
-            }
-            for (int kb = 0; kb < nk; ++kb, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                if (!wait_bar(&ctrl->empty[s], ph ^ 1, abort, p.err)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *dst = sA + s * kABytes + rg * 128 + swz;
-                const bool colok = kb * BK + c * V < p.K;
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    if (okmask & (1u << q))
-                        cp_async16(dst + q * 16 * 128, colok ? (const void *)(src[q] + kb * BK) : (const void *)x,
-                                   colok ? 16 : 0);
-                cp_async_commit();
-                // the barrier receives this thread's arrival once its copies have landed
-                cp_async_arrive_noinc(&ctrl->full[s]);
-            }
-        }
-        cp_async_wait<0>();
+        gather_rows<T, kStages, BM>(p, threadIdx.x - kGatherWarp0 * 32, blockIdx.x, gridDim.x, total, n_tiles,
+                                    tile_start, seg_off, seg_end, nE, nk, 0, sA, ctrl->full, ctrl->empty, abort);
     }
 
     tc_fence_before();
@@ -473,6 +325,7 @@ cudaError_t launch_bn(const GemmLaunch &L, cudaStream_t s) {
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s) {
     const GemmParams &p = L.p;
     if (p.rows <= 0) return cudaSuccess;
+    if (L.pair) return launch_grouped_gemm_pair(L, s);
     const bool f32 = L.dtype == MOE_F32;
     if (L.mode == gg::GATEUP) {
         if (L.gather)

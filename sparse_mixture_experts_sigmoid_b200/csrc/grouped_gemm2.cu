@@ -1,0 +1,340 @@
+// Grouped expert GEMMs on two SMs per tile (tcgen05.mma.cta_group::2), for
+// layers whose experts hold many rows (the tensor-bound regime).
+//
+// Same math and tile order as grouped_gemm.cu ("Tutorial 11: Mixture of
+// Experts (MoE)", section 3 "Expert Computation"), with the tiles doubled in
+// M: a cluster of two CTAs computes 256 grouped rows x BN columns.  Each CTA
+// stages its own 128 rows of A and its own half of the B columns (for gate/up:
+// CTA 0 the gate rows, CTA 1 the up rows), so per K block a CTA moves 32 KB
+// into shared memory for the same MMA work that costs 48 KB on one SM: the
+// operand traffic per FLOP, which bounds the one-SM kernel on these layers,
+// drops by a third.  The even CTA issues M=256 MMAs that read both CTAs'
+// shared memory and write each CTA's half of D into its own TMEM.
+//
+// Synchronisation across the pair:
+//  * both CTAs' TMA loads complete on the even CTA's full[s] barrier (the
+//    even CTA posts the expected bytes of both); gathered token rows of the
+//    odd CTA are signalled by a relay thread that waits for the local cp.async
+//    arrivals and arrives on the even CTA's full[s];
+//  * tcgen05.commit multicasts the stage release (empty[s]) and the
+//    accumulator-ready signal (tfull) to both CTAs;
+//  * each CTA's epilogue warps release the accumulator on the even CTA's
+//    tempty barrier (the odd CTA's by remote arrive);
+//  * cluster barriers after set-up and before exit keep every barrier and
+//    shared buffer alive while the peer may still touch it.
+// Every mbarrier wait is bounded as in the one-SM kernel.
+#include <algorithm>
+#include <mutex>
+
+#include "grouped_parts.cuh"
+
+namespace moe {
+namespace gg {
+namespace {
+
+constexpr int BM2 = 256;                  // grouped rows per pair tile
+constexpr int kHalfRows = 128;            // rows per CTA
+constexpr int kABytes = kHalfRows * 128;  // one A stage: 128 rows x 128 bytes
+constexpr int kMaxStages = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kTmaWarp = 4;
+constexpr int kMmaWarp = 5;               // MMA issuer in the even CTA, gather relay in the odd one
+constexpr int kGatherWarp0 = 6;
+constexpr int kGatherThreads = 128;
+constexpr int kTmemCols = 512;
+
+// Ring depth for an MMA N of BN (each CTA holds BN / 2 rows of B per stage).
+constexpr int pair_stages(int BN) {
+    const int s = 196608 / (kABytes + BN * 64);
+    return s > kMaxStages ? kMaxStages : s;
+}
+
+struct Ctrl2 {
+    uint64_t full[kMaxStages];    // even CTA: operands of a K block landed (both CTAs)
+    uint64_t empty[kMaxStages];   // both: the MMAs of a K block are done
+    uint64_t gfull[kMaxStages];   // odd CTA: its gathered rows landed (relayed to the even CTA)
+    uint64_t tfull[2];            // both: accumulator ready
+    uint64_t tempty[2];           // even CTA: accumulator released by both epilogues
+    uint64_t done;                // both: all MMAs of the CTA pair completed
+    uint32_t tmem_base;
+    int abort;
+    int n_mtiles;
+    int pad;
+};
+
+template <int MODE, bool GATHER, typename T, int BN>
+__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                             const __grid_constant__ CUtensorMap tmB1, GemmParams p) {
+    constexpr int BK = 128 / (int)sizeof(T);
+    constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
+    constexpr int kStages = pair_stages(BN);
+    constexpr int kBBytes = BN * 64;                 // this CTA's half of a B stage
+    constexpr uint32_t kIdesc = instr_desc<T>(BM2, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + kStages * kABytes;
+    Ctrl2 *ctrl = reinterpret_cast<Ctrl2 *>(sB + kStages * kBBytes);
+    int *tile_start = reinterpret_cast<int *>(ctrl + 1);
+    int *seg_off = tile_start + (p.E + 1);
+    int *seg_end = seg_off + (p.E + 1);
+    volatile int *abort = &ctrl->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool lead = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            // the even CTA's expect_tx arrival (+ its 128 gather threads and the
+            // odd CTA's relay when the rows are gathered)
+            mbar_init(&ctrl->full[s], GATHER ? 1 + kGatherThreads + 1 : 1);
+            mbar_init(&ctrl->empty[s], 1);
+            mbar_init(&ctrl->gfull[s], kGatherThreads);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&ctrl->tfull[a], 1);
+            mbar_init(&ctrl->tempty[a], 2 * kEpiWarps);
+        }
+        mbar_init(&ctrl->done, 1);
+        ctrl->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) tmem_alloc2(&ctrl->tmem_base, kTmemCols);
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tmap(&tmB0);
+        if (MODE == GATEUP) prefetch_tmap(&tmB1);
+        if (!GATHER) prefetch_tmap(&tmA);
+    }
+    pdl_wait();
+    if (warp == kTmaWarp) build_tiles<BM2>(p, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cluster_sync_all();   // both CTAs' barriers exist before any remote arrive
+    pdl_launch_dependents();
+
+    const uint32_t tmem = ctrl->tmem_base;
+    const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
+    const int total = ctrl->n_mtiles * n_tiles;
+    const int nk = (p.K + BK - 1) / BK;
+    const int nE = p.offsets ? p.E : 1;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int row_off = (int)rank * kHalfRows;   // this CTA's rows inside a 256-row tile
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            // this CTA's A rows (when contiguous) and its half of the B columns,
+            // completing on the even CTA's full[s]; the even CTA posts the bytes
+            // of both CTAs
+            constexpr uint32_t kTx = 2u * (uint32_t)(kBBytes + (GATHER ? 0 : kABytes));
+            const uint32_t full_lead = mapa_shared(&ctrl->full[0], 0);   // the even CTA's full[0]
+            const CUtensorMap *mb = (MODE == GATEUP && !lead) ? &tmB1 : &tmB0;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int id = pair; id < total && ok; id += npairs) {
+                const Tile tl = decode(id, n_tiles, tile_start, nE);
+                const int a_row = seg_off[tl.e] + tl.m * BM2 + row_off;
+                // gate/up: the gate rows from CTA 0, the up rows from CTA 1;
+                // down: the first and second half of the BN weight rows
+                const int b_row = tl.e * p.N + tl.n * BN_OUT + (MODE == GATEUP ? 0 : (int)rank * (BN / 2));
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lead) mbar_expect_tx(&ctrl->full[s], kTx);
+                    const uint32_t fb = full_lead + s * (uint32_t)sizeof(uint64_t);
+                    if (!GATHER) tma_load_2d_pair(&tmA, sA + s * kABytes, fb, kb * BK, a_row);
+                    tma_load_2d_pair(mb, sB + s * kBBytes, fb, kb * BK, b_row);
+                }
+            }
+            if (!ok) {
+                // aborting: let this CTA's copies land before it leaves (the last
+                // stages it filled are released by the MMAs or time out)
+                for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j) {
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait(&ctrl->empty[j % kStages], (j / kStages) & 1) &&
+                           globaltimer() - t0 < 100000000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0 && lead) {
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int id = pair; id < total && ok; id += npairs, ++tc) {
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * BN;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    bool got = mbar_try_wait_cluster(&ctrl->full[s], ph);
+                    if (!got) got = wait_bar(&ctrl->full[s], ph, abort, p.err) && mbar_try_wait_cluster(&ctrl->full[s], ph);
+                    if (!got) {
+                        ok = false;
+                        break;
+                    }
+                    if constexpr (GATHER) fence_proxy_async();
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc(sA + s * kABytes);
+                    const uint64_t bd = smem_desc(sB + s * kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma2<T>(d_tmem, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb | kk) != 0);
+                    mma_commit2(&ctrl->empty[s], 0x3);
+                }
+                if (ok) mma_commit2(&ctrl->tfull[acc], 0x3);
+            }
+            mma_commit2(&ctrl->done, 0x3);
+        } else if (lane == 0 && GATHER) {
+            // odd CTA: relay its gathered rows of each K block to the even CTA
+            uint32_t it = 0;
+            bool ok = true;
+            for (int id = pair; id < total && ok; id += npairs) {
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!wait_bar(&ctrl->gfull[s], (it / kStages) & 1, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async();   // cp.async writes before the MMA's async-proxy reads
+                    mbar_arrive_remote(mapa_shared(&ctrl->full[s], 0));   // the even CTA's full[s]
+                }
+            }
+        }
+    } else if (warp < kEpiWarps) {
+        if (MODE == GATEUP && p.zero) {
+            const int64_t n4 = p.zero_floats / 4;
+            const int64_t per = (n4 + gridDim.x - 1) / gridDim.x;
+            const int64_t b = (int64_t)blockIdx.x * per, e = min(n4, b + per);
+            float4 *z = reinterpret_cast<float4 *>(p.zero);
+            for (int64_t i = b + threadIdx.x; i < e; i += kEpiWarps * 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        uint32_t tc = 0;
+        const int row = warp * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t tempty_lead = mapa_shared(&ctrl->tempty[0], 0);
+        for (int id = pair; id < total; id += npairs, ++tc) {
+            const Tile tl = decode(id, n_tiles, tile_start, nE);
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
+            tc_fence_after();
+            const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM2 + row_off + row;
+            epilogue_row<MODE, T, BN>(p, tl.n, r, r < seg_end[tl.e], tmem + acc * BN + lane_base);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (lead) mbar_arrive(&ctrl->tempty[acc]);
+                else mbar_arrive_remote(tempty_lead + acc * (uint32_t)sizeof(uint64_t));
+            }
+        }
+    } else if (GATHER && warp >= kGatherWarp0) {
+        gather_rows<T, kStages, BM2>(p, threadIdx.x - kGatherWarp0 * 32, pair, npairs, total, n_tiles, tile_start,
+                                     seg_off, seg_end, nE, nk, row_off, sA, lead ? ctrl->full : ctrl->gfull,
+                                     ctrl->empty, abort);
+    }
+
+    // every MMA of the pair has completed (its arrivals on this CTA's barriers
+    // included) before the pair meets for the last time and frees TMEM
+    if (threadIdx.x == 0) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&ctrl->done, 0) && globaltimer() - t0 < kWaitLimitNs) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc2(tmem, kTmemCols);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host side
+
+template <int MODE, bool GATHER, typename T, int BN>
+cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
+    const GemmParams &p = L.p;
+    constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
+    constexpr int kStages = pair_stages(BN);
+    const bool f32 = sizeof(T) == 4;
+    CUtensorMap mA, mB0, mB1;
+    const int nE = p.offsets ? p.E : 1;
+    // B boxes hold this CTA's half of the tile's weight rows
+    if (!make_map(&mB0, L.b0, f32, (uint64_t)nE * p.N, p.K, BN / 2)) return cudaErrorInvalidValue;
+    if (MODE == GATEUP) {
+        if (!make_map(&mB1, L.b1, f32, (uint64_t)nE * p.N, p.K, BN / 2)) return cudaErrorInvalidValue;
+    } else {
+        mB1 = mB0;
+    }
+    if (!GATHER) {
+        if (!make_map(&mA, L.a_src, f32, (uint64_t)p.rows, p.K, kHalfRows)) return cudaErrorInvalidValue;
+    } else {
+        mA = mB0;   // unused: gather mode reads x with cp.async
+    }
+    const size_t smem = 1024 + (size_t)kStages * (kABytes + BN * 64) + sizeof(Ctrl2) + 3 * sizeof(int) * (p.E + 1);
+    auto kern = grouped_gemm_pair_kernel<MODE, GATHER, T, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // as many CTA pairs as can be resident at once (one CTA per SM), capped by
+    // the tile count
+    static std::mutex mu;
+    static int max_pairs[8] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 8) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!max_pairs[dev]) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
+            cfg.blockDim = dim3(GATHER ? 320 : 192);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+            if (e != cudaSuccess) return e;
+            max_pairs[dev] = n > 0 ? n : 1;
+        }
+    }
+    const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
+    const int64_t max_tiles = (p.rows / BM2 + nE) * (int64_t)n_tiles;
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs[dev], max_tiles));
+    return launch_kernel_pair(kern, 2 * pairs, GATHER ? 320 : 192, smem, s, mA, mB0, mB1, p);
+}
+
+template <int MODE, bool GATHER, typename T>
+cudaError_t launch_pair_bn(const GemmLaunch &L, cudaStream_t s) {
+    return L.narrow ? launch_pair_t<MODE, GATHER, T, 128>(L, s) : launch_pair_t<MODE, GATHER, T, 256>(L, s);
+}
+
+}  // namespace gg
+
+cudaError_t launch_grouped_gemm_pair(const GemmLaunch &L, cudaStream_t s) {
+    const GemmParams &p = L.p;
+    if (p.rows <= 0) return cudaSuccess;
+    const bool f32 = L.dtype == MOE_F32;
+    if (L.mode == gg::GATEUP) {
+        if (L.gather)
+            return f32 ? gg::launch_pair_bn<gg::GATEUP, true, float>(L, s)
+                       : gg::launch_pair_bn<gg::GATEUP, true, __nv_bfloat16>(L, s);
+        return f32 ? gg::launch_pair_bn<gg::GATEUP, false, float>(L, s)
+                   : gg::launch_pair_bn<gg::GATEUP, false, __nv_bfloat16>(L, s);
+    }
+    return f32 ? gg::launch_pair_bn<gg::DOWN, false, float>(L, s)
+               : gg::launch_pair_bn<gg::DOWN, false, __nv_bfloat16>(L, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,192 @@
+// Pieces shared by the one-SM and the two-SM grouped GEMM kernels: the
+// epilogue of one accumulator row and the token-row gather producer.
+//
+//   GATEUP: act[i, n] = silu(W_gate[e, n] . a_i) * (W_up[e, n] . a_i)
+//   DOWN  : y_acc[t_i, n] += g_i * (W_down[e, n] . a_i)
+//
+// "Tutorial 11: Mixture of Experts (MoE)", section 3 "Expert Computation"
+// (silu(gate) * up; the weighted sum back in token order).
+#pragma once
+
+#include "grouped_tiles.cuh"
+#include "moe_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace gg {
+
+using namespace tc;
+
+enum { GATEUP = 0, DOWN = 1 };
+
+// Epilogue of one grouped row r (valid: r lies inside its expert's segment)
+// of a tile in column tile n, whose fp32 accumulator row starts at TMEM
+// address tbase (this thread's lane).  GATEUP holds BN/2 gate columns then
+// BN/2 up columns and stores silu(g) * u into act; DOWN scales the BN
+// columns by the row's gate and adds them into y_acc with 16-byte reductions.
+// Several TMEM loads are in flight per wait.
+template <int MODE, typename T, int BN>
+__device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t r, bool valid, uint32_t tbase) {
+    constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
+    if constexpr (MODE == GATEUP) {
+        T *act = static_cast<T *>(p.act);
+        // silu(g) * u for 16 output columns from column c of the tile
+        auto store16 = [&](int c, const float(&g)[16], const float(&u)[16]) {
+            const int col = n * BN_OUT + c;
+            if (!valid || col >= p.N) return;
+            T *dst = act + r * p.N + col;
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                if (col + 8 * h8 >= p.N) continue;
+                if constexpr (sizeof(T) == 2) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int i0 = 8 * h8 + 2 * q;
+                        __nv_bfloat162 b2 =
+                            __floats2bfloat162_rn(silu_f(g[i0]) * u[i0], silu_f(g[i0 + 1]) * u[i0 + 1]);
+                        w[q] = *reinterpret_cast<uint32_t *>(&b2);
+                    }
+                    *reinterpret_cast<uint4 *>(dst + 8 * h8) = make_uint4(w[0], w[1], w[2], w[3]);
+                } else {
+                    float o[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) o[q] = silu_f(g[8 * h8 + q]) * u[8 * h8 + q];
+                    float *fd = reinterpret_cast<float *>(dst + 8 * h8);
+                    *reinterpret_cast<float4 *>(fd) = make_float4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<float4 *>(fd + 4) = make_float4(o[4], o[5], o[6], o[7]);
+                }
+            }
+        };
+        // 32 output columns per TMEM wait: four loads in flight at a time
+#pragma unroll 1
+        for (int c = 0; c < BN_OUT; c += 32) {
+            float g[2][16], u[2][16];
+            tmem_ld16(tbase + c, g[0]);
+            tmem_ld16(tbase + c + 16, g[1]);
+            tmem_ld16(tbase + BN_OUT + c, u[0]);
+            tmem_ld16(tbase + BN_OUT + c + 16, u[1]);
+            tmem_wait_ld();
+            store16(c, g[0], u[0]);
+            store16(c + 16, g[1], u[1]);
+        }
+    } else {
+        int64_t t = -1;
+        float gate = 0.f;
+        if (valid) {
+            if (p.sorted_rows) {
+                const int v = p.sorted_rows[r];
+                t = v / p.k;
+                gate = (v >= 0 && v < p.rows) ? p.gates[v] : 0.f;
+            } else {
+                t = r;
+                gate = p.gates[r];
+            }
+            if (t < 0 || t >= p.T) {
+                atomicOr(p.err, kErrInput);
+                t = -1;
+            }
+        }
+        // 32 columns per TMEM wait: two loads in flight at a time
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            float v[2][16];
+            tmem_ld16(tbase + c, v[0]);
+            tmem_ld16(tbase + c + 16, v[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int hh = 0; hh < 2 && t >= 0; ++hh) {
+                const int col = n * BN + c + 16 * hh;
+                float *dst = p.y_acc + t * p.N + col;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (col + 4 * q < p.N)
+                        atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
+                                  make_float4(gate * v[hh][4 * q], gate * v[hh][4 * q + 1], gate * v[hh][4 * q + 2],
+                                              gate * v[hh][4 * q + 3]));
+            }
+        }
+    }
+}
+
+// Gather producer (128 threads, g = 0..127): the token rows x[t] of the routed
+// gate/up GEMM, read in place by index with 16-byte cp.async into the
+// 128-byte-swizzled K-major layout the MMA descriptor reads (8 threads per
+// row, 16 rows per pass).  Tile id runs from `first` in steps of `stride`;
+// the rows of a tile start `row_off` rows into its RB-row block.  Stage s of
+// the S-deep ring is written once empty[s] shows the previous use consumed,
+// and its arrival lands on full[s] when the thread's copies have (non-blocking
+// cp.async.mbarrier.arrive.noinc).  The assignment ids are loaded one tile
+// ahead so their loads overlap the copies.  Returns false on abort.
+template <typename T, int S, int RB>
+__device__ bool gather_rows(const GemmParams &p, int g, int first, int stride, int total, int n_tiles,
+                            const int *tile_start, const int *seg_off, const int *seg_end, int nE, int nk,
+                            int row_off, uint8_t *sA, uint64_t *full, uint64_t *empty, volatile int *abort) {
+    constexpr int BK = 128 / (int)sizeof(T);
+    constexpr int V = 16 / (int)sizeof(T);
+    constexpr int kABytes = 128 * 128;
+    const int c = g & 7;                             // 16-byte chunk of the 128-byte row
+    const int rg = g >> 3;                           // rows rg, rg + 16, ..., rg + 112
+    const int swz = (c ^ (rg & 7)) << 4;             // 128-byte swizzle: chunk ^ (row mod 8)
+    const T *x = static_cast<const T *>(p.x);
+    auto load_ids = [&](int id, int (&v)[8]) {
+        if (id >= total) return;
+        const Tile tl = decode(id, n_tiles, tile_start, nE);
+        const int64_t row0 = (int64_t)seg_off[tl.e] + (int64_t)tl.m * RB + row_off;
+        const int64_t rend = seg_end[tl.e];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int64_t r = row0 + rg + 16 * q;
+            v[q] = r < rend ? p.sorted_rows[r] : -1;
+        }
+    };
+    int vnext[8];
+    load_ids(first, vnext);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int id = first; id < total && ok; id += stride) {
+        int vcur[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) vcur[q] = vnext[q];
+        load_ids(id + stride, vnext);
+        const T *src[8];
+        uint32_t okmask = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            src[q] = x;
+            const int v = vcur[q];
+            if (v != -1) {
+                const int64_t t = v / p.k;
+                if (v >= 0 && t < p.T) {
+                    src[q] = x + t * p.K + c * V;
+                    okmask |= 1u << q;
+                } else {
+                    atomicOr(p.err, kErrInput);
+                }
+            }
+        }
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % S;
+            const uint32_t ph = (it / S) & 1;
+            if (!wait_bar(&empty[s], ph ^ 1, abort, p.err)) {
+                ok = false;
+                break;
+            }
+            uint8_t *dst = sA + s * kABytes + rg * 128 + swz;
+            const bool colok = kb * BK + c * V < p.K;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (okmask & (1u << q))
+                    cp_async16(dst + q * 16 * 128, colok ? (const void *)(src[q] + kb * BK) : (const void *)x,
+                               colok ? 16 : 0);
+            cp_async_commit();
+            // the barrier receives this thread's arrival once its copies have landed
+            cp_async_arrive_noinc(&full[s]);
+        }
+    }
+    cp_async_wait<0>();
+    return ok;
+}
+
+}  // namespace gg
+}  // namespace moe

@@ -106,6 +106,22 @@ bool narrow_down(const moe_config &c) { return c.d % 256 != 0; }
 // Experts average at most one 128-row tile: every weight tile is read once.
 bool one_tile_per_expert(const moe_config &c) { return (int64_t)c.T * c.k <= 128LL * c.E; }
 
+// Two SMs per tile (M = 256 across a CTA pair) for GEMMs whose A operand comes
+// by TMA and whose groups average at least 512 rows: the layer is tensor-bound
+// and the operand traffic per SM drops by a third (measured: mixtral_prefill
+// down 874 -> 732 us, the shared expert's gate/up and down of qwen_shared -17%).
+// With gathered token rows the pair is slower (the odd CTA's rows reach the
+// MMA through a relay) and with fewer rows the 256-row tiles waste work, so
+// those keep one SM per tile.  MOE_GG_PAIR=1 / 0 forces it on / off.
+bool pair_tiles(int64_t rows, int groups, bool gather) {
+    static const int force = [] {
+        const char *v = std::getenv("MOE_GG_PAIR");
+        return v ? (v[0] == '1' ? 1 : 0) : -1;
+    }();
+    if (force >= 0) return force == 1;
+    return !gather && rows >= 512LL * groups;
+}
+
 GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const void *wu, const int32_t *offsets,
                        const int32_t *srt, void *act, uint32_t *err) {
     GemmLaunch L{};
@@ -115,6 +131,7 @@ GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.d, c.h, x, act, nullptr, nullptr, err};
     L.narrow = narrow_gateup(c);
     L.p.stream_weights = one_tile_per_expert(c);
+    L.pair = pair_tiles(c.T * c.k, c.E, true);
     L.b0 = wg;
     L.b1 = wu;
     return L;
@@ -126,6 +143,7 @@ GemmLaunch gemm_gateup_dense(const moe_config &c, const void *x, const void *wg,
     L.gather = false;
     L.dtype = c.dtype;
     L.p = GemmParams{nullptr, nullptr, 1, 1, c.T, c.T, c.d, c.h_shared, x, act, nullptr, nullptr, err};
+    L.pair = pair_tiles(c.T, 1, false);
     L.a_src = x;
     L.b0 = wg;
     L.b1 = wu;
@@ -140,6 +158,7 @@ GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.h, c.d, nullptr, nullptr, acc, gates, err};
     L.narrow = narrow_down(c);
     L.p.stream_weights = one_tile_per_expert(c);
+    L.pair = pair_tiles(c.T * c.k, c.E, false);
     L.a_src = act;
     L.b0 = wd;
     return L;
@@ -151,6 +170,7 @@ GemmLaunch gemm_down_dense(const moe_config &c, const void *act, const void *wd,
     L.gather = false;
     L.dtype = c.dtype;
     L.p = GemmParams{nullptr, nullptr, 1, 1, c.T, c.T, c.h_shared, c.d, nullptr, nullptr, acc, sg, err};
+    L.pair = pair_tiles(c.T, 1, false);
     L.a_src = act;
     L.b0 = wd;
     return L;

@@ -175,11 +175,13 @@ struct GemmLaunch {
     bool gather;          // A rows gathered from x by index (routed gate/up); else TMA from a_src
     int dtype;            // MOE_BF16 or MOE_F32 (tf32 MMA)
     bool narrow;          // MMA N = 128 (6-stage ring) instead of N = 256 (4 stages)
+    bool pair;            // two SMs per tile (clusters of two CTAs, M = 256 MMAs)
     GemmParams p;
     const void *a_src;    // contiguous A operand [rows, K] when !gather
     const void *b0, *b1;  // weights [E*N, K] (b1: up projection for gate/up)
 };
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s);
+cudaError_t launch_grouped_gemm_pair(const GemmLaunch &L, cudaStream_t s);
 
 // Launch planning shared by the entry points (defined in moe_api.cu).
 uint32_t *device_error_word();   // the library's device error word on the current device
@@ -227,6 +229,29 @@ cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size_t smem
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<A &&>(args)...);
+    note_launch();
+    return e;
+}
+
+// The same for a kernel launched in clusters of two CTAs along x.
+template <typename... P, typename... A>
+cudaError_t launch_kernel_pair(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                               A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<A &&>(args)...);
     note_launch();
     return e;
