@@ -204,8 +204,13 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                         ok = false;
                         break;
                     }
-                    fence_proxy_async();   // cp.async writes before the MMA's async-proxy reads
-                    mbar_arrive_remote(mapa_shared(&ctrl->full[s], 0));   // the even CTA's full[s]
+                    // the rows sit in this CTA's shared memory: the fence makes the
+                    // cp.async writes visible to the async proxy that the MMAs read
+                    // them through, and the MMAs are issued only after this arrival.
+                    // (A release arrive stalls the relay ~1 us per K block, which
+                    // measured 1.6x slower on the whole kernel.)
+                    fence_proxy_async();
+                    mbar_arrive_remote_relaxed(mapa_shared(&ctrl->full[s], 0));   // the even CTA's full[s]
                 }
             }
         }
