@@ -246,6 +246,17 @@ int64_t moe_launch_count(void);
  * reports an error.  Blocking; meant for tests and debugging. */
 moe_status moe_device_status(void *stream);
 
+/* Self-test of the device failure path (the pages have no counterpart; it
+ * exists so the timeout path can be exercised without faulting a GPU).
+ * Enqueues on `stream` one kernel whose mbarrier wait can never complete,
+ * through the same bounded wait the tensor-core kernels use, with a limit of
+ * limit_ms milliseconds (1..10000).  When it runs out the kernel raises the
+ * device flag and returns: the next moe_device_status() reports
+ * MOE_ERR_DEVICE_TIMEOUT, and the context and stream stay usable.
+ * Returns MOE_ERR_INVALID_ARG for a limit outside the range, MOE_ERR_CUDA if
+ * the launch failed, MOE_OK otherwise. */
+moe_status moe_selftest_wait_timeout(uint32_t limit_ms, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

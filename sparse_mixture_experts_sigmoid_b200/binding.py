@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTED = ["moe_status_string", "moe_validate", "moe_workspace_size", "moe_workspace_layout", "moe_route",
             "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_decode_max_rows",
             "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size",
+            "moe_selftest_wait_timeout",
             "moe_route_workspace_size"]
 STAGES = ["route", "permute", "gate_up", "shared_gate_up", "down", "shared_down", "finalize"]
 
@@ -71,6 +72,7 @@ def lib() -> ctypes.CDLL:
             "moe_forward": ([C, P, P, P, P, P, P, P, P, P, P, P, S, P], ctypes.c_int),
             "moe_decode_max_rows": ([], ctypes.c_int32),
             "moe_device_status": ([P], ctypes.c_int),
+            "moe_selftest_wait_timeout": ([ctypes.c_uint32, P], ctypes.c_int),
             "moe_profile_events": ([ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32], ctypes.c_int),
             "moe_launch_count": ([], ctypes.c_int64),
             "moe_combine_noalloc": ([C, P, P, P, P, P, P, P], ctypes.c_int),
@@ -292,6 +294,12 @@ def device_status(stream=None) -> int:
 
 def decode_max_rows() -> int:
     return lib().moe_decode_max_rows()
+
+
+def selftest_wait_timeout(limit_ms: int, stream=None) -> int:
+    """Enqueues the bounded-wait self-test kernel (see moe_selftest_wait_timeout);
+    returns the launch status (the timeout itself shows in device_status())."""
+    return lib().moe_selftest_wait_timeout(int(limit_ms), _stream(stream))
 
 
 def launch_count() -> int:

@@ -65,7 +65,10 @@ constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kGatherWarp0 = 6;
-constexpr int kGatherThreads = 128;
+#ifndef MOE_GATHER_THREADS
+#define MOE_GATHER_THREADS 256
+#endif
+constexpr int kGatherThreads = MOE_GATHER_THREADS;   // 128 or 256
 constexpr int kTmemCols = 512;
 
 using Params = GemmParams;
@@ -84,7 +87,7 @@ struct Ctrl {
 // ------------------------------------------------------------------ kernel
 
 template <int MODE, bool GATHER, typename T, int BN>
-__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+__global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, Params p) {
     constexpr int BK = 128 / (int)sizeof(T);   // elements per 128-byte K block
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             mbar_arrive(&ctrl->tempty[acc]);
         }
     } else if (GATHER && warp >= kGatherWarp0) {
-        gather_rows<T, kStages, BM>(p, threadIdx.x - kGatherWarp0 * 32, blockIdx.x, gridDim.x, total, n_tiles,
+        gather_rows<T, kStages, BM, kGatherThreads>(p, threadIdx.x - kGatherWarp0 * 32, blockIdx.x, gridDim.x, total, n_tiles,
                                     tile_start, seg_off, seg_end, nE, nk, 0, sA, ctrl->full, ctrl->empty, abort);
     }
 
@@ -312,7 +315,7 @@ cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
     auto kern = grouped_gemm_kernel<MODE, GATHER, T, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(kern, grid, GATHER ? 320 : 192, smem, s, mA, mB0, mB1, p);
+    return launch_kernel(kern, grid, GATHER ? 192 + kGatherThreads : 192, smem, s, mA, mB0, mB1, p);
 }
 
 template <int MODE, bool GATHER, typename T>

@@ -109,50 +109,52 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
     }
 }
 
-// Gather producer (128 threads, g = 0..127): the token rows x[t] of the routed
+// Gather producer (NG threads, g = 0..NG-1): the token rows x[t] of the routed
 // gate/up GEMM, read in place by index with 16-byte cp.async into the
 // 128-byte-swizzled K-major layout the MMA descriptor reads (8 threads per
-// row, 16 rows per pass).  Tile id runs from `first` in steps of `stride`;
+// row, NG / 8 rows per pass).  Tile id runs from `first` in steps of `stride`;
 // the rows of a tile start `row_off` rows into its RB-row block.  Stage s of
 // the S-deep ring is written once empty[s] shows the previous use consumed,
 // and its arrival lands on full[s] when the thread's copies have (non-blocking
 // cp.async.mbarrier.arrive.noinc).  The assignment ids are loaded one tile
 // ahead so their loads overlap the copies.  Returns false on abort.
-template <typename T, int S, int RB>
+template <typename T, int S, int RB, int NG = 128>
 __device__ bool gather_rows(const GemmParams &p, int g, int first, int stride, int total, int n_tiles,
                             const int *tile_start, const int *seg_off, const int *seg_end, int nE, int nk,
                             int row_off, uint8_t *sA, uint64_t *full, uint64_t *empty, volatile int *abort) {
     constexpr int BK = 128 / (int)sizeof(T);
     constexpr int V = 16 / (int)sizeof(T);
     constexpr int kABytes = 128 * 128;
+    constexpr int RG = NG / 8;                       // rows per pass (a multiple of 8)
+    constexpr int RPT = 128 / RG;                    // rows per thread
     const int c = g & 7;                             // 16-byte chunk of the 128-byte row
-    const int rg = g >> 3;                           // rows rg, rg + 16, ..., rg + 112
+    const int rg = g >> 3;                           // rows rg, rg + RG, ..., of the 128
     const int swz = (c ^ (rg & 7)) << 4;             // 128-byte swizzle: chunk ^ (row mod 8)
     const T *x = static_cast<const T *>(p.x);
-    auto load_ids = [&](int id, int (&v)[8]) {
+    auto load_ids = [&](int id, int (&v)[RPT]) {
         if (id >= total) return;
         const Tile tl = decode(id, n_tiles, tile_start, nE);
         const int64_t row0 = (int64_t)seg_off[tl.e] + (int64_t)tl.m * RB + row_off;
         const int64_t rend = seg_end[tl.e];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int64_t r = row0 + rg + 16 * q;
+        for (int q = 0; q < RPT; ++q) {
+            const int64_t r = row0 + rg + RG * q;
             v[q] = r < rend ? p.sorted_rows[r] : -1;
         }
     };
-    int vnext[8];
+    int vnext[RPT];
     load_ids(first, vnext);
     uint32_t it = 0;
     bool ok = true;
     for (int id = first; id < total && ok; id += stride) {
-        int vcur[8];
+        int vcur[RPT];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) vcur[q] = vnext[q];
+        for (int q = 0; q < RPT; ++q) vcur[q] = vnext[q];
         load_ids(id + stride, vnext);
-        const T *src[8];
+        const T *src[RPT];
         uint32_t okmask = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < RPT; ++q) {
             src[q] = x;
             const int v = vcur[q];
             if (v != -1) {
@@ -175,9 +177,9 @@ __device__ bool gather_rows(const GemmParams &p, int g, int first, int stride, i
             uint8_t *dst = sA + s * kABytes + rg * 128 + swz;
             const bool colok = kb * BK + c * V < p.K;
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
+            for (int q = 0; q < RPT; ++q)
                 if (okmask & (1u << q))
-                    cp_async16(dst + q * 16 * 128, colok ? (const void *)(src[q] + kb * BK) : (const void *)x,
+                    cp_async16(dst + q * RG * 128, colok ? (const void *)(src[q] + kb * BK) : (const void *)x,
                                colok ? 16 : 0);
             cp_async_commit();
             // the barrier receives this thread's arrival once its copies have landed

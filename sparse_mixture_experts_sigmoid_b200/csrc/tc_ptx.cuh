@@ -45,14 +45,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
 }
 // Bounded wait for the phase of parity `parity` to complete.  Returns false if
 // the CTA is aborting or the limit ran out (which raises the device flag).
-static __device__ __noinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int *abort, uint32_t *err) {
+static __device__ __noinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int *abort, uint32_t *err,
+                                             uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(b, parity)) return true;
         if ((i & 63) == 0) {
             if (*abort) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort = 1;
                 atomicOr(err, kErrTimeout);
                 return false;
