@@ -34,11 +34,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
 L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
 # stage -> (kernel name in the ncu launch list, source file whose hash keys the traffic figure)
+GG_SRC = "grouped_gemm.cu+grouped_gemm2.cu"   # one-SM and two-SM grouped GEMM kernels
 STAGE_KERNEL = {"route": ("router_logits_kernel", "router_tc.cu"), "permute": ("scatter_kernel", "permute.cu"),
-                "gate_up": ("grouped_gemm_kernel", "grouped_gemm.cu"),
-                "shared_gate_up": ("grouped_gemm_kernel", "grouped_gemm.cu"),
-                "down": ("grouped_gemm_kernel", "grouped_gemm.cu"),
-                "shared_down": ("grouped_gemm_kernel", "grouped_gemm.cu"),
+                "gate_up": ("grouped_gemm_kernel", GG_SRC),
+                "shared_gate_up": ("grouped_gemm_kernel", GG_SRC),
+                "down": ("grouped_gemm_kernel", GG_SRC),
+                "shared_down": ("grouped_gemm_kernel", GG_SRC),
                 "finalize": ("finalize_kernel", "segment.cu")}
 # kernels of the small-batch path (at most 64 assignments)
 STAGE_KERNEL_SMALL = {"route": ("router_kernel", "router.cu"), "gate_up": ("seg_gateup_kernel", "segment.cu"),
@@ -145,10 +146,11 @@ def barrier(ws: int):
 
 
 def source_hash(src: str) -> str:
-    """Hash of a kernel's translation unit plus the shared device headers."""
+    """Hash of a kernel's translation units ('+'-separated) plus the shared
+    device headers."""
     d = os.path.join(ROOT, "sparse_mixture_experts_sigmoid_b200", "csrc")
     h = hashlib.sha256()
-    for f in [src] + sorted(x for x in os.listdir(d) if x.endswith(".cuh")):
+    for f in src.split("+") + sorted(x for x in os.listdir(d) if x.endswith(".cuh")):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
