@@ -53,9 +53,10 @@ using namespace tc;
 constexpr int BM = 128;
 constexpr int kABytes = BM * 128;     // one A stage: 128 rows x 128 bytes
 constexpr int kMaxStages = 8;
-// Shared-memory ring depth for an MMA N of BN: as many stages as fit in 192 KB.
-constexpr int stages_for(int BN) {
-    const int s = 196608 / (kABytes + BN * 128);
+// Shared-memory ring depth for an MMA N of BN and A stages of a_bytes: as many
+// stages as fit in 192 KB.
+constexpr int stages_for(int BN, int a_bytes = kABytes) {
+    const int s = 196608 / (a_bytes + BN * 128);
     return s > kMaxStages ? kMaxStages : s;
 }
 #ifndef MOE_GG_L2_PROMOTION
@@ -86,20 +87,31 @@ struct Ctrl {
 
 // ------------------------------------------------------------------ kernel
 
-template <int MODE, bool GATHER, typename T, int BN>
+// HALF (contiguous A only): 64-row tiles whose A stage holds 64 rows, for
+// experts of at most 64 rows, where the weights stream from HBM and the rows
+// of a 128-row A stage would mostly sit empty.  The MMA still has M = 128: its
+// rows 64-127 read the next 8 KB of shared memory (the following stage, or a
+// pad after the last one) and land in TMEM lanes no epilogue thread reads.
+// The smaller stages fit 8 in the ring instead of 6, a third more weight bytes
+// in flight per SM.
+template <int MODE, bool GATHER, typename T, int BN, bool HALF>
 __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, Params p) {
     constexpr int BK = 128 / (int)sizeof(T);   // elements per 128-byte K block
     constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;   // output columns per tile
-    constexpr int kStages = stages_for(BN);
+    static_assert(!(HALF && GATHER), "half-height A tiles are loaded by TMA");
+    constexpr int RB = HALF ? BM / 2 : BM;                 // grouped rows per tile
+    constexpr int kAStage = RB * 128;                      // one A stage: RB rows x 128 bytes
+    constexpr int kAPad = kABytes - kAStage;               // room for the MMA's reads past the last stage
+    constexpr int kStages = stages_for(BN, kAStage);
     constexpr int kBBytes = BN * 128;                      // one B stage: BN rows x 128 bytes
     constexpr uint32_t kIdesc = instr_desc<T>(BM, BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
-    uint8_t *sB = smem + kStages * kABytes;
+    uint8_t *sB = smem + kStages * kAStage + kAPad;
     Ctrl *ctrl = reinterpret_cast<Ctrl *>(sB + kStages * kBBytes);
     int *tile_start = reinterpret_cast<int *>(ctrl + 1);
     int *seg_off = tile_start + (p.E + 1);
@@ -133,7 +145,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     // is read before it, so the first weight tiles are in flight early.
     const bool early_tiles = (p.early & kEarlyTiles) != 0;
     if (!early_tiles) pdl_wait();
-    if (warp == kTmaWarp) build_tiles<BM>(p, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
+    if (warp == kTmaWarp) build_tiles<RB>(p, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -177,11 +189,11 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             if (early_tiles) {
                 for (int id = blockIdx.x; id < total && pre < (uint32_t)kStages; id += gridDim.x) {
                     const Tile tl = decode(id, n_tiles, tile_start, nE);
-                    const int a_row = seg_off[tl.e] + tl.m * BM;
+                    const int a_row = seg_off[tl.e] + tl.m * RB;
                     const int b_row = tl.e * p.N + tl.n * BN_OUT;
                     for (int kb = 0; kb < nk && pre < (uint32_t)kStages; ++kb, ++pre) {
-                        mbar_expect_tx(&ctrl->full[pre], kBBytes + (GATHER ? 0 : kABytes));
-                        if (early_a) tma_load_2d(&tmA, sA + pre * kABytes, &ctrl->full[pre], kb * BK, a_row);
+                        mbar_expect_tx(&ctrl->full[pre], kBBytes + (GATHER ? 0 : kAStage));
+                        if (early_a) tma_load_2d(&tmA, sA + pre * kAStage, &ctrl->full[pre], kb * BK, a_row);
                         load_b((int)pre, kb, b_row);
                     }
                 }
@@ -192,22 +204,22 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
                 const Tile tl = decode(id, n_tiles, tile_start, nE);
-                const int a_row = seg_off[tl.e] + tl.m * BM;
+                const int a_row = seg_off[tl.e] + tl.m * RB;
                 const int b_row = tl.e * p.N + tl.n * BN_OUT;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     if (it < pre) {
                         // issued above; only the A tile may still be missing
-                        if (!GATHER && !early_a) tma_load_2d(&tmA, sA + s * kABytes, &ctrl->full[s], kb * BK, a_row);
+                        if (!GATHER && !early_a) tma_load_2d(&tmA, sA + s * kAStage, &ctrl->full[s], kb * BK, a_row);
                         continue;
                     }
                     if (!wait_bar(&ctrl->empty[s], ph ^ 1, abort, p.err)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&ctrl->full[s], kBBytes + (GATHER ? 0 : kABytes));
-                    if (!GATHER) tma_load_2d(&tmA, sA + s * kABytes, &ctrl->full[s], kb * BK, a_row);
+                    mbar_expect_tx(&ctrl->full[s], kBBytes + (GATHER ? 0 : kAStage));
+                    if (!GATHER) tma_load_2d(&tmA, sA + s * kAStage, &ctrl->full[s], kb * BK, a_row);
                     load_b(s, kb, b_row);
                 }
             }
@@ -241,7 +253,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                     // MMA reads them through the async proxy
                     if constexpr (GATHER) fence_proxy_async();
                     tc_fence_after();
-                    const uint64_t ad = smem_desc(sA + s * kABytes);
+                    const uint64_t ad = smem_desc(sA + s * kAStage);
                     const uint64_t bd = smem_desc(sB + s * kBBytes);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)   // four 32-byte K slices per 128-byte block
@@ -269,13 +281,13 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
-            const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM + row;
-            epilogue_row<MODE, T, BN>(p, tl.n, r, r < seg_end[tl.e], tmem + acc * BN + lane_base);
+            const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * RB + row;
+            epilogue_row<MODE, T, BN>(p, tl.n, r, row < RB && r < seg_end[tl.e], tmem + acc * BN + lane_base);
             tc_fence_before();
             mbar_arrive(&ctrl->tempty[acc]);
         }
     } else if (GATHER && warp >= kGatherWarp0) {
-        gather_rows<T, kStages, BM, kGatherThreads>(p, threadIdx.x - kGatherWarp0 * 32, blockIdx.x, gridDim.x, total, n_tiles,
+        gather_rows<T, kStages, RB, kGatherThreads>(p, threadIdx.x - kGatherWarp0 * 32, blockIdx.x, gridDim.x, total, n_tiles,
                                     tile_start, seg_off, seg_end, nE, nk, 0, sA, ctrl->full, ctrl->empty, abort);
     }
 
@@ -287,11 +299,12 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
 
 // ------------------------------------------------------------------ host side
 
-template <int MODE, bool GATHER, typename T, int BN>
+template <int MODE, bool GATHER, typename T, int BN, bool HALF>
 cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
     const Params &p = L.p;
     constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
-    constexpr int kStages = stages_for(BN);
+    constexpr int RB = HALF ? BM / 2 : BM;
+    constexpr int kStages = stages_for(BN, RB * 128);
     const bool f32 = sizeof(T) == 4;
     CUtensorMap mA, mB0, mB1;
     const int nE = p.offsets ? p.E : 1;
@@ -303,16 +316,17 @@ cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
         mB1 = mB0;
     }
     if (!GATHER) {
-        if (!make_map(&mA, L.a_src, f32, (uint64_t)p.rows, p.K, 128)) return cudaErrorInvalidValue;
+        if (!make_map(&mA, L.a_src, f32, (uint64_t)p.rows, p.K, RB)) return cudaErrorInvalidValue;
     } else {
         mA = mB0;   // unused: gather mode reads x with cp.async
     }
     const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
-    const int64_t max_m = p.rows / BM + nE;
+    const int64_t max_m = p.rows / RB + nE;
     const int64_t max_tiles = max_m * n_tiles;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
-    const size_t smem = 1024 + (size_t)kStages * (kABytes + BN * 128) + sizeof(Ctrl) + 3 * sizeof(int) * (p.E + 1);
-    auto kern = grouped_gemm_kernel<MODE, GATHER, T, BN>;
+    const size_t smem = 1024 + (size_t)kStages * (RB * 128 + BN * 128) + (kABytes - RB * 128) + sizeof(Ctrl) +
+                        3 * sizeof(int) * (p.E + 1);
+    auto kern = grouped_gemm_kernel<MODE, GATHER, T, BN, HALF>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_kernel(kern, grid, GATHER ? 192 + kGatherThreads : 192, smem, s, mA, mB0, mB1, p);
@@ -320,7 +334,11 @@ cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
 
 template <int MODE, bool GATHER, typename T>
 cudaError_t launch_bn(const GemmLaunch &L, cudaStream_t s) {
-    return L.narrow ? launch_t<MODE, GATHER, T, 128>(L, s) : launch_t<MODE, GATHER, T, 256>(L, s);
+    if constexpr (!GATHER) {
+        if (L.half)
+            return L.narrow ? launch_t<MODE, GATHER, T, 128, true>(L, s) : launch_t<MODE, GATHER, T, 256, true>(L, s);
+    }
+    return L.narrow ? launch_t<MODE, GATHER, T, 128, false>(L, s) : launch_t<MODE, GATHER, T, 256, false>(L, s);
 }
 
 }  // namespace gg

@@ -122,6 +122,18 @@ bool pair_tiles(int64_t rows, int groups, bool gather) {
     return !gather && rows >= 512LL * groups;
 }
 
+// 64-row tiles for a contiguous A when the groups average at most 64 rows
+// (the weights stream from HBM; see grouped_gemm.cu).  MOE_GG_HALF=1 / 0
+// forces it on / off.
+bool half_tiles(int64_t rows, int groups) {
+    static const int force = [] {
+        const char *v = std::getenv("MOE_GG_HALF");
+        return v ? (v[0] == '1' ? 1 : 0) : -1;
+    }();
+    if (force >= 0) return force == 1;
+    return rows <= 64LL * groups;
+}
+
 GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const void *wu, const int32_t *offsets,
                        const int32_t *srt, void *act, uint32_t *err) {
     GemmLaunch L{};
@@ -159,6 +171,7 @@ GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const
     L.narrow = narrow_down(c);
     L.p.stream_weights = one_tile_per_expert(c);
     L.pair = pair_tiles(c.T * c.k, c.E, false);
+    L.half = !L.pair && half_tiles(c.T * c.k, c.E);
     L.a_src = act;
     L.b0 = wd;
     return L;

@@ -176,6 +176,7 @@ struct GemmLaunch {
     int dtype;            // MOE_BF16 or MOE_F32 (tf32 MMA)
     bool narrow;          // MMA N = 128 (6-stage ring) instead of N = 256 (4 stages)
     bool pair;            // two SMs per tile (clusters of two CTAs, M = 256 MMAs)
+    bool half;            // contiguous A only: 64-row tiles with 64-row A stages (few rows per group)
     GemmParams p;
     const void *a_src;    // contiguous A operand [rows, K] when !gather
     const void *b0, *b1;  // weights [E*N, K] (b1: up projection for gate/up)
