@@ -11,33 +11,41 @@
 // everything" (read each token's expert weights in place, no gathered weight
 // copies, no padding of groups to a common length).
 //
-// Design (sm_100a):
+// Design (sm_100a), one SM per tile (grouped_gemm2.cu holds the two-SM form):
 //  * Persistent CTAs, one per SM, walk a tile list derived on the device from
-//    the expert offsets: tiles are 128 grouped rows x (128 gate + 128 up
-//    columns) for GATEUP, 128 x 256 for DOWN; expert-major, and inside an
-//    expert the row tiles vary fastest so CTAs running at the same time share
-//    one weight tile through L2.  Partial row tiles at a segment's end are
-//    computed and masked, never padded in memory.
+//    the expert offsets: tiles are 128 grouped rows (64 with HALF) x (128 gate
+//    + 128 up columns) for GATEUP, x 256 (or 128 when the output width is not
+//    a multiple of 256) for DOWN; expert-major, and inside an expert the row
+//    tiles vary fastest so CTAs running at the same time share one weight
+//    tile through L2.  Partial row tiles at a segment's end are computed and
+//    masked, never padded in memory.
 //  * Warp roles: warps 0-3 epilogue (TMEM lane quarters 0-3), warp 4 TMA
-//    producer, warp 5 TMEM allocator + single-thread MMA issuer.
+//    producer, warp 5 TMEM allocator + single-thread MMA issuer, warps 6-13
+//    token-row gather (routed gate/up).
 //  * Weights (and contiguous A operands) arrive by TMA 2D tiles, 128-byte
-//    swizzle, no multicast.  Token rows x[t] of the routed gate/up GEMM are
-//    read in place by index: warps 6-9 issue 16-byte cp.async copies straight
-//    into the 128-byte-swizzled K-major layout the MMA descriptor reads, and
-//    signal each stage with a non-blocking cp.async.mbarrier.arrive.noinc (the
-//    arrival lands when the thread's copies have), so the gather runs as far
-//    ahead as the ring allows; no copy of x is ever made.  (TMA tile::gather4
-//    was measured 2.3x slower here.)  A 4-stage shared-memory ring (48 KB per stage)
-//    is guarded by full/empty mbarriers; the MMA thread frees a stage with
+//    swizzle, no multicast; weights read by one tile only carry an
+//    evict-first L2 policy.  Token rows x[t] of the routed gate/up GEMM are
+//    read in place by index: the gather warps issue 16-byte cp.async copies
+//    straight into the 128-byte-swizzled K-major layout the MMA descriptor
+//    reads, and signal each stage with a non-blocking
+//    cp.async.mbarrier.arrive.noinc (the arrival lands when the thread's
+//    copies have), so the gather runs as far ahead as the ring allows; no copy
+//    of x is ever made.  (TMA tile::gather4 was measured 2.3x slower here.)  A
+//    192 KB shared-memory ring (4 stages of 48 KB, 6 of 32 KB, 8 of 24 KB) is
+//    guarded by full/empty mbarriers; the MMA thread frees a stage with
 //    tcgen05.commit.
-//  * One tcgen05.mma.cta_group::1 of M=128, N=256 per 32-byte K slice
+//  * One tcgen05.mma.cta_group::1 of M=128, N=BN per 32-byte K slice
 //    (kind::f16 for bf16, kind::tf32 for fp32), fp32 accumulators in TMEM,
 //    double-buffered (2 x 256 columns) so the epilogue of tile i overlaps the
 //    main loop of tile i+1.
-//  * Epilogues: GATEUP reads gate and up columns of the same row from TMEM
-//    (tcgen05.ld 32x32b), applies silu(g)*u and stores act; DOWN scales each
-//    row by its gate and adds it into the fp32 accumulator with 16-byte vector
-//    reductions (the combine over the k experts of a token).
+//  * Epilogues (grouped_parts.cuh): GATEUP reads gate and up columns of the
+//    same row from TMEM (tcgen05.ld 32x32b), applies silu(g)*u and stores act;
+//    DOWN scales each row by its gate and adds it into the fp32 accumulator
+//    with 16-byte vector reductions (the combine over the k experts of a
+//    token).
+//  * With programmatic dependent launch the prologue overlaps the previous
+//    kernel; when the offsets are known complete (two kernels back) the first
+//    ring of weight tiles is issued before waiting for it.
 //  * Every mbarrier wait is bounded (4 s of %globaltimer); on expiry the CTA
 //    raises the device timeout flag, the other roles stop at their next wait,
 //    outstanding copies are drained and TMEM is released before exit.

@@ -174,7 +174,7 @@ struct GemmLaunch {
     int mode;             // 0: gate/up with SwiGLU epilogue, 1: down with gate-weighted combine
     bool gather;          // A rows gathered from x by index (routed gate/up); else TMA from a_src
     int dtype;            // MOE_BF16 or MOE_F32 (tf32 MMA)
-    bool narrow;          // MMA N = 128 (6-stage ring) instead of N = 256 (4 stages)
+    bool narrow;          // MMA N = 128 instead of N = 256
     bool pair;            // two SMs per tile (clusters of two CTAs, M = 256 MMAs)
     bool half;            // contiguous A only: 64-row tiles with 64-row A stages (few rows per group)
     GemmParams p;
