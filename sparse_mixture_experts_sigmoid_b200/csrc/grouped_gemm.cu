@@ -115,12 +115,14 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     constexpr int kStages = stages_for(BN, kAStage);
     constexpr int kBBytes = BN * 128;                      // one B stage: BN rows x 128 bytes
     constexpr uint32_t kIdesc = instr_desc<T>(BM, BN);
+    constexpr int kStageBytes = MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + kStages * kAStage + kAPad;
-    Ctrl *ctrl = reinterpret_cast<Ctrl *>(sB + kStages * kBBytes);
+    uint8_t *sEpi = sB + kStages * kBBytes;                // DOWN epilogue staging
+    Ctrl *ctrl = reinterpret_cast<Ctrl *>(sEpi + kStageBytes);
     int *tile_start = reinterpret_cast<int *>(ctrl + 1);
     int *seg_off = tile_start + (p.E + 1);
     int *seg_end = seg_off + (p.E + 1);
@@ -290,7 +292,8 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * RB + row;
-            epilogue_row<MODE, T, BN>(p, tl.n, r, row < RB && r < seg_end[tl.e], tmem + acc * BN + lane_base);
+            epilogue_row<MODE, T, BN>(p, tl.n, r, row < RB && r < seg_end[tl.e], tmem + acc * BN + lane_base,
+                                      reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
             tc_fence_before();
             mbar_arrive(&ctrl->tempty[acc]);
         }
@@ -332,8 +335,8 @@ cudaError_t launch_t(const GemmLaunch &L, cudaStream_t s) {
     const int64_t max_m = p.rows / RB + nE;
     const int64_t max_tiles = max_m * n_tiles;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
-    const size_t smem = 1024 + (size_t)kStages * (RB * 128 + BN * 128) + (kABytes - RB * 128) + sizeof(Ctrl) +
-                        3 * sizeof(int) * (p.E + 1);
+    const size_t smem = 1024 + (size_t)kStages * (RB * 128 + BN * 128) + (kABytes - RB * 128) +
+                        (MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0) + sizeof(Ctrl) + 3 * sizeof(int) * (p.E + 1);
     auto kern = grouped_gemm_kernel<MODE, GATHER, T, BN, HALF>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -71,12 +71,14 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     constexpr int kStages = pair_stages(BN);
     constexpr int kBBytes = BN * 64;                 // this CTA's half of a B stage
     constexpr uint32_t kIdesc = instr_desc<T>(BM2, BN);
+    constexpr int kStageBytes = MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + kStages * kABytes;
-    Ctrl2 *ctrl = reinterpret_cast<Ctrl2 *>(sB + kStages * kBBytes);
+    uint8_t *sEpi = sB + kStages * kBBytes;                // DOWN epilogue staging
+    Ctrl2 *ctrl = reinterpret_cast<Ctrl2 *>(sEpi + kStageBytes);
     int *tile_start = reinterpret_cast<int *>(ctrl + 1);
     int *seg_off = tile_start + (p.E + 1);
     int *seg_end = seg_off + (p.E + 1);
@@ -232,7 +234,8 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM2 + row_off + row;
-            epilogue_row<MODE, T, BN>(p, tl.n, r, r < seg_end[tl.e], tmem + acc * BN + lane_base);
+            epilogue_row<MODE, T, BN>(p, tl.n, r, r < seg_end[tl.e], tmem + acc * BN + lane_base,
+                                      reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -284,7 +287,8 @@ cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
     } else {
         mA = mB0;   // unused: gather mode reads x with cp.async
     }
-    const size_t smem = 1024 + (size_t)kStages * (kABytes + BN * 64) + sizeof(Ctrl2) + 3 * sizeof(int) * (p.E + 1);
+    const size_t smem = 1024 + (size_t)kStages * (kABytes + BN * 64) + (MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0) +
+                        sizeof(Ctrl2) + 3 * sizeof(int) * (p.E + 1);
     auto kern = grouped_gemm_pair_kernel<MODE, GATHER, T, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

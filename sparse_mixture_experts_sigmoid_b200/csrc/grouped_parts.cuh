@@ -19,16 +19,22 @@ using namespace tc;
 
 enum { GATEUP = 0, DOWN = 1 };
 
+// shared-memory staging of the DOWN epilogue: 32 rows x 32 fp32 per warp
+constexpr int kEpiStageBytes = 32 * 32 * 4;
+
 // Epilogue of one grouped row r (valid: r lies inside its expert's segment)
 // of a tile in column tile n, whose fp32 accumulator row starts at TMEM
 // address tbase (this thread's lane).  GATEUP holds BN/2 gate columns then
 // BN/2 up columns and stores silu(g) * u into act; DOWN scales the BN
-// columns by the row's gate and adds them into y_acc with 16-byte reductions.
-// Several TMEM loads are in flight per wait.
+// columns by the row's gate and adds them into y_acc with 16-byte reductions,
+// through the warp's 4 KB shared-memory staging block `stage`.  Several TMEM
+// loads are in flight per wait.  Called by all 32 lanes of an epilogue warp.
 template <int MODE, typename T, int BN>
-__device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t r, bool valid, uint32_t tbase) {
+__device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t r, bool valid, uint32_t tbase,
+                                             float *stage) {
     constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
     if constexpr (MODE == GATEUP) {
+        if (!__any_sync(0xffffffffu, valid)) return;   // no row of this warp lies in the segment
         T *act = static_cast<T *>(p.act);
         // silu(g) * u for 16 output columns from column c of the tile
         auto store16 = [&](int c, const float(&g)[16], const float(&u)[16]) {
@@ -71,7 +77,7 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
             store16(c + 16, g[1], u[1]);
         }
     } else {
-        int64_t t = -1;
+        int t = -1;
         float gate = 0.f;
         if (valid) {
             if (p.sorted_rows) {
@@ -79,7 +85,7 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
                 t = v / p.k;
                 gate = (v >= 0 && v < p.rows) ? p.gates[v] : 0.f;
             } else {
-                t = r;
+                t = (int)r;
                 gate = p.gates[r];
             }
             if (t < 0 || t >= p.T) {
@@ -87,6 +93,19 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
                 t = -1;
             }
         }
+        if (!__any_sync(0xffffffffu, t >= 0)) return;   // no row of this warp lies in the segment
+        // The gate-scaled rows go through a 32 x 32 fp32 staging block so that
+        // each reduction instruction covers four whole 128-byte row segments of
+        // y_acc instead of 16 bytes in each of 32 rows: lane l reduces the
+        // 16-byte chunk l % 8 of staged row 4i + l / 8 in pass i.  Chunk q of
+        // row w is stored at slot q ^ (w % 8), so neither the row-wise writes
+        // nor the column-wise reads hit a shared-memory bank twice per phase.
+        const int lane = threadIdx.x & 31;
+        const int j = lane & 7;
+        int tok[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tok[i] = __shfl_sync(0xffffffffu, t, 4 * i + (lane >> 3));
+        float4 *st = reinterpret_cast<float4 *>(stage);
         // 32 columns per TMEM wait: two loads in flight at a time
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -95,16 +114,20 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
             tmem_ld16(tbase + c + 16, v[1]);
             tmem_wait_ld();
 #pragma unroll
-            for (int hh = 0; hh < 2 && t >= 0; ++hh) {
-                const int col = n * BN + c + 16 * hh;
-                float *dst = p.y_acc + t * p.N + col;
+            for (int q = 0; q < 8; ++q)
+                st[lane * 8 + (q ^ (lane & 7))] =
+                    make_float4(gate * v[q >> 2][4 * (q & 3)], gate * v[q >> 2][4 * (q & 3) + 1],
+                                gate * v[q >> 2][4 * (q & 3) + 2], gate * v[q >> 2][4 * (q & 3) + 3]);
+            __syncwarp();
+            const int col = n * BN + c + 4 * j;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (col + 4 * q < p.N)
-                        atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
-                                  make_float4(gate * v[hh][4 * q], gate * v[hh][4 * q + 1], gate * v[hh][4 * q + 2],
-                                              gate * v[hh][4 * q + 3]));
+            for (int i = 0; i < 8; ++i) {
+                const int w = 4 * i + (lane >> 3);
+                const float4 val = st[w * 8 + (j ^ (w & 7))];
+                if (tok[i] >= 0 && col < p.N)
+                    atomicAdd(reinterpret_cast<float4 *>(p.y_acc + (int64_t)tok[i] * p.N + col), val);
             }
+            __syncwarp();
         }
     }
 }
