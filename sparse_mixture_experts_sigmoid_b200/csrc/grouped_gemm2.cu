@@ -40,7 +40,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;               // MMA issuer in the even CTA, gather relay in the odd one
 constexpr int kGatherWarp0 = 6;
-constexpr int kGatherThreads = 128;
+constexpr int kGatherThreads = 256;
 constexpr int kTmemCols = 512;
 
 // Ring depth for an MMA N of BN (each CTA holds BN / 2 rows of B per stage).
@@ -62,14 +62,22 @@ struct Ctrl2 {
     int pad;
 };
 
-template <int MODE, bool GATHER, typename T, int BN>
-__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+// W = 2 (gathered gate/up): each pair tile issues two N = BN MMAs per K slice
+// into one 2 x BN column accumulator, so every gathered token row feeds twice
+// the output columns and the gather, which bounds this GEMM, is needed at half
+// the rate per FLOP.  The accumulator then fills TMEM and is not double
+// buffered: the epilogue of a tile does not overlap the next tile's MMAs.
+template <int MODE, bool GATHER, typename T, int BN, int W>
+__global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1, GemmParams p) {
     constexpr int BK = 128 / (int)sizeof(T);
-    constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
-    constexpr int kStages = pair_stages(BN);
-    constexpr int kBBytes = BN * 64;                 // this CTA's half of a B stage
+    static_assert(W == 1 || (W == 2 && MODE == GATEUP), "wide tiles are for gate/up");
+    constexpr int BN_OUT = MODE == GATEUP ? W * BN / 2 : BN;   // output columns per tile
+    constexpr int kStages = pair_stages(W * BN);
+    constexpr int kBSub = BN * 64;                   // this CTA's half of one MMA's B
+    constexpr int kBBytes = W * kBSub;               // this CTA's B per stage
+    constexpr int kAccBufs = W == 1 ? 2 : 1;         // TMEM accumulators of W x BN columns
     constexpr uint32_t kIdesc = instr_desc<T>(BM2, BN);
     constexpr int kStageBytes = MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0;
 
@@ -96,7 +104,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             mbar_init(&ctrl->empty[s], 1);
             mbar_init(&ctrl->gfull[s], kGatherThreads);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < kAccBufs; ++a) {
             mbar_init(&ctrl->tfull[a], 1);
             mbar_init(&ctrl->tempty[a], 2 * kEpiWarps);
         }
@@ -139,8 +147,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             for (int id = pair; id < total && ok; id += npairs) {
                 const Tile tl = decode(id, n_tiles, tile_start, nE);
                 const int a_row = seg_off[tl.e] + tl.m * BM2 + row_off;
-                // gate/up: the gate rows from CTA 0, the up rows from CTA 1;
-                // down: the first and second half of the BN weight rows
+                // gate/up: the gate rows from CTA 0, the up rows from CTA 1 (W x
+                // BN / 2 of them, one box); down: the first and second half of
+                // the BN weight rows
                 const int b_row = tl.e * p.N + tl.n * BN_OUT + (MODE == GATEUP ? 0 : (int)rank * (BN / 2));
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
@@ -170,7 +179,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             uint32_t it = 0, tc = 0;
             bool ok = true;
             for (int id = pair; id < total && ok; id += npairs, ++tc) {
-                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                const uint32_t acc = tc % kAccBufs, aph = (tc / kAccBufs) & 1;
                 if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + acc * BN;
@@ -186,10 +195,14 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                     if constexpr (GATHER) fence_proxy_async();
                     tc_fence_after();
                     const uint64_t ad = smem_desc(sA + s * kABytes);
-                    const uint64_t bd = smem_desc(sB + s * kBBytes);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma2<T>(d_tmem, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb | kk) != 0);
+                    for (int j = 0; j < W; ++j) {
+                        // MMA j: B rows j * BN / 2 .. of each CTA -> accumulator columns j * BN ..
+                        const uint64_t bd = smem_desc(sB + s * kBBytes + j * kBSub);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma2<T>(d_tmem + j * BN, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb | kk) != 0);
+                    }
                     mma_commit2(&ctrl->empty[s], 0x3);
                 }
                 if (ok) mma_commit2(&ctrl->tfull[acc], 0x3);
@@ -230,12 +243,14 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         const uint32_t tempty_lead = mapa_shared(&ctrl->tempty[0], 0);
         for (int id = pair; id < total; id += npairs, ++tc) {
             const Tile tl = decode(id, n_tiles, tile_start, nE);
-            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            const uint32_t acc = tc % kAccBufs, aph = (tc / kAccBufs) & 1;
             if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM2 + row_off + row;
-            epilogue_row<MODE, T, BN>(p, tl.n, r, r < seg_end[tl.e], tmem + acc * BN + lane_base,
-                                      reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
+#pragma unroll 1
+            for (int j = 0; j < W; ++j)
+                epilogue_row<MODE, T, BN>(p, tl.n * W + j, r, r < seg_end[tl.e], tmem + (acc + j) * BN + lane_base,
+                                          reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -244,7 +259,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             }
         }
     } else if (GATHER && warp >= kGatherWarp0) {
-        gather_rows<T, kStages, BM2>(p, threadIdx.x - kGatherWarp0 * 32, pair, npairs, total, n_tiles, tile_start,
+        gather_rows<T, kStages, BM2, kGatherThreads>(p, threadIdx.x - kGatherWarp0 * 32, pair, npairs, total, n_tiles, tile_start,
                                      seg_off, seg_end, nE, nk, row_off, sA, lead ? ctrl->full : ctrl->gfull,
                                      ctrl->empty, abort);
     }
@@ -267,18 +282,18 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
 // ------------------------------------------------------------------ host side
 
-template <int MODE, bool GATHER, typename T, int BN>
+template <int MODE, bool GATHER, typename T, int BN, int W>
 cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
     const GemmParams &p = L.p;
-    constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
-    constexpr int kStages = pair_stages(BN);
+    constexpr int BN_OUT = MODE == GATEUP ? W * BN / 2 : BN;
+    constexpr int kStages = pair_stages(W * BN);
     const bool f32 = sizeof(T) == 4;
     CUtensorMap mA, mB0, mB1;
     const int nE = p.offsets ? p.E : 1;
     // B boxes hold this CTA's half of the tile's weight rows
-    if (!make_map(&mB0, L.b0, f32, (uint64_t)nE * p.N, p.K, BN / 2)) return cudaErrorInvalidValue;
+    if (!make_map(&mB0, L.b0, f32, (uint64_t)nE * p.N, p.K, W * BN / 2)) return cudaErrorInvalidValue;
     if (MODE == GATEUP) {
-        if (!make_map(&mB1, L.b1, f32, (uint64_t)nE * p.N, p.K, BN / 2)) return cudaErrorInvalidValue;
+        if (!make_map(&mB1, L.b1, f32, (uint64_t)nE * p.N, p.K, W * BN / 2)) return cudaErrorInvalidValue;
     } else {
         mB1 = mB0;
     }
@@ -287,9 +302,9 @@ cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
     } else {
         mA = mB0;   // unused: gather mode reads x with cp.async
     }
-    const size_t smem = 1024 + (size_t)kStages * (kABytes + BN * 64) + (MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0) +
+    const size_t smem = 1024 + (size_t)kStages * (kABytes + W * BN * 64) + (MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0) +
                         sizeof(Ctrl2) + 3 * sizeof(int) * (p.E + 1);
-    auto kern = grouped_gemm_pair_kernel<MODE, GATHER, T, BN>;
+    auto kern = grouped_gemm_pair_kernel<MODE, GATHER, T, BN, W>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // as many CTA pairs as can be resident at once (one CTA per SM), capped by
@@ -303,7 +318,7 @@ cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
         if (!max_pairs[dev]) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
-            cfg.blockDim = dim3(GATHER ? 320 : 192);
+            cfg.blockDim = dim3(GATHER ? 192 + kGatherThreads : 192);
             cfg.dynamicSmemBytes = smem;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -321,12 +336,18 @@ cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
     const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
     const int64_t max_tiles = (p.rows / BM2 + nE) * (int64_t)n_tiles;
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs[dev], max_tiles));
-    return launch_kernel_pair(kern, 2 * pairs, GATHER ? 320 : 192, smem, s, mA, mB0, mB1, p);
+    return launch_kernel_pair(kern, 2 * pairs, GATHER ? 192 + kGatherThreads : 192, smem, s, mA, mB0, mB1, p);
 }
 
 template <int MODE, bool GATHER, typename T>
 cudaError_t launch_pair_bn(const GemmLaunch &L, cudaStream_t s) {
-    return L.narrow ? launch_pair_t<MODE, GATHER, T, 128>(L, s) : launch_pair_t<MODE, GATHER, T, 256>(L, s);
+    if (L.narrow) return launch_pair_t<MODE, GATHER, T, 128, 1>(L, s);
+#ifndef MOE_GG_WIDE
+#define MOE_GG_WIDE 1
+#endif
+    if constexpr (MODE == GATEUP && GATHER && MOE_GG_WIDE)
+        if (L.p.N >= 256) return launch_pair_t<MODE, GATHER, T, 256, 2>(L, s);
+    return launch_pair_t<MODE, GATHER, T, 256, 1>(L, s);
 }
 
 }  // namespace gg

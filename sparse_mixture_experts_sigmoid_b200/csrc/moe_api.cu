@@ -106,20 +106,25 @@ bool narrow_down(const moe_config &c) { return c.d % 256 != 0; }
 // Experts average at most one 128-row tile: every weight tile is read once.
 bool one_tile_per_expert(const moe_config &c) { return (int64_t)c.T * c.k <= 128LL * c.E; }
 
-// Two SMs per tile (M = 256 across a CTA pair) for GEMMs whose A operand comes
-// by TMA and whose groups average at least 512 rows: the layer is tensor-bound
-// and the operand traffic per SM drops by a third (measured: mixtral_prefill
-// down 874 -> 732 us, the shared expert's gate/up and down of qwen_shared -17%).
-// With gathered token rows the pair is slower (the odd CTA's rows reach the
-// MMA through a relay) and with fewer rows the 256-row tiles waste work, so
-// those keep one SM per tile.  MOE_GG_PAIR=1 / 0 forces it on / off.
-bool pair_tiles(int64_t rows, int groups, bool gather) {
+// Two SMs per tile (M = 256 across a CTA pair) for GEMMs whose groups average
+// at least 512 rows: the layer is tensor-bound and the operand traffic per SM
+// drops by a third (measured: mixtral_prefill down 874 -> 732 us, the shared
+// expert's gate/up and down of qwen_shared -17%).  With gathered token rows
+// the pair pays only with its wide tiles (two MMAs of N = 256 per K slice, so
+// the gather is needed at half the rate per FLOP), which want the output width
+// to be a multiple of 256; with fewer rows the 256-row tiles waste work.
+// MOE_GG_PAIR=1 / 0 forces it on / off.
+#ifndef MOE_GG_PAIR_GATHER
+#define MOE_GG_PAIR_GATHER 1
+#endif
+bool pair_tiles(int64_t rows, int groups, bool gather, int64_t out_cols) {
     static const int force = [] {
         const char *v = std::getenv("MOE_GG_PAIR");
         return v ? (v[0] == '1' ? 1 : 0) : -1;
     }();
     if (force >= 0) return force == 1;
-    return !gather && rows >= 512LL * groups;
+    if (gather) return MOE_GG_PAIR_GATHER && out_cols % 256 == 0 && rows >= 512LL * groups;
+    return rows >= 512LL * groups;
 }
 
 // 64-row tiles for a contiguous A when the groups average at most 64 rows
@@ -143,7 +148,7 @@ GemmLaunch gemm_gateup(const moe_config &c, const void *x, const void *wg, const
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.d, c.h, x, act, nullptr, nullptr, err};
     L.narrow = narrow_gateup(c);
     L.p.stream_weights = one_tile_per_expert(c);
-    L.pair = pair_tiles(c.T * c.k, c.E, true);
+    L.pair = pair_tiles(c.T * c.k, c.E, true, c.h);
     L.b0 = wg;
     L.b1 = wu;
     return L;
@@ -155,7 +160,7 @@ GemmLaunch gemm_gateup_dense(const moe_config &c, const void *x, const void *wg,
     L.gather = false;
     L.dtype = c.dtype;
     L.p = GemmParams{nullptr, nullptr, 1, 1, c.T, c.T, c.d, c.h_shared, x, act, nullptr, nullptr, err};
-    L.pair = pair_tiles(c.T, 1, false);
+    L.pair = pair_tiles(c.T, 1, false, c.h_shared);
     L.a_src = x;
     L.b0 = wg;
     L.b1 = wu;
@@ -170,7 +175,7 @@ GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const
     L.p = GemmParams{offsets, srt, c.E, c.k, c.T * c.k, c.T, c.h, c.d, nullptr, nullptr, acc, gates, err};
     L.narrow = narrow_down(c);
     L.p.stream_weights = one_tile_per_expert(c);
-    L.pair = pair_tiles(c.T * c.k, c.E, false);
+    L.pair = pair_tiles(c.T * c.k, c.E, false, c.d);
     L.half = !L.pair && half_tiles(c.T * c.k, c.E);
     L.a_src = act;
     L.b0 = wd;
@@ -183,7 +188,7 @@ GemmLaunch gemm_down_dense(const moe_config &c, const void *act, const void *wd,
     L.gather = false;
     L.dtype = c.dtype;
     L.p = GemmParams{nullptr, nullptr, 1, 1, c.T, c.T, c.h_shared, c.d, nullptr, nullptr, acc, sg, err};
-    L.pair = pair_tiles(c.T, 1, false);
+    L.pair = pair_tiles(c.T, 1, false, c.d);
     L.a_src = act;
     L.b0 = wd;
     return L;
