@@ -65,8 +65,11 @@ struct Ctrl2 {
 // W = 2 (gathered gate/up): each pair tile issues two N = BN MMAs per K slice
 // into one 2 x BN column accumulator, so every gathered token row feeds twice
 // the output columns and the gather, which bounds this GEMM, is needed at half
-// the rate per FLOP.  The accumulator then fills TMEM and is not double
-// buffered: the epilogue of a tile does not overlap the next tile's MMAs.
+// the rate per FLOP.  The accumulator then fills TMEM, so instead of two
+// accumulators its two halves (MMA j = 0 and 1) are handed over separately:
+// in a tile's last ring of K blocks the MMAs of half 0 run first and half 0
+// goes to the epilogue while half 1 finishes, and in the next tile's first
+// ring of K blocks half 0 is started while the epilogue still drains half 1.
 template <int MODE, bool GATHER, typename T, int BN, int W>
 __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -77,7 +80,6 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     constexpr int kStages = pair_stages(W * BN);
     constexpr int kBSub = BN * 64;                   // this CTA's half of one MMA's B
     constexpr int kBBytes = W * kBSub;               // this CTA's B per stage
-    constexpr int kAccBufs = W == 1 ? 2 : 1;         // TMEM accumulators of W x BN columns
     constexpr uint32_t kIdesc = instr_desc<T>(BM2, BN);
     constexpr int kStageBytes = MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0;
 
@@ -104,7 +106,8 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             mbar_init(&ctrl->empty[s], 1);
             mbar_init(&ctrl->gfull[s], kGatherThreads);
         }
-        for (int a = 0; a < kAccBufs; ++a) {
+        // W = 1: two accumulators; W = 2: the two halves of one
+        for (int a = 0; a < 2; ++a) {
             mbar_init(&ctrl->tfull[a], 1);
             mbar_init(&ctrl->tempty[a], 2 * kEpiWarps);
         }
@@ -178,34 +181,92 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
         if (lane == 0 && lead) {
             uint32_t it = 0, tc = 0;
             bool ok = true;
-            for (int id = pair; id < total && ok; id += npairs, ++tc) {
-                const uint32_t acc = tc % kAccBufs, aph = (tc / kAccBufs) & 1;
-                if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + acc * BN;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1;
-                    bool got = mbar_try_wait_cluster(&ctrl->full[s], ph);
-                    if (!got) got = wait_bar(&ctrl->full[s], ph, abort, p.err) && mbar_try_wait_cluster(&ctrl->full[s], ph);
-                    if (!got) {
-                        ok = false;
-                        break;
-                    }
+            // the operands of ring position i have landed (both CTAs)
+            auto wait_full = [&](uint32_t i) -> bool {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                bool got = mbar_try_wait_cluster(&ctrl->full[s], ph);
+                if (!got) got = wait_bar(&ctrl->full[s], ph, abort, p.err) && mbar_try_wait_cluster(&ctrl->full[s], ph);
+                if (got) {
                     if constexpr (GATHER) fence_proxy_async();
                     tc_fence_after();
-                    const uint64_t ad = smem_desc(sA + s * kABytes);
-#pragma unroll
-                    for (int j = 0; j < W; ++j) {
-                        // MMA j: B rows j * BN / 2 .. of each CTA -> accumulator columns j * BN ..
-                        const uint64_t bd = smem_desc(sB + s * kBBytes + j * kBSub);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma2<T>(d_tmem + j * BN, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb | kk) != 0);
-                    }
-                    mma_commit2(&ctrl->empty[s], 0x3);
                 }
-                if (ok) mma_commit2(&ctrl->tfull[acc], 0x3);
+                return got;
+            };
+            // MMA j of K block kb from ring position i into accumulator columns d
+            auto issue = [&](uint32_t i, int kb, int j, uint32_t d) {
+                const int s = i % kStages;
+                const uint64_t ad = smem_desc(sA + s * kABytes);
+                // B rows j * BN / 2 .. of each CTA
+                const uint64_t bd = smem_desc(sB + s * kBBytes + j * kBSub);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma2<T>(d + j * BN, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb | kk) != 0);
+            };
+            auto release = [&](uint32_t i) { mma_commit2(&ctrl->empty[i % kStages], 0x3); };
+            for (int id = pair; id < total && ok; id += npairs, ++tc) {
+                if constexpr (W == 1) {
+                    const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                    if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int kb = 0; kb < nk; ++kb, ++it) {
+                        if (!wait_full(it)) {
+                            ok = false;
+                            break;
+                        }
+                        issue(it, kb, 0, tmem + acc * BN);
+                        release(it);
+                    }
+                    if (ok) mma_commit2(&ctrl->tfull[acc], 0x3);
+                } else {
+                    const uint32_t aph = tc & 1;
+                    const int H = nk < kStages ? nk : kStages;                      // head K blocks
+                    const int Tb = nk - H < kStages ? nk - H : kStages;            // tail K blocks
+                    // head: half 0 over the first ring once the epilogue has
+                    // released it, then half 1 once that is released too
+                    if (!wait_bar(&ctrl->tempty[0], aph ^ 1, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int kb = 0; kb < H && ok; ++kb) {
+                        if (wait_full(it + kb)) issue(it + kb, kb, 0, tmem);
+                        else ok = false;
+                    }
+                    if (!ok) break;
+                    if (H == nk) mma_commit2(&ctrl->tfull[0], 0x3);
+                    if (!wait_bar(&ctrl->tempty[1], aph ^ 1, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int kb = 0; kb < H; ++kb) {
+                        issue(it + kb, kb, 1, tmem);
+                        release(it + kb);
+                    }
+                    it += H;
+                    // body: both halves per K block
+                    for (int kb = H; kb < nk - Tb; ++kb, ++it) {
+                        if (!wait_full(it)) {
+                            ok = false;
+                            break;
+                        }
+                        issue(it, kb, 0, tmem);
+                        issue(it, kb, 1, tmem);
+                        release(it);
+                    }
+                    if (!ok) break;
+                    // tail: half 0 over the last ring, handed to the epilogue,
+                    // then half 1
+                    if (Tb > 0) {
+                        for (int q = 0; q < Tb && ok; ++q) {
+                            if (wait_full(it + q)) issue(it + q, nk - Tb + q, 0, tmem);
+                            else ok = false;
+                        }
+                        if (!ok) break;
+                        mma_commit2(&ctrl->tfull[0], 0x3);
+                        for (int q = 0; q < Tb; ++q) {
+                            issue(it + q, nk - Tb + q, 1, tmem);
+                            release(it + q);
+                        }
+                        it += Tb;
+                    }
+                    mma_commit2(&ctrl->tfull[1], 0x3);
+                }
             }
             mma_commit2(&ctrl->done, 0x3);
         } else if (lane == 0 && GATHER) {
@@ -241,21 +302,28 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
         const int row = warp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const uint32_t tempty_lead = mapa_shared(&ctrl->tempty[0], 0);
-        for (int id = pair; id < total; id += npairs, ++tc) {
+        bool ok = true;
+        for (int id = pair; id < total && ok; id += npairs, ++tc) {
             const Tile tl = decode(id, n_tiles, tile_start, nE);
-            const uint32_t acc = tc % kAccBufs, aph = (tc / kAccBufs) & 1;
-            if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
-            tc_fence_after();
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM2 + row_off + row;
 #pragma unroll 1
-            for (int j = 0; j < W; ++j)
-                epilogue_row<MODE, T, BN>(p, tl.n * W + j, r, r < seg_end[tl.e], tmem + (acc + j) * BN + lane_base,
+            for (int j = 0; j < W; ++j) {
+                // W = 1: accumulator tc % 2; W = 2: half j of the one accumulator
+                const uint32_t b = W == 1 ? (tc & 1) : (uint32_t)j;
+                const uint32_t ph = W == 1 ? ((tc >> 1) & 1) : (tc & 1);
+                if (!wait_bar(&ctrl->tfull[b], ph, abort, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                epilogue_row<MODE, T, BN>(p, tl.n * W + j, r, r < seg_end[tl.e], tmem + b * BN + lane_base,
                                           reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (lead) mbar_arrive(&ctrl->tempty[acc]);
-                else mbar_arrive_remote(tempty_lead + acc * (uint32_t)sizeof(uint64_t));
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (lead) mbar_arrive(&ctrl->tempty[b]);
+                    else mbar_arrive_remote(tempty_lead + b * (uint32_t)sizeof(uint64_t));
+                }
             }
         }
     } else if (GATHER && warp >= kGatherWarp0) {
