@@ -9,7 +9,8 @@
 // into shared memory for the same MMA work that costs 48 KB on one SM: the
 // operand traffic per FLOP, which bounds the one-SM kernel on these layers,
 // drops by a third.  The even CTA issues M=256 MMAs that read both CTAs'
-// shared memory and write each CTA's half of D into its own TMEM.
+// shared memory and write each CTA's half of D into its own TMEM.  The
+// gathered gate/up runs with wide tiles (two MMAs per K slice, see W below).
 //
 // Synchronisation across the pair:
 //  * both CTAs' TMA loads complete on the even CTA's full[s] barrier (the
