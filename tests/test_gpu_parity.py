@@ -138,6 +138,9 @@ SMALL = [
     small("single_expert", E=1, k=1, seed=58),
     small("decode_T1", T=1, seed=59),
     small("decode_T3", T=3, E=64, k=8, seed=60),
+    small("decode_T1_shared", T=1, h_shared=64, seed=65),
+    small("decode_T1_ragged_widths", T=1, d=200, h=136, h_shared=72, score="sigmoid", seed=66),
+    small("decode_T1_k16", T=1, E=64, k=16, d=128, h=64, router_std=0.2, seed=67),
     small("width_not_mult_64", d=200, h=136, seed=61),
     small("many_experts", E=512, k=16, T=200, d=128, h=64, router_std=0.2, seed=62),
     small("zipf_hot_expert", recipe="zipf", E=32, k=2, seed=63),
