@@ -11,6 +11,9 @@
 // expert linears, silu(gate) * up, weighted sum); "Small MoE Architecture, in
 // depth", Expert.forward (the SwiGLU expert) and the batch-1 decode remarks in
 // "Why small changes the MoE trade-off" (decode reads only the chosen experts).
+#include <mutex>
+#include <unordered_map>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -301,8 +304,26 @@ __global__ void finalize_kernel(const float *y_acc, T *y, int64_t n) {
     }
 }
 
-int grid_for(int64_t items) {
-    const int64_t cap = 4LL * num_sms();
+// One warp per item, but no more CTAs than fit on the GPU at once: the
+// kernels stream weights, so the warps resident per SM (and with them the
+// bytes in flight) are what sets their rate.  The residency of each kernel is
+// asked for once.
+template <typename K>
+int grid_for(K kern, int64_t items, size_t smem) {
+    static std::mutex mu;
+    static std::unordered_map<const void *, int> per_sm;
+    int b = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = per_sm.find(reinterpret_cast<const void *>(kern));
+        if (it != per_sm.end()) {
+            b = it->second;
+        } else {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, smem) != cudaSuccess || b < 1) b = 1;
+            per_sm[reinterpret_cast<const void *>(kern)] = b;
+        }
+    }
+    const int64_t cap = (int64_t)b * num_sms();
     const int64_t need = (items + kWarps - 1) / kWarps;
     return (int)(need < cap ? (need > 0 ? need : 1) : cap);
 }
@@ -312,29 +333,24 @@ int grid_for(int64_t items) {
 cudaError_t launch_seg_gateup(const SegGateUpArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
     if (a.seg.rows <= 0) return cudaSuccess;
     const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
-    const int grid = grid_for((int64_t)a.seg.E * a.hid);
-    if (dtype == MOE_F32)
-        return a.T == 1 ? launch_kernel(seg_gateup_kernel<float, 1>, grid, kThreads, smem, s, a, err)
-                        : launch_kernel(seg_gateup_kernel<float, RB>, grid, kThreads, smem, s, a, err);
-    return a.T == 1 ? launch_kernel(seg_gateup_kernel<__nv_bfloat16, 1>, grid, kThreads, smem, s, a, err)
-                    : launch_kernel(seg_gateup_kernel<__nv_bfloat16, RB>, grid, kThreads, smem, s, a, err);
+    const int64_t items = (int64_t)a.seg.E * a.hid;
+    auto go = [&](auto kern) { return launch_kernel(kern, grid_for(kern, items, smem), kThreads, smem, s, a, err); };
+    if (dtype == MOE_F32) return a.T == 1 ? go(seg_gateup_kernel<float, 1>) : go(seg_gateup_kernel<float, RB>);
+    return a.T == 1 ? go(seg_gateup_kernel<__nv_bfloat16, 1>) : go(seg_gateup_kernel<__nv_bfloat16, RB>);
 }
 
 cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
     if (a.seg.rows <= 0) return cudaSuccess;
     const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
-    const int grid = grid_for((int64_t)a.seg.E * a.d);
-    if (dtype == MOE_F32)
-        return launch_kernel(seg_down_kernel<float>, grid, kThreads, smem, s, a, err);
-    return launch_kernel(seg_down_kernel<__nv_bfloat16>, grid, kThreads, smem, s, a, err);
+    const int64_t items = (int64_t)a.seg.E * a.d;
+    auto go = [&](auto kern) { return launch_kernel(kern, grid_for(kern, items, smem), kThreads, smem, s, a, err); };
+    return dtype == MOE_F32 ? go(seg_down_kernel<float>) : go(seg_down_kernel<__nv_bfloat16>);
 }
 
 cudaError_t launch_down_direct(const DownDirectArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
     if (a.T <= 0) return cudaSuccess;
-    const int grid = grid_for(a.T * a.d);
-    if (dtype == MOE_F32)
-        return launch_kernel(down_direct_kernel<float>, grid, kThreads, 0, s, a, err);
-    return launch_kernel(down_direct_kernel<__nv_bfloat16>, grid, kThreads, 0, s, a, err);
+    auto go = [&](auto kern) { return launch_kernel(kern, grid_for(kern, a.T * a.d, 0), kThreads, 0, s, a, err); };
+    return dtype == MOE_F32 ? go(down_direct_kernel<float>) : go(down_direct_kernel<__nv_bfloat16>);
 }
 
 cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s) {
