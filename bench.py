@@ -42,7 +42,7 @@ STAGE_KERNEL = {"route": ("router_logits_kernel", "router_tc.cu"), "permute": ("
                 "shared_down": ("grouped_gemm_kernel", GG_SRC),
                 "finalize": ("finalize_kernel", "segment.cu")}
 # kernels of the small-batch path (at most 64 assignments)
-STAGE_KERNEL_SMALL = {"route": ("router_kernel", "router.cu"), "gate_up": ("seg_gateup_kernel", "segment.cu"),
+STAGE_KERNEL_SMALL = {"route": ("router_small_kernel", "router.cu"), "gate_up": ("seg_gateup_kernel", "segment.cu"),
                       "down": ("down_direct_kernel", "segment.cu")}
 
 
