@@ -44,7 +44,7 @@ using namespace tc;
 
 constexpr int BM = 128;
 constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4, kTmaWarp = 4, kMmaWarp = 5;
+constexpr int kTmaWarp = 4, kMmaWarp = 5;   // warps 0-3: epilogue
 constexpr uint32_t kCols = 256;       // TMEM columns per CTA: two CTAs share an SM
 #ifndef MOE_ROUTER_TARGET_CTAS
 #define MOE_ROUTER_TARGET_CTAS 256
