@@ -87,15 +87,21 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     P = ctypes.c_void_p
     I64 = ctypes.c_int64
-    lib.oracle_route.argtypes = [ctypes.POINTER(_CCfg), P, P, P, I64, I64, P, P, P, P, ctypes.c_int]
+    lib.oracle_route.argtypes = [ctypes.POINTER(_CCfg), P, P, P, P, I64, I64, P, P, P, P, ctypes.c_int]
     lib.oracle_route.restype = ctypes.c_int
-    lib.oracle_topk_margin.argtypes = [ctypes.POINTER(_CCfg), P, P, I64, I64, P, ctypes.c_int]
+    lib.oracle_topk_margin.argtypes = [ctypes.POINTER(_CCfg), P, P, P, I64, I64, P, ctypes.c_int]
     lib.oracle_topk_margin.restype = ctypes.c_int
     lib.oracle_permute.argtypes = [ctypes.POINTER(_CCfg), P, P, P, P, P]
     lib.oracle_permute.restype = ctypes.c_int
-    lib.oracle_forward.argtypes = [ctypes.POINTER(_CCfg), P, P, P, P, P, P, P, P, P, P, I64, P,
+    lib.oracle_forward.argtypes = [ctypes.POINTER(_CCfg), P, P, P, P, P, P, P, P, P, P, P, I64, P,
                                    ctypes.c_int]
     lib.oracle_forward.restype = ctypes.c_int
+    lib.oracle_update_bias.argtypes = [ctypes.POINTER(_CCfg), P, ctypes.c_float, P, P]
+    lib.oracle_update_bias.restype = ctypes.c_int
+    lib.oracle_score_mean.argtypes = [ctypes.POINTER(_CCfg), P, P, P, ctypes.c_int]
+    lib.oracle_score_mean.restype = ctypes.c_int
+    lib.oracle_balance_loss.argtypes = [ctypes.POINTER(_CCfg), P, P, ctypes.c_double, P, P]
+    lib.oracle_balance_loss.restype = ctypes.c_int
     _lib_cache[path] = lib
     return lib
 
@@ -114,34 +120,48 @@ def _check_dtype(c: Cfg, *arrays):
             raise TypeError(f"oracle expects {np.dtype(want)} arrays for dtype {c.dtype}, got {a.dtype}")
 
 
+def _bias(c: Cfg, bias):
+    """The balance bias as a C-contiguous float32 [E] array (or None)."""
+    if bias is None:
+        return None
+    b = np.ascontiguousarray(bias, dtype=np.float32).reshape(-1)
+    if b.size != c.E:
+        raise ValueError(f"bias must have {c.E} entries, got {b.size}")
+    return b
+
+
 def route(c: Cfg, x, wr, w_sg=None, t0: int = 0, t1: int | None = None, want_probs=False,
-          nthreads: int = 0, lib: ctypes.CDLL | None = None):
+          nthreads: int = 0, lib: ctypes.CDLL | None = None, bias=None):
     """Routes tokens [t0, t1).  Returns (ids[T,k] int32, gates[T,k], probs[T,E] | None,
-    shared_gate[T] | None); rows outside [t0, t1) are left zero."""
+    shared_gate[T] | None); rows outside [t0, t1) are left zero.  ``bias`` is the
+    optional [E] float32 balance bias (selection only)."""
     lib = lib or load()
     _check_dtype(c, x, wr, w_sg)
+    bias = _bias(c, bias)
     t1 = c.T if t1 is None else t1
     ids = np.zeros((c.T, c.k), np.int32)
     gates = np.zeros((c.T, c.k), np.float64)
     probs = np.zeros((c.T, c.E), np.float64) if want_probs else None
     sg = np.zeros((c.T,), np.float64) if (c.h_shared > 0 and w_sg is not None) else None
     cc = _ccfg(c)
-    rc = lib.oracle_route(ctypes.byref(cc), _ptr(x), _ptr(wr), _ptr(w_sg), t0, t1, _ptr(ids),
-                          _ptr(gates), _ptr(probs), _ptr(sg), nthreads)
+    rc = lib.oracle_route(ctypes.byref(cc), _ptr(x), _ptr(wr), _ptr(w_sg), _ptr(bias), t0, t1,
+                          _ptr(ids), _ptr(gates), _ptr(probs), _ptr(sg), nthreads)
     if rc != 0:
         raise ValueError("oracle_route rejected its arguments")
     return ids, gates, probs, sg
 
 
 def topk_margin(c: Cfg, x, wr, t0: int = 0, t1: int | None = None, nthreads: int = 0,
-                lib: ctypes.CDLL | None = None):
+                lib: ctypes.CDLL | None = None, bias=None):
     """Per-token smallest gap between adjacent keys among the top min(k+1, E)."""
     lib = lib or load()
     _check_dtype(c, x, wr)
+    bias = _bias(c, bias)
     t1 = c.T if t1 is None else t1
     out = np.zeros((t1 - t0,), np.float64)
     cc = _ccfg(c)
-    if lib.oracle_topk_margin(ctypes.byref(cc), _ptr(x), _ptr(wr), t0, t1, _ptr(out), nthreads):
+    if lib.oracle_topk_margin(ctypes.byref(cc), _ptr(x), _ptr(wr), _ptr(bias), t0, t1, _ptr(out),
+                              nthreads):
         raise ValueError("oracle_topk_margin rejected its arguments")
     return out
 
@@ -164,10 +184,12 @@ def permute(c: Cfg, ids, lib: ctypes.CDLL | None = None):
 
 
 def forward(c: Cfg, x, wr, wg, wu, wd, shared=None, tokens=None, nthreads: int = 0,
-            lib: ctypes.CDLL | None = None, return_threads=False):
+            lib: ctypes.CDLL | None = None, return_threads=False, bias=None):
     """Layer output rows (float64) for ``tokens`` (default: all).  ``shared`` is
-    (W_shared_gate[h_s,d], W_shared_up[h_s,d], W_shared_down[d,h_s], w_s[d]) or None."""
+    (W_shared_gate[h_s,d], W_shared_up[h_s,d], W_shared_down[d,h_s], w_s[d]) or None;
+    ``bias`` the optional [E] float32 balance bias."""
     lib = lib or load()
+    bias = _bias(c, bias)
     sh = shared if shared is not None else (None, None, None, None)
     _check_dtype(c, x, wr, wg, wu, wd, *sh)
     if tokens is None:
@@ -176,8 +198,44 @@ def forward(c: Cfg, x, wr, wg, wu, wd, shared=None, tokens=None, nthreads: int =
     y = np.zeros((tokens.size, c.d), np.float64)
     cc = _ccfg(c)
     rc = lib.oracle_forward(ctypes.byref(cc), _ptr(x), _ptr(wr), _ptr(wg), _ptr(wu), _ptr(wd),
-                            _ptr(sh[0]), _ptr(sh[1]), _ptr(sh[2]), _ptr(sh[3]), _ptr(tokens),
-                            tokens.size, _ptr(y), nthreads)
+                            _ptr(sh[0]), _ptr(sh[1]), _ptr(sh[2]), _ptr(sh[3]), _ptr(bias),
+                            _ptr(tokens), tokens.size, _ptr(y), nthreads)
     if rc < 0:
         raise ValueError("oracle_forward rejected its arguments")
     return (y, rc) if return_threads else y
+
+
+def update_bias(c: Cfg, counts, lr: float, bias, lib: ctypes.CDLL | None = None):
+    """The balance bias after one step: bias + lr * sign(mean(counts) - counts), float32."""
+    lib = lib or load()
+    counts = np.ascontiguousarray(counts, dtype=np.int32).reshape(-1)
+    assert counts.size == c.E
+    b = _bias(c, bias)
+    out = np.zeros(c.E, np.float32)
+    if lib.oracle_update_bias(ctypes.byref(_ccfg(c)), _ptr(counts), ctypes.c_float(lr), _ptr(b), _ptr(out)):
+        raise ValueError("oracle_update_bias rejected its arguments")
+    return out
+
+
+def score_mean(c: Cfg, x, wr, nthreads: int = 0, lib: ctypes.CDLL | None = None):
+    """P_e: the mean over the T tokens of each expert's score (float64 [E])."""
+    lib = lib or load()
+    _check_dtype(c, x, wr)
+    out = np.zeros(c.E, np.float64)
+    if lib.oracle_score_mean(ctypes.byref(_ccfg(c)), _ptr(x), _ptr(wr), _ptr(out), nthreads):
+        raise ValueError("oracle_score_mean rejected its arguments")
+    return out
+
+
+def balance_loss(c: Cfg, counts, score_mean_, alpha: float, lib: ctypes.CDLL | None = None):
+    """(loss, f[E]): the Switch term alpha * E * sum_e f_e * P_e with f_e = counts[e] / T."""
+    lib = lib or load()
+    counts = np.ascontiguousarray(counts, dtype=np.int32).reshape(-1)
+    pm = np.ascontiguousarray(score_mean_, dtype=np.float64).reshape(-1)
+    assert counts.size == c.E and pm.size == c.E
+    frac = np.zeros(c.E, np.float64)
+    loss = np.zeros(1, np.float64)
+    if lib.oracle_balance_loss(ctypes.byref(_ccfg(c)), _ptr(counts), _ptr(pm), ctypes.c_double(alpha),
+                               _ptr(frac), _ptr(loss)):
+        raise ValueError("oracle_balance_loss rejected its arguments")
+    return float(loss[0]), frac

@@ -40,18 +40,28 @@ def _silu(u):
     return u * _sigmoid(u)
 
 
-def route_matrix(X, Wr, k, score="softmax", norm_topk=True):
-    """Routing as matrix operations.  Returns (ids[T,k], gates[T,k], G[T,E]) where
-    G is the dense gate matrix: G[t, ids[t,j]] = gates[t,j], zero elsewhere."""
-    T, E = X.shape[0], Wr.shape[0]
+def score_matrix(X, Wr, score="softmax"):
+    """The [T, E] score matrix: row-wise softmax of the logits X Wr^T, or their
+    element-wise sigmoid."""
     L = X @ Wr.T
     if score == "sigmoid":
-        S = _sigmoid(L)
-        key = S
-    else:
-        Z = np.exp(L - L.max(axis=1, keepdims=True))
-        S = Z / Z.sum(axis=1, keepdims=True)
-        key = L
+        return _sigmoid(L)
+    Z = np.exp(L - L.max(axis=1, keepdims=True))
+    return Z / Z.sum(axis=1, keepdims=True)
+
+
+def route_matrix(X, Wr, k, score="softmax", norm_topk=True, bias=None):
+    """Routing as matrix operations.  Returns (ids[T,k], gates[T,k], G[T,E]) where
+    G is the dense gate matrix: G[t, ids[t,j]] = gates[t,j], zero elsewhere.
+    With a balance bias [E] the selection key is the score plus the bias and the
+    gates stay the unbiased scores ("Small MoE Architecture, in depth",
+    SmallMoE.forward: topk of scores + balance_bias, gates gathered from scores)."""
+    T, E = X.shape[0], Wr.shape[0]
+    L = X @ Wr.T
+    S = score_matrix(X, Wr, score)
+    key = S if score == "sigmoid" else L
+    if bias is not None:
+        key = S + np.asarray(bias, np.float32).astype(np.float64)[None, :]
     # full sort by (key descending, expert index ascending)
     idx = np.broadcast_to(np.arange(E), (T, E))
     order = np.lexsort((idx, -key), axis=-1)
@@ -69,10 +79,10 @@ def dense_swiglu(X, Wg, Wu, Wd):
     return (_silu(X @ Wg.T) * (X @ Wu.T)) @ Wd.T
 
 
-def dense_forward(cfg, x, wr, wg, wu, wd, shared=None):
+def dense_forward(cfg, x, wr, wg, wu, wd, shared=None, bias=None):
     """All experts on all tokens, masked by the gate matrix.  Returns (y[T,d], ids, gates)."""
     X, Wr = to_f64(x), to_f64(wr)
-    ids, gates, G = route_matrix(X, Wr, cfg.k, cfg.score, cfg.norm_topk)
+    ids, gates, G = route_matrix(X, Wr, cfg.k, cfg.score, cfg.norm_topk, bias)
     WG, WU, WD = to_f64(wg), to_f64(wu), to_f64(wd)
     Y = np.zeros((cfg.T, cfg.d))
     for e in range(cfg.E):
@@ -83,10 +93,10 @@ def dense_forward(cfg, x, wr, wg, wu, wd, shared=None):
     return Y, ids, gates
 
 
-def loop_over_experts_forward(cfg, x, wr, wg, wu, wd, shared=None):
+def loop_over_experts_forward(cfg, x, wr, wg, wu, wd, shared=None, bias=None):
     """Per-expert gather / batch / index_add.  Returns y[T,d]."""
     X, Wr = to_f64(x), to_f64(wr)
-    ids, gates, _ = route_matrix(X, Wr, cfg.k, cfg.score, cfg.norm_topk)
+    ids, gates, _ = route_matrix(X, Wr, cfg.k, cfg.score, cfg.norm_topk, bias)
     WG, WU, WD = to_f64(wg), to_f64(wu), to_f64(wd)
     out = np.zeros((cfg.T, cfg.d))
     if shared is not None and cfg.h_shared > 0:

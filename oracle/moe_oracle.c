@@ -21,6 +21,13 @@
  *   permute    "Tutorial 11", section 3 "Expert Computation", Step 1 (sort the
  *              flattened expert ids; the grouped order) and "Small MoE
  *              Architecture, in depth" (per-expert counts by bincount).
+ *   balance    "Small MoE Architecture, in depth", SmallMoE.forward and the
+ *              paragraph on auxiliary-loss-free balancing after it (a
+ *              per-expert bias added to the scores only when choosing the
+ *              top k, and its update from the per-expert load after a step);
+ *              "Mixture-of-Experts -- more capacity per byte of weight",
+ *              section "What's wired today" (the Switch load-balancing term
+ *              alpha * N * sum_e f_e * P_e and the statistics it needs).
  *   forward    "Tutorial 11", section 3 Steps 2-3 and section 4 "The Complete
  *              MoE Layer" (per-row expert SwiGLU, weighted sum over the k
  *              selected experts); the SwiGLU expert is down(silu(gate x) *
@@ -38,7 +45,13 @@
  *     kept probabilities; that configuration is {softmax, norm_topk = 1}.
  *   - the shared expert's gate is sigmoid(w_s . x); its logit takes no part
  *     in the top-k selection.
- *   - silu(u) = u / (1 + exp(-u)); no biases anywhere.
+ *   - silu(u) = u / (1 + exp(-u)); no biases in any linear layer.
+ *   - the balance bias is added to the score s_e (softmax probability or
+ *     sigmoid score, whichever the layer uses) to form the selection key;
+ *     the gates are gathered from the unbiased scores.
+ *   - the Switch statistics: f_e = counts[e] / T, the fraction of the T
+ *     tokens dispatched to expert e, and P_e = the mean over the T tokens of
+ *     the score s_e (the full score row, before selection).
  *
  * Pins: this file is checked, not trusted -- see tests/test_oracle_pins.py
  * (the route_topk worked example, a dense all-experts formulation, a
@@ -105,11 +118,19 @@ static void router_logits(const oracle_cfg *c, const void *x, const void *wr,
     }
 }
 
-/* Selection keys: logits under softmax (monotone map), sigmoid otherwise. */
-static void selection_keys(const oracle_cfg *c, const double *logits, double *keys)
+/* Selection keys.  Without a balance bias: the logit under softmax (a
+ * monotone map, so ranking logits ranks probabilities) and the sigmoid score
+ * under sigmoid.  With a bias (SmallMoE.forward: topk of scores +
+ * balance_bias): key_e = s_e + bias_e, the score plus the bias. */
+static void selection_keys(const oracle_cfg *c, const double *logits, const double *scores,
+                           const float *bias, double *keys)
 {
-    for (int32_t e = 0; e < c->E; ++e)
-        keys[e] = (c->score == ORACLE_SIGMOID) ? sigmoid(logits[e]) : logits[e];
+    for (int32_t e = 0; e < c->E; ++e) {
+        if (bias)
+            keys[e] = scores[e] + (double)bias[e];
+        else
+            keys[e] = (c->score == ORACLE_SIGMOID) ? sigmoid(logits[e]) : logits[e];
+    }
 }
 
 /* The k best experts, best first: repeatedly take the largest key not yet
@@ -148,16 +169,17 @@ static void expert_scores(const oracle_cfg *c, const double *logits, double *sco
 
 /* Routes one token: ids[0..k), gates[0..k), the full score row and the
  * shared-expert gate.  Gates are the selected scores ("Tutorial 11" section 2
- * step 4), divided by their sum when norm_topk is set (step 5; the worked
- * example under "Why Normalize Selected Probabilities?"). */
+ * step 4; with a balance bias still the unbiased scores, SmallMoE.forward),
+ * divided by their sum when norm_topk is set (step 5; the worked example
+ * under "Why Normalize Selected Probabilities?").  bias may be NULL. */
 static void route_one(const oracle_cfg *c, const void *x, const void *wr, const void *w_sg,
-                      int64_t t, double *logits, double *keys, double *scores, char *taken,
-                      int32_t *ids, double *gates, double *shared_gate)
+                      const float *bias, int64_t t, double *logits, double *keys, double *scores,
+                      char *taken, int32_t *ids, double *gates, double *shared_gate)
 {
     router_logits(c, x, wr, t, logits);
-    selection_keys(c, logits, keys);
-    select_topk(c, keys, taken, ids);
     expert_scores(c, logits, scores);
+    selection_keys(c, logits, scores, bias, keys);
+    select_topk(c, keys, taken, ids);
     double sum = 0.0;
     for (int32_t j = 0; j < c->k; ++j) {
         gates[j] = scores[ids[j]];
@@ -190,10 +212,11 @@ static int nthreads_used(int requested)
 
 /* Routes tokens [t0, t1).  ids and gates are [T, k] (indexed by absolute
  * token), probs is an optional [T, E] score matrix, shared_gate an optional
- * [T] vector.  Returns 0 on success, -1 on a bad argument. */
+ * [T] vector, bias an optional [E] fp32 balance bias.  Returns 0 on success,
+ * -1 on a bad argument. */
 int oracle_route(const oracle_cfg *c, const void *x, const void *wr, const void *w_sg,
-                 int64_t t0, int64_t t1, int32_t *ids, double *gates, double *probs,
-                 double *shared_gate, int nthreads)
+                 const float *bias, int64_t t0, int64_t t1, int32_t *ids, double *gates,
+                 double *probs, double *shared_gate, int nthreads)
 {
     if (!cfg_ok(c) || !x || !wr || !ids || !gates || t0 < 0 || t1 > c->T || t0 > t1) return -1;
     int nt = nthreads_used(nthreads);
@@ -209,7 +232,7 @@ int oracle_route(const oracle_cfg *c, const void *x, const void *wr, const void 
             double *keys = logits + c->E, *scores = logits + 2 * c->E;
 #pragma omp for schedule(dynamic, 16)
             for (int64_t t = t0; t < t1; ++t) {
-                route_one(c, x, wr, w_sg, t, logits, keys, scores, taken, ids + t * c->k,
+                route_one(c, x, wr, w_sg, bias, t, logits, keys, scores, taken, ids + t * c->k,
                           gates + t * c->k, shared_gate ? shared_gate + t : NULL);
                 if (probs)
                     for (int32_t e = 0; e < c->E; ++e) probs[t * c->E + e] = scores[e];
@@ -222,11 +245,12 @@ int oracle_route(const oracle_cfg *c, const void *x, const void *wr, const void 
 }
 
 /* Margin of the selection for tokens [t0, t1): the smallest gap between
- * adjacent keys among the top min(k + 1, E) keys in descending order.  A
+ * adjacent keys (with the balance bias when given) among the top
+ * min(k + 1, E) keys in descending order.  A
  * margin above the numerical error of a faster implementation means that it
  * must find the same experts in the same slot order. */
-int oracle_topk_margin(const oracle_cfg *c, const void *x, const void *wr, int64_t t0, int64_t t1,
-                       double *margin, int nthreads)
+int oracle_topk_margin(const oracle_cfg *c, const void *x, const void *wr, const float *bias,
+                       int64_t t0, int64_t t1, double *margin, int nthreads)
 {
     if (!cfg_ok(c) || !x || !wr || !margin || t0 < 0 || t1 > c->T || t0 > t1) return -1;
     int nt = nthreads_used(nthreads);
@@ -234,20 +258,21 @@ int oracle_topk_margin(const oracle_cfg *c, const void *x, const void *wr, int64
     int bad = 0;
 #pragma omp parallel num_threads(nt)
     {
-        double *logits = malloc(sizeof(double) * (size_t)c->E * 2);
+        double *logits = malloc(sizeof(double) * (size_t)c->E * 3);
         char *taken = malloc((size_t)c->E);
         int32_t *order = malloc(sizeof(int32_t) * (size_t)m);
         if (!logits || !taken || !order) {
 #pragma omp atomic write
             bad = 1;
         } else {
-            double *keys = logits + c->E;
+            double *keys = logits + c->E, *scores = logits + 2 * c->E;
             oracle_cfg cm = *c;
             cm.k = m;
 #pragma omp for schedule(dynamic, 16)
             for (int64_t t = t0; t < t1; ++t) {
                 router_logits(c, x, wr, t, logits);
-                selection_keys(c, logits, keys);
+                expert_scores(c, logits, scores);
+                selection_keys(c, logits, scores, bias, keys);
                 select_topk(&cm, keys, taken, order);
                 double g = INFINITY;
                 for (int32_t j = 0; j + 1 < m; ++j) {
@@ -320,12 +345,12 @@ static void swiglu_expert_add(const oracle_cfg *c, const void *x, int64_t t, con
  * output row, y = sum_j gate_j * expert_{ids_j}(x) (+ sigmoid(w_s . x) *
  * shared(x) when h_shared > 0).  W_gate/W_up are [E, h, d], W_down [E, d, h];
  * the shared expert's weights are [h_shared, d], [h_shared, d], [d, h_shared]
- * and w_s is [d].  Routing is recomputed per token, so any subset of tokens
+ * and w_s is [d]; bias is the optional [E] balance bias.  Routing is recomputed per token, so any subset of tokens
  * can be evaluated on its own.  Returns the number of threads used, or -1. */
 int oracle_forward(const oracle_cfg *c, const void *x, const void *wr, const void *wg,
                    const void *wu, const void *wd, const void *sh_g, const void *sh_u,
-                   const void *sh_d, const void *w_sg, const int64_t *tokens, int64_t n_tokens,
-                   double *y, int nthreads)
+                   const void *sh_d, const void *w_sg, const float *bias, const int64_t *tokens,
+                   int64_t n_tokens, double *y, int nthreads)
 {
     if (!cfg_ok(c) || !x || !wr || !wg || !wu || !wd || !tokens || !y || n_tokens < 0) return -1;
     if (c->h_shared > 0 && (!sh_g || !sh_u || !sh_d || !w_sg)) return -1;
@@ -349,7 +374,7 @@ int oracle_forward(const oracle_cfg *c, const void *x, const void *wr, const voi
             for (int64_t i = 0; i < n_tokens; ++i) {
                 int64_t t = tokens[i];
                 double sg = 0.0;
-                route_one(c, x, wr, w_sg, t, logits, keys, scores, taken, ids, gates, &sg);
+                route_one(c, x, wr, w_sg, bias, t, logits, keys, scores, taken, ids, gates, &sg);
                 double *out = y + i * c->d;
                 for (int32_t q = 0; q < c->d; ++q) out[q] = 0.0;
                 for (int32_t j = 0; j < c->k; ++j) {
@@ -366,4 +391,88 @@ int oracle_forward(const oracle_cfg *c, const void *x, const void *wr, const voi
         free(ids);
     }
     return bad ? -1 : nt;
+}
+
+/* Balance-bias update after a step ("Small MoE Architecture, in depth",
+ * SmallMoE.forward in training, and the paragraph on auxiliary-loss-free
+ * balancing after it): the load of expert e is counts[e] (the bincount of
+ * the chosen ids), and bias_e moves by lr * sign(mean load - load_e): down by
+ * lr for an expert above the mean load, up by lr below it, unchanged at it.
+ * The bias is a stored fp32 buffer: each new value is formed in double and
+ * rounded once to fp32.  bias_out may alias bias_in. */
+int oracle_update_bias(const oracle_cfg *c, const int32_t *counts, float lr, const float *bias_in,
+                       float *bias_out)
+{
+    if (!cfg_ok(c) || !counts || !bias_in || !bias_out) return -1;
+    double total = 0.0;
+    for (int32_t e = 0; e < c->E; ++e) total += (double)counts[e];
+    double mean = total / (double)c->E;
+    for (int32_t e = 0; e < c->E; ++e) {
+        double load = (double)counts[e];
+        double sign = 0.0;
+        if (mean > load) sign = 1.0;
+        if (mean < load) sign = -1.0;
+        bias_out[e] = (float)((double)bias_in[e] + (double)lr * sign);
+    }
+    return 0;
+}
+
+/* Mean score per expert over the T tokens, P_e = (1/T) sum_t s_e(t), with
+ * s(t) the full score row of token t (softmax probabilities or sigmoid
+ * scores, before selection): the router-probability statistic of the Switch
+ * load-balancing term ("Mixture-of-Experts -- more capacity per byte of
+ * weight", "What's wired today").  Scores are formed per token in parallel
+ * and summed over tokens in increasing t.  T = 0 gives zeros. */
+int oracle_score_mean(const oracle_cfg *c, const void *x, const void *wr, double *mean, int nthreads)
+{
+    if (!cfg_ok(c) || !x || !wr || !mean) return -1;
+    for (int32_t e = 0; e < c->E; ++e) mean[e] = 0.0;
+    if (c->T == 0) return 0;
+    double *rows = malloc(sizeof(double) * (size_t)c->T * (size_t)c->E);
+    if (!rows) return -1;
+    int nt = nthreads_used(nthreads);
+    int bad = 0;
+#pragma omp parallel num_threads(nt)
+    {
+        double *logits = malloc(sizeof(double) * (size_t)c->E);
+        if (!logits) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = 0; t < c->T; ++t) {
+                router_logits(c, x, wr, t, logits);
+                expert_scores(c, logits, rows + t * c->E);
+            }
+        }
+        free(logits);
+    }
+    if (!bad) {
+        for (int32_t e = 0; e < c->E; ++e) {
+            double s = 0.0;
+            for (int64_t t = 0; t < c->T; ++t) s += rows[t * c->E + e];
+            mean[e] = s / (double)c->T;
+        }
+    }
+    free(rows);
+    return bad ? -1 : 0;
+}
+
+/* The Switch load-balancing term ("Mixture-of-Experts -- more capacity per
+ * byte of weight", "What's wired today"): loss = alpha * N * sum_e f_e * P_e
+ * with N = E experts, f_e = counts[e] / T (the fraction of the T tokens
+ * dispatched to expert e) and P_e = score_mean[e].  frac may be NULL.  T = 0
+ * gives f = 0 and loss = 0. */
+int oracle_balance_loss(const oracle_cfg *c, const int32_t *counts, const double *score_mean,
+                        double alpha, double *frac, double *loss)
+{
+    if (!cfg_ok(c) || !counts || !score_mean || !loss) return -1;
+    double sum = 0.0;
+    for (int32_t e = 0; e < c->E; ++e) {
+        double f = c->T > 0 ? (double)counts[e] / (double)c->T : 0.0;
+        if (frac) frac[e] = f;
+        sum += f * score_mean[e];
+    }
+    *loss = alpha * (double)c->E * sum;
+    return 0;
 }

@@ -38,6 +38,15 @@ MUTANTS = [
     ("selection_by_raw_logit_under_sigmoid",
      "keys[e] = (c->score == ORACLE_SIGMOID) ? sigmoid(logits[e]) : logits[e];",
      "keys[e] = (c->score == ORACLE_SIGMOID) ? -logits[e] : logits[e];"),
+    ("balance_bias_ignored", "if (bias)\n            keys[e] = scores[e]", "if (0 && bias)\n            keys[e] = scores[e]"),
+    ("balance_bias_subtracted", "keys[e] = scores[e] + (double)bias[e];", "keys[e] = scores[e] - (double)bias[e];"),
+    ("balance_bias_on_logits", "keys[e] = scores[e] + (double)bias[e];", "keys[e] = logits[e] + (double)bias[e];"),
+    ("balance_bias_leaks_into_gates", "gates[j] = scores[ids[j]];", "gates[j] = keys[ids[j]];"),
+    ("bias_update_sign", "if (mean > load) sign = 1.0;", "if (mean > load) sign = -1.0;"),
+    ("bias_update_mean_over_tokens", "double mean = total / (double)c->E;", "double mean = total / (double)c->T;"),
+    ("score_mean_not_divided", "mean[e] = s / (double)c->T;", "mean[e] = s;"),
+    ("switch_loss_without_N", "*loss = alpha * (double)c->E * sum;", "*loss = alpha * sum;"),
+    ("switch_frac_over_assignments", "(double)counts[e] / (double)c->T", "(double)counts[e] / (double)(c->T * c->k)"),
 ]
 
 

@@ -10,7 +10,15 @@
   loop-over-experts index_add formulation (numpy, float64, matrix ops);
 * the E = 1, k = 1 special case, which is the textbook dense SwiGLU FFN;
 * invariants: distinct ids, counts summing to T*k, a stable permutation
-  (numpy's stable argsort), gates summing to one under renormalisation.
+  (numpy's stable argsort), gates summing to one under renormalisation;
+* selection with a balance bias and the bias update: hand-computed examples
+  of "Small MoE Architecture, in depth" ("A small MoE layer in PyTorch"),
+  brute force over k-subsets of the biased keys, and the dense and
+  loop-over-experts formulations with the bias;
+* the Switch statistics ("Mixture-of-Experts -- more capacity per byte of
+  weight", "What's wired today"): a hand-computed example, the uniform router
+  (P_e = 1/E) and uniform load (loss = alpha * k) closed forms, and the mean
+  of the numpy score matrix.
 """
 import itertools
 import math
@@ -326,9 +334,144 @@ def test_oracle_rejects_bad_arguments():
         oracle.permute(c, np.array([3], np.int32))                 # id out of range
 
 
+# ---------------------------------------------------------------- balance bias and Switch statistics
+
+def _bias_example(norm=True, bias=True):
+    g = _golden("balance_bias_example.txt")
+    s = np.array([float(v) for v in g["scores"]])
+    E, d = s.size, 4
+    c = oracle.Cfg(T=1, d=d, E=E, h=8, k=int(g["top_k"][0]), norm_topk=norm, score="sigmoid", dtype="f32")
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0                                              # logit_e = Wr[e, 0]
+    wr = np.zeros((E, d), np.float32)
+    wr[:, 0] = np.log(s / (1.0 - s)).astype(np.float32)       # sigmoid(logit(s)) = s
+    b = np.array([float(v) for v in g["bias"]], np.float32) if bias else None
+    return g, c, x, wr, b
+
+
+def check_balance_bias_example():
+    g, c, x, wr, b = _bias_example()
+    ids, gates, probs, _ = oracle.route(c, x, wr, want_probs=True, bias=b, lib=lib())
+    np.testing.assert_array_equal(ids[0], [int(v) for v in g["ids"]])
+    np.testing.assert_allclose(gates[0], [float(v) for v in g["gates_normalised"]], atol=1e-6)
+    np.testing.assert_allclose(probs[0], [float(v) for v in g["scores"]], atol=1e-6)   # scores stay unbiased
+    _, c0, _, _, _ = _bias_example(norm=False)
+    ids0, gates0, _, _ = oracle.route(c0, x, wr, bias=b, lib=lib())
+    np.testing.assert_array_equal(ids0[0], ids[0])
+    np.testing.assert_allclose(gates0[0], [float(v) for v in g["gates_raw"]], atol=1e-6)
+    idsu, gatesu, _, _ = oracle.route(c, x, wr, lib=lib())
+    np.testing.assert_array_equal(idsu[0], [int(v) for v in g["ids_unbiased"]])
+    np.testing.assert_allclose(gatesu[0], [float(v) for v in g["gates_unbiased_normalised"]], atol=1e-6)
+    # the margin sees the biased keys: 0.95 - 0.9 and 0.9 - 0.8 -> 0.05
+    m = oracle.topk_margin(c, x, wr, bias=b, lib=lib())
+    np.testing.assert_allclose(m, [0.05], atol=1e-6)
+
+
+def test_balance_bias_example():
+    check_balance_bias_example()
+
+
+def check_biased_routing_brute_force_and_formulations():
+    rng = np.random.default_rng(21)
+    for score in ("sigmoid", "softmax"):
+        for norm in (True, False):
+            c, x, wr = _random_case(rng, 30, 12, 9, 3, score=score, norm=norm)
+            # biases of the size of the score spread, so they change many choices
+            b = (rng.standard_normal(9) * (0.3 if score == "sigmoid" else 0.1)).astype(np.float32)
+            ids, gates, _, _ = oracle.route(c, x, wr, bias=b, lib=lib())
+            ids_plain, _, _, _ = oracle.route(c, x, wr, lib=lib())
+            assert (ids != ids_plain).any(), "the bias should change some selections"
+            S = dense.score_matrix(dense.to_f64(x), dense.to_f64(wr), score)
+            key = S + b.astype(np.float64)[None, :]
+            for t in range(c.T):
+                best = max(itertools.combinations(range(c.E), c.k), key=lambda s_: key[t, list(s_)].sum())
+                assert set(ids[t].tolist()) == set(best)
+                assert all(key[t, ids[t, j]] > key[t, ids[t, j + 1]] for j in range(c.k - 1))
+                g = S[t, ids[t]]
+                np.testing.assert_allclose(gates[t], g / g.sum() if norm else g, rtol=1e-13, atol=1e-15)
+    # the whole layer with a bias: C loop == dense masking == loop over experts
+    w, a = _small_layer((27, 16, 7, 12, 2, "sigmoid", True, 12, "bf16"), 300)
+    c = ocfg(w)
+    b = (np.random.default_rng(22).standard_normal(w.E) * 0.3).astype(np.float32)
+    y = oracle.forward(c, a.x, a.wr, a.wg, a.wu, a.wd, a.shared, bias=b, lib=lib())
+    y_dense, ids_d, _ = dense.dense_forward(c, a.x, a.wr, a.wg, a.wu, a.wd, a.shared, bias=b)
+    y_loop = dense.loop_over_experts_forward(c, a.x, a.wr, a.wg, a.wu, a.wd, a.shared, bias=b)
+    scale = np.abs(y_dense).max()
+    np.testing.assert_allclose(y, y_dense, rtol=0, atol=1e-12 * scale)
+    np.testing.assert_allclose(y, y_loop, rtol=0, atol=1e-12 * scale)
+    ids, _, _, _ = oracle.route(c, a.x, a.wr, a.w_sg, bias=b, lib=lib())
+    np.testing.assert_array_equal(ids, ids_d)
+
+
+def test_biased_routing_brute_force_and_formulations():
+    check_biased_routing_brute_force_and_formulations()
+
+
+def check_bias_update_example():
+    g = _golden("bias_update_example.txt")
+    E, T, k = int(g["E"][0]), int(g["T"][0]), int(g["top_k"][0])
+    c = oracle.Cfg(T=T, d=8, E=E, h=8, k=k)
+    counts = np.array([int(v) for v in g["counts"]], np.int32)
+    assert counts.sum() == T * k
+    before = np.array([float(v) for v in g["bias_before"]], np.float32)
+    after = oracle.update_bias(c, counts, float(g["lr"][0]), before, lib=lib())
+    np.testing.assert_array_equal(after, np.array([float(v) for v in g["bias_after"]], np.float32))
+    # an exactly balanced load leaves the bias unchanged; a second step moves it again
+    np.testing.assert_array_equal(oracle.update_bias(c, np.full(E, 3, np.int32), 0.001, before, lib=lib()),
+                                  before)
+    twice = oracle.update_bias(c, counts, 0.001, after, lib=lib())
+    np.testing.assert_allclose(twice - before, [-0.002, 0.002, 0.0, 0.0], atol=1e-9)
+
+
+def test_bias_update_example():
+    check_bias_update_example()
+
+
+def check_switch_statistics():
+    g = _golden("switch_balance_example.txt")
+    E, T, k = int(g["E"][0]), int(g["T"][0]), int(g["top_k"][0])
+    c = oracle.Cfg(T=T, d=T, E=E, h=8, k=k, norm_topk=False, dtype="f32")
+    x = np.eye(T, dtype=np.float32)                            # token t reads router column t
+    wr = np.zeros((E, T), np.float32)
+    for t in range(T):
+        wr[:, t] = np.log([float(v) for v in g[f"probs_t{t}"]]).astype(np.float32)
+    ids, _, _, _ = oracle.route(c, x, wr, lib=lib())
+    counts, _, _, _ = oracle.permute(c, ids, lib=lib())
+    np.testing.assert_array_equal(counts, [int(v) for v in g["counts"]])
+    P = oracle.score_mean(c, x, wr, lib=lib())
+    np.testing.assert_allclose(P, [float(v) for v in g["P"]], atol=1e-7)
+    loss, f = oracle.balance_loss(c, counts, P, float(g["alpha"][0]), lib=lib())
+    np.testing.assert_allclose(f, [float(v) for v in g["f"]], rtol=0, atol=0)
+    np.testing.assert_allclose(loss, float(g["loss"][0]), rtol=1e-6)
+    # closed forms: a zero router gives every expert the score 1/E (softmax) or
+    # 1/2 (sigmoid); a uniform load then gives alpha * k
+    for score, p in (("softmax", 1 / 8), ("sigmoid", 0.5)):
+        c8 = oracle.Cfg(T=16, d=4, E=8, h=8, k=2, score=score, dtype="f32")
+        xz = np.random.default_rng(3).standard_normal((16, 4)).astype(np.float32)
+        P8 = oracle.score_mean(c8, xz, np.zeros((8, 4), np.float32), lib=lib())
+        np.testing.assert_allclose(P8, np.full(8, p), rtol=1e-15)
+    c8 = oracle.Cfg(T=16, d=4, E=8, h=8, k=2, dtype="f32")
+    loss8, f8 = oracle.balance_loss(c8, np.full(8, 4, np.int32), np.full(8, 1 / 8), 0.01, lib=lib())
+    np.testing.assert_allclose(f8, np.full(8, 0.25), rtol=0)
+    np.testing.assert_allclose(loss8, 0.01 * 2, rtol=1e-15)
+    # random router: the mean of the score matrix
+    rng = np.random.default_rng(23)
+    for score in ("softmax", "sigmoid"):
+        cr, xr, wrr = _random_case(rng, 40, 10, 6, 2, score=score, dtype="bf16")
+        Pr = oracle.score_mean(cr, xr, wrr, lib=lib())
+        S = dense.score_matrix(dense.to_f64(xr), dense.to_f64(wrr), score)
+        np.testing.assert_allclose(Pr, S.mean(axis=0), rtol=1e-13)
+
+
+def test_switch_statistics():
+    check_switch_statistics()
+
+
 # The checks the mutation tests run against deliberately broken builds.
 PIN_CHECKS = [check_worked_example, check_routing_brute_force, check_routing_vs_full_sort_and_ties,
               check_margin, check_dense_formulation, check_tiny_workload, check_loop_over_experts,
-              check_single_expert_is_dense_swiglu, check_permutation_invariants]
+              check_single_expert_is_dense_swiglu, check_permutation_invariants, check_balance_bias_example,
+              check_biased_routing_brute_force_and_formulations, check_bias_update_example,
+              check_switch_statistics]
 
 assert math.isclose(64 ** (1 / 3), 4.0)
