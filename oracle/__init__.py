@@ -35,7 +35,7 @@ _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 SOFTMAX, SIGMOID = 0, 1
-BF16, F32 = 0, 1
+BF16, F32, F64 = 0, 1, 2
 
 
 @dataclass(frozen=True)
@@ -49,7 +49,7 @@ class Cfg:
     norm_topk: bool = True
     score: str = "softmax"      # "softmax" | "sigmoid"
     h_shared: int = 0
-    dtype: str = "bf16"         # "bf16" | "f32"
+    dtype: str = "bf16"         # "bf16" | "f32" | "f64" (f64: pins only)
 
 
 class _CCfg(ctypes.Structure):
@@ -61,7 +61,7 @@ class _CCfg(ctypes.Structure):
 def _ccfg(c: Cfg) -> _CCfg:
     return _CCfg(c.T, c.d, c.E, c.h, c.k, int(bool(c.norm_topk)),
                  SIGMOID if c.score == "sigmoid" else SOFTMAX, c.h_shared,
-                 F32 if c.dtype == "f32" else BF16)
+                 {"f32": F32, "f64": F64}.get(c.dtype, BF16))
 
 
 def build(force: bool = False, source: str = _SRC, output: str = _LIB) -> str:
@@ -102,6 +102,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.oracle_score_mean.restype = ctypes.c_int
     lib.oracle_balance_loss.argtypes = [ctypes.POINTER(_CCfg), P, P, ctypes.c_double, P, P]
     lib.oracle_balance_loss.restype = ctypes.c_int
+    lib.oracle_backward.argtypes = [ctypes.POINTER(_CCfg)] + [P] * 20 + [ctypes.c_int]
+    lib.oracle_backward.restype = ctypes.c_int
     _lib_cache[path] = lib
     return lib
 
@@ -114,7 +116,7 @@ def _ptr(a):
 
 
 def _check_dtype(c: Cfg, *arrays):
-    want = np.float32 if c.dtype == "f32" else np.uint16
+    want = {"f32": np.float32, "f64": np.float64}.get(c.dtype, np.uint16)
     for a in arrays:
         if a is not None and a.dtype != want:
             raise TypeError(f"oracle expects {np.dtype(want)} arrays for dtype {c.dtype}, got {a.dtype}")
@@ -239,3 +241,27 @@ def balance_loss(c: Cfg, counts, score_mean_, alpha: float, lib: ctypes.CDLL | N
                                _ptr(frac), _ptr(loss)):
         raise ValueError("oracle_balance_loss rejected its arguments")
     return float(loss[0]), frac
+
+
+def backward(c: Cfg, x, wr, wg, wu, wd, dy, shared=None, bias=None, nthreads: int = 0,
+             lib: ctypes.CDLL | None = None) -> dict:
+    """Gradients (float64) of the layer given the upstream gradient dy[T, d] (the
+    layer's dtype): dx, dw_router, dw_gate, dw_up, dw_down and, with a shared
+    expert, dsh_gate, dsh_up, dsh_down, dw_shared_gate."""
+    lib = lib or load()
+    sh = shared if shared is not None else (None, None, None, None)
+    _check_dtype(c, x, wr, wg, wu, wd, dy, *sh)
+    bias = _bias(c, bias)
+    g = {"dx": np.zeros((c.T, c.d)), "dw_router": np.zeros((c.E, c.d)), "dw_gate": np.zeros((c.E, c.h, c.d)),
+         "dw_up": np.zeros((c.E, c.h, c.d)), "dw_down": np.zeros((c.E, c.d, c.h))}
+    if c.h_shared > 0:
+        g.update(dsh_gate=np.zeros((c.h_shared, c.d)), dsh_up=np.zeros((c.h_shared, c.d)),
+                 dsh_down=np.zeros((c.d, c.h_shared)), dw_shared_gate=np.zeros(c.d))
+    rc = lib.oracle_backward(ctypes.byref(_ccfg(c)), _ptr(x), _ptr(wr), _ptr(wg), _ptr(wu), _ptr(wd),
+                             _ptr(sh[0]), _ptr(sh[1]), _ptr(sh[2]), _ptr(sh[3]), _ptr(bias), _ptr(dy),
+                             _ptr(g["dx"]), _ptr(g["dw_router"]), _ptr(g["dw_gate"]), _ptr(g["dw_up"]),
+                             _ptr(g["dw_down"]), _ptr(g.get("dsh_gate")), _ptr(g.get("dsh_up")),
+                             _ptr(g.get("dsh_down")), _ptr(g.get("dw_shared_gate")), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_backward rejected its arguments")
+    return g

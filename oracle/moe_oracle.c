@@ -65,7 +65,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_BF16 = 0, ORACLE_F32 = 1 };
+enum { ORACLE_BF16 = 0, ORACLE_F32 = 1, ORACLE_F64 = 2 };
 enum { ORACLE_SOFTMAX = 0, ORACLE_SIGMOID = 1 };
 
 /* Layer shape and options.  T tokens of width d, E routed experts of hidden
@@ -79,9 +79,12 @@ typedef struct {
     int32_t dtype;
 } oracle_cfg;
 
-/* Element i of a stored tensor, widened exactly to double. */
+/* Element i of a stored tensor, widened exactly to double.  (float64 inputs
+ * exist only so that the pins can difference the layer finely.) */
 static double elem(const void *base, int64_t i, int32_t dtype)
 {
+    if (dtype == ORACLE_F64)
+        return ((const double *)base)[i];
     if (dtype == ORACLE_F32)
         return (double)((const float *)base)[i];
     uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
@@ -94,12 +97,19 @@ static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
 
 static double silu(double u) { return u / (1.0 + exp(-u)); }
 
+/* d silu(u) / du = sigmoid(u) * (1 + u * (1 - sigmoid(u))). */
+static double dsilu(double u)
+{
+    double s = sigmoid(u);
+    return s * (1.0 + u * (1.0 - s));
+}
+
 static int cfg_ok(const oracle_cfg *c)
 {
     if (!c || c->T < 0 || c->d < 1 || c->E < 1 || c->h < 1) return 0;
     if (c->k < 1 || c->k > c->E) return 0;
     if (c->score != ORACLE_SOFTMAX && c->score != ORACLE_SIGMOID) return 0;
-    if (c->dtype != ORACLE_BF16 && c->dtype != ORACLE_F32) return 0;
+    if (c->dtype != ORACLE_BF16 && c->dtype != ORACLE_F32 && c->dtype != ORACLE_F64) return 0;
     if (c->h_shared < 0) return 0;
     return 1;
 }
@@ -475,4 +485,248 @@ int oracle_balance_loss(const oracle_cfg *c, const int32_t *counts, const double
     }
     *loss = alpha * (double)c->E * sum;
     return 0;
+}
+
+/* ------------------------------------------------------------------ backward
+ *
+ * The gradient of the layer, written out by the chain rule through the same
+ * steps as the forward pass above (the pages train this layer -- "Small
+ * models, sparse experts", "Dispatch decides everything" reports training
+ * tokens/s; "Small MoE Architecture, in depth", SmallMoE -- but print no
+ * backward; the backward of a composition of these plain steps has one
+ * definition).  Given the upstream gradient dy[T, d] of the output y:
+ *
+ *   expert j of token t (e = ids_j, gate g_j):
+ *     u = Wg[e] x, v = Wu[e] x, a = silu(u) * v, o = Wd[e] a
+ *     r  = Wd[e]^T dy            (dy . o = r . a, so dL/dg_j = r . a)
+ *     da = g_j r, du = da * v * silu'(u), dv = da * silu(u)
+ *     dx += Wg[e]^T du + Wu[e]^T dv
+ *     dWd[e] += g_j dy a^T, dWg[e] += du x^T, dWu[e] += dv x^T
+ *   shared expert (gate sg = sigmoid(w_s . x)): the same with sg in place of
+ *     g_j, and dL/dsg = r_s . a_s, so dl_s = dL/dsg * sg * (1 - sg),
+ *     dw_s += dl_s x, dx += dl_s w_s
+ *   router: the kept raw scores q_j = s_{ids_j}; with renormalisation
+ *     g_j = q_j / Q (Q = sum q), dq_j = (dg_j - sum_i dg_i g_i) / Q, else
+ *     dq_j = dg_j; ds_{ids_j} = dq_j and 0 elsewhere; softmax:
+ *     dl_e = s_e (ds_e - sum_e' s_e' ds_e'), sigmoid: dl_e = ds_e s_e (1 - s_e);
+ *     dWr[e] += dl_e x, dx += sum_e dl_e Wr[e]
+ *
+ * The top-k selection (with or without the balance bias) is piecewise
+ * constant, so it passes no gradient; the bias gets none.
+ */
+
+/* Gradient of the router logits of one token from the gradients dg of its k
+ * gates (ids, gates, the full score row as route_one leaves them). */
+static void router_backward(const oracle_cfg *c, const double *scores, const int32_t *ids,
+                            const double *gates, const double *dg, double *ds, double *dl)
+{
+    double q = 0.0, dot = 0.0;
+    for (int32_t j = 0; j < c->k; ++j) {
+        q += scores[ids[j]];
+        dot += dg[j] * gates[j];
+    }
+    for (int32_t e = 0; e < c->E; ++e) ds[e] = 0.0;
+    for (int32_t j = 0; j < c->k; ++j)
+        ds[ids[j]] = c->norm_topk ? (dg[j] - dot) / q : dg[j];
+    if (c->score == ORACLE_SIGMOID) {
+        for (int32_t e = 0; e < c->E; ++e) dl[e] = ds[e] * scores[e] * (1.0 - scores[e]);
+        return;
+    }
+    double sd = 0.0;
+    for (int32_t e = 0; e < c->E; ++e) sd += scores[e] * ds[e];
+    for (int32_t e = 0; e < c->E; ++e) dl[e] = scores[e] * (ds[e] - sd);
+}
+
+/* u, v and a = silu(u) * v of one expert (rows w_off_in.. of Wg, Wu) on token t. */
+static void expert_hidden(const oracle_cfg *c, const void *x, int64_t t, const void *wg, const void *wu,
+                          int64_t w_off_in, int32_t hid, double *u, double *v, double *a)
+{
+    for (int32_t n = 0; n < hid; ++n) {
+        double su = 0.0, sv = 0.0;
+        for (int32_t i = 0; i < c->d; ++i) {
+            double xi = elem(x, t * c->d + i, c->dtype);
+            su += elem(wg, w_off_in + (int64_t)n * c->d + i, c->dtype) * xi;
+            sv += elem(wu, w_off_in + (int64_t)n * c->d + i, c->dtype) * xi;
+        }
+        u[n] = su;
+        v[n] = sv;
+        a[n] = silu(su) * sv;
+    }
+}
+
+/* r = Wd^T dy_t for one expert (Wd = rows w_off_out.. of [d, hid]). */
+static void down_transpose(const oracle_cfg *c, const void *dy, int64_t t, const void *wd, int64_t w_off_out,
+                           int32_t hid, double *r)
+{
+    for (int32_t n = 0; n < hid; ++n) {
+        double s = 0.0;
+        for (int32_t i = 0; i < c->d; ++i)
+            s += elem(wd, w_off_out + (int64_t)i * hid + n, c->dtype) * elem(dy, t * c->d + i, c->dtype);
+        r[n] = s;
+    }
+}
+
+/* Backward of one expert on token t with gate g: returns dL/dg = r . a and
+ * adds Wg^T du + Wu^T dv into dx_t. */
+static double expert_backward_dx(const oracle_cfg *c, const void *x, const void *dy, int64_t t, const void *wg,
+                                 const void *wu, const void *wd, int64_t w_off_in, int64_t w_off_out,
+                                 int32_t hid, double g, double *u, double *v, double *a, double *r, double *dx_t)
+{
+    expert_hidden(c, x, t, wg, wu, w_off_in, hid, u, v, a);
+    down_transpose(c, dy, t, wd, w_off_out, hid, r);
+    double dgate = 0.0;
+    for (int32_t n = 0; n < hid; ++n) dgate += r[n] * a[n];
+    for (int32_t n = 0; n < hid; ++n) {
+        double da = g * r[n];
+        double du = da * v[n] * dsilu(u[n]);
+        double dv = da * silu(u[n]);
+        for (int32_t i = 0; i < c->d; ++i)
+            dx_t[i] += elem(wg, w_off_in + (int64_t)n * c->d + i, c->dtype) * du +
+                       elem(wu, w_off_in + (int64_t)n * c->d + i, c->dtype) * dv;
+    }
+    return dgate;
+}
+
+/* Weight gradients of hidden unit n of one expert from one token with gate
+ * g: row n of dWg / dWu and column n of dWd (stride hid). */
+static void expert_backward_w(const oracle_cfg *c, const void *x, const void *dy, int64_t t, const void *wg,
+                              const void *wu, const void *wd, int64_t w_off_in, int64_t w_off_out, int32_t hid,
+                              int32_t n, double g, double *dwg_row, double *dwu_row, double *dwd_col)
+{
+    double u = 0.0, v = 0.0, r = 0.0;
+    for (int32_t i = 0; i < c->d; ++i) {
+        double xi = elem(x, t * c->d + i, c->dtype);
+        u += elem(wg, w_off_in + (int64_t)n * c->d + i, c->dtype) * xi;
+        v += elem(wu, w_off_in + (int64_t)n * c->d + i, c->dtype) * xi;
+        r += elem(wd, w_off_out + (int64_t)i * hid + n, c->dtype) * elem(dy, t * c->d + i, c->dtype);
+    }
+    double a = silu(u) * v;
+    double da = g * r;
+    double du = da * v * dsilu(u);
+    double dv = da * silu(u);
+    for (int32_t i = 0; i < c->d; ++i) {
+        double xi = elem(x, t * c->d + i, c->dtype);
+        dwg_row[i] += du * xi;
+        dwu_row[i] += dv * xi;
+        dwd_col[(int64_t)i * hid] += g * elem(dy, t * c->d + i, c->dtype) * a;
+    }
+}
+
+/* The layer's backward for all T tokens.  dy has the layer's dtype; every
+ * output is float64 and overwritten: dx [T, d], dwr [E, d], dwg and dwu
+ * [E, h, d], dwd [E, d, h]; with a shared expert dshg, dshu [h_shared, d],
+ * dshd [d, h_shared] and dwsg [d] (else those may be NULL).  bias is the
+ * optional balance bias (it changes the selection only).  Tokens are
+ * independent in the first pass (dx and the router gradient, parallel over
+ * tokens); each weight gradient is then a sum over tokens in increasing t,
+ * parallel over experts and hidden units.  Returns 0, or -1 on a bad
+ * argument or allocation failure. */
+int oracle_backward(const oracle_cfg *c, const void *x, const void *wr, const void *wg, const void *wu,
+                    const void *wd, const void *sh_g, const void *sh_u, const void *sh_d, const void *w_sg,
+                    const float *bias, const void *dy, double *dx, double *dwr, double *dwg, double *dwu,
+                    double *dwd, double *dshg, double *dshu, double *dshd, double *dwsg, int nthreads)
+{
+    if (!cfg_ok(c) || !x || !wr || !wg || !wu || !wd || !dy || !dx || !dwr || !dwg || !dwu || !dwd) return -1;
+    const int shared = c->h_shared > 0;
+    if (shared && (!sh_g || !sh_u || !sh_d || !w_sg || !dshg || !dshu || !dshd || !dwsg)) return -1;
+    const int64_t T = c->T;
+    const int32_t E = c->E, d = c->d, h = c->h, k = c->k, hs = c->h_shared;
+    int nt = nthreads_used(nthreads);
+    int32_t *ids = malloc(sizeof(int32_t) * (size_t)(T * k > 0 ? T * k : 1));
+    double *gates = malloc(sizeof(double) * (size_t)(T * k > 0 ? T * k : 1));
+    double *dl = malloc(sizeof(double) * (size_t)(T * E > 0 ? T * E : 1));
+    double *sgs = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    double *dls = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!ids || !gates || !dl || !sgs || !dls) {
+        free(ids); free(gates); free(dl); free(sgs); free(dls);
+        return -1;
+    }
+    int bad = 0;
+    int32_t hmax = h > hs ? h : hs;
+    /* pass 1: per token -- routing, the gate gradients, dx, the router's logit gradient */
+#pragma omp parallel num_threads(nt)
+    {
+        double *buf = malloc(sizeof(double) * ((size_t)E * 5 + (size_t)k + 4 * (size_t)hmax));
+        char *taken = malloc((size_t)E);
+        if (!buf || !taken) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            double *logits = buf, *keys = buf + E, *scores = buf + 2 * E, *ds = buf + 3 * E;
+            double *dlt = buf + 4 * E, *dg = buf + 5 * E, *u = dg + k, *v = u + hmax, *a = v + hmax,
+                   *r = a + hmax;
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < T; ++t) {
+                double sg = 0.0;
+                route_one(c, x, wr, w_sg, bias, t, logits, keys, scores, taken, ids + t * k, gates + t * k,
+                          &sg);
+                double *dxt = dx + t * d;
+                for (int32_t i = 0; i < d; ++i) dxt[i] = 0.0;
+                for (int32_t j = 0; j < k; ++j) {
+                    int64_t e = ids[t * k + j];
+                    dg[j] = expert_backward_dx(c, x, dy, t, wg, wu, wd, e * h * d, e * d * h, h,
+                                               gates[t * k + j], u, v, a, r, dxt);
+                }
+                router_backward(c, scores, ids + t * k, gates + t * k, dg, ds, dlt);
+                for (int32_t e = 0; e < E; ++e) {
+                    dl[t * E + e] = dlt[e];
+                    for (int32_t i = 0; i < d; ++i) dxt[i] += dlt[e] * elem(wr, (int64_t)e * d + i, c->dtype);
+                }
+                sgs[t] = sg;
+                dls[t] = 0.0;
+                if (shared) {
+                    double dsg = expert_backward_dx(c, x, dy, t, sh_g, sh_u, sh_d, 0, 0, hs, sg, u, v, a, r, dxt);
+                    dls[t] = dsg * sg * (1.0 - sg);
+                    for (int32_t i = 0; i < d; ++i) dxt[i] += dls[t] * elem(w_sg, i, c->dtype);
+                }
+            }
+        }
+        free(buf);
+        free(taken);
+    }
+    if (!bad) {
+        /* pass 2: weight gradients, each a sum over tokens in increasing t */
+        memset(dwg, 0, sizeof(double) * (size_t)E * h * d);
+        memset(dwu, 0, sizeof(double) * (size_t)E * h * d);
+        memset(dwd, 0, sizeof(double) * (size_t)E * d * h);
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+        for (int32_t e = 0; e < E; ++e)
+            for (int32_t i = 0; i < d; ++i) {
+                double s = 0.0;
+                for (int64_t t = 0; t < T; ++t) s += dl[t * E + e] * elem(x, t * d + i, c->dtype);
+                dwr[(int64_t)e * d + i] = s;
+            }
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+        for (int64_t en = 0; en < (int64_t)E * h; ++en) {
+            int32_t e = (int32_t)(en / h), n = (int32_t)(en % h);
+            double *dwg_row = dwg + ((int64_t)e * h + n) * d, *dwu_row = dwu + ((int64_t)e * h + n) * d;
+            double *dwd_col = dwd + (int64_t)e * d * h + n;
+            for (int64_t t = 0; t < T; ++t)
+                for (int32_t j = 0; j < k; ++j)
+                    if (ids[t * k + j] == e)
+                        expert_backward_w(c, x, dy, t, wg, wu, wd, (int64_t)e * h * d, (int64_t)e * d * h, h, n,
+                                          gates[t * k + j], dwg_row, dwu_row, dwd_col);
+        }
+        if (shared) {
+            memset(dshg, 0, sizeof(double) * (size_t)hs * d);
+            memset(dshu, 0, sizeof(double) * (size_t)hs * d);
+            memset(dshd, 0, sizeof(double) * (size_t)d * hs);
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+            for (int32_t n = 0; n < hs; ++n)
+                for (int64_t t = 0; t < T; ++t)
+                    expert_backward_w(c, x, dy, t, sh_g, sh_u, sh_d, 0, 0, hs, n, sgs[t], dshg + (int64_t)n * d,
+                                      dshu + (int64_t)n * d, dshd + n);
+            for (int32_t i = 0; i < d; ++i) {
+                double s = 0.0;
+                for (int64_t t = 0; t < T; ++t) s += dls[t] * elem(x, t * d + i, c->dtype);
+                dwsg[i] = s;
+            }
+        }
+    }
+    free(ids);
+    free(gates);
+    free(dl);
+    free(sgs);
+    free(dls);
+    return bad ? -1 : 0;
 }

@@ -22,8 +22,10 @@ MUTANTS = [
     ("silu_sign", "return u / (1.0 + exp(-u));", "return u / (1.0 + exp(u));"),
     ("renorm_dropped", "if (c->norm_topk)\n", "if (0 && c->norm_topk)\n"),
     ("gate_from_slot_index", "gates[j] = scores[ids[j]];", "gates[j] = scores[j];"),
-    ("down_transposed", "elem(wd, w_off_out + (int64_t)i * hid + n, c->dtype)",
-     "elem(wd, w_off_out + (int64_t)n * c->d + i, c->dtype)"),
+    ("down_transposed", "o += elem(wd, w_off_out + (int64_t)i * hid + n, c->dtype) * a[n];",
+     "o += elem(wd, w_off_out + (int64_t)n * c->d + i, c->dtype) * a[n];"),
+    ("bwd_down_transposed", "s += elem(wd, w_off_out + (int64_t)i * hid + n, c->dtype) * elem(dy",
+     "s += elem(wd, w_off_out + (int64_t)n * c->d + i, c->dtype) * elem(dy"),
     ("gate_up_swapped", "a[n] = silu(u) * v;", "a[n] = silu(v) * u;"),
     ("router_transposed", "elem(wr, (int64_t)e * c->d + i, c->dtype)",
      "elem(wr, (int64_t)i * c->E + e, c->dtype)"),
@@ -47,6 +49,18 @@ MUTANTS = [
     ("score_mean_not_divided", "mean[e] = s / (double)c->T;", "mean[e] = s;"),
     ("switch_loss_without_N", "*loss = alpha * (double)c->E * sum;", "*loss = alpha * sum;"),
     ("switch_frac_over_assignments", "(double)counts[e] / (double)c->T", "(double)counts[e] / (double)(c->T * c->k)"),
+    ("bwd_dsilu", "return s * (1.0 + u * (1.0 - s));", "return s * (1.0 + u * s);"),
+    ("bwd_renorm_dropped", "ds[ids[j]] = c->norm_topk ? (dg[j] - dot) / q : dg[j];", "ds[ids[j]] = dg[j];"),
+    ("bwd_softmax_not_centred", "dl[e] = scores[e] * (ds[e] - sd);", "dl[e] = scores[e] * ds[e];"),
+    ("bwd_sigmoid_factor", "dl[e] = ds[e] * scores[e] * (1.0 - scores[e]);", "dl[e] = ds[e] * scores[e];"),
+    ("bwd_gate_missing", "double da = g * r[n];", "double da = r[n];"),
+    ("bwd_dv_uses_dsilu", "double dv = da * silu(u[n]);", "double dv = da * dsilu(u[n]);"),
+    ("bwd_dwd_without_gate", "dwd_col[(int64_t)i * hid] += g * elem(dy", "dwd_col[(int64_t)i * hid] += elem(dy"),
+    ("bwd_dwg_from_dv", "dwg_row[i] += du * xi;", "dwg_row[i] += dv * xi;"),
+    ("bwd_router_dx_dropped", "for (int32_t i = 0; i < d; ++i) dxt[i] += dlt[e]", "for (int32_t i = 0; i < 0; ++i) dxt[i] += dlt[e]"),
+    ("bwd_shared_gate_sign", "dls[t] = dsg * sg * (1.0 - sg);", "dls[t] = -dsg * sg * (1.0 - sg);"),
+    ("bwd_dwr_reversed", "s += dl[t * E + e] * elem(x, t * d + i, c->dtype);",
+     "s += dl[t * E + e] * elem(x, t * d + (d - 1 - i), c->dtype);"),
 ]
 
 

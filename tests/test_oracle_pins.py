@@ -18,7 +18,10 @@
 * the Switch statistics ("Mixture-of-Experts -- more capacity per byte of
   weight", "What's wired today"): a hand-computed example, the uniform router
   (P_e = 1/E) and uniform load (loss = alpha * k) closed forms, and the mean
-  of the numpy score matrix.
+  of the numpy score matrix;
+* the backward pass: central finite differences of the oracle's own forward
+  in float64 (every input element), and torch autograd (float64, CPU) on the
+  dense all-experts-then-mask formulation.
 """
 import itertools
 import math
@@ -467,11 +470,127 @@ def test_switch_statistics():
     check_switch_statistics()
 
 
+# ---------------------------------------------------------------- backward
+
+BWD_CASES = [
+    # (T, d, E, h, k, score, norm, h_shared, biased)
+    (5, 6, 4, 5, 2, "softmax", True, 0, False),
+    (4, 5, 5, 4, 3, "softmax", False, 3, False),
+    (5, 6, 4, 5, 2, "sigmoid", True, 3, True),
+    (4, 6, 3, 4, 1, "sigmoid", False, 0, False),
+    (3, 4, 1, 3, 1, "softmax", True, 2, False),      # E = 1: the gate is constant 1
+]
+
+
+def _bwd_case(case, seed):
+    """float64 inputs of a small layer with every token's selection margin >= 1e-3."""
+    T, d, E, h, k, score, norm, hs, biased = case
+    rng = np.random.default_rng(seed)
+    c = oracle.Cfg(T=T, d=d, E=E, h=h, k=k, norm_topk=norm, score=score, h_shared=hs, dtype="f64")
+    wr = rng.standard_normal((E, d)) * 0.7
+    b = (rng.standard_normal(E) * 0.1).astype(np.float32) if biased else None
+    x = rng.standard_normal((T, d))
+    for _ in range(200):
+        m = oracle.topk_margin(c, x, wr, bias=b, lib=lib())
+        bad = ~(m >= 1e-3)
+        if not bad.any():
+            break
+        x[bad] = rng.standard_normal((int(bad.sum()), d))
+    t = {"x": x, "wr": wr, "wg": rng.standard_normal((E, h, d)) * 0.5, "wu": rng.standard_normal((E, h, d)) * 0.5,
+         "wd": rng.standard_normal((E, d, h)) * 0.5, "dy": rng.standard_normal((T, d))}
+    if hs:
+        t.update(shg=rng.standard_normal((hs, d)) * 0.5, shu=rng.standard_normal((hs, d)) * 0.5,
+                 shd=rng.standard_normal((d, hs)) * 0.5, ws=rng.standard_normal(d) * 0.5)
+    return c, t, b
+
+
+def _fwd_loss(c, t, b):
+    sh = (t["shg"], t["shu"], t["shd"], t["ws"]) if c.h_shared else None
+    y = oracle.forward(c, t["x"], t["wr"], t["wg"], t["wu"], t["wd"], sh, bias=b, nthreads=1, lib=lib())
+    return float((y * t["dy"]).sum())
+
+
+_GRAD_OF = {"x": "dx", "wr": "dw_router", "wg": "dw_gate", "wu": "dw_up", "wd": "dw_down",
+            "shg": "dsh_gate", "shu": "dsh_up", "shd": "dsh_down", "ws": "dw_shared_gate"}
+
+
+def _oracle_grads(c, t, b):
+    sh = (t["shg"], t["shu"], t["shd"], t["ws"]) if c.h_shared else None
+    return oracle.backward(c, t["x"], t["wr"], t["wg"], t["wu"], t["wd"], t["dy"], sh, bias=b, lib=lib())
+
+
+def check_backward_finite_differences():
+    for i, case in enumerate(BWD_CASES):
+        c, t, b = _bwd_case(case, 500 + i)
+        g = _oracle_grads(c, t, b)
+        for name, gname in _GRAD_OF.items():
+            if name not in t:
+                continue
+            arr = t[name]
+            fd = np.zeros_like(arr)
+            for idx in np.ndindex(arr.shape):
+                v = arr[idx]
+                eps = 1e-6 * max(1.0, abs(v))
+                arr[idx] = v + eps
+                lp = _fwd_loss(c, t, b)
+                arr[idx] = v - eps
+                lm = _fwd_loss(c, t, b)
+                arr[idx] = v
+                fd[idx] = (lp - lm) / (2 * eps)
+            scale = max(np.abs(fd).max(), 1e-3)
+            np.testing.assert_allclose(g[gname], fd, rtol=0, atol=1e-6 * scale, err_msg=f"case {i} {gname}")
+
+
+def test_backward_finite_differences():
+    check_backward_finite_differences()
+
+
+def _torch_dense_grads(c, t, b):
+    """Autograd of the dense all-experts-then-mask formulation (float64, CPU)."""
+    import torch
+    T_ = {k_: torch.tensor(v, dtype=torch.float64, requires_grad=(k_ != "dy")) for k_, v in t.items()}
+    X, Wr = T_["x"], T_["wr"]
+    L = X @ Wr.T
+    S = torch.sigmoid(L) if c.score == "sigmoid" else torch.softmax(L, dim=1)
+    key = (S if c.score == "sigmoid" else L).detach().numpy()
+    if b is not None:
+        key = S.detach().numpy() + b.astype(np.float64)[None, :]
+    idx = np.broadcast_to(np.arange(c.E), key.shape)
+    order = torch.tensor(np.lexsort((idx, -key), axis=-1)[:, :c.k].copy())
+    gates = S.gather(1, order)
+    if c.norm_topk:
+        gates = gates / gates.sum(dim=1, keepdim=True)
+    G = torch.zeros(c.T, c.E, dtype=torch.float64).scatter(1, order, gates)
+    Y = torch.zeros(c.T, c.d, dtype=torch.float64)
+    for e in range(c.E):
+        a = torch.nn.functional.silu(X @ T_["wg"][e].T) * (X @ T_["wu"][e].T)
+        Y = Y + G[:, e:e + 1] * (a @ T_["wd"][e].T)
+    if c.h_shared:
+        a = torch.nn.functional.silu(X @ T_["shg"].T) * (X @ T_["shu"].T)
+        Y = Y + torch.sigmoid(X @ T_["ws"])[:, None] * (a @ T_["shd"].T)
+    (Y * T_["dy"]).sum().backward()
+    return {_GRAD_OF[k_]: v.grad.numpy() for k_, v in T_.items() if k_ != "dy"}
+
+
+def check_backward_vs_autograd_dense():
+    for i, case in enumerate(BWD_CASES):
+        c, t, b = _bwd_case(case, 600 + i)
+        g = _oracle_grads(c, t, b)
+        ref = _torch_dense_grads(c, t, b)
+        for gname, r in ref.items():
+            scale = max(np.abs(r).max(), 1e-12)
+            np.testing.assert_allclose(g[gname], r, rtol=0, atol=1e-12 * scale, err_msg=f"case {i} {gname}")
+
+
+def test_backward_vs_autograd_dense():
+    check_backward_vs_autograd_dense()
+
+
 # The checks the mutation tests run against deliberately broken builds.
 PIN_CHECKS = [check_worked_example, check_routing_brute_force, check_routing_vs_full_sort_and_ties,
               check_margin, check_dense_formulation, check_tiny_workload, check_loop_over_experts,
               check_single_expert_is_dense_swiglu, check_permutation_invariants, check_balance_bias_example,
               check_biased_routing_brute_force_and_formulations, check_bias_update_example,
-              check_switch_statistics]
+              check_switch_statistics, check_backward_finite_differences, check_backward_vs_autograd_dense]
 
 assert math.isclose(64 ** (1 / 3), 4.0)
