@@ -104,6 +104,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.oracle_balance_loss.restype = ctypes.c_int
     lib.oracle_backward.argtypes = [ctypes.POINTER(_CCfg)] + [P] * 20 + [ctypes.c_int]
     lib.oracle_backward.restype = ctypes.c_int
+    lib.oracle_quantize_q4.argtypes = [P, ctypes.c_int32, I64, ctypes.c_int32, P, P]
+    lib.oracle_quantize_q4.restype = ctypes.c_int
+    lib.oracle_dequantize_q4.argtypes = [P, P, I64, ctypes.c_int32, P]
+    lib.oracle_dequantize_q4.restype = ctypes.c_int
     _lib_cache[path] = lib
     return lib
 
@@ -265,3 +269,48 @@ def backward(c: Cfg, x, wr, wg, wu, wd, dy, shared=None, bias=None, nthreads: in
     if rc != 0:
         raise ValueError("oracle_backward rejected its arguments")
     return g
+
+
+def quantize_q4(w, lib: ctypes.CDLL | None = None):
+    """4-bit codes of a [..., cols] weight tensor (stored bits: uint16 bf16 or float32),
+    cols a multiple of 64: (packed nibbles uint8 [..., cols / 2], scales float32
+    [..., cols / 64])."""
+    lib = lib or load()
+    w = np.ascontiguousarray(w)
+    dt = {np.dtype(np.uint16): BF16, np.dtype(np.float32): F32}[w.dtype]
+    cols = w.shape[-1]
+    rows = w.size // cols
+    q = np.zeros(w.shape[:-1] + (cols // 2,), np.uint8)
+    sc = np.zeros(w.shape[:-1] + (cols // 64,), np.float32)
+    if lib.oracle_quantize_q4(_ptr(w), dt, rows, cols, _ptr(q), _ptr(sc)):
+        raise ValueError("oracle_quantize_q4 rejected its arguments")
+    return q, sc
+
+
+def dequantize_q4(q, scales, lib: ctypes.CDLL | None = None):
+    """The float64 values of a 4-bit tensor."""
+    lib = lib or load()
+    q = np.ascontiguousarray(q, np.uint8)
+    scales = np.ascontiguousarray(scales, np.float32)
+    cols = q.shape[-1] * 2
+    rows = q.size // q.shape[-1]
+    out = np.zeros(q.shape[:-1] + (cols,), np.float64)
+    if lib.oracle_dequantize_q4(_ptr(q), _ptr(scales), rows, cols, _ptr(out)):
+        raise ValueError("oracle_dequantize_q4 rejected its arguments")
+    return out
+
+
+def forward_q4(c: Cfg, x, wr, qg, sg_, qu, su, qd, sd, shared=None, tokens=None, bias=None, nthreads: int = 0,
+               lib: ctypes.CDLL | None = None):
+    """The layer with 4-bit routed experts: the routed weights are the values
+    their codes represent, everything else as stored; evaluated by the float64
+    forward on exact float64 copies of every input."""
+    from . import dense
+    f64 = Cfg(T=c.T, d=c.d, E=c.E, h=c.h, k=c.k, norm_topk=c.norm_topk, score=c.score, h_shared=c.h_shared,
+              dtype="f64")
+    sh = None
+    if shared is not None:
+        sh = tuple(np.ascontiguousarray(dense.to_f64(a)) for a in shared)
+    return forward(f64, np.ascontiguousarray(dense.to_f64(x)), np.ascontiguousarray(dense.to_f64(wr)),
+                   dequantize_q4(qg, sg_, lib), dequantize_q4(qu, su, lib), dequantize_q4(qd, sd, lib), sh,
+                   tokens=tokens, bias=bias, nthreads=nthreads, lib=lib)

@@ -730,3 +730,66 @@ int oracle_backward(const oracle_cfg *c, const void *x, const void *wr, const vo
     free(dls);
     return bad ? -1 : 0;
 }
+
+/* ------------------------------------------------------------------ 4-bit routed experts
+ *
+ * "Small MoE Architecture, in depth", section "Running experts that do not
+ * fit: offloading and quantisation" (routed experts quantised more
+ * aggressively than the shared expert and the router) and "Worked example:
+ * the batch-1 budget on a device" (4-bit weights, about half a byte per
+ * parameter).  The pages fix no format; the one read here: a weight matrix
+ * [rows, cols] (cols a multiple of 64) is cut into groups of 64 consecutive
+ * elements of a row; each group has the scale s = max|w| / 7 and each element
+ * the code q = round(w / s) in [-7, 7] (round to nearest, ties to even),
+ * stored as the nibble q + 8, two per byte (element 2i in the low nibble of
+ * byte i).  A group of zeros has s = 0 and codes 0.  The value represented is
+ * (nibble - 8) * s.  The code is decided in fp32 (s = fp32(max|w|) / 7 and
+ * w / s both rounded to fp32), the precision of the kernel that quantises.
+ */
+int oracle_quantize_q4(const void *w, int32_t dtype, int64_t rows, int32_t cols, uint8_t *q, float *scales)
+{
+    if (!w || !q || !scales || rows < 0 || cols <= 0 || cols % 64) return -1;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_F32) return -1;
+    const int32_t groups = cols / 64;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t g = 0; g < groups; ++g) {
+            float m = 0.0f;
+            for (int32_t i = 0; i < 64; ++i) {
+                float v = (float)elem(w, r * cols + g * 64 + i, dtype);
+                if (fabsf(v) > m) m = fabsf(v);
+            }
+            volatile float s = m / 7.0f;   /* one fp32 division, correctly rounded */
+            scales[r * groups + g] = s;
+            for (int32_t i = 0; i < 64; i += 2) {
+                int code[2];
+                for (int z = 0; z < 2; ++z) {
+                    float v = (float)elem(w, r * cols + g * 64 + i + z, dtype);
+                    if (s == 0.0f) {
+                        code[z] = 0;
+                    } else {
+                        volatile float ratio = v / s;
+                        float c = rintf(ratio);
+                        if (c > 7.0f) c = 7.0f;
+                        if (c < -7.0f) c = -7.0f;
+                        code[z] = (int)c;
+                    }
+                }
+                q[r * (cols / 2) + (g * 64 + i) / 2] = (uint8_t)((code[0] + 8) | ((code[1] + 8) << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* The values a 4-bit matrix represents, (nibble - 8) * scale, in double. */
+int oracle_dequantize_q4(const uint8_t *q, const float *scales, int64_t rows, int32_t cols, double *out)
+{
+    if (!q || !scales || !out || rows < 0 || cols <= 0 || cols % 64) return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t c = 0; c < cols; ++c) {
+            uint8_t b = q[r * (cols / 2) + c / 2];
+            int nib = (c % 2 == 0) ? (b & 15) : (b >> 4);
+            out[r * cols + c] = (double)(nib - 8) * (double)scales[r * (cols / 64) + c / 64];
+        }
+    return 0;
+}

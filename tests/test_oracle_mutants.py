@@ -59,6 +59,10 @@ MUTANTS = [
     ("bwd_dwg_from_dv", "dwg_row[i] += du * xi;", "dwg_row[i] += dv * xi;"),
     ("bwd_router_dx_dropped", "for (int32_t i = 0; i < d; ++i) dxt[i] += dlt[e]", "for (int32_t i = 0; i < 0; ++i) dxt[i] += dlt[e]"),
     ("bwd_shared_gate_sign", "dls[t] = dsg * sg * (1.0 - sg);", "dls[t] = -dsg * sg * (1.0 - sg);"),
+    ("q4_round_down", "float c = rintf(ratio);", "float c = floorf(ratio);"),
+    ("q4_scale_over_8", "volatile float s = m / 7.0f;", "volatile float s = m / 8.0f;"),
+    ("q4_nibbles_swapped", "(uint8_t)((code[0] + 8) | ((code[1] + 8) << 4))", "(uint8_t)((code[1] + 8) | ((code[0] + 8) << 4))"),
+    ("q4_dequant_offset", "out[r * cols + c] = (double)(nib - 8)", "out[r * cols + c] = (double)(nib - 7)"),
     ("bwd_dwr_reversed", "s += dl[t * E + e] * elem(x, t * d + i, c->dtype);",
      "s += dl[t * E + e] * elem(x, t * d + (d - 1 - i), c->dtype);"),
 ]

@@ -586,11 +586,90 @@ def test_backward_vs_autograd_dense():
     check_backward_vs_autograd_dense()
 
 
+# ---------------------------------------------------------------- 4-bit routed experts
+
+def check_q4_group_example():
+    g = _golden("q4_group_example.txt")
+    w = np.zeros((1, 64), np.float32)
+    w[0, :8] = [float(v) for v in g["weights"]]
+    for stored in (w, _to_bf16_bits(w)):
+        q, sc = oracle.quantize_q4(stored, lib=lib())
+        assert sc.shape == (1, 1) and sc[0, 0] == float(g["scale"][0])
+        np.testing.assert_array_equal(q[0, :4], [int(b, 16) for b in g["bytes"]])
+        assert (q[0, 4:] == 0x88).all()          # zeros: code 0, nibble 8
+        deq = oracle.dequantize_q4(q, sc, lib=lib())
+        np.testing.assert_array_equal(deq[0, :8], [float(v) for v in g["dequantised"]])
+        assert (deq[0, 8:] == 0).all()
+    # a group of zeros: scale 0, codes 0
+    q, sc = oracle.quantize_q4(np.zeros((2, 128), np.float32), lib=lib())
+    assert (sc == 0).all() and (q == 0x88).all()
+
+
+def test_q4_group_example():
+    check_q4_group_example()
+
+
+def check_q4_nearest_code():
+    """Every code is the nearest of -7..7 to w / scale in fp32 (ties to the even
+    code), the scale is fp32(max|w|) / 7 in fp32, and every represented value is
+    within half a scale of the weight."""
+    rng = np.random.default_rng(31)
+    w = (rng.standard_normal((6, 192)) * rng.uniform(0.01, 3.0, (6, 1))).astype(np.float32)
+    w[2, 64:128] *= 0                           # one all-zero group
+    q, sc = oracle.quantize_q4(w, lib=lib())
+    deq = oracle.dequantize_q4(q, sc, lib=lib())
+    cand = np.arange(-7, 8, dtype=np.float64)
+    for r in range(w.shape[0]):
+        for gi in range(3):
+            grp = w[r, 64 * gi:64 * gi + 64]
+            s_ref = np.float32(np.abs(grp).max()) / np.float32(7)
+            assert sc[r, gi] == s_ref
+            nib = np.stack([q[r, 32 * gi:32 * gi + 32] & 15, q[r, 32 * gi:32 * gi + 32] >> 4], 1).reshape(-1)
+            codes = nib.astype(np.int64) - 8
+            for i, v in enumerate(grp):
+                if s_ref == 0:
+                    assert codes[i] == 0
+                    continue
+                ratio = np.float64(np.float32(v) / s_ref)
+                dist = np.abs(cand - ratio)
+                best = cand[dist == dist.min()]
+                want = best[0] if best.size == 1 else best[np.abs(best) % 2 == 0][0]
+                assert codes[i] == want, (r, gi, i)
+            assert np.all(np.abs(deq[r, 64 * gi:64 * gi + 64] - grp) <= s_ref / 2 * (1 + 1e-6))
+
+
+def test_q4_nearest_code():
+    check_q4_nearest_code()
+
+
+def check_q4_forward_is_the_dense_layer_on_the_represented_weights():
+    from oracle import dense
+    w, a = _small_layer((21, 64, 5, 128, 2, "softmax", True, 64, "bf16"), 700)
+    c = ocfg(w)
+    qs = [oracle.quantize_q4(t, lib=lib()) for t in (a.wg, a.wu, a.wd)]
+    y = oracle.forward_q4(c, a.x, a.wr, *qs[0], *qs[1], *qs[2], a.shared, lib=lib())
+    deq = [oracle.dequantize_q4(q, s_, lib=lib()) for q, s_ in qs]
+    X, Wr = dense.to_f64(a.x), dense.to_f64(a.wr)
+    _, _, G = dense.route_matrix(X, Wr, c.k, c.score, c.norm_topk)
+    Y = np.zeros((c.T, c.d))
+    for e in range(c.E):
+        Y += G[:, e:e + 1] * dense.dense_swiglu(X, deq[0][e], deq[1][e], deq[2][e])
+    sg, su, sd, ws = (dense.to_f64(t) for t in a.shared)
+    Y += 1 / (1 + np.exp(-(X @ ws)))[:, None] * dense.dense_swiglu(X, sg, su, sd)
+    np.testing.assert_allclose(y, Y, rtol=0, atol=1e-12 * np.abs(Y).max())
+
+
+def test_q4_forward_is_the_dense_layer_on_the_represented_weights():
+    check_q4_forward_is_the_dense_layer_on_the_represented_weights()
+
+
 # The checks the mutation tests run against deliberately broken builds.
 PIN_CHECKS = [check_worked_example, check_routing_brute_force, check_routing_vs_full_sort_and_ties,
               check_margin, check_dense_formulation, check_tiny_workload, check_loop_over_experts,
               check_single_expert_is_dense_swiglu, check_permutation_invariants, check_balance_bias_example,
               check_biased_routing_brute_force_and_formulations, check_bias_update_example,
-              check_switch_statistics, check_backward_finite_differences, check_backward_vs_autograd_dense]
+              check_switch_statistics, check_backward_finite_differences, check_backward_vs_autograd_dense,
+              check_q4_group_example, check_q4_nearest_code,
+              check_q4_forward_is_the_dense_layer_on_the_represented_weights]
 
 assert math.isclose(64 ** (1 / 3), 4.0)
