@@ -5,6 +5,13 @@ buffers, and the float64 oracle timed on the host cores as a baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+The headline (`value`, `roofline`, `e2e`, `cpu_baseline`) is measured on
+--workload, by default the largest layer that fits one GPU (the Mixtral-like
+prefill).  The same line carries a `per_workload` block with every reported
+layer shape timed the same way (--per-workload-steps steps each): tokens/s,
+both roofline fractions of the layer and of its dominant kernel, the clocks
+seen during that workload's timed region, and the realised per-expert load.
+
 One process per GPU (torchrun for N > 1).  Every rank runs the whole layer on
 its own batch of T tokens (token-sharded replicas: the forward pass has no
 exchange step, so there is no collective on the data path); the timed region
@@ -28,7 +35,7 @@ import torch
 
 from sparse_mixture_experts_sigmoid_b200 import binding as B
 from sparse_mixture_experts_sigmoid_b200 import roofline, synth
-from sparse_mixture_experts_sigmoid_b200.workloads import HEADLINE, WORKLOADS
+from sparse_mixture_experts_sigmoid_b200.workloads import HEADLINE, REPORTED, WORKLOADS
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
@@ -44,6 +51,8 @@ STAGE_KERNEL = {"route": ("router_logits_kernel", "router_tc.cu"), "permute": ("
 # kernels of the small-batch path (at most 64 assignments)
 STAGE_KERNEL_SMALL = {"route": ("router_small_kernel", "router.cu"), "gate_up": ("seg_gateup_kernel", "segment.cu"),
                       "down": ("down_direct_kernel", "segment.cu")}
+# ... with 4-bit routed experts
+STAGE_KERNEL_Q4 = {"gate_up": ("seg_gateup_q4_kernel", "segment_q4.cu"), "down": ("down_direct_q4_kernel", "segment_q4.cu")}
 
 
 def parse():
@@ -56,6 +65,12 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-workload", action="store_true",
+                   help="time only --workload (no per_workload block)")
+    p.add_argument("--per-workload-steps", type=int, default=50)
+    p.add_argument("--train-workloads", default="",
+                   help="comma-separated workloads whose training step (forward + backward) is timed too")
+    p.add_argument("--train-steps", type=int, default=20)
     return p.parse_args()
 
 
@@ -219,12 +234,31 @@ def run_oracle_sample(w, layer_cpu, seconds: float, max_tokens: int | None = Non
 
 # ----------------------------------------------------------------------------- arms
 
-def bench_ours(args, w, ws_n, rank, local):
-    torch.cuda.set_device(local)
+def tensor_peak(peaks, clocks):
+    """The bf16 tensor peak to divide by: the sustained cuBLAS figure when the
+    timed region ran under the power cap (the regime it was measured in), the
+    burst figure otherwise."""
+    if "sw_power_cap" in (clocks.get("reasons") or []):
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
+
+
+def time_workload(args, w, ws_n, rank, local, steps, warmup, headline, q4=False):
+    """Times moe_forward on workload w (inputs resident in HBM, L2 flushed between
+    steps).  The headline workload also gets the end-to-end pass through the
+    public API with host buffers and the oracle baseline on the host cores.
+    q4: the routed experts in 4 bits (moe_forward_q4; quantised before timing)."""
     dev = torch.device("cuda", local)
     layer = synth.make_layer(w, dev)
     cfg = B.config_of(w)
     wsbuf = B.alloc_workspace(cfg, dev)
+    if q4:
+        qw = B.quantize_experts_q4(layer)
+        layer.w_gate = layer.w_up = layer.w_down = None   # only the 4-bit copies stay resident
+        torch.cuda.empty_cache()
+        fwd = lambda lay, **kw: B.forward_q4(cfg, lay, qw, **kw)
+    else:
+        fwd = lambda lay, **kw: B.forward_layer(cfg, lay, **kw)
     y = torch.empty(w.T, w.d, dtype=layer.x.dtype, device=dev)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -235,10 +269,9 @@ def bench_ours(args, w, ws_n, rank, local):
         flush_w.zero_()
         flush_r.sum()
 
-    K, W = args.steps, args.warmup
-
+    K, W = steps, warmup
     for _ in range(W):
-        B.forward_layer(cfg, layer, y=y, ws=wsbuf)
+        fwd(layer, y=y, ws=wsbuf)
     torch.cuda.synchronize()
     counts = B.workspace_views(cfg, wsbuf)["counts"].cpu().numpy()
 
@@ -252,30 +285,52 @@ def bench_ours(args, w, ws_n, rank, local):
         for i in range(K):
             flush()
             starts[i].record()
-            B.forward_layer(cfg, layer, y=y, ws=wsbuf)
+            fwd(layer, y=y, ws=wsbuf)
             stops[i].record()
         barrier(ws_n)
         launches = B.launch_count() - l0
     assert B.device_status() == 0, "device error flag set during the timed region"
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
-    ms_local = statistics.fmean(step_ms)
-    ms = reduce_max(ms_local, ws_n)
-    value = job_value(ws_n, w.T, ms)
+    ms = reduce_max(statistics.fmean(step_ms), ws_n)
+    clocks = sampler.summary()
 
-    # per-kernel breakdown: the same steps again with the library recording an
-    # event after each stage (the dominant kernel's roofline comes from these)
+    # per-stage breakdown: the same steps again with the library recording an
+    # event after each stage (an upper bound on each kernel's time: the events
+    # also stop the next kernel's prologue from overlapping this one's tail)
     ev = [B.StageEvents() for _ in range(K)]
     barrier(ws_n)
     for i in range(K):
         flush()
         with ev[i]:
-            B.forward_layer(cfg, layer, y=y, ws=wsbuf)
+            fwd(layer, y=y, ws=wsbuf)
     barrier(ws_n)
     stage = {n: statistics.fmean(e.stage_ms()[n] for e in ev) for n in B.STAGES}
+    stage = {n: reduce_max(v, ws_n) for n, v in stage.items()}
 
-    # end to end through the public API: pinned host x in, y back to pinned host
-    e2e = None
-    if not args.no_e2e:
+    peaks = roofline.measured_peaks()
+    tpk, tpk_kind = tensor_peak(peaks, clocks)
+    work = roofline.stage_work(w, counts, q4=q4)
+    dom = max((n for n in stage if n in work), key=lambda n: stage[n])
+    kname, ksrc = STAGE_KERNEL[dom]
+    if w.R <= B.decode_max_rows() and dom in STAGE_KERNEL_SMALL:
+        kname, ksrc = STAGE_KERNEL_SMALL[dom]
+    if q4 and dom in STAGE_KERNEL_Q4:
+        kname, ksrc = STAGE_KERNEL_Q4[dom]
+    dfr = roofline.fractions(work[dom]["flops"], work[dom]["bytes"], stage[dom] / 1e3, peaks, tpk)
+    lw = roofline.layer_work(w, counts, q4=q4)
+    lfr = roofline.fractions(lw["flops"], lw["bytes"], ms / 1e3, peaks, tpk)
+    lfr["tensor_frac_of_burst"] = lfr["tflops"] / peaks["bf16_tflops"]
+    res = {"workload": w.name + ("_q4" if q4 else ""), "tokens_per_s": job_value(ws_n, w.T, ms), "ms_per_step": ms,
+           "steps": K, "weights": "routed experts 4-bit (64-weight groups, fp32 scales)" if q4 else w.dtype,
+           "warmup": W, "gpu_launches": launches, "layer": lfr,
+           "dominant": {"stage": dom, "kernel": kname, "ms_per_launch": stage[dom],
+                        "algorithmic_flops": work[dom]["flops"], "algorithmic_bytes": work[dom]["bytes"], **dfr},
+           "stages_ms": stage, "clocks": clocks, "tensor_peak": tpk, "tensor_peak_kind": tpk_kind,
+           "load": roofline.load_spread(counts)}
+    res["_roof"] = (dom, kname, ksrc, dfr, peaks, tpk, tpk_kind)
+
+    if headline and not args.no_e2e:
+        # end to end through the public API: pinned host x in, y back to pinned host
         xh = layer.x.cpu().pin_memory()
         yh = torch.empty(w.T, w.d, dtype=y.dtype).pin_memory()
         xd = torch.empty_like(layer.x)
@@ -299,45 +354,115 @@ def bench_ours(args, w, ws_n, rank, local):
             tot += s0.elapsed_time(s1)
         barrier(ws_n)
         e2e_ms = reduce_max(tot / K, ws_n)
-        e2e = {"value": job_value(ws_n, w.T, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
-               "d2h_bytes_per_step": yh.numel() * yh.element_size()}
+        res["e2e"] = {"value": job_value(ws_n, w.T, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                      "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+                      "d2h_bytes_per_step": yh.numel() * yh.element_size()}
 
-    # roofline of the dominant kernel
-    peaks = roofline.measured_peaks()
-    work = roofline.stage_work(w, counts)
-    dom = max((n for n in stage if n in work), key=lambda n: stage[n])
-    fl, by = work[dom]["flops"], work[dom]["bytes"]
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    t = stage[dom] / 1e3
-    kname, ksrc = STAGE_KERNEL[dom]
-    if w.R <= B.decode_max_rows() and dom in STAGE_KERNEL_SMALL:
-        kname, ksrc = STAGE_KERNEL_SMALL[dom]
-    if by > 0 and fl / by < ridge:
-        roof = {"bound": "hbm", "achieved": by / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": fl / t / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for(dom, ksrc, w.name)
-    roof.update({"kernel": kname, "stage": dom, "ms_per_launch": stage[dom],
-                 "algorithmic_bytes": by, "algorithmic_flops": fl, "peak_source": peaks["source"]})
-    lw = roofline.layer_work(w, counts)
-    layer_roof = {"tflops": lw["flops"] / (ms / 1e3) / 1e12, "gbs": lw["bytes"] / (ms / 1e3) / 1e9,
-                  "tensor_frac": lw["flops"] / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
-                  "hbm_frac": lw["bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
-
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n, "steps": K, "warmup": W,
-           "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-           "dtype": dtype_name(w), "data": "synthetic (seeded; shapes and distributions of the workload)",
-           "config": config_json(w, ws_n), "roofline": roof, "layer_roofline": layer_roof,
-           "stages_ms": stage, "gpu_launches": launches, "clocks": sampler.summary(), "e2e": e2e,
-           "active_experts": int(np.count_nonzero(counts))}
-
-    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+    if headline and rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         layer_cpu = layer.to("cpu")
         n, el, used, desc = run_oracle_sample(w, layer_cpu, args.cpu_seconds)
-        out["cpu_baseline"] = {"value": n / el, "unit": "tokens/s", "cores": used, "kind": "oracle",
+        res["cpu_baseline"] = {"value": n / el, "unit": "tokens/s", "cores": used, "kind": "oracle",
                                "sample": desc, "seconds": el}
+        del layer_cpu
+    del layer, wsbuf, y, flush_w, flush_r
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_train(args, w, ws_n, local, steps, warmup):
+    """Times one training step of the layer -- moe_forward_train then
+    moe_backward with a seeded upstream gradient -- with L2 flushed between
+    steps.  Work counted: the forward's FLOPs plus twice them for the backward
+    (the data and weight gradients of every GEMM)."""
+    dev = torch.device("cuda", local)
+    layer = synth.make_layer(w, dev)
+    cfg = B.config_of(w)
+    ws = B.alloc_train_workspace(cfg, dev)
+    g = torch.Generator(device=dev).manual_seed(w.seed + 7)
+    dy = torch.randn(w.T, w.d, generator=g, device=dev).to(layer.x.dtype)
+    y = torch.empty(w.T, w.d, dtype=layer.x.dtype, device=dev)
+    grads = None
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        B.forward_train(cfg, layer, ws, y=y)
+        grads = B.backward(cfg, layer, dy, ws, grads=grads)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier(ws_n)
+        for i in range(steps):
+            flush_w.zero_()
+            flush_r.sum()
+            ev[i][0].record()
+            B.forward_train(cfg, layer, ws, y=y)
+            ev[i][1].record()
+            B.backward(cfg, layer, dy, ws, grads=grads)
+            ev[i][2].record()
+        barrier(ws_n)
+    assert B.device_status() == 0, "device error flag set during the training steps"
+    fwd = reduce_max(statistics.fmean(e[0].elapsed_time(e[1]) for e in ev), ws_n)
+    bwd = reduce_max(statistics.fmean(e[1].elapsed_time(e[2]) for e in ev), ws_n)
+    clocks = sampler.summary()
+    peaks = roofline.measured_peaks()
+    tpk, tpk_kind = tensor_peak(peaks, clocks)
+    ms = fwd + bwd
+    flops = 3.0 * w.flops()
+    res = {"tokens_per_s": job_value(ws_n, w.T, ms), "ms_per_step": ms, "forward_ms": fwd, "backward_ms": bwd,
+           "steps": steps, "tflops": flops / (ms / 1e3) / 1e12,
+           "tensor_frac": flops / (ms / 1e3) / 1e12 / tpk, "tensor_peak_kind": tpk_kind, "clocks": clocks}
+    del layer, ws, dy, y, grads, flush_w, flush_r
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_ours(args, w, ws_n, rank, local):
+    torch.cuda.set_device(local)
+    head = time_workload(args, w, ws_n, rank, local, args.steps, args.warmup, headline=True)
+    dom, kname, ksrc, dfr, peaks, tpk, tpk_kind = head.pop("_roof")
+    bound = dfr["bound"]
+    if bound == "tensor":
+        roof = {"bound": "tensor", "achieved": dfr["tflops"], "peak": tpk, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": dfr["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for(dom, ksrc, w.name)
+    roof.update({"tensor_frac": dfr["tensor_frac"], "hbm_frac": dfr["hbm_frac"],
+                 "tensor_frac_of_burst": dfr["tflops"] / peaks["bf16_tflops"],
+                 "kernel": kname, "stage": dom, "ms_per_launch": head["dominant"]["ms_per_launch"],
+                 "algorithmic_bytes": head["dominant"]["algorithmic_bytes"],
+                 "algorithmic_flops": head["dominant"]["algorithmic_flops"],
+                 "peak_source": f"{peaks['source']} ({'cuBLAS bf16 ' + tpk_kind if bound == 'tensor' else 'HBM copy'})"})
+    ms = head["ms_per_step"]
+    out = {"metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": ws_n,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w),
+           "data": "synthetic (seeded; shapes and distributions of the workload)",
+           "config": config_json(w, ws_n), "roofline": roof, "layer_roofline": head["layer"],
+           "stages_ms": head["stages_ms"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+           "e2e": head.get("e2e"), "load": head["load"]}
+    if "cpu_baseline" in head:
+        out["cpu_baseline"] = head["cpu_baseline"]
+    if not args.no_per_workload:
+        per = {}
+        for name in REPORTED:
+            if name == w.name:
+                entry = {k: v for k, v in head.items() if k not in ("e2e", "cpu_baseline")}
+            else:
+                entry = time_workload(args, WORKLOADS[name], ws_n, rank, local, args.per_workload_steps,
+                                      args.warmup, headline=False)
+                entry.pop("_roof")
+            per[name] = entry
+        # the batch-1 decode step again with 4-bit routed experts
+        entry = time_workload(args, WORKLOADS["mixtral_decode"], ws_n, rank, local, args.per_workload_steps,
+                              args.warmup, headline=False, q4=True)
+        entry.pop("_roof")
+        per["mixtral_decode_q4"] = entry
+        out["per_workload"] = per
+    if args.train_workloads:
+        out["train"] = {name: time_train(args, WORKLOADS[name], ws_n, local, args.train_steps, args.warmup)
+                        for name in args.train_workloads.split(",") if name}
     return out
 
 

@@ -7,7 +7,8 @@
  *   l_e    = x . W_router[e]                       e = 0..E-1, bias-free
  *   s_e    = softmax(l)_e  or  sigmoid(l_e)        score function
  *   ids    = the k experts with the largest keys, best first; the key is
- *            l_e under softmax (same order as s_e) and s_e under sigmoid;
+ *            s_e + b_e with a balance bias b, else s_e (which the library
+ *            ranks through l_e: both score functions are increasing in it);
  *            equal keys go to the lower expert index
  *   g_j    = s_{ids_j}, divided by sum_j s_{ids_j} when norm_topk is set
  *   y      = sum_j g_j * W_down[ids_j] (silu(W_gate[ids_j] x) * (W_up[ids_j] x))
@@ -20,9 +21,13 @@
  * scores, optional renormalisation), section 3 "Expert Computation" (group
  * rows by expert, grouped expert linears, unsort and weighted sum), section 4
  * "The Complete MoE Layer" (weight shapes); "Small MoE Architecture, in depth"
- * -- section "A small MoE layer in PyTorch" (sigmoid scores, SwiGLU experts,
- * shared expert added to every token).  The sigmoid gate on the shared expert
- * and the tie rule are this library's readings where the pages are silent.
+ * -- section "A small MoE layer in PyTorch" (sigmoid scores, a balance bias
+ * that only steers the selection, SwiGLU experts, shared expert added to every
+ * token) and the paragraph on auxiliary-loss-free balancing after it;
+ * "Mixture-of-Experts -- more capacity per byte of weight", section "What's
+ * wired today" (the Switch load-balancing term).  The sigmoid gate on the
+ * shared expert and the tie rule are this library's readings where the pages
+ * are silent.
  *
  * Conventions for every entry point:
  *  - Tensors are row-major and contiguous, in DEVICE memory owned by the
@@ -97,6 +102,23 @@ typedef struct {
     float *y_acc;         /* [T, d]  fp32 accumulator; NULL when dtype is MOE_F32 */
 } moe_workspace_views;
 
+/* Options of the routing step for training; every field is optional (NULL
+ * turns it off) and so is the struct (opts == NULL turns all off).  Both
+ * pointers are device memory owned by the caller.
+ *   balance_bias [E] fp32: added to the scores only to choose the top k; the
+ *       gates still come from the unbiased scores ("Small MoE Architecture,
+ *       in depth", SmallMoE.forward and the auxiliary-loss-free balancing
+ *       paragraph after it).  Update it after a step with moe_update_bias.
+ *   score_mean [E] fp32, out: P_e = (1/T) sum_t s_e(t), the mean over the T
+ *       tokens of each expert's score (the whole score row, before
+ *       selection): the router statistic of the Switch load-balancing term
+ *       (moe_balance_loss).  Added in a fixed order, so repeated calls give
+ *       identical bits. */
+typedef struct {
+    const float *balance_bias;
+    float *score_mean;
+} moe_route_opts;
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *moe_status_string(moe_status status);
 
@@ -114,6 +136,7 @@ moe_status moe_workspace_layout(const moe_config *cfg, void *ws, size_t ws_bytes
                                 moe_workspace_views *views);
 
 /* Router: logits, scores, top-k selection and gates for all T tokens.
+ *   opts     routing options (balance bias, score statistic), or NULL
  *   x        [T, d]        dtype
  *   w_router [E, d]        dtype
  *   w_shared_gate [d]      dtype, or NULL (then shared_gate must be NULL)
@@ -122,16 +145,40 @@ moe_status moe_workspace_layout(const moe_config *cfg, void *ws, size_t ws_bytes
  *   probs    [T, E] fp32   out, optional (NULL): every expert's score s_e
  *   shared_gate [T] fp32   out, optional: sigmoid(w_s . x)
  *   ws, ws_bytes: device scratch of at least moe_route_workspace_size(cfg)
- *            bytes, 256-byte aligned (may be NULL when that size is 0)
+ *            bytes, 256-byte aligned
  * "Tutorial 11", section 2 (route_topk); "Small MoE Architecture, in depth",
- * forward of SmallMoE (sigmoid scores, gates from the raw scores). */
-moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router,
-                     const void *w_shared_gate, int32_t *ids, float *gates, float *probs,
-                     float *shared_gate, void *ws, size_t ws_bytes, void *stream);
+ * forward of SmallMoE (sigmoid scores, balance bias, gates from the raw
+ * scores). */
+moe_status moe_route(const moe_config *cfg, const moe_route_opts *opts, const void *x,
+                     const void *w_router, const void *w_shared_gate, int32_t *ids, float *gates,
+                     float *probs, float *shared_gate, void *ws, size_t ws_bytes, void *stream);
 
-/* Bytes of scratch that moe_route needs for cfg (host only; 0 for batches
- * served by the CUDA-core router). */
+/* Bytes of scratch that moe_route needs for cfg (host only). */
 moe_status moe_route_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/* Balance-bias update after a training step ("Small MoE Architecture, in
+ * depth", SmallMoE.forward in training, and the auxiliary-loss-free balancing
+ * paragraph after it): with load_e = counts[e] and mean = sum(counts) / E,
+ *   bias[e] += lr * sign(mean - load_e)
+ * so an expert above the mean load loses lr, one below it gains lr and one at
+ * the mean keeps its bias (the comparison is exact, in integers).
+ *   counts [E] int32 (from moe_permute, or the workspace after moe_forward);
+ *   bias   [E] fp32, updated in place (fp32 add, round to nearest).
+ *   lr must be finite, else MOE_ERR_INVALID_ARG. */
+moe_status moe_update_bias(const moe_config *cfg, const int32_t *counts, float lr, float *bias,
+                           void *stream);
+
+/* The Switch load-balancing term ("Mixture-of-Experts -- more capacity per
+ * byte of weight", "What's wired today"):
+ *   loss = alpha * E * sum_e f_e * P_e,   f_e = counts[e] / T
+ * (f_e: the fraction of the T tokens dispatched to expert e; P_e: the mean
+ * score from moe_route_opts.score_mean).  fp32; the sum over experts is a
+ * fixed tree, so repeated calls give identical bits.
+ *   counts [E] int32; score_mean [E] fp32; frac [E] fp32 out (f_e) or NULL;
+ *   loss [1] fp32 out.  T = 0 gives f = 0 and loss = 0.  alpha must be
+ *   finite, else MOE_ERR_INVALID_ARG. */
+moe_status moe_balance_loss(const moe_config *cfg, const int32_t *counts, const float *score_mean,
+                            float alpha, float *frac, float *loss, void *stream);
 
 /* Grouping: counts, offsets and the stable permutation of the T*k
  * assignments by expert, and its inverse.
@@ -189,10 +236,14 @@ moe_status moe_combine(const moe_config *cfg, const void *act, const void *w_dow
  *   MOE_ERR_WORKSPACE and enqueues nothing.  The call allocates nothing and
  *   calls no allocating routine.
  *   The first call on a device looks up the array's device address (a
- *   one-time, per-device set-up with that device current); make that first
- *   call before any stream capture.  All calls share the array and it keeps
- *   the last call's contents: each call clears the part it uses, and calls
- *   that overlap on the GPU (unordered streams) race on it. */
+ *   one-time, per-device set-up with that device current).  With CUDA's lazy
+ *   module loading (the default) that look-up is also when the driver loads
+ *   this part of the library onto the device and backs the array with device
+ *   memory, so the first call may allocate: make it at start-up, outside any
+ *   region that must not allocate and before any stream capture.  Later
+ *   calls allocate nothing.  All calls share the array and it keeps the last
+ *   call's contents: each call clears the part it uses, and calls that
+ *   overlap on the GPU (unordered streams) race on it. */
 #define MOE_NOALLOC_MAX_ACC_FLOATS (4u << 20)
 moe_status moe_combine_noalloc(const moe_config *cfg, const void *act, const void *w_down,
                                const int32_t *offsets, const int32_t *sorted_rows, const float *gates,
@@ -200,6 +251,7 @@ moe_status moe_combine_noalloc(const moe_config *cfg, const void *act, const voi
 
 /* The whole layer: route, group, grouped SwiGLU, down projection and combine,
  * plus the shared expert when cfg->h_shared > 0.
+ *   opts: routing options (balance bias, score statistic) or NULL;
  *   x [T, d]; w_router [E, d]; w_gate, w_up [E, h, d]; w_down [E, d, h];
  *   sh_gate, sh_up [h_shared, d], sh_down [d, h_shared], w_shared_gate [d]
  *   (all four NULL when h_shared == 0); y [T, d] out (dtype).
@@ -207,11 +259,84 @@ moe_status moe_combine_noalloc(const moe_config *cfg, const void *act, const voi
  *   aligned; afterwards it holds the routing results (moe_workspace_layout).
  * "Tutorial 11", section 4 (Moe.__call__); "Small MoE Architecture, in
  * depth", SmallMoE.forward (shared expert). */
-moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
-                       const void *w_gate, const void *w_up, const void *w_down,
+moe_status moe_forward(const moe_config *cfg, const moe_route_opts *opts, const void *x,
+                       const void *w_router, const void *w_gate, const void *w_up, const void *w_down,
                        const void *sh_gate, const void *sh_up, const void *sh_down,
                        const void *w_shared_gate, void *y, void *ws, size_t ws_bytes,
                        void *stream);
+
+/* ---- training: the forward pass that keeps what the backward needs, and the
+ * backward pass.  bf16 layers only (MOE_F32 returns MOE_ERR_UNSUPPORTED).
+ * The pages train this layer ("Small models, sparse experts", "Dispatch
+ * decides everything" quotes training tokens/s; "Small MoE Architecture, in
+ * depth", SmallMoE) but print no backward: the gradient here is the chain rule
+ * through the forward's steps.  The top-k selection (and the balance bias)
+ * passes no gradient. */
+
+/* Bytes of the workspace of one training step (moe_forward_train followed by
+ * moe_backward on the same workspace; host only). */
+moe_status moe_train_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/* moe_forward for training: the same arguments and output, plus it keeps in
+ * ws what moe_backward needs (every token's score row and each grouped row's
+ * pre-activations W_gate x and W_up x, in bf16).  It always takes the
+ * tensor-core path.  ws: at least moe_train_workspace_size(cfg) bytes,
+ * 256-byte aligned; pass it unchanged to moe_backward. */
+moe_status moe_forward_train(const moe_config *cfg, const moe_route_opts *opts, const void *x,
+                             const void *w_router, const void *w_gate, const void *w_up,
+                             const void *w_down, const void *sh_gate, const void *sh_up,
+                             const void *sh_down, const void *w_shared_gate, void *y, void *ws,
+                             size_t ws_bytes, void *stream);
+
+/* Gradients of the layer, given dy = dL/dy [T, d] (bf16), after
+ * moe_forward_train with the same inputs on the same workspace ws:
+ *   dx [T, d] bf16;  dw_router [E, d] fp32;  dw_gate, dw_up [E, h, d] bf16;
+ *   dw_down [E, d, h] bf16;  with a shared expert dsh_gate, dsh_up [h_s, d]
+ *   and dsh_down [d, h_s] bf16 and dw_shared_gate [d] fp32 (else NULL).
+ * Every output is overwritten (an expert that received no rows gets a zero
+ * gradient).  Accumulation is fp32; the routed rows' gradients reach the
+ * weights in grouped order, dx through fp32 additions in token order (their
+ * order over the k experts is not fixed).  ws also serves as the backward's
+ * scratch, so it no longer holds the forward's activations afterwards. */
+moe_status moe_backward(const moe_config *cfg, const void *x, const void *w_router,
+                        const void *w_gate, const void *w_up, const void *w_down,
+                        const void *sh_gate, const void *sh_up, const void *sh_down,
+                        const void *w_shared_gate, const void *dy, void *ws, size_t ws_bytes,
+                        void *dx, float *dw_router, void *dw_gate, void *dw_up, void *dw_down,
+                        void *dsh_gate, void *dsh_up, void *dsh_down, float *dw_shared_gate,
+                        void *stream);
+
+/* ---- 4-bit routed experts ("Small MoE Architecture, in depth": "Worked
+ * example: the batch-1 budget on a device" -- 4-bit weights, about half a
+ * byte per parameter, so a decode step reads a quarter of the bf16 bytes --
+ * and "Running experts that do not fit: offloading and quantisation" --
+ * routed experts quantised, shared expert and router kept at higher
+ * precision).  The pages fix no format; this library's: a weight matrix
+ * [rows, cols] (cols a multiple of 64) is cut into groups of 64 consecutive
+ * elements of a row; scale s = max|w| / 7 (fp32); code = round(w / s) in
+ * [-7, 7], ties to even, both decided in fp32; stored as the nibble code + 8,
+ * two per byte, the even element in the low nibble.  The value represented
+ * is (nibble - 8) * s. */
+
+/* Quantises w [rows, cols] (device, dtype MOE_BF16 or MOE_F32, cols a
+ * multiple of 64, else MOE_ERR_UNSUPPORTED) into q [rows, cols / 2] bytes and
+ * scales [rows, cols / 64] fp32 (device, caller-owned; w and q 16-byte
+ * aligned).  For a layer: W_gate and W_up as [E * h, d], W_down as [E * d, h]. */
+moe_status moe_quantize_q4(const void *w, int32_t dtype, int64_t rows, int32_t cols, uint8_t *q,
+                           float *scales, void *stream);
+
+/* moe_forward with 4-bit routed experts (q_* / s_* from moe_quantize_q4 of
+ * W_gate, W_up [E * h, d] and W_down [E * d, h]); x, the router and the shared
+ * expert stay bf16.  Served by the small-batch kernels, which stream the
+ * chosen experts' 4-bit rows once: T * k <= moe_decode_max_rows(), bf16, d and
+ * h multiples of 64 (else MOE_ERR_UNSUPPORTED).  ws: moe_workspace_size(cfg)
+ * bytes.  The result is the layer evaluated on the represented weights. */
+moe_status moe_forward_q4(const moe_config *cfg, const moe_route_opts *opts, const void *x,
+                          const void *w_router, const uint8_t *q_gate, const float *s_gate,
+                          const uint8_t *q_up, const float *s_up, const uint8_t *q_down,
+                          const float *s_down, const void *sh_gate, const void *sh_up,
+                          const void *sh_down, const void *w_shared_gate, void *y, void *ws,
+                          size_t ws_bytes, void *stream);
 
 /* Largest T*k that moe_forward serves with the CUDA-core small-batch kernels
  * (one warp per weight row, weights streamed once); larger batches use the
@@ -232,7 +357,7 @@ typedef enum {
 
 /* Profiling hook for the calling host thread.  With events != NULL (n must be
  * MOE_STAGE_COUNT + 1 cudaEvent_t handles, created by the caller), every later
- * moe_forward call on this thread records events[0] on its stream before its
+ * moe_forward (or moe_forward_q4) call on this thread records events[0] on its stream before its
  * first launch and events[i + 1] after stage i; a stage that does not run
  * records an empty interval.  events == NULL turns the hook off.  Host only. */
 moe_status moe_profile_events(void *const *events, int32_t n);

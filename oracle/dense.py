@@ -74,9 +74,14 @@ def route_matrix(X, Wr, k, score="softmax", norm_topk=True, bias=None):
     return ids, gates, G
 
 
+def swiglu_act(X, Wg, Wu):
+    """The expert's hidden activation silu(X Wg^T) * (X Wu^T) for X [n, d], Wg/Wu [h, d]."""
+    return _silu(X @ Wg.T) * (X @ Wu.T)
+
+
 def dense_swiglu(X, Wg, Wu, Wd):
     """down(silu(X Wg^T) * (X Wu^T)) for X [n, d], Wg/Wu [h, d], Wd [d, h]."""
-    return (_silu(X @ Wg.T) * (X @ Wu.T)) @ Wd.T
+    return swiglu_act(X, Wg, Wu) @ Wd.T
 
 
 def dense_forward(cfg, x, wr, wg, wu, wd, shared=None, bias=None):

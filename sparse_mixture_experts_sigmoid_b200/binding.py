@@ -24,7 +24,8 @@ EXPORTED = ["moe_status_string", "moe_validate", "moe_workspace_size", "moe_work
             "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_decode_max_rows",
             "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size",
             "moe_selftest_wait_timeout",
-            "moe_route_workspace_size"]
+            "moe_route_workspace_size", "moe_update_bias", "moe_balance_loss", "moe_train_workspace_size",
+            "moe_forward_train", "moe_backward", "moe_quantize_q4", "moe_forward_q4"]
 STAGES = ["route", "permute", "gate_up", "shared_gate_up", "down", "shared_down", "finalize"]
 
 
@@ -38,6 +39,11 @@ class MoEConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("h", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("norm_topk", ctypes.c_int32), ("score", ctypes.c_int32),
                 ("h_shared", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class RouteOpts(ctypes.Structure):
+    """moe_route_opts: balance bias (selection only) and the score-mean output."""
+    _fields_ = [("balance_bias", ctypes.c_void_p), ("score_mean", ctypes.c_void_p)]
 
 
 class WorkspaceViews(ctypes.Structure):
@@ -63,13 +69,22 @@ def lib() -> ctypes.CDLL:
             "moe_validate": ([C], ctypes.c_int),
             "moe_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_workspace_layout": ([C, P, S, ctypes.POINTER(WorkspaceViews)], ctypes.c_int),
-            "moe_route": ([C, P, P, P, P, P, P, P, P, S, P], ctypes.c_int),
+            "moe_route": ([C, ctypes.POINTER(RouteOpts), P, P, P, P, P, P, P, P, S, P], ctypes.c_int),
             "moe_route_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_permute": ([C, P, P, P, P, P, P, S, P], ctypes.c_int),
             "moe_permute_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_grouped_swiglu": ([C, P, P, P, P, P, P, P], ctypes.c_int),
             "moe_combine": ([C, P, P, P, P, P, P, P, S, P], ctypes.c_int),
-            "moe_forward": ([C, P, P, P, P, P, P, P, P, P, P, P, S, P], ctypes.c_int),
+            "moe_forward": ([C, ctypes.POINTER(RouteOpts), P, P, P, P, P, P, P, P, P, P, P, S, P],
+                            ctypes.c_int),
+            "moe_update_bias": ([C, P, ctypes.c_float, P, P], ctypes.c_int),
+            "moe_train_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
+            "moe_forward_train": ([C, ctypes.POINTER(RouteOpts), P, P, P, P, P, P, P, P, P, P, P, S, P],
+                                  ctypes.c_int),
+            "moe_backward": ([C] + [P] * 11 + [S] + [P] * 10, ctypes.c_int),
+            "moe_quantize_q4": ([P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, P, P, P], ctypes.c_int),
+            "moe_forward_q4": ([C, ctypes.POINTER(RouteOpts)] + [P] * 14 + [P, S, P], ctypes.c_int),
+            "moe_balance_loss": ([C, P, P, ctypes.c_float, P, P, P], ctypes.c_int),
             "moe_decode_max_rows": ([], ctypes.c_int32),
             "moe_device_status": ([P], ctypes.c_int),
             "moe_selftest_wait_timeout": ([ctypes.c_uint32, P], ctypes.c_int),
@@ -176,8 +191,20 @@ def route_workspace_size(cfg: MoEConfig) -> int:
     return n.value
 
 
-def route(cfg: MoEConfig, x, w_router, w_shared_gate=None, want_probs=False, ws=None, stream=None):
-    """Returns (ids[T,k] int32, gates[T,k] f32, probs[T,E] | None, shared_gate[T] | None)."""
+def route_opts(cfg: MoEConfig, balance_bias=None, score_mean=None):
+    """A moe_route_opts for ctypes (None when both are absent).  balance_bias and
+    score_mean are [E] float32 CUDA tensors (score_mean is written)."""
+    if balance_bias is None and score_mean is None:
+        return None
+    return ctypes.byref(RouteOpts(_ptr(balance_bias, "balance_bias", (cfg.E,), torch.float32),
+                                  _ptr(score_mean, "score_mean", (cfg.E,), torch.float32)))
+
+
+def route(cfg: MoEConfig, x, w_router, w_shared_gate=None, want_probs=False, ws=None, stream=None,
+          balance_bias=None, score_mean=None):
+    """Returns (ids[T,k] int32, gates[T,k] f32, probs[T,E] | None, shared_gate[T] | None).
+    balance_bias: optional [E] float32 selection bias; score_mean: optional [E]
+    float32 tensor that receives the mean score per expert."""
     et = _elem_dtype(cfg)
     dev = x.device
     if ws is None:
@@ -187,7 +214,8 @@ def route(cfg: MoEConfig, x, w_router, w_shared_gate=None, want_probs=False, ws=
     gates = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
     probs = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev) if want_probs else None
     sg = torch.empty(cfg.T, dtype=torch.float32, device=dev) if w_shared_gate is not None else None
-    _check(lib().moe_route(ctypes.byref(cfg), _ptr(x, "x", (cfg.T, cfg.d), et),
+    _check(lib().moe_route(ctypes.byref(cfg), route_opts(cfg, balance_bias, score_mean),
+                           _ptr(x, "x", (cfg.T, cfg.d), et),
                            _ptr(w_router, "w_router", (cfg.E, cfg.d), et),
                            _ptr(w_shared_gate, "w_shared_gate", (cfg.d,), et), _ptr(ids, "ids"),
                            _ptr(gates, "gates"), _ptr(probs, "probs"), _ptr(sg, "shared_gate"), _ptr(ws, "ws"),
@@ -262,15 +290,17 @@ def combine_noalloc(cfg: MoEConfig, act, w_down, offsets, sorted_rows, gates, y=
 
 
 def forward(cfg: MoEConfig, x, w_router, w_gate, w_up, w_down, sh_gate=None, sh_up=None, sh_down=None,
-            w_shared_gate=None, y=None, ws=None, stream=None):
-    """The whole layer.  Returns y[T,d] (allocated unless given); ws is allocated if not given."""
+            w_shared_gate=None, y=None, ws=None, stream=None, balance_bias=None, score_mean=None):
+    """The whole layer.  Returns y[T,d] (allocated unless given); ws is allocated if not given.
+    balance_bias / score_mean: the routing options (see route())."""
     et = _elem_dtype(cfg)
     if y is None:
         y = torch.empty(cfg.T, cfg.d, dtype=et, device=x.device)
     if ws is None:
         ws = alloc_workspace(cfg, x.device)
     hs = cfg.h_shared
-    _check(lib().moe_forward(ctypes.byref(cfg), _ptr(x, "x", (cfg.T, cfg.d), et),
+    _check(lib().moe_forward(ctypes.byref(cfg), route_opts(cfg, balance_bias, score_mean),
+                             _ptr(x, "x", (cfg.T, cfg.d), et),
                              _ptr(w_router, "w_router", (cfg.E, cfg.d), et),
                              _ptr(w_gate, "w_gate", (cfg.E, cfg.h, cfg.d), et),
                              _ptr(w_up, "w_up", (cfg.E, cfg.h, cfg.d), et),
@@ -282,10 +312,31 @@ def forward(cfg: MoEConfig, x, w_router, w_gate, w_up, w_down, sh_gate=None, sh_
     return y
 
 
-def forward_layer(cfg: MoEConfig, layer, y=None, ws=None, stream=None):
+def forward_layer(cfg: MoEConfig, layer, y=None, ws=None, stream=None, balance_bias=None, score_mean=None):
     """moe_forward on a synth.Layer (device tensors)."""
     return forward(cfg, layer.x, layer.w_router, layer.w_gate, layer.w_up, layer.w_down, layer.sh_gate,
-                   layer.sh_up, layer.sh_down, layer.w_shared_gate, y=y, ws=ws, stream=stream)
+                   layer.sh_up, layer.sh_down, layer.w_shared_gate, y=y, ws=ws, stream=stream,
+                   balance_bias=balance_bias, score_mean=score_mean)
+
+
+def update_bias(cfg: MoEConfig, counts, lr: float, bias, stream=None):
+    """moe_update_bias: bias[E] (float32, in place) += lr * sign(mean(counts) - counts)."""
+    _check(lib().moe_update_bias(ctypes.byref(cfg), _ptr(counts, "counts", (cfg.E,), torch.int32),
+                                 ctypes.c_float(lr), _ptr(bias, "bias", (cfg.E,), torch.float32),
+                                 _stream(stream)), "moe_update_bias")
+    return bias
+
+
+def balance_loss(cfg: MoEConfig, counts, score_mean, alpha: float, want_frac=False, stream=None):
+    """moe_balance_loss: returns (loss[1] float32, f[E] float32 | None) on the device."""
+    dev = counts.device
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    frac = torch.empty(cfg.E, dtype=torch.float32, device=dev) if want_frac else None
+    _check(lib().moe_balance_loss(ctypes.byref(cfg), _ptr(counts, "counts", (cfg.E,), torch.int32),
+                                  _ptr(score_mean, "score_mean", (cfg.E,), torch.float32),
+                                  ctypes.c_float(alpha), _ptr(frac, "frac"), _ptr(loss, "loss"),
+                                  _stream(stream)), "moe_balance_loss")
+    return loss, frac
 
 
 def device_status(stream=None) -> int:
@@ -327,3 +378,126 @@ class StageEvents:
     def stage_ms(self) -> dict:
         """Per-stage milliseconds of the last recorded moe_forward (call after a synchronize)."""
         return {n: self.events[i].elapsed_time(self.events[i + 1]) for i, n in enumerate(STAGES)}
+
+
+# ----------------------------------------------------------------------------- training
+
+def train_workspace_size(cfg: MoEConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_train_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "moe_train_workspace_size")
+    return n.value
+
+
+def alloc_train_workspace(cfg: MoEConfig, device=None) -> torch.Tensor:
+    """A uint8 device tensor of moe_train_workspace_size bytes."""
+    return torch.empty(max(train_workspace_size(cfg), 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def forward_train(cfg: MoEConfig, layer, ws, y=None, stream=None, balance_bias=None, score_mean=None):
+    """moe_forward_train on a synth.Layer: y[T,d]; ws (alloc_train_workspace) keeps what
+    backward() needs."""
+    et = _elem_dtype(cfg)
+    if y is None:
+        y = torch.empty(cfg.T, cfg.d, dtype=et, device=layer.x.device)
+    hs = cfg.h_shared
+    _check(lib().moe_forward_train(ctypes.byref(cfg), route_opts(cfg, balance_bias, score_mean),
+                                   _ptr(layer.x, "x", (cfg.T, cfg.d), et),
+                                   _ptr(layer.w_router, "w_router", (cfg.E, cfg.d), et),
+                                   _ptr(layer.w_gate, "w_gate", (cfg.E, cfg.h, cfg.d), et),
+                                   _ptr(layer.w_up, "w_up", (cfg.E, cfg.h, cfg.d), et),
+                                   _ptr(layer.w_down, "w_down", (cfg.E, cfg.d, cfg.h), et),
+                                   _ptr(layer.sh_gate, "sh_gate", (hs, cfg.d), et),
+                                   _ptr(layer.sh_up, "sh_up", (hs, cfg.d), et),
+                                   _ptr(layer.sh_down, "sh_down", (cfg.d, hs), et),
+                                   _ptr(layer.w_shared_gate, "w_shared_gate", (cfg.d,), et),
+                                   _ptr(y, "y", (cfg.T, cfg.d), et), _ptr(ws, "ws", dtype=torch.uint8), ws.numel(),
+                                   _stream(stream)), "moe_forward_train")
+    return y
+
+
+def backward(cfg: MoEConfig, layer, dy, ws, grads=None, stream=None) -> dict:
+    """moe_backward after forward_train(cfg, layer, ws): the gradients (allocated
+    unless ``grads`` holds them) dx, dw_router (fp32), dw_gate, dw_up, dw_down and,
+    with a shared expert, dsh_gate, dsh_up, dsh_down, dw_shared_gate (fp32)."""
+    et = _elem_dtype(cfg)
+    dev = layer.x.device
+    hs = cfg.h_shared
+    if grads is None:
+        grads = {"dx": torch.empty(cfg.T, cfg.d, dtype=et, device=dev),
+                 "dw_router": torch.empty(cfg.E, cfg.d, dtype=torch.float32, device=dev),
+                 "dw_gate": torch.empty(cfg.E, cfg.h, cfg.d, dtype=et, device=dev),
+                 "dw_up": torch.empty(cfg.E, cfg.h, cfg.d, dtype=et, device=dev),
+                 "dw_down": torch.empty(cfg.E, cfg.d, cfg.h, dtype=et, device=dev)}
+        if hs:
+            grads.update(dsh_gate=torch.empty(hs, cfg.d, dtype=et, device=dev),
+                         dsh_up=torch.empty(hs, cfg.d, dtype=et, device=dev),
+                         dsh_down=torch.empty(cfg.d, hs, dtype=et, device=dev),
+                         dw_shared_gate=torch.empty(cfg.d, dtype=torch.float32, device=dev))
+    g = grads
+    _check(lib().moe_backward(ctypes.byref(cfg), _ptr(layer.x, "x", (cfg.T, cfg.d), et),
+                              _ptr(layer.w_router, "w_router", (cfg.E, cfg.d), et),
+                              _ptr(layer.w_gate, "w_gate", (cfg.E, cfg.h, cfg.d), et),
+                              _ptr(layer.w_up, "w_up", (cfg.E, cfg.h, cfg.d), et),
+                              _ptr(layer.w_down, "w_down", (cfg.E, cfg.d, cfg.h), et),
+                              _ptr(layer.sh_gate, "sh_gate", (hs, cfg.d), et),
+                              _ptr(layer.sh_up, "sh_up", (hs, cfg.d), et),
+                              _ptr(layer.sh_down, "sh_down", (cfg.d, hs), et),
+                              _ptr(layer.w_shared_gate, "w_shared_gate", (cfg.d,), et),
+                              _ptr(dy, "dy", (cfg.T, cfg.d), et), _ptr(ws, "ws", dtype=torch.uint8), ws.numel(),
+                              _ptr(g["dx"], "dx", (cfg.T, cfg.d), et),
+                              _ptr(g["dw_router"], "dw_router", (cfg.E, cfg.d), torch.float32),
+                              _ptr(g["dw_gate"], "dw_gate", (cfg.E, cfg.h, cfg.d), et),
+                              _ptr(g["dw_up"], "dw_up", (cfg.E, cfg.h, cfg.d), et),
+                              _ptr(g["dw_down"], "dw_down", (cfg.E, cfg.d, cfg.h), et),
+                              _ptr(g.get("dsh_gate"), "dsh_gate", (hs, cfg.d), et),
+                              _ptr(g.get("dsh_up"), "dsh_up", (hs, cfg.d), et),
+                              _ptr(g.get("dsh_down"), "dsh_down", (cfg.d, hs), et),
+                              _ptr(g.get("dw_shared_gate"), "dw_shared_gate", (cfg.d,), torch.float32),
+                              _stream(stream)), "moe_backward")
+    return grads
+
+
+# ----------------------------------------------------------------------------- 4-bit routed experts
+
+def quantize_q4(w: torch.Tensor, stream=None):
+    """moe_quantize_q4 of a [..., cols] bf16/fp32 CUDA tensor: (codes uint8
+    [..., cols / 2], scales float32 [..., cols / 64])."""
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    q = torch.empty(*w.shape[:-1], cols // 2, dtype=torch.uint8, device=w.device)
+    sc = torch.empty(*w.shape[:-1], cols // 64, dtype=torch.float32, device=w.device)
+    _check(lib().moe_quantize_q4(_ptr(w, "w"), 1 if w.dtype == torch.float32 else 0, rows, cols, _ptr(q, "q"),
+                                 _ptr(sc, "scales"), _stream(stream)), "moe_quantize_q4")
+    return q, sc
+
+
+def quantize_experts_q4(layer, stream=None) -> dict:
+    """The routed experts of a synth.Layer in 4 bits: {"q_gate", "s_gate", "q_up", "s_up", "q_down", "s_down"}."""
+    out = {}
+    for name, w in (("gate", layer.w_gate), ("up", layer.w_up), ("down", layer.w_down)):
+        out["q_" + name], out["s_" + name] = quantize_q4(w, stream)
+    return out
+
+
+def forward_q4(cfg: MoEConfig, layer, q4: dict, y=None, ws=None, stream=None, balance_bias=None, score_mean=None):
+    """moe_forward_q4: the layer with 4-bit routed experts (q4 from quantize_experts_q4)."""
+    et = _elem_dtype(cfg)
+    if y is None:
+        y = torch.empty(cfg.T, cfg.d, dtype=et, device=layer.x.device)
+    if ws is None:
+        ws = alloc_workspace(cfg, layer.x.device)
+    hs = cfg.h_shared
+    E, h, d = cfg.E, cfg.h, cfg.d
+    _check(lib().moe_forward_q4(ctypes.byref(cfg), route_opts(cfg, balance_bias, score_mean),
+                                _ptr(layer.x, "x", (cfg.T, d), et), _ptr(layer.w_router, "w_router", (E, d), et),
+                                _ptr(q4["q_gate"], "q_gate", (E, h, d // 2), torch.uint8),
+                                _ptr(q4["s_gate"], "s_gate", (E, h, d // 64), torch.float32),
+                                _ptr(q4["q_up"], "q_up", (E, h, d // 2), torch.uint8),
+                                _ptr(q4["s_up"], "s_up", (E, h, d // 64), torch.float32),
+                                _ptr(q4["q_down"], "q_down", (E, d, h // 2), torch.uint8),
+                                _ptr(q4["s_down"], "s_down", (E, d, h // 64), torch.float32),
+                                _ptr(layer.sh_gate, "sh_gate", (hs, d), et), _ptr(layer.sh_up, "sh_up", (hs, d), et),
+                                _ptr(layer.sh_down, "sh_down", (d, hs), et),
+                                _ptr(layer.w_shared_gate, "w_shared_gate", (d,), et), _ptr(y, "y", (cfg.T, d), et),
+                                _ptr(ws, "ws", dtype=torch.uint8), ws.numel(), _stream(stream)), "moe_forward_q4")
+    return y

@@ -1,0 +1,391 @@
+// moe_backward: the gradient of the MoE layer after moe_forward_train.
+//
+// The chain rule through the forward's steps (the layer of "Tutorial 11:
+// Mixture of Experts (MoE)", sections 2-4, with the sigmoid scores, shared
+// expert and balance bias of "Small MoE Architecture, in depth", SmallMoE;
+// "Small models, sparse experts", "Dispatch decides everything" trains it):
+//
+//   1. routed experts, rows grouped by expert:  r = W_down^T dy;  the gate
+//      gradient r . a;  du, dv through silu(u) * v;  gate * a kept for dW_down
+//      (grouped_bwd.cu, SWIGLU)
+//   2. the shared expert, the same on one dense segment with gate sigmoid(w_s.x)
+//   3. router: the gate gradients through the (renormalised) softmax or the
+//      sigmoid to the logits (router_bwd_kernel, one warp per token)
+//   4. dx: W_gate^T du + W_up^T dv added into token order (SCATTER), the
+//      shared expert's, and dl W_router; then fp32 -> bf16 with the shared
+//      gate's w_s term (finalize_dx_kernel)
+//   5. weight gradients: dW_down, dW_gate / dW_up per expert over its rows,
+//      the shared expert's over all tokens, dW_router = dl^T x (WEIGHT), and
+//      dw_s = sum_t dl_s x_t (shared_gate_grad_kernel)
+//
+// The top-k selection (and the balance bias) passes no gradient.
+#include <algorithm>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+struct RouterBwdArgs {
+    int64_t T;
+    int E, k, norm_topk, score, ep;   // ep: row stride of dl
+    const int32_t *ids;
+    const float *gates, *probs, *dgate;
+    const float *sg, *dsg;            // shared gate and its gradient (or null)
+    __nv_bfloat16 *dl;                // [T, ep] out, zero past E
+    float *dls;                       // [T] out: gradient of the shared gate's logit (or null)
+};
+
+// One warp per token.  q_j = s_{ids_j} are the kept raw scores; with
+// renormalisation g_j = q_j / Q and dq_j = (dg_j - sum_i dg_i g_i) / Q, else
+// dq_j = dg_j.  ds is dq on the kept experts and 0 elsewhere; softmax:
+// dl_e = s_e (ds_e - sum_e' s_e' ds_e'), sigmoid: dl_e = ds_e s_e (1 - s_e).
+__global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+    if (t >= a.T) return;
+    const float *s = a.probs + t * a.E;
+    int id = -1;
+    float dg = 0.f, g = 0.f, q = 0.f;
+    if (lane < a.k) {
+        id = a.ids[t * a.k + lane];
+        if (id < 0 || id >= a.E) id = -1;
+        dg = a.dgate[t * a.k + lane];
+        g = a.gates[t * a.k + lane];
+        q = id >= 0 ? s[id] : 0.f;
+    }
+    const float Q = warp_sum(q);
+    const float dot = warp_sum(dg * g);
+    const float dq = a.norm_topk ? (dg - dot) / Q : dg;
+    const bool sigm = a.score == MOE_SCORE_SIGMOID;
+    const float sd = sigm ? 0.f : warp_sum(id >= 0 ? q * dq : 0.f);   // sum_e s_e ds_e
+    // every lane takes the k (id, dq) pairs (a uniform loop, so all lanes shuffle)
+    int idj[MOE_MAX_TOPK];
+    float dqj[MOE_MAX_TOPK];
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+        idj[j] = -1;
+        dqj[j] = 0.f;
+        if (j < a.k) {
+            idj[j] = __shfl_sync(0xffffffffu, id, j);
+            dqj[j] = __shfl_sync(0xffffffffu, dq, j);
+        }
+    }
+    for (int e = lane; e < a.ep; e += 32) {
+        float ds = 0.f;
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_TOPK; ++j)
+            if (idj[j] == e) ds = dqj[j];
+        float dl = 0.f;
+        if (e < a.E) dl = sigm ? ds * s[e] * (1.f - s[e]) : s[e] * (ds - sd);
+        a.dl[t * a.ep + e] = __float2bfloat16_rn(dl);
+    }
+    if (lane == 0 && a.dls) a.dls[t] = a.dsg[t] * a.sg[t] * (1.f - a.sg[t]);
+}
+
+// dx[t, i] = bf16(acc[t, i] + dls[t] * w_s[i]) (the w_s term only with a shared expert).
+__global__ void finalize_dx_kernel(const float *acc, const float *dls, const __nv_bfloat16 *ws, __nv_bfloat16 *dx,
+                                   int64_t T, int d) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t n = T * d;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float v = acc[i];
+        if (dls) v += dls[i / d] * __bfloat162float(ws[i % d]);
+        dx[i] = __float2bfloat16_rn(v);
+    }
+}
+
+// dw_s[i] = sum over t (in increasing order) of dls[t] * x[t, i].
+__global__ void shared_gate_grad_kernel(const float *dls, const __nv_bfloat16 *x, float *dws, int64_t T, int d) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= d) return;
+    float s = 0.f;
+    for (int64_t t = 0; t < T; ++t) s = fmaf(dls[t], __bfloat162float(x[t * d + i]), s);
+    dws[i] = s;
+}
+
+cudaError_t set0(void *p, size_t bytes, cudaStream_t s) { return p && bytes ? cudaMemsetAsync(p, 0, bytes, s) : cudaSuccess; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status moe_backward(const moe_config *c, const void *x, const void *w_router, const void *w_gate,
+                                   const void *w_up, const void *w_down, const void *sh_gate, const void *sh_up,
+                                   const void *sh_down, const void *w_shared_gate, const void *dy, void *ws,
+                                   size_t ws_bytes, void *dx, float *dw_router, void *dw_gate, void *dw_up,
+                                   void *dw_down, void *dsh_gate, void *dsh_up, void *dsh_down,
+                                   float *dw_shared_gate, void *stream) {
+    moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!dw_router || !dw_gate || !dw_up || !dw_down || !w_router || !w_gate || !w_up || !w_down)
+        return MOE_ERR_INVALID_ARG;
+    const bool shared = c->h_shared > 0;
+    if (shared && (!sh_gate || !sh_up || !sh_down || !w_shared_gate || !dsh_gate || !dsh_up || !dsh_down ||
+                   !dw_shared_gate))
+        return MOE_ERR_INVALID_ARG;
+    if (c->T > 0 && (!x || !dy || !dx)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*c, true);
+    if (c->T > 0 && (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255))) return MOE_ERR_WORKSPACE;
+    uint32_t *err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t T = c->T, R = T * c->k;
+    const int d = c->d, E = c->E, h = c->h, hs = c->h_shared, ep = dl_stride(E);
+    if (T == 0) {
+        // no tokens: every weight gradient is zero
+        cudaError_t e = set0(dw_router, sizeof(float) * (size_t)E * d, s);
+        if (e == cudaSuccess) e = set0(dw_gate, 2 * (size_t)E * h * d, s);
+        if (e == cudaSuccess) e = set0(dw_up, 2 * (size_t)E * h * d, s);
+        if (e == cudaSuccess) e = set0(dw_down, 2 * (size_t)E * d * h, s);
+        if (shared) {
+            if (e == cudaSuccess) e = set0(dsh_gate, 2 * (size_t)hs * d, s);
+            if (e == cudaSuccess) e = set0(dsh_up, 2 * (size_t)hs * d, s);
+            if (e == cudaSuccess) e = set0(dsh_down, 2 * (size_t)d * hs, s);
+            if (e == cudaSuccess) e = set0(dw_shared_gate, sizeof(float) * d, s);
+        }
+        return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
+
+    const int32_t *ids = ws_part<int32_t>(ws, L, P_IDS);
+    const float *gates = ws_part<float>(ws, L, P_GATES);
+    const float *sg = ws_part<float>(ws, L, P_SG);
+    const int32_t *offsets = ws_part<int32_t>(ws, L, P_OFFSETS);
+    const int32_t *srt = ws_part<int32_t>(ws, L, P_SORTED);
+    const float *probs = ws_part<float>(ws, L, P_PROBS);
+    char *hpre = ws_part<char>(ws, L, P_HPRE);
+    char *hpres = ws_part<char>(ws, L, P_HPRES);
+    float *dg = ws_part<float>(ws, L, P_DG);
+    float *dsg = ws_part<float>(ws, L, P_DSG);
+    char *dh = ws_part<char>(ws, L, P_DH);
+    char *dhs = ws_part<char>(ws, L, P_DHS);
+    void *ga = ws_part<void>(ws, L, P_ACT);      // gate * a of the routed rows (act is not needed any more)
+    void *gas = ws_part<void>(ws, L, P_GAS);
+    void *dlb = ws_part<void>(ws, L, P_DLB);
+    float *dls = ws_part<float>(ws, L, P_DLS);
+    float *acc = ws_part<float>(ws, L, P_YACC);  // the dx accumulator
+
+    cudaError_t e = set0(dg, sizeof(float) * R, s);
+    if (e == cudaSuccess) e = set0(dsg, shared ? sizeof(float) * T : 0, s);
+    if (e == cudaSuccess) e = set0(acc, sizeof(float) * T * d, s);
+
+    auto base = [](const BwdGemm::Kind kind) {
+        BwdGemm g{};
+        g.kind = kind;
+        return g;
+    };
+    // 1. routed: r = W_down^T dy over grouped rows (dy gathered by token)
+    if (e == cudaSuccess) {
+        BwdGemm g = base(BwdGemm::SWIGLU);
+        g.gather_a = true;
+        g.b0 = {w_down, (uint64_t)E * d, (uint64_t)h, (uint64_t)h};
+        g.offsets = offsets;
+        g.sorted_rows = srt;
+        g.groups = E;
+        g.k = c->k;
+        g.rows = R;
+        g.T = T;
+        g.nranges = 1;
+        g.Kr = d;
+        g.N = h;
+        g.gsrc = dy;
+        g.gwidth = d;
+        g.hpre = hpre;
+        g.gate = gates;
+        g.dh = dh;
+        g.ga = ga;
+        g.dgate = dg;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    // 2. shared expert: the same on the dense segment (gate sigmoid(w_s . x))
+    if (e == cudaSuccess && shared) {
+        BwdGemm g = base(BwdGemm::SWIGLU);
+        g.a0 = {dy, (uint64_t)T, (uint64_t)d, (uint64_t)d};
+        g.b0 = {sh_down, (uint64_t)d, (uint64_t)hs, (uint64_t)hs};
+        g.groups = 1;
+        g.k = 1;
+        g.rows = T;
+        g.T = T;
+        g.nranges = 1;
+        g.Kr = d;
+        g.N = hs;
+        g.hpre = hpres;
+        g.gate = sg;
+        g.dh = dhs;
+        g.ga = gas;
+        g.dgate = dsg;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    // 3. router: gate gradients -> logit gradients
+    if (e == cudaSuccess) {
+        RouterBwdArgs a{T, E, c->k, c->norm_topk, c->score, ep, ids, gates, probs, dg, shared ? sg : nullptr,
+                        shared ? dsg : nullptr, static_cast<__nv_bfloat16 *>(dlb), shared ? dls : nullptr};
+        e = launch_kernel(router_bwd_kernel, (unsigned)((T + 7) / 8), 256, 0, s, a);
+    }
+    // 4. dx: the routed experts' gate/up (two K ranges: du with W_gate, dv with W_up), the shared expert's,
+    //    and the router's
+    if (e == cudaSuccess) {
+        BwdGemm g = base(BwdGemm::SCATTER);
+        g.a0 = {dh, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
+        g.a1 = {dh + (size_t)h * 2, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
+        g.b0 = {w_gate, (uint64_t)E * h, (uint64_t)d, (uint64_t)d};
+        g.b1 = {w_up, (uint64_t)E * h, (uint64_t)d, (uint64_t)d};
+        g.offsets = offsets;
+        g.sorted_rows = srt;
+        g.groups = E;
+        g.k = c->k;
+        g.rows = R;
+        g.T = T;
+        g.nranges = 2;
+        g.Kr = h;
+        g.N = d;
+        g.acc = acc;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess && shared) {
+        BwdGemm g = base(BwdGemm::SCATTER);
+        g.a0 = {dhs, (uint64_t)T, (uint64_t)hs, 2 * (uint64_t)hs};
+        g.a1 = {dhs + (size_t)hs * 2, (uint64_t)T, (uint64_t)hs, 2 * (uint64_t)hs};
+        g.b0 = {sh_gate, (uint64_t)hs, (uint64_t)d, (uint64_t)d};
+        g.b1 = {sh_up, (uint64_t)hs, (uint64_t)d, (uint64_t)d};
+        g.groups = 1;
+        g.k = 1;
+        g.rows = T;
+        g.T = T;
+        g.nranges = 2;
+        g.Kr = hs;
+        g.N = d;
+        g.acc = acc;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess) {
+        BwdGemm g = base(BwdGemm::SCATTER);
+        g.a0 = {dlb, (uint64_t)T, (uint64_t)E, (uint64_t)ep};
+        g.b0 = {w_router, (uint64_t)E, (uint64_t)d, (uint64_t)d};
+        g.groups = 1;
+        g.k = 1;
+        g.rows = T;
+        g.T = T;
+        g.nranges = 1;
+        g.Kr = E;
+        g.N = d;
+        g.acc = acc;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess) {
+        const int64_t n = T * d;
+        const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, 4LL * num_sms() * 8);
+        e = launch_kernel(finalize_dx_kernel, blocks, 256, 0, s, static_cast<const float *>(acc),
+                          static_cast<const float *>(shared ? dls : nullptr),
+                          static_cast<const __nv_bfloat16 *>(shared ? w_shared_gate : nullptr),
+                          static_cast<__nv_bfloat16 *>(dx), T, d);
+    }
+    // 5. weight gradients
+    if (e == cudaSuccess) {
+        // dW_down[e] = sum over the expert's rows of dy_t (x) (gate * a)
+        BwdGemm g = base(BwdGemm::WEIGHT);
+        g.gather_a = true;
+        g.b0 = {ga, (uint64_t)R, (uint64_t)h, (uint64_t)h};
+        g.offsets = offsets;
+        g.sorted_rows = srt;
+        g.groups = E;
+        g.k = c->k;
+        g.rows = R;
+        g.T = T;
+        g.M = d;
+        g.halves = 1;
+        g.N = h;
+        g.gsrc = dy;
+        g.gwidth = d;
+        g.out0 = dw_down;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess) {
+        // dW_gate[e] / dW_up[e] = sum over the expert's rows of du / dv (x) x_t
+        BwdGemm g = base(BwdGemm::WEIGHT);
+        g.gather_b = true;
+        g.a0 = {dh, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
+        g.a1 = {dh + (size_t)h * 2, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
+        g.offsets = offsets;
+        g.sorted_rows = srt;
+        g.groups = E;
+        g.k = c->k;
+        g.rows = R;
+        g.T = T;
+        g.M = h;
+        g.halves = 2;
+        g.N = d;
+        g.gsrc = x;
+        g.gwidth = d;
+        g.out0 = dw_gate;
+        g.out1 = dw_up;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess && shared) {
+        BwdGemm g = base(BwdGemm::WEIGHT);
+        g.a0 = {dy, (uint64_t)T, (uint64_t)d, (uint64_t)d};
+        g.b0 = {gas, (uint64_t)T, (uint64_t)hs, (uint64_t)hs};
+        g.groups = 1;
+        g.k = 1;
+        g.rows = T;
+        g.T = T;
+        g.M = d;
+        g.halves = 1;
+        g.N = hs;
+        g.out0 = dsh_down;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess && shared) {
+        BwdGemm g = base(BwdGemm::WEIGHT);
+        g.a0 = {dhs, (uint64_t)T, (uint64_t)hs, 2 * (uint64_t)hs};
+        g.a1 = {dhs + (size_t)hs * 2, (uint64_t)T, (uint64_t)hs, 2 * (uint64_t)hs};
+        g.b0 = {x, (uint64_t)T, (uint64_t)d, (uint64_t)d};
+        g.groups = 1;
+        g.k = 1;
+        g.rows = T;
+        g.T = T;
+        g.M = hs;
+        g.halves = 2;
+        g.N = d;
+        g.out0 = dsh_gate;
+        g.out1 = dsh_up;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess) {
+        // dW_router = dl^T x
+        BwdGemm g = base(BwdGemm::WEIGHT);
+        g.a0 = {dlb, (uint64_t)T, (uint64_t)E, (uint64_t)ep};
+        g.b0 = {x, (uint64_t)T, (uint64_t)d, (uint64_t)d};
+        g.groups = 1;
+        g.k = 1;
+        g.rows = T;
+        g.T = T;
+        g.M = E;
+        g.halves = 1;
+        g.N = d;
+        g.out0 = dw_router;
+        g.out_f32 = true;
+        g.err = err;
+        e = launch_bwd_gemm(g, s);
+    }
+    if (e == cudaSuccess && shared)
+        e = launch_kernel(shared_gate_grad_kernel, (unsigned)((d + 127) / 128), 128, 0, s,
+                          static_cast<const float *>(dls), static_cast<const __nv_bfloat16 *>(x), dw_shared_gate, T, d);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

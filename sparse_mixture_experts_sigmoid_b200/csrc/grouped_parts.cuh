@@ -36,11 +36,32 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
     if constexpr (MODE == GATEUP) {
         if (!__any_sync(0xffffffffu, valid)) return;   // no row of this warp lies in the segment
         T *act = static_cast<T *>(p.act);
-        // silu(g) * u for 16 output columns from column c of the tile
+        // silu(g) * u for 16 output columns from column c of the tile (and, in
+        // training, g and u themselves into the pre-activation rows)
         auto store16 = [&](int c, const float(&g)[16], const float(&u)[16]) {
             const int col = n * BN_OUT + c;
             if (!valid || col >= p.N) return;
             T *dst = act + r * p.N + col;
+            if constexpr (sizeof(T) == 2) {
+                if (p.hpre) {
+                    T *hg = static_cast<T *>(p.hpre) + r * 2 * (int64_t)p.N + col;
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        if (col + 8 * h8 >= p.N) continue;
+                        uint32_t wg[4], wu[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int i0 = 8 * h8 + 2 * q;
+                            __nv_bfloat162 a2 = __floats2bfloat162_rn(g[i0], g[i0 + 1]);
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(u[i0], u[i0 + 1]);
+                            wg[q] = *reinterpret_cast<uint32_t *>(&a2);
+                            wu[q] = *reinterpret_cast<uint32_t *>(&b2);
+                        }
+                        *reinterpret_cast<uint4 *>(hg + 8 * h8) = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+                        *reinterpret_cast<uint4 *>(hg + p.N + 8 * h8) = make_uint4(wu[0], wu[1], wu[2], wu[3]);
+                    }
+                }
+            }
 #pragma unroll
             for (int h8 = 0; h8 < 2; ++h8) {
                 if (col + 8 * h8 >= p.N) continue;
@@ -80,13 +101,20 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
         int t = -1;
         float gate = 0.f;
         if (valid) {
+            // gates == nullptr: every row is added with weight 1
             if (p.sorted_rows) {
+                // range-check the assignment before deriving its token: a value in
+                // (-k, 0) would otherwise truncate to token 0
                 const int v = p.sorted_rows[r];
-                t = v / p.k;
-                gate = (v >= 0 && v < p.rows) ? p.gates[v] : 0.f;
+                if (v >= 0 && v < p.rows) {
+                    t = v / p.k;
+                    gate = p.gates ? p.gates[v] : 1.f;
+                } else {
+                    t = -2;   // reported below
+                }
             } else {
                 t = (int)r;
-                gate = p.gates[r];
+                gate = p.gates ? p.gates[r] : 1.f;
             }
             if (t < 0 || t >= p.T) {
                 atomicOr(p.err, kErrInput);

@@ -18,6 +18,8 @@ std::mutex g_mu;
 uint32_t *g_err_ptr[kMaxDevices];
 int g_sms[kMaxDevices];
 
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
 int current_device() {
     int d = 0;
     if (cudaGetDevice(&d) != cudaSuccess) return -1;
@@ -37,22 +39,19 @@ uint32_t *err_ptr() {
     return g_err_ptr[dev];
 }
 
-size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
-
-enum Part { P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_PERM, P_LOGITS, P_N };
-
-struct Layout {
-    size_t off[P_N];
-    size_t size[P_N];
-    size_t total;
-};
+using Layout = WsLayout;
+using Part = WsPart;
 
 // Scratch of the tensor-core router (fp32 logits), 0 when the CUDA-core router runs.
 size_t router_scratch_bytes(const moe_config &c) {
     return router_tc_supported(c.T, c.E, c.dtype) ? router_tc_workspace_bytes(c.T, c.d, c.E, c.h_shared > 0) : 0;
 }
+// Per-CTA score sums of the score-mean statistic.
+size_t router_stats_bytes(const moe_config &c) { return sizeof(float) * (size_t)router_stats_rows(c.T) * c.E; }
+// moe_route's scratch: the logits part, then (256-byte aligned) the statistic part.
+size_t route_ws_total(const moe_config &c) { return align256(router_scratch_bytes(c)) + router_stats_bytes(c); }
 
-Layout make_layout(const moe_config &c) {
+Layout make_layout(const moe_config &c, bool train = false) {
     Layout L{};
     const size_t R = (size_t)c.T * c.k, esz = c.dtype == MOE_F32 ? 4 : 2;
     L.size[P_IDS] = R * 4;
@@ -67,6 +66,22 @@ Layout make_layout(const moe_config &c) {
     L.size[P_YACC] = c.dtype == MOE_BF16 ? (size_t)c.T * c.d * 4 : 0;
     L.size[P_PERM] = permute_workspace_bytes((int64_t)R, c.E);
     L.size[P_LOGITS] = router_scratch_bytes(c);
+    L.size[P_STATS] = router_stats_bytes(c);
+    if (train) {
+        // kept for the backward pass (ga reuses act, the dx accumulator reuses y_acc)
+        const size_t hs = (size_t)c.h_shared;
+        L.size[P_PROBS] = (size_t)c.T * c.E * 4;
+        L.size[P_HPRE] = R * 2 * (size_t)c.h * esz;
+        L.size[P_HPRES] = (size_t)c.T * 2 * hs * esz;
+        L.size[P_DG] = R * 4;
+        L.size[P_DSG] = hs ? (size_t)c.T * 4 : 0;
+        L.size[P_DH] = R * 2 * (size_t)c.h * esz;
+        L.size[P_DHS] = (size_t)c.T * 2 * hs * esz;
+        L.size[P_GAS] = (size_t)c.T * hs * esz;
+        L.size[P_DLB] = (size_t)c.T * dl_stride(c.E) * 2;
+        L.size[P_DLS] = hs ? (size_t)c.T * 4 : 0;
+        if (c.dtype == MOE_BF16 && L.size[P_YACC] == 0) L.size[P_YACC] = (size_t)c.T * c.d * 4;
+    }
     size_t o = 0;
     for (int i = 0; i < P_N; ++i) {
         L.off[i] = o;
@@ -78,7 +93,7 @@ Layout make_layout(const moe_config &c) {
 
 template <typename T>
 T *part(void *ws, const Layout &L, Part p) {
-    return L.size[p] ? reinterpret_cast<T *>(static_cast<char *>(ws) + L.off[p]) : nullptr;
+    return ws_part<T>(ws, L, p);
 }
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -195,10 +210,25 @@ GemmLaunch gemm_down_dense(const moe_config &c, const void *act, const void *wd,
 }
 bool use_gemm(const moe_config &c) { return c.T * c.k > kDecodeMaxRows; }
 
+// The fused expert kernel (gate/up, SwiGLU, down and combine in one pass over
+// the weights) when the experts average at most one 128-row tile and the
+// hidden width is a multiple of its 128-column slices.  MOE_FUSED=1 / 0
+// forces it on (where the shape allows) / off.
+bool use_fused(const moe_config &c) {
+    static const int force = [] {
+        const char *v = std::getenv("MOE_FUSED");
+        return v ? (v[0] == '1' ? 1 : 0) : -1;
+    }();
+    if (c.dtype != MOE_BF16 || c.h % 128 != 0) return false;
+    if (force >= 0) return force == 1;
+    return fused_expert_supported(c);
+}
+
 
 }  // namespace
 
 uint32_t *device_error_word() { return err_ptr(); }
+WsLayout ws_layout(const moe_config &c, bool train) { return make_layout(c, train); }
 bool gemm_path(const moe_config &c) { return use_gemm(c); }
 GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const int32_t *offsets,
                      const int32_t *srt, const float *gates, float *acc, uint32_t *err) {
@@ -294,19 +324,22 @@ moe_status moe_route_workspace_size(const moe_config *c, size_t *bytes) {
     if (!bytes) return MOE_ERR_INVALID_ARG;
     const moe_status st = moe_validate(c);
     if (st != MOE_OK) return st;
-    *bytes = router_scratch_bytes(*c);
+    *bytes = route_ws_total(*c);
     return MOE_OK;
 }
 
-moe_status moe_route(const moe_config *c, const void *x, const void *w_router, const void *w_shared_gate,
-                     int32_t *ids, float *gates, float *probs, float *shared_gate, void *ws, size_t ws_bytes,
-                     void *stream) {
+moe_status moe_route(const moe_config *c, const moe_route_opts *opts, const void *x, const void *w_router,
+                     const void *w_shared_gate, int32_t *ids, float *gates, float *probs, float *shared_gate,
+                     void *ws, size_t ws_bytes, void *stream) {
     moe_status st = moe_validate(c);
     if (st != MOE_OK) return st;
     if (c->T == 0) return MOE_OK;
     if (!x || !w_router || !ids || !gates) return MOE_ERR_INVALID_ARG;
     if (shared_gate && !w_shared_gate) return MOE_ERR_INVALID_ARG;
-    const size_t need = router_scratch_bytes(*c);
+    const bool stats = opts && opts->score_mean;
+    const size_t logits = router_scratch_bytes(*c);
+    // the statistic part is needed only when the statistic is asked for
+    const size_t need = stats ? route_ws_total(*c) : logits;
     if (need && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255))) return MOE_ERR_WORKSPACE;
     RouterArgs a{};
     a.x = x;
@@ -323,9 +356,12 @@ moe_status moe_route(const moe_config *c, const void *x, const void *w_router, c
     a.probs = probs;
     a.shared_gate = shared_gate;
     a.zero_rows = nullptr;
+    a.bias = opts ? opts->balance_bias : nullptr;
+    a.score_mean = stats ? opts->score_mean : nullptr;
+    a.stats = stats ? reinterpret_cast<float *>(static_cast<char *>(ws) + align256(logits)) : nullptr;
     a.err = err_ptr();
     if (!a.err) return MOE_ERR_CUDA;
-    return cuda_status(launch_router(a, c->dtype, need ? static_cast<float *>(ws) : nullptr,
+    return cuda_status(launch_router(a, c->dtype, logits ? static_cast<float *>(ws) : nullptr,
                                      static_cast<cudaStream_t>(stream)));
 }
 
@@ -406,17 +442,24 @@ moe_status moe_combine(const moe_config *c, const void *act, const void *w_down,
     return cuda_status(e);
 }
 
-moe_status moe_forward(const moe_config *c, const void *x, const void *w_router, const void *w_gate,
-                       const void *w_up, const void *w_down, const void *sh_gate, const void *sh_up,
-                       const void *sh_down, const void *w_shared_gate, void *y, void *ws, size_t ws_bytes,
-                       void *stream) {
+}  // extern "C"
+
+namespace moe {
+// The forward pass; `train` also keeps what moe_backward needs (the full score
+// rows and the pre-activations of every grouped row) and always takes the
+// tensor-core path, whose gate/up epilogue writes them.
+moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const void *x, const void *w_router,
+                        const void *w_gate, const void *w_up, const void *w_down, const void *sh_gate,
+                        const void *sh_up, const void *sh_down, const void *w_shared_gate, void *y, void *ws,
+                        size_t ws_bytes, void *stream, bool train) {
     moe_status st = moe_validate(c);
     if (st != MOE_OK) return st;
+    if (train && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     if (c->T == 0) return MOE_OK;
     if (!x || !w_router || !w_gate || !w_up || !w_down || !y) return MOE_ERR_INVALID_ARG;
     const bool shared = c->h_shared > 0;
     if (shared && (!sh_gate || !sh_up || !sh_down || !w_shared_gate)) return MOE_ERR_INVALID_ARG;
-    const Layout L = make_layout(*c);
+    const Layout L = make_layout(*c, train);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
     uint32_t *err = err_ptr();
     if (!err) return MOE_ERR_CUDA;
@@ -446,10 +489,17 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     ra.score = c->score;
     ra.ids = ids;
     ra.gates = gates;
-    ra.probs = nullptr;
+    ra.probs = train ? part<float>(ws, L, P_PROBS) : nullptr;
     ra.shared_gate = sg;
-    ra.zero_rows = nullptr;   // the gate/up GEMM clears the accumulator; the small-batch path writes y
+    const bool gemm = train || use_gemm(*c);
+    const bool fused = gemm && !train && use_fused(*c);
+    // the fused expert kernel adds into the accumulator from its first unit on, so
+    // the router clears it; otherwise the gate/up GEMM does (the small-batch path writes y)
+    ra.zero_rows = fused ? acc : nullptr;
     ra.err = err;
+    ra.bias = opts ? opts->balance_bias : nullptr;
+    ra.score_mean = opts ? opts->score_mean : nullptr;
+    ra.stats = ra.score_mean ? part<float>(ws, L, P_STATS) : nullptr;
     // the tensor-core router also builds the grouping histogram
     const bool fused_hist = L.size[P_LOGITS] && c->T * c->k > permute_chunk();
     ra.hist = fused_hist ? part<int32_t>(ws, L, P_PERM) : nullptr;
@@ -466,12 +516,14 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     mark(1 + MOE_STAGE_PERMUTE, s);
     const Segments routed{offsets, srt, c->E, c->k, (int64_t)R};
     const Segments dense{nullptr, nullptr, 1, 1, c->T};
-    const bool gemm = use_gemm(*c);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && fused) {
+        e = launch_fused_expert(*c, x, w_gate, w_up, w_down, offsets, srt, gates, acc, err, s);
+    } else if (e == cudaSuccess) {
         SegGateUpArgs ga{x, w_gate, w_up, routed, c->T, c->d, c->h, act};
         GemmLaunch gl = gemm_gateup(*c, x, w_gate, w_up, offsets, srt, act, err);
         gl.p.zero = acc;   // the down GEMM accumulates into it two kernels later
         gl.p.zero_floats = c->T * c->d;
+        gl.p.hpre = train ? part<void>(ws, L, P_HPRE) : nullptr;
         e = gemm ? launch_grouped_gemm(gl, s) : launch_seg_gateup(ga, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_GATE_UP, s);
@@ -479,6 +531,7 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
         SegGateUpArgs ga{x, sh_gate, sh_up, dense, c->T, c->d, c->h_shared, acts};
         GemmLaunch gl = gemm_gateup_dense(*c, x, sh_gate, sh_up, acts, err);
         gl.p.early = kEarlyTiles | kEarlyA;   // x and the weights are layer inputs
+        gl.p.hpre = train ? part<void>(ws, L, P_HPRES) : nullptr;
         e = gemm ? launch_grouped_gemm(gl, s) : launch_seg_gateup(ga, c->dtype, s, err);
     }
     mark(1 + MOE_STAGE_SHARED_GATE_UP, s);
@@ -499,16 +552,135 @@ moe_status moe_forward(const moe_config *c, const void *x, const void *w_router,
     // complete when the down GEMM starts; act is read after the wait
     GemmLaunch dl = gemm_down(*c, act, w_down, offsets, srt, gates, acc, err);
     dl.p.early = kEarlyTiles;
-    if (e == cudaSuccess) e = launch_grouped_gemm(dl, s);
+    if (e == cudaSuccess && !fused) e = launch_grouped_gemm(dl, s);   // fused: done in the gate/up stage
     mark(1 + MOE_STAGE_DOWN, s);
     // the shared expert's act came from the kernel before the routed down GEMM
+    // (with the fused expert kernel, from the kernel right before this one)
     GemmLaunch sdl = gemm_down_dense(*c, acts, sh_down, sg, acc, err);
-    sdl.p.early = kEarlyTiles | kEarlyA;
+    sdl.p.early = fused ? kEarlyTiles : (kEarlyTiles | kEarlyA);
     if (e == cudaSuccess && shared) e = launch_grouped_gemm(sdl, s);
     mark(1 + MOE_STAGE_SHARED_DOWN, s);
     if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
     mark(1 + MOE_STAGE_FINALIZE, s);
     return cuda_status(e);
+}
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_forward(const moe_config *c, const moe_route_opts *opts, const void *x, const void *w_router,
+                       const void *w_gate, const void *w_up, const void *w_down, const void *sh_gate,
+                       const void *sh_up, const void *sh_down, const void *w_shared_gate, void *y, void *ws,
+                       size_t ws_bytes, void *stream) {
+    return forward_impl(c, opts, x, w_router, w_gate, w_up, w_down, sh_gate, sh_up, sh_down, w_shared_gate, y, ws,
+                        ws_bytes, stream, false);
+}
+
+moe_status moe_forward_train(const moe_config *c, const moe_route_opts *opts, const void *x, const void *w_router,
+                             const void *w_gate, const void *w_up, const void *w_down, const void *sh_gate,
+                             const void *sh_up, const void *sh_down, const void *w_shared_gate, void *y, void *ws,
+                             size_t ws_bytes, void *stream) {
+    return forward_impl(c, opts, x, w_router, w_gate, w_up, w_down, sh_gate, sh_up, sh_down, w_shared_gate, y, ws,
+                        ws_bytes, stream, true);
+}
+
+moe_status moe_quantize_q4(const void *w, int32_t dtype, int64_t rows, int32_t cols, uint8_t *q, float *scales,
+                           void *stream) {
+    if ((dtype != MOE_BF16 && dtype != MOE_F32) || rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 64) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!w || !q || !scales) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(q)) & 15) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_quantize_q4(w, dtype, rows, cols, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward_q4(const moe_config *c, const moe_route_opts *opts, const void *x, const void *w_router,
+                          const uint8_t *q_gate, const float *s_gate, const uint8_t *q_up, const float *s_up,
+                          const uint8_t *q_down, const float *s_down, const void *sh_gate, const void *sh_up,
+                          const void *sh_down, const void *w_shared_gate, void *y, void *ws, size_t ws_bytes,
+                          void *stream) {
+    moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (c->dtype != MOE_BF16 || c->d % 64 || c->h % 64 || c->T * c->k > kDecodeMaxRows) return MOE_ERR_UNSUPPORTED;
+    if (c->T == 0) return MOE_OK;
+    if (!x || !w_router || !q_gate || !s_gate || !q_up || !s_up || !q_down || !s_down || !y)
+        return MOE_ERR_INVALID_ARG;
+    const uintptr_t qa = reinterpret_cast<uintptr_t>(q_gate) | reinterpret_cast<uintptr_t>(q_up) |
+                         reinterpret_cast<uintptr_t>(q_down);
+    if (qa & 15) return MOE_ERR_INVALID_ARG;
+    const bool shared = c->h_shared > 0;
+    if (shared && (!sh_gate || !sh_up || !sh_down || !w_shared_gate)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*c);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
+    uint32_t *err = err_ptr();
+    if (!err) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t *ids = part<int32_t>(ws, L, P_IDS);
+    float *gates = part<float>(ws, L, P_GATES);
+    float *sg = part<float>(ws, L, P_SG);
+    int32_t *counts = part<int32_t>(ws, L, P_COUNTS);
+    int32_t *offsets = part<int32_t>(ws, L, P_OFFSETS);
+    int32_t *srt = part<int32_t>(ws, L, P_SORTED);
+    int32_t *inv = part<int32_t>(ws, L, P_INV);
+    void *act = part<void>(ws, L, P_ACT);
+    void *acts = part<void>(ws, L, P_ACTS);
+
+    RouterArgs ra{};
+    ra.x = x;
+    ra.w_router = w_router;
+    ra.w_shared_gate = shared ? w_shared_gate : nullptr;
+    ra.T = c->T;
+    ra.d = c->d;
+    ra.E = c->E;
+    ra.k = c->k;
+    ra.norm_topk = c->norm_topk != 0;
+    ra.score = c->score;
+    ra.ids = ids;
+    ra.gates = gates;
+    ra.shared_gate = sg;
+    ra.err = err;
+    ra.bias = opts ? opts->balance_bias : nullptr;
+    ra.score_mean = opts ? opts->score_mean : nullptr;
+    ra.stats = ra.score_mean ? part<float>(ws, L, P_STATS) : nullptr;
+    ra.hist_chunk = permute_chunk();
+    mark(0, s);
+    cudaError_t e = launch_router(ra, c->dtype, part<float>(ws, L, P_LOGITS), s);
+    mark(1 + MOE_STAGE_ROUTE, s);
+    const int R = (int)(c->T * c->k);
+    if (e == cudaSuccess) {
+        PermuteArgs pa{ids, R, c->E, counts, offsets, srt, inv, err};
+        e = launch_permute(pa, part<int32_t>(ws, L, P_PERM), false, s);
+    }
+    mark(1 + MOE_STAGE_PERMUTE, s);
+    if (e == cudaSuccess) {
+        SegGateUpQ4Args ga{x, q_gate, q_up, s_gate, s_up, Segments{offsets, srt, c->E, c->k, (int64_t)R}, c->T, c->d,
+                           c->h, act};
+        e = launch_seg_gateup_q4(ga, s, err);
+    }
+    mark(1 + MOE_STAGE_GATE_UP, s);
+    if (e == cudaSuccess && shared) {
+        SegGateUpArgs ga{x, sh_gate, sh_up, Segments{nullptr, nullptr, 1, 1, c->T}, c->T, c->d, c->h_shared, acts};
+        e = launch_seg_gateup(ga, c->dtype, s, err);
+    }
+    mark(1 + MOE_STAGE_SHARED_GATE_UP, s);
+    if (e == cudaSuccess) {
+        DownDirectQ4Args da{act, q_down, s_down, ids, inv, gates, shared ? acts : nullptr, shared ? sh_down : nullptr,
+                            sg, c->T, c->d, c->h, c->E, c->k, c->h_shared, y};
+        e = launch_down_direct_q4(da, s, err);
+    }
+    mark(1 + MOE_STAGE_DOWN, s);
+    mark(1 + MOE_STAGE_SHARED_DOWN, s);
+    mark(1 + MOE_STAGE_FINALIZE, s);
+    return cuda_status(e);
+}
+
+moe_status moe_train_workspace_size(const moe_config *c, size_t *bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const moe_status st = moe_validate(c);
+    if (st != MOE_OK) return st;
+    if (c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    *bytes = make_layout(*c, true).total;
+    return MOE_OK;
 }
 
 moe_status moe_profile_events(void *const *events, int32_t n) {

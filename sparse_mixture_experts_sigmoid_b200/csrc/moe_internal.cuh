@@ -81,7 +81,18 @@ struct RouterArgs {
     uint32_t *err;      // device error word
     int32_t *hist;      // optional [B, E+1] block histogram for grouping (tensor-core router only)
     int hist_chunk;     // assignments per histogram block
+    const float *bias;  // optional [E] balance bias: selection key = score + bias
+    float *stats;       // optional [router_stats_rows(T), E] per-CTA score sums (fixed order)
+    float *score_mean;  // optional [E] out: mean score per expert (needs stats)
 };
+// Rows of per-CTA score sums the routers write for the score-mean statistic:
+// one per token for the one-token-per-CTA router (T <= 64), else at most one
+// per 8 tokens.
+inline int64_t router_stats_rows(int64_t T) { return T <= 64 ? T : (T + 7) / 8; }
+// Sums the rows of a [rows, E] partial array in a fixed order and divides by
+// T into score_mean (router_stats.cu).
+cudaError_t launch_router_stats(const float *partial, int64_t rows, int E, int64_t T, float *score_mean,
+                                cudaStream_t s);
 // Router: the tensor-core logits GEMM + warp-per-token selection (router_tc.cu)
 // when supported and scratch is given, else the CUDA-core routers (router.cu).
 cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaStream_t s);
@@ -145,6 +156,35 @@ cudaError_t launch_down_direct(const DownDirectArgs &a, int dtype, cudaStream_t 
 
 cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s);
 
+// 4-bit routed experts on the small-batch path (segment_q4.cu).  A 4-bit
+// weight matrix [rows, cols] is q [rows, cols / 2] (nibble code + 8, even
+// element low) and scales [rows, cols / 64] (fp32, per group of 64).
+struct SegGateUpQ4Args {
+    const void *x;                       // [T, d] bf16
+    const uint8_t *q_gate, *q_up;        // [E * hid, d / 2]
+    const float *s_gate, *s_up;          // [E * hid, d / 64]
+    Segments seg;
+    int64_t T;
+    int d, hid;
+    void *act;                           // [rows, hid] bf16
+};
+struct DownDirectQ4Args {
+    const void *act;                     // [R, h] bf16, grouped order
+    const uint8_t *q_down;               // [E * d, h / 2]
+    const float *s_down;                 // [E * d, h / 64]
+    const int32_t *ids, *inv_rows;
+    const float *gates;
+    const void *act_shared, *sh_down;    // bf16 shared expert, or null
+    const float *shared_gate;
+    int64_t T;
+    int d, h, E, k, h_shared;
+    void *y;                             // [T, d] bf16
+};
+cudaError_t launch_quantize_q4(const void *w, int dtype, int64_t rows, int cols, uint8_t *q, float *scales,
+                               cudaStream_t s);
+cudaError_t launch_seg_gateup_q4(const SegGateUpQ4Args &a, cudaStream_t s, uint32_t *err);
+cudaError_t launch_down_direct_q4(const DownDirectQ4Args &a, cudaStream_t s, uint32_t *err);
+
 // Tensor-core grouped GEMM (grouped_gemm.cu).
 struct GemmParams {
     const int32_t *offsets;      // [E + 1] grouped row offsets; nullptr: one dense segment of `rows` rows
@@ -165,6 +205,8 @@ struct GemmParams {
     // stream has completed (see pdl_wait).  Set only where every kernel between
     // the producer of that data and this one is known.
     int early;
+    void *hpre;                  // gate/up only, optional: [rows, 2N] pre-activations (gate | up) kept
+                                 // for the backward pass
 };
 enum : int {
     kEarlyTiles = 1,   // offsets (and hence the tile list) and the weights
@@ -183,6 +225,65 @@ struct GemmLaunch {
 };
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s);
 cudaError_t launch_grouped_gemm_pair(const GemmLaunch &L, cudaStream_t s);
+
+// Fused gate/up + SwiGLU + down + combine for layers whose experts average at
+// most one 128-row tile (grouped_fused.cu).  y_acc must be zero on entry.
+bool fused_expert_supported(const moe_config &c);
+cudaError_t launch_fused_expert(const moe_config &c, const void *x, const void *wg, const void *wu, const void *wd,
+                                const int32_t *offsets, const int32_t *srt, const float *gates, float *y_acc,
+                                uint32_t *err, cudaStream_t s);
+
+// Backward grouped GEMMs (grouped_bwd.cu).  An operand tensor: row-major
+// [rows, cols] bf16 with a row stride of ld elements.
+struct BwdOperand {
+    const void *base;
+    uint64_t rows, cols, ld;
+};
+struct BwdGemm {
+    // SWIGLU: rows x N tiles, r = W^T dy with the SwiGLU-backward epilogue;
+    // SCATTER: rows x N tiles added (weight 1) into acc[token];
+    // WEIGHT: per group, M x N weight-gradient tiles reduced over the group's rows.
+    enum Kind { SWIGLU, SCATTER, WEIGHT } kind;
+    bool gather_a, gather_b;      // operand gathered from gsrc by token index
+    BwdOperand a0, a1, b0, b1;    // TMA operands (a1/b1: second K range or second half)
+    const int32_t *offsets, *sorted_rows;   // grouping (offsets == nullptr: one dense segment)
+    int groups, k;
+    int64_t rows, T;
+    int nranges, Kr, N, M, halves;
+    const void *gsrc;             // [T, gwidth] bf16
+    int gwidth;
+    const void *hpre;             // SWIGLU: [rows, 2N] pre-activations (u | v)
+    const float *gate;            // SWIGLU: routed [R] by assignment / dense [T]
+    void *dh, *ga;                // SWIGLU out: [rows, 2N] du | dv, [rows, N] gate * a
+    float *dgate;                 // SWIGLU: accumulated gate gradients
+    float *acc;                   // SCATTER: [T, N] fp32
+    void *out0, *out1;            // WEIGHT: [groups * M, N] per half
+    bool out_f32;
+    uint32_t *err;
+};
+cudaError_t launch_bwd_gemm(const BwdGemm &L, cudaStream_t s);
+
+// Parts of the workspace (see moe_workspace_layout); the training parts exist
+// only in the layout of a training step.
+enum WsPart {
+    P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_PERM, P_LOGITS,
+    P_STATS,
+    // training: kept by moe_forward_train for moe_backward, and the backward's scratch
+    P_PROBS, P_HPRE, P_HPRES, P_DG, P_DSG, P_DH, P_DHS, P_GAS, P_DLB, P_DLS,
+    P_N
+};
+struct WsLayout {
+    size_t off[P_N];
+    size_t size[P_N];
+    size_t total;
+};
+WsLayout ws_layout(const moe_config &c, bool train);
+template <typename T>
+T *ws_part(void *ws, const WsLayout &L, WsPart p) {
+    return L.size[p] ? reinterpret_cast<T *>(static_cast<char *>(ws) + L.off[p]) : nullptr;
+}
+// Row stride (elements) of the bf16 router-gradient rows: E rounded up to 8.
+inline int dl_stride(int E) { return (E + 7) / 8 * 8; }
 
 // Launch planning shared by the entry points (defined in moe_api.cu).
 uint32_t *device_error_word();   // the library's device error word on the current device

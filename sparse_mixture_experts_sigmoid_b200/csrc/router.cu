@@ -4,7 +4,8 @@
 // "Tutorial 11: Mixture of Experts (MoE)", section 2 "The Router" (route_topk:
 // logits = x . W_router^T, softmax over all experts, top-k, gather, optional
 // renormalisation); "Small MoE Architecture, in depth", SmallMoE.forward
-// (sigmoid scores; gates are the kept raw scores).
+// (sigmoid scores; top k of scores + balance_bias; gates are the kept raw
+// scores) and the paragraph on auxiliary-loss-free balancing after it.
 //
 // Layout of the work: a CTA of 8 warps owns 8*TW consecutive tokens, each warp
 // TW of them.  W_router (plus the shared-expert gate vector w_s as row E) is
@@ -14,7 +15,11 @@
 // CG = 32 / EL lane groups split the chunk's columns; the CG partial sums are
 // folded with shuffles.  All arithmetic is fp32 on exact bf16/fp32 inputs.
 // Selection is k rounds of a warp arg-max over (key, -index), so equal keys
-// resolve to the lower expert index.
+// resolve to the lower expert index.  The key is the logit (it orders experts
+// as either score function does), or the score plus the balance bias when one
+// is given; gates always come from the unbiased scores.  With the score
+// statistic requested, each CTA adds its tokens' score rows, in token order,
+// into one partial row of a.stats.
 #include <float.h>
 
 #include "moe_internal.cuh"
@@ -149,6 +154,10 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
     }
 
     const bool sigm = a.score == MOE_SCORE_SIGMOID;
+    const bool want_s = a.probs || a.stats || a.bias;
+    float ssum[EPL];   // this warp's score sums per owned expert (score statistic)
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) ssum[q] = 0.f;
 #pragma unroll
     for (int i = 0; i < TW; ++i) {
         const int64_t t = t0 + warp * TW + i;
@@ -171,9 +180,17 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
             }
             z = warp_sum(z);
         }
-        float key[EPL];
+        float sc_e[EPL], key[EPL];
 #pragma unroll
-        for (int q = 0; q < EPL; ++q) key[q] = sigm ? 1.f / (1.f + expf(-acc[i][q])) : acc[i][q];
+        for (int q = 0; q < EPL; ++q) {
+            const int e = le + g.EL * q;
+            const bool own = cg == 0 && e < a.E;
+            sc_e[q] = 0.f;
+            if (want_s && own) sc_e[q] = sigm ? 1.f / (1.f + expf(-acc[i][q])) : expf(acc[i][q] - m) / z;
+            ssum[q] += sc_e[q];
+            key[q] = acc[i][q];
+            if (a.bias) key[q] = own ? sc_e[q] + a.bias[e] : -FLT_MAX;
+        }
 
         uint32_t taken = 0;
         int my_e = 0;
@@ -213,8 +230,8 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
         float sc = 0.f;
         if (lane < a.k) sc = sigm ? 1.f / (1.f + expf(-my_l)) : expf(my_l - m) / z;
         if (a.norm_topk) {
-            const float ssum = warp_sum(lane < a.k ? sc : 0.f);
-            sc = sc / ssum;
+            const float gsum = warp_sum(lane < a.k ? sc : 0.f);
+            sc = sc / gsum;
         }
         if (lane < a.k) {
             a.ids[t * a.k + lane] = my_e;
@@ -224,8 +241,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
 #pragma unroll
             for (int q = 0; q < EPL; ++q) {
                 const int e = le + g.EL * q;
-                if (cg == 0 && e < a.E)
-                    a.probs[t * a.E + e] = sigm ? 1.f / (1.f + expf(-acc[i][q])) : expf(acc[i][q] - m) / z;
+                if (cg == 0 && e < a.E) a.probs[t * a.E + e] = sc_e[q];
             }
         }
         if (a.shared_gate && a.w_shared_gate) {
@@ -234,6 +250,22 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
                 const int e = le + g.EL * q;
                 if (cg == 0 && e == a.E) a.shared_gate[t] = 1.f / (1.f + expf(-acc[i][q]));
             }
+        }
+    }
+    if (a.stats) {
+        // the staging buffers are idle (the chunk loop ended with a barrier):
+        // per-warp score sums, then their sum in warp order
+        float *ws = reinterpret_cast<float *>(smem_raw);   // [kWarps, E]
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = le + g.EL * q;
+            if (cg == 0 && e < a.E) ws[warp * a.E + e] = ssum[q];
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < a.E; e += kThreads) {
+            float v = 0.f;
+            for (int w = 0; w < kWarps; ++w) v += ws[w * a.E + e];
+            a.stats[(int64_t)blockIdx.x * a.E + e] = v;
         }
     }
 }
@@ -284,12 +316,11 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     if (warp != 0) return;
     constexpr int EPL = MOE_MAX_EXPERTS / 32;
     const bool sigm = a.score == MOE_SCORE_SIGMOID;
-    float l[EPL], key[EPL];
+    float l[EPL], key[EPL], sc_e[EPL];
 #pragma unroll
     for (int q = 0; q < EPL; ++q) {
         const int e = lane + 32 * q;
         l[q] = e < a.E ? lg[e] : -FLT_MAX;
-        key[q] = sigm ? 1.f / (1.f + expf(-l[q])) : l[q];
     }
     float m = -FLT_MAX;
 #pragma unroll
@@ -303,6 +334,15 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
         for (int q = 0; q < EPL; ++q)
             if (lane + 32 * q < a.E) z += expf(l[q] - m);
         z = warp_sum(z);
+    }
+    // scores when needed; key = the logit, or the score plus the balance bias
+    const bool want_s = a.probs || a.stats || a.bias;
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) {
+        const int e = lane + 32 * q;
+        sc_e[q] = (want_s && e < a.E) ? (sigm ? 1.f / (1.f + expf(-l[q])) : expf(l[q] - m) / z) : 0.f;
+        key[q] = l[q];
+        if (a.bias) key[q] = e < a.E ? sc_e[q] + a.bias[e] : -FLT_MAX;
     }
     uint32_t taken = 0;
     int my_e = 0;
@@ -351,7 +391,15 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
 #pragma unroll
         for (int q = 0; q < EPL; ++q) {
             const int e = lane + 32 * q;
-            if (e < a.E) a.probs[t * a.E + e] = sigm ? key[q] : expf(l[q] - m) / z;
+            if (e < a.E) a.probs[t * a.E + e] = sc_e[q];
+        }
+    }
+    if (a.stats) {
+        // one token per CTA: its score row is the CTA's partial row
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane + 32 * q;
+            if (e < a.E) a.stats[t * a.E + e] = sc_e[q];
         }
     }
     if (lane == 0 && a.shared_gate && a.w_shared_gate) a.shared_gate[t] = 1.f / (1.f + expf(-lg[a.E]));
@@ -371,7 +419,9 @@ cudaError_t launch_t(const RouterArgs &a, const Geo &g, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((a.T + NT - 1) / NT);
-    return launch_kernel(kern, grid, kThreads, smem, s, a, g);
+    e = launch_kernel(kern, grid, kThreads, smem, s, a, g);
+    if (e == cudaSuccess && a.stats && a.score_mean) e = launch_router_stats(a.stats, grid, a.E, a.T, a.score_mean, s);
+    return e;
 }
 
 template <typename Tin, int EPL>
@@ -429,17 +479,12 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaSt
     if (scratch && router_tc_supported(a.T, a.E, dtype)) return launch_router_tc(a, scratch, s);
     if (a.T <= kSmallT) {
         const size_t smem = sizeof(float) * ((size_t)a.d + a.E + 1);
-        if (dtype == MOE_F32) {
-            cudaError_t e = cudaFuncSetAttribute(router_small_kernel<float>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            return launch_kernel(router_small_kernel<float>, (unsigned)a.T, kThreads, smem, s, a);
-        } else {
-            cudaError_t e = cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            return launch_kernel(router_small_kernel<__nv_bfloat16>, (unsigned)a.T, kThreads, smem, s, a);
-        }
+        auto kern = dtype == MOE_F32 ? router_small_kernel<float> : router_small_kernel<__nv_bfloat16>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess) e = launch_kernel(kern, (unsigned)a.T, kThreads, smem, s, a);
+        if (e == cudaSuccess && a.stats && a.score_mean)
+            e = launch_router_stats(a.stats, a.T, a.E, a.T, a.score_mean, s);
+        return e;
     }
     return dtype == MOE_F32 ? launch_dt<float>(a, s) : launch_dt<__nv_bfloat16>(a, s);
 }

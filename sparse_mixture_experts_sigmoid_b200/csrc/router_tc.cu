@@ -11,12 +11,18 @@
 //     chunk order, forms softmax statistics or sigmoid scores, takes the top k
 //     by k rounds of a warp arg-max over (key, -index) -- equal keys go to the
 //     lower expert index -- and writes ids, gates (optionally renormalised),
-//     the full score row and the shared gate.
+//     the full score row and the shared gate.  The key is the logit (it
+//     orders experts as either score does), or, with a balance bias, the
+//     score plus the bias; the gates always come from the unbiased scores.
+//     With the score statistic requested, the CTA's 8 score rows are added
+//     in token order into one partial row per CTA.
 //
 // "Tutorial 11: Mixture of Experts (MoE)", section 2 "The Router" (route_topk:
 // logits = x . W_router^T, softmax over all experts, top-k, gather of the kept
 // scores, optional renormalisation); "Small MoE Architecture, in depth",
-// SmallMoE.forward (sigmoid scores; gates are the kept raw scores).
+// SmallMoE.forward (sigmoid scores; top k of scores + balance_bias; gates are
+// the kept raw scores) and the paragraph on auxiliary-loss-free balancing
+// after it.
 //
 // Exactness: x and W_router are bf16, so every product is exact in fp32.  The
 // K range is cut into S chunks (one per CTA) and, inside a CTA, k-block kb of
@@ -262,10 +268,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == kMmaWarp) tmem_dealloc(tmem, kCols);
 }
 
-// The selection for token t by one warp (see router_select_kernel).
+// The selection for token t by one warp (see router_select_kernel).  With
+// stat_row != NULL the lanes also write the token's score row there.
 template <int EPL>
 __device__ __forceinline__ void select_token(const RouterArgs &a, const float *partial, int LSP, int S, int nrw,
-                                             int64_t t, int lane) {
+                                             int64_t t, int lane, float *stat_row) {
     const bool sigm = a.score == MOE_SCORE_SIGMOID;
     // the token's logits: lane owns experts lane * EPL .. + EPL - 1; its S
     // partial rows are read with vector loads, a group of chunks at a time with
@@ -309,10 +316,8 @@ __device__ __forceinline__ void select_token(const RouterArgs &a, const float *p
         }
     }
 #pragma unroll
-    for (int q = 0; q < EPL; ++q) {
+    for (int q = 0; q < EPL; ++q)
         if (!mine || e0 + q >= a.E) l[q] = -FLT_MAX;
-        key[q] = sigm ? 1.f / (1.f + expf(-l[q])) : l[q];
-    }
     if (a.zero_rows) {
         float4 *z = reinterpret_cast<float4 *>(a.zero_rows + t * a.d);
         for (int i = lane; i < a.d / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -329,6 +334,22 @@ __device__ __forceinline__ void select_token(const RouterArgs &a, const float *p
         for (int q = 0; q < EPL; ++q)
             if (e0 + q < a.E) z += expf(l[q] - m);
         z = warp_sum(z);
+    }
+    // every expert's score, when the score row, its statistic or a biased
+    // key needs it
+    float sc_e[EPL];
+    if (a.probs || stat_row || a.bias) {
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+            sc_e[q] = e0 + q < a.E ? (sigm ? 1.f / (1.f + expf(-l[q])) : expf(l[q] - m) / z) : 0.f;
+    }
+    // selection key: the logit (monotone in the score under either function),
+    // or the score plus the balance bias
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) {
+        const int e = e0 + q;
+        key[q] = l[q];
+        if (a.bias) key[q] = e < a.E ? sc_e[q] + a.bias[e] : -FLT_MAX;
     }
     uint32_t taken = 0;
     int my_e = 0;
@@ -382,8 +403,13 @@ __device__ __forceinline__ void select_token(const RouterArgs &a, const float *p
 #pragma unroll
         for (int q = 0; q < EPL; ++q) {
             const int e = e0 + q;
-            if (e < a.E) a.probs[t * a.E + e] = sigm ? key[q] : expf(l[q] - m) / z;
+            if (e < a.E) a.probs[t * a.E + e] = sc_e[q];
         }
+    }
+    if (stat_row) {
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+            if (e0 + q < a.E) stat_row[e0 + q] = sc_e[q];
     }
     if (lane == 0 && a.shared_gate && a.w_shared_gate) {
         float ls = 0.f;
@@ -392,15 +418,33 @@ __device__ __forceinline__ void select_token(const RouterArgs &a, const float *p
     }
 }
 
-// One warp per token: scoring, top-k and gates from a row of logits.
+// One warp per token: scoring, top-k and gates from a row of logits.  With
+// the score statistic requested (a.stats), the 8 tokens' score rows are
+// staged in shared memory and added in token order into row blockIdx.x of
+// a.stats (tokens past T count as zero rows).
 template <int EPL>
 __global__ void __launch_bounds__(256) router_select_kernel(RouterArgs a, const float *partial, int LSP, int S,
                                                             int nrw) {
+    extern __shared__ float s_rows[];   // [8, E] when a.stats
     pdl_wait();
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-    if (t < a.T) select_token<EPL>(a, partial, LSP, S, nrw, t, lane);
+    float *stat_row = a.stats ? s_rows + warp * a.E : nullptr;
+    if (t < a.T) {
+        select_token<EPL>(a, partial, LSP, S, nrw, t, lane, stat_row);
+    } else if (stat_row) {
+        for (int e = lane; e < a.E; e += 32) stat_row[e] = 0.f;
+    }
+    if (a.stats) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < a.E; e += 256) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) v += s_rows[w * a.E + e];
+            a.stats[(int64_t)blockIdx.x * a.E + e] = v;
+        }
+    }
 }
 
 // Tiling of the logits GEMM for a batch (a pure function of the shape).
@@ -478,10 +522,13 @@ cudaError_t launch_router_tc(const RouterArgs &a, float *scratch, cudaStream_t s
     if (e != cudaSuccess) return e;
     const unsigned sgrid = (unsigned)((a.T + 7) / 8);
     const float *pt = scratch;
-    if (a.E <= 64) return launch_kernel(router_select_kernel<2>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
-    if (a.E <= 128) return launch_kernel(router_select_kernel<4>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
-    if (a.E <= 256) return launch_kernel(router_select_kernel<8>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
-    return launch_kernel(router_select_kernel<16>, sgrid, 256, 0, s, a, pt, p.LSP, p.S, p.nrw);
+    const size_t ssm = a.stats ? sizeof(float) * 8 * (size_t)a.E : 0;
+    if (a.E <= 64) e = launch_kernel(router_select_kernel<2>, sgrid, 256, ssm, s, a, pt, p.LSP, p.S, p.nrw);
+    else if (a.E <= 128) e = launch_kernel(router_select_kernel<4>, sgrid, 256, ssm, s, a, pt, p.LSP, p.S, p.nrw);
+    else if (a.E <= 256) e = launch_kernel(router_select_kernel<8>, sgrid, 256, ssm, s, a, pt, p.LSP, p.S, p.nrw);
+    else e = launch_kernel(router_select_kernel<16>, sgrid, 256, ssm, s, a, pt, p.LSP, p.S, p.nrw);
+    if (e == cudaSuccess && a.stats && a.score_mean) e = launch_router_stats(a.stats, sgrid, a.E, a.T, a.score_mean, s);
+    return e;
 }
 
 }  // namespace moe

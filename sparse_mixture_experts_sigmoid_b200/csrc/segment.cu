@@ -11,66 +11,16 @@
 // expert linears, silu(gate) * up, weighted sum); "Small MoE Architecture, in
 // depth", Expert.forward (the SwiGLU expert) and the batch-1 decode remarks in
 // "Why small changes the MoE trade-off" (decode reads only the chosen experts).
-#include <mutex>
-#include <unordered_map>
-
-#include "moe_internal.cuh"
+#include "segment_parts.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+using seg::kThreads;
+using seg::kWarps;
+using seg::list_experts;
+using seg::grid_for;
 constexpr int RB = 4;  // grouped rows per pass over a weight row
-
-// Builds, in shared memory, the list of experts that own at least one row.
-__device__ int list_experts(const Segments &sg, int *list, int *beg, int *end) {
-    __shared__ int s_n;
-    if (sg.offsets == nullptr) {
-        if (threadIdx.x == 0) {
-            list[0] = 0;
-            beg[0] = 0;
-            end[0] = (int)sg.rows;
-            s_n = 1;
-        }
-        __syncthreads();
-        return s_n;
-    }
-    if (threadIdx.x == 0) s_n = 0;
-    __syncthreads();
-    // ordered compaction: each warp takes 32 experts at a time
-    for (int base = 0; base < sg.E; base += kThreads) {
-        const int e = base + threadIdx.x;
-        int b = 0, en = 0;
-        bool has = false;
-        if (e < sg.E) {
-            b = sg.offsets[e];
-            en = sg.offsets[e + 1];
-            has = en > b;
-        }
-        __shared__ int wcount[kWarps];
-        const unsigned m = __ballot_sync(0xffffffffu, has);
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-        if (lane == 0) wcount[warp] = __popc(m);
-        __syncthreads();
-        int before = s_n;
-        for (int w = 0; w < warp; ++w) before += wcount[w];
-        if (has) {
-            const int pos = before + __popc(m & ((1u << lane) - 1u));
-            list[pos] = e;
-            beg[pos] = b;
-            end[pos] = en;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int add = 0;
-            for (int w = 0; w < kWarps; ++w) add += wcount[w];
-            s_n += add;
-        }
-        __syncthreads();
-    }
-    return s_n;
-}
 
 __device__ __forceinline__ float dot8(const float (&a)[8], const float (&b)[8], float acc) {
 #pragma unroll
@@ -110,7 +60,9 @@ __global__ void __launch_bounds__(kThreads) seg_gateup_kernel(SegGateUpArgs a, u
                 const int r = r0 + b;
                 int64_t t = -1;
                 if (r < end[li]) {
-                    t = a.seg.sorted_rows ? a.seg.sorted_rows[r] / a.seg.k : r;
+                    // range-check the assignment before deriving its token
+                    const int v = a.seg.sorted_rows ? a.seg.sorted_rows[r] : r;
+                    t = (v >= 0 && v < a.seg.rows) ? (a.seg.sorted_rows ? v / a.seg.k : v) : -1;
                     if (t < 0 || t >= a.T) {
                         if (lane == 0) atomicOr(err, kErrInput);
                         t = -1;
@@ -302,30 +254,6 @@ __global__ void finalize_kernel(const float *y_acc, T *y, int64_t n) {
     } else {
         for (int64_t j = i; j < n; ++j) y[j] = __float2bfloat16_rn(y_acc[j]);
     }
-}
-
-// One warp per item, but no more CTAs than fit on the GPU at once: the
-// kernels stream weights, so the warps resident per SM (and with them the
-// bytes in flight) are what sets their rate.  The residency of each kernel is
-// asked for once.
-template <typename K>
-int grid_for(K kern, int64_t items, size_t smem) {
-    static std::mutex mu;
-    static std::unordered_map<const void *, int> per_sm;
-    int b = 0;
-    {
-        std::lock_guard<std::mutex> lk(mu);
-        auto it = per_sm.find(reinterpret_cast<const void *>(kern));
-        if (it != per_sm.end()) {
-            b = it->second;
-        } else {
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, smem) != cudaSuccess || b < 1) b = 1;
-            per_sm[reinterpret_cast<const void *>(kern)] = b;
-        }
-    }
-    const int64_t cap = (int64_t)b * num_sms();
-    const int64_t need = (items + kWarps - 1) / kWarps;
-    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
 }
 
 }  // namespace

@@ -1,0 +1,261 @@
+// 4-bit routed experts for the small-batch (decode) path.
+//
+// "Small MoE Architecture, in depth": "Worked example: the batch-1 budget on
+// a device" (4-bit weights, about half a byte per parameter: decode reads the
+// k chosen experts' weights, so tokens/s follows the bytes per parameter) and
+// "Running experts that do not fit: offloading and quantisation" (routed
+// experts quantised more aggressively; shared expert and router kept at
+// higher precision).  Format (this library's reading; the pages fix none):
+// groups of 64 consecutive weights along a row (the reduction dimension),
+// scale s = max|w| / 7 in fp32, code round(w / s) in [-7, 7] (ties to even),
+// stored as nibble code + 8, two per byte, even element in the low nibble;
+// the value represented is (nibble - 8) * s.
+//
+//   quantize_q4_kernel: one thread per group of 64 weights.
+//   seg_gateup_q4_kernel: one warp per (expert, hidden row): the warp streams
+//     the 4-bit gate and up rows once (16 bytes = 32 weights per lane per
+//     load, the group's scale alongside) and applies them to every grouped row
+//     of the expert; act = silu(gate) * up in bf16.
+//   down_direct_q4_kernel: one warp per output element (t, n):
+//     y = sum_j g_j (W_down[e_j, n] . act) (+ the bf16 shared expert), written
+//     straight into y.
+// The weights are dequantised in registers; accumulation is fp32.
+#include <algorithm>
+
+#include "segment_parts.cuh"
+
+namespace moe {
+namespace {
+
+using seg::grid_for;
+using seg::kThreads;
+using seg::kWarps;
+using seg::list_experts;
+
+// One group of 64 weights -> 32 bytes of nibbles and one fp32 scale.  The
+// code is decided in fp32: s = max|w| / 7 and w / s, each rounded once.
+template <typename T>
+__global__ void quantize_q4_kernel(const T *w, int64_t groups, int gpr, uint8_t *q, float *scales) {
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (int64_t)gridDim.x * blockDim.x) {
+        const T *src = w + g * 64;
+        float v[64];
+#pragma unroll
+        for (int i = 0; i < 64; i += 8) {
+            float t[8];
+            load8(src + i, t);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[i + j] = t[j];
+        }
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) m = fmaxf(m, fabsf(v[i]));
+        const float s = __fdiv_rn(m, 7.f);
+        scales[g] = s;
+        uint32_t out[8];
+#pragma unroll
+        for (int wd = 0; wd < 8; ++wd) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                int code = 0;
+                if (s != 0.f) {
+                    float c = rintf(__fdiv_rn(v[wd * 8 + j], s));
+                    c = fminf(7.f, fmaxf(-7.f, c));
+                    code = (int)c;
+                }
+                word |= (uint32_t)(code + 8) << (4 * j);
+            }
+            out[wd] = word;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(q + g * 32);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        (void)gpr;
+    }
+}
+
+// 32 weights (one 16-byte load of nibbles, even element in the low nibble)
+// times scale s, dotted with 32 consecutive bf16 values of v.
+__device__ __forceinline__ float dot32_q4(const uint4 &qw, float s, const __nv_bfloat16 *v, float acc) {
+    const uint32_t words[4] = {qw.x, qw.y, qw.z, qw.w};
+    float part = 0.f;
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+        float xv[8];
+        load8(v + 8 * wd, xv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part = fmaf((float)((int)((words[wd] >> (4 * j)) & 15u) - 8), xv[j], part);
+    }
+    return fmaf(part, s, acc);
+}
+
+// Dot of one 4-bit weight row (n weights, n a multiple of 64) with a bf16
+// vector; lane l takes the 32-weight halves l, l + 32, ...; four loads in
+// flight per round.
+__device__ __forceinline__ float row_dot_q4(const uint8_t *q, const float *sc, const __nv_bfloat16 *v, int n,
+                                            int lane) {
+    float acc = 0.f;
+    int c = lane * 32;
+    for (; c + 3 * 1024 < n; c += 4 * 1024) {
+        uint4 qw[4];
+        float sv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            qw[u] = __ldcs(reinterpret_cast<const uint4 *>(q + (c + u * 1024) / 2));
+            sv[u] = __ldg(sc + (c + u * 1024) / 64);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc = dot32_q4(qw[u], sv[u], v + c + u * 1024, acc);
+    }
+    for (; c < n; c += 1024) {
+        const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(q + c / 2));
+        acc = dot32_q4(q0, __ldg(sc + c / 64), v + c, acc);
+    }
+    return acc;
+}
+
+__device__ __forceinline__ float row_dot_bf16(const __nv_bfloat16 *w, const __nv_bfloat16 *v, int n, int lane) {
+    float acc = 0.f;
+    for (int c = lane * 8; c < n; c += 256) {
+        float wv[8], av[8];
+        load8_stream(w + c, wv);
+        load8(v + c, av);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc = fmaf(wv[u], av[u], acc);
+    }
+    return acc;
+}
+
+// Grouped gate/up of the routed experts from 4-bit weights: one warp per
+// (listed expert, hidden row n), RG grouped rows per pass over the weight rows.
+template <int RG>
+__global__ void __launch_bounds__(kThreads) seg_gateup_q4_kernel(SegGateUpQ4Args a, uint32_t *err) {
+    pdl_wait();
+    pdl_launch_dependents();
+    extern __shared__ int sm[];
+    int *list = sm, *beg = sm + a.seg.E, *end = sm + 2 * a.seg.E;
+    const int ne = list_experts(a.seg, list, beg, end);
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
+    __nv_bfloat16 *act = static_cast<__nv_bfloat16 *>(a.act);
+    const int lane = threadIdx.x & 31;
+    const int qpr = a.d / 2, spr = a.d / 64;   // bytes and scales per weight row
+    const int64_t nitems = (int64_t)ne * a.hid;
+    const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t nw = (int64_t)gridDim.x * kWarps;
+    for (int64_t item = gw; item < nitems; item += nw) {
+        const int li = (int)(item / a.hid);
+        const int n = (int)(item - (int64_t)li * a.hid);
+        const int64_t wrow = (int64_t)list[li] * a.hid + n;
+        const uint8_t *qg = a.q_gate + wrow * qpr, *qu = a.q_up + wrow * qpr;
+        const float *sg = a.s_gate + wrow * spr, *su = a.s_up + wrow * spr;
+        for (int r0 = beg[li]; r0 < end[li]; r0 += RG) {
+            int64_t tok[RG];
+#pragma unroll
+            for (int b = 0; b < RG; ++b) {
+                const int r = r0 + b;
+                int64_t t = -1;
+                if (r < end[li]) {
+                    // range-check the assignment before deriving its token
+                    const int v = a.seg.sorted_rows[r];
+                    t = (v >= 0 && v < a.seg.rows) ? v / a.seg.k : -1;
+                    if (t < 0 || t >= a.T) {
+                        if (lane == 0) atomicOr(err, kErrInput);
+                        t = -1;
+                    }
+                }
+                tok[b] = t;
+            }
+            float ag[RG], au[RG];
+#pragma unroll
+            for (int b = 0; b < RG; ++b) ag[b] = au[b] = 0.f;
+#pragma unroll 4
+            for (int c = lane * 32; c < a.d; c += 1024) {
+                const uint4 wg = __ldcs(reinterpret_cast<const uint4 *>(qg + c / 2));
+                const uint4 wu = __ldcs(reinterpret_cast<const uint4 *>(qu + c / 2));
+                const float s_g = __ldg(sg + c / 64), s_u = __ldg(su + c / 64);
+#pragma unroll
+                for (int b = 0; b < RG; ++b) {
+                    if (tok[b] >= 0) {
+                        ag[b] = dot32_q4(wg, s_g, x + tok[b] * a.d + c, ag[b]);
+                        au[b] = dot32_q4(wu, s_u, x + tok[b] * a.d + c, au[b]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < RG; ++b) {
+                const float g = warp_sum(ag[b]);
+                const float u = warp_sum(au[b]);
+                if (lane == b && tok[b] >= 0) act[(int64_t)(r0 + b) * a.hid + n] = __float2bfloat16_rn(silu_f(g) * u);
+            }
+        }
+    }
+}
+
+// y[t, n] = sum_j g_j (W_down[e_j, n] . act[inv(t*k + j)]) (4-bit W_down)
+//         (+ shared_gate[t] * (S_down[n] . act_shared[t]), bf16).
+__global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Args a, uint32_t *err) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const __nv_bfloat16 *act = static_cast<const __nv_bfloat16 *>(a.act);
+    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(a.y);
+    const int lane = threadIdx.x & 31;
+    const int qpr = a.h / 2, spr = a.h / 64;
+    const int64_t nitems = a.T * a.d;
+    const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t nw = (int64_t)gridDim.x * kWarps;
+    for (int64_t item = gw; item < nitems; item += nw) {
+        const int64_t t = item / a.d;
+        const int n = (int)(item - t * a.d);
+        float acc = 0.f;
+        for (int j = 0; j < a.k; ++j) {
+            const int64_t slot = t * a.k + j;
+            const int e = a.ids[slot];
+            const int r = a.inv_rows[slot];
+            if (e < 0 || e >= a.E || r < 0 || r >= a.T * a.k) {
+                if (lane == 0) atomicOr(err, kErrInput);
+                continue;
+            }
+            const int64_t wrow = (int64_t)e * a.d + n;
+            acc += a.gates[slot] * row_dot_q4(a.q_down + wrow * qpr, a.s_down + wrow * spr, act + (int64_t)r * a.h,
+                                              a.h, lane);
+        }
+        if (a.sh_down) {
+            const __nv_bfloat16 *sd = static_cast<const __nv_bfloat16 *>(a.sh_down);
+            const __nv_bfloat16 *as = static_cast<const __nv_bfloat16 *>(a.act_shared);
+            acc += a.shared_gate[t] * row_dot_bf16(sd + (int64_t)n * a.h_shared, as + t * a.h_shared, a.h_shared, lane);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) y[item] = __float2bfloat16_rn(acc);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_q4(const void *w, int dtype, int64_t rows, int cols, uint8_t *q, float *scales,
+                               cudaStream_t s) {
+    const int64_t groups = rows * (cols / 64);
+    if (groups <= 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)std::min<int64_t>((groups + 255) / 256, 32LL * num_sms());
+    if (dtype == MOE_F32)
+        return launch_kernel(quantize_q4_kernel<float>, blocks, 256, 0, s, static_cast<const float *>(w), groups,
+                             cols / 64, q, scales);
+    return launch_kernel(quantize_q4_kernel<__nv_bfloat16>, blocks, 256, 0, s, static_cast<const __nv_bfloat16 *>(w),
+                         groups, cols / 64, q, scales);
+}
+
+cudaError_t launch_seg_gateup_q4(const SegGateUpQ4Args &a, cudaStream_t s, uint32_t *err) {
+    if (a.seg.rows <= 0) return cudaSuccess;
+    const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
+    const int64_t items = (int64_t)a.seg.E * a.hid;
+    auto go = [&](auto kern) { return launch_kernel(kern, grid_for(kern, items, smem), kThreads, smem, s, a, err); };
+    return a.T == 1 ? go(seg_gateup_q4_kernel<1>) : go(seg_gateup_q4_kernel<4>);
+}
+
+cudaError_t launch_down_direct_q4(const DownDirectQ4Args &a, cudaStream_t s, uint32_t *err) {
+    if (a.T <= 0) return cudaSuccess;
+    return launch_kernel(down_direct_q4_kernel, grid_for(down_direct_q4_kernel, a.T * a.d, 0), kThreads, 0, s, a, err);
+}
+
+}  // namespace moe

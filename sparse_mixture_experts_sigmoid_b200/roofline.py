@@ -31,10 +31,15 @@ def active_experts(counts) -> int:
     return int(np.count_nonzero(np.asarray(counts)))
 
 
-def stage_work(w: Workload, counts) -> dict:
+# 4-bit routed expert weights: half a byte per parameter plus one fp32 scale per 64
+Q4_BYTES_PER_PARAM = 0.5 + 4.0 / 64
+
+
+def stage_work(w: Workload, counts, q4: bool = False) -> dict:
     """Algorithmic FLOPs and bytes of each stage of the forward pass, given the
-    per-expert row counts the router produced."""
+    per-expert row counts the router produced (q4: routed experts in 4 bits)."""
     esz = w.elem_bytes()
+    wsz = Q4_BYTES_PER_PARAM if q4 else esz   # bytes per routed expert parameter
     R, T, d, h, hs = w.R, w.T, w.d, w.h, w.h_shared
     na = active_experts(counts)
     work = {
@@ -42,9 +47,9 @@ def stage_work(w: Workload, counts) -> dict:
                   "bytes": T * d * esz + w.E * d * esz + R * 8 + (d * esz + T * 4 if hs else 0)},
         "permute": {"flops": 0.0, "bytes": R * 4 * 3 + (2 * w.E + 1) * 4},
         "gate_up": {"flops": 2.0 * R * 2 * h * d,
-                    "bytes": na * 2 * h * d * esz + T * d * esz + R * h * esz},
+                    "bytes": na * 2 * h * d * wsz + T * d * esz + R * h * esz},
         "down": {"flops": 2.0 * R * h * d,
-                 "bytes": na * d * h * esz + R * h * esz + R * 8 + T * d * 4},
+                 "bytes": na * d * h * wsz + R * h * esz + R * 8 + T * d * 4},
         "finalize": {"flops": 0.0, "bytes": T * d * (4 + esz) if w.dtype == "bf16" else 0},
     }
     if hs:
@@ -55,12 +60,13 @@ def stage_work(w: Workload, counts) -> dict:
     return work
 
 
-def layer_work(w: Workload, counts) -> dict:
+def layer_work(w: Workload, counts, q4: bool = False) -> dict:
     """Whole-layer algorithmic FLOPs and minimum bytes (weights of the chosen
-    experts, router, x and y)."""
+    experts, router, x and y; q4: routed experts in 4 bits)."""
     esz = w.elem_bytes()
     na = active_experts(counts)
-    b = na * 3 * w.h * w.d * esz + w.E * w.d * esz + 2 * w.T * w.d * esz
+    wsz = Q4_BYTES_PER_PARAM if q4 else esz
+    b = na * 3 * w.h * w.d * wsz + w.E * w.d * esz + 2 * w.T * w.d * esz
     if w.h_shared:
         b += 3 * w.h_shared * w.d * esz + w.d * esz
     return {"flops": w.flops(), "bytes": b}
@@ -78,3 +84,28 @@ def measured_peaks(path: str | None = None) -> dict:
     except (OSError, KeyError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "source": "fallback"}
+
+
+def load_spread(counts) -> dict:
+    """The realised per-expert load: rows per expert (max, min, mean), their
+    coefficient of variation, and how many experts received rows."""
+    c = np.asarray(counts, dtype=np.float64)
+    mean = float(c.mean()) if c.size else 0.0
+    return {"active_experts": int(np.count_nonzero(c)), "max": int(c.max()) if c.size else 0,
+            "min": int(c.min()) if c.size else 0, "mean": mean,
+            "cv": float(c.std() / mean) if mean > 0 else 0.0}
+
+
+def fractions(flops: float, nbytes: float, seconds: float, peaks: dict, tensor_peak: float) -> dict:
+    """Both roofline fractions of one timed piece of work and the binding one.
+
+    tensor_frac = (flops / t) / tensor_peak and hbm_frac = (bytes / t) / HBM
+    peak; the roofline's lower bound on the time is max(flops / tensor_peak,
+    bytes / HBM peak), so frac = that bound / t = max(tensor_frac, hbm_frac),
+    and `bound` names the resource that sets it."""
+    tf = flops / seconds / 1e12 / tensor_peak if seconds > 0 else 0.0
+    hf = nbytes / seconds / 1e9 / peaks["hbm_gbs"] if seconds > 0 else 0.0
+    bound = "tensor" if tf >= hf else "hbm"
+    return {"bound": bound, "tensor_frac": tf, "hbm_frac": hf, "frac": max(tf, hf),
+            "tflops": flops / seconds / 1e12 if seconds > 0 else 0.0,
+            "gbs": nbytes / seconds / 1e9 if seconds > 0 else 0.0}

@@ -56,13 +56,14 @@ class OracleInputs:
 
 
 def enforce_margin(w: Workload, layer: synth.Layer, margin: float = MARGIN,
-                   max_attempts: int = 80) -> int:
+                   max_attempts: int = 80, bias=None) -> int:
     """Redraws x rows (in place, CPU tensor) until every token's selection margin
-    is >= margin.  Returns the number of row redraws."""
+    (with the balance bias, when given) is >= margin.  Returns the number of row
+    redraws."""
     c = ocfg(w)
     redraws = 0
     for attempt in range(1, max_attempts + 1):
-        m = oracle.topk_margin(c, bits(layer.x), bits(layer.w_router))
+        m = oracle.topk_margin(c, bits(layer.x), bits(layer.w_router), bias=bias)
         bad = np.nonzero(~(m >= margin))[0]
         if bad.size == 0:
             return redraws

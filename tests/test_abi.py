@@ -61,23 +61,26 @@ def test_null_pointers_rejected_before_launch():
     L = B.lib()
     P = ctypes.c_void_p
     fake = P(0x1000)
-    assert L.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, None, None, None, 0, None) == 1
-    assert L.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None, 0, None) == 1  # no w_s
+    assert L.moe_route(ctypes.byref(cfg), None, None, fake, None, fake, fake, None, None, None, 0, None) == 1
+    assert L.moe_route(ctypes.byref(cfg), None, fake, fake, None, fake, fake, None, fake, None, 0, None) == 1  # no w_s
     big = B.config_of(WORKLOADS["olmoe_zipf"])
-    # fp32 partial logits: one [T, 64] slab per chunk of the K range
+    # fp32 partial logits, one [T, 64] slab per chunk of the K range, then the
+    # per-CTA score sums of the score-mean statistic ([T / 8, E] fp32)
     n = B.route_workspace_size(big)
-    assert n >= 8192 * 64 * 4 and n % (8192 * 64 * 4) == 0 and n // (8192 * 64 * 4) <= 2048 // 64
-    assert L.moe_route(ctypes.byref(big), fake, fake, None, fake, fake, None, None, None, 0, None) == 3
+    stats = 8192 // 8 * 64 * 4
+    logits = n - stats
+    assert logits >= 8192 * 64 * 4 and logits % (8192 * 64 * 4) == 0 and logits // (8192 * 64 * 4) <= 2048 // 64
+    assert L.moe_route(ctypes.byref(big), None, fake, fake, None, fake, fake, None, None, None, 0, None) == 3
     assert L.moe_permute(ctypes.byref(cfg), fake, None, fake, fake, fake, fake, 1 << 20, None) == 1
     assert L.moe_permute(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, 0, None) == 3
     assert L.moe_permute(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, 4, None) == 3
     assert L.moe_grouped_swiglu(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, None) == 1
     assert L.moe_combine(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, None, 0, None) == 1
     args = [fake] * 5 + [None] * 4 + [fake]
-    assert L.moe_forward(ctypes.byref(cfg), *args, None, 0, None) == 3        # no workspace
-    assert L.moe_forward(ctypes.byref(cfg), *args, P(0x10000), 16, None) == 3  # too small
+    assert L.moe_forward(ctypes.byref(cfg), None, *args, None, 0, None) == 3        # no workspace
+    assert L.moe_forward(ctypes.byref(cfg), None, *args, P(0x10000), 16, None) == 3  # too small
     qcfg = B.config_of(WORKLOADS["qwen_shared"])
-    assert L.moe_forward(ctypes.byref(qcfg), *args, P(0x10000), 1 << 40, None) == 1  # shared weights missing
+    assert L.moe_forward(ctypes.byref(qcfg), None, *args, P(0x10000), 1 << 40, None) == 1  # shared weights missing
     bf = B.config(16, 64, 8, 128, 2)
     assert L.moe_combine(ctypes.byref(bf), fake, fake, fake, fake, fake, fake, None, 0, None) == 3
 
@@ -85,8 +88,39 @@ def test_null_pointers_rejected_before_launch():
 def test_zero_tokens_is_a_no_op():
     cfg = B.config(0, 64, 8, 128, 2)
     P = ctypes.c_void_p
-    assert B.lib().moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None, 0, None) == 0
-    assert B.lib().moe_forward(ctypes.byref(cfg), *([None] * 10), None, 0, None) == 0
+    assert B.lib().moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, 0, None) == 0
+    assert B.lib().moe_forward(ctypes.byref(cfg), None, *([None] * 10), None, 0, None) == 0
+
+
+def test_route_statistic_needs_its_workspace_part():
+    """With a score-mean output the route scratch must also hold the per-CTA
+    partial rows; without it the logits part alone suffices."""
+    L = B.lib()
+    fake = ctypes.c_void_p(0x1000)
+    for T in (1, 64, 100, 4096):
+        cfg = B.config(T, 256, 16, 128, 2)
+        total = B.route_workspace_size(cfg)
+        rows = T if T <= 64 else (T + 7) // 8
+        assert total >= rows * 16 * 4
+        opts = B.RouteOpts(None, 0x2000)
+        ws = ctypes.c_void_p(1 << 20)
+        assert L.moe_route(ctypes.byref(cfg), ctypes.byref(opts), fake, fake, None, fake, fake, None, None,
+                           ws, total - 1, None) == 3
+        assert L.moe_route(ctypes.byref(cfg), ctypes.byref(opts), fake, fake, None, fake, fake, None, None,
+                           None, 0, None) == 3
+
+
+def test_balance_entry_points_validate_on_the_host():
+    L = B.lib()
+    cfg = B.config(16, 64, 8, 128, 2)
+    fake = ctypes.c_void_p(0x1000)
+    assert L.moe_update_bias(ctypes.byref(cfg), None, ctypes.c_float(1e-3), fake, None) == 1
+    assert L.moe_update_bias(ctypes.byref(cfg), fake, ctypes.c_float(float("nan")), fake, None) == 1
+    assert L.moe_update_bias(ctypes.byref(cfg), fake, ctypes.c_float(float("inf")), fake, None) == 1
+    assert L.moe_balance_loss(ctypes.byref(cfg), fake, fake, ctypes.c_float(0.01), None, None, None) == 1
+    assert L.moe_balance_loss(ctypes.byref(cfg), fake, None, ctypes.c_float(0.01), None, fake, None) == 1
+    bad = B.config(16, 64, 8, 128, 9)                      # k > E
+    assert L.moe_update_bias(ctypes.byref(bad), fake, ctypes.c_float(1e-3), fake, None) == 1
 
 
 def test_workspace_layout_is_disjoint_and_aligned():

@@ -6,7 +6,11 @@ forced on every small parity case against the oracle:
   (gathered and contiguous operands, gate/up and down, fp32 (tf32) and bf16,
   partial 256-row tiles, the shared expert, 128-wide tiles);
 * 64-row down tiles with 64-row A stages, chosen when experts average at most
-  64 rows; MOE_GG_HALF=1 forces them.
+  64 rows; MOE_GG_HALF=1 forces them;
+* the fused expert kernel (gate/up, SwiGLU, down and combine in one pass),
+  chosen when experts average at most one 128-row tile; MOE_FUSED=1 forces it
+  wherever the hidden width is a multiple of 128 (experts with several row
+  tiles included).
 
 The switches are read once per process, so each run is a child process."""
 import os
@@ -36,3 +40,8 @@ def test_forward_small_with_two_sm_tiles():
 @pytest.mark.gpu
 def test_forward_small_with_half_height_down_tiles():
     run_small_cases(MOE_GG_PAIR="0", MOE_GG_HALF="1")
+
+
+@pytest.mark.gpu
+def test_forward_small_with_fused_expert_kernel():
+    run_small_cases(MOE_FUSED="1")

@@ -51,3 +51,22 @@ def test_layer_work_closed_forms():
 def test_peaks_file_or_fallback(tmp_path):
     p = roofline.measured_peaks(str(tmp_path / "missing.json"))
     assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0
+
+
+def test_fractions_name_the_binding_resource():
+    """frac = max(F / peak_F, B / peak_B) / t, whichever side of the ridge the
+    work lies on; both components are reported."""
+    peaks = {"hbm_gbs": 6000.0}
+    # 1 TFLOP and 1 GB in 1 ms: 1000 TFLOP/s (of 2000) and 1000 GB/s (of 6000)
+    r = roofline.fractions(1e12, 1e9, 1e-3, peaks, 2000.0)
+    assert r["bound"] == "tensor" and abs(r["tensor_frac"] - 0.5) < 1e-12
+    assert abs(r["hbm_frac"] - 1 / 6) < 1e-12 and r["frac"] == r["tensor_frac"]
+    # near the ridge (intensity 250 vs a ridge of 333): the bigger fraction wins
+    r = roofline.fractions(250e9, 1e9, 1e-3, peaks, 2000.0)
+    assert r["bound"] == "hbm" and abs(r["frac"] - 1 / 6) < 1e-12 and abs(r["tensor_frac"] - 0.125) < 1e-12
+
+
+def test_load_spread():
+    s = roofline.load_spread([4, 0, 2, 2])
+    assert s["active_experts"] == 3 and s["max"] == 4 and s["min"] == 0 and s["mean"] == 2.0
+    assert abs(s["cv"] - np.std([4, 0, 2, 2]) / 2.0) < 1e-15

@@ -3,10 +3,11 @@ allocate device memory (its fp32 accumulator is a static device array inside
 the library instead of a caller workspace).
 
 Called through the C ABI and compared with moe_combine, the entry point that
-takes a workspace, on two calls in a row (the static array keeps the first
-call's sums, so the second call checks that it is cleared).  This file is
-collected last so that a run stopping at the first failure has already run
-every other test; it also passes on its own in a fresh process.
+takes a workspace, and with the float64 oracle's layer output, on two calls in
+a row (the static array keeps the first call's sums, so the second call checks
+that it is cleared).  This file is collected last so that a run stopping at the
+first failure has already run every other test; it also passes on its own in a
+fresh process.
 """
 import ctypes
 
@@ -14,9 +15,11 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from sparse_mixture_experts_sigmoid_b200 import binding as B
-from sparse_mixture_experts_sigmoid_b200 import synth
 from sparse_mixture_experts_sigmoid_b200.workloads import Workload
+
+from support import OracleInputs, make_checked_layer, ocfg
 
 pytestmark = pytest.mark.gpu
 
@@ -30,27 +33,33 @@ CASES = [
 
 
 def _stages(w):
-    layer = synth.make_layer(w, "cuda")
+    cpu = make_checked_layer(w)      # routing margin enforced, so the oracle routes alike
+    layer = cpu.to("cuda")
     cfg = B.config_of(w)
     ids, gates, _, _ = B.route(cfg, layer.x, layer.w_router)
     _, offsets, srt, _ = B.permute(cfg, ids)
     act = B.grouped_swiglu(cfg, layer.x, layer.w_gate, layer.w_up, offsets, srt)
-    return cfg, layer, act, offsets, srt, gates
+    return cfg, cpu, layer, act, offsets, srt, gates
 
 
 @pytest.mark.parametrize("w", CASES, ids=[w.name for w in CASES])
 def test_noalloc_matches_workspace_combine_twice(w):
-    cfg, layer, act, offsets, srt, gates = _stages(w)
+    cfg, cpu, layer, act, offsets, srt, gates = _stages(w)
     y_ref = B.combine(cfg, act, layer.w_down, offsets, srt, gates).float()
     torch.cuda.synchronize()
     scale = y_ref.abs().max().item()
     assert scale > 0
+    a = OracleInputs(cpu)
+    y_oracle = oracle.forward(ocfg(w), a.x, a.wr, a.wg, a.wu, a.wd)
+    o_scale = np.abs(y_oracle).max()
     for call in range(2):
         y = B.combine_noalloc(cfg, act, layer.w_down, offsets, srt, gates)
         torch.cuda.synchronize()
         assert B.device_status() == 0
         err = (y.float() - y_ref).abs().max().item()
         assert np.isfinite(err) and err <= Y_TOL * scale, f"call {call}: {err} > {Y_TOL} * {scale}"
+        o_err = np.abs(y.float().cpu().numpy() - y_oracle).max()
+        assert o_err <= Y_TOL * o_scale, f"call {call} vs oracle: {o_err} > {Y_TOL} * {o_scale}"
 
 
 def test_noalloc_rejects_sizes_beyond_its_static_scratch():
