@@ -71,6 +71,8 @@ def parse():
     p.add_argument("--train-workloads", default="",
                    help="comma-separated workloads whose training step (forward + backward) is timed too")
     p.add_argument("--train-steps", type=int, default=20)
+    p.add_argument("--q4", action="store_true",
+                   help="time --workload with 4-bit routed experts (moe_forward_q4; decode-sized batches)")
     return p.parse_args()
 
 
@@ -320,12 +322,17 @@ def time_workload(args, w, ws_n, rank, local, steps, warmup, headline, q4=False)
     lw = roofline.layer_work(w, counts, q4=q4)
     lfr = roofline.fractions(lw["flops"], lw["bytes"], ms / 1e3, peaks, tpk)
     lfr["tensor_frac_of_burst"] = lfr["tflops"] / peaks["bf16_tflops"]
+    # both roofline fractions of every stage that ran (event-timed, so an upper bound on each kernel's time)
+    per_stage = {n: {"ms": stage[n], **{k_: v for k_, v in roofline.fractions(
+        work[n]["flops"], work[n]["bytes"], stage[n] / 1e3, peaks, tpk).items() if k_ in ("bound", "tensor_frac",
+                                                                                         "hbm_frac", "frac")}}
+                 for n in stage if n in work and stage[n] > 0.004}
     res = {"workload": w.name + ("_q4" if q4 else ""), "tokens_per_s": job_value(ws_n, w.T, ms), "ms_per_step": ms,
            "steps": K, "weights": "routed experts 4-bit (64-weight groups, fp32 scales)" if q4 else w.dtype,
            "warmup": W, "gpu_launches": launches, "layer": lfr,
            "dominant": {"stage": dom, "kernel": kname, "ms_per_launch": stage[dom],
                         "algorithmic_flops": work[dom]["flops"], "algorithmic_bytes": work[dom]["bytes"], **dfr},
-           "stages_ms": stage, "clocks": clocks, "tensor_peak": tpk, "tensor_peak_kind": tpk_kind,
+           "stages_ms": stage, "stages": per_stage, "clocks": clocks, "tensor_peak": tpk, "tensor_peak_kind": tpk_kind,
            "load": roofline.load_spread(counts)}
     res["_roof"] = (dom, kname, ksrc, dfr, peaks, tpk, tpk_kind)
 
@@ -419,7 +426,9 @@ def time_train(args, w, ws_n, local, steps, warmup):
 
 def bench_ours(args, w, ws_n, rank, local):
     torch.cuda.set_device(local)
-    head = time_workload(args, w, ws_n, rank, local, args.steps, args.warmup, headline=True)
+    if args.q4:
+        args.no_per_workload = True   # the 4-bit line is a single-workload measurement
+    head = time_workload(args, w, ws_n, rank, local, args.steps, args.warmup, headline=not args.q4, q4=args.q4)
     dom, kname, ksrc, dfr, peaks, tpk, tpk_kind = head.pop("_roof")
     bound = dfr["bound"]
     if bound == "tensor":
@@ -440,7 +449,8 @@ def bench_ours(args, w, ws_n, rank, local):
            "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w),
            "data": "synthetic (seeded; shapes and distributions of the workload)",
            "config": config_json(w, ws_n), "roofline": roof, "layer_roofline": head["layer"],
-           "stages_ms": head["stages_ms"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+           "stages_ms": head["stages_ms"], "stages": head["stages"], "gpu_launches": head["gpu_launches"],
+           "clocks": head["clocks"],
            "e2e": head.get("e2e"), "load": head["load"]}
     if "cpu_baseline" in head:
         out["cpu_baseline"] = head["cpu_baseline"]

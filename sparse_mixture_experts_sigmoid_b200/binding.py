@@ -83,7 +83,7 @@ def lib() -> ctypes.CDLL:
                                   ctypes.c_int),
             "moe_backward": ([C] + [P] * 11 + [S] + [P] * 10, ctypes.c_int),
             "moe_quantize_q4": ([P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, P, P, P], ctypes.c_int),
-            "moe_forward_q4": ([C, ctypes.POINTER(RouteOpts)] + [P] * 14 + [P, S, P], ctypes.c_int),
+            "moe_forward_q4": ([C, ctypes.POINTER(RouteOpts)] + [P] * 13 + [P, S, P], ctypes.c_int),
             "moe_balance_loss": ([C, P, P, ctypes.c_float, P, P, P], ctypes.c_int),
             "moe_decode_max_rows": ([], ctypes.c_int32),
             "moe_device_status": ([P], ctypes.c_int),

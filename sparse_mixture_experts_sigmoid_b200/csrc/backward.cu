@@ -5,6 +5,8 @@
 // expert and balance bias of "Small MoE Architecture, in depth", SmallMoE;
 // "Small models, sparse experts", "Dispatch decides everything" trains it):
 //
+//   0. x and dy rows copied into the padded grouped layout the backward GEMMs
+//      read by TMA (gather_pad_kernel)
 //   1. routed experts, rows grouped by expert:  r = W_down^T dy;  the gate
 //      gradient r . a;  du, dv through silu(u) * v;  gate * a kept for dW_down
 //      (grouped_bwd.cu, SWIGLU)
@@ -21,10 +23,81 @@
 // The top-k selection (and the balance bias) passes no gradient.
 #include <algorithm>
 
+#include "grouped_tiles.cuh"
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
+
+// The routed rows of x and dy copied into the padded grouped layout of the
+// backward GEMMs (expert e's rows from row 64 * sum_{e' < e} ceil(count_e' /
+// 64), in grouped order), with the padding rows -- past each segment's end up
+// to the next multiple of 64 -- zeroed in x_g, dy_g, dH and ga.  CTA-strided
+// over 64-row blocks; 16-byte copies.
+struct GatherPadArgs {
+    const __nv_bfloat16 *x, *dy;
+    const int32_t *offsets, *sorted_rows;
+    int E, k, d, h;
+    int64_t T, R;
+    __nv_bfloat16 *xg, *dyg, *dh, *ga;
+    uint32_t *err;
+};
+__global__ void __launch_bounds__(256) gather_pad_kernel(GatherPadArgs a) {
+    __shared__ int blk[MOE_MAX_EXPERTS + 1], off[MOE_MAX_EXPERTS + 1], end[MOE_MAX_EXPERTS + 1];
+    __shared__ int nblk;
+    pdl_wait();
+    pdl_launch_dependents();
+    if (threadIdx.x < 32) {
+        GemmParams g{};
+        g.offsets = a.offsets;
+        g.E = a.E;
+        g.rows = a.R;
+        g.err = a.err;
+        int n = 0;
+        gg::build_tiles<64>(g, blk, off, end, &n);
+        if (threadIdx.x == 31) nblk = n;
+    }
+    __syncthreads();
+    const int cpr = a.d / 8;                 // 16-byte chunks per x / dy row
+    for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
+        const gg::Tile tl = gg::decode(b, 1, blk, a.E);
+        const int64_t pr0 = (int64_t)b * 64;               // first padded row of the block
+        const int64_t r0 = (int64_t)off[tl.e] + tl.m * 64;  // its first grouped row
+        // x_g and dy_g: copy or zero, 16 bytes per thread step
+        for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
+            const int q = i / cpr, c = i - q * cpr;
+            const int64_t r = r0 + q;
+            int64_t t = -1;
+            if (r < end[tl.e]) {
+                const int v = a.sorted_rows[r];
+                t = (v >= 0 && v < a.R) ? v / a.k : -1;
+                if (t < 0 || t >= a.T) {
+                    atomicOr(a.err, kErrInput);
+                    t = -1;
+                }
+            }
+            uint4 vx = make_uint4(0, 0, 0, 0), vd = vx;
+            if (t >= 0) {
+                vx = *reinterpret_cast<const uint4 *>(a.x + t * a.d + 8 * c);
+                vd = *reinterpret_cast<const uint4 *>(a.dy + t * a.d + 8 * c);
+            }
+            *reinterpret_cast<uint4 *>(a.xg + (pr0 + q) * a.d + 8 * c) = vx;
+            *reinterpret_cast<uint4 *>(a.dyg + (pr0 + q) * a.d + 8 * c) = vd;
+        }
+        // dH and ga: zero the padding rows (the SWIGLU epilogue writes the others)
+        const int64_t rem = (int64_t)end[tl.e] - r0;
+        const int64_t valid = rem < 64 ? rem : 64;
+        const int hc = a.h / 8;
+        for (int64_t q = valid; q < 64; ++q) {
+            uint4 *dh = reinterpret_cast<uint4 *>(a.dh + (pr0 + q) * 2 * a.h);
+            uint4 *ga = reinterpret_cast<uint4 *>(a.ga + (pr0 + q) * a.h);
+            for (int i = threadIdx.x; i < 3 * hc; i += blockDim.x) {
+                if (i < 2 * hc) dh[i] = make_uint4(0, 0, 0, 0);
+                else ga[i - 2 * hc] = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+}
 
 struct RouterBwdArgs {
     int64_t T;
@@ -166,7 +239,10 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
     float *dsg = ws_part<float>(ws, L, P_DSG);
     char *dh = ws_part<char>(ws, L, P_DH);
     char *dhs = ws_part<char>(ws, L, P_DHS);
-    void *ga = ws_part<void>(ws, L, P_ACT);      // gate * a of the routed rows (act is not needed any more)
+    void *ga = ws_part<void>(ws, L, P_GA);       // gate * a of the routed rows, padded layout
+    void *xg = ws_part<void>(ws, L, P_XG);       // x and dy rows in the padded grouped layout
+    void *dyg = ws_part<void>(ws, L, P_DYG);
+    const uint64_t Rp = (uint64_t)padded_rows(R, E);
     void *gas = ws_part<void>(ws, L, P_GAS);
     void *dlb = ws_part<void>(ws, L, P_DLB);
     float *dls = ws_part<float>(ws, L, P_DLS);
@@ -181,10 +257,19 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
         g.kind = kind;
         return g;
     };
-    // 1. routed: r = W_down^T dy over grouped rows (dy gathered by token)
+    // 0. x and dy rows into the padded grouped layout; zero padding rows
+    if (e == cudaSuccess) {
+        GatherPadArgs a{static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(dy), offsets, srt,
+                        E, c->k, d, h, T, R, static_cast<__nv_bfloat16 *>(xg), static_cast<__nv_bfloat16 *>(dyg),
+                        reinterpret_cast<__nv_bfloat16 *>(dh), static_cast<__nv_bfloat16 *>(ga), err};
+        const unsigned blocks = (unsigned)std::min<int64_t>((int64_t)(Rp / 64), 8LL * num_sms());
+        e = launch_kernel(gather_pad_kernel, std::max(1u, blocks), 256, 0, s, a);
+    }
+    // 1. routed: r = W_down^T dy over grouped rows
     if (e == cudaSuccess) {
         BwdGemm g = base(BwdGemm::SWIGLU);
-        g.gather_a = true;
+        g.padded = true;
+        g.a0 = {dyg, Rp, (uint64_t)d, (uint64_t)d};
         g.b0 = {w_down, (uint64_t)E * d, (uint64_t)h, (uint64_t)h};
         g.offsets = offsets;
         g.sorted_rows = srt;
@@ -195,8 +280,6 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
         g.nranges = 1;
         g.Kr = d;
         g.N = h;
-        g.gsrc = dy;
-        g.gwidth = d;
         g.hpre = hpre;
         g.gate = gates;
         g.dh = dh;
@@ -235,8 +318,9 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
     //    and the router's
     if (e == cudaSuccess) {
         BwdGemm g = base(BwdGemm::SCATTER);
-        g.a0 = {dh, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
-        g.a1 = {dh + (size_t)h * 2, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
+        g.padded = true;
+        g.a0 = {dh, Rp, (uint64_t)h, 2 * (uint64_t)h};
+        g.a1 = {dh + (size_t)h * 2, Rp, (uint64_t)h, 2 * (uint64_t)h};
         g.b0 = {w_gate, (uint64_t)E * h, (uint64_t)d, (uint64_t)d};
         g.b1 = {w_up, (uint64_t)E * h, (uint64_t)d, (uint64_t)d};
         g.offsets = offsets;
@@ -296,8 +380,9 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
     if (e == cudaSuccess) {
         // dW_down[e] = sum over the expert's rows of dy_t (x) (gate * a)
         BwdGemm g = base(BwdGemm::WEIGHT);
-        g.gather_a = true;
-        g.b0 = {ga, (uint64_t)R, (uint64_t)h, (uint64_t)h};
+        g.padded = true;
+        g.a0 = {dyg, Rp, (uint64_t)d, (uint64_t)d};
+        g.b0 = {ga, Rp, (uint64_t)h, (uint64_t)h};
         g.offsets = offsets;
         g.sorted_rows = srt;
         g.groups = E;
@@ -307,8 +392,6 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
         g.M = d;
         g.halves = 1;
         g.N = h;
-        g.gsrc = dy;
-        g.gwidth = d;
         g.out0 = dw_down;
         g.err = err;
         e = launch_bwd_gemm(g, s);
@@ -316,9 +399,10 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
     if (e == cudaSuccess) {
         // dW_gate[e] / dW_up[e] = sum over the expert's rows of du / dv (x) x_t
         BwdGemm g = base(BwdGemm::WEIGHT);
-        g.gather_b = true;
-        g.a0 = {dh, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
-        g.a1 = {dh + (size_t)h * 2, (uint64_t)R, (uint64_t)h, 2 * (uint64_t)h};
+        g.padded = true;
+        g.a0 = {dh, Rp, (uint64_t)h, 2 * (uint64_t)h};
+        g.a1 = {dh + (size_t)h * 2, Rp, (uint64_t)h, 2 * (uint64_t)h};
+        g.b0 = {xg, Rp, (uint64_t)d, (uint64_t)d};
         g.offsets = offsets;
         g.sorted_rows = srt;
         g.groups = E;
@@ -328,8 +412,6 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
         g.M = h;
         g.halves = 2;
         g.N = d;
-        g.gsrc = x;
-        g.gwidth = d;
         g.out0 = dw_gate;
         g.out1 = dw_up;
         g.err = err;

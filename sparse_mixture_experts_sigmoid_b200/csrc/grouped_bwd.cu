@@ -15,22 +15,25 @@
 // and the same for the shared expert (one dense segment, gate sigmoid(w_s.x))
 // and for the router (dx += dl W_router, dW_router = dl^T x).
 //
+// Every operand comes by TMA.  The routed rows live in a padded grouped
+// layout: expert e's rows start at row 64 * (sum over e' < e of
+// ceil(count_e' / 64)), and the rows from the end of its segment to the next
+// multiple of 64 are zero (x and dy are copied into that layout by the
+// backward's first kernel; du | dv and gate * a are written into it by the
+// SWIGLU epilogue).  So a weight-gradient tile reads whole 64-row K blocks of
+// both operands and the rows past a segment's end add nothing.
+//
 // Two tile schemes share one persistent kernel (one CTA per SM; warps 0-3
-// epilogue, warp 4 TMA producer, warp 5 TMEM allocator + MMA issuer, warps
-// 6-13 gather):
+// epilogue, warp 4 TMA producer, warp 5 TMEM allocator + MMA issuer):
 //  * ROWS: tiles of 128 grouped rows x 256 output columns, K over the
 //    weight's reduction dimension in blocks of 64, split into up to two K
-//    ranges (the gate half and the up half of [du | dv]).  A is K-major
-//    (grouped rows: gathered by token index with cp.async, or TMA); B is a
-//    weight read MN-major (its rows are the K index, contiguous along N), four
-//    64 x 64 TMA boxes per K block.
+//    ranges (the gate half and the up half of [du | dv]).  A is K-major; B is
+//    a weight read MN-major (its rows are the K index, contiguous along N),
+//    four 64 x 64 TMA boxes per K block.
 //  * WGRAD: tiles of 128 weight rows x 256 weight columns of one expert, K
-//    over that expert's grouped rows (a ragged length) in blocks of 64.  Both
-//    operands are MN-major: each grouped row contributes one 128-byte k-row per
-//    64 columns, by TMA from a grouped tensor or gathered by token index.  Rows
-//    past the segment's end are zero-filled in the gathered operand (or read
-//    past the tensor's end, where TMA fills zeros), so the next expert's rows
-//    add nothing.  An expert without rows writes a zero gradient.
+//    over that expert's (padded) rows in blocks of 64.  Both operands are
+//    MN-major: each row contributes one 128-byte k-row per 64 columns.  An
+//    expert without rows writes a zero gradient.
 // MN-major shared-memory operands use the canonical 128-byte-swizzled layout:
 // 64-element atoms along M/N 8 KB apart (leading offset), 8-row k groups
 // 1 KB apart (stride offset); a K slice of 16 advances the start by 2 KB.
@@ -58,8 +61,7 @@ constexpr int kAtom = 8192;               // one MN-major atom column: 64 k-rows
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
-constexpr int kGatherWarp0 = 6;
-constexpr int kGatherThreads = 256;
+constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 
 enum { ROWS = 0, WGRAD = 1 };
@@ -94,87 +96,30 @@ constexpr uint32_t idesc_bwd() {
 struct Params {
     GemmParams g;            // grouping (offsets, sorted_rows, E = groups, k, rows, T, err) and, for
                              // SCATTER, N = output width, y_acc, gates (nullptr: weight 1)
+    bool padded;             // routed operands in the padded grouped layout (see the top of the file)
     int nranges;             // ROWS: K ranges (1 or 2)
     int Kr;                  // ROWS: K extent of each range (weight rows per group per range)
     int N;                   // output columns (ROWS) / weight columns (WGRAD)
     int M;                   // WGRAD: weight rows per group per half
     int halves;              // WGRAD: 1 or 2 (gate | up)
-    const __nv_bfloat16 *gsrc;   // gathered operand [T, gwidth] (rows picked by token index)
-    int gwidth;
     // SWIGLU epilogue
-    const __nv_bfloat16 *hpre;   // [rows, 2N] kept pre-activations (u | v)
+    const __nv_bfloat16 *hpre;   // [rows, 2N] kept pre-activations (u | v), unpadded grouped rows
     const float *gate;           // routed: [R] by assignment; dense: [T]
-    __nv_bfloat16 *dh;           // [rows, 2N] out: du | dv
-    __nv_bfloat16 *ga;           // [rows, N] out: gate * a
+    __nv_bfloat16 *dh;           // [rows (padded), 2N] out: du | dv
+    __nv_bfloat16 *ga;           // [rows (padded), N] out: gate * a
     float *dgate;                // routed: [R] by assignment; dense: [T]; accumulated
     // STORE epilogue: row-major [groups * M, N] per half
     void *out0, *out1;
     bool out_f32;
 };
 
-// ------------------------------------------------------------------ gathers
-
-// ROWS: the 128 grouped rows of tile `tl` for K block kb of a K-major A
-// operand gathered from gsrc (one 128-byte segment per row).  Thread g
-// handles rows g / 8 + 32 q and chunk g % 8.
-__device__ __forceinline__ void gather_rows_kmajor(const Params &p, const int *seg_off, const int *seg_end,
-                                                   const Tile &tl, int kb, int g, uint8_t *dst) {
-    const int c = g & 7, rg = g >> 3;
-    const int64_t row0 = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM;
-    const int col = kb * BK + c * 8;
-    const bool colok = col < p.gwidth;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int row = rg + 32 * q;
-        const int64_t r = row0 + row;
-        int64_t t = -1;
-        if (r < seg_end[tl.e]) {
-            const int v = p.g.sorted_rows ? p.g.sorted_rows[r] : (int)r;
-            if (v >= 0 && v < p.g.rows) t = p.g.sorted_rows ? v / p.g.k : v;
-            if (t >= p.g.T) t = -1;
-            if (t < 0) atomicOr(p.g.err, kErrInput);
-        }
-        const bool ok = t >= 0 && colok;
-        cp_async16(dst + row * 128 + ((c ^ (row & 7)) << 4), ok ? (const void *)(p.gsrc + t * p.gwidth + col)
-                                                               : (const void *)p.gsrc, ok ? 16 : 0);
-    }
-}
-
-// WGRAD: the 64 grouped rows of K block kb of group e as k-rows of an
-// MN-major operand covering NSEG x 64 columns from c0, gathered from gsrc.
-// Row q of the block lands at byte q * 128 of each 8 KB atom column (chunks
-// swizzled by q % 8); rows past the segment are zero-filled.
-template <int NSEG>
-__device__ __forceinline__ void gather_rows_mnmajor(const Params &p, int64_t seg0, int64_t seg1, int kb, int c0,
-                                                    int g, uint8_t *dst) {
-    constexpr int CPR = NSEG * 8;                 // 16-byte chunks per row
-    constexpr int PER = 64 * CPR / kGatherThreads; // chunks per thread (4 or 8)
-    const int row = g / (kGatherThreads / 64);    // 4 threads per row
-    const int cbase = (g % (kGatherThreads / 64)) * PER;
-    const int64_t r = seg0 + (int64_t)kb * 64 + row;
-    int64_t t = -1;
-    if (r < seg1) {
-        const int v = p.g.sorted_rows ? p.g.sorted_rows[r] : (int)r;
-        if (v >= 0 && v < p.g.rows) t = p.g.sorted_rows ? v / p.g.k : v;
-        if (t >= p.g.T) t = -1;
-        if (t < 0) atomicOr(p.g.err, kErrInput);
-    }
-#pragma unroll
-    for (int q = 0; q < PER; ++q) {
-        const int ch = cbase + q;
-        const int seg = ch >> 3, c = ch & 7;
-        const int col = c0 + seg * 64 + c * 8;
-        const bool ok = t >= 0 && col < p.gwidth;
-        cp_async16(dst + seg * kAtom + row * 128 + ((c ^ (row & 7)) << 4),
-                   ok ? (const void *)(p.gsrc + t * p.gwidth + col) : (const void *)p.gsrc, ok ? 16 : 0);
-    }
-}
-
 // ------------------------------------------------------------------ epilogues
 
 // ROWS / SWIGLU: grouped row r (valid) of column tile nt; D = r_i over 256
-// columns from TMEM address tbase.
-__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int64_t r, bool valid, uint32_t tbase) {
+// columns from TMEM address tbase.  The outputs go to row ro (r in the padded
+// layout).
+__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int64_t r, int64_t ro, bool valid,
+                                                uint32_t tbase) {
     if (!__any_sync(0xffffffffu, valid)) return;
     const int N = p.N;
     float g = 0.f;
@@ -231,10 +176,10 @@ __device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int64_t
                     b = __floats2bfloat162_rn(ga[0], ga[1]);
                     ga2[q] = *reinterpret_cast<uint32_t *>(&b);
                 }
-                *reinterpret_cast<uint4 *>(p.dh + r * 2 * (int64_t)N + col) = make_uint4(du2[0], du2[1], du2[2], du2[3]);
-                *reinterpret_cast<uint4 *>(p.dh + r * 2 * (int64_t)N + N + col) =
+                *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + col) = make_uint4(du2[0], du2[1], du2[2], du2[3]);
+                *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + N + col) =
                     make_uint4(dv2[0], dv2[1], dv2[2], dv2[3]);
-                *reinterpret_cast<uint4 *>(p.ga + r * (int64_t)N + col) = make_uint4(ga2[0], ga2[1], ga2[2], ga2[3]);
+                *reinterpret_cast<uint4 *>(p.ga + ro * (int64_t)N + col) = make_uint4(ga2[0], ga2[1], ga2[2], ga2[3]);
             }
         }
     }
@@ -305,16 +250,12 @@ __device__ __forceinline__ WTile wdecode(int id, int mtiles, int ntiles, int hal
     return w;
 }
 
-template <int MODE, bool AG, bool BG, int EPI>
-__global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
+template <int MODE, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1, Params p) {
-    static_assert(!(MODE == ROWS && BG), "ROWS reads its weights by TMA");
-    constexpr bool GATHER = AG || BG;
     constexpr uint32_t kIdesc = idesc_bwd<MODE>();
     constexpr int kEpiStage = EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0;
-    constexpr uint32_t kTxA = AG ? 0 : kAStage;
-    constexpr uint32_t kTxB = BG ? 0 : kBStage;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -325,12 +266,13 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
     int *tile_start = reinterpret_cast<int *>(ctrl + 1);
     int *seg_off = tile_start + (p.g.E + 1);
     int *seg_end = seg_off + (p.g.E + 1);
+    int *blk64 = seg_end + (p.g.E + 1);   // padded layout: group e starts at row 64 * blk64[e]
     volatile int *abort = &ctrl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&ctrl->full[s], GATHER ? 1 + kGatherThreads : 1);
+            mbar_init(&ctrl->full[s], 1);
             mbar_init(&ctrl->empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -342,11 +284,15 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
     }
     if (warp == kMmaWarp) tmem_alloc(&ctrl->tmem_base, kTmemCols);
     if (warp == kTmaWarp && lane == 0) {
-        if (!AG) prefetch_tmap(&tmA0);
-        if (!BG) prefetch_tmap(&tmB0);
+        prefetch_tmap(&tmA0);
+        prefetch_tmap(&tmB0);
     }
     pdl_wait();
-    if (warp == kTmaWarp) build_tiles<(MODE == ROWS ? BM : 64)>(p.g, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
+    if (warp == kTmaWarp) {
+        int blocks64;
+        build_tiles<64>(p.g, blk64, seg_off, seg_end, &blocks64);
+        if (MODE == ROWS) build_tiles<BM>(p.g, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -357,12 +303,13 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
     const int ntiles = (p.N + BN - 1) / BN;
     const int mtiles = MODE == WGRAD ? (p.M + BM - 1) / BM : 0;
     const int total = MODE == ROWS ? ctrl->n_mtiles * ntiles : nE * p.halves * mtiles * ntiles;
-    const int nk_rows = MODE == ROWS ? p.nranges * ((p.Kr + BK - 1) / BK) : 0;
     const int kpr = (p.Kr + BK - 1) / BK;   // ROWS: K blocks per range
+    // first row of group e in the operands' layout
+    auto op_row0 = [&](int e) -> int { return p.padded ? 64 * blk64[e] : seg_off[e]; };
     // K blocks of a tile
     auto tile_nk = [&](int id) -> int {
         if constexpr (MODE == ROWS) {
-            return nk_rows;
+            return p.nranges * kpr;
         } else {
             const WTile w = wdecode(id, mtiles, ntiles, p.halves);
             return (seg_end[w.e] - seg_off[w.e] + 63) / 64;
@@ -370,7 +317,7 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
     };
 
     if (warp == kTmaWarp) {
-        if (lane == 0 && (kTxA + kTxB) > 0) {
+        if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
@@ -381,36 +328,36 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&ctrl->full[s], kTxA + kTxB);
+                    mbar_expect_tx(&ctrl->full[s], kAStage + kBStage);
                     uint8_t *a = sA + s * kAStage, *b = sB + s * kBStage;
                     if constexpr (MODE == ROWS) {
                         const Tile tl = decode(id, ntiles, tile_start, nE);
                         const int range = kb / kpr, kr = kb - range * kpr;
                         const CUtensorMap *ma = range ? &tmA1 : &tmA0;
                         const CUtensorMap *mb = range ? &tmB1 : &tmB0;
-                        if (!AG) tma_load_2d(ma, a, &ctrl->full[s], kr * BK, seg_off[tl.e] + tl.m * BM);
+                        tma_load_2d(ma, a, &ctrl->full[s], kr * BK, op_row0(tl.e) + tl.m * BM);
                         const int brow = tl.e * p.Kr + kr * BK;
 #pragma unroll
-                        for (int j = 0; j < BN / 64; ++j) tma_load_2d(mb, b + j * kAtom, &ctrl->full[s], tl.n * BN + 64 * j, brow);
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(mb, b + j * kAtom, &ctrl->full[s], tl.n * BN + 64 * j, brow);
                     } else {
                         const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                        const int krow = seg_off[w.e] + kb * 64;
-                        if (!AG) {
-                            const CUtensorMap *ma = w.half ? &tmA1 : &tmA0;
+                        const int krow = op_row0(w.e) + kb * 64;
+                        const CUtensorMap *ma = w.half ? &tmA1 : &tmA0;
 #pragma unroll
-                            for (int j = 0; j < BM / 64; ++j) tma_load_2d(ma, a + j * kAtom, &ctrl->full[s], w.mt * BM + 64 * j, krow);
-                        }
-                        if (!BG) {
+                        for (int j = 0; j < BM / 64; ++j)
+                            tma_load_2d(ma, a + j * kAtom, &ctrl->full[s], w.mt * BM + 64 * j, krow);
 #pragma unroll
-                            for (int j = 0; j < BN / 64; ++j) tma_load_2d(&tmB0, b + j * kAtom, &ctrl->full[s], w.nt * BN + 64 * j, krow);
-                        }
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(&tmB0, b + j * kAtom, &ctrl->full[s], w.nt * BN + 64 * j, krow);
                     }
                 }
             }
             if (!ok) {
                 for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j) {
                     const uint64_t t0 = globaltimer();
-                    while (!mbar_try_wait(&ctrl->full[j % kStages], (j / kStages) & 1) && globaltimer() - t0 < 100000000ull) {
+                    while (!mbar_try_wait(&ctrl->full[j % kStages], (j / kStages) & 1) &&
+                           globaltimer() - t0 < 100000000ull) {
                     }
                 }
             }
@@ -431,7 +378,6 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
                         ok = false;
                         break;
                     }
-                    if constexpr (GATHER) fence_proxy_async();
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
@@ -456,11 +402,15 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
             const uint32_t tb = tmem + acc * BN + lane_base;
             if constexpr (MODE == ROWS) {
                 const Tile tl = decode(id, ntiles, tile_start, nE);
-                const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM + row;
+                const int64_t local = (int64_t)tl.m * BM + row;
+                const int64_t r = (int64_t)seg_off[tl.e] + local;
                 const bool valid = r < seg_end[tl.e];
-                if constexpr (EPI == EPI_SWIGLU) epilogue_swiglu(p, tl.n, r, valid, tb);
-                else gg::epilogue_row<gg::DOWN, __nv_bfloat16, BN>(p.g, tl.n, r, valid, tb,
-                                                                    reinterpret_cast<float *>(sEpi + warp * gg::kEpiStageBytes));
+                if constexpr (EPI == EPI_SWIGLU) {
+                    epilogue_swiglu(p, tl.n, r, op_row0(tl.e) + local, valid, tb);
+                } else {
+                    gg::epilogue_row<gg::DOWN, __nv_bfloat16, BN>(
+                        p.g, tl.n, r, valid, tb, reinterpret_cast<float *>(sEpi + warp * gg::kEpiStageBytes));
+                }
             } else {
                 const WTile w = wdecode(id, mtiles, ntiles, p.halves);
                 epilogue_store(p, w.e, w.half, w.mt * BM + row, w.nt * BN, seg_end[w.e] > seg_off[w.e], tb);
@@ -468,31 +418,6 @@ __global__ void __launch_bounds__((AG || BG) ? 192 + kGatherThreads : 192, 1)
             tc_fence_before();
             mbar_arrive(&ctrl->tempty[acc]);
         }
-    } else if (GATHER && warp >= kGatherWarp0) {
-        const int g = threadIdx.x - kGatherWarp0 * 32;
-        uint32_t it = 0;
-        bool ok = true;
-        for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-            const int nk = tile_nk(id);
-            for (int kb = 0; kb < nk; ++kb, ++it) {
-                const int s = it % kStages;
-                if (!wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, p.g.err)) {
-                    ok = false;
-                    break;
-                }
-                if constexpr (MODE == ROWS) {
-                    const Tile tl = decode(id, ntiles, tile_start, nE);
-                    gather_rows_kmajor(p, seg_off, seg_end, tl, kb, g, sA + s * kAStage);
-                } else {
-                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                    if constexpr (AG) gather_rows_mnmajor<BM / 64>(p, seg_off[w.e], seg_end[w.e], kb, w.mt * BM, g, sA + s * kAStage);
-                    else gather_rows_mnmajor<BN / 64>(p, seg_off[w.e], seg_end[w.e], kb, w.nt * BN, g, sB + s * kBStage);
-                }
-                cp_async_commit();
-                cp_async_arrive_noinc(&ctrl->full[s]);
-            }
-        }
-        cp_async_wait<0>();
     }
 
     tc_fence_before();
@@ -521,27 +446,25 @@ bool map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, bool AG, bool BG, int EPI>
+template <int MODE, int EPI>
 cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOperand &b0, const BwdOperand &b1,
                        const gb::Params &p, cudaStream_t s) {
     using namespace gb;
     CUtensorMap mA0, mA1, mB0, mB1;
     // ROWS: A K-major boxes of 128 rows; otherwise MN-major boxes of 64 k-rows
     const uint32_t a_box = MODE == ROWS ? BM : 64;
-    if (!AG && !map_bf16(&mA0, a0.base, a0.rows, a0.cols, a0.ld, a_box)) return cudaErrorInvalidValue;
-    if (!BG && !map_bf16(&mB0, b0.base, b0.rows, b0.cols, b0.ld, 64)) return cudaErrorInvalidValue;
-    if (!AG && a1.base) {
+    if (!map_bf16(&mA0, a0.base, a0.rows, a0.cols, a0.ld, a_box)) return cudaErrorInvalidValue;
+    if (!map_bf16(&mB0, b0.base, b0.rows, b0.cols, b0.ld, 64)) return cudaErrorInvalidValue;
+    if (a1.base) {
         if (!map_bf16(&mA1, a1.base, a1.rows, a1.cols, a1.ld, a_box)) return cudaErrorInvalidValue;
     } else {
-        mA1 = AG ? mB0 : mA0;
+        mA1 = mA0;
     }
-    if (!BG && b1.base) {
+    if (b1.base) {
         if (!map_bf16(&mB1, b1.base, b1.rows, b1.cols, b1.ld, 64)) return cudaErrorInvalidValue;
     } else {
-        mB1 = BG ? mA0 : mB0;
+        mB1 = mB0;
     }
-    if (AG) mA0 = mA1 = mB0;   // unused
-    if (BG) mB0 = mB1 = mA0;   // unused
     const int nE = p.g.offsets ? p.g.E : 1;
     const int ntiles = (p.N + BN - 1) / BN;
     int64_t max_tiles;
@@ -550,11 +473,11 @@ cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOper
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
     const size_t smem = 1024 + (size_t)kStages * (kAStage + kBStage) +
                         (EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0) + sizeof(Ctrl) +
-                        3 * sizeof(int) * (p.g.E + 1);
-    auto kern = bwd_gemm_kernel<MODE, AG, BG, EPI>;
+                        4 * sizeof(int) * (p.g.E + 1);
+    auto kern = bwd_gemm_kernel<MODE, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(kern, grid, (AG || BG) ? 192 + kGatherThreads : 192, smem, s, mA0, mA1, mB0, mB1, p);
+    return launch_kernel(kern, grid, kThreads, smem, s, mA0, mA1, mB0, mB1, p);
 }
 
 }  // namespace
@@ -564,13 +487,12 @@ cudaError_t launch_bwd_gemm(const BwdGemm &L, cudaStream_t s) {
     Params p{};
     p.g = GemmParams{L.offsets, L.sorted_rows, L.groups, L.k, L.rows, L.T, 0, L.N, nullptr, nullptr, L.acc,
                      nullptr, L.err};
+    p.padded = L.padded;
     p.nranges = L.nranges;
     p.Kr = L.Kr;
     p.N = L.N;
     p.M = L.M;
     p.halves = L.halves;
-    p.gsrc = static_cast<const __nv_bfloat16 *>(L.gsrc);
-    p.gwidth = L.gwidth;
     p.hpre = static_cast<const __nv_bfloat16 *>(L.hpre);
     p.gate = L.gate;
     p.dh = static_cast<__nv_bfloat16 *>(L.dh);
@@ -581,15 +503,9 @@ cudaError_t launch_bwd_gemm(const BwdGemm &L, cudaStream_t s) {
     p.out_f32 = L.out_f32;
     if (L.rows <= 0 && L.kind != BwdGemm::WEIGHT) return cudaSuccess;
     switch (L.kind) {
-        case BwdGemm::SWIGLU:
-            return L.gather_a ? launch_bwd<ROWS, true, false, EPI_SWIGLU>(L.a0, L.a1, L.b0, L.b1, p, s)
-                              : launch_bwd<ROWS, false, false, EPI_SWIGLU>(L.a0, L.a1, L.b0, L.b1, p, s);
-        case BwdGemm::SCATTER:
-            return launch_bwd<ROWS, false, false, EPI_SCATTER>(L.a0, L.a1, L.b0, L.b1, p, s);
-        default:
-            if (L.gather_a) return launch_bwd<WGRAD, true, false, EPI_STORE>(L.a0, L.a1, L.b0, L.b1, p, s);
-            if (L.gather_b) return launch_bwd<WGRAD, false, true, EPI_STORE>(L.a0, L.a1, L.b0, L.b1, p, s);
-            return launch_bwd<WGRAD, false, false, EPI_STORE>(L.a0, L.a1, L.b0, L.b1, p, s);
+        case BwdGemm::SWIGLU: return launch_bwd<ROWS, EPI_SWIGLU>(L.a0, L.a1, L.b0, L.b1, p, s);
+        case BwdGemm::SCATTER: return launch_bwd<ROWS, EPI_SCATTER>(L.a0, L.a1, L.b0, L.b1, p, s);
+        default: return launch_bwd<WGRAD, EPI_STORE>(L.a0, L.a1, L.b0, L.b1, p, s);
     }
 }
 

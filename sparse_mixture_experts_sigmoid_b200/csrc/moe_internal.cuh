@@ -244,14 +244,12 @@ struct BwdGemm {
     // SCATTER: rows x N tiles added (weight 1) into acc[token];
     // WEIGHT: per group, M x N weight-gradient tiles reduced over the group's rows.
     enum Kind { SWIGLU, SCATTER, WEIGHT } kind;
-    bool gather_a, gather_b;      // operand gathered from gsrc by token index
+    bool padded;                  // routed operands in the padded grouped layout (64-row aligned segments)
     BwdOperand a0, a1, b0, b1;    // TMA operands (a1/b1: second K range or second half)
     const int32_t *offsets, *sorted_rows;   // grouping (offsets == nullptr: one dense segment)
     int groups, k;
     int64_t rows, T;
     int nranges, Kr, N, M, halves;
-    const void *gsrc;             // [T, gwidth] bf16
-    int gwidth;
     const void *hpre;             // SWIGLU: [rows, 2N] pre-activations (u | v)
     const float *gate;            // SWIGLU: routed [R] by assignment / dense [T]
     void *dh, *ga;                // SWIGLU out: [rows, 2N] du | dv, [rows, N] gate * a
@@ -269,7 +267,7 @@ enum WsPart {
     P_IDS, P_GATES, P_SG, P_COUNTS, P_OFFSETS, P_SORTED, P_INV, P_ACT, P_ACTS, P_YACC, P_PERM, P_LOGITS,
     P_STATS,
     // training: kept by moe_forward_train for moe_backward, and the backward's scratch
-    P_PROBS, P_HPRE, P_HPRES, P_DG, P_DSG, P_DH, P_DHS, P_GAS, P_DLB, P_DLS,
+    P_PROBS, P_HPRE, P_HPRES, P_DG, P_DSG, P_DH, P_DHS, P_GAS, P_DLB, P_DLS, P_XG, P_DYG, P_GA,
     P_N
 };
 struct WsLayout {
@@ -284,6 +282,9 @@ T *ws_part(void *ws, const WsLayout &L, WsPart p) {
 }
 // Row stride (elements) of the bf16 router-gradient rows: E rounded up to 8.
 inline int dl_stride(int E) { return (E + 7) / 8 * 8; }
+// Rows of the backward's padded grouped layout (each expert's segment rounded
+// up to a multiple of 64 rows): at most R + 63 E.
+inline int64_t padded_rows(int64_t R, int E) { return R + 63LL * E; }
 
 // Launch planning shared by the entry points (defined in moe_api.cu).
 uint32_t *device_error_word();   // the library's device error word on the current device
