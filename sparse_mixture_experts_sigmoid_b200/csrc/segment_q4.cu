@@ -12,11 +12,11 @@
 // the value represented is (nibble - 8) * s.
 //
 //   quantize_q4_kernel: one thread per group of 64 weights.
-//   seg_gateup_q4_kernel: one warp per (expert, hidden row): the warp streams
-//     the 4-bit gate and up rows once (16 bytes = 32 weights per lane per
-//     load, the group's scale alongside) and applies them to every grouped row
-//     of the expert; act = silu(gate) * up in bf16.
-//   down_direct_q4_kernel: one warp per output element (t, n):
+//   seg_gateup_q4_kernel: one warp per (expert, block of hidden rows): the
+//     warp streams the 4-bit gate and up rows once (16 bytes = 32 weights per
+//     lane per load, the group's scale alongside) and applies them to every
+//     grouped row of the expert; act = silu(gate) * up in bf16.
+//   down_direct_q4_kernel: one warp per block of 4 output elements (t, n):
 //     y = sum_j g_j (W_down[e_j, n] . act) (+ the bf16 shared expert), written
 //     straight into y.
 // The weights are dequantised in registers; accumulation is fp32.
@@ -76,43 +76,40 @@ __global__ void quantize_q4_kernel(const T *w, int64_t groups, int gpr, uint8_t 
     }
 }
 
-// 32 weights (one 16-byte load of nibbles, even element in the low nibble)
-// times scale s, dotted with 32 consecutive bf16 values of v.
-__device__ __forceinline__ float dot32_q4(const uint4 &qw, float s, const __nv_bfloat16 *v, float acc) {
-    const uint32_t words[4] = {qw.x, qw.y, qw.z, qw.w};
-    float part = 0.f;
-#pragma unroll
-    for (int wd = 0; wd < 4; ++wd) {
-        float xv[8];
-        load8(v + 8 * wd, xv);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) part = fmaf((float)((int)((words[wd] >> (4 * j)) & 15u) - 8), xv[j], part);
-    }
-    return fmaf(part, s, acc);
+// Dequantisation in the dot products: nibble n placed in the low mantissa
+// bits of 128.0f (one bit operation) is the float 128 + n exactly, so for a
+// 32-weight half group with scale s and activations x
+//   sum_i (n_i - 8) s x_i = s (sum_i (128 + n_i) x_i - 136 sum_i x_i),
+// and sum_i x_i is formed once per activation chunk and shared by every
+// weight row that the chunk meets.
+__device__ __forceinline__ float nib_f(uint32_t word, int j) {
+    return __uint_as_float(0x43000000u | (((word >> (4 * j)) & 15u) << 16));
 }
 
-// Dot of one 4-bit weight row (n weights, n a multiple of 64) with a bf16
-// vector; lane l takes the 32-weight halves l, l + 32, ...; four loads in
-// flight per round.
-__device__ __forceinline__ float row_dot_q4(const uint8_t *q, const float *sc, const __nv_bfloat16 *v, int n,
-                                            int lane) {
-    float acc = 0.f;
-    int c = lane * 32;
-    for (; c + 3 * 1024 < n; c += 4 * 1024) {
-        uint4 qw[4];
-        float sv[4];
+// 32 consecutive bf16 activations -> fp32 registers and their sum.
+__device__ __forceinline__ float load32(const __nv_bfloat16 *v, float (&x)[32]) {
+    float sum = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            qw[u] = __ldcs(reinterpret_cast<const uint4 *>(q + (c + u * 1024) / 2));
-            sv[u] = __ldg(sc + (c + u * 1024) / 64);
+    for (int wd = 0; wd < 4; ++wd) {
+        float t[8];
+        load8(v + 8 * wd, t);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            x[8 * wd + j] = t[j];
+            sum += t[j];
         }
+    }
+    return sum;
+}
+
+// sum_i (128 + n_i) x_i over the 32 nibbles of one 16-byte load.
+__device__ __forceinline__ float dot32_raw(const uint4 &qw, const float (&x)[32]) {
+    const uint32_t words[4] = {qw.x, qw.y, qw.z, qw.w};
+    float acc = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) acc = dot32_q4(qw[u], sv[u], v + c + u * 1024, acc);
-    }
-    for (; c < n; c += 1024) {
-        const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(q + c / 2));
-        acc = dot32_q4(q0, __ldg(sc + c / 64), v + c, acc);
-    }
+    for (int wd = 0; wd < 4; ++wd)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc = fmaf(nib_f(words[wd], j), x[8 * wd + j], acc);
     return acc;
 }
 
@@ -129,8 +126,9 @@ __device__ __forceinline__ float row_dot_bf16(const __nv_bfloat16 *w, const __nv
 }
 
 // Grouped gate/up of the routed experts from 4-bit weights: one warp per
-// (listed expert, hidden row n), RG grouped rows per pass over the weight rows.
-template <int RG>
+// (listed expert, block of NR hidden rows), RG grouped rows per pass; each
+// activation chunk a lane loads (32 values) feeds the NR gate and NR up rows.
+template <int RG, int NR>
 __global__ void __launch_bounds__(kThreads) seg_gateup_q4_kernel(SegGateUpQ4Args a, uint32_t *err) {
     pdl_wait();
     pdl_launch_dependents();
@@ -141,15 +139,14 @@ __global__ void __launch_bounds__(kThreads) seg_gateup_q4_kernel(SegGateUpQ4Args
     __nv_bfloat16 *act = static_cast<__nv_bfloat16 *>(a.act);
     const int lane = threadIdx.x & 31;
     const int qpr = a.d / 2, spr = a.d / 64;   // bytes and scales per weight row
-    const int64_t nitems = (int64_t)ne * a.hid;
+    const int nblk = (a.hid + NR - 1) / NR;
+    const int64_t nitems = (int64_t)ne * nblk;
     const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
     const int64_t nw = (int64_t)gridDim.x * kWarps;
     for (int64_t item = gw; item < nitems; item += nw) {
-        const int li = (int)(item / a.hid);
-        const int n = (int)(item - (int64_t)li * a.hid);
-        const int64_t wrow = (int64_t)list[li] * a.hid + n;
-        const uint8_t *qg = a.q_gate + wrow * qpr, *qu = a.q_up + wrow * qpr;
-        const float *sg = a.s_gate + wrow * spr, *su = a.s_up + wrow * spr;
+        const int li = (int)(item / nblk);
+        const int n0 = (int)(item - (int64_t)li * nblk) * NR;
+        const int64_t wrow0 = (int64_t)list[li] * a.hid + n0;
         for (int r0 = beg[li]; r0 < end[li]; r0 += RG) {
             int64_t tok[RG];
 #pragma unroll
@@ -167,34 +164,53 @@ __global__ void __launch_bounds__(kThreads) seg_gateup_q4_kernel(SegGateUpQ4Args
                 }
                 tok[b] = t;
             }
-            float ag[RG], au[RG];
+            float ag[RG][NR], au[RG][NR];
 #pragma unroll
-            for (int b = 0; b < RG; ++b) ag[b] = au[b] = 0.f;
-#pragma unroll 4
+            for (int b = 0; b < RG; ++b)
+#pragma unroll
+                for (int q = 0; q < NR; ++q) ag[b][q] = au[b][q] = 0.f;
             for (int c = lane * 32; c < a.d; c += 1024) {
-                const uint4 wg = __ldcs(reinterpret_cast<const uint4 *>(qg + c / 2));
-                const uint4 wu = __ldcs(reinterpret_cast<const uint4 *>(qu + c / 2));
-                const float s_g = __ldg(sg + c / 64), s_u = __ldg(su + c / 64);
+                uint4 wg[NR], wu[NR];
+                float sg[NR], su[NR];
+#pragma unroll
+                for (int q = 0; q < NR; ++q) {
+                    const bool ok = n0 + q < a.hid;
+                    const int64_t wr = ok ? wrow0 + q : wrow0;
+                    wg[q] = __ldcs(reinterpret_cast<const uint4 *>(a.q_gate + wr * qpr + c / 2));
+                    wu[q] = __ldcs(reinterpret_cast<const uint4 *>(a.q_up + wr * qpr + c / 2));
+                    sg[q] = __ldg(a.s_gate + wr * spr + c / 64);
+                    su[q] = __ldg(a.s_up + wr * spr + c / 64);
+                }
 #pragma unroll
                 for (int b = 0; b < RG; ++b) {
-                    if (tok[b] >= 0) {
-                        ag[b] = dot32_q4(wg, s_g, x + tok[b] * a.d + c, ag[b]);
-                        au[b] = dot32_q4(wu, s_u, x + tok[b] * a.d + c, au[b]);
+                    if (tok[b] < 0) continue;
+                    float xv[32];
+                    const float xs = 136.f * load32(x + tok[b] * a.d + c, xv);
+#pragma unroll
+                    for (int q = 0; q < NR; ++q) {
+                        ag[b][q] = fmaf(sg[q], dot32_raw(wg[q], xv) - xs, ag[b][q]);
+                        au[b][q] = fmaf(su[q], dot32_raw(wu[q], xv) - xs, au[b][q]);
                     }
                 }
             }
 #pragma unroll
             for (int b = 0; b < RG; ++b) {
-                const float g = warp_sum(ag[b]);
-                const float u = warp_sum(au[b]);
-                if (lane == b && tok[b] >= 0) act[(int64_t)(r0 + b) * a.hid + n] = __float2bfloat16_rn(silu_f(g) * u);
+#pragma unroll
+                for (int q = 0; q < NR; ++q) {
+                    const float g = warp_sum(ag[b][q]);
+                    const float u = warp_sum(au[b][q]);
+                    if (lane == b * NR + q && tok[b] >= 0 && n0 + q < a.hid)
+                        act[(int64_t)(r0 + b) * a.hid + n0 + q] = __float2bfloat16_rn(silu_f(g) * u);
+                }
             }
         }
     }
 }
 
 // y[t, n] = sum_j g_j (W_down[e_j, n] . act[inv(t*k + j)]) (4-bit W_down)
-//         (+ shared_gate[t] * (S_down[n] . act_shared[t]), bf16).
+//         (+ shared_gate[t] * (S_down[n] . act_shared[t]), bf16), for NR
+// consecutive outputs n per warp, which share the activation chunks.
+template <int NR>
 __global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Args a, uint32_t *err) {
     pdl_wait();
     pdl_launch_dependents();
@@ -202,13 +218,16 @@ __global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Ar
     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(a.y);
     const int lane = threadIdx.x & 31;
     const int qpr = a.h / 2, spr = a.h / 64;
-    const int64_t nitems = a.T * a.d;
+    const int nblk = (a.d + NR - 1) / NR;
+    const int64_t nitems = a.T * nblk;
     const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
     const int64_t nw = (int64_t)gridDim.x * kWarps;
     for (int64_t item = gw; item < nitems; item += nw) {
-        const int64_t t = item / a.d;
-        const int n = (int)(item - t * a.d);
-        float acc = 0.f;
+        const int64_t t = item / nblk;
+        const int n0 = (int)(item - t * nblk) * NR;
+        float acc[NR];
+#pragma unroll
+        for (int q = 0; q < NR; ++q) acc[q] = 0.f;
         for (int j = 0; j < a.k; ++j) {
             const int64_t slot = t * a.k + j;
             const int e = a.ids[slot];
@@ -217,17 +236,42 @@ __global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Ar
                 if (lane == 0) atomicOr(err, kErrInput);
                 continue;
             }
-            const int64_t wrow = (int64_t)e * a.d + n;
-            acc += a.gates[slot] * row_dot_q4(a.q_down + wrow * qpr, a.s_down + wrow * spr, act + (int64_t)r * a.h,
-                                              a.h, lane);
+            const float g = a.gates[slot];
+            const int64_t wrow0 = (int64_t)e * a.d + n0;
+            float part[NR];
+#pragma unroll
+            for (int q = 0; q < NR; ++q) part[q] = 0.f;
+            for (int c = lane * 32; c < a.h; c += 1024) {
+                uint4 w[NR];
+                float sc[NR];
+#pragma unroll
+                for (int q = 0; q < NR; ++q) {
+                    const int64_t wr = n0 + q < a.d ? wrow0 + q : wrow0;
+                    w[q] = __ldcs(reinterpret_cast<const uint4 *>(a.q_down + wr * qpr + c / 2));
+                    sc[q] = __ldg(a.s_down + wr * spr + c / 64);
+                }
+                float xv[32];
+                const float xs = 136.f * load32(act + (int64_t)r * a.h + c, xv);
+#pragma unroll
+                for (int q = 0; q < NR; ++q) part[q] = fmaf(sc[q], dot32_raw(w[q], xv) - xs, part[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < NR; ++q) acc[q] = fmaf(g, part[q], acc[q]);
         }
         if (a.sh_down) {
             const __nv_bfloat16 *sd = static_cast<const __nv_bfloat16 *>(a.sh_down);
             const __nv_bfloat16 *as = static_cast<const __nv_bfloat16 *>(a.act_shared);
-            acc += a.shared_gate[t] * row_dot_bf16(sd + (int64_t)n * a.h_shared, as + t * a.h_shared, a.h_shared, lane);
+#pragma unroll
+            for (int q = 0; q < NR; ++q)
+                if (n0 + q < a.d)
+                    acc[q] += a.shared_gate[t] *
+                              row_dot_bf16(sd + (int64_t)(n0 + q) * a.h_shared, as + t * a.h_shared, a.h_shared, lane);
         }
-        acc = warp_sum(acc);
-        if (lane == 0) y[item] = __float2bfloat16_rn(acc);
+#pragma unroll
+        for (int q = 0; q < NR; ++q) {
+            const float v = warp_sum(acc[q]);
+            if (lane == q && n0 + q < a.d) y[t * a.d + n0 + q] = __float2bfloat16_rn(v);
+        }
     }
 }
 
@@ -248,14 +292,20 @@ cudaError_t launch_quantize_q4(const void *w, int dtype, int64_t rows, int cols,
 cudaError_t launch_seg_gateup_q4(const SegGateUpQ4Args &a, cudaStream_t s, uint32_t *err) {
     if (a.seg.rows <= 0) return cudaSuccess;
     const size_t smem = sizeof(int) * 3 * (size_t)a.seg.E;
-    const int64_t items = (int64_t)a.seg.E * a.hid;
-    auto go = [&](auto kern) { return launch_kernel(kern, grid_for(kern, items, smem), kThreads, smem, s, a, err); };
-    return a.T == 1 ? go(seg_gateup_q4_kernel<1>) : go(seg_gateup_q4_kernel<4>);
+    auto go = [&](auto kern, int nr) {
+        const int64_t items = (int64_t)a.seg.E * ((a.hid + nr - 1) / nr);
+        return launch_kernel(kern, grid_for(kern, items, smem), kThreads, smem, s, a, err);
+    };
+    // one token: four hidden rows per warp share each activation chunk; more
+    // tokens: four grouped rows per pass share each weight load
+    return a.T == 1 ? go(seg_gateup_q4_kernel<1, 4>, 4) : go(seg_gateup_q4_kernel<4, 1>, 1);
 }
 
 cudaError_t launch_down_direct_q4(const DownDirectQ4Args &a, cudaStream_t s, uint32_t *err) {
     if (a.T <= 0) return cudaSuccess;
-    return launch_kernel(down_direct_q4_kernel, grid_for(down_direct_q4_kernel, a.T * a.d, 0), kThreads, 0, s, a, err);
+    constexpr int NR = 4;
+    auto kern = down_direct_q4_kernel<NR>;
+    return launch_kernel(kern, grid_for(kern, a.T * ((a.d + NR - 1) / NR), 0), kThreads, 0, s, a, err);
 }
 
 }  // namespace moe

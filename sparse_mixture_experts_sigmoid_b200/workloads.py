@@ -82,6 +82,10 @@ WORKLOADS: dict[str, Workload] = {
     # small case of the Mixtral-like expert shape (2 experts, 0.7 GB of weights) for
     # full profiler captures, which must stay a few GB on the device
     "mixtral_e2_profile": Workload("mixtral_e2_profile", T=2048, d=4096, E=2, h=14336, k=2, seed=6),
+    # small case of the OLMoE-like expert shape (a quarter of the tokens, half the
+    # experts: 0.4 GB of weights) for full profiler
+    # captures of the training step's kernels
+    "olmoe_profile": Workload("olmoe_profile", T=2048, d=2048, E=32, h=1024, k=8, norm_topk=False, seed=7),
 }
 
 # The workload that the headline benchmark line is quoted on: the largest
