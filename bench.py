@@ -71,6 +71,8 @@ def parse():
     p.add_argument("--train-workloads", default="",
                    help="comma-separated workloads whose training step (forward + backward) is timed too")
     p.add_argument("--train-steps", type=int, default=20)
+    p.add_argument("--combine", default="add", choices=["add", "ordered"],
+                   help="combine mode: fp32 reductions (add) or slot rows summed in slot order (ordered)")
     p.add_argument("--q4", action="store_true",
                    help="time --workload with 4-bit routed experts (moe_forward_q4; decode-sized batches)")
     return p.parse_args()
@@ -252,7 +254,7 @@ def time_workload(args, w, ws_n, rank, local, steps, warmup, headline, q4=False)
     q4: the routed experts in 4 bits (moe_forward_q4; quantised before timing)."""
     dev = torch.device("cuda", local)
     layer = synth.make_layer(w, dev)
-    cfg = B.config_of(w)
+    cfg = B.config_of(w, combine=args.combine)
     wsbuf = B.alloc_workspace(cfg, dev)
     if q4:
         qw = B.quantize_experts_q4(layer)
@@ -383,7 +385,7 @@ def time_train(args, w, ws_n, local, steps, warmup):
     (the data and weight gradients of every GEMM)."""
     dev = torch.device("cuda", local)
     layer = synth.make_layer(w, dev)
-    cfg = B.config_of(w)
+    cfg = B.config_of(w, combine=args.combine)
     ws = B.alloc_train_workspace(cfg, dev)
     g = torch.Generator(device=dev).manual_seed(w.seed + 7)
     dy = torch.randn(w.T, w.d, generator=g, device=dev).to(layer.x.dtype)
@@ -448,7 +450,7 @@ def bench_ours(args, w, ws_n, rank, local):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w),
            "data": "synthetic (seeded; shapes and distributions of the workload)",
-           "config": config_json(w, ws_n), "roofline": roof, "layer_roofline": head["layer"],
+           "config": dict(config_json(w, ws_n), combine=args.combine), "roofline": roof, "layer_roofline": head["layer"],
            "stages_ms": head["stages_ms"], "stages": head["stages"], "gpu_launches": head["gpu_launches"],
            "clocks": head["clocks"],
            "e2e": head.get("e2e"), "load": head["load"]}

@@ -72,6 +72,18 @@ typedef enum {
 
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_fn;
 typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
+/* How the k expert outputs of a token are summed ("Tutorial 11", section 3,
+ * Step 3: unsort, then the gate-weighted sum over the k experts).
+ *   MOE_COMBINE_ADD: each expert row is added into an fp32 accumulator by
+ *       vector reductions as its tile finishes; the order of the additions
+ *       varies from run to run, so y may differ in the last bits.
+ *   MOE_COMBINE_ORDERED: each gate-weighted expert row is stored in its own
+ *       fp32 slot row (T*k*d floats of workspace), and a final pass adds the
+ *       slots of a token in slot order j = 0..k-1, then the shared expert:
+ *       y is bit-identical from run to run.  Costs one more write and read
+ *       of T*k*d floats.  Applies to the forward combine only (moe_backward
+ *       still accumulates dx by reductions). */
+typedef enum { MOE_COMBINE_ADD = 0, MOE_COMBINE_ORDERED = 1 } moe_combine_mode;
 
 /* Layer shape and options.  All fields are plain integers so the struct has
  * one layout in every language binding. */
@@ -85,6 +97,7 @@ typedef struct {
     int32_t score;     /* moe_score_fn */
     int32_t h_shared;  /* hidden width of the always-on shared expert; 0 = none */
     int32_t dtype;     /* moe_dtype of x, the weights, act and y */
+    int32_t combine;   /* moe_combine_mode; 0 (MOE_COMBINE_ADD) by default */
 } moe_config;
 
 /* Device pointers into a moe_forward workspace (see moe_workspace_layout).
@@ -100,6 +113,8 @@ typedef struct {
     void *act;            /* [T*k, h] silu(gate)*up rows in grouped order (dtype) */
     void *act_shared;     /* [T, h_shared] shared-expert activations; NULL if absent */
     float *y_acc;         /* [T, d]  fp32 accumulator; NULL when dtype is MOE_F32 */
+    float *y_slots;       /* [T*k, d] fp32 gate-weighted expert rows by assignment
+                             r = t*k + j (MOE_COMBINE_ORDERED only; else NULL) */
 } moe_workspace_views;
 
 /* Options of the routing step for training; every field is optional (NULL
@@ -216,9 +231,11 @@ moe_status moe_grouped_swiglu(const moe_config *cfg, const void *x, const void *
  *   y[t, :] = sum over the k assignments r = t*k + j of gates[r] * W_down[e] act[inv(r), :]
  *   act [T*k, h] (dtype, grouped order); w_down [E, d, h]; offsets [E + 1];
  *   sorted_rows [T*k]; gates [T, k] fp32; y [T, d] out (dtype, overwritten).
- *   ws / ws_bytes: for MOE_BF16 an fp32 accumulator of T*d floats is needed
- *   (any workspace of moe_workspace_size bytes works); for MOE_F32 ws may be
- *   NULL.  The summation order over the k experts is not fixed.
+ *   ws / ws_bytes: with MOE_COMBINE_ADD, for MOE_BF16 an fp32 accumulator
+ *   of T*d floats is needed, for MOE_F32 ws may be NULL, and the summation
+ *   order over the k experts is not fixed; with MOE_COMBINE_ORDERED, T*k*d
+ *   floats of slot rows are needed (either dtype) and the k rows of a token
+ *   are added in slot order.  Any workspace of moe_workspace_size bytes works.
  * "Tutorial 11", section 3, Steps 2-3 (grouped down linear, unsort, weighted
  * sum over the k experts). */
 moe_status moe_combine(const moe_config *cfg, const void *act, const void *w_down,
@@ -233,7 +250,9 @@ moe_status moe_combine(const moe_config *cfg, const void *act, const void *w_dow
  *   MOE_BF16 the fp32 accumulator is a static device array of
  *   MOE_NOALLOC_MAX_ACC_FLOATS floats (16 MiB) that every GPU loading the
  *   library holds until exit; T * d above that limit returns
- *   MOE_ERR_WORKSPACE and enqueues nothing.  The call allocates nothing and
+ *   MOE_ERR_WORKSPACE and enqueues nothing.  With MOE_COMBINE_ORDERED the
+ *   same array holds the T*k*d floats of slot rows (either dtype), and the
+ *   limit applies to T*k*d.  The call allocates nothing and
  *   calls no allocating routine.
  *   The first call on a device looks up the array's device address (a
  *   one-time, per-device set-up with that device current).  With CUDA's lazy

@@ -38,7 +38,7 @@ class MoEError(RuntimeError):
 class MoEConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("h", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("norm_topk", ctypes.c_int32), ("score", ctypes.c_int32),
-                ("h_shared", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("h_shared", ctypes.c_int32), ("dtype", ctypes.c_int32), ("combine", ctypes.c_int32)]
 
 
 class RouteOpts(ctypes.Structure):
@@ -48,7 +48,8 @@ class RouteOpts(ctypes.Structure):
 
 class WorkspaceViews(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("ids", "gates", "shared_gate", "counts", "offsets",
-                                               "sorted_rows", "inv_rows", "act", "act_shared", "y_acc")]
+                                               "sorted_rows", "inv_rows", "act", "act_shared", "y_acc",
+                                               "y_slots")]
 
 
 _lib = None
@@ -111,13 +112,22 @@ def _check(status: int, where: str):
         raise MoEError(status, where)
 
 
-def config(T, d, E, h, k, norm_topk=True, score="softmax", h_shared=0, dtype="bf16") -> MoEConfig:
+COMBINE_MODES = {"add": 0, "ordered": 1}
+
+
+def config(T, d, E, h, k, norm_topk=True, score="softmax", h_shared=0, dtype="bf16", combine="add") -> MoEConfig:
+    """moe_config.  combine: "add" (fp32 reductions, summation order not fixed) or
+    "ordered" (per-assignment slot rows added in slot order: bit-reproducible y)."""
+    if combine not in COMBINE_MODES:
+        raise ValueError(f"combine must be one of {sorted(COMBINE_MODES)}, got {combine!r}")
     return MoEConfig(int(T), int(d), int(E), int(h), int(k), int(bool(norm_topk)),
-                     1 if score == "sigmoid" else 0, int(h_shared), 1 if dtype == "f32" else 0)
+                     1 if score == "sigmoid" else 0, int(h_shared), 1 if dtype == "f32" else 0,
+                     COMBINE_MODES[combine])
 
 
-def config_of(w: Workload, T: int | None = None) -> MoEConfig:
-    return config(w.T if T is None else T, w.d, w.E, w.h, w.k, w.norm_topk, w.score, w.h_shared, w.dtype)
+def config_of(w: Workload, T: int | None = None, combine: str = "add") -> MoEConfig:
+    return config(w.T if T is None else T, w.d, w.E, w.h, w.k, w.norm_topk, w.score, w.h_shared, w.dtype,
+                  combine)
 
 
 def _elem_dtype(cfg: MoEConfig):
@@ -169,7 +179,8 @@ def workspace_views(cfg: MoEConfig, ws: torch.Tensor) -> dict:
     spec = {"ids": ((T, k), torch.int32), "gates": ((T, k), torch.float32), "shared_gate": ((T,), torch.float32),
             "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32),
             "sorted_rows": ((R,), torch.int32), "inv_rows": ((R,), torch.int32), "act": ((R, cfg.h), et),
-            "act_shared": ((T, cfg.h_shared), et), "y_acc": ((T, cfg.d), torch.float32)}
+            "act_shared": ((T, cfg.h_shared), et), "y_acc": ((T, cfg.d), torch.float32),
+            "y_slots": ((R, cfg.d), torch.float32)}
     out = {}
     for name, (shape, dt) in spec.items():
         p = getattr(v, name)
@@ -262,8 +273,10 @@ def grouped_swiglu(cfg: MoEConfig, x, w_gate, w_up, offsets, sorted_rows, stream
 def combine(cfg: MoEConfig, act, w_down, offsets, sorted_rows, gates, ws=None, stream=None):
     et = _elem_dtype(cfg)
     y = torch.empty(cfg.T, cfg.d, dtype=et, device=act.device)
-    if ws is None and cfg.dtype == 0:
-        ws = torch.empty(cfg.T * cfg.d * 4, dtype=torch.uint8, device=act.device)
+    if ws is None and (cfg.dtype == 0 or cfg.combine == COMBINE_MODES["ordered"]):
+        # the fp32 accumulator [T, d], or the ordered combine's slot rows [T*k, d]
+        rows = cfg.T * cfg.k if cfg.combine == COMBINE_MODES["ordered"] else cfg.T
+        ws = torch.empty(rows * cfg.d * 4, dtype=torch.uint8, device=act.device)
     _check(lib().moe_combine(ctypes.byref(cfg), _ptr(act, "act", (cfg.T * cfg.k, cfg.h), et),
                              _ptr(w_down, "w_down", (cfg.E, cfg.d, cfg.h), et),
                              _ptr(offsets, "offsets", (cfg.E + 1,), torch.int32),

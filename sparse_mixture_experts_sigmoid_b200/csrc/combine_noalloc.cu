@@ -14,7 +14,8 @@
 // Costs and rules of the static array:
 //  - every GPU that loads the library holds it (kNoAllocAccFloats floats,
 //    16 MiB) until the process exits;
-//  - it bounds the call: T * d must not exceed kNoAllocAccFloats;
+//  - it bounds the call: T * d (T * k * d for the ordered combine, whose slot
+//    rows it then holds) must not exceed kNoAllocAccFloats;
 //  - every call on a device shares it and leaves the previous call's sums in
 //    it; each call clears the part it uses before accumulating, and calls
 //    whose executions overlap on the GPU (different streams, no ordering)
@@ -62,29 +63,12 @@ extern "C" moe_status moe_combine_noalloc(const moe_config *c, const void *act, 
     if (st != MOE_OK) return st;
     if (c->T == 0) return MOE_OK;
     if (!act || !w_down || !offsets || !sorted_rows || !gates || !y) return MOE_ERR_INVALID_ARG;
-    const bool bf16 = c->dtype == MOE_BF16;
-    if (bf16 && (size_t)c->T * (size_t)c->d > kNoAllocAccFloats) return MOE_ERR_WORKSPACE;
+    const size_t need = combine_scratch_floats(*c);
+    if (need > kNoAllocAccFloats) return MOE_ERR_WORKSPACE;
     uint32_t *err = device_error_word();
-    float *acc = bf16 ? acc_ptr() : static_cast<float *>(y);
-    if (!err || !acc) return MOE_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)c->T * c->d * sizeof(float), s);
-    if (e == cudaSuccess) {
-        if (gemm_path(*c)) {
-            e = launch_grouped_gemm(down_plan(*c, act, w_down, offsets, sorted_rows, gates, acc, err), s);
-        } else {
-            SegDownArgs a{};
-            a.act = act;
-            a.w_down = w_down;
-            a.seg = Segments{offsets, sorted_rows, c->E, c->k, c->T * c->k};
-            a.T = c->T;
-            a.d = c->d;
-            a.hid = c->h;
-            a.gates = gates;
-            a.y_acc = acc;
-            e = launch_seg_down(a, c->dtype, s, err);
-        }
-    }
-    if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
+    float *buf = need ? acc_ptr() : nullptr;
+    if (!err || (need && !buf)) return MOE_ERR_CUDA;
+    const cudaError_t e = launch_combine(*c, act, w_down, offsets, sorted_rows, gates, y, buf,
+                                         static_cast<cudaStream_t>(stream), err);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

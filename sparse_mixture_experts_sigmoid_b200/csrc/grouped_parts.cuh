@@ -3,6 +3,8 @@
 //
 //   GATEUP: act[i, n] = silu(W_gate[e, n] . a_i) * (W_up[e, n] . a_i)
 //   DOWN  : y_acc[t_i, n] += g_i * (W_down[e, n] . a_i)
+//           (ordered combine: slot_out[v_i, n] = g_i * (W_down[e, n] . a_i),
+//            v_i the row's assignment)
 //
 // "Tutorial 11: Mixture of Experts (MoE)", section 3 "Expert Computation"
 // (silu(gate) * up; the weighted sum back in token order).
@@ -98,6 +100,8 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
             store16(c + 16, g[1], u[1]);
         }
     } else {
+        // t: the destination row, the token (accumulated into y_acc) or, with
+        // slot_out, the assignment (stored into its own slot row)
         int t = -1;
         float gate = 0.f;
         if (valid) {
@@ -107,7 +111,7 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
                 // (-k, 0) would otherwise truncate to token 0
                 const int v = p.sorted_rows[r];
                 if (v >= 0 && v < p.rows) {
-                    t = v / p.k;
+                    t = p.slot_out ? v : v / p.k;
                     gate = p.gates ? p.gates[v] : 1.f;
                 } else {
                     t = -2;   // reported below
@@ -116,7 +120,7 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
                 t = (int)r;
                 gate = p.gates ? p.gates[r] : 1.f;
             }
-            if (t < 0 || t >= p.T) {
+            if (t < 0 || t >= (p.slot_out ? p.rows : p.T)) {
                 atomicOr(p.err, kErrInput);
                 t = -1;
             }
@@ -152,8 +156,12 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
             for (int i = 0; i < 8; ++i) {
                 const int w = 4 * i + (lane >> 3);
                 const float4 val = st[w * 8 + (j ^ (w & 7))];
-                if (tok[i] >= 0 && col < p.N)
-                    atomicAdd(reinterpret_cast<float4 *>(p.y_acc + (int64_t)tok[i] * p.N + col), val);
+                if (tok[i] >= 0 && col < p.N) {
+                    if (p.slot_out)
+                        *reinterpret_cast<float4 *>(p.slot_out + (int64_t)tok[i] * p.N + col) = val;
+                    else
+                        atomicAdd(reinterpret_cast<float4 *>(p.y_acc + (int64_t)tok[i] * p.N + col), val);
+                }
             }
             __syncwarp();
         }

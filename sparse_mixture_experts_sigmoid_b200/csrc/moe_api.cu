@@ -67,6 +67,7 @@ Layout make_layout(const moe_config &c, bool train = false) {
     L.size[P_PERM] = permute_workspace_bytes((int64_t)R, c.E);
     L.size[P_LOGITS] = router_scratch_bytes(c);
     L.size[P_STATS] = router_stats_bytes(c);
+    L.size[P_SLOTS] = c.combine == MOE_COMBINE_ORDERED ? R * (size_t)c.d * 4 : 0;
     if (train) {
         // kept for the backward pass, and the backward's scratch (the dx accumulator reuses y_acc)
         const size_t hs = (size_t)c.h_shared;
@@ -232,10 +233,39 @@ bool use_fused(const moe_config &c) {
 
 uint32_t *device_error_word() { return err_ptr(); }
 WsLayout ws_layout(const moe_config &c, bool train) { return make_layout(c, train); }
-bool gemm_path(const moe_config &c) { return use_gemm(c); }
-GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const int32_t *offsets,
-                     const int32_t *srt, const float *gates, float *acc, uint32_t *err) {
-    return gemm_down(c, act, wd, offsets, srt, gates, acc, err);
+size_t combine_scratch_floats(const moe_config &c) {
+    if (c.combine == MOE_COMBINE_ORDERED) return (size_t)c.T * c.k * c.d;
+    return c.dtype == MOE_BF16 ? (size_t)c.T * c.d : 0;
+}
+
+cudaError_t launch_combine(const moe_config &c, const void *act, const void *w_down, const int32_t *offsets,
+                           const int32_t *srt, const float *gates, void *y, float *buf, cudaStream_t s,
+                           uint32_t *err) {
+    const bool ordered = c.combine == MOE_COMBINE_ORDERED;
+    // ordered: every slot row is stored once, so nothing needs clearing
+    float *acc = ordered ? nullptr : (c.dtype == MOE_BF16 ? buf : static_cast<float *>(y));
+    cudaError_t e = ordered ? cudaSuccess : cudaMemsetAsync(acc, 0, (size_t)c.T * c.d * sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    if (use_gemm(c)) {
+        GemmLaunch dl = gemm_down(c, act, w_down, offsets, srt, gates, acc, err);
+        dl.p.slot_out = ordered ? buf : nullptr;
+        e = launch_grouped_gemm(dl, s);
+    } else {
+        SegDownArgs a{};
+        a.act = act;
+        a.w_down = w_down;
+        a.seg = Segments{offsets, srt, c.E, c.k, c.T * c.k};
+        a.T = c.T;
+        a.d = c.d;
+        a.hid = c.h;
+        a.gates = gates;
+        a.y_acc = acc;
+        a.slots = ordered ? buf : nullptr;
+        e = launch_seg_down(a, c.dtype, s, err);
+    }
+    if (e != cudaSuccess) return e;
+    if (ordered) return launch_finalize_ordered(buf, nullptr, y, c.T, c.d, c.k, c.dtype, s);
+    return c.dtype == MOE_BF16 ? launch_finalize(acc, y, c.T * c.d, s) : cudaSuccess;
 }
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -285,6 +315,7 @@ moe_status moe_validate(const moe_config *c) {
         return MOE_ERR_INVALID_ARG;
     if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
     if (c->dtype != MOE_BF16 && c->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+    if (c->combine != MOE_COMBINE_ADD && c->combine != MOE_COMBINE_ORDERED) return MOE_ERR_INVALID_ARG;
     if (c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
     if (c->d % 8 || c->h % 8 || c->h_shared % 8) return MOE_ERR_UNSUPPORTED;
     if (c->T * (int64_t)c->k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
@@ -318,6 +349,7 @@ moe_status moe_workspace_layout(const moe_config *c, void *ws, size_t ws_bytes, 
     v->act = part<void>(ws, L, P_ACT);
     v->act_shared = part<void>(ws, L, P_ACTS);
     v->y_acc = part<float>(ws, L, P_YACC);
+    v->y_slots = part<float>(ws, L, P_SLOTS);
     return MOE_OK;
 }
 
@@ -421,28 +453,12 @@ moe_status moe_combine(const moe_config *c, const void *act, const void *w_down,
     if (st != MOE_OK) return st;
     if (c->T == 0) return MOE_OK;
     if (!act || !w_down || !offsets || !sorted_rows || !gates || !y) return MOE_ERR_INVALID_ARG;
-    const bool bf16 = c->dtype == MOE_BF16;
-    const size_t need = bf16 ? (size_t)c->T * c->d * 4 : 0;
-    if (bf16 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15))) return MOE_ERR_WORKSPACE;
+    const size_t need = combine_scratch_floats(*c) * 4;
+    if (need && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15))) return MOE_ERR_WORKSPACE;
     uint32_t *err = err_ptr();
     if (!err) return MOE_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    float *acc = bf16 ? static_cast<float *>(ws) : static_cast<float *>(y);
-    cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)c->T * c->d * 4, s);
-    SegDownArgs a{};
-    a.act = act;
-    a.w_down = w_down;
-    a.seg = Segments{offsets, sorted_rows, c->E, c->k, c->T * c->k};
-    a.T = c->T;
-    a.d = c->d;
-    a.hid = c->h;
-    a.gates = gates;
-    a.y_acc = acc;
-    if (e == cudaSuccess)
-        e = use_gemm(*c) ? launch_grouped_gemm(gemm_down(*c, act, w_down, offsets, sorted_rows, gates, acc, err), s)
-                         : launch_seg_down(a, c->dtype, s, err);
-    if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
-    return cuda_status(e);
+    return cuda_status(launch_combine(*c, act, w_down, offsets, sorted_rows, gates, y, static_cast<float *>(ws),
+                                      static_cast<cudaStream_t>(stream), err));
 }
 
 }  // extern "C"
@@ -495,7 +511,11 @@ moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const v
     ra.probs = train ? part<float>(ws, L, P_PROBS) : nullptr;
     ra.shared_gate = sg;
     const bool gemm = train || use_gemm(*c);
-    const bool fused = gemm && !train && use_fused(*c);
+    // ordered combine: the routed rows go to their slot rows and a last pass adds
+    // them in slot order (the small-batch path already sums in slot order)
+    const bool ordered = gemm && c->combine == MOE_COMBINE_ORDERED;
+    float *slots = ordered ? part<float>(ws, L, P_SLOTS) : nullptr;
+    const bool fused = gemm && !train && !ordered && use_fused(*c);
     // the fused expert kernel adds into the accumulator from its first unit on, so
     // the router clears it; otherwise the gate/up GEMM does (the small-batch path writes y)
     ra.zero_rows = fused ? acc : nullptr;
@@ -524,7 +544,8 @@ moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const v
     } else if (e == cudaSuccess) {
         SegGateUpArgs ga{x, w_gate, w_up, routed, c->T, c->d, c->h, act};
         GemmLaunch gl = gemm_gateup(*c, x, w_gate, w_up, offsets, srt, act, err);
-        gl.p.zero = acc;   // the down GEMM accumulates into it two kernels later
+        // the down GEMMs accumulate into it two kernels later (ordered: only the shared one)
+        gl.p.zero = !ordered || shared ? acc : nullptr;
         gl.p.zero_floats = c->T * c->d;
         gl.p.hpre = train ? part<void>(ws, L, P_HPRE) : nullptr;
         e = gemm ? launch_grouped_gemm(gl, s) : launch_seg_gateup(ga, c->dtype, s, err);
@@ -555,6 +576,7 @@ moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const v
     // complete when the down GEMM starts; act is read after the wait
     GemmLaunch dl = gemm_down(*c, act, w_down, offsets, srt, gates, acc, err);
     dl.p.early = kEarlyTiles;
+    dl.p.slot_out = slots;
     if (e == cudaSuccess && !fused) e = launch_grouped_gemm(dl, s);   // fused: done in the gate/up stage
     mark(1 + MOE_STAGE_DOWN, s);
     // the shared expert's act came from the kernel before the routed down GEMM
@@ -563,7 +585,12 @@ moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const v
     sdl.p.early = fused ? kEarlyTiles : (kEarlyTiles | kEarlyA);
     if (e == cudaSuccess && shared) e = launch_grouped_gemm(sdl, s);
     mark(1 + MOE_STAGE_SHARED_DOWN, s);
-    if (e == cudaSuccess && bf16) e = launch_finalize(acc, y, c->T * c->d, s);
+    // ordered: y = the slot rows in slot order, then the shared expert's row (its
+    // down GEMM is the only writer of each accumulator element, so that sum is exact)
+    if (e == cudaSuccess && ordered)
+        e = launch_finalize_ordered(slots, shared ? acc : nullptr, y, c->T, c->d, c->k, c->dtype, s);
+    else if (e == cudaSuccess && bf16)
+        e = launch_finalize(acc, y, c->T * c->d, s);
     mark(1 + MOE_STAGE_FINALIZE, s);
     return cuda_status(e);
 }

@@ -138,6 +138,8 @@ struct SegDownArgs {
     int d, hid;
     const float *gates;              // routed: [R] gate per assignment; dense: [T] per token
     float *y_acc;                    // [T, d] fp32, accumulated into
+    float *slots;                    // optional, routed only: [R, d] fp32 rows by assignment,
+                                     // stored instead of added into y_acc (ordered combine)
 };
 cudaError_t launch_seg_down(const SegDownArgs &a, int dtype, cudaStream_t s, uint32_t *err);
 
@@ -155,6 +157,10 @@ struct DownDirectArgs {
 cudaError_t launch_down_direct(const DownDirectArgs &a, int dtype, cudaStream_t s, uint32_t *err);
 
 cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t s);
+// Ordered combine: y[t] = ((slots[t*k] + slots[t*k + 1]) + ... + slots[t*k + k-1]) (+ shared[t]),
+// each row d floats; shared may be nullptr and may alias y (dtype MOE_F32).
+cudaError_t launch_finalize_ordered(const float *slots, const float *shared, void *y, int64_t T, int d, int k,
+                                    int dtype, cudaStream_t s);
 
 // 4-bit routed experts on the small-batch path (segment_q4.cu).  A 4-bit
 // weight matrix [rows, cols] is q [rows, cols / 2] (nibble code + 8, even
@@ -207,6 +213,8 @@ struct GemmParams {
     int early;
     void *hpre;                  // gate/up only, optional: [rows, 2N] pre-activations (gate | up) kept
                                  // for the backward pass
+    float *slot_out;             // down only, optional: [R, N] fp32 rows by assignment (routed) or
+                                 // token (dense), stored instead of added into y_acc
 };
 enum : int {
     kEarlyTiles = 1,   // offsets (and hence the tile list) and the weights
@@ -268,6 +276,7 @@ enum WsPart {
     P_STATS,
     // training: kept by moe_forward_train for moe_backward, and the backward's scratch
     P_PROBS, P_HPRE, P_HPRES, P_DG, P_DSG, P_DH, P_DHS, P_GAS, P_DLB, P_DLS, P_XG, P_DYG, P_GA,
+    P_SLOTS,   // ordered combine: [T*k, d] fp32 gate-weighted expert rows by assignment
     P_N
 };
 struct WsLayout {
@@ -288,9 +297,14 @@ inline int64_t padded_rows(int64_t R, int E) { return R + 63LL * E; }
 
 // Launch planning shared by the entry points (defined in moe_api.cu).
 uint32_t *device_error_word();   // the library's device error word on the current device
-bool gemm_path(const moe_config &c);   // tensor-core GEMM (true) or segment kernels (false)
-GemmLaunch down_plan(const moe_config &c, const void *act, const void *wd, const int32_t *offsets,
-                     const int32_t *srt, const float *gates, float *acc, uint32_t *err);
+// Down projection and combine of moe_combine / moe_combine_noalloc.  buf holds
+// combine_scratch_floats(c) floats: the fp32 accumulator [T, d] (MOE_COMBINE_ADD
+// with bf16; unused with f32, where y accumulates) or the slot rows [T*k, d]
+// (MOE_COMBINE_ORDERED).
+size_t combine_scratch_floats(const moe_config &c);
+cudaError_t launch_combine(const moe_config &c, const void *act, const void *w_down, const int32_t *offsets,
+                           const int32_t *srt, const float *gates, void *y, float *buf, cudaStream_t s,
+                           uint32_t *err);
 
 int num_sms();
 

@@ -11,6 +11,8 @@
 // expert linears, silu(gate) * up, weighted sum); "Small MoE Architecture, in
 // depth", Expert.forward (the SwiGLU expert) and the batch-1 decode remarks in
 // "Why small changes the MoE trade-off" (decode reads only the chosen experts).
+#include <algorithm>
+
 #include "segment_parts.cuh"
 
 namespace moe {
@@ -161,8 +163,10 @@ __global__ void __launch_bounds__(kThreads) seg_down_kernel(SegDownArgs a, uint3
                     const int r = r0 + b;
                     const int64_t slot = a.seg.sorted_rows ? a.seg.sorted_rows[r] : r;
                     const int64_t t = a.seg.sorted_rows ? slot / a.seg.k : r;
-                    if (t < 0 || t >= a.T) {
+                    if (slot < 0 || t >= a.T) {
                         atomicOr(err, kErrInput);
+                    } else if (a.slots) {
+                        a.slots[slot * a.d + n] = a.gates[slot] * v;   // ordered combine: own slot row
                     } else {
                         atomicAdd(a.y_acc + t * a.d + n, a.gates[slot] * v);
                     }
@@ -256,6 +260,46 @@ __global__ void finalize_kernel(const float *y_acc, T *y, int64_t n) {
     }
 }
 
+// Ordered combine: each thread adds eight columns of a token's k slot rows in
+// slot order, then the shared expert's row, and writes y.  d % 8 == 0.
+template <typename T>
+__global__ void finalize_ordered_kernel(const float *slots, const float *shared, T *y, int64_t chunks, int d,
+                                        int k) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int cpr = d / 8;   // chunks per row
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / cpr;
+        const int c = (int)(i - t * cpr) * 8;
+        const float *src = slots + t * k * (int64_t)d + c;
+        float4 a = *reinterpret_cast<const float4 *>(src);
+        float4 b = *reinterpret_cast<const float4 *>(src + 4);
+        for (int j = 1; j < k; ++j) {
+            const float4 p = *reinterpret_cast<const float4 *>(src + (int64_t)j * d);
+            const float4 q = *reinterpret_cast<const float4 *>(src + (int64_t)j * d + 4);
+            a = make_float4(a.x + p.x, a.y + p.y, a.z + p.z, a.w + p.w);
+            b = make_float4(b.x + q.x, b.y + q.y, b.z + q.z, b.w + q.w);
+        }
+        if (shared) {
+            const float4 p = *reinterpret_cast<const float4 *>(shared + t * d + c);
+            const float4 q = *reinterpret_cast<const float4 *>(shared + t * d + c + 4);
+            a = make_float4(a.x + p.x, a.y + p.y, a.z + p.z, a.w + p.w);
+            b = make_float4(b.x + q.x, b.y + q.y, b.z + q.z, b.w + q.w);
+        }
+        T *dst = y + t * d + c;
+        if constexpr (sizeof(T) == 2) {
+            __align__(16) __nv_bfloat16 o[8] = {__float2bfloat16_rn(a.x), __float2bfloat16_rn(a.y),
+                                                __float2bfloat16_rn(a.z), __float2bfloat16_rn(a.w),
+                                                __float2bfloat16_rn(b.x), __float2bfloat16_rn(b.y),
+                                                __float2bfloat16_rn(b.z), __float2bfloat16_rn(b.w)};
+            *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(o);
+        } else {
+            *reinterpret_cast<float4 *>(dst) = a;
+            *reinterpret_cast<float4 *>(dst + 4) = b;
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_seg_gateup(const SegGateUpArgs &a, int dtype, cudaStream_t s, uint32_t *err) {
@@ -287,6 +331,19 @@ cudaError_t launch_finalize(const float *y_acc, void *y, int64_t n, cudaStream_t
     const int64_t blocks = (n / 8 + threads) / threads + 1;
     return launch_kernel(finalize_kernel<__nv_bfloat16>, (unsigned)blocks, threads, 0, s, y_acc,
                          static_cast<__nv_bfloat16 *>(y), n);
+}
+
+cudaError_t launch_finalize_ordered(const float *slots, const float *shared, void *y, int64_t T, int d, int k,
+                                    int dtype, cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    const int64_t chunks = T * (d / 8);
+    const int threads = 256;
+    const unsigned blocks = (unsigned)std::min<int64_t>((chunks + threads - 1) / threads, 8 * num_sms());
+    if (dtype == MOE_F32)
+        return launch_kernel(finalize_ordered_kernel<float>, blocks, threads, 0, s, slots, shared,
+                             static_cast<float *>(y), chunks, d, k);
+    return launch_kernel(finalize_ordered_kernel<__nv_bfloat16>, blocks, threads, 0, s, slots, shared,
+                         static_cast<__nv_bfloat16 *>(y), chunks, d, k);
 }
 
 }  // namespace moe

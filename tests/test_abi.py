@@ -42,7 +42,8 @@ def test_status_strings():
 @pytest.mark.parametrize("kw,status", [
     (dict(k=0), 1), (dict(k=9), 1), (dict(T=-1), 1), (dict(d=0), 1), (dict(score=2), 1),
     (dict(E=513, k=2), 2), (dict(k=17, E=32), 2), (dict(d=12), 2), (dict(h=100), 2),
-    (dict(h_shared=12), 2), (dict(h_shared=-8), 1), (dict(T=1 << 30, k=4), 2),
+    (dict(h_shared=12), 2), (dict(h_shared=-8), 1), (dict(T=1 << 30, k=4), 2), (dict(combine=2), 1),
+    (dict(combine=-1), 1),
 ])
 def test_validate_rejects(kw, status):
     base = dict(T=16, d=64, E=8, h=128, k=2, norm_topk=1, score=0, h_shared=0, dtype=0)
@@ -164,3 +165,28 @@ def test_workspace_never_holds_per_token_weight_copies():
     assert naive == 2_684_354_560
     w = WORKLOADS["gemma_upcycle"]
     assert B.workspace_size(B.config_of(w)) < naive / 50
+
+
+def test_ordered_combine_workspace():
+    """The ordered combine adds a [T*k, d] fp32 slot part to the workspace (and
+    to the training workspace); moe_combine then needs T*k*d floats of ws."""
+    L = B.lib()
+    fake = ctypes.c_void_p(0x1000)
+    for name in ("tiny", "olmoe_zipf", "mixtral_decode"):
+        w = WORKLOADS[name]
+        add, ordered = B.config_of(w), B.config_of(w, combine="ordered")
+        slot = w.T * w.k * w.d * 4
+        extra = B.workspace_size(ordered) - B.workspace_size(add)
+        assert slot <= extra <= slot + 255
+        if w.dtype == "bf16":
+            extra_t = B.train_workspace_size(ordered) - B.train_workspace_size(add)
+            assert slot <= extra_t <= slot + 255
+        n = slot if w.dtype == "f32" else w.T * w.d * 4
+        # the add mode's accumulator size is too small for the slot rows
+        if w.k > 1:
+            assert L.moe_combine(ctypes.byref(ordered), fake, fake, fake, fake, fake, fake, fake, w.T * w.d * 4,
+                                 None) == 3
+        assert L.moe_combine(ctypes.byref(ordered), fake, fake, fake, fake, fake, fake, None, 0, None) == 3
+    with pytest.raises(ValueError):
+        B.config(16, 64, 8, 128, 2, combine="sorted")
+
