@@ -112,7 +112,8 @@ typedef struct {
     int32_t *inv_rows;    /* [T*k]   inverse permutation: inv_rows[sorted_rows[i]] = i */
     void *act;            /* [T*k, h] silu(gate)*up rows in grouped order (dtype) */
     void *act_shared;     /* [T, h_shared] shared-expert activations; NULL if absent */
-    float *y_acc;         /* [T, d]  fp32 accumulator; NULL when dtype is MOE_F32 */
+    float *y_acc;         /* [T, d]  fp32 accumulator (scratch: undefined after the
+                             call); NULL when dtype is MOE_F32 */
     float *y_slots;       /* [T*k, d] fp32 gate-weighted expert rows by assignment
                              r = t*k + j (MOE_COMBINE_ORDERED only; else NULL) */
 } moe_workspace_views;
@@ -260,9 +261,9 @@ moe_status moe_combine(const moe_config *cfg, const void *act, const void *w_dow
  *   this part of the library onto the device and backs the array with device
  *   memory, so the first call may allocate: make it at start-up, outside any
  *   region that must not allocate and before any stream capture.  Later
- *   calls allocate nothing.  All calls share the array and it keeps the last
- *   call's contents: each call clears the part it uses, and calls that
- *   overlap on the GPU (unordered streams) race on it. */
+ *   calls allocate nothing.  All calls share the array, whose contents are
+ *   undefined between calls: each call clears the part it uses, and calls
+ *   that overlap on the GPU (unordered streams) race on it. */
 #define MOE_NOALLOC_MAX_ACC_FLOATS (4u << 20)
 moe_status moe_combine_noalloc(const moe_config *cfg, const void *act, const void *w_down,
                                const int32_t *offsets, const int32_t *sorted_rows, const float *gates,

@@ -16,10 +16,10 @@
 //    16 MiB) until the process exits;
 //  - it bounds the call: T * d (T * k * d for the ordered combine, whose slot
 //    rows it then holds) must not exceed kNoAllocAccFloats;
-//  - every call on a device shares it and leaves the previous call's sums in
-//    it; each call clears the part it uses before accumulating, and calls
-//    whose executions overlap on the GPU (different streams, no ordering)
-//    race on it and produce wrong results.
+//  - every call on a device shares it, and its contents are undefined
+//    between calls; each call clears the part it uses before accumulating,
+//    and calls whose executions overlap on the GPU (different streams, no
+//    ordering) race on it and produce wrong results.
 #include <mutex>
 
 #include "moe_internal.cuh"

@@ -40,6 +40,7 @@
 // The instruction descriptor marks each operand's major-ness.
 // Every mbarrier wait is bounded as in the forward kernels.
 #include <algorithm>
+#include <cstdlib>
 
 #include "grouped_parts.cuh"
 
@@ -63,6 +64,9 @@ constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
+// K blocks brought into L2 ahead of the ring: the first touch of an operand
+// line waits on HBM, and the ring alone does not cover that latency
+constexpr int kPrefetchAhead = 8;
 
 enum { ROWS = 0, WGRAD = 1 };
 enum { EPI_SWIGLU = 0, EPI_SCATTER = 1, EPI_STORE = 2 };
@@ -115,72 +119,87 @@ struct Params {
 
 // ------------------------------------------------------------------ epilogues
 
-// ROWS / SWIGLU: grouped row r (valid) of column tile nt; D = r_i over 256
-// columns from TMEM address tbase.  The outputs go to row ro (r in the padded
-// layout).
-__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int64_t r, int64_t ro, bool valid,
-                                                uint32_t tbase) {
-    if (!__any_sync(0xffffffffu, valid)) return;
-    const int N = p.N;
-    float g = 0.f;
-    int64_t gidx = -1;
-    if (valid) {
-        gidx = p.g.sorted_rows ? (int64_t)p.g.sorted_rows[r] : r;
-        if (gidx < 0 || gidx >= (p.g.sorted_rows ? p.g.rows : p.g.T)) {
-            atomicOr(p.g.err, kErrInput);
-            gidx = -1;
-        } else {
-            g = p.gate[gidx];
+// ROWS / SWIGLU: the kept pre-activations u | v of 32 columns from col0 of
+// grouped row r, as raw bf16 (four 16-byte loads each).
+struct UV {
+    uint4 u[4], v[4];
+};
+__device__ __forceinline__ void load_uv(const Params &p, int64_t r, int col0, bool ok, UV &b) {
+    if (!ok) return;
+    const __nv_bfloat16 *row = p.hpre + r * 2 * (int64_t)p.N;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int col = col0 + 8 * q;
+        if (col < p.N) {
+            b.u[q] = __ldg(reinterpret_cast<const uint4 *>(row + col));
+            b.v[q] = __ldg(reinterpret_cast<const uint4 *>(row + p.N + col));
         }
     }
+}
+
+// ROWS / SWIGLU epilogue of grouped row r of column tile nt (gidx: its
+// assignment, or token for the dense expert; -1 if the row is not valid; g:
+// its gate); D = r_i over 256 columns from TMEM address tbase.  The outputs
+// go to row ro (r in the padded layout).  buf[0] holds the first 32 columns'
+// u | v already (loaded before the accumulator was ready); each later chunk's
+// loads are issued before the TMEM wait of the chunk before it, so one L2
+// round trip is in flight while a chunk is computed.
+__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int64_t r, int64_t ro, int64_t gidx, float g,
+                                                uint32_t tbase, UV (&buf)[2]) {
+    const int N = p.N;
     float dot = 0.f;
+    // two chunks per iteration, so the buffers are named statically while the
+    // loop body stays small enough for the instruction cache
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c2 = 0; c2 < BN / 64; ++c2)
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+        const int ci = 2 * c2 + hc;
         float v[2][16];
-        tmem_ld16(tbase + c, v[0]);
-        tmem_ld16(tbase + c + 16, v[1]);
+        tmem_ld16(tbase + 32 * ci, v[0]);
+        tmem_ld16(tbase + 32 * ci + 16, v[1]);
+        if (ci + 1 < BN / 32) load_uv(p, r, nt * BN + 32 * (ci + 1), gidx >= 0, buf[hc ^ 1]);
         tmem_wait_ld();
-        const int col0 = nt * BN + c;
         if (gidx < 0) continue;
+        const UV &b = buf[hc];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int q = 0; q < 4; ++q) {
+            const int col = nt * BN + 32 * ci + 8 * q;
+            if (col >= N) continue;
+            const __nv_bfloat162 *u2 = reinterpret_cast<const __nv_bfloat162 *>(&b.u[q]);
+            const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&b.v[q]);
+            uint32_t du2[4], dv2[4], ga2[4];
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-                const int col = col0 + 16 * h + 8 * h8;
-                if (col >= N) continue;
-                float u[8], w[8];
-                load8(p.hpre + r * 2 * (int64_t)N + col, u);
-                load8(p.hpre + r * 2 * (int64_t)N + N + col, w);
-                uint32_t du2[4], dv2[4], ga2[4];
+            for (int z2 = 0; z2 < 4; ++z2) {
+                const float2 uf = __bfloat1622float2(u2[z2]);
+                const float2 wf = __bfloat1622float2(w2[z2]);
+                const float uu[2] = {uf.x, uf.y}, ww[2] = {wf.x, wf.y};
+                float du[2], dv[2], ga[2];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float du[2], dv[2], ga[2];
-#pragma unroll
-                    for (int z = 0; z < 2; ++z) {
-                        const int i = 2 * q + z;
-                        const float rv = v[h][8 * h8 + i];
-                        const float sg = 1.f / (1.f + __expf(-u[i]));
-                        const float su = u[i] * sg;   // silu(u)
-                        const float a = su * w[i];
-                        dot = fmaf(rv, a, dot);
-                        const float da = g * rv;
-                        du[z] = da * w[i] * sg * (1.f + u[i] * (1.f - sg));
-                        dv[z] = da * su;
-                        ga[z] = g * a;
-                    }
-                    __nv_bfloat162 b;
-                    b = __floats2bfloat162_rn(du[0], du[1]);
-                    du2[q] = *reinterpret_cast<uint32_t *>(&b);
-                    b = __floats2bfloat162_rn(dv[0], dv[1]);
-                    dv2[q] = *reinterpret_cast<uint32_t *>(&b);
-                    b = __floats2bfloat162_rn(ga[0], ga[1]);
-                    ga2[q] = *reinterpret_cast<uint32_t *>(&b);
+                for (int z = 0; z < 2; ++z) {
+                    const int i = 8 * q + 2 * z2 + z;   // column within the 32-column chunk
+                    const float rv = v[i >> 4][i & 15];
+                    const float sg = 1.f / (1.f + __expf(-uu[z]));
+                    const float su = uu[z] * sg;   // silu(u)
+                    const float a = su * ww[z];
+                    dot = fmaf(rv, a, dot);
+                    const float da = g * rv;
+                    du[z] = da * ww[z] * sg * (1.f + uu[z] * (1.f - sg));
+                    dv[z] = da * su;
+                    ga[z] = g * a;
                 }
-                *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + col) = make_uint4(du2[0], du2[1], du2[2], du2[3]);
-                *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + N + col) =
-                    make_uint4(dv2[0], dv2[1], dv2[2], dv2[3]);
-                *reinterpret_cast<uint4 *>(p.ga + ro * (int64_t)N + col) = make_uint4(ga2[0], ga2[1], ga2[2], ga2[3]);
+                __nv_bfloat162 bb;
+                bb = __floats2bfloat162_rn(du[0], du[1]);
+                du2[z2] = *reinterpret_cast<uint32_t *>(&bb);
+                bb = __floats2bfloat162_rn(dv[0], dv[1]);
+                dv2[z2] = *reinterpret_cast<uint32_t *>(&bb);
+                bb = __floats2bfloat162_rn(ga[0], ga[1]);
+                ga2[z2] = *reinterpret_cast<uint32_t *>(&bb);
             }
+            *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + col) = make_uint4(du2[0], du2[1], du2[2], du2[3]);
+            *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + N + col) =
+                make_uint4(dv2[0], dv2[1], dv2[2], dv2[3]);
+            *reinterpret_cast<uint4 *>(p.ga + ro * (int64_t)N + col) = make_uint4(ga2[0], ga2[1], ga2[2], ga2[3]);
         }
     }
     if (gidx >= 0) atomicAdd(p.dgate + gidx, dot);
@@ -318,6 +337,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
+            // the boxes of K block kb of tile id: loaded into stage s, or (s < 0)
+            // only brought into L2
+            auto boxes = [&](int id, int kb, int s) {
+                uint8_t *a = sA + (s < 0 ? 0 : s) * kAStage, *b = sB + (s < 0 ? 0 : s) * kBStage;
+                uint64_t *bar = &ctrl->full[s < 0 ? 0 : s];
+                auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) {
+                    if (s < 0) tma_prefetch_2d(m, c0, c1);
+                    else tma_load_2d(m, dst, bar, c0, c1);
+                };
+                if constexpr (MODE == ROWS) {
+                    const Tile tl = decode(id, ntiles, tile_start, nE);
+                    const int range = kb / kpr, kr = kb - range * kpr;
+                    const CUtensorMap *ma = range ? &tmA1 : &tmA0;
+                    const CUtensorMap *mb = range ? &tmB1 : &tmB0;
+                    box(ma, a, kr * BK, op_row0(tl.e) + tl.m * BM);
+                    const int brow = tl.e * p.Kr + kr * BK;
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j) box(mb, b + j * kAtom, tl.n * BN + 64 * j, brow);
+                } else {
+                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
+                    const int krow = op_row0(w.e) + kb * 64;
+                    const CUtensorMap *ma = w.half ? &tmA1 : &tmA0;
+#pragma unroll
+                    for (int j = 0; j < BM / 64; ++j) box(ma, a + j * kAtom, w.mt * BM + 64 * j, krow);
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j) box(&tmB0, b + j * kAtom, w.nt * BN + 64 * j, krow);
+                }
+            };
+            // prefetch cursor: the K block kStages + kPrefetchAhead blocks after
+            // the last one loaded (it walks the same tiles in the same order)
+            int pf_id = blockIdx.x, pf_kb = -1, pf_nk = blockIdx.x < total ? tile_nk(blockIdx.x) : 0;
+            auto pf_step = [&]() {
+                if (pf_id >= total) return;
+                ++pf_kb;
+                while (pf_kb >= pf_nk) {
+                    pf_id += gridDim.x;
+                    pf_kb = 0;
+                    if (pf_id >= total) return;
+                    pf_nk = tile_nk(pf_id);
+                }
+                boxes(pf_id, pf_kb, -1);
+            };
+            for (int q = 0; q < kStages + kPrefetchAhead; ++q) pf_step();
             uint32_t it = 0;
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
@@ -329,28 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_expect_tx(&ctrl->full[s], kAStage + kBStage);
-                    uint8_t *a = sA + s * kAStage, *b = sB + s * kBStage;
-                    if constexpr (MODE == ROWS) {
-                        const Tile tl = decode(id, ntiles, tile_start, nE);
-                        const int range = kb / kpr, kr = kb - range * kpr;
-                        const CUtensorMap *ma = range ? &tmA1 : &tmA0;
-                        const CUtensorMap *mb = range ? &tmB1 : &tmB0;
-                        tma_load_2d(ma, a, &ctrl->full[s], kr * BK, op_row0(tl.e) + tl.m * BM);
-                        const int brow = tl.e * p.Kr + kr * BK;
-#pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            tma_load_2d(mb, b + j * kAtom, &ctrl->full[s], tl.n * BN + 64 * j, brow);
-                    } else {
-                        const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                        const int krow = op_row0(w.e) + kb * 64;
-                        const CUtensorMap *ma = w.half ? &tmA1 : &tmA0;
-#pragma unroll
-                        for (int j = 0; j < BM / 64; ++j)
-                            tma_load_2d(ma, a + j * kAtom, &ctrl->full[s], w.mt * BM + 64 * j, krow);
-#pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            tma_load_2d(&tmB0, b + j * kAtom, &ctrl->full[s], w.nt * BN + 64 * j, krow);
-                    }
+                    boxes(id, kb, s);
+                    pf_step();
                 }
             }
             if (!ok) {
@@ -397,6 +439,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++tc) {
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            if constexpr (MODE == ROWS && EPI == EPI_SWIGLU) {
+                // the row's gate and first pre-activation columns are read while
+                // the accumulator is still being computed
+                const Tile tl = decode(id, ntiles, tile_start, nE);
+                const int64_t local = (int64_t)tl.m * BM + row;
+                const int64_t r = (int64_t)seg_off[tl.e] + local;
+                const bool valid = r < seg_end[tl.e];
+                int64_t gidx = -1;
+                float g = 0.f;
+                if (valid) {
+                    gidx = p.g.sorted_rows ? (int64_t)p.g.sorted_rows[r] : r;
+                    if (gidx < 0 || gidx >= (p.g.sorted_rows ? p.g.rows : p.g.T)) {
+                        atomicOr(p.g.err, kErrInput);
+                        gidx = -1;
+                    } else {
+                        g = p.gate[gidx];
+                    }
+                }
+                UV buf[2];
+                load_uv(p, r, tl.n * BN, gidx >= 0, buf[0]);
+                if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err)) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, valid))
+                    epilogue_swiglu(p, tl.n, r, op_row0(tl.e) + local, gidx, g, tmem + acc * BN + lane_base, buf);
+                tc_fence_before();
+                mbar_arrive(&ctrl->tempty[acc]);
+                continue;
+            }
             if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err)) break;
             tc_fence_after();
             const uint32_t tb = tmem + acc * BN + lane_base;
@@ -406,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int64_t r = (int64_t)seg_off[tl.e] + local;
                 const bool valid = r < seg_end[tl.e];
                 if constexpr (EPI == EPI_SWIGLU) {
-                    epilogue_swiglu(p, tl.n, r, op_row0(tl.e) + local, valid, tb);
+                    // handled above
                 } else {
                     gg::epilogue_row<gg::DOWN, __nv_bfloat16, BN>(
                         p.g, tl.n, r, valid, tb, reinterpret_cast<float *>(sEpi + warp * gg::kEpiStageBytes));
@@ -424,6 +494,288 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ two-SM kernel
+//
+// The same tile schemes with tiles doubled in M, on clusters of two CTAs
+// (tcgen05.mma.cta_group::2, M = 256): each CTA stages its own 128 rows of A
+// (ROWS: 128 grouped rows; WGRAD: 128 weight rows) and its own 128 of the 256
+// output columns of B, so per K block a CTA moves 32 KB into shared memory
+// for the MMA work that costs 48 KB on one SM, and the ring holds six K
+// blocks instead of four.  The even CTA issues the MMAs; each CTA's half of D
+// lands in its own TMEM and its epilogue warps drain it.  Synchronisation as
+// in the forward two-SM kernel: both CTAs' loads complete on the even CTA's
+// full[s]; tcgen05.commit multicasts stage releases and accumulator-ready
+// signals to both; the epilogue warps of both release an accumulator on the
+// even CTA's tempty; cluster barriers after set-up and before exit.
+constexpr int kPStages = 6;
+constexpr int kPStage = 128 * 128;   // 16 KB: this CTA's A (or B) of one K block
+
+struct Ctrl2 {
+    uint64_t full[kPStages];   // even CTA: operands of a K block landed (both CTAs)
+    uint64_t empty[kPStages];  // both: the MMAs of a K block are done
+    uint64_t tfull[2];         // both: accumulator ready
+    uint64_t tempty[2];        // even CTA: accumulator released by both CTAs' epilogue warps
+    uint64_t done;             // both: all MMAs of the pair completed
+    uint32_t tmem_base;
+    int abort;
+    int n_mtiles;
+    int pad;
+};
+
+template <int MODE>
+constexpr uint32_t idesc_bwd2() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(MODE == WGRAD) << 15) | (1u << 16) |
+           ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+template <int MODE, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                         Params p) {
+    constexpr uint32_t kIdesc = idesc_bwd2<MODE>();
+    constexpr int kEpiStage = EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0;
+    constexpr int BM2 = 256;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sB = smem;                          // B stages first, then A
+    uint8_t *sA = smem + kPStages * kPStage;
+    uint8_t *sEpi = sA + kPStages * kPStage;
+    Ctrl2 *ctrl = reinterpret_cast<Ctrl2 *>(sEpi + kEpiStage);
+    int *tile_start = reinterpret_cast<int *>(ctrl + 1);
+    int *seg_off = tile_start + (p.g.E + 1);
+    int *seg_end = seg_off + (p.g.E + 1);
+    int *blk64 = seg_end + (p.g.E + 1);
+    volatile int *abort = &ctrl->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool lead = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(&ctrl->full[s], 1);
+            mbar_init(&ctrl->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&ctrl->tfull[a], 1);
+            mbar_init(&ctrl->tempty[a], 2 * kEpiWarps);
+        }
+        mbar_init(&ctrl->done, 1);
+        ctrl->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) tmem_alloc2(&ctrl->tmem_base, kTmemCols);
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tmap(&tmA0);
+        prefetch_tmap(&tmB0);
+    }
+    pdl_wait();
+    if (warp == kTmaWarp) {
+        int blocks64;
+        build_tiles<64>(p.g, blk64, seg_off, seg_end, &blocks64);
+        if (MODE == ROWS) build_tiles<BM2>(p.g, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cluster_sync_all();   // both CTAs' barriers exist before any remote arrive
+    pdl_launch_dependents();
+
+    const uint32_t tmem = ctrl->tmem_base;
+    const int nE = p.g.offsets ? p.g.E : 1;
+    const int ntiles = (p.N + BN - 1) / BN;
+    const int mtiles = MODE == WGRAD ? (p.M + BM2 - 1) / BM2 : 0;
+    const int total = MODE == ROWS ? ctrl->n_mtiles * ntiles : nE * p.halves * mtiles * ntiles;
+    const int kpr = (p.Kr + BK - 1) / BK;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int half_off = (int)rank * 128;   // this CTA's rows of A / columns of B inside a tile
+    auto op_row0 = [&](int e) -> int { return p.padded ? 64 * blk64[e] : seg_off[e]; };
+    auto tile_nk = [&](int id) -> int {
+        if constexpr (MODE == ROWS) {
+            return p.nranges * kpr;
+        } else {
+            const WTile w = wdecode(id, mtiles, ntiles, p.halves);
+            return (seg_end[w.e] - seg_off[w.e] + 63) / 64;
+        }
+    };
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t kTx = 2u * 2u * kPStage;   // A and B of both CTAs
+            const uint32_t full_lead = mapa_shared(&ctrl->full[0], 0);
+            // this CTA's boxes of K block kb of tile id: loaded into stage s, or
+            // (s < 0) only brought into L2
+            auto boxes = [&](int id, int kb, int s) {
+                uint8_t *a = sA + (s < 0 ? 0 : s) * kPStage, *b = sB + (s < 0 ? 0 : s) * kPStage;
+                const uint32_t fb = full_lead + (s < 0 ? 0 : s) * (uint32_t)sizeof(uint64_t);
+                auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) {
+                    if (s < 0) tma_prefetch_2d(m, c0, c1);
+                    else tma_load_2d_pair(m, dst, fb, c0, c1);
+                };
+                if constexpr (MODE == ROWS) {
+                    const Tile tl = decode(id, ntiles, tile_start, nE);
+                    const int range = kb / kpr, kr = kb - range * kpr;
+                    const CUtensorMap *ma = range ? &tmA1 : &tmA0;
+                    const CUtensorMap *mb = range ? &tmB1 : &tmB0;
+                    box(ma, a, kr * BK, op_row0(tl.e) + tl.m * BM2 + half_off);
+                    const int brow = tl.e * p.Kr + kr * BK;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) box(mb, b + j * kAtom, tl.n * BN + half_off + 64 * j, brow);
+                } else {
+                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
+                    const int krow = op_row0(w.e) + kb * 64;
+                    const CUtensorMap *ma = w.half ? &tmA1 : &tmA0;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) box(ma, a + j * kAtom, w.mt * BM2 + half_off + 64 * j, krow);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) box(&tmB0, b + j * kAtom, w.nt * BN + half_off + 64 * j, krow);
+                }
+            };
+            int pf_id = pair, pf_kb = -1, pf_nk = pair < total ? tile_nk(pair) : 0;
+            auto pf_step = [&]() {
+                if (pf_id >= total) return;
+                ++pf_kb;
+                while (pf_kb >= pf_nk) {
+                    pf_id += npairs;
+                    pf_kb = 0;
+                    if (pf_id >= total) return;
+                    pf_nk = tile_nk(pf_id);
+                }
+                boxes(pf_id, pf_kb, -1);
+            };
+            for (int q = 0; q < kPStages + kPrefetchAhead; ++q) pf_step();
+            uint32_t it = 0;
+            bool ok = true;
+            for (int id = pair; id < total && ok; id += npairs) {
+                const int nk = tile_nk(id);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kPStages;
+                    if (!wait_bar(&ctrl->empty[s], ((it / kPStages) & 1) ^ 1, abort, p.g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lead) mbar_expect_tx(&ctrl->full[s], kTx);
+                    boxes(id, kb, s);
+                    pf_step();
+                }
+            }
+            if (!ok) {
+                // aborting: let this CTA's copies land before it leaves
+                for (uint32_t j = it > (uint32_t)kPStages ? it - kPStages : 0; j < it; ++j) {
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait(&ctrl->empty[j % kPStages], (j / kPStages) & 1) &&
+                           globaltimer() - t0 < 100000000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0 && lead) {
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int id = pair; id < total && ok; id += npairs, ++tc) {
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.g.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * BN;
+                const int nk = tile_nk(id);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kPStages;
+                    const uint32_t ph = (it / kPStages) & 1;
+                    // the operands of both CTAs have landed (acquire at cluster scope)
+                    bool got = mbar_try_wait_cluster(&ctrl->full[s], ph);
+                    if (!got)
+                        got = wait_bar(&ctrl->full[s], ph, abort, p.g.err) && mbar_try_wait_cluster(&ctrl->full[s], ph);
+                    if (!got) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = MODE == ROWS ? smem_desc(sA + s * kPStage) + 2 * kk
+                                                         : desc_mn(sA + s * kPStage + kk * 2048, kAtom);
+                        const uint64_t bd = desc_mn(sB + s * kPStage + kk * 2048, kAtom);
+                        mma2<__nv_bfloat16>(d_tmem, ad, bd, kIdesc, (kb | kk) != 0);
+                    }
+                    mma_commit2(&ctrl->empty[s], 0x3);
+                }
+                if (ok) mma_commit2(&ctrl->tfull[acc], 0x3);
+            }
+            mma_commit2(&ctrl->done, 0x3);
+        }
+    } else if (warp < kEpiWarps) {
+        uint32_t tc = 0;
+        const int row = warp * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t tempty_lead = mapa_shared(&ctrl->tempty[0], 0);
+        for (int id = pair; id < total; id += npairs, ++tc) {
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            const uint32_t tb = tmem + acc * BN + lane_base;
+            bool got;
+            if constexpr (MODE == ROWS) {
+                const Tile tl = decode(id, ntiles, tile_start, nE);
+                const int64_t local = (int64_t)tl.m * BM2 + half_off + row;
+                const int64_t r = (int64_t)seg_off[tl.e] + local;
+                const bool valid = r < seg_end[tl.e];
+                if constexpr (EPI == EPI_SWIGLU) {
+                    int64_t gidx = -1;
+                    float g = 0.f;
+                    if (valid) {
+                        gidx = p.g.sorted_rows ? (int64_t)p.g.sorted_rows[r] : r;
+                        if (gidx < 0 || gidx >= (p.g.sorted_rows ? p.g.rows : p.g.T)) {
+                            atomicOr(p.g.err, kErrInput);
+                            gidx = -1;
+                        } else {
+                            g = p.gate[gidx];
+                        }
+                    }
+                    UV buf[2];
+                    load_uv(p, r, tl.n * BN, gidx >= 0, buf[0]);
+                    got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+                    if (!got) break;
+                    tc_fence_after();
+                    if (__any_sync(0xffffffffu, valid))
+                        epilogue_swiglu(p, tl.n, r, op_row0(tl.e) + local, gidx, g, tb, buf);
+                } else {
+                    got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+                    if (!got) break;
+                    tc_fence_after();
+                    gg::epilogue_row<gg::DOWN, __nv_bfloat16, BN>(
+                        p.g, tl.n, r, valid, tb, reinterpret_cast<float *>(sEpi + warp * gg::kEpiStageBytes));
+                }
+            } else {
+                got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+                if (!got) break;
+                tc_fence_after();
+                const WTile w = wdecode(id, mtiles, ntiles, p.halves);
+                epilogue_store(p, w.e, w.half, w.mt * BM2 + half_off + row, w.nt * BN, seg_end[w.e] > seg_off[w.e],
+                               tb);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (lead) mbar_arrive(&ctrl->tempty[acc]);
+                else mbar_arrive_remote(tempty_lead + acc * (uint32_t)sizeof(uint64_t));
+            }
+        }
+    }
+
+    // every MMA of the pair has completed (its arrivals on this CTA's barriers
+    // included) before the pair meets for the last time and frees TMEM
+    if (threadIdx.x == 0) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&ctrl->done, 0) && globaltimer() - t0 < kWaitLimitNs) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc2(tmem, kTmemCols);
 }
 
 }  // namespace gb
@@ -480,6 +832,66 @@ cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOper
     return launch_kernel(kern, grid, kThreads, smem, s, mA0, mA1, mB0, mB1, p);
 }
 
+template <int MODE, int EPI>
+cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const BwdOperand &b0, const BwdOperand &b1,
+                            const gb::Params &p, cudaStream_t s) {
+    using namespace gb;
+    CUtensorMap mA0, mA1, mB0, mB1;
+    const uint32_t a_box = MODE == ROWS ? 128 : 64;
+    if (!map_bf16(&mA0, a0.base, a0.rows, a0.cols, a0.ld, a_box)) return cudaErrorInvalidValue;
+    if (!map_bf16(&mB0, b0.base, b0.rows, b0.cols, b0.ld, 64)) return cudaErrorInvalidValue;
+    if (a1.base) {
+        if (!map_bf16(&mA1, a1.base, a1.rows, a1.cols, a1.ld, a_box)) return cudaErrorInvalidValue;
+    } else {
+        mA1 = mA0;
+    }
+    if (b1.base) {
+        if (!map_bf16(&mB1, b1.base, b1.rows, b1.cols, b1.ld, 64)) return cudaErrorInvalidValue;
+    } else {
+        mB1 = mB0;
+    }
+    const size_t smem = 1024 + (size_t)kPStages * 2 * kPStage + (EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0) +
+                        sizeof(Ctrl2) + 4 * sizeof(int) * (p.g.E + 1);
+    auto kern = bwd_gemm_pair_kernel<MODE, EPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // as many CTA pairs as can be resident at once, capped by the tile count
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int max_pairs = 0;
+    e = cudaOccupancyMaxActiveClusters(&max_pairs, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    const int nE = p.g.offsets ? p.g.E : 1;
+    const int ntiles = (p.N + BN - 1) / BN;
+    int64_t max_tiles;
+    if (MODE == ROWS) max_tiles = (p.g.rows / 256 + nE) * (int64_t)ntiles;
+    else max_tiles = (int64_t)nE * p.halves * ((p.M + 255) / 256) * ntiles;
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(std::max(max_pairs, 1), max_tiles));
+    return launch_kernel_pair(kern, 2 * pairs, kThreads, smem, s, mA0, mA1, mB0, mB1, p);
+}
+
+// Two-SM tiles where there is enough work for them: ROWS when the groups
+// average at least 512 rows (as in the forward), WGRAD when a group's weight
+// has at least 512 rows.  MOE_BWD_PAIR=1 / 0 forces them on / off.
+bool bwd_pair(const BwdGemm &L) {
+    static const int force = [] {
+        const char *v = std::getenv("MOE_BWD_PAIR");
+        return v ? (v[0] == '1' ? 1 : 0) : -1;
+    }();
+    if (force >= 0) return force == 1;
+    if (L.kind == BwdGemm::WEIGHT) return L.M >= 512;
+    return L.rows >= 512LL * (L.offsets ? L.groups : 1);
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_gemm(const BwdGemm &L, cudaStream_t s) {
@@ -502,6 +914,13 @@ cudaError_t launch_bwd_gemm(const BwdGemm &L, cudaStream_t s) {
     p.out1 = L.out1;
     p.out_f32 = L.out_f32;
     if (L.rows <= 0 && L.kind != BwdGemm::WEIGHT) return cudaSuccess;
+    if (bwd_pair(L)) {
+        switch (L.kind) {
+            case BwdGemm::SWIGLU: return launch_bwd_pair<ROWS, EPI_SWIGLU>(L.a0, L.a1, L.b0, L.b1, p, s);
+            case BwdGemm::SCATTER: return launch_bwd_pair<ROWS, EPI_SCATTER>(L.a0, L.a1, L.b0, L.b1, p, s);
+            default: return launch_bwd_pair<WGRAD, EPI_STORE>(L.a0, L.a1, L.b0, L.b1, p, s);
+        }
+    }
     switch (L.kind) {
         case BwdGemm::SWIGLU: return launch_bwd<ROWS, EPI_SWIGLU>(L.a0, L.a1, L.b0, L.b1, p, s);
         case BwdGemm::SCATTER: return launch_bwd<ROWS, EPI_SCATTER>(L.a0, L.a1, L.b0, L.b1, p, s);

@@ -138,6 +138,9 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
 #pragma unroll
         for (int i = 0; i < 8; ++i) tok[i] = __shfl_sync(0xffffffffu, t, 4 * i + (lane >> 3));
         float4 *st = reinterpret_cast<float4 *>(stage);
+        // the accumulator is reduced into k times per token, by tiles far apart in
+        // time: keep its lines in L2 over the streamed weights and activations
+        const uint64_t acc_pol = l2_evict_last_policy();
         // 32 columns per TMEM wait: two loads in flight at a time
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -160,7 +163,7 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
                     if (p.slot_out)
                         *reinterpret_cast<float4 *>(p.slot_out + (int64_t)tok[i] * p.N + col) = val;
                     else
-                        atomicAdd(reinterpret_cast<float4 *>(p.y_acc + (int64_t)tok[i] * p.N + col), val);
+                        red_add_v4_hint(p.y_acc + (int64_t)tok[i] * p.N + col, val, acc_pol);
                 }
             }
             __syncwarp();

@@ -14,6 +14,7 @@
 #include <algorithm>
 
 #include "segment_parts.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -258,6 +259,14 @@ __global__ void finalize_kernel(const float *y_acc, T *y, int64_t n) {
     } else {
         for (int64_t j = i; j < n; ++j) y[j] = __float2bfloat16_rn(y_acc[j]);
     }
+    // The accumulator is scratch that the next call clears before use: once the
+    // four lanes sharing a 128-byte line have consumed their values, drop the
+    // line from L2 instead of writing it back to HBM.  Only whole, aligned lines
+    // inside [y_acc, y_acc + n) are dropped (a caller's workspace need only be
+    // 16-byte aligned).
+    __syncwarp();
+    if ((threadIdx.x & 3) == 0 && i + 32 <= n && (reinterpret_cast<uintptr_t>(y_acc + i) & 127) == 0)
+        tc::l2_discard_line(y_acc + i);
 }
 
 // Ordered combine: each thread adds eight columns of a token's k slot rows in

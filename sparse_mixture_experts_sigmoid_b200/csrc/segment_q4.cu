@@ -16,9 +16,9 @@
 //     warp streams the 4-bit gate and up rows once (16 bytes = 32 weights per
 //     lane per load, the group's scale alongside) and applies them to every
 //     grouped row of the expert; act = silu(gate) * up in bf16.
-//   down_direct_q4_kernel: one warp per block of 4 output elements (t, n):
-//     y = sum_j g_j (W_down[e_j, n] . act) (+ the bf16 shared expert), written
-//     straight into y.
+//   down_direct_q4_kernel: one CTA per block of 4 output elements (t, n), the
+//     reduction split over its warps: y = sum_j g_j (W_down[e_j, n] . act)
+//     (+ the bf16 shared expert), written straight into y.
 // The weights are dequantised in registers; accumulation is fp32.
 #include <algorithm>
 
@@ -76,14 +76,18 @@ __global__ void quantize_q4_kernel(const T *w, int64_t groups, int gpr, uint8_t 
     }
 }
 
-// Dequantisation in the dot products: nibble n placed in the low mantissa
-// bits of 128.0f (one bit operation) is the float 128 + n exactly, so for a
-// 32-weight half group with scale s and activations x
+// Dequantisation in the dot products: a nibble n placed in the low mantissa
+// bits of 128.0f is the float 128 + n exactly, so for a 32-weight half group
+// with scale s and activations x
 //   sum_i (n_i - 8) s x_i = s (sum_i (128 + n_i) x_i - 136 sum_i x_i),
 // and sum_i x_i is formed once per activation chunk and shared by every
-// weight row that the chunk meets.
-__device__ __forceinline__ float nib_f(uint32_t word, int j) {
-    return __uint_as_float(0x43000000u | (((word >> (4 * j)) & 15u) << 16));
+// weight row that the chunk meets.  The products (128 + n) x are exact in
+// fp32 (8 by 8 significant bits).  A 32-bit word of codes is split into its
+// low nibbles (elements 0, 2, 4, 6, one per byte) and high nibbles (elements
+// 1, 3, 5, 7) with one mask each, and a byte permute then builds each float
+// from 0x43, the nibble's byte and two zero bytes.
+__device__ __forceinline__ float nib_byte_f(uint32_t nibbles, int b) {
+    return __uint_as_float(__byte_perm(nibbles, 0x43000000u, 0x7044u | ((uint32_t)b << 8)));
 }
 
 // 32 consecutive bf16 activations -> fp32 registers and their sum.
@@ -102,27 +106,22 @@ __device__ __forceinline__ float load32(const __nv_bfloat16 *v, float (&x)[32]) 
     return sum;
 }
 
-// sum_i (128 + n_i) x_i over the 32 nibbles of one 16-byte load.
+// sum_i (128 + n_i) x_i over the 32 nibbles of one 16-byte load (two
+// accumulators, so the fma chain is half as long).
 __device__ __forceinline__ float dot32_raw(const uint4 &qw, const float (&x)[32]) {
     const uint32_t words[4] = {qw.x, qw.y, qw.z, qw.w};
-    float acc = 0.f;
+    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-    for (int wd = 0; wd < 4; ++wd)
+    for (int wd = 0; wd < 4; ++wd) {
+        const uint32_t lo = words[wd] & 0x0F0F0F0Fu;
+        const uint32_t hi = (words[wd] >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc = fmaf(nib_f(words[wd], j), x[8 * wd + j], acc);
-    return acc;
-}
-
-__device__ __forceinline__ float row_dot_bf16(const __nv_bfloat16 *w, const __nv_bfloat16 *v, int n, int lane) {
-    float acc = 0.f;
-    for (int c = lane * 8; c < n; c += 256) {
-        float wv[8], av[8];
-        load8_stream(w + c, wv);
-        load8(v + c, av);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc = fmaf(wv[u], av[u], acc);
+        for (int b = 0; b < 4; ++b) {
+            acc0 = fmaf(nib_byte_f(lo, b), x[8 * wd + 2 * b], acc0);
+            acc1 = fmaf(nib_byte_f(hi, b), x[8 * wd + 2 * b + 1], acc1);
+        }
     }
-    return acc;
+    return acc0 + acc1;
 }
 
 // Grouped gate/up of the routed experts from 4-bit weights: one warp per
@@ -209,20 +208,23 @@ __global__ void __launch_bounds__(kThreads) seg_gateup_q4_kernel(SegGateUpQ4Args
 
 // y[t, n] = sum_j g_j (W_down[e_j, n] . act[inv(t*k + j)]) (4-bit W_down)
 //         (+ shared_gate[t] * (S_down[n] . act_shared[t]), bf16), for NR
-// consecutive outputs n per warp, which share the activation chunks.
+// consecutive outputs n per CTA.  The reduction dimension is split over the
+// CTA's warps (warp w takes the 1024-element steps w, w + 8, ...), each warp's
+// NR rows share its activation chunks, and the warps' partial sums are added
+// in warp order through shared memory: enough warps in flight to cover the
+// weight loads' latency even at one token.
 template <int NR>
 __global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Args a, uint32_t *err) {
     pdl_wait();
     pdl_launch_dependents();
+    __shared__ float red[kWarps][NR];
     const __nv_bfloat16 *act = static_cast<const __nv_bfloat16 *>(a.act);
     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(a.y);
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int qpr = a.h / 2, spr = a.h / 64;
     const int nblk = (a.d + NR - 1) / NR;
     const int64_t nitems = a.T * nblk;
-    const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-    const int64_t nw = (int64_t)gridDim.x * kWarps;
-    for (int64_t item = gw; item < nitems; item += nw) {
+    for (int64_t item = blockIdx.x; item < nitems; item += gridDim.x) {
         const int64_t t = item / nblk;
         const int n0 = (int)(item - t * nblk) * NR;
         float acc[NR];
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Ar
             const int e = a.ids[slot];
             const int r = a.inv_rows[slot];
             if (e < 0 || e >= a.E || r < 0 || r >= a.T * a.k) {
-                if (lane == 0) atomicOr(err, kErrInput);
+                if (threadIdx.x == 0) atomicOr(err, kErrInput);
                 continue;
             }
             const float g = a.gates[slot];
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Ar
             float part[NR];
 #pragma unroll
             for (int q = 0; q < NR; ++q) part[q] = 0.f;
-            for (int c = lane * 32; c < a.h; c += 1024) {
+            for (int c = (warp * 32 + lane) * 32; c < a.h; c += kWarps * 1024) {
                 uint4 w[NR];
                 float sc[NR];
 #pragma unroll
@@ -260,18 +262,36 @@ __global__ void __launch_bounds__(kThreads) down_direct_q4_kernel(DownDirectQ4Ar
         }
         if (a.sh_down) {
             const __nv_bfloat16 *sd = static_cast<const __nv_bfloat16 *>(a.sh_down);
-            const __nv_bfloat16 *as = static_cast<const __nv_bfloat16 *>(a.act_shared);
+            const __nv_bfloat16 *as = static_cast<const __nv_bfloat16 *>(a.act_shared) + t * a.h_shared;
+            const float sg = a.shared_gate[t];
 #pragma unroll
-            for (int q = 0; q < NR; ++q)
-                if (n0 + q < a.d)
-                    acc[q] += a.shared_gate[t] *
-                              row_dot_bf16(sd + (int64_t)(n0 + q) * a.h_shared, as + t * a.h_shared, a.h_shared, lane);
+            for (int q = 0; q < NR; ++q) {
+                if (n0 + q >= a.d) continue;
+                const __nv_bfloat16 *row = sd + (int64_t)(n0 + q) * a.h_shared;
+                float p = 0.f;
+                for (int c = (warp * 32 + lane) * 8; c < a.h_shared; c += kWarps * 256) {
+                    float wv[8], av[8];
+                    load8_stream(row + c, wv);
+                    load8(as + c, av);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) p = fmaf(wv[u], av[u], p);
+                }
+                acc[q] = fmaf(sg, p, acc[q]);
+            }
         }
 #pragma unroll
         for (int q = 0; q < NR; ++q) {
             const float v = warp_sum(acc[q]);
-            if (lane == q && n0 + q < a.d) y[t * a.d + n0 + q] = __float2bfloat16_rn(v);
+            if (lane == 0) red[warp][q] = v;
         }
+        __syncthreads();
+        if (warp == 0 && lane < NR && n0 + lane < a.d) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) v += red[w][lane];
+            y[t * a.d + n0 + lane] = __float2bfloat16_rn(v);
+        }
+        __syncthreads();
     }
 }
 
@@ -296,16 +316,18 @@ cudaError_t launch_seg_gateup_q4(const SegGateUpQ4Args &a, cudaStream_t s, uint3
         const int64_t items = (int64_t)a.seg.E * ((a.hid + nr - 1) / nr);
         return launch_kernel(kern, grid_for(kern, items, smem), kThreads, smem, s, a, err);
     };
-    // one token: four hidden rows per warp share each activation chunk; more
+    // one token: two hidden rows per warp share each activation chunk; more
     // tokens: four grouped rows per pass share each weight load
-    return a.T == 1 ? go(seg_gateup_q4_kernel<1, 4>, 4) : go(seg_gateup_q4_kernel<4, 1>, 1);
+    return a.T == 1 ? go(seg_gateup_q4_kernel<1, 2>, 2) : go(seg_gateup_q4_kernel<4, 1>, 1);
 }
 
 cudaError_t launch_down_direct_q4(const DownDirectQ4Args &a, cudaStream_t s, uint32_t *err) {
     if (a.T <= 0) return cudaSuccess;
     constexpr int NR = 4;
     auto kern = down_direct_q4_kernel<NR>;
-    return launch_kernel(kern, grid_for(kern, a.T * ((a.d + NR - 1) / NR), 0), kThreads, 0, s, a, err);
+    // one CTA per item (grid_for counts warps)
+    const int64_t items = a.T * ((a.d + NR - 1) / NR);
+    return launch_kernel(kern, grid_for(kern, items * kWarps, 0), kThreads, 0, s, a, err);
 }
 
 }  // namespace moe

@@ -85,12 +85,39 @@ __device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap *m, void *dst
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
+// Brings a 2D box of a tensor into L2 without copying it anywhere (a later
+// TMA load of the box then waits on L2 instead of HBM).  Boxes reaching
+// outside the tensor are clipped as for a load.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *m, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1)
+                 : "memory");
+}
 // L2 policy under which the lines a streamed operand brings in are evicted
 // first, so data reused through L2 (activations, the combine accumulator) stays.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+// L2 policy under which the lines touched are kept over normal and
+// evict-first lines: for the combine accumulator, reduced into many times.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// 16-byte fp32 vector reduction into global memory (performed in L2) under an
+// L2 cache policy.
+__device__ __forceinline__ void red_add_v4_hint(float *addr, float4 v, uint64_t policy) {
+    asm volatile("red.relaxed.gpu.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;"
+                 ::"l"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(policy)
+                 : "memory");
+}
+// Drops the 128-byte L2 line at addr without writing it back: its contents
+// become undefined (for scratch that is rewritten before it is read again).
+__device__ __forceinline__ void l2_discard_line(const void *addr) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(addr) : "memory");
 }
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)

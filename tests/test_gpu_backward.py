@@ -10,7 +10,8 @@ Cases cover the tensor-core paths the backward takes: gathered and dense
 operands, widths that are not multiples of the 64-wide K blocks (the gate/up
 K split), experts without rows (zero gradients), renormalised and raw
 softmax, sigmoid with a balance bias, the shared expert, one expert, single
-tokens, and the full-size Gemma-upcycle layer.
+tokens, layers large enough for the two-SM tiles (whole and partial), and the
+full-size Gemma-upcycle layer.
 """
 import numpy as np
 import pytest
@@ -46,6 +47,9 @@ CASES = [
     case("few_tokens_shared", T=5, h_shared=64, seed=127),
     case("zipf_empty_experts", recipe="zipf", E=32, k=2, seed=128),
     case("many_experts", E=130, k=6, T=200, d=128, h=64, router_std=0.2, seed=129),
+    # enough rows per expert (>= 512) and weight rows (>= 512) for the two-SM tiles
+    case("pair_tiles", T=1024, d=512, E=4, h=512, k=2, seed=133),
+    case("pair_ragged", T=800, d=576, E=3, h=640, k=2, seed=134),   # partial 256-row and 256-column tiles
 ]
 
 
