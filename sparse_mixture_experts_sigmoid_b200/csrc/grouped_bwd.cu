@@ -64,9 +64,6 @@ constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
-// K blocks brought into L2 ahead of the ring: the first touch of an operand
-// line waits on HBM, and the ring alone does not cover that latency
-constexpr int kPrefetchAhead = 8;
 
 enum { ROWS = 0, WGRAD = 1 };
 enum { EPI_SWIGLU = 0, EPI_SCATTER = 1, EPI_STORE = 2 };
@@ -337,15 +334,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
-            // the boxes of K block kb of tile id: loaded into stage s, or (s < 0)
-            // only brought into L2
+            // the boxes of K block kb of tile id, into stage s
             auto boxes = [&](int id, int kb, int s) {
-                uint8_t *a = sA + (s < 0 ? 0 : s) * kAStage, *b = sB + (s < 0 ? 0 : s) * kBStage;
-                uint64_t *bar = &ctrl->full[s < 0 ? 0 : s];
-                auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) {
-                    if (s < 0) tma_prefetch_2d(m, c0, c1);
-                    else tma_load_2d(m, dst, bar, c0, c1);
-                };
+                uint8_t *a = sA + s * kAStage, *b = sB + s * kBStage;
+                uint64_t *bar = &ctrl->full[s];
+                auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) { tma_load_2d(m, dst, bar, c0, c1); };
                 if constexpr (MODE == ROWS) {
                     const Tile tl = decode(id, ntiles, tile_start, nE);
                     const int range = kb / kpr, kr = kb - range * kpr;
@@ -365,21 +358,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < BN / 64; ++j) box(&tmB0, b + j * kAtom, w.nt * BN + 64 * j, krow);
                 }
             };
-            // prefetch cursor: the K block kStages + kPrefetchAhead blocks after
-            // the last one loaded (it walks the same tiles in the same order)
-            int pf_id = blockIdx.x, pf_kb = -1, pf_nk = blockIdx.x < total ? tile_nk(blockIdx.x) : 0;
-            auto pf_step = [&]() {
-                if (pf_id >= total) return;
-                ++pf_kb;
-                while (pf_kb >= pf_nk) {
-                    pf_id += gridDim.x;
-                    pf_kb = 0;
-                    if (pf_id >= total) return;
-                    pf_nk = tile_nk(pf_id);
-                }
-                boxes(pf_id, pf_kb, -1);
-            };
-            for (int q = 0; q < kStages + kPrefetchAhead; ++q) pf_step();
             uint32_t it = 0;
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
@@ -392,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mbar_expect_tx(&ctrl->full[s], kAStage + kBStage);
                     boxes(id, kb, s);
-                    pf_step();
                 }
             }
             if (!ok) {
@@ -606,14 +583,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t kTx = 2u * 2u * kPStage;   // A and B of both CTAs
             const uint32_t full_lead = mapa_shared(&ctrl->full[0], 0);
-            // this CTA's boxes of K block kb of tile id: loaded into stage s, or
-            // (s < 0) only brought into L2
+            // this CTA's boxes of K block kb of tile id, into stage s
             auto boxes = [&](int id, int kb, int s) {
-                uint8_t *a = sA + (s < 0 ? 0 : s) * kPStage, *b = sB + (s < 0 ? 0 : s) * kPStage;
-                const uint32_t fb = full_lead + (s < 0 ? 0 : s) * (uint32_t)sizeof(uint64_t);
+                uint8_t *a = sA + s * kPStage, *b = sB + s * kPStage;
+                const uint32_t fb = full_lead + s * (uint32_t)sizeof(uint64_t);
                 auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) {
-                    if (s < 0) tma_prefetch_2d(m, c0, c1);
-                    else tma_load_2d_pair(m, dst, fb, c0, c1);
+                    tma_load_2d_pair(m, dst, fb, c0, c1);
                 };
                 if constexpr (MODE == ROWS) {
                     const Tile tl = decode(id, ntiles, tile_start, nE);
@@ -634,19 +609,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 2; ++j) box(&tmB0, b + j * kAtom, w.nt * BN + half_off + 64 * j, krow);
                 }
             };
-            int pf_id = pair, pf_kb = -1, pf_nk = pair < total ? tile_nk(pair) : 0;
-            auto pf_step = [&]() {
-                if (pf_id >= total) return;
-                ++pf_kb;
-                while (pf_kb >= pf_nk) {
-                    pf_id += npairs;
-                    pf_kb = 0;
-                    if (pf_id >= total) return;
-                    pf_nk = tile_nk(pf_id);
-                }
-                boxes(pf_id, pf_kb, -1);
-            };
-            for (int q = 0; q < kPStages + kPrefetchAhead; ++q) pf_step();
             uint32_t it = 0;
             bool ok = true;
             for (int id = pair; id < total && ok; id += npairs) {
@@ -659,7 +621,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (lead) mbar_expect_tx(&ctrl->full[s], kTx);
                     boxes(id, kb, s);
-                    pf_step();
                 }
             }
             if (!ok) {
@@ -881,15 +842,21 @@ cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const Bw
 
 // Two-SM tiles where there is enough work for them: ROWS when the groups
 // average at least 512 rows (as in the forward), WGRAD when a group's weight
-// has at least 512 rows.  MOE_BWD_PAIR=1 / 0 forces them on / off.
+// has at least 512 rows and the groups average at least 256 rows (the K
+// extent of its tiles).  Measured on training steps: the two-SM weight
+// gradients take olmoe_zipf's backward from 3.09 to 2.95 ms and
+// mixtral_prefill's from 8.64 to 8.15 ms; on gemma_upcycle (32 rows per
+// expert) they were slower (0.71 vs 0.51 ms).  MOE_BWD_PAIR=1 / 0 forces them
+// on / off.
 bool bwd_pair(const BwdGemm &L) {
     static const int force = [] {
         const char *v = std::getenv("MOE_BWD_PAIR");
         return v ? (v[0] == '1' ? 1 : 0) : -1;
     }();
     if (force >= 0) return force == 1;
-    if (L.kind == BwdGemm::WEIGHT) return L.M >= 512;
-    return L.rows >= 512LL * (L.offsets ? L.groups : 1);
+    const int64_t groups = L.offsets ? L.groups : 1;
+    if (L.kind == BwdGemm::WEIGHT) return L.M >= 512 && L.rows >= 256LL * groups;
+    return L.rows >= 512LL * groups;
 }
 
 }  // namespace

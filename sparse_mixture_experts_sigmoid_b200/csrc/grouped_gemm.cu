@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             uint32_t pre = 0;
             if (early_tiles) {
                 for (int id = blockIdx.x; id < total && pre < (uint32_t)kStages; id += gridDim.x) {
-                    const Tile tl = decode(id, n_tiles, tile_start, nE);
+                    const Tile tl = decode_n(id, n_tiles, p.n_groups, ctrl->n_mtiles, tile_start, nE);
                     const int a_row = seg_off[tl.e] + tl.m * RB;
                     const int b_row = tl.e * p.N + tl.n * BN_OUT;
                     for (int kb = 0; kb < nk && pre < (uint32_t)kStages; ++kb, ++pre) {
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-                const Tile tl = decode(id, n_tiles, tile_start, nE);
+                const Tile tl = decode_n(id, n_tiles, p.n_groups, ctrl->n_mtiles, tile_start, nE);
                 const int a_row = seg_off[tl.e] + tl.m * RB;
                 const int b_row = tl.e * p.N + tl.n * BN_OUT;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
         const int row = warp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++tc) {
-            const Tile tl = decode(id, n_tiles, tile_start, nE);
+            const Tile tl = decode_n(id, n_tiles, p.n_groups, ctrl->n_mtiles, tile_start, nE);
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();

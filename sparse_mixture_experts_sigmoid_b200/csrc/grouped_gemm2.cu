@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int id = pair; id < total && ok; id += npairs) {
-                const Tile tl = decode(id, n_tiles, tile_start, nE);
+                const Tile tl = decode_n(id, n_tiles, p.n_groups, ctrl->n_mtiles, tile_start, nE);
                 const int a_row = seg_off[tl.e] + tl.m * BM2 + row_off;
                 // gate/up: the gate rows from CTA 0, the up rows from CTA 1 (W x
                 // BN / 2 of them, one box); down: the first and second half of
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
         const uint32_t tempty_lead = mapa_shared(&ctrl->tempty[0], 0);
         bool ok = true;
         for (int id = pair; id < total && ok; id += npairs, ++tc) {
-            const Tile tl = decode(id, n_tiles, tile_start, nE);
+            const Tile tl = decode_n(id, n_tiles, p.n_groups, ctrl->n_mtiles, tile_start, nE);
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * BM2 + row_off + row;
 #pragma unroll 1
             for (int j = 0; j < W; ++j) {

@@ -97,5 +97,23 @@ __device__ __forceinline__ Tile decode(int id, int n_tiles, const int *tile_star
     return t;
 }
 
+// The same tiles with the column tiles split into G consecutive groups that
+// run one after another: all tiles of columns [0, gs) (expert-major as in
+// decode), then all of [gs, 2 gs), ... (gs = ceil(n_tiles / G)).  For the down
+// GEMM this bounds the part of the combine accumulator that the CTAs running
+// at one time reduce into (T x gs columns), so it stays in L2 across the k
+// experts of a token; each row of act is then read once per group.  G <= 1 is
+// decode.
+__device__ __forceinline__ Tile decode_n(int id, int n_tiles, int G, int n_mtiles, const int *tile_start, int E) {
+    if (G <= 1) return decode(id, n_tiles, tile_start, E);
+    const int gs = (n_tiles + G - 1) / G;
+    const int per = n_mtiles * gs;
+    const int g = id / per;
+    const int gsz = min(gs, n_tiles - g * gs);
+    Tile t = decode(id - g * per, gsz, tile_start, E);
+    t.n += g * gs;
+    return t;
+}
+
 }  // namespace gg
 }  // namespace moe

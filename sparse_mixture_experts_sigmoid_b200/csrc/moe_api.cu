@@ -186,6 +186,22 @@ GemmLaunch gemm_gateup_dense(const moe_config &c, const void *x, const void *wg,
     L.b1 = wu;
     return L;
 }
+// Column groups of the routed down GEMM (see decode_n).  Two groups halve the
+// part of the fp32 accumulator [T, d] that the CTAs reduce into at one time,
+// so that it stays in L2 while the k experts of each token add into it, at
+// the price of reading act twice: taken when the accumulator is larger than
+// 48 MB and act at most 2.5 times its size.  MOE_DOWN_GROUPS=n forces n.
+int down_groups(const moe_config &c, int n_tiles) {
+    static const int force = [] {
+        const char *v = std::getenv("MOE_DOWN_GROUPS");
+        return v ? std::atoi(v) : 0;
+    }();
+    const int64_t acc = (int64_t)c.T * c.d * 4;
+    const int64_t act = (int64_t)c.T * c.k * c.h * (c.dtype == MOE_F32 ? 4 : 2);
+    int g = force > 0 ? force : (acc > (48LL << 20) && 2 * act <= 5 * acc ? 2 : 1);
+    return g < 1 ? 1 : (g > n_tiles ? n_tiles : g);
+}
+
 GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const int32_t *offsets,
                      const int32_t *srt, const float *gates, float *acc, uint32_t *err) {
     GemmLaunch L{};
@@ -197,6 +213,7 @@ GemmLaunch gemm_down(const moe_config &c, const void *act, const void *wd, const
     L.p.stream_weights = one_tile_per_expert(c);
     L.pair = pair_tiles(c.T * c.k, c.E, false, c.d);
     L.half = !L.pair && half_tiles(c.T * c.k, c.E);
+    L.p.n_groups = down_groups(c, (c.d + (L.narrow ? 127 : 255)) / (L.narrow ? 128 : 256));
     L.a_src = act;
     L.b0 = wd;
     return L;

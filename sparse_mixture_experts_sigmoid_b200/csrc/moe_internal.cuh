@@ -215,6 +215,7 @@ struct GemmParams {
                                  // for the backward pass
     float *slot_out;             // down only, optional: [R, N] fp32 rows by assignment (routed) or
                                  // token (dense), stored instead of added into y_acc
+    int n_groups;                // column tiles run in this many consecutive groups (decode_n); 0, 1: one
 };
 enum : int {
     kEarlyTiles = 1,   // offsets (and hence the tile list) and the weights

@@ -85,14 +85,6 @@ __device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap *m, void *dst
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
-// Brings a 2D box of a tensor into L2 without copying it anywhere (a later
-// TMA load of the box then waits on L2 instead of HBM).  Boxes reaching
-// outside the tensor are clipped as for a load.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *m, int c0, int c1) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1)
-                 : "memory");
-}
 // L2 policy under which the lines a streamed operand brings in are evicted
 // first, so data reused through L2 (activations, the combine accumulator) stays.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {

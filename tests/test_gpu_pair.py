@@ -10,6 +10,8 @@ the small parity cases against the oracle:
 * the fused expert kernel (gate/up, SwiGLU, down and combine in one pass),
   opt-in; MOE_FUSED=1 forces it wherever the hidden width is a multiple of 64
   (experts with several row tiles included);
+* the routed down GEMM's column tiles in consecutive groups (chosen when
+  the combine accumulator is large): MOE_DOWN_GROUPS=3 forces three;
 * the backward GEMMs on two-SM tiles (chosen when groups average at least 512
   rows, or a weight gradient has at least 512 rows): MOE_BWD_PAIR=1 forces
   them on the small training cases, MOE_BWD_PAIR=0 forces one-SM tiles on the
@@ -48,6 +50,13 @@ def test_forward_small_with_half_height_down_tiles():
 @pytest.mark.gpu
 def test_forward_small_with_fused_expert_kernel():
     run_small_cases(MOE_FUSED="1")
+
+
+@pytest.mark.gpu
+def test_forward_small_with_down_column_groups():
+    """The down GEMM's column tiles in three consecutive groups (one-SM and two-SM tiles)."""
+    run_small_cases(MOE_DOWN_GROUPS="3")
+    run_small_cases(MOE_DOWN_GROUPS="3", MOE_GG_PAIR="1")
 
 
 @pytest.mark.gpu

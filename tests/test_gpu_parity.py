@@ -177,6 +177,7 @@ SMALL = [
     small("many_experts", E=512, k=16, T=200, d=128, h=64, router_std=0.2, seed=62),
     small("zipf_hot_expert", recipe="zipf", E=32, k=2, seed=63),
     small("f32_sigmoid_shared", dtype="f32", score="sigmoid", h_shared=64, seed=64),
+    small("wide_model_width", d=832, h=256, seed=68),   # seven 128-column down tiles (column groups)
 ]
 
 
