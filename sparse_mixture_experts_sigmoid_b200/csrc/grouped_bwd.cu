@@ -66,6 +66,30 @@ constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 
 enum { ROWS = 0, WGRAD = 1 };
+
+// Pipeline trace of the one-SM kernel, compiled in only with -DMOE_PIPE_TRACE
+// (a diagnostic build): per kernel variant (ROWS/SWIGLU, ROWS/SCATTER,
+// WGRAD), SM cycles summed over CTAs for [0] the whole kernel, [1] the MMA
+// issuer waiting for operands, [2] the MMA issuer waiting for a free
+// accumulator, [3] the producer waiting for a free stage, [4] epilogue warp 0
+// waiting for an accumulator, [5] epilogue warp 0 draining one, and [6] the
+// number of CTAs.  Read with moe_debug_pipe_trace (same build only).
+#ifdef MOE_PIPE_TRACE
+__device__ unsigned long long g_pipe_trace[4][8];
+struct PipeClock {
+    unsigned long long acc = 0;
+    long long t0 = 0;
+    __device__ void start() { t0 = clock64(); }
+    __device__ void stop() { acc += (unsigned long long)(clock64() - t0); }
+    __device__ void flush(int var, int slot) { atomicAdd(&g_pipe_trace[var][slot], acc); }
+};
+#else
+struct PipeClock {
+    __device__ void start() {}
+    __device__ void stop() {}
+    __device__ void flush(int, int) {}
+};
+#endif
 enum { EPI_SWIGLU = 0, EPI_SCATTER = 1, EPI_STORE = 2 };
 
 struct Ctrl {
@@ -112,6 +136,10 @@ struct Params {
     // STORE epilogue: row-major [groups * M, N] per half
     void *out0, *out1;
     bool out_f32;
+    // the MN-major operands (B; A too in WGRAD) come through 3D tensor maps
+    // {64 columns, rows, 64-column blocks}: one TMA instruction fetches all
+    // of a stage's 64-column atoms of an operand
+    bool mn3d;
 };
 
 // ------------------------------------------------------------------ epilogues
@@ -313,6 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     pdl_launch_dependents();
+    constexpr int kPtVar = MODE == WGRAD ? 2 : EPI;
+    PipeClock ck_total, ck_a, ck_b;
+    ck_total.start();
 
     const uint32_t tmem = ctrl->tmem_base;
     const int nE = p.g.offsets ? p.g.E : 1;
@@ -339,23 +370,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t *a = sA + s * kAStage, *b = sB + s * kBStage;
                 uint64_t *bar = &ctrl->full[s];
                 auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) { tma_load_2d(m, dst, bar, c0, c1); };
+                // an MN-major operand: `blocks` 64-column atoms from column c, k-rows from krow
+                auto mn = [&](const CUtensorMap *m, uint8_t *dst, int c, int krow, int blocks) {
+                    if (p.mn3d) {
+                        tma_load_3d(m, dst, bar, 0, krow, c / 64);
+                    } else {
+                        for (int j = 0; j < blocks; ++j) box(m, dst + j * kAtom, c + 64 * j, krow);
+                    }
+                };
                 if constexpr (MODE == ROWS) {
                     const Tile tl = decode(id, ntiles, tile_start, nE);
                     const int range = kb / kpr, kr = kb - range * kpr;
                     const CUtensorMap *ma = range ? &tmA1 : &tmA0;
                     const CUtensorMap *mb = range ? &tmB1 : &tmB0;
                     box(ma, a, kr * BK, op_row0(tl.e) + tl.m * BM);
-                    const int brow = tl.e * p.Kr + kr * BK;
-#pragma unroll
-                    for (int j = 0; j < BN / 64; ++j) box(mb, b + j * kAtom, tl.n * BN + 64 * j, brow);
+                    mn(mb, b, tl.n * BN, tl.e * p.Kr + kr * BK, BN / 64);
                 } else {
                     const WTile w = wdecode(id, mtiles, ntiles, p.halves);
                     const int krow = op_row0(w.e) + kb * 64;
-                    const CUtensorMap *ma = w.half ? &tmA1 : &tmA0;
-#pragma unroll
-                    for (int j = 0; j < BM / 64; ++j) box(ma, a + j * kAtom, w.mt * BM + 64 * j, krow);
-#pragma unroll
-                    for (int j = 0; j < BN / 64; ++j) box(&tmB0, b + j * kAtom, w.nt * BN + 64 * j, krow);
+                    mn(w.half ? &tmA1 : &tmA0, a, w.mt * BM, krow, BM / 64);
+                    mn(&tmB0, b, w.nt * BN, krow, BN / 64);
                 }
             };
             uint32_t it = 0;
@@ -364,7 +398,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nk = tile_nk(id);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
-                    if (!wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, p.g.err)) {
+                    ck_a.start();
+                    const bool got = wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, p.g.err);
+                    ck_a.stop();
+                    if (!got) {
                         ok = false;
                         break;
                     }
@@ -372,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     boxes(id, kb, s);
                 }
             }
+            ck_a.flush(kPtVar, 3);
             if (!ok) {
                 for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j) {
                     const uint64_t t0 = globaltimer();
@@ -387,13 +425,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++tc) {
                 const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-                if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.g.err)) break;
+                ck_b.start();
+                const bool free_acc = wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.g.err);
+                ck_b.stop();
+                if (!free_acc) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + acc * BN;
                 const int nk = tile_nk(id);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
-                    if (!wait_bar(&ctrl->full[s], (it / kStages) & 1, abort, p.g.err)) {
+                    ck_a.start();
+                    const bool got = wait_bar(&ctrl->full[s], (it / kStages) & 1, abort, p.g.err);
+                    ck_a.stop();
+                    if (!got) {
                         ok = false;
                         break;
                     }
@@ -409,6 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (ok) mma_commit(&ctrl->tfull[acc]);
             }
+            ck_a.flush(kPtVar, 1);
+            ck_b.flush(kPtVar, 2);
         }
     } else if (warp < kEpiWarps) {
         uint32_t tc = 0;
@@ -436,16 +482,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 UV buf[2];
                 load_uv(p, r, tl.n * BN, gidx >= 0, buf[0]);
-                if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err)) break;
+                ck_a.start();
+                const bool ready = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+                ck_a.stop();
+                if (!ready) break;
                 tc_fence_after();
+                ck_b.start();
                 if (__any_sync(0xffffffffu, valid))
                     epilogue_swiglu(p, tl.n, r, op_row0(tl.e) + local, gidx, g, tmem + acc * BN + lane_base, buf);
+                ck_b.stop();
                 tc_fence_before();
                 mbar_arrive(&ctrl->tempty[acc]);
                 continue;
             }
-            if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err)) break;
+            ck_a.start();
+            const bool ready = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+            ck_a.stop();
+            if (!ready) break;
             tc_fence_after();
+            ck_b.start();
             const uint32_t tb = tmem + acc * BN + lane_base;
             if constexpr (MODE == ROWS) {
                 const Tile tl = decode(id, ntiles, tile_start, nE);
@@ -462,8 +517,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const WTile w = wdecode(id, mtiles, ntiles, p.halves);
                 epilogue_store(p, w.e, w.half, w.mt * BM + row, w.nt * BN, seg_end[w.e] > seg_off[w.e], tb);
             }
+            ck_b.stop();
             tc_fence_before();
             mbar_arrive(&ctrl->tempty[acc]);
+        }
+        if (threadIdx.x == 0) {
+            ck_a.flush(kPtVar, 4);
+            ck_b.flush(kPtVar, 5);
         }
     }
 
@@ -471,6 +531,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    ck_total.stop();
+    if (threadIdx.x == 0) {
+        ck_total.flush(kPtVar, 0);
+#ifdef MOE_PIPE_TRACE
+        atomicAdd(&g_pipe_trace[kPtVar][6], 1ull);
+#endif
+    }
 }
 
 // ------------------------------------------------------------------ two-SM kernel
@@ -590,23 +657,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) {
                     tma_load_2d_pair(m, dst, fb, c0, c1);
                 };
+                // an MN-major operand: this CTA's two 64-column atoms from column c
+                auto mn = [&](const CUtensorMap *m, uint8_t *dst, int c, int krow) {
+                    if (p.mn3d) {
+                        tma_load_3d_pair(m, dst, fb, 0, krow, c / 64);
+                    } else {
+                        for (int j = 0; j < 2; ++j) box(m, dst + j * kAtom, c + 64 * j, krow);
+                    }
+                };
                 if constexpr (MODE == ROWS) {
                     const Tile tl = decode(id, ntiles, tile_start, nE);
                     const int range = kb / kpr, kr = kb - range * kpr;
                     const CUtensorMap *ma = range ? &tmA1 : &tmA0;
                     const CUtensorMap *mb = range ? &tmB1 : &tmB0;
                     box(ma, a, kr * BK, op_row0(tl.e) + tl.m * BM2 + half_off);
-                    const int brow = tl.e * p.Kr + kr * BK;
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) box(mb, b + j * kAtom, tl.n * BN + half_off + 64 * j, brow);
+                    mn(mb, b, tl.n * BN + half_off, tl.e * p.Kr + kr * BK);
                 } else {
                     const WTile w = wdecode(id, mtiles, ntiles, p.halves);
                     const int krow = op_row0(w.e) + kb * 64;
-                    const CUtensorMap *ma = w.half ? &tmA1 : &tmA0;
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) box(ma, a + j * kAtom, w.mt * BM2 + half_off + 64 * j, krow);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) box(&tmB0, b + j * kAtom, w.nt * BN + half_off + 64 * j, krow);
+                    mn(w.half ? &tmA1 : &tmA0, a, w.mt * BM2 + half_off, krow);
+                    mn(&tmB0, b, w.nt * BN + half_off, krow);
                 }
             };
             uint32_t it = 0;
@@ -759,25 +829,64 @@ bool map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same tensor viewed as {64 columns, rows, cols / 64 blocks} (block stride
+// 128 bytes), box of 64 x box_rows x box_blocks: one box holds box_blocks
+// 64-column atoms of box_rows rows, each atom 64 * box_rows * 2 bytes after
+// the previous one in shared memory.  Needs cols % 64 == 0, so that every
+// in-range coordinate is an element of the tensor.
+bool map_bf16_3d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows,
+                 uint32_t box_blocks) {
+    auto fn = tc::encode_fn();
+    if (!fn || ld % 8 || cols % 64 || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {ld * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, box_blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps of a backward GEMM: A (K-major boxes of a_box rows in ROWS, else
+// MN-major) and B (MN-major), 3D for the MN-major operands when every one of
+// them allows it (p.mn3d), else 2D boxes of one 64-column atom.
+template <int MODE>
+bool bwd_maps(const BwdOperand &a0, const BwdOperand &a1, const BwdOperand &b0, const BwdOperand &b1, uint32_t a_box,
+              uint32_t mn_blocks_a, uint32_t mn_blocks_b, CUtensorMap *mA0, CUtensorMap *mA1, CUtensorMap *mB0,
+              CUtensorMap *mB1, bool *mn3d) {
+    const BwdOperand *ops[4] = {&a0, &a1, &b0, &b1};
+    CUtensorMap *maps[4] = {mA0, mA1, mB0, mB1};
+    for (int pass = 0; pass < 2; ++pass) {
+        const bool three = pass == 0;
+        bool ok = true;
+        for (int i = 0; i < 4 && ok; ++i) {
+            const BwdOperand &o = *ops[i];
+            if (!o.base) {
+                *maps[i] = *maps[i & 2];   // a1 / b1 absent: the first map of the pair
+                continue;
+            }
+            const bool mn_major = i >= 2 || MODE == gb::WGRAD;
+            if (!mn_major) ok = map_bf16(maps[i], o.base, o.rows, o.cols, o.ld, a_box);
+            else if (three) ok = map_bf16_3d(maps[i], o.base, o.rows, o.cols, o.ld, 64, i >= 2 ? mn_blocks_b : mn_blocks_a);
+            else ok = map_bf16(maps[i], o.base, o.rows, o.cols, o.ld, 64);
+        }
+        if (ok) {
+            *mn3d = three;
+            return true;
+        }
+    }
+    return false;
+}
+
 template <int MODE, int EPI>
 cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOperand &b0, const BwdOperand &b1,
                        const gb::Params &p, cudaStream_t s) {
     using namespace gb;
     CUtensorMap mA0, mA1, mB0, mB1;
+    Params q = p;
     // ROWS: A K-major boxes of 128 rows; otherwise MN-major boxes of 64 k-rows
-    const uint32_t a_box = MODE == ROWS ? BM : 64;
-    if (!map_bf16(&mA0, a0.base, a0.rows, a0.cols, a0.ld, a_box)) return cudaErrorInvalidValue;
-    if (!map_bf16(&mB0, b0.base, b0.rows, b0.cols, b0.ld, 64)) return cudaErrorInvalidValue;
-    if (a1.base) {
-        if (!map_bf16(&mA1, a1.base, a1.rows, a1.cols, a1.ld, a_box)) return cudaErrorInvalidValue;
-    } else {
-        mA1 = mA0;
-    }
-    if (b1.base) {
-        if (!map_bf16(&mB1, b1.base, b1.rows, b1.cols, b1.ld, 64)) return cudaErrorInvalidValue;
-    } else {
-        mB1 = mB0;
-    }
+    if (!bwd_maps<MODE>(a0, a1, b0, b1, MODE == ROWS ? BM : 64, BM / 64, BN / 64, &mA0, &mA1, &mB0, &mB1, &q.mn3d))
+        return cudaErrorInvalidValue;
     const int nE = p.g.offsets ? p.g.E : 1;
     const int ntiles = (p.N + BN - 1) / BN;
     int64_t max_tiles;
@@ -790,7 +899,7 @@ cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOper
     auto kern = bwd_gemm_kernel<MODE, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(kern, grid, kThreads, smem, s, mA0, mA1, mB0, mB1, p);
+    return launch_kernel(kern, grid, kThreads, smem, s, mA0, mA1, mB0, mB1, q);
 }
 
 template <int MODE, int EPI>
@@ -798,19 +907,10 @@ cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const Bw
                             const gb::Params &p, cudaStream_t s) {
     using namespace gb;
     CUtensorMap mA0, mA1, mB0, mB1;
-    const uint32_t a_box = MODE == ROWS ? 128 : 64;
-    if (!map_bf16(&mA0, a0.base, a0.rows, a0.cols, a0.ld, a_box)) return cudaErrorInvalidValue;
-    if (!map_bf16(&mB0, b0.base, b0.rows, b0.cols, b0.ld, 64)) return cudaErrorInvalidValue;
-    if (a1.base) {
-        if (!map_bf16(&mA1, a1.base, a1.rows, a1.cols, a1.ld, a_box)) return cudaErrorInvalidValue;
-    } else {
-        mA1 = mA0;
-    }
-    if (b1.base) {
-        if (!map_bf16(&mB1, b1.base, b1.rows, b1.cols, b1.ld, 64)) return cudaErrorInvalidValue;
-    } else {
-        mB1 = mB0;
-    }
+    Params q = p;
+    // each CTA of the pair: 128 rows of A (ROWS), two 64-column atoms of each MN-major operand
+    if (!bwd_maps<MODE>(a0, a1, b0, b1, MODE == ROWS ? 128 : 64, 2, 2, &mA0, &mA1, &mB0, &mB1, &q.mn3d))
+        return cudaErrorInvalidValue;
     const size_t smem = 1024 + (size_t)kPStages * 2 * kPStage + (EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0) +
                         sizeof(Ctrl2) + 4 * sizeof(int) * (p.g.E + 1);
     auto kern = bwd_gemm_pair_kernel<MODE, EPI>;
@@ -837,7 +937,7 @@ cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const Bw
     if (MODE == ROWS) max_tiles = (p.g.rows / 256 + nE) * (int64_t)ntiles;
     else max_tiles = (int64_t)nE * p.halves * ((p.M + 255) / 256) * ntiles;
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(std::max(max_pairs, 1), max_tiles));
-    return launch_kernel_pair(kern, 2 * pairs, kThreads, smem, s, mA0, mA1, mB0, mB1, p);
+    return launch_kernel_pair(kern, 2 * pairs, kThreads, smem, s, mA0, mA1, mB0, mB1, q);
 }
 
 // Two-SM tiles where there is enough work for them: ROWS when the groups
@@ -896,3 +996,17 @@ cudaError_t launch_bwd_gemm(const BwdGemm &L, cudaStream_t s) {
 }
 
 }  // namespace moe
+
+#ifdef MOE_PIPE_TRACE
+// Diagnostic build only: copies the pipeline trace (4 x 8 counters, see
+// above) to host memory and optionally clears it.
+extern "C" int moe_debug_pipe_trace(unsigned long long *out, int reset) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return 1;
+    if (cudaMemcpyFromSymbol(out, moe::gb::g_pipe_trace, sizeof(moe::gb::g_pipe_trace)) != cudaSuccess) return 1;
+    if (reset) {
+        static const unsigned long long zero[4][8] = {};
+        if (cudaMemcpyToSymbol(moe::gb::g_pipe_trace, zero, sizeof(zero)) != cudaSuccess) return 1;
+    }
+    return 0;
+}
+#endif

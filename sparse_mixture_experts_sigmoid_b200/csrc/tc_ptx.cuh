@@ -76,6 +76,14 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *m, void *dst, uin
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
+// A 3D box (c0 innermost) into this CTA's shared memory, completion on an
+// mbarrier of this CTA.
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
 // The same load with an L2 cache policy (from createpolicy).
 __device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int c1,
                                                  uint64_t policy) {
@@ -255,6 +263,16 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *m, void *dst
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(bar_cluster)
+        : "memory");
+}
+
+// The 3D form of tma_load_2d_pair.
+__device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap *m, void *dst, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(bar_cluster)
         : "memory");
 }
 
