@@ -699,10 +699,12 @@ moe_status moe_forward_q4(const moe_config *c, const moe_route_opts *opts, const
         e = launch_permute(pa, part<int32_t>(ws, L, P_PERM), false, s);
     }
     mark(1 + MOE_STAGE_PERMUTE, s);
+    // the ring-streamed kernels where the shapes and alignments allow them
+    const bool tma = q4_tma_supported(c->d, c->h, x, q_gate, s_gate, q_up, s_up, q_down, s_down);
     if (e == cudaSuccess) {
         SegGateUpQ4Args ga{x, q_gate, q_up, s_gate, s_up, Segments{offsets, srt, c->E, c->k, (int64_t)R}, c->T, c->d,
                            c->h, act};
-        e = launch_seg_gateup_q4(ga, s, err);
+        e = tma ? launch_q4t_gateup(ga, s) : launch_seg_gateup_q4(ga, s, err);
     }
     mark(1 + MOE_STAGE_GATE_UP, s);
     if (e == cudaSuccess && shared) {
@@ -713,7 +715,28 @@ moe_status moe_forward_q4(const moe_config *c, const moe_route_opts *opts, const
     if (e == cudaSuccess) {
         DownDirectQ4Args da{act, q_down, s_down, ids, inv, gates, shared ? acts : nullptr, shared ? sh_down : nullptr,
                             sg, c->T, c->d, c->h, c->E, c->k, c->h_shared, y};
-        e = launch_down_direct_q4(da, s, err);
+        if (!tma) {
+            e = launch_down_direct_q4(da, s, err);
+        } else {
+            // the shared expert's gated rows first, into the (cleared) fp32
+            // accumulator, one contribution per element; the 4-bit kernel adds
+            // them after the routed experts
+            float *acc = shared ? part<float>(ws, L, P_YACC) : nullptr;
+            if (shared) {
+                e = cudaMemsetAsync(acc, 0, (size_t)c->T * c->d * sizeof(float), s);
+                SegDownArgs sa{};
+                sa.act = acts;
+                sa.w_down = sh_down;
+                sa.seg = Segments{nullptr, nullptr, 1, 1, c->T};
+                sa.T = c->T;
+                sa.d = c->d;
+                sa.hid = c->h_shared;
+                sa.gates = sg;
+                sa.y_acc = acc;
+                if (e == cudaSuccess) e = launch_seg_down(sa, c->dtype, s, err);
+            }
+            if (e == cudaSuccess) e = launch_q4t_down(da, acc, s);
+        }
     }
     mark(1 + MOE_STAGE_DOWN, s);
     mark(1 + MOE_STAGE_SHARED_DOWN, s);

@@ -189,7 +189,15 @@ struct DownDirectQ4Args {
 cudaError_t launch_quantize_q4(const void *w, int dtype, int64_t rows, int cols, uint8_t *q, float *scales,
                                cudaStream_t s);
 cudaError_t launch_seg_gateup_q4(const SegGateUpQ4Args &a, cudaStream_t s, uint32_t *err);
+// The same two steps with the codes streamed through a shared-memory ring by
+// TMA (segment_q4_tma.cu), for d and h multiples of 256 and 16-byte aligned
+// codes and scales; the down kernel writes y, adding shared_add [T, d] fp32
+// (the shared expert's rows) when it is not null.
+bool q4_tma_supported(int d, int h, const void *x, const void *q_gate, const float *s_gate, const void *q_up, const float *s_up,
+                      const void *q_down, const float *s_down);
+cudaError_t launch_q4t_gateup(const SegGateUpQ4Args &a, cudaStream_t s);
 cudaError_t launch_down_direct_q4(const DownDirectQ4Args &a, cudaStream_t s, uint32_t *err);
+cudaError_t launch_q4t_down(const DownDirectQ4Args &a, const float *shared_add, cudaStream_t s);
 
 // Tensor-core grouped GEMM (grouped_gemm.cu).
 struct GemmParams {

@@ -84,6 +84,13 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *m, void *dst, uin
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
 }
+// Contiguous global -> shared copy by the TMA unit (both addresses 16-byte
+// aligned, bytes a multiple of 16), completion on an mbarrier of this CTA.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 // The same load with an L2 cache policy (from createpolicy).
 __device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int c1,
                                                  uint64_t policy) {

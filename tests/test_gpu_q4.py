@@ -54,6 +54,13 @@ CASES = [
     case("decode_T3_k8", T=3, E=64, k=8, d=256, h=128, router_std=0.2, seed=142),
     case("decode_T16_k4", T=16, seed=143),
     case("decode_sigmoid_nonorm", score="sigmoid", norm_topk=False, T=2, seed=144),
+    # d and h multiples of 256: the kernels that stream the codes through a
+    # shared-memory ring (a last partial 1024-element chunk in the second and
+    # third; experts holding more than two rows, so several passes, in the others)
+    case("ring_decode_T1", h=512, seed=145),
+    case("ring_T16_shared_ragged_chunks", T=16, d=768, h=1280, h_shared=256, seed=146),
+    case("ring_T16_E4_k1", T=16, E=4, k=1, d=256, h=1280, seed=147),
+    case("ring_T3_k8", T=3, E=64, k=8, d=256, h=256, router_std=0.2, seed=148),
 ]
 
 
