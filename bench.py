@@ -52,7 +52,8 @@ STAGE_KERNEL = {"route": ("router_logits_kernel", "router_tc.cu"), "permute": ("
 STAGE_KERNEL_SMALL = {"route": ("router_small_kernel", "router.cu"), "gate_up": ("seg_gateup_kernel", "segment.cu"),
                       "down": ("down_direct_kernel", "segment.cu")}
 # ... with 4-bit routed experts
-STAGE_KERNEL_Q4 = {"gate_up": ("seg_gateup_q4_kernel", "segment_q4.cu"), "down": ("down_direct_q4_kernel", "segment_q4.cu")}
+# (the ring-streamed kernels, which the library picks for d and h multiples of 256)
+STAGE_KERNEL_Q4 = {"gate_up": ("q4t_gateup_kernel", "segment_q4_tma.cu"), "down": ("q4t_down_kernel", "segment_q4_tma.cu")}
 
 
 def parse():
@@ -333,7 +334,8 @@ def time_workload(args, w, ws_n, rank, local, steps, warmup, headline, q4=False)
            "steps": K, "weights": "routed experts 4-bit (64-weight groups, fp32 scales)" if q4 else w.dtype,
            "warmup": W, "gpu_launches": launches, "layer": lfr,
            "dominant": {"stage": dom, "kernel": kname, "ms_per_launch": stage[dom],
-                        "algorithmic_flops": work[dom]["flops"], "algorithmic_bytes": work[dom]["bytes"], **dfr},
+                        "algorithmic_flops": work[dom]["flops"], "algorithmic_bytes": work[dom]["bytes"],
+                        "traffic": traffic_for(dom, ksrc, w.name + ("_q4" if q4 else "")), **dfr},
            "stages_ms": stage, "stages": per_stage, "clocks": clocks, "tensor_peak": tpk, "tensor_peak_kind": tpk_kind,
            "load": roofline.load_spread(counts)}
     res["_roof"] = (dom, kname, ksrc, dfr, peaks, tpk, tpk_kind)
@@ -438,7 +440,7 @@ def bench_ours(args, w, ws_n, rank, local):
     else:
         roof = {"bound": "hbm", "achieved": dfr["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for(dom, ksrc, w.name)
+    roof["traffic"] = head["dominant"]["traffic"]
     roof.update({"tensor_frac": dfr["tensor_frac"], "hbm_frac": dfr["hbm_frac"],
                  "tensor_frac_of_burst": dfr["tflops"] / peaks["bf16_tflops"],
                  "kernel": kname, "stage": dom, "ms_per_launch": head["dominant"]["ms_per_launch"],

@@ -294,6 +294,16 @@ __device__ __forceinline__ WTile wdecode(int id, int mtiles, int ntiles, int hal
     return w;
 }
 
+// A tile's operand coordinates, worked out once per tile by the producer
+// (the tile decode walks the tile table in shared memory, too slow to repeat
+// for every K block): ROWS: the first A row and the weights' first row and
+// column; WGRAD: the A map, the weight row and column of the tile and the
+// expert's first K row.
+struct TileAt {
+    int a_row, b_row, b_col;   // ROWS
+    int half, m0, n0, krow0;   // WGRAD
+};
+
 template <int MODE, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -366,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kTmaWarp) {
         if (lane == 0) {
             // the boxes of K block kb of tile id, into stage s
-            auto boxes = [&](int id, int kb, int s) {
+            auto boxes = [&](const TileAt &t, int kb, int s) {
                 uint8_t *a = sA + s * kAStage, *b = sB + s * kBStage;
                 uint64_t *bar = &ctrl->full[s];
                 auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) { tma_load_2d(m, dst, bar, c0, c1); };
@@ -379,23 +389,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 };
                 if constexpr (MODE == ROWS) {
-                    const Tile tl = decode(id, ntiles, tile_start, nE);
-                    const int range = kb / kpr, kr = kb - range * kpr;
-                    const CUtensorMap *ma = range ? &tmA1 : &tmA0;
-                    const CUtensorMap *mb = range ? &tmB1 : &tmB0;
-                    box(ma, a, kr * BK, op_row0(tl.e) + tl.m * BM);
-                    mn(mb, b, tl.n * BN, tl.e * p.Kr + kr * BK, BN / 64);
+                    const int range = kb >= kpr, kr = kb - range * kpr;
+                    box(range ? &tmA1 : &tmA0, a, kr * BK, t.a_row);
+                    mn(range ? &tmB1 : &tmB0, b, t.b_col, t.b_row + kr * BK, BN / 64);
                 } else {
-                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                    const int krow = op_row0(w.e) + kb * 64;
-                    mn(w.half ? &tmA1 : &tmA0, a, w.mt * BM, krow, BM / 64);
-                    mn(&tmB0, b, w.nt * BN, krow, BN / 64);
+                    const int krow = t.krow0 + kb * 64;
+                    mn(t.half ? &tmA1 : &tmA0, a, t.m0, krow, BM / 64);
+                    mn(&tmB0, b, t.n0, krow, BN / 64);
                 }
             };
             uint32_t it = 0;
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
                 const int nk = tile_nk(id);
+                TileAt t{};
+                if constexpr (MODE == ROWS) {
+                    const Tile tl = decode(id, ntiles, tile_start, nE);
+                    t.a_row = op_row0(tl.e) + tl.m * BM;
+                    t.b_row = tl.e * p.Kr;
+                    t.b_col = tl.n * BN;
+                } else {
+                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
+                    t.half = w.half;
+                    t.m0 = w.mt * BM;
+                    t.n0 = w.nt * BN;
+                    t.krow0 = op_row0(w.e);
+                }
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
                     ck_a.start();
@@ -406,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_expect_tx(&ctrl->full[s], kAStage + kBStage);
-                    boxes(id, kb, s);
+                    boxes(t, kb, s);
                 }
             }
             ck_a.flush(kPtVar, 3);
@@ -651,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kTx = 2u * 2u * kPStage;   // A and B of both CTAs
             const uint32_t full_lead = mapa_shared(&ctrl->full[0], 0);
             // this CTA's boxes of K block kb of tile id, into stage s
-            auto boxes = [&](int id, int kb, int s) {
+            auto boxes = [&](const TileAt &t, int kb, int s) {
                 uint8_t *a = sA + s * kPStage, *b = sB + s * kPStage;
                 const uint32_t fb = full_lead + s * (uint32_t)sizeof(uint64_t);
                 auto box = [&](const CUtensorMap *m, uint8_t *dst, int c0, int c1) {
@@ -666,23 +685,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 };
                 if constexpr (MODE == ROWS) {
-                    const Tile tl = decode(id, ntiles, tile_start, nE);
-                    const int range = kb / kpr, kr = kb - range * kpr;
-                    const CUtensorMap *ma = range ? &tmA1 : &tmA0;
-                    const CUtensorMap *mb = range ? &tmB1 : &tmB0;
-                    box(ma, a, kr * BK, op_row0(tl.e) + tl.m * BM2 + half_off);
-                    mn(mb, b, tl.n * BN + half_off, tl.e * p.Kr + kr * BK);
+                    const int range = kb >= kpr, kr = kb - range * kpr;
+                    box(range ? &tmA1 : &tmA0, a, kr * BK, t.a_row);
+                    mn(range ? &tmB1 : &tmB0, b, t.b_col, t.b_row + kr * BK);
                 } else {
-                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                    const int krow = op_row0(w.e) + kb * 64;
-                    mn(w.half ? &tmA1 : &tmA0, a, w.mt * BM2 + half_off, krow);
-                    mn(&tmB0, b, w.nt * BN + half_off, krow);
+                    const int krow = t.krow0 + kb * 64;
+                    mn(t.half ? &tmA1 : &tmA0, a, t.m0, krow);
+                    mn(&tmB0, b, t.n0, krow);
                 }
             };
             uint32_t it = 0;
             bool ok = true;
             for (int id = pair; id < total && ok; id += npairs) {
                 const int nk = tile_nk(id);
+                TileAt t{};
+                if constexpr (MODE == ROWS) {
+                    const Tile tl = decode(id, ntiles, tile_start, nE);
+                    t.a_row = op_row0(tl.e) + tl.m * BM2 + half_off;
+                    t.b_row = tl.e * p.Kr;
+                    t.b_col = tl.n * BN + half_off;
+                } else {
+                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
+                    t.half = w.half;
+                    t.m0 = w.mt * BM2 + half_off;
+                    t.n0 = w.nt * BN + half_off;
+                    t.krow0 = op_row0(w.e);
+                }
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kPStages;
                     if (!wait_bar(&ctrl->empty[s], ((it / kPStages) & 1) ^ 1, abort, p.g.err)) {
@@ -690,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (lead) mbar_expect_tx(&ctrl->full[s], kTx);
-                    boxes(id, kb, s);
+                    boxes(t, kb, s);
                 }
             }
             if (!ok) {
