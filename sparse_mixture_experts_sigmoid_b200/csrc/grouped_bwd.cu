@@ -59,10 +59,12 @@ constexpr int kAStage = BM * 128;         // 16 KB
 constexpr int kBStage = BN * 128;         // 32 KB
 constexpr int kStages = 4;
 constexpr int kAtom = 8192;               // one MN-major atom column: 64 k-rows x 128 bytes
-constexpr int kEpiWarps = 4;
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+// Warp roles: epilogue warps first, then the TMA producer and the MMA issuer.
+// The SwiGLU and weight-gradient epilogues run on eight warps (warp w drains
+// TMEM lanes 32 (w mod 4) .. + 31, columns 128 (w / 4) .. + 127 of the 256),
+// the scatter epilogue, which is not the bottleneck and needs 4 KB of
+// staging per warp, on four.
+constexpr int kScatterEpiWarps = 4;
 constexpr int kTmemCols = 512;
 
 enum { ROWS = 0, WGRAD = 1 };
@@ -91,6 +93,14 @@ struct PipeClock {
 };
 #endif
 enum { EPI_SWIGLU = 0, EPI_SCATTER = 1, EPI_STORE = 2 };
+template <int EPI>
+constexpr int epi_warps() {
+    return EPI == EPI_SCATTER ? kScatterEpiWarps : 8;
+}
+template <int EPI>
+constexpr int kernel_threads() {
+    return (epi_warps<EPI>() + 2) * 32;
+}
 
 struct Ctrl {
     uint64_t full[kStages];
@@ -164,32 +174,36 @@ __device__ __forceinline__ void load_uv(const Params &p, int64_t r, int col0, bo
 
 // ROWS / SWIGLU epilogue of grouped row r of column tile nt (gidx: its
 // assignment, or token for the dense expert; -1 if the row is not valid; g:
-// its gate); D = r_i over 256 columns from TMEM address tbase.  The outputs
-// go to row ro (r in the padded layout).  buf[0] holds the first 32 columns'
-// u | v already (loaded before the accumulator was ready); each later chunk's
-// loads are issued before the TMEM wait of the chunk before it, so one L2
-// round trip is in flight while a chunk is computed.
-__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int64_t r, int64_t ro, int64_t gidx, float g,
-                                                uint32_t tbase, UV (&buf)[2]) {
+// its gate); D = r_i from TMEM.  The outputs go to row ro (r in the padded
+// layout).  buf[0] holds the first 32 columns' u | v already (loaded before
+// the accumulator was ready); each later chunk's loads are issued before the
+// TMEM wait of the chunk before it, so one L2 round trip is in flight while
+// a chunk is computed.  With two warps per row each adds its partial dot
+// product into the row's gate gradient.
+// This warp drains NC columns from column c0 of the tile (tbase points at
+// column c0).
+template <int NC>
+__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int c0, int64_t r, int64_t ro, int64_t gidx,
+                                                float g, uint32_t tbase, UV (&buf)[2]) {
     const int N = p.N;
     float dot = 0.f;
     // two chunks per iteration, so the buffers are named statically while the
     // loop body stays small enough for the instruction cache
 #pragma unroll 1
-    for (int c2 = 0; c2 < BN / 64; ++c2)
+    for (int c2 = 0; c2 < NC / 64; ++c2)
 #pragma unroll
     for (int hc = 0; hc < 2; ++hc) {
         const int ci = 2 * c2 + hc;
         float v[2][16];
         tmem_ld16(tbase + 32 * ci, v[0]);
         tmem_ld16(tbase + 32 * ci + 16, v[1]);
-        if (ci + 1 < BN / 32) load_uv(p, r, nt * BN + 32 * (ci + 1), gidx >= 0, buf[hc ^ 1]);
+        if (ci + 1 < NC / 32) load_uv(p, r, nt * BN + c0 + 32 * (ci + 1), gidx >= 0, buf[hc ^ 1]);
         tmem_wait_ld();
         if (gidx < 0) continue;
         const UV &b = buf[hc];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int col = nt * BN + 32 * ci + 8 * q;
+            const int col = nt * BN + c0 + 32 * ci + 8 * q;
             if (col >= N) continue;
             const __nv_bfloat162 *u2 = reinterpret_cast<const __nv_bfloat162 *>(&b.u[q]);
             const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&b.v[q]);
@@ -230,8 +244,9 @@ __device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int64_t
     if (gidx >= 0) atomicAdd(p.dgate + gidx, dot);
 }
 
-// WGRAD / STORE: weight row m (of M, in half `half`) of group e, 256 columns
-// from n0; zero when the group had no rows.
+// WGRAD / STORE: weight row m (of M, in half `half`) of group e, NC columns
+// from n0 (TMEM from tbase); zero when the group had no rows.
+template <int NC>
 __device__ __forceinline__ void epilogue_store(const Params &p, int e, int half, int m, int n0, bool has_rows,
                                                uint32_t tbase) {
     const bool valid = m < p.M;
@@ -239,7 +254,7 @@ __device__ __forceinline__ void epilogue_store(const Params &p, int e, int half,
     const int64_t orow = (int64_t)e * p.M + m;
     void *out = half ? p.out1 : p.out0;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = 0; c < NC; c += 32) {
         float v[2][16];
         if (has_rows) {
             tmem_ld16(tbase + c, v[0]);
@@ -305,10 +320,12 @@ struct TileAt {
 };
 
 template <int MODE, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1, Params p) {
     constexpr uint32_t kIdesc = idesc_bwd<MODE>();
+    constexpr int kEpiWarps = epi_warps<EPI>(), kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
+    constexpr int kCols = BN / (kEpiWarps / 4);   // columns one epilogue warp drains
     constexpr int kEpiStage = EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0;
 
     extern __shared__ uint8_t smem_raw[];
@@ -477,8 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kEpiWarps) {
         uint32_t tc = 0;
-        const int row = warp * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int row = (warp & 3) * 32 + lane;
+        const int c0 = (warp >> 2) * kCols;   // this warp's first column of the tile
+        const uint32_t lane_base = ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c0;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++tc) {
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             if constexpr (MODE == ROWS && EPI == EPI_SWIGLU) {
@@ -500,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 UV buf[2];
-                load_uv(p, r, tl.n * BN, gidx >= 0, buf[0]);
+                load_uv(p, r, tl.n * BN + c0, gidx >= 0, buf[0]);
                 ck_a.start();
                 const bool ready = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
                 ck_a.stop();
@@ -508,7 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 ck_b.start();
                 if (__any_sync(0xffffffffu, valid))
-                    epilogue_swiglu(p, tl.n, r, op_row0(tl.e) + local, gidx, g, tmem + acc * BN + lane_base, buf);
+                    epilogue_swiglu<kCols>(p, tl.n, c0, r, op_row0(tl.e) + local, gidx, g, tmem + acc * BN + lane_base,
+                                           buf);
                 ck_b.stop();
                 tc_fence_before();
                 mbar_arrive(&ctrl->tempty[acc]);
@@ -534,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
                 const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                epilogue_store(p, w.e, w.half, w.mt * BM + row, w.nt * BN, seg_end[w.e] > seg_off[w.e], tb);
+                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM + row, w.nt * BN + c0, seg_end[w.e] > seg_off[w.e], tb);
             }
             ck_b.stop();
             tc_fence_before();
@@ -594,11 +613,13 @@ constexpr uint32_t idesc_bwd2() {
 }
 
 template <int MODE, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     bwd_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                          const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                          Params p) {
     constexpr uint32_t kIdesc = idesc_bwd2<MODE>();
+    constexpr int kEpiWarps = epi_warps<EPI>(), kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
+    constexpr int kCols = BN / (kEpiWarps / 4);   // columns one epilogue warp drains
     constexpr int kEpiStage = EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0;
     constexpr int BM2 = 256;
 
@@ -768,8 +789,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kEpiWarps) {
         uint32_t tc = 0;
-        const int row = warp * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int row = (warp & 3) * 32 + lane;
+        const int c0 = (warp >> 2) * kCols;   // this warp's first column of the tile
+        const uint32_t lane_base = ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c0;
         const uint32_t tempty_lead = mapa_shared(&ctrl->tempty[0], 0);
         for (int id = pair; id < total; id += npairs, ++tc) {
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
@@ -793,12 +815,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     UV buf[2];
-                    load_uv(p, r, tl.n * BN, gidx >= 0, buf[0]);
+                    load_uv(p, r, tl.n * BN + c0, gidx >= 0, buf[0]);
                     got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
                     if (!got) break;
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, valid))
-                        epilogue_swiglu(p, tl.n, r, op_row0(tl.e) + local, gidx, g, tb, buf);
+                        epilogue_swiglu<kCols>(p, tl.n, c0, r, op_row0(tl.e) + local, gidx, g, tb, buf);
                 } else {
                     got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
                     if (!got) break;
@@ -811,7 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!got) break;
                 tc_fence_after();
                 const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                epilogue_store(p, w.e, w.half, w.mt * BM2 + half_off + row, w.nt * BN, seg_end[w.e] > seg_off[w.e],
+                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM2 + half_off + row, w.nt * BN + c0, seg_end[w.e] > seg_off[w.e],
                                tb);
             }
             tc_fence_before();
@@ -922,12 +944,12 @@ cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOper
     else max_tiles = (int64_t)nE * p.halves * ((p.M + BM - 1) / BM) * ntiles;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
     const size_t smem = 1024 + (size_t)kStages * (kAStage + kBStage) +
-                        (EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0) + sizeof(Ctrl) +
+                        (EPI == EPI_SCATTER ? kScatterEpiWarps * gg::kEpiStageBytes : 0) + sizeof(Ctrl) +
                         4 * sizeof(int) * (p.g.E + 1);
     auto kern = bwd_gemm_kernel<MODE, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(kern, grid, kThreads, smem, s, mA0, mA1, mB0, mB1, q);
+    return launch_kernel(kern, grid, kernel_threads<EPI>(), smem, s, mA0, mA1, mB0, mB1, q);
 }
 
 template <int MODE, int EPI>
@@ -939,7 +961,7 @@ cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const Bw
     // each CTA of the pair: 128 rows of A (ROWS), two 64-column atoms of each MN-major operand
     if (!bwd_maps<MODE>(a0, a1, b0, b1, MODE == ROWS ? 128 : 64, 2, 2, &mA0, &mA1, &mB0, &mB1, &q.mn3d))
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + (size_t)kPStages * 2 * kPStage + (EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0) +
+    const size_t smem = 1024 + (size_t)kPStages * 2 * kPStage + (EPI == EPI_SCATTER ? kScatterEpiWarps * gg::kEpiStageBytes : 0) +
                         sizeof(Ctrl2) + 4 * sizeof(int) * (p.g.E + 1);
     auto kern = bwd_gemm_pair_kernel<MODE, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -947,7 +969,7 @@ cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const Bw
     // as many CTA pairs as can be resident at once, capped by the tile count
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kernel_threads<EPI>());
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -965,7 +987,7 @@ cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const Bw
     if (MODE == ROWS) max_tiles = (p.g.rows / 256 + nE) * (int64_t)ntiles;
     else max_tiles = (int64_t)nE * p.halves * ((p.M + 255) / 256) * ntiles;
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(std::max(max_pairs, 1), max_tiles));
-    return launch_kernel_pair(kern, 2 * pairs, kThreads, smem, s, mA0, mA1, mB0, mB1, q);
+    return launch_kernel_pair(kern, 2 * pairs, kernel_threads<EPI>(), smem, s, mA0, mA1, mB0, mB1, q);
 }
 
 // Two-SM tiles where there is enough work for them: ROWS when the groups
