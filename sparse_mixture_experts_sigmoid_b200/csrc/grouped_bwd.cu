@@ -78,19 +78,9 @@ enum { ROWS = 0, WGRAD = 1 };
 // number of CTAs.  Read with moe_debug_pipe_trace (same build only).
 #ifdef MOE_PIPE_TRACE
 __device__ unsigned long long g_pipe_trace[4][8];
-struct PipeClock {
-    unsigned long long acc = 0;
-    long long t0 = 0;
-    __device__ void start() { t0 = clock64(); }
-    __device__ void stop() { acc += (unsigned long long)(clock64() - t0); }
-    __device__ void flush(int var, int slot) { atomicAdd(&g_pipe_trace[var][slot], acc); }
-};
+#define PIPE_SLOT(var, slot) (&g_pipe_trace[var][slot])
 #else
-struct PipeClock {
-    __device__ void start() {}
-    __device__ void stop() {}
-    __device__ void flush(int, int) {}
-};
+#define PIPE_SLOT(var, slot) nullptr
 #endif
 enum { EPI_SWIGLU = 0, EPI_SCATTER = 1, EPI_STORE = 2 };
 template <int EPI>
@@ -445,7 +435,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                     boxes(t, kb, s);
                 }
             }
-            ck_a.flush(kPtVar, 3);
+            ck_a.flush(PIPE_SLOT(kPtVar, 3));
             if (!ok) {
                 for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j) {
                     const uint64_t t0 = globaltimer();
@@ -489,8 +479,8 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                 }
                 if (ok) mma_commit(&ctrl->tfull[acc]);
             }
-            ck_a.flush(kPtVar, 1);
-            ck_b.flush(kPtVar, 2);
+            ck_a.flush(PIPE_SLOT(kPtVar, 1));
+            ck_b.flush(PIPE_SLOT(kPtVar, 2));
         }
     } else if (warp < kEpiWarps) {
         uint32_t tc = 0;
@@ -560,8 +550,8 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
             mbar_arrive(&ctrl->tempty[acc]);
         }
         if (threadIdx.x == 0) {
-            ck_a.flush(kPtVar, 4);
-            ck_b.flush(kPtVar, 5);
+            ck_a.flush(PIPE_SLOT(kPtVar, 4));
+            ck_b.flush(PIPE_SLOT(kPtVar, 5));
         }
     }
 
@@ -571,7 +561,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
     ck_total.stop();
     if (threadIdx.x == 0) {
-        ck_total.flush(kPtVar, 0);
+        ck_total.flush(PIPE_SLOT(kPtVar, 0));
 #ifdef MOE_PIPE_TRACE
         atomicAdd(&g_pipe_trace[kPtVar][6], 1ull);
 #endif

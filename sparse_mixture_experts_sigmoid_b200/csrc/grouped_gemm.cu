@@ -95,6 +95,20 @@ struct Ctrl {
 
 // ------------------------------------------------------------------ kernel
 
+// Pipeline trace of this kernel in a diagnostic build (-DMOE_PIPE_TRACE; read
+// with moe_debug_fwd_trace): per variant (gate/up, down, 64-row down), SM
+// cycles summed over CTAs for [0] the whole kernel, [1] the MMA issuer
+// waiting for operands, [2] it waiting for a free accumulator, [3] the TMA
+// producer waiting for a free stage, [4] epilogue warp 0 waiting for an
+// accumulator, [5] it draining one, [6] the number of CTAs, [7] the first
+// gather thread waiting for a free stage.
+#ifdef MOE_PIPE_TRACE
+__device__ unsigned long long g_fwd_trace[4][8];
+#define FWD_SLOT(var, slot) (&g_fwd_trace[var][slot])
+#else
+#define FWD_SLOT(var, slot) nullptr
+#endif
+
 // HALF (contiguous A only): 64-row tiles whose A stage holds 64 rows, for
 // experts of at most 64 rows, where the weights stream from HBM and the rows
 // of a 128-row A stage would mostly sit empty.  The MMA still has M = 128: its
@@ -174,6 +188,9 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     const int total = ctrl->n_mtiles * n_tiles;
     const int nk = (p.K + BK - 1) / BK;
     const int nE = p.offsets ? p.E : 1;
+    constexpr int kPtVar = MODE == GATEUP ? 0 : (HALF ? 2 : 1);
+    PipeClock ck_total, ck_a, ck_b;
+    ck_total.start();
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
@@ -224,7 +241,10 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                         if (!GATHER && !early_a) tma_load_2d(&tmA, sA + s * kAStage, &ctrl->full[s], kb * BK, a_row);
                         continue;
                     }
-                    if (!wait_bar(&ctrl->empty[s], ph ^ 1, abort, p.err)) {
+                    ck_a.start();
+                    const bool got = wait_bar(&ctrl->empty[s], ph ^ 1, abort, p.err);
+                    ck_a.stop();
+                    if (!got) {
                         ok = false;
                         break;
                     }
@@ -233,6 +253,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                     load_b(s, kb, b_row);
                 }
             }
+            ck_a.flush(FWD_SLOT(kPtVar, 3));
             if (!ok) {
                 // aborting: let the copies already issued land before the CTA exits
                 for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j) {
@@ -249,13 +270,19 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++tc) {
                 const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-                if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
+                ck_b.start();
+                const bool free_acc = wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err);
+                ck_b.stop();
+                if (!free_acc) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + acc * BN;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
-                    if (!wait_bar(&ctrl->full[s], ph, abort, p.err)) {
+                    ck_a.start();
+                    const bool got = wait_bar(&ctrl->full[s], ph, abort, p.err);
+                    ck_a.stop();
+                    if (!got) {
                         ok = false;
                         break;
                     }
@@ -272,6 +299,8 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                 }
                 if (ok) mma_commit(&ctrl->tfull[acc]);
             }
+            ck_a.flush(FWD_SLOT(kPtVar, 1));
+            ck_b.flush(FWD_SLOT(kPtVar, 2));
         }
     } else if (warp < kEpiWarps) {
         if (MODE == GATEUP && p.zero) {
@@ -289,23 +318,42 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++tc) {
             const Tile tl = decode_n(id, n_tiles, p.n_groups, ctrl->n_mtiles, tile_start, nE);
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-            if (!wait_bar(&ctrl->tfull[acc], aph, abort, p.err)) break;
+            ck_a.start();
+            const bool ready = wait_bar(&ctrl->tfull[acc], aph, abort, p.err);
+            ck_a.stop();
+            if (!ready) break;
             tc_fence_after();
+            ck_b.start();
             const int64_t r = (int64_t)seg_off[tl.e] + (int64_t)tl.m * RB + row;
             epilogue_row<MODE, T, BN>(p, tl.n, r, row < RB && r < seg_end[tl.e], tmem + acc * BN + lane_base,
                                       reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
+            ck_b.stop();
             tc_fence_before();
             mbar_arrive(&ctrl->tempty[acc]);
         }
+        if (threadIdx.x == 0) {
+            ck_a.flush(FWD_SLOT(kPtVar, 4));
+            ck_b.flush(FWD_SLOT(kPtVar, 5));
+        }
     } else if (GATHER && warp >= kGatherWarp0) {
+        PipeClock ck_g;
         gather_rows<T, kStages, RB, kGatherThreads>(p, threadIdx.x - kGatherWarp0 * 32, blockIdx.x, gridDim.x, total, n_tiles,
-                                    tile_start, seg_off, seg_end, nE, nk, 0, sA, ctrl->full, ctrl->empty, abort);
+                                    tile_start, seg_off, seg_end, nE, nk, 0, sA, ctrl->full, ctrl->empty, abort,
+                                    &ck_g);
+        if (threadIdx.x == kGatherWarp0 * 32) ck_g.flush(FWD_SLOT(kPtVar, 7));
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    ck_total.stop();
+    if (threadIdx.x == 0) {
+        ck_total.flush(FWD_SLOT(kPtVar, 0));
+#ifdef MOE_PIPE_TRACE
+        atomicAdd(&g_fwd_trace[kPtVar][6], 1ull);
+#endif
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -370,3 +418,17 @@ cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t s) {
 }
 
 }  // namespace moe
+
+#ifdef MOE_PIPE_TRACE
+// Diagnostic build only: copies the forward pipeline trace (4 x 8 counters,
+// see above) to host memory and optionally clears it.
+extern "C" int moe_debug_fwd_trace(unsigned long long *out, int reset) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return 1;
+    if (cudaMemcpyFromSymbol(out, moe::gg::g_fwd_trace, sizeof(moe::gg::g_fwd_trace)) != cudaSuccess) return 1;
+    if (reset) {
+        static const unsigned long long zero[4][8] = {};
+        if (cudaMemcpyToSymbol(moe::gg::g_fwd_trace, zero, sizeof(zero)) != cudaSuccess) return 1;
+    }
+    return 0;
+}
+#endif

@@ -183,7 +183,8 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
 template <typename T, int S, int RB, int NG = 128>
 __device__ bool gather_rows(const GemmParams &p, int g, int first, int stride, int total, int n_tiles,
                             const int *tile_start, const int *seg_off, const int *seg_end, int nE, int nk,
-                            int row_off, uint8_t *sA, uint64_t *full, uint64_t *empty, volatile int *abort) {
+                            int row_off, uint8_t *sA, uint64_t *full, uint64_t *empty, volatile int *abort,
+                            PipeClock *ck = nullptr) {
     constexpr int BK = 128 / (int)sizeof(T);
     constexpr int V = 16 / (int)sizeof(T);
     constexpr int kABytes = 128 * 128;
@@ -232,7 +233,10 @@ __device__ bool gather_rows(const GemmParams &p, int g, int first, int stride, i
         for (int kb = 0; kb < nk; ++kb, ++it) {
             const int s = it % S;
             const uint32_t ph = (it / S) & 1;
-            if (!wait_bar(&empty[s], ph ^ 1, abort, p.err)) {
+            if (ck) ck->start();
+            const bool got = wait_bar(&empty[s], ph ^ 1, abort, p.err);
+            if (ck) ck->stop();
+            if (!got) {
                 ok = false;
                 break;
             }

@@ -182,6 +182,25 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
+// Cycle counter for the pipeline traces of the GEMM kernels; with
+// -DMOE_PIPE_TRACE (a diagnostic build) it accumulates clock64() spans and
+// adds them into a device array, otherwise it compiles to nothing.
+#ifdef MOE_PIPE_TRACE
+struct PipeClock {
+    unsigned long long acc = 0;
+    long long t0 = 0;
+    __device__ void start() { t0 = clock64(); }
+    __device__ void stop() { acc += (unsigned long long)(clock64() - t0); }
+    __device__ void flush(unsigned long long *slot) { atomicAdd(slot, acc); }
+};
+#else
+struct PipeClock {
+    __device__ void start() {}
+    __device__ void stop() {}
+    __device__ void flush(unsigned long long *) {}
+};
+#endif
+
 // ---- two-SM (cta_group::2) forms, for kernels launched in clusters of two CTAs.
 // The even CTA of the pair (rank 0) issues the MMAs; each CTA holds its half of
 // A (M rows 0-127 / 128-255) and of B (N columns 0-N/2 / N/2-N) at the same
