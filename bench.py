@@ -176,15 +176,39 @@ def source_hash(src: str) -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_for(stage: str, src: str, workload: str):
-    """DRAM bytes per launch of a stage's kernel from a committed ncu capture
-    (profiles/traffic.json), if the kernel's source is unchanged since."""
+def _capture(stage: str, src: str, workload: str):
+    """A stage's entry in profiles/traffic.json (from a committed ncu capture),
+    if the kernel's source is unchanged since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             ent = json.load(f)[stage][workload]
-        return float(ent["bytes_per_launch"]) if ent.get("src_sha") == source_hash(src) else None
+        return ent if ent.get("src_sha") == source_hash(src) else None
     except (OSError, KeyError, ValueError):
         return None
+
+
+def traffic_for(stage: str, src: str, workload: str):
+    """DRAM bytes per launch of a stage's kernel (dram__bytes_read.sum +
+    dram__bytes_write.sum), or None."""
+    ent = _capture(stage, src, workload)
+    return float(ent["bytes_per_launch"]) if ent else None
+
+
+def ncu_ms_for(stage: str, src: str, workload: str):
+    """The stage's kernel time per launch in the same capture
+    (gpu__time_duration.sum: serialised, cold-cache, no event boundaries), or None."""
+    ent = _capture(stage, src, workload)
+    return float(ent["us_per_launch"]) / 1e3 if ent and "us_per_launch" in ent else None
+
+
+def kernel_of(stage: str, w, q4: bool):
+    """(kernel name, source) of a stage for workload w."""
+    kname, ksrc = STAGE_KERNEL[stage]
+    if w.R <= B.decode_max_rows() and stage in STAGE_KERNEL_SMALL:
+        kname, ksrc = STAGE_KERNEL_SMALL[stage]
+    if q4 and stage in STAGE_KERNEL_Q4:
+        kname, ksrc = STAGE_KERNEL_Q4[stage]
+    return kname, ksrc
 
 
 def config_json(w, n):
@@ -316,26 +340,26 @@ def time_workload(args, w, ws_n, rank, local, steps, warmup, headline, q4=False)
     tpk, tpk_kind = tensor_peak(peaks, clocks)
     work = roofline.stage_work(w, counts, q4=q4)
     dom = max((n for n in stage if n in work), key=lambda n: stage[n])
-    kname, ksrc = STAGE_KERNEL[dom]
-    if w.R <= B.decode_max_rows() and dom in STAGE_KERNEL_SMALL:
-        kname, ksrc = STAGE_KERNEL_SMALL[dom]
-    if q4 and dom in STAGE_KERNEL_Q4:
-        kname, ksrc = STAGE_KERNEL_Q4[dom]
+    kname, ksrc = kernel_of(dom, w, q4)
+    cap_name = w.name + ("_q4" if q4 else "")
     dfr = roofline.fractions(work[dom]["flops"], work[dom]["bytes"], stage[dom] / 1e3, peaks, tpk)
     lw = roofline.layer_work(w, counts, q4=q4)
     lfr = roofline.fractions(lw["flops"], lw["bytes"], ms / 1e3, peaks, tpk)
     lfr["tensor_frac_of_burst"] = lfr["tflops"] / peaks["bf16_tflops"]
-    # both roofline fractions of every stage that ran (event-timed, so an upper bound on each kernel's time)
-    per_stage = {n: {"ms": stage[n], **{k_: v for k_, v in roofline.fractions(
-        work[n]["flops"], work[n]["bytes"], stage[n] / 1e3, peaks, tpk).items() if k_ in ("bound", "tensor_frac",
-                                                                                         "hbm_frac", "frac")}}
+    # both roofline fractions of every stage that ran (event-timed, so an upper bound on each kernel's time),
+    # next to the kernel's time in the committed ncu capture (serialised, cold-cache) when it still applies
+    per_stage = {n: {"ms": stage[n], "ncu_ms": ncu_ms_for(n, kernel_of(n, w, q4)[1], cap_name),
+                     **{k_: v for k_, v in roofline.fractions(
+                         work[n]["flops"], work[n]["bytes"], stage[n] / 1e3, peaks, tpk).items()
+                        if k_ in ("bound", "tensor_frac", "hbm_frac", "frac")}}
                  for n in stage if n in work and stage[n] > 0.004}
     res = {"workload": w.name + ("_q4" if q4 else ""), "tokens_per_s": job_value(ws_n, w.T, ms), "ms_per_step": ms,
            "steps": K, "weights": "routed experts 4-bit (64-weight groups, fp32 scales)" if q4 else w.dtype,
            "warmup": W, "gpu_launches": launches, "layer": lfr,
            "dominant": {"stage": dom, "kernel": kname, "ms_per_launch": stage[dom],
                         "algorithmic_flops": work[dom]["flops"], "algorithmic_bytes": work[dom]["bytes"],
-                        "traffic": traffic_for(dom, ksrc, w.name + ("_q4" if q4 else "")), **dfr},
+                        "ncu_ms_per_launch": ncu_ms_for(dom, ksrc, cap_name),
+                        "traffic": traffic_for(dom, ksrc, cap_name), **dfr},
            "stages_ms": stage, "stages": per_stage, "clocks": clocks, "tensor_peak": tpk, "tensor_peak_kind": tpk_kind,
            "load": roofline.load_spread(counts)}
     res["_roof"] = (dom, kname, ksrc, dfr, peaks, tpk, tpk_kind)
@@ -444,6 +468,7 @@ def bench_ours(args, w, ws_n, rank, local):
     roof.update({"tensor_frac": dfr["tensor_frac"], "hbm_frac": dfr["hbm_frac"],
                  "tensor_frac_of_burst": dfr["tflops"] / peaks["bf16_tflops"],
                  "kernel": kname, "stage": dom, "ms_per_launch": head["dominant"]["ms_per_launch"],
+                 "ncu_ms_per_launch": head["dominant"]["ncu_ms_per_launch"],
                  "algorithmic_bytes": head["dominant"]["algorithmic_bytes"],
                  "algorithmic_flops": head["dominant"]["algorithmic_flops"],
                  "peak_source": f"{peaks['source']} ({'cuBLAS bf16 ' + tpk_kind if bound == 'tensor' else 'HBM copy'})"})
