@@ -382,6 +382,13 @@ typedef enum {
  * records an empty interval.  events == NULL turns the hook off.  Host only. */
 moe_status moe_profile_events(void *const *events, int32_t n);
 
+/* NVTX ranges for the calling host thread: with on != 0, every later
+ * moe_forward (or moe_forward_q4) call on this thread opens an NVTX range
+ * named "moe <stage>" around the launches of each stage, so a profiler that
+ * records NVTX shows which host calls issued which kernels.  on == 0 turns
+ * them off (the default).  Host only; never fails. */
+moe_status moe_profile_nvtx(int32_t on);
+
 /* Number of kernels this library has launched in this process (all threads). */
 int64_t moe_launch_count(void);
 

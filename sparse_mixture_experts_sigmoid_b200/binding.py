@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_DEVICE_INPUT"}
 EXPORTED = ["moe_status_string", "moe_validate", "moe_workspace_size", "moe_workspace_layout", "moe_route",
             "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_decode_max_rows",
-            "moe_device_status", "moe_profile_events", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size",
+            "moe_device_status", "moe_profile_events", "moe_profile_nvtx", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size",
             "moe_selftest_wait_timeout",
             "moe_route_workspace_size", "moe_update_bias", "moe_balance_loss", "moe_train_workspace_size",
             "moe_forward_train", "moe_backward", "moe_quantize_q4", "moe_forward_q4"]
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "moe_balance_loss": ([C, P, P, ctypes.c_float, P, P, P], ctypes.c_int),
             "moe_decode_max_rows": ([], ctypes.c_int32),
             "moe_device_status": ([P], ctypes.c_int),
+            "moe_profile_nvtx": ([ctypes.c_int32], ctypes.c_int),
             "moe_selftest_wait_timeout": ([ctypes.c_uint32, P], ctypes.c_int),
             "moe_profile_events": ([ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32], ctypes.c_int),
             "moe_launch_count": ([], ctypes.c_int64),
@@ -514,3 +515,9 @@ def forward_q4(cfg: MoEConfig, layer, q4: dict, y=None, ws=None, stream=None, ba
                                 _ptr(layer.w_shared_gate, "w_shared_gate", (d,), et), _ptr(y, "y", (cfg.T, d), et),
                                 _ptr(ws, "ws", dtype=torch.uint8), ws.numel(), _stream(stream)), "moe_forward_q4")
     return y
+
+
+def profile_nvtx(on: bool = True) -> None:
+    """moe_profile_nvtx: NVTX ranges around each forward stage on this thread."""
+    _check(lib().moe_profile_nvtx(int(bool(on))), "moe_profile_nvtx")
+

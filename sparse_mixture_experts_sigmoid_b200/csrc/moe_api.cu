@@ -1,6 +1,8 @@
 // C ABI of libmoe.so: argument validation, workspace layout and the launch
 // sequence of the MoE layer forward pass.  Declarations and contracts are in
 // include/moe.h.
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <cstdlib>
 #include <mutex>
@@ -109,8 +111,19 @@ std::atomic<int64_t> g_launches{0};
 thread_local cudaEvent_t t_events[MOE_STAGE_COUNT + 1];
 thread_local bool t_profile = false;
 
+// Per-thread NVTX stage ranges (moe_profile_nvtx).
+thread_local bool t_nvtx = false;
+const char *const kStageNames[MOE_STAGE_COUNT] = {"moe route",      "moe permute",     "moe gate_up",
+                                                  "moe shared gate_up", "moe down", "moe shared down",
+                                                  "moe finalize"};
+
+// Boundary i of a forward call: 0 before the first launch, 1 + s after stage s.
 void mark(int i, cudaStream_t s) {
     if (t_profile) cudaEventRecord(t_events[i], s);
+    if (t_nvtx) {
+        if (i > 0) nvtxRangePop();
+        if (i < MOE_STAGE_COUNT) nvtxRangePushA(kStageNames[i]);
+    }
 }
 
 // The tensor-core grouped GEMM serves batches above this many assignments;
@@ -764,6 +777,11 @@ moe_status moe_profile_events(void *const *events, int32_t n) {
         t_events[i] = static_cast<cudaEvent_t>(events[i]);
     }
     t_profile = true;
+    return MOE_OK;
+}
+
+moe_status moe_profile_nvtx(int32_t on) {
+    t_nvtx = on != 0;
     return MOE_OK;
 }
 

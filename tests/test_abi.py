@@ -190,3 +190,9 @@ def test_ordered_combine_workspace():
     with pytest.raises(ValueError):
         B.config(16, 64, 8, 128, 2, combine="sorted")
 
+
+
+def test_profile_nvtx_is_host_only():
+    """Turning the NVTX stage ranges on and off needs no GPU and never fails."""
+    assert B.lib().moe_profile_nvtx(1) == 0
+    assert B.lib().moe_profile_nvtx(0) == 0

@@ -269,3 +269,19 @@ def test_zero_tokens():
     B.forward(cfg, x, z, wgt, wgt, wd, y=y, ws=torch.empty(256, dtype=torch.uint8, device="cuda"))
     torch.cuda.synchronize()
     assert B.device_status() == 0
+
+
+def test_forward_with_nvtx_ranges_gives_the_same_bits():
+    """moe_profile_nvtx only adds host-side ranges: y is bit-identical with them on."""
+    w = SMALL[0]
+    layer, dev, a = checked(w)
+    cfg = B.config_of(w, combine="ordered")
+    y0 = B.forward_layer(cfg, dev).cpu()
+    B.profile_nvtx(True)
+    try:
+        y1 = B.forward_layer(cfg, dev).cpu()
+    finally:
+        B.profile_nvtx(False)
+    assert B.device_status() == 0
+    assert torch.equal(y0, y1)
+
