@@ -18,7 +18,7 @@
 //      gate's w_s term (finalize_dx_kernel)
 //   5. weight gradients: dW_down, dW_gate / dW_up per expert over its rows,
 //      the shared expert's over all tokens, dW_router = dl^T x (WEIGHT), and
-//      dw_s = sum_t dl_s x_t (shared_gate_grad_kernel)
+//      dw_s = sum_t dl_s x_t (shared_gate_grad_kernel, fixed summation order)
 //
 // The top-k selection (and the balance bias) passes no gradient.
 #include <algorithm>
@@ -59,16 +59,17 @@ __global__ void __launch_bounds__(256) gather_pad_kernel(GatherPadArgs a) {
     }
     __syncthreads();
     const int cpr = a.d / 8;                 // 16-byte chunks per x / dy row
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
         const gg::Tile tl = gg::decode(b, 1, blk, a.E);
         const int64_t pr0 = (int64_t)b * 64;               // first padded row of the block
         const int64_t r0 = (int64_t)off[tl.e] + tl.m * 64;  // its first grouped row
-        // x_g and dy_g: copy or zero, 16 bytes per thread step
-        for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
-            const int q = i / cpr, c = i - q * cpr;
+        // x_g and dy_g: one warp per row (its token looked up once), each lane
+        // four 16-byte chunks of x and of dy in flight before it stores them
+        for (int q = warp; q < 64; q += 8) {
             const int64_t r = r0 + q;
             int64_t t = -1;
-            if (r < end[tl.e]) {
+            if (lane == 0 && r < end[tl.e]) {
                 const int v = a.sorted_rows[r];
                 t = (v >= 0 && v < a.R) ? v / a.k : -1;
                 if (t < 0 || t >= a.T) {
@@ -76,13 +77,31 @@ __global__ void __launch_bounds__(256) gather_pad_kernel(GatherPadArgs a) {
                     t = -1;
                 }
             }
-            uint4 vx = make_uint4(0, 0, 0, 0), vd = vx;
-            if (t >= 0) {
-                vx = *reinterpret_cast<const uint4 *>(a.x + t * a.d + 8 * c);
-                vd = *reinterpret_cast<const uint4 *>(a.dy + t * a.d + 8 * c);
+            t = __shfl_sync(0xffffffffu, t, 0);
+            uint4 *xo = reinterpret_cast<uint4 *>(a.xg + (pr0 + q) * a.d);
+            uint4 *dyo = reinterpret_cast<uint4 *>(a.dyg + (pr0 + q) * a.d);
+            const uint4 *xi = reinterpret_cast<const uint4 *>(a.x + (t < 0 ? 0 : t) * a.d);
+            const uint4 *dyi = reinterpret_cast<const uint4 *>(a.dy + (t < 0 ? 0 : t) * a.d);
+            for (int c0 = lane; c0 < cpr; c0 += 4 * 32) {
+                uint4 vx[4], vd[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + 32 * u;
+                    vx[u] = vd[u] = make_uint4(0, 0, 0, 0);
+                    if (t >= 0 && c < cpr) {
+                        vx[u] = xi[c];
+                        vd[u] = dyi[c];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + 32 * u;
+                    if (c < cpr) {
+                        __stcs(xo + c, vx[u]);
+                        __stcs(dyo + c, vd[u]);
+                    }
+                }
             }
-            *reinterpret_cast<uint4 *>(a.xg + (pr0 + q) * a.d + 8 * c) = vx;
-            *reinterpret_cast<uint4 *>(a.dyg + (pr0 + q) * a.d + 8 * c) = vd;
         }
         // dH and ga: zero the padding rows (the SWIGLU epilogue writes the others)
         const int64_t rem = (int64_t)end[tl.e] - r0;
@@ -158,28 +177,74 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdArgs a) {
     if (lane == 0 && a.dls) a.dls[t] = a.dsg[t] * a.sg[t] * (1.f - a.sg[t]);
 }
 
-// dx[t, i] = bf16(acc[t, i] + dls[t] * w_s[i]) (the w_s term only with a shared expert).
+// dx[t, i] = bf16(acc[t, i] + dls[t] * w_s[i]) (the w_s term only with a
+// shared expert), eight elements per thread step (d % 8 == 0): two 16-byte
+// loads and one 16-byte store.
 __global__ void finalize_dx_kernel(const float *acc, const float *dls, const __nv_bfloat16 *ws, __nv_bfloat16 *dx,
                                    int64_t T, int d) {
     pdl_wait();
     pdl_launch_dependents();
-    const int64_t n = T * d;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        float v = acc[i];
-        if (dls) v += dls[i / d] * __bfloat162float(ws[i % d]);
-        dx[i] = __float2bfloat16_rn(v);
+    const int cpr = d / 8;
+    const int64_t chunks = T * cpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = *reinterpret_cast<const float4 *>(acc + 8 * i);
+        const float4 b = *reinterpret_cast<const float4 *>(acc + 8 * i + 4);
+        float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        if (dls) {
+            const int64_t t = i / cpr;
+            const int c = (int)(i - t * cpr) * 8;
+            const float g = dls[t];
+            float w[8];
+            load8(ws + c, w);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = fmaf(g, w[j], v[j]);
+        }
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            o[j] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(dx + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
-// dw_s[i] = sum over t (in increasing order) of dls[t] * x[t, i].
-__global__ void shared_gate_grad_kernel(const float *dls, const __nv_bfloat16 *x, float *dws, int64_t T, int d) {
+// dw_s[i] = sum over t of dls[t] * x[t, i], in a fixed order: a CTA takes 32
+// columns (one per lane); warp w of its 32 sums the w-th 32nd of the tokens
+// in increasing order, eight loads in flight at a time, and the 32 partial
+// sums are added in warp order.
+__global__ void __launch_bounds__(1024) shared_gate_grad_kernel(const float *dls, const __nv_bfloat16 *x, float *dws,
+                                                                int64_t T, int d) {
+    __shared__ float part[32][33];
     pdl_wait();
     pdl_launch_dependents();
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= d) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int i = blockIdx.x * 32 + lane;
+    const int64_t per = (T + 31) / 32, t0 = warp * per, t1 = t0 + per < T ? t0 + per : T;
     float s = 0.f;
-    for (int64_t t = 0; t < T; ++t) s = fmaf(dls[t], __bfloat162float(x[t * d + i]), s);
-    dws[i] = s;
+    if (i < d) {
+        int64_t t = t0;
+        for (; t + 8 <= t1; t += 8) {
+            float xv[8], g[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                xv[u] = __bfloat162float(x[(t + u) * d + i]);
+                g[u] = dls[t + u];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s = fmaf(g[u], xv[u], s);
+        }
+        for (; t < t1; ++t) s = fmaf(dls[t], __bfloat162float(x[t * d + i]), s);
+    }
+    part[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0 && i < d) {
+        float r = 0.f;
+#pragma unroll
+        for (int w = 0; w < 32; ++w) r += part[w][lane];
+        dws[i] = r;
+    }
 }
 
 cudaError_t set0(void *p, size_t bytes, cudaStream_t s) { return p && bytes ? cudaMemsetAsync(p, 0, bytes, s) : cudaSuccess; }
@@ -369,7 +434,7 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
         e = launch_bwd_gemm(g, s);
     }
     if (e == cudaSuccess) {
-        const int64_t n = T * d;
+        const int64_t n = T * (d / 8);
         const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, 4LL * num_sms() * 8);
         e = launch_kernel(finalize_dx_kernel, blocks, 256, 0, s, static_cast<const float *>(acc),
                           static_cast<const float *>(shared ? dls : nullptr),
@@ -467,7 +532,7 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
         e = launch_bwd_gemm(g, s);
     }
     if (e == cudaSuccess && shared)
-        e = launch_kernel(shared_gate_grad_kernel, (unsigned)((d + 127) / 128), 128, 0, s,
+        e = launch_kernel(shared_gate_grad_kernel, (unsigned)((d + 31) / 32), 1024, 0, s,
                           static_cast<const float *>(dls), static_cast<const __nv_bfloat16 *>(x), dw_shared_gate, T, d);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
