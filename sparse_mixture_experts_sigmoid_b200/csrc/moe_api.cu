@@ -557,12 +557,20 @@ moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const v
     const bool fused_hist = L.size[P_LOGITS] && c->T * c->k > permute_chunk();
     ra.hist = fused_hist ? part<int32_t>(ws, L, P_PERM) : nullptr;
     ra.hist_chunk = permute_chunk();
+    // one token (decode): the router writes the grouping itself
+    const bool one_token = c->T == 1 && !L.size[P_LOGITS];
+    if (one_token) {
+        ra.counts = counts;
+        ra.offsets = offsets;
+        ra.sorted_rows = srt;
+        ra.inv_rows = inv;
+    }
     mark(0, s);
     cudaError_t e = launch_router(ra, c->dtype, part<float>(ws, L, P_LOGITS), s);
     mark(1 + MOE_STAGE_ROUTE, s);
 
     const int R = (int)(c->T * c->k);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && !one_token) {
         PermuteArgs pa{ids, R, c->E, counts, offsets, srt, inv, err};
         e = launch_permute(pa, part<int32_t>(ws, L, P_PERM), fused_hist, s);
     }
@@ -703,11 +711,18 @@ moe_status moe_forward_q4(const moe_config *c, const moe_route_opts *opts, const
     ra.score_mean = opts ? opts->score_mean : nullptr;
     ra.stats = ra.score_mean ? part<float>(ws, L, P_STATS) : nullptr;
     ra.hist_chunk = permute_chunk();
+    const bool one_token = c->T == 1 && !L.size[P_LOGITS];
+    if (one_token) {
+        ra.counts = counts;
+        ra.offsets = offsets;
+        ra.sorted_rows = srt;
+        ra.inv_rows = inv;
+    }
     mark(0, s);
     cudaError_t e = launch_router(ra, c->dtype, part<float>(ws, L, P_LOGITS), s);
     mark(1 + MOE_STAGE_ROUTE, s);
     const int R = (int)(c->T * c->k);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && !one_token) {
         PermuteArgs pa{ids, R, c->E, counts, offsets, srt, inv, err};
         e = launch_permute(pa, part<int32_t>(ws, L, P_PERM), false, s);
     }

@@ -84,6 +84,9 @@ struct RouterArgs {
     const float *bias;  // optional [E] balance bias: selection key = score + bias
     float *stats;       // optional [router_stats_rows(T), E] per-CTA score sums (fixed order)
     float *score_mean;  // optional [E] out: mean score per expert (needs stats)
+    // optional, T == 1 only (the one-token router): the grouping of the token's
+    // k assignments, written by the router itself (no separate grouping step)
+    int32_t *counts, *offsets, *sorted_rows, *inv_rows;
 };
 // Rows of per-CTA score sums the routers write for the score-mean statistic:
 // one per token for the one-token-per-CTA router (T <= 64), else at most one
