@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
 // 16-byte loads, all issued before the reduction), so the router weights are
 // streamed by the whole CTA at once.  Warp 0 then selects the top k with the
 // same arg-max rounds as the batched router.
-template <typename Tin, int EP>
+template <typename Tin>
 __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     pdl_wait();
     pdl_launch_dependents();
@@ -299,55 +299,18 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     __syncthreads();
     const Tin *wr = static_cast<const Tin *>(a.w_router);
     const int Ep = a.E + (a.w_shared_gate ? 1 : 0);
-    auto row_of = [&](int e) { return e < a.E ? wr + (int64_t)e * a.d : static_cast<const Tin *>(a.w_shared_gate); };
-    if (EP > 0) {
-        // few logits: every thread takes its eight-column chunks of all Ep rows
-        // at once (Ep loads in flight), then the CTA adds the partial sums,
-        // each warp's in a fixed shuffle order and the warps' in warp order
-        __shared__ float red[kWarps][EP > 0 ? EP : 1];
-        float part[EP > 0 ? EP : 1];
-#pragma unroll
-        for (int e = 0; e < EP; ++e) part[e] = 0.f;
-        for (int c = threadIdx.x * 8; c < a.d; c += kThreads * 8) {
-            float xv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) xv[u] = sx[c + u];
-#pragma unroll
-            for (int e = 0; e < EP; ++e) {
-                if (e < Ep) {
-                    float w[8];
-                    load8(row_of(e) + c, w);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) part[e] = fmaf(w[u], xv[u], part[e]);
-                }
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < EP; ++e) {
-            const float v = warp_sum(part[e]);
-            if (lane == 0) red[warp][e] = v;
-        }
-        __syncthreads();
-        if (threadIdx.x < Ep) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) v += red[w][threadIdx.x];
-            lg[threadIdx.x] = v;
-        }
-    } else {
-        for (int e = warp; e < Ep; e += kWarps) {
-            const Tin *row = row_of(e);
-            float acc = 0.f;
+    for (int e = warp; e < Ep; e += kWarps) {
+        const Tin *row = e < a.E ? wr + (int64_t)e * a.d : static_cast<const Tin *>(a.w_shared_gate);
+        float acc = 0.f;
 #pragma unroll 4
-            for (int c = lane * 8; c < a.d; c += 256) {
-                float w[8];
-                load8(row + c, w);
+        for (int c = lane * 8; c < a.d; c += 256) {
+            float w[8];
+            load8(row + c, w);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) acc = fmaf(w[u], sx[c + u], acc);
-            }
-            acc = warp_sum(acc);
-            if (lane == 0) lg[e] = acc;
+            for (int u = 0; u < 8; ++u) acc = fmaf(w[u], sx[c + u], acc);
         }
+        acc = warp_sum(acc);
+        if (lane == 0) lg[e] = acc;
     }
     __syncthreads();
     if (warp != 0) return;
@@ -464,13 +427,6 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     if (lane == 0 && a.shared_gate && a.w_shared_gate) a.shared_gate[t] = 1.f / (1.f + expf(-lg[a.E]));
 }
 
-// Logit columns up to which the one-token router reads all router rows in
-// one pass (each thread its chunks of every row) instead of a warp per row.
-#ifndef MOE_ONE_PASS_LOGITS
-#define MOE_ONE_PASS_LOGITS 16
-#endif
-constexpr int kOnePassLogits = MOE_ONE_PASS_LOGITS;
-
 int pow2ceil(int v) {
     int p = 1;
     while (p < v) p <<= 1;
@@ -545,10 +501,7 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaSt
     if (scratch && router_tc_supported(a.T, a.E, dtype)) return launch_router_tc(a, scratch, s);
     if (a.T <= kSmallT) {
         const size_t smem = sizeof(float) * ((size_t)a.d + a.E + 1);
-        const int Ep = a.E + (a.w_shared_gate ? 1 : 0);
-        auto pick = [&](auto f32, auto bf16) { return dtype == MOE_F32 ? f32 : bf16; };
-        auto kern = Ep <= kOnePassLogits ? pick(router_small_kernel<float, 16>, router_small_kernel<__nv_bfloat16, 16>)
-                                         : pick(router_small_kernel<float, 0>, router_small_kernel<__nv_bfloat16, 0>);
+        auto kern = dtype == MOE_F32 ? router_small_kernel<float> : router_small_kernel<__nv_bfloat16>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess) e = launch_kernel(kern, (unsigned)a.T, kThreads, smem, s, a);
         if (e == cudaSuccess && a.stats && a.score_mean)
