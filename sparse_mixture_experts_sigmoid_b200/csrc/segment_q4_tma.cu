@@ -38,7 +38,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int kQWarps = 16;                            // consumer warps
+#ifndef MOE_Q4_WARPS
+#define MOE_Q4_WARPS 16
+#endif
+constexpr int kQWarps = MOE_Q4_WARPS;                  // consumer warps
+static_assert(kQWarps == 8 || kQWarps == 16, "32 rows per item over the consumer warps, within 1024 threads");
 constexpr int kQThreads = (kQWarps + 1) * 32;          // + the producer warp
 constexpr int kQRows = 32;                             // weight rows per work item
 constexpr int kQRW = kQRows / kQWarps;                 // weight rows per consumer warp
