@@ -69,15 +69,16 @@ constexpr int kTmemCols = 512;
 
 enum { ROWS = 0, WGRAD = 1 };
 
-// Pipeline trace of the one-SM kernel, compiled in only with -DMOE_PIPE_TRACE
-// (a diagnostic build): per kernel variant (ROWS/SWIGLU, ROWS/SCATTER,
-// WGRAD), SM cycles summed over CTAs for [0] the whole kernel, [1] the MMA
+// Pipeline trace of the backward kernels, compiled in only with
+// -DMOE_PIPE_TRACE (a diagnostic build): per kernel variant (rows 0-2: the
+// one-SM kernel's ROWS/SWIGLU, ROWS/SCATTER and WGRAD; rows 4-6: the same for
+// the two-SM kernel, summed over both CTAs of a pair), SM cycles summed over CTAs for [0] the whole kernel, [1] the MMA
 // issuer waiting for operands, [2] the MMA issuer waiting for a free
 // accumulator, [3] the producer waiting for a free stage, [4] epilogue warp 0
 // waiting for an accumulator, [5] epilogue warp 0 draining one, and [6] the
 // number of CTAs.  Read with moe_debug_pipe_trace (same build only).
 #ifdef MOE_PIPE_TRACE
-__device__ unsigned long long g_pipe_trace[4][8];
+__device__ unsigned long long g_pipe_trace[8][8];
 #define PIPE_SLOT(var, slot) (&g_pipe_trace[var][slot])
 #else
 #define PIPE_SLOT(var, slot) nullptr
@@ -144,60 +145,118 @@ struct Params {
 
 // ------------------------------------------------------------------ epilogues
 
-// ROWS / SWIGLU: the kept pre-activations u | v of 32 columns from col0 of
-// grouped row r, as raw bf16 (four 16-byte loads each).
+// Row exchange through shared memory.  An epilogue thread owns one row of
+// the accumulator (TMEM lane = row), so a thread-per-row global access makes
+// each warp instruction touch 32 rows, 16 bytes each.  Instead every warp
+// moves 64-byte pieces of its 32 rows through 2 KB of its own shared memory:
+// global memory is read and written as 8 rows x 64 contiguous bytes per
+// instruction (4 threads per row), and the row-wise side stays in registers.
+// The 16-byte word j of row i sits at i * 64 + 16 * (j ^ ((i >> 1) & 3)), so
+// both the row-wise and the column-wise shared accesses are free of bank
+// conflicts (each group of 8 threads covers all 32 banks once).
+constexpr int kXBytes = 32 * 64;   // one warp's exchange buffer
+
+// Shared memory of the epilogue warps: the scatter's row staging, else the
+// exchange buffers (16 KB either way).
+template <int EPI>
+constexpr int epi_stage_bytes() {
+    return EPI == EPI_SCATTER ? kScatterEpiWarps * gg::kEpiStageBytes : epi_warps<EPI>() * kXBytes;
+}
+
+__device__ __forceinline__ uint32_t x_slot(int i, int j) { return (uint32_t)(i * 64 + ((j ^ ((i >> 1) & 3)) << 4)); }
+
+// Column-wise -> row-wise: w[t] is word (lane & 3) of row 8 t + lane / 4;
+// out[j] becomes word j of row `lane`.
+__device__ __forceinline__ void x_to_rows(uint8_t *buf, const uint4 (&w)[4], uint4 (&out)[4]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+        *reinterpret_cast<uint4 *>(buf + x_slot(8 * t + (lane >> 2), lane & 3)) = w[t];
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[j] = *reinterpret_cast<const uint4 *>(buf + x_slot(lane, j));
+    __syncwarp();
+}
+
+// Row-wise -> global: in[j] is word j of row `lane`; row i = 8 t + lane / 4
+// goes to base + (row0 + i) * ld (bytes) when i < nrows, word j = lane & 3
+// only when j < nwords.
+__device__ __forceinline__ void x_store_rows(uint8_t *buf, const uint4 (&in)[4], uint8_t *base, int64_t row0,
+                                             int64_t ld, int nrows, int nwords) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4 *>(buf + x_slot(lane, j)) = in[j];
+    __syncwarp();
+    const int j = lane & 3;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int i = 8 * t + (lane >> 2);
+        const uint4 w = *reinterpret_cast<const uint4 *>(buf + x_slot(i, j));
+        if (i < nrows && j < nwords) *reinterpret_cast<uint4 *>(base + (row0 + i) * ld + 16 * j) = w;
+    }
+    __syncwarp();
+}
+
+// ROWS / SWIGLU: the kept pre-activations u | v of 32 columns from col0 for
+// the warp's 32 grouped rows r0 .. r0 + 31 (the first nrows valid), read
+// column-wise: u[t] / v[t] hold word (lane & 3) of row 8 t + lane / 4.
 struct UV {
     uint4 u[4], v[4];
 };
-__device__ __forceinline__ void load_uv(const Params &p, int64_t r, int col0, bool ok, UV &b) {
-    if (!ok) return;
-    const __nv_bfloat16 *row = p.hpre + r * 2 * (int64_t)p.N;
+__device__ __forceinline__ void load_uv(const Params &p, int64_t r0, int nrows, int col0, UV &b) {
+    const int lane = threadIdx.x & 31;
+    const int col = col0 + 8 * (lane & 3);
+    if (col >= p.N) return;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int col = col0 + 8 * q;
-        if (col < p.N) {
-            b.u[q] = __ldg(reinterpret_cast<const uint4 *>(row + col));
-            b.v[q] = __ldg(reinterpret_cast<const uint4 *>(row + p.N + col));
+    for (int t = 0; t < 4; ++t) {
+        const int i = 8 * t + (lane >> 2);
+        if (i < nrows) {
+            const __nv_bfloat16 *row = p.hpre + (r0 + i) * 2 * (int64_t)p.N;
+            b.u[t] = __ldg(reinterpret_cast<const uint4 *>(row + col));
+            b.v[t] = __ldg(reinterpret_cast<const uint4 *>(row + p.N + col));
         }
     }
 }
 
-// ROWS / SWIGLU epilogue of grouped row r of column tile nt (gidx: its
-// assignment, or token for the dense expert; -1 if the row is not valid; g:
-// its gate); D = r_i from TMEM.  The outputs go to row ro (r in the padded
-// layout).  buf[0] holds the first 32 columns' u | v already (loaded before
-// the accumulator was ready); each later chunk's loads are issued before the
-// TMEM wait of the chunk before it, so one L2 round trip is in flight while
-// a chunk is computed.  With two warps per row each adds its partial dot
-// product into the row's gate gradient.
-// This warp drains NC columns from column c0 of the tile (tbase points at
-// column c0).
+// ROWS / SWIGLU epilogue of column tile nt for the warp's grouped rows r0 ..
+// r0 + 31 (the first nrows valid; this thread's row is r0 + lane, gidx its
+// assignment, or token for the dense expert, -1 if not valid; g its gate);
+// D = r_i from TMEM.  The outputs go to rows ro0 .. (r in the padded
+// layout).  buf holds the first 32 columns' u | v already (loaded before the
+// accumulator was ready); once a chunk's u | v are in registers row-wise, the
+// next chunk's loads are issued into buf, so one L2 round trip is in flight
+// while a chunk is computed and stored.  With two warps per row each adds its
+// partial dot product into the row's gate gradient.  This warp drains NC
+// columns from column c0 of the tile (tbase points at column c0); xb is its
+// exchange buffer.
 template <int NC>
-__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int c0, int64_t r, int64_t ro, int64_t gidx,
-                                                float g, uint32_t tbase, UV (&buf)[2]) {
+__device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int c0, int64_t r0, int64_t ro0, int nrows,
+                                                int64_t gidx, float g, uint32_t tbase, UV &buf, uint8_t *xb) {
     const int N = p.N;
     float dot = 0.f;
-    // two chunks per iteration, so the buffers are named statically while the
-    // loop body stays small enough for the instruction cache
 #pragma unroll 1
-    for (int c2 = 0; c2 < NC / 64; ++c2)
-#pragma unroll
-    for (int hc = 0; hc < 2; ++hc) {
-        const int ci = 2 * c2 + hc;
+    for (int ci = 0; ci < NC / 32; ++ci) {
+        const int col0 = nt * BN + c0 + 32 * ci;
+        uint4 ur[4], vr[4];
+        x_to_rows(xb, buf.u, ur);
+        x_to_rows(xb, buf.v, vr);
         float v[2][16];
         tmem_ld16(tbase + 32 * ci, v[0]);
         tmem_ld16(tbase + 32 * ci + 16, v[1]);
-        if (ci + 1 < NC / 32) load_uv(p, r, nt * BN + c0 + 32 * (ci + 1), gidx >= 0, buf[hc ^ 1]);
+        if (ci + 1 < NC / 32) {
+            int64_t r = r0;
+            asm volatile("" : "+l"(r));
+            load_uv(p, r, nrows, col0 + 32, buf);
+        }
         tmem_wait_ld();
-        if (gidx < 0) continue;
-        const UV &b = buf[hc];
+        uint4 dur[4], dvr[4], gar[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int col = nt * BN + c0 + 32 * ci + 8 * q;
-            if (col >= N) continue;
-            const __nv_bfloat162 *u2 = reinterpret_cast<const __nv_bfloat162 *>(&b.u[q]);
-            const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&b.v[q]);
-            uint32_t du2[4], dv2[4], ga2[4];
+            const __nv_bfloat162 *u2 = reinterpret_cast<const __nv_bfloat162 *>(&ur[q]);
+            const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&vr[q]);
+            uint32_t *du2 = reinterpret_cast<uint32_t *>(&dur[q]), *dv2 = reinterpret_cast<uint32_t *>(&dvr[q]),
+                     *ga2 = reinterpret_cast<uint32_t *>(&gar[q]);
+            const bool in = col0 + 8 * q < N;
 #pragma unroll
             for (int z2 = 0; z2 < 4; ++z2) {
                 const float2 uf = __bfloat1622float2(u2[z2]);
@@ -208,10 +267,10 @@ __device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int c0,
                 for (int z = 0; z < 2; ++z) {
                     const int i = 8 * q + 2 * z2 + z;   // column within the 32-column chunk
                     const float rv = v[i >> 4][i & 15];
-                    const float sg = 1.f / (1.f + __expf(-uu[z]));
+                    const float sg = __fdividef(1.f, 1.f + __expf(-uu[z]));   // sigmoid(u), as the forward
                     const float su = uu[z] * sg;   // silu(u)
                     const float a = su * ww[z];
-                    dot = fmaf(rv, a, dot);
+                    if (in) dot = fmaf(rv, a, dot);
                     const float da = g * rv;
                     du[z] = da * ww[z] * sg * (1.f + uu[z] * (1.f - sg));
                     dv[z] = da * su;
@@ -225,26 +284,34 @@ __device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int c0,
                 bb = __floats2bfloat162_rn(ga[0], ga[1]);
                 ga2[z2] = *reinterpret_cast<uint32_t *>(&bb);
             }
-            *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + col) = make_uint4(du2[0], du2[1], du2[2], du2[3]);
-            *reinterpret_cast<uint4 *>(p.dh + ro * 2 * (int64_t)N + N + col) =
-                make_uint4(dv2[0], dv2[1], dv2[2], dv2[3]);
-            *reinterpret_cast<uint4 *>(p.ga + ro * (int64_t)N + col) = make_uint4(ga2[0], ga2[1], ga2[2], ga2[3]);
         }
+        const int nw = min(4, (N - col0) / 8);
+        // the row addresses are worked out afresh for each chunk rather than
+        // held in registers across the loop
+        int64_t ro = ro0;
+        asm volatile("" : "+l"(ro));
+        uint8_t *dh = reinterpret_cast<uint8_t *>(p.dh + col0);
+        x_store_rows(xb, dur, dh, ro, 4 * (int64_t)N, nrows, nw);
+        x_store_rows(xb, dvr, dh + 2 * (int64_t)N, ro, 4 * (int64_t)N, nrows, nw);
+        x_store_rows(xb, gar, reinterpret_cast<uint8_t *>(p.ga + col0), ro, 2 * (int64_t)N, nrows, nw);
     }
     if (gidx >= 0) atomicAdd(p.dgate + gidx, dot);
 }
 
-// WGRAD / STORE: weight row m (of M, in half `half`) of group e, NC columns
-// from n0 (TMEM from tbase); zero when the group had no rows.
+// WGRAD / STORE: the warp's weight rows m0 .. m0 + 31 (of M, in half `half`)
+// of group e, NC columns from n0 (TMEM from tbase); zero when the group had
+// no rows.  xb: the warp's exchange buffer.
 template <int NC>
-__device__ __forceinline__ void epilogue_store(const Params &p, int e, int half, int m, int n0, bool has_rows,
-                                               uint32_t tbase) {
-    const bool valid = m < p.M;
-    if (!__any_sync(0xffffffffu, valid)) return;
-    const int64_t orow = (int64_t)e * p.M + m;
-    void *out = half ? p.out1 : p.out0;
+__device__ __forceinline__ void epilogue_store(const Params &p, int e, int half, int m0, int n0, bool has_rows,
+                                               uint32_t tbase, uint8_t *xb) {
+    const int nrows = min(32, p.M - m0);
+    if (nrows <= 0) return;
+    const int64_t orow0 = (int64_t)e * p.M + m0;
+    uint8_t *out = static_cast<uint8_t *>(half ? p.out1 : p.out0);
 #pragma unroll 1
     for (int c = 0; c < NC; c += 32) {
+        const int col0 = n0 + c;
+        if (col0 >= p.N) break;
         float v[2][16];
         if (has_rows) {
             tmem_ld16(tbase + c, v[0]);
@@ -254,29 +321,32 @@ __device__ __forceinline__ void epilogue_store(const Params &p, int e, int half,
 #pragma unroll
             for (int q = 0; q < 16; ++q) v[0][q] = v[1][q] = 0.f;
         }
-        if (!valid) continue;
+        if (p.out_f32) {
+            // two 16-column halves of 64 bytes per row
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < 2; ++h) {
+                uint4 w[4];
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-                const int col = n0 + c + 16 * h + 8 * h8;
-                if (col >= p.N) continue;
-                const float *s = &v[h][8 * h8];
-                if (p.out_f32) {
-                    float *d = static_cast<float *>(out) + orow * p.N + col;
-                    *reinterpret_cast<float4 *>(d) = make_float4(s[0], s[1], s[2], s[3]);
-                    *reinterpret_cast<float4 *>(d + 4) = make_float4(s[4], s[5], s[6], s[7]);
-                } else {
-                    uint32_t w[4];
+                for (int q = 0; q < 4; ++q)
+                    w[q] = make_uint4(__float_as_uint(v[h][4 * q]), __float_as_uint(v[h][4 * q + 1]),
+                                      __float_as_uint(v[h][4 * q + 2]), __float_as_uint(v[h][4 * q + 3]));
+                const int c16 = col0 + 16 * h;
+                if (c16 < p.N)
+                    x_store_rows(xb, w, out + 4 * (int64_t)c16, orow0, 4 * (int64_t)p.N, nrows, min(4, (p.N - c16) / 4));
+            }
+        } else {
+            uint4 w[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(s[2 * q], s[2 * q + 1]);
-                        w[q] = *reinterpret_cast<uint32_t *>(&b);
-                    }
-                    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + orow * p.N + col) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
+            for (int q = 0; q < 4; ++q) {
+                uint32_t *wq = reinterpret_cast<uint32_t *>(&w[q]);
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                    const int i = 8 * q + 2 * z;
+                    __nv_bfloat162 b = __floats2bfloat162_rn(v[i >> 4][i & 15], v[i >> 4][(i & 15) + 1]);
+                    wq[z] = *reinterpret_cast<uint32_t *>(&b);
                 }
             }
+            x_store_rows(xb, w, out + 2 * (int64_t)col0, orow0, 2 * (int64_t)p.N, nrows, min(4, (p.N - col0) / 8));
         }
     }
 }
@@ -316,7 +386,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     constexpr uint32_t kIdesc = idesc_bwd<MODE>();
     constexpr int kEpiWarps = epi_warps<EPI>(), kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
     constexpr int kCols = BN / (kEpiWarps / 4);   // columns one epilogue warp drains
-    constexpr int kEpiStage = EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0;
+    constexpr int kEpiStage = epi_stage_bytes<EPI>();
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -358,7 +428,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     __syncthreads();
     tc_fence_after();
     pdl_launch_dependents();
-    constexpr int kPtVar = MODE == WGRAD ? 2 : EPI;
+    [[maybe_unused]] constexpr int kPtVar = MODE == WGRAD ? 2 : EPI;
     PipeClock ck_total, ck_a, ck_b;
     ck_total.start();
 
@@ -507,17 +577,20 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                         g = p.gate[gidx];
                     }
                 }
-                UV buf[2];
-                load_uv(p, r, tl.n * BN + c0, gidx >= 0, buf[0]);
+                const int64_t r0 = r - lane;   // the warp's first row
+                const int64_t left = seg_end[tl.e] - r0;
+                const int nrows = left <= 0 ? 0 : (left >= 32 ? 32 : (int)left);
+                UV buf;
+                load_uv(p, r0, nrows, tl.n * BN + c0, buf);
                 ck_a.start();
                 const bool ready = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
                 ck_a.stop();
                 if (!ready) break;
                 tc_fence_after();
                 ck_b.start();
-                if (__any_sync(0xffffffffu, valid))
-                    epilogue_swiglu<kCols>(p, tl.n, c0, r, op_row0(tl.e) + local, gidx, g, tmem + acc * BN + lane_base,
-                                           buf);
+                if (nrows > 0)
+                    epilogue_swiglu<kCols>(p, tl.n, c0, r0, op_row0(tl.e) + local - lane, nrows, gidx, g,
+                                           tmem + acc * BN + lane_base, buf, sEpi + warp * kXBytes);
                 ck_b.stop();
                 tc_fence_before();
                 mbar_arrive(&ctrl->tempty[acc]);
@@ -543,7 +616,8 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                 }
             } else {
                 const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM + row, w.nt * BN + c0, seg_end[w.e] > seg_off[w.e], tb);
+                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM + row - lane, w.nt * BN + c0, seg_end[w.e] > seg_off[w.e], tb,
+                                      sEpi + warp * kXBytes);
             }
             ck_b.stop();
             tc_fence_before();
@@ -581,7 +655,10 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
 // full[s]; tcgen05.commit multicasts stage releases and accumulator-ready
 // signals to both; the epilogue warps of both release an accumulator on the
 // even CTA's tempty; cluster barriers after set-up and before exit.
-constexpr int kPStages = 6;
+#ifndef MOE_BWD_PSTAGES
+#define MOE_BWD_PSTAGES 6
+#endif
+constexpr int kPStages = MOE_BWD_PSTAGES;
 constexpr int kPStage = 128 * 128;   // 16 KB: this CTA's A (or B) of one K block
 
 struct Ctrl2 {
@@ -610,7 +687,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     constexpr uint32_t kIdesc = idesc_bwd2<MODE>();
     constexpr int kEpiWarps = epi_warps<EPI>(), kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
     constexpr int kCols = BN / (kEpiWarps / 4);   // columns one epilogue warp drains
-    constexpr int kEpiStage = EPI == EPI_SCATTER ? kEpiWarps * gg::kEpiStageBytes : 0;
+    constexpr int kEpiStage = epi_stage_bytes<EPI>();
     constexpr int BM2 = 256;
 
     extern __shared__ uint8_t smem_raw[];
@@ -657,6 +734,9 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     tc_fence_after();
     cluster_sync_all();   // both CTAs' barriers exist before any remote arrive
     pdl_launch_dependents();
+    [[maybe_unused]] constexpr int kPtVar = 4 + (MODE == WGRAD ? 2 : EPI);   // two-SM kernels: rows 4-6
+    PipeClock ck_total, ck_a, ck_b;
+    ck_total.start();
 
     const uint32_t tmem = ctrl->tmem_base;
     const int nE = p.g.offsets ? p.g.E : 1;
@@ -724,7 +804,10 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                 }
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kPStages;
-                    if (!wait_bar(&ctrl->empty[s], ((it / kPStages) & 1) ^ 1, abort, p.g.err)) {
+                    ck_a.start();
+                    const bool free_stage = wait_bar(&ctrl->empty[s], ((it / kPStages) & 1) ^ 1, abort, p.g.err);
+                    ck_a.stop();
+                    if (!free_stage) {
                         ok = false;
                         break;
                     }
@@ -741,6 +824,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                     }
                 }
             }
+            ck_a.flush(PIPE_SLOT(kPtVar, 3));
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0 && lead) {
@@ -748,7 +832,10 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
             bool ok = true;
             for (int id = pair; id < total && ok; id += npairs, ++tc) {
                 const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-                if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.g.err)) break;
+                ck_b.start();
+                const bool free_acc = wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.g.err);
+                ck_b.stop();
+                if (!free_acc) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + acc * BN;
                 const int nk = tile_nk(id);
@@ -756,9 +843,11 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                     const int s = it % kPStages;
                     const uint32_t ph = (it / kPStages) & 1;
                     // the operands of both CTAs have landed (acquire at cluster scope)
+                    ck_a.start();
                     bool got = mbar_try_wait_cluster(&ctrl->full[s], ph);
                     if (!got)
                         got = wait_bar(&ctrl->full[s], ph, abort, p.g.err) && mbar_try_wait_cluster(&ctrl->full[s], ph);
+                    ck_a.stop();
                     if (!got) {
                         ok = false;
                         break;
@@ -776,6 +865,8 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                 if (ok) mma_commit2(&ctrl->tfull[acc], 0x3);
             }
             mma_commit2(&ctrl->done, 0x3);
+            ck_a.flush(PIPE_SLOT(kPtVar, 1));
+            ck_b.flush(PIPE_SLOT(kPtVar, 2));
         }
     } else if (warp < kEpiWarps) {
         uint32_t tc = 0;
@@ -804,27 +895,43 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                             g = p.gate[gidx];
                         }
                     }
-                    UV buf[2];
-                    load_uv(p, r, tl.n * BN + c0, gidx >= 0, buf[0]);
+                    const int64_t r0 = r - lane;   // the warp's first row
+                    const int64_t left = seg_end[tl.e] - r0;
+                    const int nrows = left <= 0 ? 0 : (left >= 32 ? 32 : (int)left);
+                    UV buf;
+                    load_uv(p, r0, nrows, tl.n * BN + c0, buf);
+                    ck_a.start();
                     got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+                    ck_a.stop();
                     if (!got) break;
                     tc_fence_after();
-                    if (__any_sync(0xffffffffu, valid))
-                        epilogue_swiglu<kCols>(p, tl.n, c0, r, op_row0(tl.e) + local, gidx, g, tb, buf);
+                    ck_b.start();
+                    if (nrows > 0)
+                        epilogue_swiglu<kCols>(p, tl.n, c0, r0, op_row0(tl.e) + local - lane, nrows, gidx, g, tb, buf,
+                                               sEpi + warp * kXBytes);
+                    ck_b.stop();
                 } else {
+                    ck_a.start();
                     got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+                    ck_a.stop();
                     if (!got) break;
                     tc_fence_after();
+                    ck_b.start();
                     gg::epilogue_row<gg::DOWN, __nv_bfloat16, BN>(
                         p.g, tl.n, r, valid, tb, reinterpret_cast<float *>(sEpi + warp * gg::kEpiStageBytes));
+                    ck_b.stop();
                 }
             } else {
+                ck_a.start();
                 got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
+                ck_a.stop();
                 if (!got) break;
                 tc_fence_after();
                 const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM2 + half_off + row, w.nt * BN + c0, seg_end[w.e] > seg_off[w.e],
-                               tb);
+                ck_b.start();
+                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM2 + half_off + row - lane, w.nt * BN + c0,
+                                      seg_end[w.e] > seg_off[w.e], tb, sEpi + warp * kXBytes);
+                ck_b.stop();
             }
             tc_fence_before();
             __syncwarp();
@@ -832,6 +939,10 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                 if (lead) mbar_arrive(&ctrl->tempty[acc]);
                 else mbar_arrive_remote(tempty_lead + acc * (uint32_t)sizeof(uint64_t));
             }
+        }
+        if (threadIdx.x == 0) {
+            ck_a.flush(PIPE_SLOT(kPtVar, 4));
+            ck_b.flush(PIPE_SLOT(kPtVar, 5));
         }
     }
 
@@ -847,6 +958,13 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     cluster_sync_all();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc2(tmem, kTmemCols);
+    ck_total.stop();
+    if (threadIdx.x == 0) {
+        ck_total.flush(PIPE_SLOT(kPtVar, 0));
+#ifdef MOE_PIPE_TRACE
+        atomicAdd(&g_pipe_trace[kPtVar][6], 1ull);
+#endif
+    }
 }
 
 }  // namespace gb
@@ -934,7 +1052,7 @@ cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOper
     else max_tiles = (int64_t)nE * p.halves * ((p.M + BM - 1) / BM) * ntiles;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
     const size_t smem = 1024 + (size_t)kStages * (kAStage + kBStage) +
-                        (EPI == EPI_SCATTER ? kScatterEpiWarps * gg::kEpiStageBytes : 0) + sizeof(Ctrl) +
+                        epi_stage_bytes<EPI>() + sizeof(Ctrl) +
                         4 * sizeof(int) * (p.g.E + 1);
     auto kern = bwd_gemm_kernel<MODE, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -951,7 +1069,7 @@ cudaError_t launch_bwd_pair(const BwdOperand &a0, const BwdOperand &a1, const Bw
     // each CTA of the pair: 128 rows of A (ROWS), two 64-column atoms of each MN-major operand
     if (!bwd_maps<MODE>(a0, a1, b0, b1, MODE == ROWS ? 128 : 64, 2, 2, &mA0, &mA1, &mB0, &mB1, &q.mn3d))
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + (size_t)kPStages * 2 * kPStage + (EPI == EPI_SCATTER ? kScatterEpiWarps * gg::kEpiStageBytes : 0) +
+    const size_t smem = 1024 + (size_t)kPStages * 2 * kPStage + epi_stage_bytes<EPI>() +
                         sizeof(Ctrl2) + 4 * sizeof(int) * (p.g.E + 1);
     auto kern = bwd_gemm_pair_kernel<MODE, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1044,7 +1162,7 @@ extern "C" int moe_debug_pipe_trace(unsigned long long *out, int reset) {
     if (cudaDeviceSynchronize() != cudaSuccess) return 1;
     if (cudaMemcpyFromSymbol(out, moe::gb::g_pipe_trace, sizeof(moe::gb::g_pipe_trace)) != cudaSuccess) return 1;
     if (reset) {
-        static const unsigned long long zero[4][8] = {};
+        static const unsigned long long zero[8][8] = {};
         if (cudaMemcpyToSymbol(moe::gb::g_pipe_trace, zero, sizeof(zero)) != cudaSuccess) return 1;
     }
     return 0;
