@@ -33,7 +33,7 @@ namespace {
 // backward GEMMs (expert e's rows from row 64 * sum_{e' < e} ceil(count_e' /
 // 64), in grouped order), with the padding rows -- past each segment's end up
 // to the next multiple of 64 -- zeroed in x_g, dy_g, dH and ga.  CTA-strided
-// over 64-row blocks; 16-byte copies.
+// over (64-row block, 1024-column slice) units; 16-byte copies.
 struct GatherPadArgs {
     const __nv_bfloat16 *x, *dy;
     const int32_t *offsets, *sorted_rows;
@@ -59,13 +59,16 @@ __global__ void __launch_bounds__(256) gather_pad_kernel(GatherPadArgs a) {
     }
     __syncthreads();
     const int cpr = a.d / 8;                 // 16-byte chunks per x / dy row
+    const int S = (cpr + 127) / 128;         // column slices of 128 chunks
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
+    for (int u = blockIdx.x; u < nblk * S; u += gridDim.x) {
+        const int b = u / S, sl = u - b * S;
         const gg::Tile tl = gg::decode(b, 1, blk, a.E);
         const int64_t pr0 = (int64_t)b * 64;               // first padded row of the block
         const int64_t r0 = (int64_t)off[tl.e] + tl.m * 64;  // its first grouped row
         // x_g and dy_g: one warp per row (its token looked up once), each lane
-        // four 16-byte chunks of x and of dy in flight before it stores them
+        // four 16-byte chunks of the slice of x and of dy in flight before it
+        // stores them
         for (int q = warp; q < 64; q += 8) {
             const int64_t r = r0 + q;
             int64_t t = -1;
@@ -82,35 +85,35 @@ __global__ void __launch_bounds__(256) gather_pad_kernel(GatherPadArgs a) {
             uint4 *dyo = reinterpret_cast<uint4 *>(a.dyg + (pr0 + q) * a.d);
             const uint4 *xi = reinterpret_cast<const uint4 *>(a.x + (t < 0 ? 0 : t) * a.d);
             const uint4 *dyi = reinterpret_cast<const uint4 *>(a.dy + (t < 0 ? 0 : t) * a.d);
-            for (int c0 = lane; c0 < cpr; c0 += 4 * 32) {
-                uint4 vx[4], vd[4];
+            const int c0 = sl * 128 + lane;
+            uint4 vx[4], vd[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + 32 * u;
-                    vx[u] = vd[u] = make_uint4(0, 0, 0, 0);
-                    if (t >= 0 && c < cpr) {
-                        vx[u] = xi[c];
-                        vd[u] = dyi[c];
-                    }
+            for (int j = 0; j < 4; ++j) {
+                const int c = c0 + 32 * j;
+                vx[j] = vd[j] = make_uint4(0, 0, 0, 0);
+                if (t >= 0 && c < cpr) {
+                    vx[j] = xi[c];
+                    vd[j] = dyi[c];
                 }
+            }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + 32 * u;
-                    if (c < cpr) {
-                        __stcs(xo + c, vx[u]);
-                        __stcs(dyo + c, vd[u]);
-                    }
+            for (int j = 0; j < 4; ++j) {
+                const int c = c0 + 32 * j;
+                if (c < cpr) {
+                    __stcs(xo + c, vx[j]);
+                    __stcs(dyo + c, vd[j]);
                 }
             }
         }
-        // dH and ga: zero the padding rows (the SWIGLU epilogue writes the others)
+        // dH and ga: zero the padding rows (the SWIGLU epilogue writes the
+        // others), the block's share of them
         const int64_t rem = (int64_t)end[tl.e] - r0;
         const int64_t valid = rem < 64 ? rem : 64;
         const int hc = a.h / 8;
         for (int64_t q = valid; q < 64; ++q) {
             uint4 *dh = reinterpret_cast<uint4 *>(a.dh + (pr0 + q) * 2 * a.h);
             uint4 *ga = reinterpret_cast<uint4 *>(a.ga + (pr0 + q) * a.h);
-            for (int i = threadIdx.x; i < 3 * hc; i += blockDim.x) {
+            for (int i = sl * blockDim.x + threadIdx.x; i < 3 * hc; i += S * blockDim.x) {
                 if (i < 2 * hc) dh[i] = make_uint4(0, 0, 0, 0);
                 else ga[i - 2 * hc] = make_uint4(0, 0, 0, 0);
             }
@@ -327,7 +330,10 @@ extern "C" moe_status moe_backward(const moe_config *c, const void *x, const voi
         GatherPadArgs a{static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(dy), offsets, srt,
                         E, c->k, d, h, T, R, static_cast<__nv_bfloat16 *>(xg), static_cast<__nv_bfloat16 *>(dyg),
                         reinterpret_cast<__nv_bfloat16 *>(dh), static_cast<__nv_bfloat16 *>(ga), err};
-        const unsigned blocks = (unsigned)std::min<int64_t>((int64_t)(Rp / 64), 8LL * num_sms());
+        // one CTA per 64-row block and slice of 1024 columns, so that enough
+        // copies are in flight for HBM (at most 32 CTAs per SM, grid-strided)
+        const int64_t slices = ((int64_t)d / 8 + 127) / 128;
+        const unsigned blocks = (unsigned)std::min<int64_t>((int64_t)(Rp / 64) * slices, 32LL * num_sms());
         e = launch_kernel(gather_pad_kernel, std::max(1u, blocks), 256, 0, s, a);
     }
     // 1. routed: r = W_down^T dy over grouped rows
