@@ -197,23 +197,22 @@ __device__ __forceinline__ void x_store_rows(uint8_t *buf, const uint4 (&in)[4],
     __syncwarp();
 }
 
-// ROWS / SWIGLU: the kept pre-activations u | v of 32 columns from col0 for
-// the warp's 32 grouped rows r0 .. r0 + 31 (the first nrows valid), read
-// column-wise: u[t] / v[t] hold word (lane & 3) of row 8 t + lane / 4.
+// ROWS / SWIGLU: the kept pre-activations u | v of 32 columns from col0 of
+// this thread's grouped row r (the row's 16-byte words; not read when ok is
+// false).  In the pre-activation layout one word of the warp's 32 rows spans
+// at most two 512-byte runs.
 struct UV {
     uint4 u[4], v[4];
 };
-__device__ __forceinline__ void load_uv(const Params &p, int64_t r0, int nrows, int col0, UV &b) {
-    const int lane = threadIdx.x & 31;
-    const int col = col0 + 8 * (lane & 3);
-    if (col >= p.N) return;
+__device__ __forceinline__ void load_uv(const Params &p, int64_t r, bool ok, int col0, UV &b) {
+    if (!ok) return;
+    const uint8_t *hp = reinterpret_cast<const uint8_t *>(p.hpre);
+    const int words = p.N / 4, j0 = col0 / 8;
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int i = 8 * t + (lane >> 2);
-        if (i < nrows) {
-            const __nv_bfloat16 *row = p.hpre + (r0 + i) * 2 * (int64_t)p.N;
-            b.u[t] = __ldg(reinterpret_cast<const uint4 *>(row + col));
-            b.v[t] = __ldg(reinterpret_cast<const uint4 *>(row + p.N + col));
+    for (int q = 0; q < 4; ++q) {
+        if (col0 + 8 * q < p.N) {
+            b.u[q] = __ldg(reinterpret_cast<const uint4 *>(hp + hpre_offset(r, j0 + q, words)));
+            b.v[q] = __ldg(reinterpret_cast<const uint4 *>(hp + hpre_offset(r, p.N / 8 + j0 + q, words)));
         }
     }
 }
@@ -223,32 +222,25 @@ __device__ __forceinline__ void load_uv(const Params &p, int64_t r0, int nrows, 
 // assignment, or token for the dense expert, -1 if not valid; g its gate);
 // D = r_i from TMEM.  The outputs go to rows ro0 .. (r in the padded
 // layout).  buf holds the first 32 columns' u | v already (loaded before the
-// accumulator was ready); once a chunk's u | v are in registers row-wise, the
-// next chunk's loads are issued into buf, so one L2 round trip is in flight
-// while a chunk is computed and stored.  With two warps per row each adds its
-// partial dot product into the row's gate gradient.  This warp drains NC
-// columns from column c0 of the tile (tbase points at column c0); xb is its
-// exchange buffer.
+// accumulator was ready); once a chunk's outputs are computed the next
+// chunk's loads are issued into buf, so they are in flight while the chunk is
+// stored.  With two warps per row each adds its partial dot product into the
+// row's gate gradient.  This warp drains NC columns from column c0 of the
+// tile (tbase points at column c0); xb is its exchange buffer.
 template <int NC>
 __device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int c0, int64_t r0, int64_t ro0, int nrows,
                                                 int64_t gidx, float g, uint32_t tbase, UV &buf, uint8_t *xb) {
     const int N = p.N;
+    const int lane = threadIdx.x & 31;
     float dot = 0.f;
 #pragma unroll 1
     for (int ci = 0; ci < NC / 32; ++ci) {
         const int col0 = nt * BN + c0 + 32 * ci;
-        uint4 ur[4], vr[4];
-        x_to_rows(xb, buf.u, ur);
-        x_to_rows(xb, buf.v, vr);
         float v[2][16];
         tmem_ld16(tbase + 32 * ci, v[0]);
         tmem_ld16(tbase + 32 * ci + 16, v[1]);
-        if (ci + 1 < NC / 32) {
-            int64_t r = r0;
-            asm volatile("" : "+l"(r));
-            load_uv(p, r, nrows, col0 + 32, buf);
-        }
         tmem_wait_ld();
+        const uint4 *ur = buf.u, *vr = buf.v;
         uint4 dur[4], dvr[4], gar[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -284,6 +276,11 @@ __device__ __forceinline__ void epilogue_swiglu(const Params &p, int nt, int c0,
                 bb = __floats2bfloat162_rn(ga[0], ga[1]);
                 ga2[z2] = *reinterpret_cast<uint32_t *>(&bb);
             }
+        }
+        if (ci + 1 < NC / 32) {
+            int64_t r = r0;
+            asm volatile("" : "+l"(r));
+            load_uv(p, r + lane, lane < nrows, col0 + 32, buf);
         }
         const int nw = min(4, (N - col0) / 8);
         // the row addresses are worked out afresh for each chunk rather than
@@ -581,7 +578,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                 const int64_t left = seg_end[tl.e] - r0;
                 const int nrows = left <= 0 ? 0 : (left >= 32 ? 32 : (int)left);
                 UV buf;
-                load_uv(p, r0, nrows, tl.n * BN + c0, buf);
+                load_uv(p, r, lane < nrows, tl.n * BN + c0, buf);
                 ck_a.start();
                 const bool ready = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
                 ck_a.stop();
@@ -899,7 +896,7 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                     const int64_t left = seg_end[tl.e] - r0;
                     const int nrows = left <= 0 ? 0 : (left >= 32 ? 32 : (int)left);
                     UV buf;
-                    load_uv(p, r0, nrows, tl.n * BN + c0, buf);
+                    load_uv(p, r, lane < nrows, tl.n * BN + c0, buf);
                     ck_a.start();
                     got = wait_bar(&ctrl->tfull[acc], aph, abort, p.g.err);
                     ck_a.stop();

@@ -46,7 +46,8 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
             T *dst = act + r * p.N + col;
             if constexpr (sizeof(T) == 2) {
                 if (p.hpre) {
-                    T *hg = static_cast<T *>(p.hpre) + r * 2 * (int64_t)p.N + col;
+                    uint8_t *hp = static_cast<uint8_t *>(p.hpre);
+                    const int words = p.N / 4, j0 = col / 8;
 #pragma unroll
                     for (int h8 = 0; h8 < 2; ++h8) {
                         if (col + 8 * h8 >= p.N) continue;
@@ -59,8 +60,10 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
                             wg[q] = *reinterpret_cast<uint32_t *>(&a2);
                             wu[q] = *reinterpret_cast<uint32_t *>(&b2);
                         }
-                        *reinterpret_cast<uint4 *>(hg + 8 * h8) = make_uint4(wg[0], wg[1], wg[2], wg[3]);
-                        *reinterpret_cast<uint4 *>(hg + p.N + 8 * h8) = make_uint4(wu[0], wu[1], wu[2], wu[3]);
+                        *reinterpret_cast<uint4 *>(hp + hpre_offset(r, j0 + h8, words)) =
+                            make_uint4(wg[0], wg[1], wg[2], wg[3]);
+                        *reinterpret_cast<uint4 *>(hp + hpre_offset(r, p.N / 8 + j0 + h8, words)) =
+                            make_uint4(wu[0], wu[1], wu[2], wu[3]);
                     }
                 }
             }

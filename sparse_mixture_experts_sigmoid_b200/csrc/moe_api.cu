@@ -74,8 +74,8 @@ Layout make_layout(const moe_config &c, bool train = false) {
         // kept for the backward pass, and the backward's scratch (the dx accumulator reuses y_acc)
         const size_t hs = (size_t)c.h_shared;
         L.size[P_PROBS] = (size_t)c.T * c.E * 4;
-        L.size[P_HPRE] = R * 2 * (size_t)c.h * esz;
-        L.size[P_HPRES] = (size_t)c.T * 2 * hs * esz;
+        L.size[P_HPRE] = (size_t)hpre_rows((int64_t)R) * 2 * (size_t)c.h * esz;
+        L.size[P_HPRES] = (size_t)hpre_rows(c.T) * 2 * hs * esz;
         const size_t Rp = (size_t)padded_rows((int64_t)R, c.E);
         L.size[P_DG] = R * 4;
         L.size[P_DSG] = hs ? (size_t)c.T * 4 : 0;

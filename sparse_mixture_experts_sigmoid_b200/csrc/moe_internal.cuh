@@ -62,6 +62,19 @@ __device__ __forceinline__ void load8_stream(const float *p, float (&v)[8]) {
 // result flushes to zero, which is silu's limit there.
 __device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
+// Layout of the pre-activations a training forward keeps for the backward:
+// rows (grouped rows, or tokens for the shared expert) of `words` 16-byte
+// words (8 bf16 columns each: the gate columns, then the up columns), in
+// blocks of 32 rows; inside a block, word j of its 32 rows is 512 contiguous
+// bytes.  An epilogue warp holds 32 consecutive rows, one per thread, so each
+// of its 16-byte stores (forward) and loads (backward) of one word covers
+// whole lines.  Byte offset of word j of row r; the buffer holds rows rounded
+// up to a multiple of 32.
+__device__ __forceinline__ int64_t hpre_offset(int64_t r, int j, int words) {
+    return (((r >> 5) * words + j) << 9) + ((r & 31) << 4);
+}
+inline int64_t hpre_rows(int64_t rows) { return (rows + 31) / 32 * 32; }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -222,8 +235,8 @@ struct GemmParams {
     // stream has completed (see pdl_wait).  Set only where every kernel between
     // the producer of that data and this one is known.
     int early;
-    void *hpre;                  // gate/up only, optional: [rows, 2N] pre-activations (gate | up) kept
-                                 // for the backward pass
+    void *hpre;                  // gate/up only, optional: the pre-activations (gate | up, 2N
+                                 // columns) kept for the backward pass, in the hpre_offset layout
     float *slot_out;             // down only, optional: [R, N] fp32 rows by assignment (routed) or
                                  // token (dense), stored instead of added into y_acc
     int n_groups;                // column tiles run in this many consecutive groups (decode_n); 0, 1: one
@@ -270,7 +283,7 @@ struct BwdGemm {
     int groups, k;
     int64_t rows, T;
     int nranges, Kr, N, M, halves;
-    const void *hpre;             // SWIGLU: [rows, 2N] pre-activations (u | v)
+    const void *hpre;             // SWIGLU: pre-activations (u | v, 2N columns), hpre_offset layout
     const float *gate;            // SWIGLU: routed [R] by assignment / dense [T]
     void *dh, *ga;                // SWIGLU out: [rows, 2N] du | dv, [rows, N] gate * a
     float *dgate;                 // SWIGLU: accumulated gate gradients
