@@ -145,56 +145,14 @@ struct Params {
 
 // ------------------------------------------------------------------ epilogues
 
-// Row exchange through shared memory.  An epilogue thread owns one row of
-// the accumulator (TMEM lane = row), so a thread-per-row global access makes
-// each warp instruction touch 32 rows, 16 bytes each.  Instead every warp
-// moves 64-byte pieces of its 32 rows through 2 KB of its own shared memory:
-// global memory is read and written as 8 rows x 64 contiguous bytes per
-// instruction (4 threads per row), and the row-wise side stays in registers.
-// The 16-byte word j of row i sits at i * 64 + 16 * (j ^ ((i >> 1) & 3)), so
-// both the row-wise and the column-wise shared accesses are free of bank
-// conflicts (each group of 8 threads covers all 32 banks once).
-constexpr int kXBytes = 32 * 64;   // one warp's exchange buffer
+using gg::kXBytes;
+using gg::x_store_rows;
 
 // Shared memory of the epilogue warps: the scatter's row staging, else the
 // exchange buffers (16 KB either way).
 template <int EPI>
 constexpr int epi_stage_bytes() {
     return EPI == EPI_SCATTER ? kScatterEpiWarps * gg::kEpiStageBytes : epi_warps<EPI>() * kXBytes;
-}
-
-__device__ __forceinline__ uint32_t x_slot(int i, int j) { return (uint32_t)(i * 64 + ((j ^ ((i >> 1) & 3)) << 4)); }
-
-// Column-wise -> row-wise: w[t] is word (lane & 3) of row 8 t + lane / 4;
-// out[j] becomes word j of row `lane`.
-__device__ __forceinline__ void x_to_rows(uint8_t *buf, const uint4 (&w)[4], uint4 (&out)[4]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-        *reinterpret_cast<uint4 *>(buf + x_slot(8 * t + (lane >> 2), lane & 3)) = w[t];
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < 4; ++j) out[j] = *reinterpret_cast<const uint4 *>(buf + x_slot(lane, j));
-    __syncwarp();
-}
-
-// Row-wise -> global: in[j] is word j of row `lane`; row i = 8 t + lane / 4
-// goes to base + (row0 + i) * ld (bytes) when i < nrows, word j = lane & 3
-// only when j < nwords.
-__device__ __forceinline__ void x_store_rows(uint8_t *buf, const uint4 (&in)[4], uint8_t *base, int64_t row0,
-                                             int64_t ld, int nrows, int nwords) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4 *>(buf + x_slot(lane, j)) = in[j];
-    __syncwarp();
-    const int j = lane & 3;
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int i = 8 * t + (lane >> 2);
-        const uint4 w = *reinterpret_cast<const uint4 *>(buf + x_slot(i, j));
-        if (i < nrows && j < nwords) *reinterpret_cast<uint4 *>(base + (row0 + i) * ld + 16 * j) = w;
-    }
-    __syncwarp();
 }
 
 // ROWS / SWIGLU: the kept pre-activations u | v of 32 columns from col0 of

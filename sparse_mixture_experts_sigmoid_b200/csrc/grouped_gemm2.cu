@@ -71,6 +71,20 @@ struct Ctrl2 {
 // in a tile's last ring of K blocks the MMAs of half 0 run first and half 0
 // goes to the epilogue while half 1 finishes, and in the next tile's first
 // ring of K blocks half 0 is started while the epilogue still drains half 1.
+// Pipeline trace of this kernel in a diagnostic build (-DMOE_PIPE_TRACE; read
+// with moe_debug_fwd2_trace): per variant (gathered gate/up, contiguous
+// gate/up, down), SM cycles summed over CTAs for [0] the whole kernel, [1] the
+// MMA issuer waiting for operands, [2] it waiting for an accumulator, [3] the
+// TMA producers waiting for a free stage, [4] epilogue warp 0 waiting for an
+// accumulator, [5] it draining one, [6] the number of CTAs, [7] the first
+// gather thread waiting for a free stage.
+#ifdef MOE_PIPE_TRACE
+__device__ unsigned long long g_fwd2_trace[4][8];
+#define FWD2_SLOT(var, slot) (&g_fwd2_trace[var][slot])
+#else
+#define FWD2_SLOT(var, slot) nullptr
+#endif
+
 template <int MODE, bool GATHER, typename T, int BN, int W>
 __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -129,6 +143,9 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     tc_fence_after();
     cluster_sync_all();   // both CTAs' barriers exist before any remote arrive
     pdl_launch_dependents();
+    [[maybe_unused]] constexpr int kPtVar = MODE == GATEUP ? (GATHER ? 0 : 1) : 2;
+    PipeClock ck_total, ck_a, ck_b;
+    ck_total.start();
 
     const uint32_t tmem = ctrl->tmem_base;
     const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
@@ -157,7 +174,10 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                 const int b_row = tl.e * p.N + tl.n * BN_OUT + (MODE == GATEUP ? 0 : (int)rank * (BN / 2));
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
-                    if (!wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, p.err)) {
+                    ck_a.start();
+                    const bool free_stage = wait_bar(&ctrl->empty[s], ((it / kStages) & 1) ^ 1, abort, p.err);
+                    ck_a.stop();
+                    if (!free_stage) {
                         ok = false;
                         break;
                     }
@@ -178,6 +198,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                 }
             }
         }
+        if (lane == 0) ck_a.flush(FWD2_SLOT(kPtVar, 3));
     } else if (warp == kMmaWarp) {
         if (lane == 0 && lead) {
             uint32_t it = 0, tc = 0;
@@ -186,8 +207,10 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             auto wait_full = [&](uint32_t i) -> bool {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
+                ck_a.start();
                 bool got = mbar_try_wait_cluster(&ctrl->full[s], ph);
                 if (!got) got = wait_bar(&ctrl->full[s], ph, abort, p.err) && mbar_try_wait_cluster(&ctrl->full[s], ph);
+                ck_a.stop();
                 if (got) {
                     if constexpr (GATHER) fence_proxy_async();
                     tc_fence_after();
@@ -208,7 +231,10 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             for (int id = pair; id < total && ok; id += npairs, ++tc) {
                 if constexpr (W == 1) {
                     const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-                    if (!wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err)) break;
+                    ck_b.start();
+                    const bool free_acc = wait_bar(&ctrl->tempty[acc], aph ^ 1, abort, p.err);
+                    ck_b.stop();
+                    if (!free_acc) break;
                     tc_fence_after();
                     for (int kb = 0; kb < nk; ++kb, ++it) {
                         if (!wait_full(it)) {
@@ -225,7 +251,10 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                     const int Tb = nk - H < kStages ? nk - H : kStages;            // tail K blocks
                     // head: half 0 over the first ring once the epilogue has
                     // released it, then half 1 once that is released too
-                    if (!wait_bar(&ctrl->tempty[0], aph ^ 1, abort, p.err)) break;
+                    ck_b.start();
+                    const bool free_half0 = wait_bar(&ctrl->tempty[0], aph ^ 1, abort, p.err);
+                    ck_b.stop();
+                    if (!free_half0) break;
                     tc_fence_after();
                     for (int kb = 0; kb < H && ok; ++kb) {
                         if (wait_full(it + kb)) issue(it + kb, kb, 0, tmem);
@@ -233,7 +262,10 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                     }
                     if (!ok) break;
                     if (H == nk) mma_commit2(&ctrl->tfull[0], 0x3);
-                    if (!wait_bar(&ctrl->tempty[1], aph ^ 1, abort, p.err)) break;
+                    ck_b.start();
+                    const bool free_half1 = wait_bar(&ctrl->tempty[1], aph ^ 1, abort, p.err);
+                    ck_b.stop();
+                    if (!free_half1) break;
                     tc_fence_after();
                     for (int kb = 0; kb < H; ++kb) {
                         issue(it + kb, kb, 1, tmem);
@@ -270,6 +302,8 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                 }
             }
             mma_commit2(&ctrl->done, 0x3);
+            ck_a.flush(FWD2_SLOT(kPtVar, 1));
+            ck_b.flush(FWD2_SLOT(kPtVar, 2));
         } else if (lane == 0 && GATHER) {
             // odd CTA: relay its gathered rows of each K block to the even CTA
             uint32_t it = 0;
@@ -312,13 +346,18 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                 // W = 1: accumulator tc % 2; W = 2: half j of the one accumulator
                 const uint32_t b = W == 1 ? (tc & 1) : (uint32_t)j;
                 const uint32_t ph = W == 1 ? ((tc >> 1) & 1) : (tc & 1);
-                if (!wait_bar(&ctrl->tfull[b], ph, abort, p.err)) {
+                ck_a.start();
+                const bool ready = wait_bar(&ctrl->tfull[b], ph, abort, p.err);
+                ck_a.stop();
+                if (!ready) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                ck_b.start();
                 epilogue_row<MODE, T, BN>(p, tl.n * W + j, r, r < seg_end[tl.e], tmem + b * BN + lane_base,
                                           reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
+                ck_b.stop();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -327,10 +366,16 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                 }
             }
         }
+        if (threadIdx.x == 0) {
+            ck_a.flush(FWD2_SLOT(kPtVar, 4));
+            ck_b.flush(FWD2_SLOT(kPtVar, 5));
+        }
     } else if (GATHER && warp >= kGatherWarp0) {
+        PipeClock ck_g;
         gather_rows<T, kStages, BM2, kGatherThreads>(p, threadIdx.x - kGatherWarp0 * 32, pair, npairs, total, n_tiles, tile_start,
                                      seg_off, seg_end, nE, nk, row_off, sA, lead ? ctrl->full : ctrl->gfull,
-                                     ctrl->empty, abort);
+                                     ctrl->empty, abort, &ck_g);
+        if (threadIdx.x == kGatherWarp0 * 32) ck_g.flush(FWD2_SLOT(kPtVar, 7));
     }
 
     // every MMA of the pair has completed (its arrivals on this CTA's barriers
@@ -345,6 +390,13 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     cluster_sync_all();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc2(tmem, kTmemCols);
+    ck_total.stop();
+    if (threadIdx.x == 0) {
+        ck_total.flush(FWD2_SLOT(kPtVar, 0));
+#ifdef MOE_PIPE_TRACE
+        atomicAdd(&g_fwd2_trace[kPtVar][6], 1ull);
+#endif
+    }
 }
 
 }  // namespace
@@ -437,3 +489,17 @@ cudaError_t launch_grouped_gemm_pair(const GemmLaunch &L, cudaStream_t s) {
 }
 
 }  // namespace moe
+
+#ifdef MOE_PIPE_TRACE
+// Diagnostic build only: copies the two-SM forward pipeline trace (4 x 8
+// counters, see above) to host memory and optionally clears it.
+extern "C" int moe_debug_fwd2_trace(unsigned long long *out, int reset) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return 1;
+    if (cudaMemcpyFromSymbol(out, moe::gg::g_fwd2_trace, sizeof(moe::gg::g_fwd2_trace)) != cudaSuccess) return 1;
+    if (reset) {
+        static const unsigned long long zero[4][8] = {};
+        if (cudaMemcpyToSymbol(moe::gg::g_fwd2_trace, zero, sizeof(zero)) != cudaSuccess) return 1;
+    }
+    return 0;
+}
+#endif
