@@ -285,6 +285,35 @@ moe_status moe_forward(const moe_config *cfg, const moe_route_opts *opts, const 
                        const void *w_shared_gate, void *y, void *ws, size_t ws_bytes,
                        void *stream);
 
+/* moe_forward for inputs and outputs in host memory: x_host [T, d] is copied
+ * in and y_host [T, d] out by the call, in `chunks` pieces of at most
+ * ceil(T / chunks) tokens each.  Piece i's layer (moe_forward on its tokens,
+ * without routing options) runs on `stream` once its rows are on the device,
+ * and its y goes back on `copy_stream` while later pieces compute, so the
+ * copies overlap the layer; each token's result is that of moe_forward on
+ * its piece (the layer treats tokens independently; only the split of the
+ * router's reductions can differ with the token count).  All copies to the
+ * device are issued first.  More pieces hide more of the copies but re-read
+ * the expert weights once per piece.
+ *   x_host, y_host: page-locked host memory (pageable memory works, but its
+ *   copies do not overlap); weights as for moe_forward, on the device.
+ *   chunks >= 1 (more than T acts as T); copy_stream: a second stream, or NULL
+ *   to issue the copies on `stream` (no overlap).
+ *   ws: device workspace of at least moe_forward_host_workspace_size(cfg,
+ *   chunks) bytes, 256-byte aligned (the device copies of x and y, then the
+ *   layer's workspace for one piece).
+ * The call returns once everything is queued; when `stream` reaches the
+ * point of the call's end, y_host is complete (the copy stream's last copy
+ * is made a dependency of `stream`).  Events are created and destroyed by
+ * the call; no device memory is allocated.  Overlapping calls that share ws
+ * race on it. */
+moe_status moe_forward_host_workspace_size(const moe_config *cfg, int32_t chunks, size_t *bytes);
+moe_status moe_forward_host(const moe_config *cfg, const void *x_host, const void *w_router,
+                            const void *w_gate, const void *w_up, const void *w_down,
+                            const void *sh_gate, const void *sh_up, const void *sh_down,
+                            const void *w_shared_gate, void *y_host, int32_t chunks, void *ws,
+                            size_t ws_bytes, void *stream, void *copy_stream);
+
 /* ---- training: the forward pass that keeps what the backward needs, and the
  * backward pass.  bf16 layers only (MOE_F32 returns MOE_ERR_UNSUPPORTED).
  * The pages train this layer ("Small models, sparse experts", "Dispatch

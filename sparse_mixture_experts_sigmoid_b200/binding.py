@@ -25,7 +25,8 @@ EXPORTED = ["moe_status_string", "moe_validate", "moe_workspace_size", "moe_work
             "moe_device_status", "moe_profile_events", "moe_profile_nvtx", "moe_launch_count", "moe_combine_noalloc", "moe_permute_workspace_size",
             "moe_selftest_wait_timeout",
             "moe_route_workspace_size", "moe_update_bias", "moe_balance_loss", "moe_train_workspace_size",
-            "moe_forward_train", "moe_backward", "moe_quantize_q4", "moe_forward_q4"]
+            "moe_forward_train", "moe_backward", "moe_quantize_q4", "moe_forward_q4",
+            "moe_forward_host_workspace_size", "moe_forward_host"]
 STAGES = ["route", "permute", "gate_up", "shared_gate_up", "down", "shared_down", "finalize"]
 
 
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
             "moe_combine": ([C, P, P, P, P, P, P, P, S, P], ctypes.c_int),
             "moe_forward": ([C, ctypes.POINTER(RouteOpts), P, P, P, P, P, P, P, P, P, P, P, S, P],
                             ctypes.c_int),
+            "moe_forward_host_workspace_size": ([C, ctypes.c_int32, ctypes.POINTER(S)], ctypes.c_int),
+            "moe_forward_host": ([C] + [P] * 10 + [ctypes.c_int32, P, S, P, P], ctypes.c_int),
             "moe_update_bias": ([C, P, ctypes.c_float, P, P], ctypes.c_int),
             "moe_train_workspace_size": ([C, ctypes.POINTER(S)], ctypes.c_int),
             "moe_forward_train": ([C, ctypes.POINTER(RouteOpts), P, P, P, P, P, P, P, P, P, P, P, S, P],
@@ -331,6 +334,47 @@ def forward_layer(cfg: MoEConfig, layer, y=None, ws=None, stream=None, balance_b
     return forward(cfg, layer.x, layer.w_router, layer.w_gate, layer.w_up, layer.w_down, layer.sh_gate,
                    layer.sh_up, layer.sh_down, layer.w_shared_gate, y=y, ws=ws, stream=stream,
                    balance_bias=balance_bias, score_mean=score_mean)
+
+
+def _host_ptr(t: torch.Tensor, name: str, shape, dtype):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {dtype} of shape {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def forward_host_workspace_size(cfg: MoEConfig, chunks: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_forward_host_workspace_size(ctypes.byref(cfg), int(chunks), ctypes.byref(n)),
+           "moe_forward_host_workspace_size")
+    return n.value
+
+
+def forward_host(cfg: MoEConfig, layer, x_host, y_host, chunks: int, ws=None, stream=None, copy_stream=None):
+    """moe_forward_host: x_host [T,d] in and y_host [T,d] out in (pinned) host memory, the weights of
+    the synth.Layer-like `layer` on the device; `chunks` pieces whose copies overlap the other pieces'
+    layers (copy_stream: a torch.cuda.Stream, or None for no overlap).  Returns y_host."""
+    et = _elem_dtype(cfg)
+    if ws is None:
+        ws = torch.empty(max(forward_host_workspace_size(cfg, chunks), 1), dtype=torch.uint8, device="cuda")
+    hs = cfg.h_shared
+    cs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
+    _check(lib().moe_forward_host(ctypes.byref(cfg), _host_ptr(x_host, "x_host", (cfg.T, cfg.d), et),
+                                  _ptr(layer.w_router, "w_router", (cfg.E, cfg.d), et),
+                                  _ptr(layer.w_gate, "w_gate", (cfg.E, cfg.h, cfg.d), et),
+                                  _ptr(layer.w_up, "w_up", (cfg.E, cfg.h, cfg.d), et),
+                                  _ptr(layer.w_down, "w_down", (cfg.E, cfg.d, cfg.h), et),
+                                  _ptr(layer.sh_gate, "sh_gate", (hs, cfg.d), et),
+                                  _ptr(layer.sh_up, "sh_up", (hs, cfg.d), et),
+                                  _ptr(layer.sh_down, "sh_down", (cfg.d, hs), et),
+                                  _ptr(layer.w_shared_gate, "w_shared_gate", (cfg.d,), et),
+                                  _host_ptr(y_host, "y_host", (cfg.T, cfg.d), et), int(chunks),
+                                  _ptr(ws, "ws", dtype=torch.uint8), ws.numel(), _stream(stream), cs),
+           "moe_forward_host")
+    return y_host
 
 
 def update_bias(cfg: MoEConfig, counts, lr: float, bias, stream=None):

@@ -3,9 +3,11 @@
 // include/moe.h.
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdlib>
 #include <mutex>
+#include <vector>
 
 #include "moe_internal.cuh"
 
@@ -642,6 +644,104 @@ moe_status moe_forward(const moe_config *c, const moe_route_opts *opts, const vo
                        size_t ws_bytes, void *stream) {
     return forward_impl(c, opts, x, w_router, w_gate, w_up, w_down, sh_gate, sh_up, sh_down, w_shared_gate, y, ws,
                         ws_bytes, stream, false);
+}
+
+namespace {
+
+// Workspace of moe_forward_host: the device copies of x and y, then the
+// layer's workspace for one piece of at most ceil(T / chunks) tokens.
+struct HostLayout {
+    size_t x_off, y_off, ws_off, total;
+    int64_t piece;
+};
+moe_status host_layout(const moe_config &c, int32_t chunks, HostLayout *h) {
+    if (chunks <= 0) return MOE_ERR_INVALID_ARG;
+    const moe_status st = moe_validate(&c);
+    if (st != MOE_OK) return st;
+    const size_t esz = c.dtype == MOE_F32 ? 4 : 2;
+    const int64_t n = chunks > c.T ? c.T : chunks;
+    h->piece = n > 0 ? (c.T + n - 1) / n : 0;
+    moe_config pc = c;
+    pc.T = h->piece;
+    const size_t rows = (size_t)c.T * c.d * esz;
+    h->x_off = 0;
+    h->y_off = align256(rows);
+    h->ws_off = h->y_off + align256(rows);
+    h->total = h->ws_off + (pc.T > 0 ? make_layout(pc).total : 0);
+    return MOE_OK;
+}
+
+}  // namespace
+
+moe_status moe_forward_host_workspace_size(const moe_config *c, int32_t chunks, size_t *bytes) {
+    if (!c || !bytes) return MOE_ERR_INVALID_ARG;
+    HostLayout h;
+    const moe_status st = host_layout(*c, chunks, &h);
+    if (st == MOE_OK) *bytes = h.total;
+    return st;
+}
+
+moe_status moe_forward_host(const moe_config *c, const void *x_host, const void *w_router, const void *w_gate,
+                            const void *w_up, const void *w_down, const void *sh_gate, const void *sh_up,
+                            const void *sh_down, const void *w_shared_gate, void *y_host, int32_t chunks, void *ws,
+                            size_t ws_bytes, void *stream, void *copy_stream) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    HostLayout h;
+    moe_status st = host_layout(*c, chunks, &h);
+    if (st != MOE_OK) return st;
+    if (c->T == 0) return MOE_OK;
+    if (!x_host || !y_host || !w_router || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
+    if (c->h_shared > 0 && (!sh_gate || !sh_up || !sh_down || !w_shared_gate)) return MOE_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < h.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
+    const size_t row_bytes = (size_t)c->d * (c->dtype == MOE_F32 ? 4 : 2);
+    char *xd = static_cast<char *>(ws) + h.x_off;
+    char *yd = static_cast<char *>(ws) + h.y_off;
+    void *lws = static_cast<char *>(ws) + h.ws_off;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaStream_t cs = copy_stream ? static_cast<cudaStream_t>(copy_stream) : s;
+    const int64_t n = (c->T + h.piece - 1) / h.piece;   // pieces
+    // events order the two streams: start (earlier work on stream is done
+    // with the device copies), in[i] (piece i is on the device), out[i]
+    // (piece i's y is ready), done (the last copy back has landed)
+    std::vector<cudaEvent_t> ev((size_t)(2 * n + 2), nullptr);
+    cudaError_t e = cudaSuccess;
+    for (auto &v : ev)
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&v, cudaEventDisableTiming);
+    cudaEvent_t &start = ev[0], &done = ev[1];
+    auto ev_in = [&](int64_t i) { return ev[2 + i]; };
+    auto ev_out = [&](int64_t i) { return ev[2 + n + i]; };
+    if (e == cudaSuccess && cs != s) e = cudaEventRecord(start, s);
+    if (e == cudaSuccess && cs != s) e = cudaStreamWaitEvent(cs, start, 0);
+    // every piece's rows in first (one copy each), so that no copy to the
+    // device waits behind a copy back on the copy stream
+    for (int64_t i = 0; i < n && e == cudaSuccess; ++i) {
+        const int64_t t0 = i * h.piece, rows = std::min<int64_t>(h.piece, c->T - t0);
+        e = cudaMemcpyAsync(xd + t0 * row_bytes, static_cast<const char *>(x_host) + t0 * row_bytes,
+                            (size_t)rows * row_bytes, cudaMemcpyHostToDevice, cs);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in(i), cs);
+    }
+    for (int64_t i = 0; i < n && e == cudaSuccess && st == MOE_OK; ++i) {
+        const int64_t t0 = i * h.piece, rows = std::min<int64_t>(h.piece, c->T - t0);
+        moe_config pc = *c;
+        pc.T = rows;
+        e = cudaStreamWaitEvent(s, ev_in(i), 0);
+        if (e != cudaSuccess) break;
+        st = forward_impl(&pc, nullptr, xd + t0 * row_bytes, w_router, w_gate, w_up, w_down, sh_gate, sh_up,
+                          sh_down, w_shared_gate, yd + t0 * row_bytes, lws, ws_bytes - h.ws_off, stream, false);
+        if (st != MOE_OK) break;
+        e = cudaEventRecord(ev_out(i), s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev_out(i), 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(static_cast<char *>(y_host) + t0 * row_bytes, yd + t0 * row_bytes,
+                                (size_t)rows * row_bytes, cudaMemcpyDeviceToHost, cs);
+    }
+    // the caller waits on `stream` alone
+    if (e == cudaSuccess && st == MOE_OK && cs != s) e = cudaEventRecord(done, cs);
+    if (e == cudaSuccess && st == MOE_OK && cs != s) e = cudaStreamWaitEvent(s, done, 0);
+    for (auto &v : ev)
+        if (v) cudaEventDestroy(v);   // released once the recorded work completes
+    if (st != MOE_OK) return st;
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_forward_train(const moe_config *c, const moe_route_opts *opts, const void *x, const void *w_router,

@@ -196,3 +196,33 @@ def test_profile_nvtx_is_host_only():
     """Turning the NVTX stage ranges on and off needs no GPU and never fails."""
     assert B.lib().moe_profile_nvtx(1) == 0
     assert B.lib().moe_profile_nvtx(0) == 0
+
+
+def test_forward_host_workspace_and_argument_checks():
+    """moe_forward_host's workspace holds the device copies of x and y plus the
+    layer's workspace for one piece of ceil(T / chunks) tokens; chunks < 1 is
+    rejected and chunks > T acts as T; bad arguments are caught on the host."""
+    L = B.lib()
+    fake = ctypes.c_void_p(0x1000)
+    for name in ("tiny", "mixtral_prefill", "mixtral_decode"):
+        w = WORKLOADS[name]
+        cfg = B.config_of(w)
+        esz = 4 if w.dtype == "f32" else 2
+        rows = -(-w.T * w.d * esz // 256) * 256
+        for chunks in (1, 2, 3, 4, 8):
+            piece = -(-w.T // min(chunks, w.T))
+            layer = B.workspace_size(B.config_of(w, T=piece))
+            assert B.forward_host_workspace_size(cfg, chunks) == 2 * rows + layer
+        assert B.forward_host_workspace_size(cfg, w.T + 5) == B.forward_host_workspace_size(cfg, w.T)
+        n = ctypes.c_size_t(0)
+        assert L.moe_forward_host_workspace_size(ctypes.byref(cfg), 0, ctypes.byref(n)) == 1
+        assert L.moe_forward_host_workspace_size(ctypes.byref(cfg), -2, ctypes.byref(n)) == 1
+        args = [fake] * 9
+        # no x or y host buffer; no workspace; a misaligned workspace
+        assert L.moe_forward_host(ctypes.byref(cfg), None, *args[1:], fake, 2, fake, 1 << 40, None, None) == 1
+        assert L.moe_forward_host(ctypes.byref(cfg), *args, None, 2, fake, 1 << 40, None, None) == 1
+        assert L.moe_forward_host(ctypes.byref(cfg), *args, fake, 2, None, 1 << 40, None, None) == 3
+        assert L.moe_forward_host(ctypes.byref(cfg), *args, fake, 2, ctypes.c_void_p(0x1010), 1 << 40, None,
+                                  None) == 3
+        assert L.moe_forward_host(ctypes.byref(cfg), *args, fake, 2, fake, 16, None, None) == 3
+        assert L.moe_forward_host(ctypes.byref(cfg), *args, fake, 0, fake, 1 << 40, None, None) == 1
