@@ -37,11 +37,29 @@ constexpr int BM2 = 256;                  // grouped rows per pair tile
 constexpr int kHalfRows = 128;            // rows per CTA
 constexpr int kABytes = kHalfRows * 128;  // one A stage: 128 rows x 128 bytes
 constexpr int kMaxStages = 8;
-constexpr int kEpiWarps = 4;
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;               // MMA issuer in the even CTA, gather relay in the odd one
-constexpr int kGatherWarp0 = 6;
-constexpr int kGatherThreads = 256;
+// Warp roles: epilogue warps 0 .. EW-1, then the TMA producer, the MMA issuer
+// (the gather relay in the odd CTA) and the gather warps.  Gate/up drains a
+// half accumulator while the MMAs of its tile's other half, or of the next
+// tile's first K blocks, run: with eight epilogue warps (two per TMEM lane
+// quarter, each half of the columns) the drain is short enough that the MMA
+// issuer rarely waits for it.
+#ifndef MOE_GG2_GATEUP_EPI_WARPS
+#define MOE_GG2_GATEUP_EPI_WARPS 8
+#endif
+#ifndef MOE_GG2_GATHER_THREADS
+#define MOE_GG2_GATHER_THREADS 128
+#endif
+constexpr int kGatherThreads = MOE_GG2_GATHER_THREADS;
+static_assert(kGatherThreads == 128 || kGatherThreads == 256, "8 threads per row, 128 rows in whole passes");
+template <int MODE>
+constexpr int epi_warps() {
+    return MODE == GATEUP ? MOE_GG2_GATEUP_EPI_WARPS : 4;
+}
+static_assert(MOE_GG2_GATEUP_EPI_WARPS == 4 || MOE_GG2_GATEUP_EPI_WARPS == 8, "one or two warps per lane quarter");
+template <int MODE, bool GATHER>
+constexpr int pair_threads() {
+    return (epi_warps<MODE>() + 2) * 32 + (GATHER ? kGatherThreads : 0);
+}
 constexpr int kTmemCols = 512;
 
 // Ring depth for an MMA N of BN (each CTA holds BN / 2 rows of B per stage).
@@ -86,9 +104,11 @@ __device__ unsigned long long g_fwd2_trace[4][8];
 #endif
 
 template <int MODE, bool GATHER, typename T, int BN, int W>
-__global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
+__global__ void __launch_bounds__(pair_threads<MODE, GATHER>(), 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1, GemmParams p) {
+    constexpr int kEpiWarps = epi_warps<MODE>(), kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1,
+                  kGatherWarp0 = kEpiWarps + 2;
     constexpr int BK = 128 / (int)sizeof(T);
     static_assert(W == 1 || (W == 2 && MODE == GATEUP), "wide tiles are for gate/up");
     constexpr int BN_OUT = MODE == GATEUP ? W * BN / 2 : BN;   // output columns per tile
@@ -97,6 +117,7 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     constexpr int kBBytes = W * kBSub;               // this CTA's B per stage
     constexpr uint32_t kIdesc = instr_desc<T>(BM2, BN);
     constexpr int kStageBytes = MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0;
+    static_assert(MODE == GATEUP || kEpiWarps == 4, "the down epilogue stages 4 warps' rows");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -334,8 +355,11 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
             for (int64_t i = b + threadIdx.x; i < e; i += kEpiWarps * 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         uint32_t tc = 0;
-        const int row = warp * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int row = (warp & 3) * 32 + lane;   // TMEM lane quarter warp % 4
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        // this warp's part of the output columns of one accumulator (half)
+        constexpr int kParts = kEpiWarps / 4, kPartCols = (MODE == GATEUP ? BN / 2 : BN) / kParts;
+        const int c_lo = (warp >> 2) * kPartCols;
         const uint32_t tempty_lead = mapa_shared(&ctrl->tempty[0], 0);
         bool ok = true;
         for (int id = pair; id < total && ok; id += npairs, ++tc) {
@@ -356,7 +380,8 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
                 tc_fence_after();
                 ck_b.start();
                 epilogue_row<MODE, T, BN>(p, tl.n * W + j, r, r < seg_end[tl.e], tmem + b * BN + lane_base,
-                                          reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes));
+                                          reinterpret_cast<float *>(sEpi + warp * kEpiStageBytes), c_lo,
+                                          c_lo + kPartCols);
                 ck_b.stop();
                 tc_fence_before();
                 __syncwarp();
@@ -423,7 +448,7 @@ cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
     } else {
         mA = mB0;   // unused: gather mode reads x with cp.async
     }
-    const size_t smem = 1024 + (size_t)kStages * (kABytes + W * BN * 64) + (MODE == DOWN ? kEpiWarps * kEpiStageBytes : 0) +
+    const size_t smem = 1024 + (size_t)kStages * (kABytes + W * BN * 64) + (MODE == DOWN ? 4 * kEpiStageBytes : 0) +
                         sizeof(Ctrl2) + 3 * sizeof(int) * (p.E + 1);
     auto kern = grouped_gemm_pair_kernel<MODE, GATHER, T, BN, W>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -439,7 +464,7 @@ cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
         if (!max_pairs[dev]) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
-            cfg.blockDim = dim3(GATHER ? 192 + kGatherThreads : 192);
+            cfg.blockDim = dim3(pair_threads<MODE, GATHER>());
             cfg.dynamicSmemBytes = smem;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -457,7 +482,7 @@ cudaError_t launch_pair_t(const GemmLaunch &L, cudaStream_t s) {
     const int n_tiles = (p.N + BN_OUT - 1) / BN_OUT;
     const int64_t max_tiles = (p.rows / BM2 + nE) * (int64_t)n_tiles;
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs[dev], max_tiles));
-    return launch_kernel_pair(kern, 2 * pairs, GATHER ? 192 + kGatherThreads : 192, smem, s, mA, mB0, mB1, p);
+    return launch_kernel_pair(kern, 2 * pairs, pair_threads<MODE, GATHER>(), smem, s, mA, mB0, mB1, p);
 }
 
 template <int MODE, bool GATHER, typename T>

@@ -61,10 +61,12 @@ constexpr int kEpiStageBytes = 32 * 32 * 4;
 // BN/2 up columns and stores silu(g) * u into act; DOWN scales the BN
 // columns by the row's gate and adds them into y_acc with 16-byte reductions,
 // through the warp's 4 KB shared-memory staging block `stage`.  Several TMEM
-// loads are in flight per wait.  Called by all 32 lanes of an epilogue warp.
+// loads are in flight per wait.  Called by all 32 lanes of an epilogue warp;
+// GATEUP drains only output columns c_lo .. c_hi of the tile (two warps per
+// TMEM lane quarter split them).
 template <int MODE, typename T, int BN>
 __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t r, bool valid, uint32_t tbase,
-                                             float *stage) {
+                                             float *stage, int c_lo = 0, int c_hi = BN) {
     constexpr int BN_OUT = MODE == GATEUP ? BN / 2 : BN;
     if constexpr (MODE == GATEUP) {
         if (!__any_sync(0xffffffffu, valid)) return;   // no row of this warp lies in the segment
@@ -121,9 +123,10 @@ __device__ __forceinline__ void epilogue_row(const GemmParams &p, int n, int64_t
                 }
             }
         };
-        // 32 output columns per TMEM wait: four loads in flight at a time
+        // 32 output columns per TMEM wait: four loads in flight at a time;
+        // output columns c_lo .. c_hi of the tile (gate/up: of BN_OUT)
 #pragma unroll 1
-        for (int c = 0; c < BN_OUT; c += 32) {
+        for (int c = c_lo; c < min(BN_OUT, c_hi); c += 32) {
             float g[2][16], u[2][16];
             tmem_ld16(tbase + c, g[0]);
             tmem_ld16(tbase + c + 16, g[1]);
