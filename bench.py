@@ -201,6 +201,12 @@ def ncu_ms_for(stage: str, src: str, workload: str):
     return float(ent["us_per_launch"]) / 1e3 if ent and "us_per_launch" in ent else None
 
 
+def captured_kernel(stage: str, src: str, workload: str):
+    """The kernel (template instance) the capture saw for the stage, or None."""
+    ent = _capture(stage, src, workload)
+    return ent.get("kernel") if ent else None
+
+
 def kernel_of(stage: str, w, q4: bool):
     """(kernel name, source) of a stage for workload w."""
     kname, ksrc = STAGE_KERNEL[stage]
@@ -342,6 +348,7 @@ def time_workload(args, w, ws_n, rank, local, steps, warmup, headline, q4=False)
     dom = max((n for n in stage if n in work), key=lambda n: stage[n])
     kname, ksrc = kernel_of(dom, w, q4)
     cap_name = w.name + ("_q4" if q4 else "")
+    kname = captured_kernel(dom, ksrc, cap_name) or kname   # the instance the library picked, when captured
     dfr = roofline.fractions(work[dom]["flops"], work[dom]["bytes"], stage[dom] / 1e3, peaks, tpk)
     lw = roofline.layer_work(w, counts, q4=q4)
     lfr = roofline.fractions(lw["flops"], lw["bytes"], ms / 1e3, peaks, tpk)
