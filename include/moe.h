@@ -297,8 +297,8 @@ moe_status moe_forward(const moe_config *cfg, const moe_route_opts *opts, const 
  * the expert weights once per piece.
  *   x_host, y_host: page-locked host memory (pageable memory works, but its
  *   copies do not overlap); weights as for moe_forward, on the device.
- *   chunks >= 1 (more than T acts as T); copy_stream: a second stream, or NULL
- *   to issue the copies on `stream` (no overlap).
+ *   chunks >= 1 (more than T acts as T, more than 256 as 256); copy_stream: a
+ *   second stream, or NULL to issue the copies on `stream` (no overlap).
  *   ws: device workspace of at least moe_forward_host_workspace_size(cfg,
  *   chunks) bytes, 256-byte aligned (the device copies of x and y, then the
  *   layer's workspace for one piece).

@@ -648,6 +648,8 @@ moe_status moe_forward(const moe_config *c, const moe_route_opts *opts, const vo
 
 namespace {
 
+constexpr int64_t kMaxHostPieces = 256;   // moe_forward_host: events per call stay few
+
 // Workspace of moe_forward_host: the device copies of x and y, then the
 // layer's workspace for one piece of at most ceil(T / chunks) tokens.
 struct HostLayout {
@@ -659,7 +661,8 @@ moe_status host_layout(const moe_config &c, int32_t chunks, HostLayout *h) {
     const moe_status st = moe_validate(&c);
     if (st != MOE_OK) return st;
     const size_t esz = c.dtype == MOE_F32 ? 4 : 2;
-    const int64_t n = chunks > c.T ? c.T : chunks;
+    int64_t n = chunks > c.T ? c.T : chunks;
+    n = n > kMaxHostPieces ? kMaxHostPieces : n;
     h->piece = n > 0 ? (c.T + n - 1) / n : 0;
     moe_config pc = c;
     pc.T = h->piece;
