@@ -168,6 +168,18 @@ __global__ void __launch_bounds__(GATHER ? 192 + kGatherThreads : 192, 1)
     // complete already (weights, the layer input, offsets from further back)
     // is read before it, so the first weight tiles are in flight early.
     const bool early_tiles = (p.early & kEarlyTiles) != 0;
+    if (!early_tiles && (p.early & kEarlyPrefetch) && warp == kTmaWarp && lane == 0) {
+        // with one row tile per expert and every expert active, tile id is
+        // (expert id / n_tiles, column tile id % n_tiles)
+        const int nt = (p.N + BN_OUT - 1) / BN_OUT, e = blockIdx.x / nt;
+        if (e < p.E) {
+            const int b_row = e * p.N + (blockIdx.x - e * nt) * BN_OUT;
+            for (int kb = 0; kb < (p.K + BK - 1) / BK; ++kb) {
+                tma_prefetch_2d(&tmB0, kb * BK, b_row);
+                if (MODE == GATEUP) tma_prefetch_2d(&tmB1, kb * BK, b_row);
+            }
+        }
+    }
     if (!early_tiles) pdl_wait();
     if (warp == kTmaWarp) build_tiles<RB>(p, tile_start, seg_off, seg_end, &ctrl->n_mtiles);
     tc_fence_before();

@@ -252,6 +252,16 @@ bool use_gemm(const moe_config &c) { return c.T * c.k > kDecodeMaxRows; }
 // on the layers it targets (experts of about one 128-row tile) it measured
 // slower than the two grouped GEMMs (gemma_upcycle: 150 us against ~104 us),
 // so the two-kernel path is the default.
+// The speculative L2 prefetch of each CTA's first gate/up weight tile
+// (kEarlyPrefetch); MOE_PREFETCH=0 turns it off.
+bool prefetch_first_tiles() {
+    static const bool on = [] {
+        const char *v = std::getenv("MOE_PREFETCH");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
+
 bool use_fused(const moe_config &c) {
     static const bool on = [] {
         const char *v = std::getenv("MOE_FUSED");
@@ -584,6 +594,7 @@ moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const v
     } else if (e == cudaSuccess) {
         SegGateUpArgs ga{x, w_gate, w_up, routed, c->T, c->d, c->h, act};
         GemmLaunch gl = gemm_gateup(*c, x, w_gate, w_up, offsets, srt, act, err);
+        if (gl.p.stream_weights && prefetch_first_tiles()) gl.p.early |= kEarlyPrefetch;
         // the down GEMMs accumulate into it two kernels later (ordered: only the shared one)
         gl.p.zero = !ordered || shared ? acc : nullptr;
         gl.p.zero_floats = c->T * c->d;

@@ -244,6 +244,10 @@ struct GemmParams {
 enum : int {
     kEarlyTiles = 1,   // offsets (and hence the tile list) and the weights
     kEarlyA = 2,       // the contiguous A operand
+    // the weights of the tile each CTA would take first if every expert had
+    // one row tile, fetched into L2 while the grouping kernels still run (a
+    // wrong guess costs only the bandwidth)
+    kEarlyPrefetch = 4,
 };
 struct GemmLaunch {
     int mode;             // 0: gate/up with SwiGLU epilogue, 1: down with gate-weighted combine

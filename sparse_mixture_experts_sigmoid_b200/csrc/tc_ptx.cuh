@@ -76,6 +76,12 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *m, void *dst, uin
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
+// A 2D box fetched into L2 only (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *m, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1)
+                 : "memory");
+}
 // A 3D box (c0 innermost) into this CTA's shared memory, completion on an
 // mbarrier of this CTA.
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap *m, void *dst, uint64_t *bar, int c0, int c1, int c2) {
