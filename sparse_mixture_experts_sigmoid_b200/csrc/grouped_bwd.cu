@@ -23,13 +23,15 @@
 // SWIGLU epilogue).  So a weight-gradient tile reads whole 64-row K blocks of
 // both operands and the rows past a segment's end add nothing.
 //
-// Two tile schemes share one persistent kernel (one CTA per SM; warps 0-3
-// epilogue, warp 4 TMA producer, warp 5 TMEM allocator + MMA issuer):
+// Two tile schemes share one persistent kernel (one CTA per SM; epilogue
+// warps first -- eight, two per TMEM lane quarter, or four for the scatter
+// epilogue -- then the TMA producer warp and the TMEM allocator + MMA issuer
+// warp), and a two-SM variant of it (see bwd_gemm_pair_kernel):
 //  * ROWS: tiles of 128 grouped rows x 256 output columns, K over the
 //    weight's reduction dimension in blocks of 64, split into up to two K
 //    ranges (the gate half and the up half of [du | dv]).  A is K-major; B is
 //    a weight read MN-major (its rows are the K index, contiguous along N),
-//    four 64 x 64 TMA boxes per K block.
+//    one 3D TMA box of 64-column atoms per K block.
 //  * WGRAD: tiles of 128 weight rows x 256 weight columns of one expert, K
 //    over that expert's (padded) rows in blocks of 64.  Both operands are
 //    MN-major: each row contributes one 128-byte k-row per 64 columns.  An
