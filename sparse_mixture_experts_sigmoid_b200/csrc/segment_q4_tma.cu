@@ -39,16 +39,22 @@ namespace {
 using namespace tc;
 
 #ifndef MOE_Q4_WARPS
-#define MOE_Q4_WARPS 16
+#define MOE_Q4_WARPS 14
 #endif
 constexpr int kQWarps = MOE_Q4_WARPS;                  // consumer warps
-static_assert(kQWarps == 8 || kQWarps == 16, "32 rows per item over the consumer warps, within 1024 threads");
+static_assert(kQWarps == 8 || kQWarps == 14 || kQWarps == 16, "consumer warps per CTA");
 constexpr int kQThreads = (kQWarps + 1) * 32;          // + the producer warp
-constexpr int kQRows = 32;                             // weight rows per work item
-constexpr int kQRW = kQRows / kQWarps;                 // weight rows per consumer warp
+constexpr int kQRW = 2;                                // weight rows per consumer warp
+// weight rows per work item: 28 makes the Mixtral shapes' item counts fit
+// the 148 SMs (1024 gate/up items, 6.9 per SM; 147 down items) where 32
+// left a seventh gate/up item on 8 SMs and 20 SMs without a down item; the
+// last item of a matrix may be partial (its extra rows are computed from
+// the next rows or TMA's zero fill, and not stored)
+constexpr int kQRows = kQRW * kQWarps;
 constexpr int kQChunk = 1024;                          // reduction elements per stage
-constexpr int kQCodeBytes = kQRows * kQChunk / 2;      // 16 KB of codes per matrix
-constexpr int kQScaleBytes = kQRows * (kQChunk / 64) * 4;   // 2 KB of scales per matrix
+constexpr int kQCodeBytes = kQRows * kQChunk / 2;      // codes per matrix (14 KB for 28 rows)
+constexpr int kQScaleBytes = kQRows * (kQChunk / 64) * 4;   // scales per matrix
+static_assert(kQCodeBytes % 128 == 0 && kQScaleBytes % 128 == 0, "TMA destinations stay 128-byte aligned");
 constexpr int kQRing = 180 * 1024;                     // shared-memory ring
 constexpr int kQTok = 2;                               // grouped rows per gate/up pass
 constexpr int kQMaxPasses = 64;                        // at most kDecodeMaxRows rows
@@ -70,6 +76,7 @@ constexpr int q_stages() {
     return kQRing / q_stage_bytes<NMAT>();
 }
 
+static_assert(q_stages<1>() <= 12 && q_stages<2>() <= 12, "ring stages fit the barrier arrays");
 struct QCtrl {
     uint64_t full[12];
     uint64_t empty[12];
@@ -238,7 +245,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     __syncthreads();
     pdl_launch_dependents();
 
-    const int nrb = a.hid / kQRows;
+    const int nrb = (a.hid + kQRows - 1) / kQRows;
     const int nitems = c->n_pass * nrb;
     const int nch = (a.d + kQChunk - 1) / kQChunk;
 
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 for (int q = 0; q < kQRW; ++q) {
                     const float g = warp_sum(ag[b][q]);
                     const float u = warp_sum(au[b][q]);
-                    if (lane == 0 && tok[b] >= 0)
+                    if (lane == 0 && tok[b] >= 0 && n0 + q < a.hid)
                         a.act[(int64_t)(c->pb[ps] + b) * a.hid + n0 + q] = __float2bfloat16_rn(silu_f(g) * u);
                 }
             }
@@ -379,7 +386,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     __syncthreads();
     pdl_launch_dependents();
 
-    const int nrb = a.d / kQRows;
+    const int nrb = (a.d + kQRows - 1) / kQRows;
     const int64_t nitems = a.T * nrb;
     const int nch = (a.h + kQChunk - 1) / kQChunk;
     const int R = (int)(a.T * a.k);
@@ -478,7 +485,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
             for (int q = 0; q < kQRW; ++q) {
                 float v = warp_sum(acc[q]);
-                if (lane == 0) {
+                if (lane == 0 && n0 + q < a.d) {
                     if (a.shared_add) v += a.shared_add[t * a.d + n0 + q];
                     a.y[t * a.d + n0 + q] = __float2bfloat16_rn(v);
                 }
@@ -524,13 +531,13 @@ int q_grid(int64_t items) { return (int)std::max<int64_t>(1, std::min<int64_t>(i
 
 bool q4_tma_supported(int d, int h, const void *x, const void *q_gate, const float *s_gate, const void *q_up, const float *s_up,
                       const void *q_down, const float *s_down) {
-    // rows of scales must be 16-byte strides (K / 64 a multiple of 4), the
-    // row blocks must not cross experts, and every base 16-byte aligned
+    // rows of scales must be 16-byte strides (K / 64 a multiple of 4) and
+    // every base 16-byte aligned
     const uintptr_t al = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(q_gate) |
                          reinterpret_cast<uintptr_t>(s_gate) |
                          reinterpret_cast<uintptr_t>(q_up) | reinterpret_cast<uintptr_t>(s_up) |
                          reinterpret_cast<uintptr_t>(q_down) | reinterpret_cast<uintptr_t>(s_down);
-    return d % 256 == 0 && h % 256 == 0 && d % kQRows == 0 && h % kQRows == 0 && (al & 15) == 0;
+    return d % 256 == 0 && h % 256 == 0 && (al & 15) == 0;
 }
 
 cudaError_t launch_q4t_gateup(const SegGateUpQ4Args &a, cudaStream_t s) {
@@ -545,7 +552,7 @@ cudaError_t launch_q4t_gateup(const SegGateUpQ4Args &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(q4t_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // passes are at most the grouped rows; items = passes x row blocks
-    const int64_t items = std::min<int64_t>(a.seg.rows, kQMaxPasses) * (a.hid / kQRows);
+    const int64_t items = std::min<int64_t>(a.seg.rows, kQMaxPasses) * ((a.hid + kQRows - 1) / kQRows);
     return launch_kernel(q4t_gateup_kernel, q_grid(items), kQThreads, smem, s, mqg, mqu, msg, msu, p,
                          device_error_word());
 }
@@ -559,7 +566,7 @@ cudaError_t launch_q4t_down(const DownDirectQ4Args &a, const float *shared_add, 
     const size_t smem = q_smem<1>();
     cudaError_t e = cudaFuncSetAttribute(q4t_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(q4t_down_kernel, q_grid(a.T * (a.d / kQRows)), kQThreads, smem, s, mq, ms, p,
+    return launch_kernel(q4t_down_kernel, q_grid(a.T * ((a.d + kQRows - 1) / kQRows)), kQThreads, smem, s, mq, ms, p,
                          device_error_word());
 }
 
