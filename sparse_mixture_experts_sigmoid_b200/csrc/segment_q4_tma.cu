@@ -12,17 +12,17 @@
 // bytes each SM keeps in flight.  Loading the codes into registers ties that
 // to the register file (the warps that fit and the loads each can have
 // outstanding); here one producer thread per CTA streams the codes and scales
-// of 32 weight rows x 1024 reduction elements per stage (16 KB of codes per
+// of 28 weight rows x 1024 reduction elements per stage (14 KB of codes per
 // matrix), with the activation chunks they meet (contiguous bulk copies),
-// into a ~180 KB ring, and sixteen consumer warps read them from shared
+// into a ~180 KB ring, and fourteen consumer warps read them from shared
 // memory, two rows per warp, each lane 32 codes of a row per stage (one
 // 16-byte shared load).  The activation chunk a lane needs (32 values) is
 // read once per stage and shared by its rows.
 //
-//   q4t_gateup_kernel: work items (expert pass, block of 32 hidden rows); a
+//   q4t_gateup_kernel: work items (expert pass, block of 28 hidden rows); a
 //     pass holds up to two of the expert's grouped rows, whose activations
 //     meet the staged gate and up codes; act = silu(gate) * up in bf16.
-//   q4t_down_kernel: work items (token, block of 32 output rows); the stages
+//   q4t_down_kernel: work items (token, block of 28 output rows); the stages
 //     walk the k chosen experts' W_down rows in slot order, so
 //     y = sum_j g_j (W_down[e_j] . act_j) is summed in a fixed order, plus the
 //     shared expert's row (computed beforehand in fp32) when there is one.
