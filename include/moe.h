@@ -286,8 +286,12 @@ moe_status moe_forward(const moe_config *cfg, const moe_route_opts *opts, const 
                        void *stream);
 
 /* moe_forward for inputs and outputs in host memory: x_host [T, d] is copied
- * in and y_host [T, d] out by the call, in `chunks` pieces of at most
- * ceil(T / chunks) tokens each.  Piece i's layer (moe_forward on its tokens,
+ * in and y_host [T, d] out by the call, in n = min(chunks, T, 256) pieces of
+ * consecutive tokens.  With n >= 3 the first and last pieces hold half as
+ * many tokens as the others (their copies are the ones no layer hides):
+ * piece i is tokens [T c_i / (2n - 2), T c_(i+1) / (2n - 2)) with c_0 = 0,
+ * c_i = 2i - 1 for 0 < i < n, c_n = 2n - 2 (integer division); with n <= 2,
+ * tokens [T i / n, T (i + 1) / n).  Piece i's layer (moe_forward on its tokens,
  * without routing options) runs on `stream` once its rows are on the device,
  * and its y goes back on `copy_stream` while later pieces compute, so the
  * copies overlap the layer; each token's result is that of moe_forward on
@@ -301,7 +305,7 @@ moe_status moe_forward(const moe_config *cfg, const moe_route_opts *opts, const 
  *   second stream, or NULL to issue the copies on `stream` (no overlap).
  *   ws: device workspace of at least moe_forward_host_workspace_size(cfg,
  *   chunks) bytes, 256-byte aligned (the device copies of x and y, then the
- *   layer's workspace for one piece).
+ *   layer's workspace for the largest piece).
  * The call returns once everything is queued; when `stream` reaches the
  * point of the call's end, y_host is complete (the copy stream's last copy
  * is made a dependency of `stream`).  Events are created and destroyed by

@@ -346,6 +346,18 @@ def _host_ptr(t: torch.Tensor, name: str, shape, dtype):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def host_piece_bounds(T: int, chunks: int) -> list[int]:
+    """The token bounds of moe_forward_host's pieces (its documented rule: n = min(chunks, T, 256);
+    with n >= 3 the first and last pieces are half as large as the others)."""
+    n = min(chunks, T, 256)
+    if n <= 0:
+        return [0]
+    if n <= 2:
+        return [T * i // n for i in range(n + 1)]
+    c = [0] + [2 * i - 1 for i in range(1, n)] + [2 * n - 2]
+    return [T * ci // (2 * n - 2) for ci in c]
+
+
 def forward_host_workspace_size(cfg: MoEConfig, chunks: int) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().moe_forward_host_workspace_size(ctypes.byref(cfg), int(chunks), ctypes.byref(n)),

@@ -661,22 +661,39 @@ namespace {
 
 constexpr int64_t kMaxHostPieces = 256;   // moe_forward_host: events per call stay few
 
+// Pieces of moe_forward_host: n = min(chunks, T, 256); with n >= 3 the first
+// and last pieces carry half the tokens of the others (the first piece's copy
+// in and the last piece's copy back are the parts no layer overlaps), so
+// piece i spans tokens [T c_i / (2n - 2), T c_{i+1} / (2n - 2)) with c_0 = 0,
+// c_i = 2i - 1 (0 < i < n), c_n = 2n - 2 (integer division); with n <= 2 the
+// pieces are T c_i / n with c_i = i.
+int64_t host_pieces(int64_t T, int32_t chunks) {
+    int64_t n = chunks > T ? T : chunks;
+    return n > kMaxHostPieces ? kMaxHostPieces : n;
+}
+int64_t host_bound(int64_t T, int64_t n, int64_t i) {
+    if (n <= 2) return T * i / n;
+    const int64_t c = i == 0 ? 0 : (i == n ? 2 * n - 2 : 2 * i - 1);
+    return T * c / (2 * n - 2);
+}
+
 // Workspace of moe_forward_host: the device copies of x and y, then the
-// layer's workspace for one piece of at most ceil(T / chunks) tokens.
+// layer's workspace for its largest piece.
 struct HostLayout {
     size_t x_off, y_off, ws_off, total;
-    int64_t piece;
+    int64_t n;   // pieces
 };
 moe_status host_layout(const moe_config &c, int32_t chunks, HostLayout *h) {
     if (chunks <= 0) return MOE_ERR_INVALID_ARG;
     const moe_status st = moe_validate(&c);
     if (st != MOE_OK) return st;
     const size_t esz = c.dtype == MOE_F32 ? 4 : 2;
-    int64_t n = chunks > c.T ? c.T : chunks;
-    n = n > kMaxHostPieces ? kMaxHostPieces : n;
-    h->piece = n > 0 ? (c.T + n - 1) / n : 0;
+    h->n = host_pieces(c.T, chunks);
+    int64_t largest = 0;
+    for (int64_t i = 0; i < h->n; ++i)
+        largest = std::max<int64_t>(largest, host_bound(c.T, h->n, i + 1) - host_bound(c.T, h->n, i));
     moe_config pc = c;
-    pc.T = h->piece;
+    pc.T = largest;
     const size_t rows = (size_t)c.T * c.d * esz;
     h->x_off = 0;
     h->y_off = align256(rows);
@@ -713,7 +730,7 @@ moe_status moe_forward_host(const moe_config *c, const void *x_host, const void 
     void *lws = static_cast<char *>(ws) + h.ws_off;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaStream_t cs = copy_stream ? static_cast<cudaStream_t>(copy_stream) : s;
-    const int64_t n = (c->T + h.piece - 1) / h.piece;   // pieces
+    const int64_t n = h.n;
     // events order the two streams: start (earlier work on stream is done
     // with the device copies), in[i] (piece i is on the device), out[i]
     // (piece i's y is ready), done (the last copy back has landed)
@@ -729,13 +746,15 @@ moe_status moe_forward_host(const moe_config *c, const void *x_host, const void 
     // every piece's rows in first (one copy each), so that no copy to the
     // device waits behind a copy back on the copy stream
     for (int64_t i = 0; i < n && e == cudaSuccess; ++i) {
-        const int64_t t0 = i * h.piece, rows = std::min<int64_t>(h.piece, c->T - t0);
+        const int64_t t0 = host_bound(c->T, n, i), rows = host_bound(c->T, n, i + 1) - t0;
+        if (rows <= 0) continue;
         e = cudaMemcpyAsync(xd + t0 * row_bytes, static_cast<const char *>(x_host) + t0 * row_bytes,
                             (size_t)rows * row_bytes, cudaMemcpyHostToDevice, cs);
         if (e == cudaSuccess) e = cudaEventRecord(ev_in(i), cs);
     }
     for (int64_t i = 0; i < n && e == cudaSuccess && st == MOE_OK; ++i) {
-        const int64_t t0 = i * h.piece, rows = std::min<int64_t>(h.piece, c->T - t0);
+        const int64_t t0 = host_bound(c->T, n, i), rows = host_bound(c->T, n, i + 1) - t0;
+        if (rows <= 0) continue;
         moe_config pc = *c;
         pc.T = rows;
         e = cudaStreamWaitEvent(s, ev_in(i), 0);

@@ -210,7 +210,11 @@ def test_forward_host_workspace_and_argument_checks():
         esz = 4 if w.dtype == "f32" else 2
         rows = -(-w.T * w.d * esz // 256) * 256
         for chunks in (1, 2, 3, 4, 8):
-            piece = -(-w.T // min(chunks, w.T))
+            b = B.host_piece_bounds(w.T, chunks)
+            assert b[0] == 0 and b[-1] == w.T and all(x <= y for x, y in zip(b, b[1:]))
+            piece = max(y - x for x, y in zip(b, b[1:]))
+            if len(b) > 3:   # three or more pieces: the outer ones hold about half the tokens
+                assert abs(2 * (b[1] - b[0]) - (b[2] - b[1])) <= 2
             layer = B.workspace_size(B.config_of(w, T=piece))
             assert B.forward_host_workspace_size(cfg, chunks) == 2 * rows + layer
         assert B.forward_host_workspace_size(cfg, w.T + 5) == B.forward_host_workspace_size(cfg, min(w.T, 256))

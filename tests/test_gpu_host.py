@@ -7,8 +7,8 @@ other pieces' layers.
   stream, bf16 and fp32, with the shared expert;
 * with the ordered combine, every piece's y bit-identical to moe_forward on
   that piece's tokens (the call is moe_forward per piece plus the copies);
-* a ragged last piece (T not a multiple of the piece size) and more pieces
-  than tokens.
+* three or more pieces (the first and last half as large as the others),
+  uneven splits, and more pieces than tokens.
 """
 import numpy as np
 import pytest
@@ -82,10 +82,10 @@ def test_forward_host_pieces_equal_forward_on_their_tokens(w, chunks):
     B.forward_host(cfg, dev, xh, yh, chunks, ws=ws, copy_stream=torch.cuda.Stream())
     torch.cuda.current_stream().synchronize()
     assert B.device_status() == 0
-    n = min(chunks, w.T)
-    piece = -(-w.T // n)
-    for t0 in range(0, w.T, piece):
-        t1 = min(w.T, t0 + piece)
+    b = B.host_piece_bounds(w.T, chunks)
+    for t0, t1 in zip(b, b[1:]):
+        if t1 == t0:
+            continue
         pc = B.config_of(w, T=t1 - t0, combine="ordered")
         y = B.forward(pc, dev.x[t0:t1].contiguous(), dev.w_router, dev.w_gate, dev.w_up, dev.w_down,
                       dev.sh_gate, dev.sh_up, dev.sh_down, dev.w_shared_gate).cpu()
