@@ -139,6 +139,11 @@ struct Params {
     // STORE epilogue: row-major [groups * M, N] per half
     void *out0, *out1;
     bool out_f32;
+    // WGRAD on one SM, fp32 output of one dense group (the router's weight
+    // gradient: few output tiles, a long K): its K blocks split into ksplit
+    // consecutive ranges, each range's product added into the zeroed output
+    // (1: stored whole)
+    int ksplit;
     // the MN-major operands (B; A too in WGRAD) come through 3D tensor maps
     // {64 columns, rows, 64-column blocks}: one TMA instruction fetches all
     // of a stage's 64-column atoms of an operand
@@ -148,7 +153,31 @@ struct Params {
 // ------------------------------------------------------------------ epilogues
 
 using gg::kXBytes;
+using gg::x_slot;
 using gg::x_store_rows;
+
+// x_store_rows with fp32 reductions into global memory instead of stores.
+__device__ __forceinline__ void x_reduce_rows(uint8_t *buf, const uint4 (&in)[4], uint8_t *base, int64_t row0,
+                                              int64_t ld, int nrows, int nwords) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4 *>(buf + x_slot(lane, j)) = in[j];
+    __syncwarp();
+    const int j = lane & 3;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int i = 8 * t + (lane >> 2);
+        const uint4 w = *reinterpret_cast<const uint4 *>(buf + x_slot(i, j));
+        if (i < nrows && j < nwords) {
+            float *dst = reinterpret_cast<float *>(base + (row0 + i) * ld + 16 * j);
+            asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                         ::"l"(dst), "f"(__uint_as_float(w.x)), "f"(__uint_as_float(w.y)), "f"(__uint_as_float(w.z)),
+                           "f"(__uint_as_float(w.w))
+                         : "memory");
+        }
+    }
+    __syncwarp();
+}
 
 // Shared memory of the epilogue warps: the scatter's row staging, else the
 // exchange buffers (16 KB either way).
@@ -262,7 +291,7 @@ template <int NC>
 __device__ __forceinline__ void epilogue_store(const Params &p, int e, int half, int m0, int n0, bool has_rows,
                                                uint32_t tbase, uint8_t *xb) {
     const int nrows = min(32, p.M - m0);
-    if (nrows <= 0) return;
+    if (nrows <= 0 || (p.ksplit > 1 && !has_rows)) return;   // split K: an empty range adds nothing
     const int64_t orow0 = (int64_t)e * p.M + m0;
     uint8_t *out = static_cast<uint8_t *>(half ? p.out1 : p.out0);
 #pragma unroll 1
@@ -288,7 +317,10 @@ __device__ __forceinline__ void epilogue_store(const Params &p, int e, int half,
                     w[q] = make_uint4(__float_as_uint(v[h][4 * q]), __float_as_uint(v[h][4 * q + 1]),
                                       __float_as_uint(v[h][4 * q + 2]), __float_as_uint(v[h][4 * q + 3]));
                 const int c16 = col0 + 16 * h;
-                if (c16 < p.N)
+                if (c16 >= p.N) continue;
+                if (p.ksplit > 1)
+                    x_reduce_rows(xb, w, out + 4 * (int64_t)c16, orow0, 4 * (int64_t)p.N, nrows, min(4, (p.N - c16) / 4));
+                else
                     x_store_rows(xb, w, out + 4 * (int64_t)c16, orow0, 4 * (int64_t)p.N, nrows, min(4, (p.N - c16) / 4));
             }
         } else {
@@ -393,17 +425,30 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
     const int nE = p.g.offsets ? p.g.E : 1;
     const int ntiles = (p.N + BN - 1) / BN;
     const int mtiles = MODE == WGRAD ? (p.M + BM - 1) / BM : 0;
-    const int total = MODE == ROWS ? ctrl->n_mtiles * ntiles : nE * p.halves * mtiles * ntiles;
+    const int wbase = nE * p.halves * mtiles * ntiles;   // WGRAD tiles per K range
+    const int total = MODE == ROWS ? ctrl->n_mtiles * ntiles : wbase * p.ksplit;
     const int kpr = (p.Kr + BK - 1) / BK;   // ROWS: K blocks per range
     // first row of group e in the operands' layout
     auto op_row0 = [&](int e) -> int { return p.padded ? 64 * blk64[e] : seg_off[e]; };
+    // WGRAD: tile id -> its weight tile and its K range's first K block and
+    // K block count (ranges of whole 64-row blocks; a range may be empty)
+    auto wtile = [&](int id, int *kb0, int *nk) -> WTile {
+        const int ks = id / wbase;
+        const WTile w = wdecode(id - ks * wbase, mtiles, ntiles, p.halves);
+        const int blocks = (seg_end[w.e] - seg_off[w.e] + 63) / 64;
+        const int per = (blocks + p.ksplit - 1) / p.ksplit;
+        *kb0 = ks * per;
+        *nk = max(0, min(per, blocks - *kb0));
+        return w;
+    };
     // K blocks of a tile
     auto tile_nk = [&](int id) -> int {
         if constexpr (MODE == ROWS) {
             return p.nranges * kpr;
         } else {
-            const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-            return (seg_end[w.e] - seg_off[w.e] + 63) / 64;
+            int kb0, nk;
+            wtile(id, &kb0, &nk);
+            return nk;
         }
     };
 
@@ -443,11 +488,12 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                     t.b_row = tl.e * p.Kr;
                     t.b_col = tl.n * BN;
                 } else {
-                    const WTile w = wdecode(id, mtiles, ntiles, p.halves);
+                    int kb0, nkw;
+                    const WTile w = wtile(id, &kb0, &nkw);
                     t.half = w.half;
                     t.m0 = w.mt * BM;
                     t.n0 = w.nt * BN;
-                    t.krow0 = op_row0(w.e);
+                    t.krow0 = op_row0(w.e) + 64 * kb0;
                 }
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % kStages;
@@ -572,8 +618,9 @@ __global__ void __launch_bounds__(kernel_threads<EPI>(), 1)
                         p.g, tl.n, r, valid, tb, reinterpret_cast<float *>(sEpi + warp * gg::kEpiStageBytes));
                 }
             } else {
-                const WTile w = wdecode(id, mtiles, ntiles, p.halves);
-                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM + row - lane, w.nt * BN + c0, seg_end[w.e] > seg_off[w.e], tb,
+                int kb0, nkw;
+                const WTile w = wtile(id, &kb0, &nkw);
+                epilogue_store<kCols>(p, w.e, w.half, w.mt * BM + row - lane, w.nt * BN + c0, nkw > 0, tb,
                                       sEpi + warp * kXBytes);
             }
             ck_b.stop();
@@ -1006,7 +1053,7 @@ cudaError_t launch_bwd(const BwdOperand &a0, const BwdOperand &a1, const BwdOper
     const int ntiles = (p.N + BN - 1) / BN;
     int64_t max_tiles;
     if (MODE == ROWS) max_tiles = (p.g.rows / BM + nE) * (int64_t)ntiles;
-    else max_tiles = (int64_t)nE * p.halves * ((p.M + BM - 1) / BM) * ntiles;
+    else max_tiles = (int64_t)nE * p.halves * ((p.M + BM - 1) / BM) * ntiles * p.ksplit;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
     const size_t smem = 1024 + (size_t)kStages * (kAStage + kBStage) +
                         epi_stage_bytes<EPI>() + sizeof(Ctrl) +
@@ -1095,12 +1142,29 @@ cudaError_t launch_bwd_gemm(const BwdGemm &L, cudaStream_t s) {
     p.out0 = L.out0;
     p.out1 = L.out1;
     p.out_f32 = L.out_f32;
+    p.ksplit = 1;
     if (L.rows <= 0 && L.kind != BwdGemm::WEIGHT) return cudaSuccess;
     if (bwd_pair(L)) {
         switch (L.kind) {
             case BwdGemm::SWIGLU: return launch_bwd_pair<ROWS, EPI_SWIGLU>(L.a0, L.a1, L.b0, L.b1, p, s);
             case BwdGemm::SCATTER: return launch_bwd_pair<ROWS, EPI_SCATTER>(L.a0, L.a1, L.b0, L.b1, p, s);
             default: return launch_bwd_pair<WGRAD, EPI_STORE>(L.a0, L.a1, L.b0, L.b1, p, s);
+        }
+    }
+    if (L.kind == BwdGemm::WEIGHT && !L.offsets && L.out_f32 && L.rows > 0) {
+        // one dense group with an fp32 output (the router's weight gradient:
+        // E x d outputs, K = T rows): split K so that about one tile runs per
+        // SM, each range adding into the zeroed output (at least 4 K blocks
+        // per range)
+        const int64_t tiles = (int64_t)L.halves * ((L.M + BM - 1) / BM) * ((L.N + BN - 1) / BN);
+        const int64_t blocks = (L.rows + 63) / 64;
+        const int64_t split = std::min<int64_t>(num_sms() / std::max<int64_t>(tiles, 1), blocks / 4);
+        if (split > 1) {
+            p.ksplit = (int)split;
+            const size_t bytes = sizeof(float) * (size_t)L.M * (size_t)L.N;
+            cudaError_t e = cudaMemsetAsync(L.out0, 0, bytes, s);
+            if (e == cudaSuccess && L.halves > 1) e = cudaMemsetAsync(L.out1, 0, bytes, s);
+            if (e != cudaSuccess) return e;
         }
     }
     switch (L.kind) {
