@@ -51,6 +51,8 @@ STAGE_KERNEL = {"route": ("router_logits_kernel", "router_tc.cu"), "permute": ("
 # kernels of the small-batch path (at most 64 assignments)
 STAGE_KERNEL_SMALL = {"route": ("router_small_kernel", "router.cu"), "gate_up": ("seg_gateup_kernel", "segment.cu"),
                       "down": ("down_direct_kernel", "segment.cu")}
+# ... the down projection of bf16 layers without a shared expert (h a multiple of 8)
+STAGE_KERNEL_SMALL_TMA = {"down": ("down_tma_kernel", "segment_tma.cu")}
 # ... with 4-bit routed experts
 # (the ring-streamed kernels, which the library picks for d and h multiples of 256)
 STAGE_KERNEL_Q4 = {"gate_up": ("q4t_gateup_kernel", "segment_q4_tma.cu"), "down": ("q4t_down_kernel", "segment_q4_tma.cu")}
@@ -212,6 +214,8 @@ def kernel_of(stage: str, w, q4: bool):
     kname, ksrc = STAGE_KERNEL[stage]
     if w.R <= B.decode_max_rows() and stage in STAGE_KERNEL_SMALL:
         kname, ksrc = STAGE_KERNEL_SMALL[stage]
+        if stage in STAGE_KERNEL_SMALL_TMA and w.dtype == "bf16" and not w.h_shared and w.h % 8 == 0:
+            kname, ksrc = STAGE_KERNEL_SMALL_TMA[stage]
     if q4 and stage in STAGE_KERNEL_Q4:
         kname, ksrc = STAGE_KERNEL_Q4[stage]
     return kname, ksrc

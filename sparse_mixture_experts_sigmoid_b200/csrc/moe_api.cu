@@ -506,6 +506,11 @@ moe_status moe_combine(const moe_config *c, const void *act, const void *w_down,
 }  // extern "C"
 
 namespace moe {
+// bf16 batch-1 down projection with the weight rows streamed by TMA through a
+// shared-memory ring (segment_tma.cu); the warp-per-row kernel serves the rest.
+bool down_tma_supported(const DownDirectArgs &a, int dtype);
+cudaError_t launch_down_tma(const DownDirectArgs &a, cudaStream_t s, uint32_t *err);
+
 // The forward pass; `train` also keeps what moe_backward needs (the full score
 // rows and the pre-activations of every grouped row) and always takes the
 // tensor-core path, whose gate/up epilogue writes them.
@@ -616,7 +621,8 @@ moe_status forward_impl(const moe_config *c, const moe_route_opts *opts, const v
         if (e == cudaSuccess) {
             DownDirectArgs da{act, w_down, ids, inv, gates, shared ? acts : nullptr, shared ? sh_down : nullptr,
                               sg, c->T, c->d, c->h, c->E, c->k, c->h_shared, y};
-            e = launch_down_direct(da, c->dtype, s, err);
+            e = down_tma_supported(da, c->dtype) ? launch_down_tma(da, s, err)
+                                                 : launch_down_direct(da, c->dtype, s, err);
         }
         mark(1 + MOE_STAGE_DOWN, s);
         mark(1 + MOE_STAGE_SHARED_DOWN, s);
