@@ -278,6 +278,16 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
 // same arg-max rounds as the batched router.
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
+    {
+        // The router rows are a layer input, not the previous kernel's output:
+        // pull them into L2 (spread over the CTAs) before waiting for it, so
+        // their DRAM latency overlaps its tail and the x row load below.  L2 is
+        // coherent, so a row written by an earlier kernel is never read stale.
+        const char *wb = static_cast<const char *>(a.w_router);
+        const int64_t lines = ((int64_t)a.E * a.d * (int64_t)sizeof(Tin) + 127) / 128;
+        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < lines; i += (int64_t)gridDim.x * kThreads)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(wb + 128 * i));
+    }
     pdl_wait();
     pdl_launch_dependents();
     extern __shared__ float sm[];

@@ -12,6 +12,9 @@ the small parity cases against the oracle:
   (experts with several row tiles included);
 * the routed down GEMM's column tiles in consecutive groups (chosen when
   the combine accumulator is large): MOE_DOWN_GROUPS=3 forces three;
+* the warp-per-output batch-1 down kernel, which the library keeps for
+  layers with a shared expert or fp32 weights: MOE_DOWN_TMA=0 forces it on
+  the bf16 decode cases instead of the TMA-ring kernel;
 * the backward GEMMs on two-SM tiles (chosen when groups average at least 512
   rows, or a weight gradient has at least 512 rows): MOE_BWD_PAIR=1 forces
   them on the small training cases, MOE_BWD_PAIR=0 forces one-SM tiles on the
@@ -57,6 +60,11 @@ def test_forward_small_with_down_column_groups():
     """The down GEMM's column tiles in three consecutive groups (one-SM and two-SM tiles)."""
     run_small_cases(MOE_DOWN_GROUPS="3")
     run_small_cases(MOE_DOWN_GROUPS="3", MOE_GG_PAIR="1")
+
+
+@pytest.mark.gpu
+def test_decode_small_with_warp_per_output_down():
+    run_small_cases(select="decode", MOE_DOWN_TMA="0")
 
 
 @pytest.mark.gpu
