@@ -378,13 +378,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         c->abort = 0;
         fence_barrier_init();
     }
-    if (warp == kQWarps && lane == 0) {
-        prefetch_tmap(&mq);
-        prefetch_tmap(&ms);
-    }
-    pdl_wait();
     __syncthreads();
-    pdl_launch_dependents();
 
     const int nrb = (a.d + kQRows - 1) / kQRows;
     const int64_t nitems = a.T * nrb;
@@ -397,6 +391,34 @@ __global__ void __launch_bounds__(kQThreads, 1)
         *r = a.inv_rows[slot];
         return (e < 0 || e >= a.E || *r < 0 || *r >= R) ? -1 : e;
     };
+
+    // The routing was written two or more kernels back and is complete when
+    // this grid starts; act (the gate/up output) and the shared expert's rows
+    // only after the wait.  The codes and scales of the first S stages are
+    // requested before it, their activation chunks after it.
+    uint32_t pre = 0;
+    if (warp == kQWarps && lane == 0) {
+        prefetch_tmap(&mq);
+        prefetch_tmap(&ms);
+        for (int64_t item = blockIdx.x; item < nitems && pre < (uint32_t)S; item += gridDim.x) {
+            const int64_t t = item / nrb;
+            const int nb = (int)(item - t * nrb);
+            for (int j = 0; j < a.k && pre < (uint32_t)S; ++j) {
+                int r;
+                const int e = expert_of(t, j, &r);
+                if (e < 0) continue;
+                for (int ch = 0; ch < nch && pre < (uint32_t)S; ++ch, ++pre) {
+                    uint8_t *st = ring + pre * SB;
+                    mbar_expect_tx(&c->full[pre],
+                                   kQCodeBytes + kQScaleBytes + 2u * (uint32_t)min(kQChunk, a.h - ch * kQChunk));
+                    tma_load_2d(&mq, st, &c->full[pre], ch * (kQChunk / 8), e * a.d + nb * kQRows);
+                    tma_load_2d(&ms, st + kQCodeBytes, &c->full[pre], ch * (kQChunk / 64), e * a.d + nb * kQRows);
+                }
+            }
+        }
+    }
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (warp == kQWarps) {
         if (lane == 0) {
@@ -412,13 +434,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
                     const int row0 = e * a.d + nb * kQRows;
                     for (int ch = 0; ch < nch; ++ch, ++it) {
                         const int s = it % S;
+                        uint8_t *st = ring + s * SB;
+                        const int k0 = ch * kQChunk;
+                        const uint32_t xbytes = 2u * (uint32_t)min(kQChunk, a.h - k0);
+                        if (it < pre) {
+                            // codes and scales requested before the wait
+                            bulk_load(st + kQXOff1, a.act + (int64_t)r * a.h + k0, xbytes, &c->full[s]);
+                            continue;
+                        }
                         if (!wait_bar(&c->empty[s], ((it / S) & 1) ^ 1, abort, err)) {
                             ok = false;
                             break;
                         }
-                        uint8_t *st = ring + s * SB;
-                        const int k0 = ch * kQChunk;
-                        const uint32_t xbytes = 2u * (uint32_t)min(kQChunk, a.h - k0);
                         mbar_expect_tx(&c->full[s], kQCodeBytes + kQScaleBytes + xbytes);
                         tma_load_2d(&mq, st, &c->full[s], ch * (kQChunk / 8), row0);
                         tma_load_2d(&ms, st + kQCodeBytes, &c->full[s], ch * (kQChunk / 64), row0);
