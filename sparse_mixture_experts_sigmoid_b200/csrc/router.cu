@@ -275,8 +275,10 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a, Geo g) {
 // w + 8, ... (lane l takes the 8-element slices l, l + 32, ... of the row with
 // 16-byte loads, all issued before the reduction), so the router weights are
 // streamed by the whole CTA at once.  Warp 0 then selects the top k with the
-// same arg-max rounds as the batched router.
-template <typename Tin>
+// same arg-max rounds as the batched router, over EPL experts per lane (the
+// smallest power of two covering E / 32: the selection is the serial tail of
+// a batch-1 step, and its code is fetched from memory each time).
+template <typename Tin, int EPL>
 __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     {
         // The router rows are a layer input, not the previous kernel's output:
@@ -295,6 +297,19 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     float *lg = sm + a.d;        // [E + 1] logits (shared gate last)
     const int64_t t = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Tin *wr = static_cast<const Tin *>(a.w_router);
+    const int Ep = a.E + (a.w_shared_gate ? 1 : 0);
+    auto row_of = [&](int e) { return e < a.E ? wr + (int64_t)e * a.d : static_cast<const Tin *>(a.w_shared_gate); };
+    // the first kPre slices of this warp's first row are loaded before the x
+    // row is staged, so the two loads overlap
+    constexpr int kPre = 8;
+    float wpre[kPre][8];
+    if (warp < Ep) {
+        const Tin *row = row_of(warp);
+#pragma unroll
+        for (int i = 0; i < kPre; ++i)
+            if (lane * 8 + 256 * i < a.d) load8(row + lane * 8 + 256 * i, wpre[i]);
+    }
     const Tin *x = static_cast<const Tin *>(a.x) + t * a.d;
     for (int c = threadIdx.x * 8; c < a.d; c += kThreads * 8) {
         float v[8];
@@ -307,13 +322,20 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
         for (int i = threadIdx.x; i < a.d / 4; i += kThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    const Tin *wr = static_cast<const Tin *>(a.w_router);
-    const int Ep = a.E + (a.w_shared_gate ? 1 : 0);
     for (int e = warp; e < Ep; e += kWarps) {
-        const Tin *row = e < a.E ? wr + (int64_t)e * a.d : static_cast<const Tin *>(a.w_shared_gate);
+        const Tin *row = row_of(e);
         float acc = 0.f;
+        int c = lane * 8;
+        if (e == warp) {
+#pragma unroll
+            for (int i = 0; i < kPre; ++i, c += 256)
+                if (c < a.d) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) acc = fmaf(wpre[i][u], sx[c + u], acc);
+                }
+        }
 #pragma unroll 4
-        for (int c = lane * 8; c < a.d; c += 256) {
+        for (; c < a.d; c += 256) {
             float w[8];
             load8(row + c, w);
 #pragma unroll
@@ -324,7 +346,6 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     }
     __syncthreads();
     if (warp != 0) return;
-    constexpr int EPL = MOE_MAX_EXPERTS / 32;
     const bool sigm = a.score == MOE_SCORE_SIGMOID;
     float l[EPL], key[EPL], sc_e[EPL];
 #pragma unroll
@@ -511,7 +532,18 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, float *scratch, cudaSt
     if (scratch && router_tc_supported(a.T, a.E, dtype)) return launch_router_tc(a, scratch, s);
     if (a.T <= kSmallT) {
         const size_t smem = sizeof(float) * ((size_t)a.d + a.E + 1);
-        auto kern = dtype == MOE_F32 ? router_small_kernel<float> : router_small_kernel<__nv_bfloat16>;
+        const int epl = pow2ceil((a.E + 31) / 32);
+        auto pick = [&](auto tin) -> void (*)(RouterArgs) {
+            using Tin = decltype(tin);
+            switch (epl) {
+                case 1: return router_small_kernel<Tin, 1>;
+                case 2: return router_small_kernel<Tin, 2>;
+                case 4: return router_small_kernel<Tin, 4>;
+                case 8: return router_small_kernel<Tin, 8>;
+                default: return router_small_kernel<Tin, MOE_MAX_EXPERTS / 32>;
+            }
+        };
+        auto kern = dtype == MOE_F32 ? pick(float{}) : pick(__nv_bfloat16{});
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess) e = launch_kernel(kern, (unsigned)a.T, kThreads, smem, s, a);
         if (e == cudaSuccess && a.stats && a.score_mean)
