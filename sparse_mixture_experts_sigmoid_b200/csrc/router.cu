@@ -300,9 +300,10 @@ __global__ void __launch_bounds__(kThreads) router_small_kernel(RouterArgs a) {
     const Tin *wr = static_cast<const Tin *>(a.w_router);
     const int Ep = a.E + (a.w_shared_gate ? 1 : 0);
     auto row_of = [&](int e) { return e < a.E ? wr + (int64_t)e * a.d : static_cast<const Tin *>(a.w_shared_gate); };
-    // the first kPre slices of this warp's first row are loaded before the x
-    // row is staged, so the two loads overlap
-    constexpr int kPre = 8;
+    // the first kPre slices of this warp's first row (all of a row of up to
+    // 4096 elements) are loaded before the x row is staged, so the two loads
+    // overlap and the row arrives in one round trip
+    constexpr int kPre = 16;
     float wpre[kPre][8];
     if (warp < Ep) {
         const Tin *row = row_of(warp);
