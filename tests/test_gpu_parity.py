@@ -174,6 +174,8 @@ SMALL = [
     small("decode_T1_ragged_widths", T=1, d=200, h=136, h_shared=72, score="sigmoid", seed=66),
     small("decode_T1_k16", T=1, E=64, k=16, d=128, h=64, router_std=0.2, seed=67),
     small("decode_T2_ragged_widths", T=2, d=200, h=136, seed=69),   # partial row block and reduction chunk
+    small("decode_T16_k4", T=16, seed=70),   # 64 assignments: more work items than SMs in the batch-1 down kernel
+    small("decode_T64_k1", T=64, k=1, d=512, h=1024, seed=71),   # the largest small batch, two 512-element chunks
     small("width_not_mult_64", d=200, h=136, seed=61),
     small("many_experts", E=512, k=16, T=200, d=128, h=64, router_std=0.2, seed=62),
     small("zipf_hot_expert", recipe="zipf", E=32, k=2, seed=63),
