@@ -70,3 +70,28 @@ def test_load_spread():
     s = roofline.load_spread([4, 0, 2, 2])
     assert s["active_experts"] == 3 and s["max"] == 4 and s["min"] == 0 and s["mean"] == 2.0
     assert abs(s["cv"] - np.std([4, 0, 2, 2]) / 2.0) < 1e-15
+
+
+def test_bench_names_the_kernel_each_stage_runs():
+    """The kernel (and source) the bench line attributes each stage to: the
+    batch-1 bf16 down projection runs the TMA-ring kernel unless the layer has
+    a shared expert, 4-bit layers run the ring-streamed 4-bit kernels, and
+    every named source exists (its hash keys the committed DRAM captures)."""
+    import dataclasses
+
+    import bench
+
+    dec = WORKLOADS["mixtral_decode"]
+    assert bench.kernel_of("down", dec, False) == ("down_tma_kernel", "segment_tma.cu")
+    assert bench.kernel_of("gate_up", dec, False) == ("seg_gateup_kernel", "segment.cu")
+    assert bench.kernel_of("down", dec, True) == ("q4t_down_kernel", "segment_q4_tma.cu")
+    shared = dataclasses.replace(dec, h_shared=1024)
+    assert bench.kernel_of("down", shared, False) == ("down_direct_kernel", "segment.cu")
+    f32 = dataclasses.replace(dec, dtype="f32")
+    assert bench.kernel_of("down", f32, False) == ("down_direct_kernel", "segment.cu")
+    pre = WORKLOADS["mixtral_prefill"]
+    assert bench.kernel_of("gate_up", pre, False) == ("grouped_gemm_kernel", bench.GG_SRC)
+    tables = (bench.STAGE_KERNEL, bench.STAGE_KERNEL_SMALL, bench.STAGE_KERNEL_SMALL_TMA, bench.STAGE_KERNEL_Q4)
+    for table in tables:
+        for _, src in table.values():
+            assert len(bench.source_hash(src)) == 16
